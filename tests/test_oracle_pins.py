@@ -1,0 +1,350 @@
+"""Pins of the oracle against what the pages and mathematics fix (CPU only).
+
+Each oracle step is checked against something other than itself: hand-derived
+golden cases (tests/golden/), closed forms, library routines (numpy matmul,
+numpy convolve, torch's bf16 conversion) and invariants the pages state.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+def _load_rows(path):
+    rows = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        rows.append(line.split())
+    return rows
+
+
+# ------------------------------------------------------------------ remap
+
+def test_remap_golden(golden_dir):
+    rows = {r[0]: [int(x) for x in r[1:]] for r in _load_rows(os.path.join(golden_dir, "remap_case.txt"))}
+    canon, bad = oracle.remap(np.array(rows["tok"]), np.array(rows["P"]))
+    assert bad == 0
+    assert canon.tolist() == rows["canon"]
+
+
+def test_remap_out_of_range_marks_invalid():
+    P = np.array([1, 0, 2, 1])
+    canon, bad = oracle.remap(np.array([0, 4, -1, 3]), P)
+    assert bad == 2
+    assert canon.tolist() == [1, -1, -1, 1]
+
+
+# ------------------------------------------------------------------ hash
+
+def test_hash_single_head_golden(golden_dir):
+    for r in _load_rows(os.path.join(golden_dir, "hash_cases.txt")):
+        n, M, a0, a1, a2, s0, s1, s2, want = (int(x) for x in r)
+        s = [s0, s1, s2][:n]
+        canon = np.array([list(reversed(s))], dtype=np.int32)  # s_0 is the last position
+        mult = np.array([[a0, a1, a2, 0]], dtype=np.uint64)
+        idx, bad = oracle.hash_ids(canon, 1 << 30, [n], 1, mult, np.array([M]), t_begin=n - 1)
+        assert bad == 0
+        assert idx.shape == (1, 1)
+        assert int(idx[0, 0]) == want, r
+
+
+def test_hash_sequence_golden_with_padding(golden_dir):
+    rows = _load_rows(os.path.join(golden_dir, "hash_sequence.txt"))
+    canon = np.array([[4, 7, 2]], dtype=np.int32)
+    mult = np.array([[1, 2, 0, 0], [1, 2, 4, 0]], dtype=np.uint64)
+    idx, bad = oracle.hash_ids(canon, 10, [2, 3], 1, mult, np.array([97, 97]))
+    assert bad == 0
+    for t, i2, i3, _ in ((int(x) for x in r) for r in rows):
+        assert idx[t].tolist() == [i2, i3]
+    idx13, _ = oracle.hash_ids(canon, 10, [2, 3], 1, mult, np.array([97, 13]))
+    for t, i2, _, i3 in ((int(x) for x in r) for r in rows):
+        assert idx13[t].tolist() == [i2, i3]
+    # decode form: only the last position, n-gram windows reach back into context
+    idx_last, _ = oracle.hash_ids(canon, 10, [2, 3], 1, mult, np.array([97, 97]), t_begin=2)
+    assert idx_last.tolist() == [idx[2].tolist()]
+
+
+def test_hash_invalid_canonical_id():
+    canon = np.array([[1, -1, 2, 3]], dtype=np.int32)
+    mult = np.array([[3, 5, 0, 0]], dtype=np.uint64)
+    idx, bad = oracle.hash_ids(canon, 10, [2], 1, mult, np.array([7]))
+    # n-grams containing position 1 (t = 1 and t = 2) are invalid
+    assert bad == 2
+    assert idx[:, 0].tolist()[1:3] == [0xFFFFFFFF, 0xFFFFFFFF]
+    assert idx[0, 0] < 7 and idx[3, 0] < 7
+
+
+@pytest.fixture(scope="module")
+def c1():
+    inp = synth.Inputs(synth.WORKLOADS["c1"])
+    canon, bad = oracle.remap(inp.tok, inp.P)
+    assert bad == 0
+    idx, badh = oracle.hash_ids(canon, inp.wl.Vc, inp.wl.orders, inp.wl.K, inp.mult, inp.rows)
+    assert badh == 0
+    return inp, canon, idx
+
+
+def _ngrams_bruteforce(seq, n, pad):
+    """Naive listing of suffix n-grams (most recent first), padded at the start."""
+    out = []
+    for t in range(len(seq)):
+        out.append(tuple(seq[t - j] if t - j >= 0 else pad for j in range(n)))
+    return out
+
+
+def test_hash_indices_in_range_and_deterministic(c1):
+    inp, canon, idx = c1
+    wl = inp.wl
+    assert idx.shape == (wl.n_tok, wl.J)
+    assert np.all(idx < wl.M)
+    for o, n in enumerate(wl.orders):
+        grams = _ngrams_bruteforce(canon[0].tolist(), n, wl.Vc)
+        seen = {}
+        for t, g in enumerate(grams):
+            tup = tuple(idx[t, o * wl.K:(o + 1) * wl.K].tolist())
+            if g in seen:
+                # equal n-grams at different positions give equal indices
+                assert seen[g] == tup
+            else:
+                seen[g] = tup
+        # distinct n-grams never collide on all K heads at this size
+        assert len(set(seen.values())) == len(seen)
+
+
+def test_hash_collisions_within_birthday_bound():
+    # many distinct n-grams into a small prime table: per-head collision count
+    # near the birthday expectation n_d^2 / (2M)
+    wl = synth.WORKLOADS["c1"].replace(T=4096, B=4)
+    inp = synth.Inputs(wl)
+    canon, _ = oracle.remap(inp.tok, inp.P)
+    M = 10007
+    idx, _ = oracle.hash_ids(canon, wl.Vc, wl.orders, wl.K, inp.mult, np.full(wl.J, M))
+    for o, n in enumerate(wl.orders):
+        distinct = {}
+        for b in range(wl.B):
+            grams = _ngrams_bruteforce(canon[b].tolist(), n, wl.Vc)
+            for t, g in enumerate(grams):
+                distinct.setdefault(g, b * wl.T + t)
+        nd = len(distinct)
+        rows = np.array(list(distinct.values()))
+        expect = nd * (nd - 1) / (2.0 * M)
+        for k in range(wl.K):
+            col = idx[rows, o * wl.K + k]
+            _, counts = np.unique(col, return_counts=True)
+            pairs = float(np.sum(counts * (counts - 1) / 2))
+            assert 0.7 * expect < pairs < 1.3 * expect, (n, k, nd, pairs, expect)
+
+
+def test_hash_depends_only_on_ids(c1):
+    inp, canon, idx = c1
+    # the same ids placed in another sequence slot give the same indices
+    wl = inp.wl
+    two = np.concatenate([canon, canon], axis=0)
+    idx2, _ = oracle.hash_ids(two, wl.Vc, wl.orders, wl.K, inp.mult, inp.rows)
+    assert np.array_equal(idx2[: wl.T], idx) and np.array_equal(idx2[wl.T:], idx)
+
+
+# ------------------------------------------------------------------ gather
+
+def test_gather_matches_numpy_take():
+    rng = np.random.default_rng(3)
+    J, M, D, n = 5, 11, 7, 40
+    tables = rng.standard_normal((J, M, D)).astype(np.float32)
+    idx = rng.integers(0, M, size=(n, J)).astype(np.uint32)
+    idx[3, 2] = M        # out of range -> zero row
+    idx[7, 0] = 0xFFFFFFFF
+    e = oracle.gather(idx, np.full(J, M), tables)
+    want = np.concatenate([np.where((idx[:, j] < M)[:, None], tables[j][np.minimum(idx[:, j], M - 1)], 0)
+                           for j in range(J)], axis=1)
+    assert np.array_equal(e, want)
+    # bit patterns (bf16 stored as uint16) are copied exactly
+    bits = rng.integers(0, 65535, size=(J, M, D)).astype(np.uint16)
+    eb = oracle.gather(idx, np.full(J, M), bits)
+    assert eb.dtype == np.uint16
+    assert np.array_equal(eb[5].reshape(J, D), np.stack([bits[j, idx[5, j]] for j in range(J)]))
+
+
+def test_gather_rows_matches_full_gather(c1):
+    inp, canon, idx = c1
+    tables = inp.all_tables()
+    e_full = oracle.gather(idx, inp.rows, tables)
+    e_rows = oracle.gather_rows(idx, inp.rows, inp.table_rows)
+    assert np.array_equal(e_full, e_rows.astype(np.float32))
+
+
+# ------------------------------------------------------------------ projections
+
+def test_project_matches_numpy_matmul():
+    rng = np.random.default_rng(5)
+    e = rng.standard_normal((9, 13))
+    W = rng.standard_normal((6, 13))
+    np.testing.assert_allclose(oracle.project(e, W), e @ W.T, rtol=1e-12, atol=1e-12)
+
+
+def test_project_identity_returns_e():
+    rng = np.random.default_rng(6)
+    e = rng.standard_normal((4, 8))
+    W = np.vstack([np.eye(8), np.zeros((3, 8))])  # d_mem <= d, W = [I; 0]
+    k = oracle.project(e, W)
+    assert np.array_equal(k[:, :8], e) and np.all(k[:, 8:] == 0)
+
+
+# ------------------------------------------------------------------ gate
+
+def test_gate_orthogonal_is_half():
+    h = np.array([[1.0, 1.0, 0.0, 0.0]])
+    k = np.array([[0.0, 0.0, 1.0, -1.0]])
+    a = oracle.gate(h, k, np.ones(4), np.ones(4), 1e-6)
+    assert a[0] == 0.5
+
+
+@pytest.mark.parametrize("c", [0.3, 1.0, 4.0])
+def test_gate_parallel_closed_form(c):
+    rng = np.random.default_rng(7)
+    d = 64
+    h = rng.standard_normal((1, d))
+    eps = 1e-6
+    m = np.mean(h * h)
+    dot = d * c * m / (math.sqrt(m + eps) * math.sqrt(c * c * m + eps))
+    want = 1.0 / (1.0 + math.exp(-dot / math.sqrt(d)))
+    got = oracle.gate(h, c * h, np.ones(d), np.ones(d), eps)[0]
+    assert abs(got - want) < 1e-14
+    got_neg = oracle.gate(h, -c * h, np.ones(d), np.ones(d), eps)[0]
+    assert abs(got_neg - (1.0 - want)) < 1e-14
+    # with d = 64 the aligned key gives sigma(~8) -> near 1, the opposed one near 0
+    assert got > 0.999 and got_neg < 0.001
+
+
+def test_gate_gains_scale_the_logit():
+    rng = np.random.default_rng(8)
+    d = 32
+    h = rng.standard_normal((3, d))
+    k = rng.standard_normal((3, d))
+    a1 = oracle.gate(h, k, np.ones(d), np.ones(d), 1e-6)
+    a6 = oracle.gate(h, k, np.full(d, 2.0), np.full(d, 3.0), 1e-6)
+    logit = lambda a: np.log(a / (1 - a))
+    np.testing.assert_allclose(logit(a6), 6.0 * logit(a1), rtol=1e-10)
+
+
+def test_gate_in_open_unit_interval():
+    rng = np.random.default_rng(9)
+    a = oracle.gate(rng.standard_normal((200, 48)) * 5, rng.standard_normal((200, 48)),
+                    np.ones(48), np.ones(48), 1e-6)
+    assert np.all(a > 0) and np.all(a < 1)
+
+
+# ------------------------------------------------------------------ conv
+
+def test_conv_matches_numpy_convolve():
+    rng = np.random.default_rng(10)
+    L, d, w = 20, 5, 4
+    vt = rng.standard_normal((L, d))
+    cw = rng.standard_normal((d, w))
+    u = oracle.conv(vt, cw)
+    for c in range(d):
+        np.testing.assert_allclose(u[:, c], np.convolve(vt[:, c], cw[c])[:L], rtol=1e-12, atol=1e-12)
+
+
+def test_conv_impulse_response_and_causality():
+    rng = np.random.default_rng(11)
+    L, d, w = 12, 3, 4
+    cw = rng.standard_normal((d, w))
+    vt = np.zeros((L, d))
+    vt[5] = 1.0
+    u = oracle.conv(vt, cw)
+    for j in range(w):
+        assert np.array_equal(u[5 + j], cw[:, j])
+    assert np.all(u[:5] == 0) and np.all(u[5 + w:] == 0)
+    base = rng.standard_normal((L, d))
+    pert = base.copy()
+    pert[7] += 3.0
+    ub, up = oracle.conv(base, cw), oracle.conv(pert, cw)
+    assert np.array_equal(ub[:7], up[:7])
+    assert not np.allclose(ub[7], up[7])
+
+
+def test_conv_history_equals_concatenation():
+    rng = np.random.default_rng(12)
+    L, d, w = 6, 4, 4
+    cw = rng.standard_normal((d, w))
+    hist = rng.standard_normal((w - 1, d))
+    vt = rng.standard_normal((L, d))
+    u = oracle.conv(vt, cw, hist)
+    u_cat = oracle.conv(np.vstack([hist, vt]), cw)[w - 1:]
+    np.testing.assert_allclose(u, u_cat, rtol=0, atol=1e-15)
+
+
+def test_output_special_cases():
+    assert oracle.silu(0.0) == 0.0
+    assert abs(oracle.silu(1.0) - 0.7310585786300049) < 1e-15
+    assert abs(oracle.silu(40.0) - 40.0) < 1e-12
+    rng = np.random.default_rng(13)
+    vt = rng.standard_normal((8, 3))
+    h = rng.standard_normal((8, 3))
+    zero_u = oracle.conv(vt, np.zeros((3, 4)))
+    assert np.array_equal(oracle.output(vt, zero_u, h, False), vt)        # conv_w = 0 -> Y = v~
+    assert np.array_equal(oracle.output(vt, zero_u, h, True), vt + h)     # plus the residual
+    cw = np.zeros((3, 4))
+    cw[:, 1] = [0.5, -2.0, 1.5]                                            # one-hot tap j = 1
+    y = oracle.output(vt, oracle.conv(vt, cw), h, False)
+    for t in range(1, 8):
+        for c in range(3):
+            x = cw[c, 1] * vt[t - 1, c]
+            assert abs(y[t, c] - (vt[t, c] + x / (1 + math.exp(-x)))) < 1e-14
+
+
+# ------------------------------------------------------------------ bf16 rounding
+
+def test_round_bf16_matches_torch_and_ties():
+    import torch
+    rng = np.random.default_rng(14)
+    x32 = (rng.standard_normal(20000) * rng.choice([1e-3, 1.0, 300.0], 20000)).astype(np.float32)
+    want = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_bf16(x32.astype(np.float64)), want)
+    # ties to even: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7
+    assert oracle.round_bf16(1.0 + 2.0 ** -8) == 1.0
+    assert oracle.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert oracle.round_bf16(-(1.0 + 3 * 2.0 ** -8)) == -(1.0 + 2.0 ** -6)
+    # a double just above the tie rounds up (no double rounding through fp32)
+    assert oracle.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -40) == 1.0 + 2.0 ** -7
+
+
+# ------------------------------------------------------------------ whole path
+
+def test_forward_full_c1_properties(c1):
+    inp, canon, idx = c1
+    r = oracle.forward_full(inp)
+    assert np.array_equal(r.idx, idx)
+    assert np.all(r.alpha > 0) and np.all(r.alpha < 1)
+    # the gate is not saturated on these inputs
+    assert 0.05 < np.std(r.alpha) < 0.45
+    assert np.all(np.isfinite(r.y))
+    assert np.max(np.abs(r.y)) < 4.0
+
+
+def test_forward_rows_equals_forward_full(c1):
+    inp, _, _ = c1
+    full = oracle.forward_full(inp, add_residual=True)
+    pos = synth.sample_positions(inp.wl, 24, seed=1)
+    rows = oracle.forward_rows(inp, pos, add_residual=True)
+    np.testing.assert_allclose(rows.y, full.y[pos], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(rows.alpha, full.alpha[pos], rtol=0, atol=1e-15)
+
+
+def test_decode_step_equals_last_prefill_row(c1):
+    inp, _, _ = c1
+    wl = inp.wl
+    full = oracle.forward_full(inp)
+    dec_wl = wl.replace(t_begin=wl.T - 1)
+    dec = synth.Inputs(dec_wl)
+    hist = full.vt[None, wl.T - wl.w:wl.T - 1]        # the last w-1 gated rows before t = T-1
+    dec.hidden_rows = lambda rows: inp.hidden_rows(np.asarray(rows) + (wl.T - 1))
+    r = oracle.forward_rows(dec, np.array([0]), hist=hist)
+    np.testing.assert_allclose(r.y[0], full.y[wl.T - 1], rtol=0, atol=1e-12)
