@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Engram forward benchmark on B200.
+
+One step = the whole forward (remap + hash, gather, W_K/W_V projections with
+gate partials, gate + causal conv) over one batch of the workload, through
+the C ABI.  Default workload: B=4 sequences x 4096 tokens, 16 tables of
+1000003 x 64 bf16 (about 2 GB), d_mem 1024, d 2560, conv width 4.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs an independent replica (no collective on the
+data path: the forward shards by sequence); timing is the max over ranks.
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "Engram forward tokens/sec on 1 B200; gather HBM GB/s as % of ~8 TB/s peak"
+L2_FLUSH_BYTES = 256 << 20
+SPEC_HBM_GBS = 8000.0
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def describe(wl) -> str:
+    return (f"{wl.name}: B={wl.B} T={wl.T} t_begin={wl.t_begin}, V={wl.V}->V'={wl.Vc}, Zipf s={wl.zipf_s}, "
+            f"orders {list(wl.orders)} x K={wl.K} ({wl.J} tables of {wl.M} x {wl.D} {wl.dtype}), "
+            f"d_mem={wl.d_mem}, d={wl.d}, conv w={wl.w}")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(self.period)
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            self.samples.append((mhz, int(rs)))
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        if not self.samples:
+            self.sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"], "samples": 0}
+        mhz = sorted(s[0] for s in self.samples)
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- oracle timing (CPU)
+
+def oracle_sample_time(wl, n_tokens: int):
+    """Time the oracle (single-threaded, as it stands) on the first n_tokens of
+    sequence 0 of the workload.  Untimed preparation: the table rows the sample
+    touches are fetched from the seeded generator into compact host tables
+    (the sample's indices remapped to them)."""
+    import oracle
+    sw = wl.replace(B=1, T=n_tokens, t_begin=0)
+    inp = synth.Inputs(sw)
+    canon, _ = oracle.remap(inp.tok, inp.P)
+    idx, _ = oracle.hash_ids(canon, sw.Vc, sw.orders, sw.K, inp.mult, inp.rows)
+    U = []
+    idx_c = np.empty_like(idx)
+    for j in range(sw.J):
+        u, inv = np.unique(idx[:, j], return_inverse=True)
+        U.append(u)
+        idx_c[:, j] = inv
+    umax = max(len(u) for u in U)
+    compact = np.zeros((sw.J, umax, sw.D), dtype=np.float32)
+    for j in range(sw.J):
+        compact[j, :len(U[j])] = inp.table_rows(j, U[j])
+    rows_c = np.array([len(u) for u in U], dtype=np.uint32)
+    h = inp.all_hidden()
+    t0 = time.perf_counter()
+    canon, _ = oracle.remap(inp.tok, inp.P)
+    idx, _ = oracle.hash_ids(canon, sw.Vc, sw.orders, sw.K, inp.mult, inp.rows)
+    e = oracle.gather(idx_c, rows_c, compact)
+    k = oracle.project(e, inp.Wk)
+    v = oracle.project(e, inp.Wv)
+    if sw.dtype == "bf16":
+        v = oracle.round_bf16(v)
+    alpha = oracle.gate(h, k, inp.gq, inp.gk, 1e-6)
+    vt = alpha[:, None] * v
+    u = oracle.conv(vt, inp.conv_w)
+    oracle.output(vt, u, h, True)
+    return time.perf_counter() - t0
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    n = args.ref_tokens
+    if n <= 0:
+        # size each step so that warm-up + timed steps take about 90 s
+        rate = 16 / oracle_sample_time(wl, 16)
+        n = int(max(8, min(1024, rate * 90.0 / (args.steps + args.warmup))))
+    for _ in range(args.warmup):
+        oracle_sample_time(wl, n)
+    ts = [oracle_sample_time(wl, n) for _ in range(args.steps)]
+    sec = float(np.mean(ts))
+    val = n / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(wl), "sample": f"first {n} tokens of sequence 0 per step"},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {n} tokens of sequence 0, single-threaded fp64 C++ oracle"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c2", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--cpu-tokens", type=int, default=2048, help="oracle sample for cpu_baseline")
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="oracle sample per reference step (0: sized so the run takes about 90 s)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_02_b200 as eb
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = synth.WORKLOADS[args.workload]
+    if world > 1:
+        wl = wl.replace(seed=wl.seed + 1000 * rank)   # each replica its own batch
+    inp = synth.Inputs(wl)
+    dd = inp.device_dense(dev)
+    tables = inp.device_tables(dev)
+    h = inp.device_hidden(dev)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    es = 2 if wl.dtype == "bf16" else 4
+    cfg = eb.make_config(orders=wl.orders, heads=wl.K, rows=[int(x) for x in inp.rows], mult=inp.mult,
+                         row_dim=wl.D, hidden=wl.d, conv_width=wl.w, vocab=wl.V, canon_vocab=wl.Vc,
+                         dtype=eb.ENGRAM_BF16 if wl.dtype == "bf16" else eb.ENGRAM_F32)
+    eng = eb.Engram(cfg, max_tok=wl.n_tok)
+    n = wl.n_tok
+    y = torch.empty(n, wl.d, dtype=tdt, device=dev)
+    state = (torch.zeros(wl.B, wl.w - 1, wl.d, dtype=torch.float32, device=dev) if wl.t_begin > 0 else None)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        eng.forward(dd["tok"], dd["P"], tables, h, dd["Wk"], dd["Wv"], dd["conv_w"], y, t_begin=wl.t_begin,
+                    gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, flags = eng.status()
+    if st != eb.ENGRAM_OK:
+        raise RuntimeError(f"device status {st} flags {flags:#x} after warm-up")
+
+    # ---- timed: K whole steps, L2 flushed before each (outside the events)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = n * world / (ms / 1e3)
+    launches = 4 * K
+
+    # ---- per-kernel durations (same workload, decomposed entry points)
+    idx = torch.empty(n, wl.J, dtype=torch.int32, device=dev)
+    e = torch.empty(n, wl.d_mem, dtype=tdt, device=dev)
+    v = torch.empty(n, wl.d, dtype=tdt, device=dev)
+    G = (wl.d + 127) // 128
+    part = torch.empty(n, G, 4, dtype=torch.float32, device=dev)
+    names = ["hash", "gather", "project", "gate_conv"]
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in names]
+           for _ in range(K)]
+    L = wl.T - wl.t_begin
+    for i in range(K + args.warmup):
+        flush.zero_()
+        rec = kev[i - args.warmup] if i >= args.warmup else None
+        calls = [
+            lambda: eb.engram_hash(eng.ctx, dd["tok"], dd["P"], wl.B, wl.T, wl.T, wl.t_begin, idx),
+            lambda: eb.engram_gather(eng.ctx, idx, n, tables, e),
+            lambda: eb.engram_project(eng.ctx, e, n, h, dd["Wk"], dd["Wv"], dd["gq"], dd["gk"], v, part),
+            lambda: eb.engram_conv(eng.ctx, v, part, h, dd["conv_w"], wl.B, L, state, y, None, 1),
+        ]
+        for j, c in enumerate(calls):
+            if rec:
+                rec[j][0].record(stream)
+            c()
+            if rec:
+                rec[j][1].record(stream)
+    torch.cuda.synchronize()
+    kms = {nm: float(np.mean([kev[i][j][0].elapsed_time(kev[i][j][1]) for i in range(K)]))
+           for j, nm in enumerate(names)}
+
+    hbm, tf_burst, tf_sust, peak_src = _peaks()
+    flops = 2.0 * n * wl.d_mem * 2 * wl.d
+    gemm_tflops = flops / (kms["project"] / 1e3) / 1e12
+    gather_bytes = n * wl.J * 4 + 2.0 * n * wl.d_mem * es          # idx read + rows read + e write
+    gather_gbs = gather_bytes / (kms["gather"] / 1e3) / 1e9
+    conv_bytes = n * (2.0 * wl.d * es + G * 16 + wl.d * es)         # v read + partials + Y write
+    if True:  # add_residual reads h
+        conv_bytes += n * wl.d * es
+    conv_gbs = conv_bytes / (kms["gate_conv"] / 1e3) / 1e9
+    dominant = max(kms, key=kms.get)
+    roofline = {"kernel": "project (W_K/W_V tcgen05 GEMM + gate partials)", "bound": "tensor",
+                "achieved": gemm_tflops, "peak": tf_burst, "unit": "TFLOP/s", "frac": gemm_tflops / tf_burst,
+                "traffic": None, "peak_source": f"{peak_src} bf16 burst",
+                "algorithmic": f"2*n*d_mem*2d = {flops:.4g} FLOP per launch"}
+
+    # ---- end to end through the public API: pinned host inputs in, host Y out
+    tok_h = torch.from_numpy(inp.tok).pin_memory()
+    h_h = h.cpu().pin_memory()
+    y_h = torch.empty(n, wl.d, dtype=tdt).pin_memory()
+    tok_d = torch.empty_like(dd["tok"])
+    h_d = torch.empty_like(h)
+    Ke = max(3, min(K, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    for i in range(Ke + 3):
+        flush.zero_()
+        if i >= 3:
+            e2e_ev[i - 3][0].record(stream)
+        tok_d.copy_(tok_h, non_blocking=True)
+        h_d.copy_(h_h, non_blocking=True)
+        eng.forward(tok_d, dd["P"], tables, h_d, dd["Wk"], dd["Wv"], dd["conv_w"], y, t_begin=wl.t_begin,
+                    gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
+        y_h.copy_(y, non_blocking=True)
+        if i >= 3:
+            e2e_ev[i - 3][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in e2e_ev]))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": n * world / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(tok_h.numel() * 4 + h_h.numel() * es),
+           "d2h_bytes_per_step": int(y_h.numel() * es), "ms_per_step": e2e_ms,
+           "path": "pinned host tok+h -> device (cudaMemcpyAsync) -> engram_forward -> Y to pinned host"}
+
+    st, flags = eng.status()
+    if st != eb.ENGRAM_OK:
+        raise RuntimeError(f"device status {st} flags {flags:#x} after timing")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec = oracle_sample_time(wl, args.cpu_tokens)
+        cpu = {"value": args.cpu_tokens / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {args.cpu_tokens} tokens of sequence 0 ({sec:.1f} s), single-threaded fp64 C++"}
+
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic: seeded Zipf tokens, counter-based N(0,s^2) tables/hidden/weights",
+        "config": {"workload": describe(wl), "B": wl.B, "seq_len": wl.T, "tokens_per_step": n * world,
+                   "parallelism": f"replicas x{world} (no collective)",
+                   "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write outside the events)"},
+        "roofline": roofline,
+        "gather": {"achieved_gbs": gather_gbs, "frac_of_8000": gather_gbs / SPEC_HBM_GBS,
+                   "frac_of_measured": gather_gbs / hbm, "bytes_per_launch": gather_bytes},
+        "gate_conv": {"achieved_gbs": conv_gbs, "frac_of_measured": conv_gbs / hbm, "bytes_per_launch": conv_bytes},
+        "kernels_ms": kms, "dominant_kernel": dominant,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

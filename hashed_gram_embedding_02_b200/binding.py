@@ -1,0 +1,192 @@
+"""ctypes binding of libengram.so: same names as the C ABI, argument
+marshalling only.
+
+Tensors are torch tensors on the context's device (PyTorch provides device
+memory and streams); every step of the path runs in the library's kernels.
+Each wrapper raises :class:`EngramError` when the C call returns a non-zero
+status.  Importing this module without the built library raises at once:
+there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libengram.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m hashed_gram_embedding_02_b200.build` "
+                      "or __graft_entry__.build(); the Engram path has no CPU fallback")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+ENGRAM_OK, ENGRAM_E_INVAL, ENGRAM_E_CUDA, ENGRAM_E_NOMEM, ENGRAM_E_UNSUPPORTED, ENGRAM_E_TIMEOUT, \
+    ENGRAM_E_HOST, ENGRAM_E_DEVICE = range(8)
+ENGRAM_F32, ENGRAM_BF16 = 0, 1
+ENGRAM_ERR_TOKEN, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+ENGRAM_INVALID_INDEX = 0xFFFFFFFF
+ENGRAM_MAX_TABLES = 32
+ENGRAM_PART_GROUP = 128
+
+# exported symbol names declared in include/engram.h
+EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_error", "engram_workspace_bytes",
+           "engram_device_status", "engram_remap", "engram_hash", "engram_gather", "engram_project",
+           "engram_conv", "engram_gate_conv", "engram_forward")
+
+
+class engram_config(ctypes.Structure):
+    _fields_ = [
+        ("n_orders", ctypes.c_int32),
+        ("orders", ctypes.c_int32 * 4),
+        ("heads", ctypes.c_int32),
+        ("rows", ctypes.c_uint32 * ENGRAM_MAX_TABLES),
+        ("mult", (ctypes.c_uint64 * 4) * ENGRAM_MAX_TABLES),
+        ("row_dim", ctypes.c_int32),
+        ("hidden", ctypes.c_int32),
+        ("conv_width", ctypes.c_int32),
+        ("vocab", ctypes.c_int32),
+        ("canon_vocab", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("eps", ctypes.c_float),
+    ]
+
+
+class EngramError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.engram_strerror(status).decode()
+        detail = _lib.engram_last_error().decode()
+        super().__init__(f"{where}: {msg}" + (f" ({detail})" if detail else ""))
+
+
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_st = ctypes.c_int
+_sigs = {
+    "engram_create": ([ctypes.POINTER(engram_config), ctypes.POINTER(_vp)], _st),
+    "engram_destroy": ([_vp], None),
+    "engram_strerror": ([_st], ctypes.c_char_p),
+    "engram_last_error": ([], ctypes.c_char_p),
+    "engram_workspace_bytes": ([_vp, _i64], _sz),
+    "engram_device_status": ([_vp, _vp, ctypes.POINTER(ctypes.c_uint32)], _st),
+    "engram_remap": ([_vp, _vp, _i64, _vp, _vp, _vp], _st),
+    "engram_hash": ([_vp, _vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp], _st),
+    "engram_gather": ([_vp, _vp, _i64, _vp, _vp, _vp], _st),
+    "engram_project": ([_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _st),
+    "engram_conv": ([_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp], _st),
+    "engram_gate_conv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _sz, _vp],
+                         _st),
+    "engram_forward": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                        _i32, _vp, _sz, _vp], _st),
+}
+for _name, (_args, _res) in _sigs.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a tensor (None for None)."""
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, where: str):
+    if status != ENGRAM_OK:
+        raise EngramError(status, where)
+
+
+def make_config(orders: Sequence[int], heads: int, rows: Sequence[int], mult, row_dim: int, hidden: int,
+                conv_width: int, vocab: int, canon_vocab: int, dtype: int, eps: float = 1e-6) -> engram_config:
+    cfg = engram_config()
+    cfg.n_orders = len(orders)
+    for i, n in enumerate(orders):
+        cfg.orders[i] = int(n)
+    cfg.heads = heads
+    for j, m in enumerate(rows):
+        cfg.rows[j] = int(m)
+    for j in range(len(rows)):
+        for q in range(4):
+            cfg.mult[j][q] = int(mult[j][q])
+    cfg.row_dim, cfg.hidden, cfg.conv_width = row_dim, hidden, conv_width
+    cfg.vocab, cfg.canon_vocab, cfg.dtype, cfg.eps = vocab, canon_vocab, dtype, eps
+    return cfg
+
+
+# ---------------------------------------------------------------- C ABI, same names
+
+def engram_create(cfg: engram_config) -> int:
+    ctx = _vp()
+    _check(_lib.engram_create(ctypes.byref(cfg), ctypes.byref(ctx)), "engram_create")
+    return ctx.value
+
+
+def engram_destroy(ctx: int) -> None:
+    _lib.engram_destroy(ctx)
+
+
+def engram_strerror(status: int) -> str:
+    return _lib.engram_strerror(status).decode()
+
+
+def engram_last_error() -> str:
+    return _lib.engram_last_error().decode()
+
+
+def engram_workspace_bytes(ctx: int, n_tok: int) -> int:
+    return int(_lib.engram_workspace_bytes(ctx, n_tok))
+
+
+def engram_device_status(ctx: int, stream=None):
+    """Returns (status, flags); does not raise."""
+    flags = ctypes.c_uint32(0)
+    st = _lib.engram_device_status(ctx, _stream(stream), ctypes.byref(flags))
+    return int(st), int(flags.value)
+
+
+def engram_remap(ctx, tok, n, P, canon, stream=None):
+    _check(_lib.engram_remap(ctx, _ptr(tok), n, _ptr(P), _ptr(canon), _stream(stream)), "engram_remap")
+
+
+def engram_hash(ctx, ids, P, B, T, stride, t_begin, idx, stream=None):
+    _check(_lib.engram_hash(ctx, _ptr(ids), _ptr(P), B, T, stride, t_begin, _ptr(idx), _stream(stream)),
+           "engram_hash")
+
+
+def engram_gather(ctx, idx, n_tok, tables, e_cat, stream=None):
+    _check(_lib.engram_gather(ctx, _ptr(idx), n_tok, _ptr(tables), _ptr(e_cat), _stream(stream)), "engram_gather")
+
+
+def engram_project(ctx, e_cat, n_tok, h, Wk, Wv, gq, gk, v, part, stream=None):
+    _check(_lib.engram_project(ctx, _ptr(e_cat), n_tok, _ptr(h), _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(v),
+                               _ptr(part), _stream(stream)), "engram_project")
+
+
+def engram_conv(ctx, v, part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, stream=None):
+    _check(_lib.engram_conv(ctx, _ptr(v), _ptr(part), _ptr(h), _ptr(conv_w), B, L, _ptr(conv_state), _ptr(y),
+                            _ptr(alpha_out), int(add_residual), _stream(stream)), "engram_conv")
+
+
+def engram_gate_conv(ctx, e_cat, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual,
+                     workspace, workspace_bytes, stream=None):
+    _check(_lib.engram_gate_conv(ctx, _ptr(e_cat), _ptr(h), _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w),
+                                 B, L, _ptr(conv_state), _ptr(y), _ptr(alpha_out), int(add_residual),
+                                 _ptr(workspace), workspace_bytes, _stream(stream)), "engram_gate_conv")
+
+
+def engram_forward(ctx, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
+                   alpha_out, add_residual, workspace, workspace_bytes, stream=None):
+    _check(_lib.engram_forward(ctx, _ptr(tok), B, T, tok_stride, t_begin, _ptr(P), _ptr(tables), _ptr(h), _ptr(Wk),
+                               _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w), _ptr(conv_state), _ptr(y),
+                               _ptr(alpha_out), int(add_residual), _ptr(workspace), workspace_bytes,
+                               _stream(stream)), "engram_forward")

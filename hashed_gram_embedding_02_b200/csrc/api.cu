@@ -1,0 +1,366 @@
+// C ABI of the Engram forward path: argument checks, workspace layout and
+// kernel sequencing.  Every entry point validates on the host and launches
+// nothing on error; kernels report data errors through the context's device
+// status word instead of trapping.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+
+using namespace engram;
+
+struct engram_ctx {
+    engram_config cfg;
+    int device;
+    int num_sms;
+    bool sm100;
+    int J;
+    int d_mem;
+    int G;
+    int es;                 // element size of the storage dtype
+    HashParams hp;
+    GatherParams gp;
+    uint32_t* d_status;     // device status word (256-byte block)
+};
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+void set_error(const char* what, cudaError_t e) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+}
+
+void set_error(const char* what) { std::snprintf(g_last_error, sizeof(g_last_error), "%s", what); }
+
+engram_status inval(const char* what) {
+    set_error(what);
+    return ENGRAM_E_INVAL;
+}
+
+engram_status cuda_fail(const char* what, cudaError_t e) {
+    set_error(what, e);
+    return ENGRAM_E_CUDA;
+}
+
+bool is_prime_u32(uint32_t n) {
+    if (n < 2) return false;
+    if (n % 2 == 0) return n == 2;
+    for (uint32_t f = 3; (uint64_t)f * f <= n; f += 2)
+        if (n % f == 0) return false;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Workspace {
+    uint32_t* idx;
+    void* e;
+    void* v;
+    float* part;
+    size_t bytes;
+};
+
+size_t idx_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->J * sizeof(uint32_t)); }
+size_t e_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->d_mem * c->es); }
+size_t v_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->cfg.hidden * c->es); }
+size_t part_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->G * 4 * sizeof(float)); }
+
+Workspace carve(const engram_ctx* c, void* base, int64_t n, bool with_idx_e) {
+    Workspace w{};
+    char* p = static_cast<char*>(base);
+    if (with_idx_e) {
+        w.idx = reinterpret_cast<uint32_t*>(p);
+        p += idx_bytes(c, n);
+        w.e = p;
+        p += e_bytes(c, n);
+    }
+    w.v = p;
+    p += v_bytes(c, n);
+    w.part = reinterpret_cast<float*>(p);
+    p += part_bytes(c, n);
+    w.bytes = (size_t)(p - static_cast<char*>(base));
+    return w;
+}
+
+engram_status check_device(const engram_ctx* c) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev != c->device) return inval("the current device is not the context's device");
+    return ENGRAM_OK;
+}
+
+engram_status launched(const char* what, cudaError_t e) {
+    if (e != cudaSuccess) return cuda_fail(what, e);
+    return ENGRAM_OK;
+}
+
+engram_status project_impl(engram_ctx* c, const void* e_cat, int64_t n, const void* h, const void* Wk,
+                           const void* Wv, const float* gq, const float* gk, void* v, float* part,
+                           cudaStream_t s) {
+    const bool bf16 = c->cfg.dtype == ENGRAM_BF16;
+    if (bf16 && c->sm100 && project_tc_supported(n, c->d_mem, c->cfg.hidden)) {
+        return launched("tcgen05 projection launch",
+                        launch_project_tc(e_cat, n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, v, part,
+                                          c->d_status, c->num_sms, s));
+    }
+    return launched("projection launch", launch_project_simt(bf16, e_cat, n, c->d_mem, h, Wk, Wv, gq, gk,
+                                                             c->cfg.hidden, v, part, s));
+}
+
+engram_status conv_impl(engram_ctx* c, const void* v, const float* part, const void* h, const float* conv_w,
+                        int32_t B, int32_t L, float* state, void* y, float* alpha_out, int32_t add_residual,
+                        cudaStream_t s) {
+    return launched("gate/conv launch",
+                    launch_gate_conv(c->cfg.dtype == ENGRAM_BF16, v, part, h, conv_w, B, L, c->cfg.hidden,
+                                     c->cfg.conv_width, c->cfg.eps, state, y, alpha_out, add_residual, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* engram_last_error(void) { return g_last_error; }
+
+const char* engram_strerror(engram_status s) {
+    switch (s) {
+        case ENGRAM_OK: return "ok";
+        case ENGRAM_E_INVAL: return "invalid argument";
+        case ENGRAM_E_CUDA: return "CUDA runtime error";
+        case ENGRAM_E_NOMEM: return "out of memory or workspace too small";
+        case ENGRAM_E_UNSUPPORTED: return "unsupported";
+        case ENGRAM_E_TIMEOUT: return "device wait timed out";
+        case ENGRAM_E_HOST: return "host-tier failure";
+        case ENGRAM_E_DEVICE: return "device reported a data error";
+    }
+    return "unknown status";
+}
+
+engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
+    if (!cfg || !out) return inval("null config or output pointer");
+    *out = nullptr;
+    const engram_config& k = *cfg;
+    if (k.n_orders < 1 || k.n_orders > 4) return inval("n_orders must be in 1..4");
+    int max_order = 0;
+    for (int o = 0; o < k.n_orders; ++o) {
+        if (k.orders[o] < 1 || k.orders[o] > 4) return inval("each order must be in 1..4");
+        if (o > 0 && k.orders[o] <= k.orders[o - 1]) return inval("orders must be strictly ascending");
+        if (k.orders[o] > max_order) max_order = k.orders[o];
+    }
+    if (k.heads < 1) return inval("heads must be >= 1");
+    const int J = k.n_orders * k.heads;
+    if (J > ENGRAM_MAX_TABLES) return inval("n_orders * heads must be <= 32");
+    for (int j = 0; j < J; ++j) {
+        if (k.rows[j] >= 0x80000000u || !is_prime_u32(k.rows[j])) return inval("every table size must be a prime < 2^31");
+    }
+    if (k.dtype != ENGRAM_F32 && k.dtype != ENGRAM_BF16) return inval("unknown dtype");
+    const int es = k.dtype == ENGRAM_F32 ? 4 : 2;
+    if (k.row_dim < 1 || ((int64_t)k.row_dim * es) % 16 != 0) return inval("row_dim * element size must be a multiple of 16 bytes");
+    if (k.hidden < 8 || k.hidden % 8 != 0) return inval("hidden must be a positive multiple of 8");
+    if (k.conv_width < 1 || k.conv_width > kMaxConv) return inval("conv_width must be in 1..8");
+    if (k.vocab < 1) return inval("vocab must be >= 1");
+    if (k.canon_vocab < 1 || k.canon_vocab >= 0x7FFFFFFF) return inval("canon_vocab must be in [1, 2^31 - 1)");
+    if (!(k.eps >= 0.f) || !std::isfinite(k.eps)) return inval("eps must be finite and >= 0");
+
+    engram_ctx* c = new (std::nothrow) engram_ctx();
+    if (!c) return ENGRAM_E_NOMEM;
+    c->cfg = k;
+    c->J = J;
+    c->es = es;
+    c->d_mem = J * k.row_dim;
+    c->G = (k.hidden + kGroup - 1) / kGroup;
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e != cudaSuccess) {
+        delete c;
+        return cuda_fail("cudaGetDevice", e);
+    }
+    int major = 0;
+    cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, c->device);
+    c->sm100 = (major == 10);
+
+    std::memset(&c->hp, 0, sizeof(c->hp));
+    for (int j = 0; j < J; ++j) {
+        for (int q = 0; q < 4; ++q) c->hp.mult[j][q] = k.mult[j][q];
+        c->hp.rows[j] = k.rows[j];
+    }
+    for (int o = 0; o < 4; ++o) c->hp.orders[o] = o < k.n_orders ? k.orders[o] : 0;
+    c->hp.n_orders = k.n_orders;
+    c->hp.K = k.heads;
+    c->hp.J = J;
+    c->hp.max_order = max_order;
+    c->hp.V = k.vocab;
+    c->hp.Vc = k.canon_vocab;
+
+    std::memset(&c->gp, 0, sizeof(c->gp));
+    int64_t off = 0;
+    for (int j = 0; j < J; ++j) {
+        c->gp.row_off[j] = off;
+        c->gp.rows[j] = k.rows[j];
+        off += k.rows[j];
+    }
+    c->gp.J = J;
+    c->gp.chunks_per_row = k.row_dim * es / 16;
+
+    e = cudaMalloc(&c->d_status, 256);
+    if (e != cudaSuccess) {
+        delete c;
+        return e == cudaErrorMemoryAllocation ? ENGRAM_E_NOMEM : cuda_fail("cudaMalloc status", e);
+    }
+    e = cudaMemset(c->d_status, 0, 256);
+    if (e != cudaSuccess) {
+        cudaFree(c->d_status);
+        delete c;
+        return cuda_fail("cudaMemset status", e);
+    }
+    *out = c;
+    return ENGRAM_OK;
+}
+
+void engram_destroy(engram_ctx* c) {
+    if (!c) return;
+    if (c->d_status) cudaFree(c->d_status);
+    delete c;
+}
+
+size_t engram_workspace_bytes(const engram_ctx* c, int64_t n_tok) {
+    if (!c || n_tok < 0) return 0;
+    return idx_bytes(c, n_tok) + e_bytes(c, n_tok) + v_bytes(c, n_tok) + part_bytes(c, n_tok);
+}
+
+engram_status engram_device_status(engram_ctx* c, cudaStream_t s, uint32_t* flags) {
+    if (!c) return inval("null context");
+    uint32_t h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, c->d_status, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail("reading the device status word", e);
+    if (h) {
+        e = cudaMemsetAsync(c->d_status, 0, sizeof(uint32_t), s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail("clearing the device status word", e);
+    }
+    if (flags) *flags = h;
+    if (h & ENGRAM_ERR_TIMEOUT) return ENGRAM_E_TIMEOUT;
+    return h ? ENGRAM_E_DEVICE : ENGRAM_OK;
+}
+
+engram_status engram_remap(engram_ctx* c, const int32_t* tok, int64_t n, const int32_t* P, int32_t* canon,
+                           cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (n < 0) return inval("n must be >= 0");
+    if (n > 0 && (!tok || !P || !canon)) return inval("null tensor pointer");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    return launched("remap launch", launch_remap(tok, n, P, c->cfg.vocab, canon, c->d_status, s));
+}
+
+engram_status engram_hash(engram_ctx* c, const int32_t* ids, const int32_t* P, int32_t B, int32_t T,
+                          int64_t stride, int32_t t_begin, uint32_t* idx, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (B < 0 || T < 0 || t_begin < 0 || t_begin > T) return inval("need B >= 0 and 0 <= t_begin <= T");
+    if (stride < T) return inval("stride must be >= T");
+    if ((int64_t)B * (T - t_begin) == 0) return ENGRAM_OK;
+    if (!ids || !idx) return inval("null tensor pointer");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    return launched("hash launch", launch_hash(ids, P, B, T, stride, t_begin, idx, c->hp, c->d_status, s));
+}
+
+engram_status engram_gather(engram_ctx* c, const uint32_t* idx, int64_t n_tok, const void* tables,
+                            void* e_cat, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (n_tok < 0) return inval("n_tok must be >= 0");
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!idx || !tables || !e_cat) return inval("null tensor pointer");
+    if (!aligned16(tables) || !aligned16(e_cat)) return inval("tables and e_cat must be 16-byte aligned");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    return launched("gather launch", launch_gather(idx, n_tok, tables, c->gp, e_cat, c->d_status, c->num_sms, s));
+}
+
+engram_status engram_project(engram_ctx* c, const void* e_cat, int64_t n_tok, const void* h, const void* Wk,
+                             const void* Wv, const float* gq, const float* gk, void* v, float* part,
+                             cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (n_tok < 0) return inval("n_tok must be >= 0");
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!e_cat || !h || !Wk || !Wv || !v || !part) return inval("null tensor pointer");
+    if (!aligned16(e_cat) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(v) || !aligned16(part))
+        return inval("e_cat, h, Wk, Wv, v and part must be 16-byte aligned");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    return project_impl(c, e_cat, n_tok, h, Wk, Wv, gq, gk, v, part, s);
+}
+
+engram_status engram_conv(engram_ctx* c, const void* v, const float* part, const void* h, const float* conv_w,
+                          int32_t B, int32_t L, float* conv_state, void* y, float* alpha_out,
+                          int32_t add_residual, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (B < 0 || L < 0) return inval("B and L must be >= 0");
+    if ((int64_t)B * L == 0) return ENGRAM_OK;
+    if (!v || !part || !conv_w || !y || (add_residual && !h)) return inval("null tensor pointer");
+    if (!aligned16(v) || !aligned16(part) || !aligned16(y) || (add_residual && !aligned16(h)) ||
+        (conv_state && !aligned16(conv_state)))
+        return inval("v, part, y, h and conv_state must be 16-byte aligned");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    return conv_impl(c, v, part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, s);
+}
+
+engram_status engram_gate_conv(engram_ctx* c, const void* e_cat, const void* h, const void* Wk, const void* Wv,
+                               const float* gq, const float* gk, const float* conv_w, int32_t B, int32_t L,
+                               float* conv_state, void* y, float* alpha_out, int32_t add_residual,
+                               void* workspace, size_t workspace_bytes, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (B < 0 || L < 0) return inval("B and L must be >= 0");
+    const int64_t n = (int64_t)B * L;
+    if (n == 0) return ENGRAM_OK;
+    if (!e_cat || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    Workspace w = carve(c, workspace, n, false);
+    if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
+    if (!aligned16(e_cat) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
+        (conv_state && !aligned16(conv_state)))
+        return inval("e_cat, h, Wk, Wv, y and conv_state must be 16-byte aligned");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    st = project_impl(c, e_cat, n, h, Wk, Wv, gq, gk, w.v, w.part, s);
+    if (st != ENGRAM_OK) return st;
+    return conv_impl(c, w.v, w.part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, s);
+}
+
+engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
+                             int32_t t_begin, const int32_t* P, const void* tables, const void* h, const void* Wk,
+                             const void* Wv, const float* gq, const float* gk, const float* conv_w,
+                             float* conv_state, void* y, float* alpha_out, int32_t add_residual, void* workspace,
+                             size_t workspace_bytes, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (B < 0 || T < 0 || t_begin < 0 || t_begin > T) return inval("need B >= 0 and 0 <= t_begin <= T");
+    if (tok_stride < T) return inval("tok_stride must be >= T");
+    const int32_t L = T - t_begin;
+    const int64_t n = (int64_t)B * L;
+    if (n == 0) return ENGRAM_OK;
+    if (!tok || !P || !tables || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    Workspace w = carve(c, workspace, n, true);
+    if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
+    if (!aligned16(tables) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
+        (conv_state && !aligned16(conv_state)))
+        return inval("tables, h, Wk, Wv, y and conv_state must be 16-byte aligned");
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    st = launched("hash launch", launch_hash(tok, P, B, T, tok_stride, t_begin, w.idx, c->hp, c->d_status, s));
+    if (st != ENGRAM_OK) return st;
+    st = launched("gather launch", launch_gather(w.idx, n, tables, c->gp, w.e, c->d_status, c->num_sms, s));
+    if (st != ENGRAM_OK) return st;
+    st = project_impl(c, w.e, n, h, Wk, Wv, gq, gk, w.v, w.part, s);
+    if (st != ENGRAM_OK) return st;
+    return conv_impl(c, w.v, w.part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, s);
+}
+
+}  // extern "C"

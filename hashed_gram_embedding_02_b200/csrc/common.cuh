@@ -1,0 +1,111 @@
+// Internal declarations shared by the Engram CUDA kernels and the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "engram.h"
+
+namespace engram {
+
+constexpr int kMaxTables = ENGRAM_MAX_TABLES;
+constexpr int kGroup = ENGRAM_PART_GROUP;   // channels per gate-partial group
+constexpr int kMaxConv = 8;
+
+// Hash configuration passed by value to the hash kernel (about 1.2 KB of
+// kernel parameters; dynamic indexing reads the constant bank).
+struct HashParams {
+    uint64_t mult[kMaxTables][4];
+    uint32_t rows[kMaxTables];
+    int32_t orders[4];
+    int32_t n_orders;
+    int32_t K;
+    int32_t J;
+    int32_t max_order;
+    int32_t V;
+    int32_t Vc;
+};
+
+// Table geometry passed by value to the gather kernel.
+struct GatherParams {
+    int64_t row_off[kMaxTables];   // first row of table j in the back-to-back table buffer
+    uint32_t rows[kMaxTables];
+    int32_t J;
+    int32_t chunks_per_row;        // 16-byte chunks per table row
+};
+
+// ---------------------------------------------------------------- launches
+// Each returns cudaGetLastError() of its launch.
+cudaError_t launch_remap(const int32_t* tok, int64_t n, const int32_t* P, int32_t V, int32_t* canon,
+                         uint32_t* status, cudaStream_t s);
+cudaError_t launch_hash(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
+                        int32_t t_begin, uint32_t* idx, const HashParams& hp, uint32_t* status,
+                        cudaStream_t s);
+cudaError_t launch_gather(const uint32_t* idx, int64_t n_tok, const void* tables, const GatherParams& gp,
+                          void* e_cat, uint32_t* status, int num_sms, cudaStream_t s);
+// CUDA-core projection (fp32 or bf16 operands, fp32 accumulation)
+cudaError_t launch_project_simt(bool bf16, const void* e, int64_t n_tok, int32_t d_mem, const void* h,
+                                const void* Wk, const void* Wv, const float* gq, const float* gk, int32_t d,
+                                void* v, float* part, cudaStream_t s);
+// tcgen05 projection (bf16 operands, fp32 accumulation in tensor memory).
+// Returns cudaErrorNotSupported when the shape does not fit its tiling.
+bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d);
+cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
+                              const void* Wv, const float* gq, const float* gk, int32_t d, void* v,
+                              float* part, uint32_t* status, int num_sms, cudaStream_t s);
+cudaError_t launch_gate_conv(bool bf16, const void* v, const float* part, const void* h, const float* conv_w,
+                             int32_t B, int32_t L, int32_t d, int32_t w, float eps, float* state, void* y,
+                             float* alpha_out, int32_t add_residual, cudaStream_t s);
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
+    if (status) atomicOr(status, bit);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+// fp32 -> bf16 round-to-nearest-even (cuda_bf16 intrinsic), two values packed
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// 16-byte vector <-> floats
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void load(const float* p, float* out) {
+        float4 q = *reinterpret_cast<const float4*>(p);
+        out[0] = q.x; out[1] = q.y; out[2] = q.z; out[3] = q.w;
+    }
+    __device__ __forceinline__ static void store(float* p, const float* in) {
+        *reinterpret_cast<float4*>(p) = make_float4(in[0], in[1], in[2], in[3]);
+    }
+};
+template <> struct Vec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out) {
+        uint4 q = *reinterpret_cast<const uint4*>(p);
+        out[0] = bf16_lo(q.x); out[1] = bf16_hi(q.x);
+        out[2] = bf16_lo(q.y); out[3] = bf16_hi(q.y);
+        out[4] = bf16_lo(q.z); out[5] = bf16_hi(q.z);
+        out[6] = bf16_lo(q.w); out[7] = bf16_hi(q.w);
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* in) {
+        uint4 q;
+        q.x = pack_bf16x2(in[0], in[1]);
+        q.y = pack_bf16x2(in[2], in[3]);
+        q.z = pack_bf16x2(in[4], in[5]);
+        q.w = pack_bf16x2(in[6], in[7]);
+        *reinterpret_cast<uint4*>(p) = q;
+    }
+};
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_f(float& dst, float x) { dst = x; }
+__device__ __forceinline__ void from_f(__nv_bfloat16& dst, float x) { dst = __float2bfloat16_rn(x); }
+
+}  // namespace engram

@@ -1,0 +1,202 @@
+/*
+ * engram.h - C ABI of the Engram conditional-memory forward path on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The method (DeepSeek Engram; "DeepSeek AI II" digest, section "DeepSeek
+ * Engram", and the Synced repost, sections "hashed N-gram sparse retrieval"
+ * and "context-aware gating") processes every position t of a token sequence
+ * in two stages:
+ *   retrieval: x'_t = P(x_t) (tokenizer compression), suffix n-grams
+ *              g_{t,n} = (x'_{t-n+1}, ..., x'_t) for each order n, K hash
+ *              heads per order indexing tables E_{n,k} of prime size M_{n,k},
+ *              the rows concatenated into e_t;
+ *   fusion:    k_t = W_K e_t, v_t = W_V e_t, a scalar gate
+ *              alpha_t = sigmoid(<RMSNorm(h_t), RMSNorm(k_t)> / sqrt(d)),
+ *              v~_t = alpha_t v_t, and a short causal depthwise convolution
+ *              over time giving Y_t (added to the residual stream by the
+ *              caller, or here when add_residual is set).
+ *
+ * Readings fixed by this library where the pages give no formula:
+ *   hash      phi_{n,k}(g) = (XOR_{j<n} (s_j + 1) * a_{n,k,j} mod 2^64) mod M,
+ *             s_j = x'_{t-j}; s_j = PAD = V' before the sequence start;
+ *             the odd 64-bit multipliers a are configuration (engram_config).
+ *   concat    table order: order ascending, then head ascending;
+ *             table j = o*K + k for order index o and head k.
+ *   gate      q^ = g_q * h / rms(h), k^ = g_k * k / rms(k),
+ *             rms(x) = sqrt(mean(x^2) + eps), alpha = sigmoid(<q^,k^>/sqrt(d)).
+ *   conv      u_t = sum_{j<w} c[ch][j] * v~_{t-j} (per channel, causal;
+ *             history before the first computed position from conv_state,
+ *             else zero), Y_t = v~_t + SiLU(u_t) (+ h_t with add_residual).
+ *   storage   bf16 configurations store e and v as bf16 and Y as bf16;
+ *             k, alpha, u and the conv history stay fp32.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are caller-owned DEVICE memory unless stated; the
+ *     library never allocates per call.  engram_create allocates one small
+ *     device status block (freed by engram_destroy).
+ *   - Every call is asynchronous on the given stream and launches nothing
+ *     when it returns an error.  Host-side checks (null pointers, sizes,
+ *     16-byte alignment) return synchronously.
+ *   - Device-side data errors (an id outside [0, V), a canonical id outside
+ *     [0, V'), a gather index >= M, a pipeline wait that ran out) never trap:
+ *     the kernel records a bit in the context's device status word and keeps
+ *     going with zero rows for the affected position.  engram_device_status
+ *     reads and clears that word.
+ *   - Matrices are row-major.  A "row" is one computed token position; rows
+ *     are ordered sequence-major: row = b * L + (t - t_begin), L = T - t_begin.
+ *   - One context per stream at a time (the status word is shared).
+ */
+#ifndef ENGRAM_H_
+#define ENGRAM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define ENGRAM_API __attribute__((visibility("default")))
+#else
+#define ENGRAM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum engram_status {
+    ENGRAM_OK = 0,
+    ENGRAM_E_INVAL = 1,        /* bad argument: null pointer, size, alignment, non-prime M */
+    ENGRAM_E_CUDA = 2,         /* a CUDA runtime call failed */
+    ENGRAM_E_NOMEM = 3,        /* workspace too small, or allocation in engram_create failed */
+    ENGRAM_E_UNSUPPORTED = 4,  /* valid but not implemented (e.g. device is not sm_100) */
+    ENGRAM_E_TIMEOUT = 5,      /* a bounded device wait ran out (device status bit) */
+    ENGRAM_E_HOST = 6,         /* host-tier worker failure */
+    ENGRAM_E_DEVICE = 7        /* device status word reports a data error */
+} engram_status;
+
+typedef enum engram_dtype {
+    ENGRAM_F32 = 0,   /* tables, e, W, h, v, Y in fp32; projections on CUDA cores */
+    ENGRAM_BF16 = 1   /* tables, e, W, h, v, Y in bf16; projections on tcgen05 tensor cores */
+} engram_dtype;
+
+/* device status word bits (engram_device_status) */
+#define ENGRAM_ERR_TOKEN   0x1u   /* raw id outside [0, V) */
+#define ENGRAM_ERR_CANON   0x2u   /* canonical id outside [0, V') */
+#define ENGRAM_ERR_INDEX   0x4u   /* gather index >= M (other than the invalid marker) */
+#define ENGRAM_ERR_TIMEOUT 0x8u   /* a bounded device wait ran out */
+
+#define ENGRAM_INVALID_INDEX 0xFFFFFFFFu  /* index of an n-gram that holds an invalid id */
+#define ENGRAM_MAX_TABLES 32
+#define ENGRAM_PART_GROUP 128             /* channels per gate-partial group */
+
+typedef struct engram_config {
+    int32_t n_orders;                        /* number of n-gram orders, 1..4 */
+    int32_t orders[4];                       /* the orders, ascending, each in 1..4 (pages: {2,3}) */
+    int32_t heads;                           /* K hash heads per order; J = n_orders*heads <= 32 */
+    uint32_t rows[ENGRAM_MAX_TABLES];        /* M_j for table j = o*K + k; each prime, < 2^31 */
+    uint64_t mult[ENGRAM_MAX_TABLES][4];     /* a_{n,k,j}: multiplier of s_j for table j (j < n) */
+    int32_t row_dim;                         /* D, elements per table row */
+    int32_t hidden;                          /* d, hidden width (query, k, v, Y) */
+    int32_t conv_width;                      /* w, causal conv taps, 1..8 */
+    int32_t vocab;                           /* V, raw vocabulary */
+    int32_t canon_vocab;                     /* V', canonical vocabulary; PAD id = V' */
+    engram_dtype dtype;
+    float eps;                               /* RMSNorm epsilon (1e-6) */
+} engram_config;
+
+typedef struct engram_ctx engram_ctx;
+
+/* Validate cfg (orders ascending in 1..4, J <= 32, every M prime and < 2^31,
+ * D*elem a multiple of 16 bytes, d a multiple of 8, V' < 2^31 - 1) and bind a
+ * context to the CURRENT device.  Allocates a 256-byte device status block.
+ * Returns ENGRAM_E_INVAL for a bad config, ENGRAM_E_CUDA/NOMEM on failure. */
+ENGRAM_API engram_status engram_create(const engram_config* cfg, engram_ctx** out);
+ENGRAM_API void engram_destroy(engram_ctx* ctx);
+ENGRAM_API const char* engram_strerror(engram_status s);
+/* Text of the last host-side failure on the calling thread (argument check
+ * or CUDA error with its call site); empty when none.  Owned by the library. */
+ENGRAM_API const char* engram_last_error(void);
+
+/* Bytes of scratch that engram_forward / engram_gate_conv need for n_tok rows:
+ * indices [n_tok][J] u32, e [n_tok][J*D], v [n_tok][d] and gate partials
+ * [n_tok][G][4] f32 with G = ceil(d / 128), each 256-byte aligned. */
+ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int64_t n_tok);
+
+/* Synchronise `stream`, return the device status word in *flags (nullable)
+ * and clear it.  ENGRAM_OK when it was zero, ENGRAM_E_TIMEOUT when the
+ * timeout bit was set, else ENGRAM_E_DEVICE. */
+ENGRAM_API engram_status engram_device_status(engram_ctx* ctx, cudaStream_t stream, uint32_t* flags);
+
+/* Tokenizer compression ("DeepSeek AI II" digest, section "DeepSeek Engram":
+ * the surjection P: V -> V').  canon[i] = P[tok[i]] for i < n; P is [V] int32.
+ * An id outside [0, V) gives canon = -1 and sets ENGRAM_ERR_TOKEN. */
+ENGRAM_API engram_status engram_remap(engram_ctx* ctx, const int32_t* tok, int64_t n, const int32_t* P,
+                           int32_t* canon, cudaStream_t stream);
+
+/* Suffix n-grams and multi-head hashing (same section: g_{t,n}, phi_{n,k},
+ * prime table sizes; Synced repost, "hashed N-gram sparse retrieval": K
+ * independent heads per order).  ids is [B] sequences of `stride` int32
+ * (positions 0..T-1 valid); rows t in [t_begin, T) are computed and the
+ * n-gram windows reach back into [0, t_begin).  When P is non-null, ids are
+ * raw token ids remapped on the fly; otherwise they are canonical ids.
+ * idx is [B*(T-t_begin)][J] uint32; an n-gram holding an invalid id gives
+ * ENGRAM_INVALID_INDEX for its order's K tables. */
+ENGRAM_API engram_status engram_hash(engram_ctx* ctx, const int32_t* ids, const int32_t* P, int32_t B, int32_t T,
+                          int64_t stride, int32_t t_begin, uint32_t* idx, cudaStream_t stream);
+
+/* Gather and concatenation (same section: e_t = concat of E_{n,k}[phi]).
+ * tables holds the J tables back to back (table j starts at row
+ * sum_{i<j} M_i; each row D elements of the context dtype); e_cat is
+ * [n_tok][J*D].  An index >= M_j writes a zero row (ENGRAM_ERR_INDEX unless
+ * it is ENGRAM_INVALID_INDEX).  tables and e_cat 16-byte aligned. */
+ENGRAM_API engram_status engram_gather(engram_ctx* ctx, const uint32_t* idx, int64_t n_tok, const void* tables,
+                            void* e_cat, cudaStream_t stream);
+
+/* Key/value projections with the gate's partial sums (same section: k = W_K e,
+ * v = W_V e; RMSNorm on query and key).  Wk and Wv are [d][J*D] (nn.Linear
+ * layout), h is [n_tok][d], gq/gk are [d] fp32 RMSNorm gains (null = ones).
+ * Writes v [n_tok][d] in the context dtype and part [n_tok][G][4] fp32,
+ * G = ceil(d/128): for channel group g, part = (sum g_q g_k h k, sum k^2,
+ * sum h^2, 0) over the group's channels.  k itself is never stored. */
+ENGRAM_API engram_status engram_project(engram_ctx* ctx, const void* e_cat, int64_t n_tok, const void* h,
+                             const void* Wk, const void* Wv, const float* gq, const float* gk,
+                             void* v, float* part, cudaStream_t stream);
+
+/* Gate and causal depthwise convolution (same section: alpha_t in (0,1),
+ * v~ = alpha v, short-kernel per-channel causal conv; residual H <- H + Y).
+ * v and part as written by engram_project for B sequences of L rows each;
+ * conv_w is [d][w] fp32 (tap j multiplies v~_{t-j}); conv_state (nullable)
+ * is [B][w-1][d] fp32 holding v~ of the w-1 positions before the first row
+ * (row w-2 most recent): read as history and overwritten with the last w-1
+ * v~ rows of the extended sequence (in place is safe).  Null: zero history.
+ * h is read only when add_residual != 0.  y is [B*L][d] (context dtype);
+ * alpha_out (nullable) [B*L] fp32. */
+ENGRAM_API engram_status engram_conv(engram_ctx* ctx, const void* v, const float* part, const void* h,
+                          const float* conv_w, int32_t B, int32_t L, float* conv_state, void* y,
+                          float* alpha_out, int32_t add_residual, cudaStream_t stream);
+
+/* engram_project followed by engram_conv, v and part in `workspace`. */
+ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, const void* h, const void* Wk,
+                               const void* Wv, const float* gq, const float* gk, const float* conv_w,
+                               int32_t B, int32_t L, float* conv_state, void* y, float* alpha_out,
+                               int32_t add_residual, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* The whole forward: engram_hash (with remap) -> engram_gather ->
+ * engram_project -> engram_conv, intermediates in `workspace`
+ * (engram_workspace_bytes(ctx, B*(T-t_begin)) bytes, 256-byte aligned).
+ * tok is [B] rows of `tok_stride` raw ids; prefill uses t_begin = 0, a
+ * decode step for the last position uses t_begin = T-1 with conv_state. */
+ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int32_t B, int32_t T,
+                             int64_t tok_stride, int32_t t_begin, const int32_t* P,
+                             const void* tables, const void* h, const void* Wk, const void* Wv,
+                             const float* gq, const float* gk, const float* conv_w,
+                             float* conv_state, void* y, float* alpha_out, int32_t add_residual,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENGRAM_H_ */

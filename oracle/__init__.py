@@ -257,6 +257,7 @@ def forward_rows(inp, positions: np.ndarray, add_residual: bool = False, eps: fl
     vt = alpha[:, None] * v
     y = np.empty((len(positions), wl.d))
     al = np.empty(len(positions))
+    win = np.zeros((len(positions), wl.w, wl.d))
     for i, p in enumerate(positions):
         b, t = divmod(int(p), L)
         lo = max(0, t - (wl.w - 1))
@@ -267,4 +268,23 @@ def forward_rows(inp, positions: np.ndarray, add_residual: bool = False, eps: fl
             u = conv(seg, inp.conv_w, None)[-1:]
         y[i] = output(vt[slot[int(p)]][None], u, h[slot[int(p)]][None], add_residual)[0]
         al[i] = alpha[slot[int(p)]]
-    return Result(idx=idx, y=y, alpha=al, positions=np.asarray(positions))
+        for j in range(wl.w):
+            if t - j >= 0:
+                win[i, j] = vt[slot[b * L + t - j]]
+            elif hist is not None:
+                win[i, j] = hist[b][wl.w - 1 + t - j]
+    return Result(idx=idx, y=y, alpha=al, vt_win=win, positions=np.asarray(positions))
+
+
+def vt_windows(vt: np.ndarray, B: int, L: int, w: int, hist: Optional[np.ndarray] = None) -> np.ndarray:
+    """[n][w][d]: the gated values v~_{t-j}, j < w, seen by each row's conv."""
+    n, d = vt.shape
+    win = np.zeros((n, w, d))
+    for r in range(n):
+        b, t = divmod(r, L)
+        for j in range(w):
+            if t - j >= 0:
+                win[r, j] = vt[b * L + t - j]
+            elif hist is not None:
+                win[r, j] = hist[b][w - 1 + t - j]
+    return win

@@ -1,0 +1,54 @@
+"""Helpers shared by the GPU parity tests: build a context from seeded inputs,
+place the inputs on the device, and the bf16 output tolerance."""
+
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+
+
+def config_for(inp, eb, eps: float = 1e-6):
+    wl = inp.wl
+    return eb.make_config(orders=wl.orders, heads=wl.K, rows=[int(x) for x in inp.rows], mult=inp.mult,
+                          row_dim=wl.D, hidden=wl.d, conv_width=wl.w, vocab=wl.V, canon_vocab=wl.Vc,
+                          dtype=eb.ENGRAM_BF16 if wl.dtype == "bf16" else eb.ENGRAM_F32, eps=eps)
+
+
+class DeviceInputs:
+    def __init__(self, inp, device="cuda:0"):
+        import torch
+        self.inp = inp
+        self.wl = inp.wl
+        dd = inp.device_dense(device)
+        self.__dict__.update(dd)
+        self.tables = inp.device_tables(device)
+        self.h = inp.device_hidden(device)
+        self.dtype = torch.float32 if self.wl.dtype == "f32" else torch.bfloat16
+        self.device = device
+
+    def empty_y(self):
+        import torch
+        return torch.empty(self.wl.n_tok, self.wl.d, dtype=self.dtype, device=self.device)
+
+
+def bf16_bound(y_ref: np.ndarray, vt_win: np.ndarray, cw: np.ndarray) -> np.ndarray:
+    """Elementwise bound on |Y_gpu - Y_oracle| for the bf16 path.
+
+    Sources: (1) Y is rounded once to bf16 (half an ulp, 2^-8 relative);
+    (2) v is stored as bf16 after an fp32 (GPU) or fp64 (oracle) accumulation,
+    so the two may land one bf16 ulp apart (2^-7 relative); such a flip in
+    v_{t-j} moves v~_{t-j} by at most 2^-7 |v~_{t-j}| and reaches Y_t through
+    the skip (j = 0, weight 1) and through SiLU(u) (weight |c_j| * max SiLU',
+    max SiLU' < 1.1); (3) fp32 arithmetic in the gate and conv, well below
+    1e-5 at these magnitudes.  A factor 1.5 covers both (1) and (2) at once."""
+    w = cw.shape[1]
+    s = np.abs(vt_win[:, 0]) * (1.0 + 1.1 * np.abs(cw[None, :, 0]))
+    for j in range(1, w):
+        s = s + 1.1 * np.abs(cw[None, :, j]) * np.abs(vt_win[:, j])
+    return 1.5 * (2.0 ** -8 * np.abs(y_ref) + 2.0 ** -7 * s) + 1e-5
+
+
+def to_np(t):
+    import torch
+    return t.detach().to(torch.float64).cpu().numpy()
