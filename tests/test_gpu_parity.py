@@ -317,3 +317,47 @@ def test_host_checks_launch_nothing(eb):
                           None, di.conv_w, None, y, None, 0, ctx.workspace, ctx.workspace_bytes)
     torch.cuda.synchronize()
     assert bool((y == 3.0).all()) and bool((ybig == 0).all())
+
+
+@pytest.mark.parametrize("name", ["b1", "b2", "b3", "c1"])
+def test_project_v_and_partials(eb, name):
+    """engram_project alone: v (storage dtype) and the per-group gate partials
+    against the oracle's fp64 projections."""
+    wl = SMALL[name]
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    ref = oracle.forward_full(inp)
+    e = torch.from_numpy(ref.e.astype(np.float32)).to(di.dtype).cuda()
+    G = (wl.d + 127) // 128
+    v = torch.empty(wl.n_tok, wl.d, dtype=di.dtype, device="cuda")
+    part = torch.full((wl.n_tok, G, 4), float("nan"), dtype=torch.float32, device="cuda")
+    eb.engram_project(ctx.ctx, e, wl.n_tok, di.h, di.Wk, di.Wv, di.gq, di.gk, v, part)
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    vg = to_np(v)
+    if wl.dtype == "f32":
+        assert np.max(np.abs(vg - ref.v)) <= 1e-5
+    else:
+        # bf16 storage: equal to the oracle's rounding up to one bf16 ulp plus
+        # the fp32 accumulation error, bounded by K 2^-23 sum_q |e_q W_q|
+        # (large relative to |v| only where the sum cancels)
+        ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref.v), 1e-30))) - 7)
+        s_abs = np.abs(ref.e.astype(np.float64)) @ np.abs(inp.Wv.astype(np.float64)).T
+        bound = ulp * 1.0001 + wl.d_mem * 2.0 ** -23 * s_abs
+        diff = np.abs(vg - ref.v)
+        assert np.all(diff <= bound), float((diff / bound).max())
+        assert np.mean(diff == 0) > 0.95
+    h = inp.all_hidden()
+    gg = inp.gq.astype(np.float64) * inp.gk.astype(np.float64)
+    pg = part.cpu().numpy().astype(np.float64)
+    for g in range(G):
+        sl = slice(g * 128, min(wl.d, g * 128 + 128))
+        want_qk = np.sum(gg[sl][None] * h[:, sl] * ref.k[:, sl], axis=1)
+        want_kk = np.sum(ref.k[:, sl] ** 2, axis=1)
+        want_hh = np.sum(h[:, sl].astype(np.float64) ** 2, axis=1)
+        scale_qk = np.sum(np.abs(gg[sl][None] * h[:, sl] * ref.k[:, sl]), axis=1)
+        np.testing.assert_allclose(pg[:, g, 0], want_qk, rtol=0, atol=1e-5 * (1 + scale_qk.max()))
+        np.testing.assert_allclose(pg[:, g, 1], want_kk, rtol=2e-5, atol=1e-7)
+        np.testing.assert_allclose(pg[:, g, 2], want_hh, rtol=2e-5, atol=1e-7)
+        assert np.all(pg[:, g, 3] == 0)
