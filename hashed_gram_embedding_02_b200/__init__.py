@@ -14,26 +14,27 @@ from .binding import (  # noqa: F401  (re-exported C ABI names)
     ENGRAM_BF16, ENGRAM_F32, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
     ENGRAM_INVALID_INDEX, ENGRAM_OK, EXPORTS, LIB_PATH, EngramError, engram_config, engram_conv, engram_create,
     engram_destroy, engram_device_status, engram_forward, engram_gate_conv, engram_gather, engram_hash,
-    engram_last_error, engram_project, engram_remap, engram_strerror, engram_workspace_bytes, make_config)
+    engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
+    engram_workspace_bytes, make_config)
 
 
 class Engram:
-    """Owns one engram_ctx (bound to the current device) and a workspace
-    sized for up to ``max_tok`` rows."""
+    """Owns one engram_ctx (bound to the current device) and a workspace,
+    grown on demand (or reserved up front for B sequences of L rows)."""
 
-    def __init__(self, cfg: engram_config, max_tok: int = 0):
+    def __init__(self, cfg: engram_config, B: int = 0, L: int = 0):
         import torch
         self.cfg = cfg
         self.ctx = engram_create(cfg)
         self.device = torch.device("cuda", torch.cuda.current_device())
         self.workspace = None
         self.workspace_bytes = 0
-        if max_tok:
-            self.reserve(max_tok)
+        if B and L:
+            self.reserve(B, L)
 
-    def reserve(self, n_tok: int):
+    def reserve(self, B: int, L: int):
         import torch
-        need = engram_workspace_bytes(self.ctx, n_tok)
+        need = engram_workspace_bytes(self.ctx, B, L)
         if need > self.workspace_bytes:
             self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
             self.workspace_bytes = need
@@ -56,7 +57,7 @@ class Engram:
     def forward(self, tok, P, tables, h, Wk, Wv, conv_w, y, *, t_begin: int = 0, gq=None, gk=None,
                 conv_state=None, alpha_out=None, add_residual: bool = False, stream=None):
         B, T = tok.shape[0], tok.shape[1]
-        self.reserve(B * (T - t_begin))
+        self.reserve(B, T - t_begin)
         engram_forward(self.ctx, tok, B, T, tok.stride(0), t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w,
                        conv_state, y, alpha_out, add_residual, self.workspace, self.workspace_bytes, stream)
         return y

@@ -33,8 +33,8 @@ ENGRAM_PART_GROUP = 128
 
 # exported symbol names declared in include/engram.h
 EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_error", "engram_workspace_bytes",
-           "engram_device_status", "engram_remap", "engram_hash", "engram_gather", "engram_project",
-           "engram_conv", "engram_gate_conv", "engram_forward")
+           "engram_profile_enable", "engram_profile_read", "engram_device_status", "engram_remap", "engram_hash",
+           "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward")
 
 
 class engram_config(ctypes.Structure):
@@ -69,7 +69,9 @@ _sigs = {
     "engram_destroy": ([_vp], None),
     "engram_strerror": ([_st], ctypes.c_char_p),
     "engram_last_error": ([], ctypes.c_char_p),
-    "engram_workspace_bytes": ([_vp, _i64], _sz),
+    "engram_workspace_bytes": ([_vp, _i32, _i32], _sz),
+    "engram_profile_enable": ([_vp, _i32], _st),
+    "engram_profile_read": ([_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p), _i32], _i32),
     "engram_device_status": ([_vp, _vp, ctypes.POINTER(ctypes.c_uint32)], _st),
     "engram_remap": ([_vp, _vp, _i64, _vp, _vp, _vp], _st),
     "engram_hash": ([_vp, _vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp], _st),
@@ -143,8 +145,20 @@ def engram_last_error() -> str:
     return _lib.engram_last_error().decode()
 
 
-def engram_workspace_bytes(ctx: int, n_tok: int) -> int:
-    return int(_lib.engram_workspace_bytes(ctx, n_tok))
+def engram_workspace_bytes(ctx: int, B: int, L: int) -> int:
+    return int(_lib.engram_workspace_bytes(ctx, B, L))
+
+
+def engram_profile_enable(ctx: int, enable: bool = True) -> None:
+    _check(_lib.engram_profile_enable(ctx, 1 if enable else 0), "engram_profile_enable")
+
+
+def engram_profile_read(ctx: int, max_kernels: int = 16):
+    """[(kernel name, ms)] of the kernels launched by the most recent call."""
+    ms = (ctypes.c_float * max_kernels)()
+    names = (ctypes.c_char_p * max_kernels)()
+    n = _lib.engram_profile_read(ctx, ms, names, max_kernels)
+    return [(names[i].decode(), float(ms[i])) for i in range(n)]
 
 
 def engram_device_status(ctx: int, stream=None):

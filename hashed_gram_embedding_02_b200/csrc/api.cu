@@ -11,6 +11,10 @@
 
 using namespace engram;
 
+namespace {
+constexpr int kMaxProf = 16;
+}
+
 struct engram_ctx {
     engram_config cfg;
     int device;
@@ -23,6 +27,11 @@ struct engram_ctx {
     HashParams hp;
     GatherParams gp;
     uint32_t* d_status;     // device status word (256-byte block)
+    // per-kernel timing (engram_profile_enable)
+    bool prof;
+    cudaEvent_t ev[2 * kMaxProf];
+    const char* prof_name[kMaxProf];
+    int prof_n;
 };
 
 namespace {
@@ -57,32 +66,57 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// ---------------------------------------------------------------- profiling
+
+void prof_reset(engram_ctx* c) { c->prof_n = 0; }
+
+void prof_begin(engram_ctx* c, cudaStream_t s, const char* name) {
+    if (!c->prof || c->prof_n >= kMaxProf) return;
+    c->prof_name[c->prof_n] = name;
+    cudaEventRecord(c->ev[2 * c->prof_n], s);
+}
+
+void prof_end(engram_ctx* c, cudaStream_t s) {
+    if (!c->prof || c->prof_n >= kMaxProf) return;
+    cudaEventRecord(c->ev[2 * c->prof_n + 1], s);
+    ++c->prof_n;
+}
+
+// ---------------------------------------------------------------- workspace
+
+bool tc_path(const engram_ctx* c, int64_t n) {
+    return c->cfg.dtype == ENGRAM_BF16 && c->sm100 && project_tc_supported(n, c->d_mem, c->cfg.hidden);
+}
+
 struct Workspace {
     uint32_t* idx;
     void* e;
-    void* v;
     float* part;
+    float* state_next;
+    float* v;
     size_t bytes;
 };
 
-size_t idx_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->J * sizeof(uint32_t)); }
-size_t e_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->d_mem * c->es); }
-size_t v_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->cfg.hidden * c->es); }
-size_t part_bytes(const engram_ctx* c, int64_t n) { return align256((size_t)n * c->G * 4 * sizeof(float)); }
-
-Workspace carve(const engram_ctx* c, void* base, int64_t n, bool with_idx_e) {
+// idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | state_next [B][w-1][d] f32 |
+// v [n][d] f32 (CUDA-core path only), each 256-byte aligned
+Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e) {
+    const int64_t n = B * L;
     Workspace w{};
     char* p = static_cast<char*>(base);
     if (with_idx_e) {
         w.idx = reinterpret_cast<uint32_t*>(p);
-        p += idx_bytes(c, n);
+        p += align256((size_t)n * c->J * sizeof(uint32_t));
         w.e = p;
-        p += e_bytes(c, n);
+        p += align256((size_t)n * c->d_mem * c->es);
     }
-    w.v = p;
-    p += v_bytes(c, n);
     w.part = reinterpret_cast<float*>(p);
-    p += part_bytes(c, n);
+    p += align256((size_t)n * c->G * 4 * sizeof(float));
+    w.state_next = reinterpret_cast<float*>(p);
+    p += align256((size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
+    if (!tc_path(c, n)) {
+        w.v = reinterpret_cast<float*>(p);
+        p += align256((size_t)n * c->cfg.hidden * sizeof(float));
+    }
     w.bytes = (size_t)(p - static_cast<char*>(base));
     return w;
 }
@@ -101,24 +135,62 @@ engram_status launched(const char* what, cudaError_t e) {
 }
 
 engram_status project_impl(engram_ctx* c, const void* e_cat, int64_t n, const void* h, const void* Wk,
-                           const void* Wv, const float* gq, const float* gk, void* v, float* part,
+                           const void* Wv, const float* gq, const float* gk, float* v, float* part,
                            cudaStream_t s) {
     const bool bf16 = c->cfg.dtype == ENGRAM_BF16;
-    if (bf16 && c->sm100 && project_tc_supported(n, c->d_mem, c->cfg.hidden)) {
-        return launched("tcgen05 projection launch",
-                        launch_project_tc(e_cat, n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, v, part,
-                                          c->d_status, c->num_sms, s));
+    if (tc_path(c, n)) {
+        prof_begin(c, s, "project_kv_tc");
+        cudaError_t e = launch_project_tc(e_cat, n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, v, part, c->d_status,
+                                          c->num_sms, s);
+        prof_end(c, s);
+        return launched("tcgen05 projection launch", e);
     }
-    return launched("projection launch", launch_project_simt(bf16, e_cat, n, c->d_mem, h, Wk, Wv, gq, gk,
-                                                             c->cfg.hidden, v, part, s));
+    prof_begin(c, s, "project_simt");
+    cudaError_t e = launch_project_simt(bf16, e_cat, n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, v, part, s);
+    prof_end(c, s);
+    return launched("projection launch", e);
 }
 
-engram_status conv_impl(engram_ctx* c, const void* v, const float* part, const void* h, const float* conv_w,
+engram_status conv_impl(engram_ctx* c, const float* v, const float* part, const void* h, const float* conv_w,
                         int32_t B, int32_t L, float* state, void* y, float* alpha_out, int32_t add_residual,
                         cudaStream_t s) {
-    return launched("gate/conv launch",
-                    launch_gate_conv(c->cfg.dtype == ENGRAM_BF16, v, part, h, conv_w, B, L, c->cfg.hidden,
-                                     c->cfg.conv_width, c->cfg.eps, state, y, alpha_out, add_residual, s));
+    prof_begin(c, s, "gate_conv");
+    cudaError_t e = launch_gate_conv(c->cfg.dtype == ENGRAM_BF16, v, part, h, conv_w, B, L, c->cfg.hidden,
+                                     c->cfg.conv_width, c->cfg.eps, state, y, alpha_out, add_residual, c->d_status,
+                                     s);
+    prof_end(c, s);
+    return launched("gate/conv launch", e);
+}
+
+// projections + gate + conv; on the tensor-core path two GEMM passes with the
+// gate and the conv fused into the second one's epilogue
+engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, const void* Wk, const void* Wv,
+                             const float* gq, const float* gk, const float* conv_w, int32_t B, int32_t L,
+                             float* state, void* y, float* alpha_out, int32_t add_residual, const Workspace& w,
+                             cudaStream_t s) {
+    const int64_t n = (int64_t)B * L;
+    if (tc_path(c, n)) {
+        prof_begin(c, s, "gate_k_tc");
+        cudaError_t e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, w.part, c->d_status,
+                                         c->num_sms, s);
+        prof_end(c, s);
+        if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
+        prof_begin(c, s, "vconv_tc");
+        e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, c->cfg.eps,
+                            w.part, state, w.state_next, y, alpha_out, add_residual, c->d_status, c->num_sms, s);
+        prof_end(c, s);
+        if (e != cudaSuccess) return cuda_fail("tcgen05 value/conv launch", e);
+        if (state) {
+            prof_begin(c, s, "state_merge");
+            e = launch_state_merge(state, w.state_next, B, L, c->cfg.conv_width, c->cfg.hidden, c->num_sms, s);
+            prof_end(c, s);
+            if (e != cudaSuccess) return cuda_fail("conv-state merge launch", e);
+        }
+        return ENGRAM_OK;
+    }
+    engram_status st = project_impl(c, e_cat, n, h, Wk, Wv, gq, gk, w.v, w.part, s);
+    if (st != ENGRAM_OK) return st;
+    return conv_impl(c, w.v, w.part, h, conv_w, B, L, state, y, alpha_out, add_residual, s);
 }
 
 }  // namespace
@@ -224,13 +296,47 @@ engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
 
 void engram_destroy(engram_ctx* c) {
     if (!c) return;
+    if (c->prof)
+        for (int i = 0; i < 2 * kMaxProf; ++i) cudaEventDestroy(c->ev[i]);
     if (c->d_status) cudaFree(c->d_status);
     delete c;
 }
 
-size_t engram_workspace_bytes(const engram_ctx* c, int64_t n_tok) {
-    if (!c || n_tok < 0) return 0;
-    return idx_bytes(c, n_tok) + e_bytes(c, n_tok) + v_bytes(c, n_tok) + part_bytes(c, n_tok);
+size_t engram_workspace_bytes(const engram_ctx* c, int32_t B, int32_t L) {
+    if (!c || B < 0 || L < 0) return 0;
+    return carve(c, nullptr, B, L, true).bytes;
+}
+
+engram_status engram_profile_enable(engram_ctx* c, int32_t enable) {
+    if (!c) return inval("null context");
+    if (enable && !c->prof) {
+        for (int i = 0; i < 2 * kMaxProf; ++i) {
+            cudaError_t e = cudaEventCreate(&c->ev[i]);
+            if (e != cudaSuccess) {
+                for (int k = 0; k < i; ++k) cudaEventDestroy(c->ev[k]);
+                return cuda_fail("cudaEventCreate", e);
+            }
+        }
+        c->prof = true;
+    } else if (!enable && c->prof) {
+        for (int i = 0; i < 2 * kMaxProf; ++i) cudaEventDestroy(c->ev[i]);
+        c->prof = false;
+    }
+    c->prof_n = 0;
+    return ENGRAM_OK;
+}
+
+int32_t engram_profile_read(engram_ctx* c, float* ms, const char** names, int32_t max) {
+    if (!c || !c->prof) return 0;
+    int n = c->prof_n < max ? c->prof_n : max;
+    for (int i = 0; i < n; ++i) {
+        cudaEventSynchronize(c->ev[2 * i + 1]);
+        float t = 0.f;
+        cudaEventElapsedTime(&t, c->ev[2 * i], c->ev[2 * i + 1]);
+        if (ms) ms[i] = t;
+        if (names) names[i] = c->prof_name[i];
+    }
+    return n;
 }
 
 engram_status engram_device_status(engram_ctx* c, cudaStream_t s, uint32_t* flags) {
@@ -256,7 +362,11 @@ engram_status engram_remap(engram_ctx* c, const int32_t* tok, int64_t n, const i
     if (n > 0 && (!tok || !P || !canon)) return inval("null tensor pointer");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
-    return launched("remap launch", launch_remap(tok, n, P, c->cfg.vocab, canon, c->d_status, s));
+    prof_reset(c);
+    prof_begin(c, s, "remap");
+    cudaError_t e = launch_remap(tok, n, P, c->cfg.vocab, canon, c->d_status, s);
+    prof_end(c, s);
+    return launched("remap launch", e);
 }
 
 engram_status engram_hash(engram_ctx* c, const int32_t* ids, const int32_t* P, int32_t B, int32_t T,
@@ -268,7 +378,11 @@ engram_status engram_hash(engram_ctx* c, const int32_t* ids, const int32_t* P, i
     if (!ids || !idx) return inval("null tensor pointer");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
-    return launched("hash launch", launch_hash(ids, P, B, T, stride, t_begin, idx, c->hp, c->d_status, s));
+    prof_reset(c);
+    prof_begin(c, s, "hash");
+    cudaError_t e = launch_hash(ids, P, B, T, stride, t_begin, idx, c->hp, c->d_status, s);
+    prof_end(c, s);
+    return launched("hash launch", e);
 }
 
 engram_status engram_gather(engram_ctx* c, const uint32_t* idx, int64_t n_tok, const void* tables,
@@ -280,11 +394,15 @@ engram_status engram_gather(engram_ctx* c, const uint32_t* idx, int64_t n_tok, c
     if (!aligned16(tables) || !aligned16(e_cat)) return inval("tables and e_cat must be 16-byte aligned");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
-    return launched("gather launch", launch_gather(idx, n_tok, tables, c->gp, e_cat, c->d_status, c->num_sms, s));
+    prof_reset(c);
+    prof_begin(c, s, "gather");
+    cudaError_t e = launch_gather(idx, n_tok, tables, c->gp, e_cat, c->d_status, c->num_sms, s);
+    prof_end(c, s);
+    return launched("gather launch", e);
 }
 
 engram_status engram_project(engram_ctx* c, const void* e_cat, int64_t n_tok, const void* h, const void* Wk,
-                             const void* Wv, const float* gq, const float* gk, void* v, float* part,
+                             const void* Wv, const float* gq, const float* gk, float* v, float* part,
                              cudaStream_t s) {
     if (!c) return inval("null context");
     if (n_tok < 0) return inval("n_tok must be >= 0");
@@ -294,10 +412,11 @@ engram_status engram_project(engram_ctx* c, const void* e_cat, int64_t n_tok, co
         return inval("e_cat, h, Wk, Wv, v and part must be 16-byte aligned");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
+    prof_reset(c);
     return project_impl(c, e_cat, n_tok, h, Wk, Wv, gq, gk, v, part, s);
 }
 
-engram_status engram_conv(engram_ctx* c, const void* v, const float* part, const void* h, const float* conv_w,
+engram_status engram_conv(engram_ctx* c, const float* v, const float* part, const void* h, const float* conv_w,
                           int32_t B, int32_t L, float* conv_state, void* y, float* alpha_out,
                           int32_t add_residual, cudaStream_t s) {
     if (!c) return inval("null context");
@@ -305,10 +424,11 @@ engram_status engram_conv(engram_ctx* c, const void* v, const float* part, const
     if ((int64_t)B * L == 0) return ENGRAM_OK;
     if (!v || !part || !conv_w || !y || (add_residual && !h)) return inval("null tensor pointer");
     if (!aligned16(v) || !aligned16(part) || !aligned16(y) || (add_residual && !aligned16(h)) ||
-        (conv_state && !aligned16(conv_state)))
-        return inval("v, part, y, h and conv_state must be 16-byte aligned");
+        (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
+        return inval("v, part, y, h, conv_w and conv_state must be 16-byte aligned");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
+    prof_reset(c);
     return conv_impl(c, v, part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, s);
 }
 
@@ -322,16 +442,15 @@ engram_status engram_gate_conv(engram_ctx* c, const void* e_cat, const void* h, 
     if (n == 0) return ENGRAM_OK;
     if (!e_cat || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
-    Workspace w = carve(c, workspace, n, false);
+    Workspace w = carve(c, workspace, B, L, false);
     if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
     if (!aligned16(e_cat) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
-        (conv_state && !aligned16(conv_state)))
-        return inval("e_cat, h, Wk, Wv, y and conv_state must be 16-byte aligned");
+        (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
+        return inval("e_cat, h, Wk, Wv, y, conv_w and conv_state must be 16-byte aligned");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
-    st = project_impl(c, e_cat, n, h, Wk, Wv, gq, gk, w.v, w.part, s);
-    if (st != ENGRAM_OK) return st;
-    return conv_impl(c, w.v, w.part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, s);
+    prof_reset(c);
+    return gate_conv_impl(c, e_cat, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
 }
 
 engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
@@ -347,20 +466,23 @@ engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32
     if (n == 0) return ENGRAM_OK;
     if (!tok || !P || !tables || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
-    Workspace w = carve(c, workspace, n, true);
+    Workspace w = carve(c, workspace, B, L, true);
     if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
     if (!aligned16(tables) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
-        (conv_state && !aligned16(conv_state)))
-        return inval("tables, h, Wk, Wv, y and conv_state must be 16-byte aligned");
+        (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
+        return inval("tables, h, Wk, Wv, y, conv_w and conv_state must be 16-byte aligned");
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
-    st = launched("hash launch", launch_hash(tok, P, B, T, tok_stride, t_begin, w.idx, c->hp, c->d_status, s));
-    if (st != ENGRAM_OK) return st;
-    st = launched("gather launch", launch_gather(w.idx, n, tables, c->gp, w.e, c->d_status, c->num_sms, s));
-    if (st != ENGRAM_OK) return st;
-    st = project_impl(c, w.e, n, h, Wk, Wv, gq, gk, w.v, w.part, s);
-    if (st != ENGRAM_OK) return st;
-    return conv_impl(c, w.v, w.part, h, conv_w, B, L, conv_state, y, alpha_out, add_residual, s);
+    prof_reset(c);
+    prof_begin(c, s, "hash");
+    cudaError_t e = launch_hash(tok, P, B, T, tok_stride, t_begin, w.idx, c->hp, c->d_status, s);
+    prof_end(c, s);
+    if (e != cudaSuccess) return cuda_fail("hash launch", e);
+    prof_begin(c, s, "gather");
+    e = launch_gather(w.idx, n, tables, c->gp, w.e, c->d_status, c->num_sms, s);
+    prof_end(c, s);
+    if (e != cudaSuccess) return cuda_fail("gather launch", e);
+    return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
 }
 
 }  // extern "C"

@@ -44,19 +44,33 @@ cudaError_t launch_hash(const int32_t* ids, const int32_t* P, int32_t B, int32_t
                         cudaStream_t s);
 cudaError_t launch_gather(const uint32_t* idx, int64_t n_tok, const void* tables, const GatherParams& gp,
                           void* e_cat, uint32_t* status, int num_sms, cudaStream_t s);
-// CUDA-core projection (fp32 or bf16 operands, fp32 accumulation)
+// CUDA-core projection (fp32 or bf16 operands, fp32 accumulation); v in fp32
 cudaError_t launch_project_simt(bool bf16, const void* e, int64_t n_tok, int32_t d_mem, const void* h,
                                 const void* Wk, const void* Wv, const float* gq, const float* gk, int32_t d,
-                                void* v, float* part, cudaStream_t s);
-// tcgen05 projection (bf16 operands, fp32 accumulation in tensor memory).
-// Returns cudaErrorNotSupported when the shape does not fit its tiling.
+                                float* v, float* part, cudaStream_t s);
+// tcgen05 kernels (bf16 operands, fp32 accumulation in tensor memory); both
+// return cudaErrorNotSupported when the shape does not fit their tiling.
 bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d);
 cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
-                              const void* Wv, const float* gq, const float* gk, int32_t d, void* v,
+                              const void* Wv, const float* gq, const float* gk, int32_t d, float* v,
                               float* part, uint32_t* status, int num_sms, cudaStream_t s);
-cudaError_t launch_gate_conv(bool bf16, const void* v, const float* part, const void* h, const float* conv_w,
+// Pass 1: k -> gate partials [n_tok][G][4].
+cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
+                             const float* gq, const float* gk, int32_t d, float* part, uint32_t* status, int num_sms,
+                             cudaStream_t s);
+// Pass 2: v -> gate, causal conv, residual, Y (fused epilogue).  When state is
+// non-null the new history goes to state_next ([B][w-1][d] fp32 scratch) and
+// launch_state_merge folds it into state afterwards.
+cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
+                            const float* conv_w, int32_t d, int32_t w, float eps, const float* part,
+                            const float* state, float* state_next, void* y, float* alpha_out, int32_t add_residual,
+                            uint32_t* status, int num_sms, cudaStream_t s);
+cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,
+                               int num_sms, cudaStream_t s);
+// gate + conv from an fp32 v (CUDA cores)
+cudaError_t launch_gate_conv(bool bf16, const float* v, const float* part, const void* h, const float* conv_w,
                              int32_t B, int32_t L, int32_t d, int32_t w, float eps, float* state, void* y,
-                             float* alpha_out, int32_t add_residual, cudaStream_t s);
+                             float* alpha_out, int32_t add_residual, uint32_t* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- device helpers
 __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {

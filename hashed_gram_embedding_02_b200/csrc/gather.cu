@@ -16,7 +16,7 @@ namespace engram {
 
 namespace {
 
-constexpr int kTokBatch = 8;
+constexpr int kTokBatch = 4;
 
 __global__ void __launch_bounds__(256)
 gather_kernel(const uint32_t* __restrict__ idx, int64_t n_tok, const uint4* __restrict__ tables,
@@ -65,7 +65,7 @@ cudaError_t launch_gather(const uint32_t* idx, int64_t n_tok, const void* tables
     const int per_tok = gp.J * gp.chunks_per_row;
     const int threads = per_tok >= 256 ? 256 : ((per_tok + 31) / 32) * 32;
     const int64_t want = (n_tok + kTokBatch - 1) / kTokBatch;
-    const int64_t cap = (int64_t)num_sms * (2048 / threads);
+    const int64_t cap = (int64_t)num_sms * (4096 / threads);
     const int64_t blocks = want < cap ? want : cap;
     gather_kernel<<<(unsigned)blocks, threads, 0, s>>>(idx, n_tok, static_cast<const uint4*>(tables), gp,
                                                        static_cast<uint4*>(e_cat), status);

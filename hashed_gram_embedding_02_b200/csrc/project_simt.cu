@@ -4,10 +4,10 @@
 // v_t = W_V e_t; RMSNorm is applied to the query h_t and to the key before
 // the scalar gate.  This kernel computes, for a tile of 32 rows and one
 // group of 128 channels, both k and v (fp32 accumulation in a fixed order),
-// writes v in the storage dtype and reduces the group's gate partials
+// writes v in fp32 and reduces the group's gate partials
 //   (sum g_q g_k h k, sum k^2, sum h^2)
 // so that k is never written to memory.  It serves the fp32 configuration
-// and bf16 shapes that the tensor-core kernel does not tile.
+// and bf16 shapes that the tensor-core kernels do not tile.
 #include "common.cuh"
 
 namespace engram {
@@ -22,7 +22,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 project_simt_kernel(const T* __restrict__ e, int64_t n_tok, int32_t d_mem, const T* __restrict__ h,
                     const T* __restrict__ Wk, const T* __restrict__ Wv, const float* __restrict__ gq,
-                    const float* __restrict__ gk, int32_t d, T* __restrict__ v, float* __restrict__ part) {
+                    const float* __restrict__ gk, int32_t d, float* __restrict__ v, float* __restrict__ part) {
     __shared__ float e_s[kRows][kKc + 1];
     __shared__ float wk_s[kGroup][kKc + 1];
     __shared__ float wv_s[kGroup][kKc + 1];
@@ -84,9 +84,7 @@ project_simt_kernel(const T* __restrict__ e, int64_t n_tok, int32_t d_mem, const
         const int64_t row = r0 + rr;
         float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
         if (row < n_tok && c < d) {
-            T vo;
-            from_f(vo, acc_v[i]);
-            v[row * d + c] = vo;
+            v[row * d + c] = acc_v[i];
             const float hv = to_f(h[row * d + c]);
             s_qk = gg * hv * acc_k[i];
             s_kk = acc_k[i] * acc_k[i];
@@ -123,19 +121,18 @@ project_simt_kernel(const T* __restrict__ e, int64_t n_tok, int32_t d_mem, const
 
 cudaError_t launch_project_simt(bool bf16, const void* e, int64_t n_tok, int32_t d_mem, const void* h,
                                 const void* Wk, const void* Wv, const float* gq, const float* gk, int32_t d,
-                                void* v, float* part, cudaStream_t s) {
+                                float* v, float* part, cudaStream_t s) {
     if (n_tok == 0) return cudaSuccess;
     dim3 grid((unsigned)((n_tok + kRows - 1) / kRows), (unsigned)((d + kGroup - 1) / kGroup));
     if (bf16) {
         using T = __nv_bfloat16;
         project_simt_kernel<T><<<grid, kThreads, 0, s>>>(
             static_cast<const T*>(e), n_tok, d_mem, static_cast<const T*>(h), static_cast<const T*>(Wk),
-            static_cast<const T*>(Wv), gq, gk, d, static_cast<T*>(v), part);
+            static_cast<const T*>(Wv), gq, gk, d, v, part);
     } else {
         project_simt_kernel<float><<<grid, kThreads, 0, s>>>(
             static_cast<const float*>(e), n_tok, d_mem, static_cast<const float*>(h),
-            static_cast<const float*>(Wk), static_cast<const float*>(Wv), gq, gk, d, static_cast<float*>(v),
-            part);
+            static_cast<const float*>(Wk), static_cast<const float*>(Wv), gq, gk, d, v, part);
     }
     return cudaGetLastError();
 }

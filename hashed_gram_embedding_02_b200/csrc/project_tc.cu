@@ -1,27 +1,37 @@
 // Key/value projections on the 5th-generation tensor cores (tcgen05), with
-// the gate's partial sums in the epilogue.
+// the gate and the causal convolution fused into the GEMM epilogues.
 //
 // "DeepSeek AI II" digest, section "DeepSeek Engram": k_t = W_K e_t and
-// v_t = W_V e_t feed an RMSNorm'd dot product with the query h_t (the
-// multi-branch variant fuses all projections into one dense GEMM "to maximise
-// GPU utilisation").  Here one GEMM computes [k | v] = e [W_K; W_V]^T:
+// v_t = W_V e_t; RMSNorm on the query h_t and on the key; a scalar gate
+// alpha_t in (0,1); v~_t = alpha_t v_t; a short-kernel per-channel causal
+// convolution; Y added to the residual stream.  (The multi-branch variant of
+// the same section fuses the projections into one dense GEMM to keep the GPU
+// busy.)  One kernel template, three epilogues:
 //
-//   A = e      [n_tok][d_mem] bf16, K-major
-//   B = W_K, W_V [d][d_mem]   bf16, K-major (nn.Linear layout)
-//   CTA tile   128 rows x (128 k-channels + the same 128 v-channels), K step 64
+//   MODE_KV    tile = 128 rows x (128 k-channels | the same 128 v-channels):
+//              writes v (fp32) and the group's gate partials; the standalone
+//              engram_project.
+//   MODE_K     tile = 128 rows x BN k-channels: writes the gate partials
+//              (sum g_q g_k h k, sum k^2, sum h^2) of its BN/128 channel
+//              groups; k never leaves the SM.
+//   MODE_VCONV tile = 128 rows x BN v-channels, row tiles overlapping by the
+//              conv history (w-1 rows): each thread owns one TMEM lane (one
+//              row), reduces its row's partials into alpha, forms v~ = alpha v,
+//              takes v~ of the w-1 previous rows from the neighbouring lanes
+//              (warp shuffles, plus a shared-memory hand-over between the four
+//              epilogue warps), applies the conv taps, SiLU, the residual, and
+//              writes Y.  v itself never reaches global memory.
 //
 // Persistent kernel, one CTA per SM, warp-specialised:
-//   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of the A tile
-//              and of the W_K and W_V tiles into a 4-stage shared-memory ring
-//   warp 1     allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
-//              issues tcgen05.mma kind::f16 (M=128, N=256, K=16) from one thread
-//   warps 4-7  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM
-//              lanes 32(w-4)..32(w-4)+31), store v as bf16, and reduce the
-//              group's gate partials (sum g_q g_k h k, sum k^2, sum h^2); the
-//              key k never leaves the SM
+//   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of the A
+//              (e) tile and the W tile(s) into a shared-memory ring
+//   warp 1     allocates TMEM (two fp32 accumulators) and issues
+//              tcgen05.mma kind::f16 (M=128, N=BN, K=16) from one thread
+//   warps 4-7  epilogue: tcgen05.ld of the accumulator; warp w reads TMEM
+//              lanes 32(w-4) .. 32(w-4)+31
 // The double-buffered accumulator lets the epilogue of tile i overlap the
-// MMAs of tile i+1.  Tiles run channel-group-fastest so that consecutive tiles
-// share the A block in L2; all of W stays L2-resident.
+// MMAs of tile i+1.  Tiles run channel-fastest so consecutive tiles share the
+// A block in L2; W stays L2-resident.
 //
 // Every mbarrier wait is bounded (about 2 s of clock64 time).  A wait that runs
 // out sets ENGRAM_ERR_TIMEOUT, raises a CTA-wide abort flag that makes the
@@ -30,29 +40,39 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace engram {
 
 namespace {
 
+constexpr int MODE_KV = 0;
+constexpr int MODE_K = 1;
+constexpr int MODE_VCONV = 2;
+
 constexpr int BM = 128;                 // rows per tile (UMMA M)
-constexpr int BNH = 128;                // channels per tile (k and v halves)
-constexpr int BN = 2 * BNH;             // UMMA N
 constexpr int BK = 64;                  // K per stage: 64 bf16 = 128 bytes = one swizzle row
 constexpr int UK = 16;                  // K per tcgen05.mma kind::f16
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;    // 16 KB
-constexpr int B_BYTES = BN * BK * 2;    // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int THREADS = 256;
-constexpr int SMEM_TILES = STAGES * STAGE_BYTES;
-constexpr int SMEM_BYTES = SMEM_TILES + 1024 /* barriers */ + 1024 /* alignment slack */;
-constexpr long long WAIT_CYCLES = 4000000000LL;   // ~2 s at 1.9 GHz
+constexpr int kMaxHist = kMaxConv - 1;
+
+template <int BN>
+struct Geo {
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int SMEM_TILES = STAGES * STAGE_BYTES;
+    // tiles | barriers (1 KB) | conv taps [2][BN * 8] fp32 | hand-over [2][4][kMaxHist][32] fp32 | slack
+    static constexpr int CW_BYTES = 2 * BN * kMaxConv * 4;
+    static constexpr int XB_BYTES = 2 * 4 * kMaxHist * 32 * 4;
+    static constexpr int SMEM_BYTES = SMEM_TILES + 1024 + CW_BYTES + XB_BYTES + 1024;
+};
 
 struct __align__(8) Barriers {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[8];
+    uint64_t empty[8];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -62,34 +82,28 @@ struct __align__(8) Barriers {
     int consumed;     // k-block stages consumed by the MMA issuer
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
+struct EpiParams {
+    const __nv_bfloat16* h;     // [n_tok][d]
+    const float* gq;            // [d] or null
+    const float* gk;            // [d] or null
+    float* v;                   // MODE_KV: [n_tok][d] fp32
+    float4* part;               // [n_tok][G]: written (KV, K), read (VCONV)
+    const float* conv_w;        // [d][w]
+    const float* state;         // [B][w-1][d] history, or null (zero history)
+    float* state_next;          // [B][w-1][d] new history (merged by a second kernel), or null
+    __nv_bfloat16* y;           // [n_tok][d]
+    float* alpha_out;           // [n_tok] or null
+    uint32_t* status;
+    int n_tok, d_mem, d, G;
+    int n_groups;               // tiles along the channel dimension
+    int num_tiles;
+    int m_stride;               // rows advanced per row tile (128, or 128 - (w-1) in MODE_VCONV)
+    int halo;                   // leading rows of a tile that are history only (MODE_VCONV)
+    int L;                      // rows per sequence
+    int w;                      // conv width
+    int add_residual;
+    float eps;
+};
 
 // Bounded wait: true when the phase with `parity` completed, false when the
 // CTA aborted or the wait ran out (then the status bit and abort flag are set).
@@ -100,7 +114,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bar
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (sb->abort_flag) return false;
-        if (clock64() - t0 > WAIT_CYCLES) {
+        if (clock64() - t0 > kWaitCycles) {
             flag(status, ENGRAM_ERR_TIMEOUT);
             sb->abort_flag = 1;
             return false;
@@ -132,16 +146,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// K-major, N = BN, M = 128.
+template <int BN>
+struct Idesc {
+    static constexpr uint32_t value =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+};
 
+template <int BN>
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
-        ::"r"(tmem_d), "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate));
+        ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN>::value), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -166,20 +184,233 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// named barrier among the four epilogue warps (id 1; id 0 is __syncthreads)
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// the same barrier as a vote: true on every epilogue thread when any passed true
+__device__ __forceinline__ bool epi_any(bool x) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)x)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float silu_bf16out(float x) {
+    // x * sigmoid(x) = hx + hx * tanh(hx), hx = x/2; hardware tanh approximation
+    // (relative error about 2^-11, below the bf16 rounding of Y)
+    const float hx = 0.5f * x;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hx));
+    return fmaf(hx, t, hx);
+}
+
+// ---------------------------------------------------------------- epilogues
+
+// gate partials of one 128-channel group from 128 k columns at taddr
+__device__ __forceinline__ void partials_128(uint32_t taddr, const EpiParams& p, int64_t row, bool valid, int c0,
+                                             float& s_qk, float& s_kk, float& s_hh) {
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t kr[32];
+        tmem_ld32(taddr + ch * 32, kr);
+        tmem_wait_ld();
+        if (valid) {
+            const uint4* hp = reinterpret_cast<const uint4*>(p.h + row * p.d + c0 + ch * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint4 hv = __ldg(hp + u);
+                const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int i = u * 8 + q * 2 + half;
+                        const int c = c0 + ch * 32 + i;
+                        const float hf = half ? bf16_hi(hw[q]) : bf16_lo(hw[q]);
+                        const float kf = __uint_as_float(kr[i]);
+                        const float gg = (p.gq ? __ldg(p.gq + c) : 1.f) * (p.gk ? __ldg(p.gk + c) : 1.f);
+                        s_qk = fmaf(gg * hf, kf, s_qk);
+                        s_kk = fmaf(kf, kf, s_kk);
+                        s_hh = fmaf(hf, hf, s_hh);
+                    }
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void epilogue_kv(uint32_t taddr, const EpiParams& p, int m0, int nt, int q, int lane) {
+    const int64_t row = (int64_t)m0 + q * 32 + lane;
+    const bool valid = row < p.n_tok;
+    const int c0 = nt * 128;
+    float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+    partials_128(taddr, p, row, valid, c0, s_qk, s_kk, s_hh);
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t vr[32];
+        tmem_ld32(taddr + 128 + ch * 32, vr);
+        tmem_wait_ld();
+        if (valid) {
+            float4* vp = reinterpret_cast<float4*>(p.v + row * p.d + c0 + ch * 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                vp[u] = make_float4(__uint_as_float(vr[4 * u]), __uint_as_float(vr[4 * u + 1]),
+                                    __uint_as_float(vr[4 * u + 2]), __uint_as_float(vr[4 * u + 3]));
+        }
+    }
+    if (valid) p.part[row * p.G + nt] = make_float4(s_qk, s_kk, s_hh, 0.f);
+}
+
+template <int BN>
+__device__ __forceinline__ void epilogue_k(uint32_t taddr, const EpiParams& p, int m0, int nt, int q, int lane) {
+    const int64_t row = (int64_t)m0 + q * 32 + lane;
+    const bool valid = row < p.n_tok;
+#pragma unroll 1
+    for (int gi = 0; gi < BN / 128; ++gi) {
+        const int g = nt * (BN / 128) + gi;
+        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+        partials_128(taddr + gi * 128, p, row, valid, g * 128, s_qk, s_kk, s_hh);
+        if (valid) p.part[row * p.G + g] = make_float4(s_qk, s_kk, s_hh, 0.f);
+    }
+}
+
+// Gate + causal depthwise conv + residual on a v tile.  TMEM lane i holds flat
+// row m0 + i; lanes below `halo` are history rows of the previous tile.
+template <int BN>
+__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const EpiParams& p, int m0, int nt, int q, int lane,
+                                               int tcount, uint32_t& xcount, float* s_cw, float* s_xb) {
+    const int i = q * 32 + lane;
+    const int64_t r = (int64_t)m0 + i;
+    const bool in_range = r >= 0 && r < p.n_tok;
+    const bool out_row = in_range && i >= p.halo;
+    const int W = p.w, H = W - 1;
+    int64_t b = 0;
+    int t = 0;
+    if (in_range) {
+        b = r / p.L;
+        t = (int)(r - b * p.L);
+    }
+    // alpha of this row: fixed-order sum of its G partials
+    float a = 0.f;
+    if (in_range) {
+        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+        const float4* pp = p.part + r * p.G;
+        for (int g = 0; g < p.G; ++g) {
+            const float4 v4 = pp[g];
+            s_qk += v4.x;
+            s_kk += v4.y;
+            s_hh += v4.z;
+        }
+        const float inv_d = 1.f / (float)p.d;
+        const float rh = sqrtf(s_hh * inv_d + p.eps);
+        const float rk = sqrtf(s_kk * inv_d + p.eps);
+        a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)p.d)));
+    }
+    if (out_row && nt == 0 && p.alpha_out) p.alpha_out[r] = a;
+
+    // conv taps of this tile's channels into shared memory (double-buffered by tile)
+    const int n0 = nt * BN;
+    float* cw = s_cw + (tcount & 1) * (BN * kMaxConv);
+    for (int k = i; k < BN * W; k += 128) cw[k] = __ldg(p.conv_w + (int64_t)n0 * W + k);
+    epi_sync();
+
+    const bool has_state = p.state != nullptr;
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t vr[32];
+        tmem_ld32(taddr + ch * 32, vr);
+        tmem_wait_ld();
+        float vt[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) vt[c] = a * __uint_as_float(vr[c]);
+        // hand the last H lanes' values to the next warp
+        float* xb = s_xb + (xcount & 1) * (4 * kMaxHist * 32);
+        if (lane >= 32 - H) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) xb[(q * kMaxHist + (lane - (32 - H))) * 32 + c] = vt[c];
+        }
+        epi_sync();
+        ++xcount;
+        const int cbase = n0 + ch * 32;
+        float yv[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) yv[c] = 0.f;
+#pragma unroll 1
+        for (int j = 1; j < W; ++j) {
+            const bool from_prev = lane < j;
+            const bool before_seq = t < j;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float pv = __shfl_up_sync(0xffffffffu, vt[c], j);
+                if (from_prev) pv = q > 0 ? xb[((q - 1) * kMaxHist + (H - j + lane)) * 32 + c] : 0.f;
+                if (before_seq) pv = has_state ? p.state[(b * H + (H + t - j)) * p.d + cbase + c] : 0.f;
+                yv[c] = fmaf(cw[(ch * 32 + c) * W + j], pv, yv[c]);
+            }
+        }
+        if (out_row) {
+            float hv[32];
+            if (p.add_residual) {
+                const uint4* hp = reinterpret_cast<const uint4*>(p.h + r * p.d + cbase);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint4 q4 = __ldg(hp + u);
+                    hv[8 * u + 0] = bf16_lo(q4.x); hv[8 * u + 1] = bf16_hi(q4.x);
+                    hv[8 * u + 2] = bf16_lo(q4.y); hv[8 * u + 3] = bf16_hi(q4.y);
+                    hv[8 * u + 4] = bf16_lo(q4.z); hv[8 * u + 5] = bf16_hi(q4.z);
+                    hv[8 * u + 6] = bf16_lo(q4.w); hv[8 * u + 7] = bf16_hi(q4.w);
+                }
+            }
+            uint4* yp = reinterpret_cast<uint4*>(p.y + r * p.d + cbase);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = 8 * u + e;
+                    const float uu = fmaf(cw[(ch * 32 + c) * W], vt[c], yv[c]);
+                    float res = vt[c] + silu_bf16out(uu);
+                    if (p.add_residual) res += hv[c];
+                    o[e] = res;
+                }
+                yp[u] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                   pack_bf16x2(o[6], o[7]));
+            }
+            // the last H rows of a sequence become its next conv history
+            if (p.state_next && t >= p.L - H) {
+                float* sp = p.state_next + (b * H + (t - (p.L - H))) * p.d + cbase;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sp[c] = vt[c];
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- kernel
+
+template <int MODE, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
-project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_wk,
-                  const __grid_constant__ CUtensorMap map_wv, const __nv_bfloat16* __restrict__ h,
-                  const float* __restrict__ gq, const float* __restrict__ gk, __nv_bfloat16* __restrict__ v,
-                  float4* __restrict__ part, uint32_t* status, int n_tok, int d_mem, int d, int G, int num_tiles) {
+project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
+                  const __grid_constant__ CUtensorMap map_b1, const EpiParams p) {
+    using GE = Geo<BN>;
+    constexpr int STAGES = GE::STAGES;
+    constexpr int STAGE_BYTES = GE::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);   // 1024-byte aligned tile base
     const uint32_t tiles_u32 = smem_u32(smem);
-    Barriers* sb = reinterpret_cast<Barriers*>(smem + SMEM_TILES);
+    Barriers* sb = reinterpret_cast<Barriers*>(smem + GE::SMEM_TILES);
+    float* s_cw = reinterpret_cast<float*>(smem + GE::SMEM_TILES + 1024);
+    float* s_xb = reinterpret_cast<float*>(smem + GE::SMEM_TILES + 1024 + GE::CW_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int KB = d_mem / BK;
+    const int KB = p.d_mem / BK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -194,15 +425,15 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         sb->abort_flag = 0;
         sb->issued = 0;
         sb->consumed = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_fence_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&map_a);
-        tma_prefetch_desc(&map_wk);
-        tma_prefetch_desc(&map_wv);
+        tma_prefetch_desc(&map_b0);
+        if (MODE == MODE_KV) tma_prefetch_desc(&map_b1);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sb->tmem_base)),
-                     "r"(TMEM_COLS)
+                     "r"(GE::TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -215,19 +446,23 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         // ---------------- TMA producer
         if (lane == 0) {
             int it = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && !sb->abort_flag; tile += gridDim.x) {
-                const int m0 = (tile / G) * BM;
-                const int c0 = (tile % G) * BNH;
+            for (int tile = blockIdx.x; tile < p.num_tiles && !sb->abort_flag; tile += gridDim.x) {
+                const int mt = tile / p.n_groups, nt = tile % p.n_groups;
+                const int m0 = mt * p.m_stride - p.halo;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!wait_bounded(&sb->empty[s], ph ^ 1u, sb, status)) break;
+                    if (!wait_bounded(&sb->empty[s], ph ^ 1u, sb, p.status)) break;
                     const uint32_t a_dst = tiles_u32 + s * STAGE_BYTES;
                     const uint32_t b_dst = a_dst + A_BYTES;
                     mbar_arrive_expect_tx(&sb->full[s], STAGE_BYTES);
                     tma_load_2d(&map_a, a_dst, &sb->full[s], kb * BK, m0);
-                    tma_load_2d(&map_wk, b_dst, &sb->full[s], kb * BK, c0);
-                    tma_load_2d(&map_wv, b_dst + BNH * BK * 2, &sb->full[s], kb * BK, c0);
+                    if (MODE == MODE_KV) {
+                        tma_load_2d(&map_b0, b_dst, &sb->full[s], kb * BK, nt * 128);
+                        tma_load_2d(&map_b1, b_dst + 128 * BK * 2, &sb->full[s], kb * BK, nt * 128);
+                    } else {
+                        tma_load_2d(&map_b0, b_dst, &sb->full[s], kb * BK, nt * BN);
+                    }
                     sb->issued = it + 1;
                 }
             }
@@ -236,17 +471,17 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         // ---------------- MMA issuer
         if (lane == 0) {
             int it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && !sb->abort_flag; tile += gridDim.x, ++tc) {
+            for (int tile = blockIdx.x; tile < p.num_tiles && !sb->abort_flag; tile += gridDim.x, ++tc) {
                 const int acc = tc & 1;
                 const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
-                if (!wait_bounded(&sb->tempty[acc], aph ^ 1u, sb, status)) break;
+                if (!wait_bounded(&sb->tempty[acc], aph ^ 1u, sb, p.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!wait_bounded(&sb->full[s], ph, sb, status)) {
+                    if (!wait_bounded(&sb->full[s], ph, sb, p.status)) {
                         ok = false;
                         break;
                     }
@@ -257,7 +492,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
                         // +32 bytes along K inside the swizzled 128-byte row
-                        umma_bf16(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
+                        umma_bf16<BN>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
                     }
                     umma_commit(&sb->empty[s]);
                     sb->consumed = it + 1;
@@ -270,67 +505,22 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         // ---------------- epilogue
         const int q = warp - 4;
         int tc = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+        uint32_t xcount = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tc) {
             const int acc = tc & 1;
             const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
-            if (!wait_bounded(&sb->tfull[acc], aph, sb, status)) break;
+            const bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
+            if (epi_any(!ok)) break;          // one decision for all four warps
             tc_fence_after();
-            const int g = tile % G;
-            const int c0 = g * BNH;
-            const int64_t row = (int64_t)(tile / G) * BM + q * 32 + lane;
-            const bool valid = row < n_tok;
+            const int mt = tile / p.n_groups, nt = tile % p.n_groups;
+            const int m0 = mt * p.m_stride - p.halo;
             const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-            float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-#pragma unroll 1
-            for (int ch = 0; ch < BNH / 32; ++ch) {
-                uint32_t kr[32];
-                tmem_ld32(taddr + ch * 32, kr);
-                tmem_wait_ld();
-                if (valid) {
-                    const uint4* hp = reinterpret_cast<const uint4*>(h + row * d + c0 + ch * 32);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint4 hv = __ldg(hp + u);
-                        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-#pragma unroll
-                            for (int half = 0; half < 2; ++half) {
-                                const int i = u * 8 + p * 2 + half;
-                                const int c = c0 + ch * 32 + i;
-                                const float hf = half ? bf16_hi(hw[p]) : bf16_lo(hw[p]);
-                                const float kf = __uint_as_float(kr[i]);
-                                const float gg = (gq ? __ldg(gq + c) : 1.f) * (gk ? __ldg(gk + c) : 1.f);
-                                s_qk = fmaf(gg * hf, kf, s_qk);
-                                s_kk = fmaf(kf, kf, s_kk);
-                                s_hh = fmaf(hf, hf, s_hh);
-                            }
-                        }
-                    }
-                }
-            }
-#pragma unroll 1
-            for (int ch = 0; ch < BNH / 32; ++ch) {
-                uint32_t vr[32];
-                tmem_ld32(taddr + BNH + ch * 32, vr);
-                tmem_wait_ld();
-                if (valid) {
-                    uint4* vp = reinterpret_cast<uint4*>(v + row * d + c0 + ch * 32);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(vr[u * 8 + 0]), __uint_as_float(vr[u * 8 + 1]));
-                        o.y = pack_bf16x2(__uint_as_float(vr[u * 8 + 2]), __uint_as_float(vr[u * 8 + 3]));
-                        o.z = pack_bf16x2(__uint_as_float(vr[u * 8 + 4]), __uint_as_float(vr[u * 8 + 5]));
-                        o.w = pack_bf16x2(__uint_as_float(vr[u * 8 + 6]), __uint_as_float(vr[u * 8 + 7]));
-                        vp[u] = o;
-                    }
-                }
-            }
+            if (MODE == MODE_KV) epilogue_kv(taddr, p, m0, nt, q, lane);
+            if (MODE == MODE_K) epilogue_k<BN>(taddr, p, m0, nt, q, lane);
+            if (MODE == MODE_VCONV) epilogue_vconv<BN>(taddr, p, m0, nt, q, lane, tc, xcount, s_cw, s_xb);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sb->tempty[acc]);
-            if (valid) part[row * G + g] = make_float4(s_qk, s_kk, s_hh, 0.f);
         }
     }
 
@@ -342,22 +532,37 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 const int s = it % STAGES;
                 const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                 const long long t0 = clock64();
-                while (!mbar_try_wait(smem_u32(&sb->full[s]), ph) && clock64() - t0 < WAIT_CYCLES) {
+                while (!mbar_try_wait(smem_u32(&sb->full[s]), ph) && clock64() - t0 < kWaitCycles) {
                 }
             }
         }
         if (warp == 1 && lane == 0) {
             umma_commit(&sb->drain);
             const long long t0 = clock64();
-            while (!mbar_try_wait(smem_u32(&sb->drain), 0) && clock64() - t0 < WAIT_CYCLES) {
+            while (!mbar_try_wait(smem_u32(&sb->drain), 0) && clock64() - t0 < kWaitCycles) {
             }
         }
         __syncthreads();
     }
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GE::TMEM_COLS)
                      : "memory");
+    }
+}
+
+// merge the new conv history: rows of the old history that are still inside
+// the window (L < w-1) shift down; the rest come from state_next.  In order
+// of increasing row, so the update is in place.
+__global__ void state_merge_kernel(float* state, const float* state_next, int B, int L, int H, int d) {
+    const int64_t n = (int64_t)B * d;
+    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t b = k / d, c = k - b * d;
+        for (int i = 0; i < H; ++i) {
+            const int p = L - H + i;
+            const float val = p >= 0 ? state_next[(b * H + i) * d + c] : state[(b * H + (L + i)) * d + c];
+            state[(b * H + i) * d + c] = val;
+        }
     }
 }
 
@@ -372,17 +577,17 @@ EncodeTiledFn encode_fn() {
     static bool tried = false;
     if (!tried) {
         tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
+        void* q = nullptr;
+        cudaDriverEntryPointQueryResult res;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &res) == cudaSuccess &&
+            res == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(q);
     }
     return fn;
 }
 
 // 2-D bf16 row-major [rows][cols] map with a box of box_rows x 64 columns
-// (128 bytes, 128-byte swizzle); rows beyond `rows` read as zero.
+// (128 bytes, 128-byte swizzle); rows outside [0, rows) read as zero.
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -395,36 +600,132 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d) {
-    return n_tok > 0 && n_tok < (int64_t)1 << 31 && d_mem % BK == 0 && d_mem >= BK && d % BNH == 0 &&
-           encode_fn() != nullptr;
-}
-
-cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
-                              const void* Wv, const float* gq, const float* gk, int32_t d, void* v, float* part,
-                              uint32_t* status, int num_sms, cudaStream_t s) {
-    if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
-    CUtensorMap ma, mk, mv;
-    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, BNH) ||
-        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, BNH))
-        return cudaErrorInvalidValue;
+template <int MODE, int BN>
+cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, EpiParams p,
+                        int64_t m_tiles, int num_sms, cudaStream_t s) {
+    using GE = Geo<BN>;
     static unsigned long long attr_set = 0;   // one bit per device ordinal
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !(attr_set >> dev & 1ull)) {
-        cudaError_t err = cudaFuncSetAttribute(project_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaError_t err = cudaFuncSetAttribute(project_tc_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               GE::SMEM_BYTES);
         if (err != cudaSuccess) return err;
         attr_set |= 1ull << dev;
     }
-    const int G = d / BNH;
-    const int64_t m_blocks = (n_tok + BM - 1) / BM;
-    const int64_t tiles = m_blocks * G;
+    const int64_t tiles = m_tiles * p.n_groups;
+    if (tiles >= (int64_t)1 << 31) return cudaErrorInvalidValue;
+    p.num_tiles = (int)tiles;
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    project_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mk, mv, static_cast<const __nv_bfloat16*>(h), gq, gk,
-                                                        static_cast<__nv_bfloat16*>(v), reinterpret_cast<float4*>(part),
-                                                        status, (int)n_tok, d_mem, d, G, (int)tiles);
+    project_tc_kernel<MODE, BN><<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, p);
+    return cudaGetLastError();
+}
+
+int pick_bn(int32_t d) { return d % 256 == 0 ? 256 : 128; }
+
+}  // namespace
+
+bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d) {
+    return n_tok > 0 && n_tok < (int64_t)1 << 30 && d_mem % BK == 0 && d_mem >= BK && d % 128 == 0 &&
+           encode_fn() != nullptr;
+}
+
+cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
+                              const void* Wv, const float* gq, const float* gk, int32_t d, float* v, float* part,
+                              uint32_t* status, int num_sms, cudaStream_t s) {
+    if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
+    CUtensorMap ma, mk, mv;
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, 128) ||
+        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, 128))
+        return cudaErrorInvalidValue;
+    EpiParams p{};
+    p.h = static_cast<const __nv_bfloat16*>(h);
+    p.gq = gq;
+    p.gk = gk;
+    p.v = v;
+    p.part = reinterpret_cast<float4*>(part);
+    p.status = status;
+    p.n_tok = (int)n_tok;
+    p.d_mem = d_mem;
+    p.d = d;
+    p.G = d / 128;
+    p.n_groups = d / 128;
+    p.m_stride = BM;
+    p.halo = 0;
+    return launch_mode<MODE_KV, 256>(ma, mk, mv, p, (n_tok + BM - 1) / BM, num_sms, s);
+}
+
+cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
+                             const float* gq, const float* gk, int32_t d, float* part, uint32_t* status, int num_sms,
+                             cudaStream_t s) {
+    if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
+    const int bn = pick_bn(d);
+    CUtensorMap ma, mk;
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn))
+        return cudaErrorInvalidValue;
+    EpiParams p{};
+    p.h = static_cast<const __nv_bfloat16*>(h);
+    p.gq = gq;
+    p.gk = gk;
+    p.part = reinterpret_cast<float4*>(part);
+    p.status = status;
+    p.n_tok = (int)n_tok;
+    p.d_mem = d_mem;
+    p.d = d;
+    p.G = d / 128;
+    p.n_groups = d / bn;
+    p.m_stride = BM;
+    p.halo = 0;
+    const int64_t mt = (n_tok + BM - 1) / BM;
+    return bn == 256 ? launch_mode<MODE_K, 256>(ma, mk, mk, p, mt, num_sms, s)
+                     : launch_mode<MODE_K, 128>(ma, mk, mk, p, mt, num_sms, s);
+}
+
+cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
+                            const float* conv_w, int32_t d, int32_t w, float eps, const float* part,
+                            const float* state, float* state_next, void* y, float* alpha_out, int32_t add_residual,
+                            uint32_t* status, int num_sms, cudaStream_t s) {
+    const int64_t n_tok = (int64_t)B * L;
+    if (!project_tc_supported(n_tok, d_mem, d) || w < 1 || w > kMaxConv) return cudaErrorNotSupported;
+    const int bn = pick_bn(d);
+    const int H = w - 1;
+    CUtensorMap ma, mv;
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn))
+        return cudaErrorInvalidValue;
+    EpiParams p{};
+    p.h = static_cast<const __nv_bfloat16*>(h);
+    p.part = const_cast<float4*>(reinterpret_cast<const float4*>(part));
+    p.conv_w = conv_w;
+    p.state = state;
+    p.state_next = state ? state_next : nullptr;
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.alpha_out = alpha_out;
+    p.status = status;
+    p.n_tok = (int)n_tok;
+    p.d_mem = d_mem;
+    p.d = d;
+    p.G = d / 128;
+    p.n_groups = d / bn;
+    p.L = L;
+    p.w = w;
+    p.add_residual = add_residual;
+    p.eps = eps;
+    // row tiles overlap by the H history rows
+    p.m_stride = BM - H;
+    p.halo = H;
+    const int64_t mt = (n_tok + p.m_stride - 1) / p.m_stride;
+    return bn == 256 ? launch_mode<MODE_VCONV, 256>(ma, mv, mv, p, mt, num_sms, s)
+                     : launch_mode<MODE_VCONV, 128>(ma, mv, mv, p, mt, num_sms, s);
+}
+
+cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,
+                               int num_sms, cudaStream_t s) {
+    const int H = w - 1;
+    if (H <= 0 || B == 0) return cudaSuccess;
+    const int64_t n = (int64_t)B * d;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > num_sms * 8) blocks = num_sms * 8;
+    state_merge_kernel<<<(unsigned)blocks, 256, 0, s>>>(state, state_next, B, L, H, d);
     return cudaGetLastError();
 }
 

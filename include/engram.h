@@ -118,10 +118,22 @@ ENGRAM_API const char* engram_strerror(engram_status s);
  * or CUDA error with its call site); empty when none.  Owned by the library. */
 ENGRAM_API const char* engram_last_error(void);
 
-/* Bytes of scratch that engram_forward / engram_gate_conv need for n_tok rows:
- * indices [n_tok][J] u32, e [n_tok][J*D], v [n_tok][d] and gate partials
- * [n_tok][G][4] f32 with G = ceil(d / 128), each 256-byte aligned. */
-ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int64_t n_tok);
+/* Bytes of scratch that engram_forward / engram_gate_conv need for B
+ * sequences of L computed rows (n_tok = B*L): indices [n_tok][J] u32,
+ * e [n_tok][J*D], gate partials [n_tok][G][4] f32 with G = ceil(d / 128), the
+ * next conv history [B][w-1][d] f32 and, where the projection runs on CUDA
+ * cores (fp32 configurations and shapes the tensor-core kernels do not tile),
+ * v [n_tok][d] f32; each part 256-byte aligned.  0 for a null context. */
+ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int32_t B, int32_t L);
+
+/* Per-kernel timing for benchmarks.  While enabled, every entry point records
+ * a pair of CUDA events (created here, on the context's device) around each
+ * kernel it launches on the caller's stream; engram_profile_read waits for
+ * the events of the most recent call and writes up to `max` durations in
+ * milliseconds and kernel names (library-owned strings) in launch order,
+ * returning how many.  Not thread-safe; disable to free the events. */
+ENGRAM_API engram_status engram_profile_enable(engram_ctx* ctx, int32_t enable);
+ENGRAM_API int32_t engram_profile_read(engram_ctx* ctx, float* ms, const char** names, int32_t max);
 
 /* Synchronise `stream`, return the device status word in *flags (nullable)
  * and clear it.  ENGRAM_OK when it was zero, ENGRAM_E_TIMEOUT when the
@@ -156,27 +168,32 @@ ENGRAM_API engram_status engram_gather(engram_ctx* ctx, const uint32_t* idx, int
 /* Key/value projections with the gate's partial sums (same section: k = W_K e,
  * v = W_V e; RMSNorm on query and key).  Wk and Wv are [d][J*D] (nn.Linear
  * layout), h is [n_tok][d], gq/gk are [d] fp32 RMSNorm gains (null = ones).
- * Writes v [n_tok][d] in the context dtype and part [n_tok][G][4] fp32,
- * G = ceil(d/128): for channel group g, part = (sum g_q g_k h k, sum k^2,
- * sum h^2, 0) over the group's channels.  k itself is never stored. */
+ * Writes v [n_tok][d] in fp32 and part [n_tok][G][4] fp32, G = ceil(d/128):
+ * for channel group g, part = (sum g_q g_k h k, sum k^2, sum h^2, 0) over the
+ * group's channels.  k itself is never stored. */
 ENGRAM_API engram_status engram_project(engram_ctx* ctx, const void* e_cat, int64_t n_tok, const void* h,
                              const void* Wk, const void* Wv, const float* gq, const float* gk,
-                             void* v, float* part, cudaStream_t stream);
+                             float* v, float* part, cudaStream_t stream);
 
 /* Gate and causal depthwise convolution (same section: alpha_t in (0,1),
  * v~ = alpha v, short-kernel per-channel causal conv; residual H <- H + Y).
- * v and part as written by engram_project for B sequences of L rows each;
- * conv_w is [d][w] fp32 (tap j multiplies v~_{t-j}); conv_state (nullable)
- * is [B][w-1][d] fp32 holding v~ of the w-1 positions before the first row
- * (row w-2 most recent): read as history and overwritten with the last w-1
- * v~ rows of the extended sequence (in place is safe).  Null: zero history.
- * h is read only when add_residual != 0.  y is [B*L][d] (context dtype);
- * alpha_out (nullable) [B*L] fp32. */
-ENGRAM_API engram_status engram_conv(engram_ctx* ctx, const void* v, const float* part, const void* h,
+ * v (fp32) and part as written by engram_project for B sequences of L rows
+ * each; conv_w is [d][w] fp32 (tap j multiplies v~_{t-j}); conv_state
+ * (nullable) is [B][w-1][d] fp32 holding v~ of the w-1 positions before the
+ * first row (row w-2 most recent): read as history and overwritten with the
+ * last w-1 v~ rows of the extended sequence (in place is safe).  Null: zero
+ * history.  h is read only when add_residual != 0.  y is [B*L][d] (context
+ * dtype); alpha_out (nullable) [B*L] fp32. */
+ENGRAM_API engram_status engram_conv(engram_ctx* ctx, const float* v, const float* part, const void* h,
                           const float* conv_w, int32_t B, int32_t L, float* conv_state, void* y,
                           float* alpha_out, int32_t add_residual, cudaStream_t stream);
 
-/* engram_project followed by engram_conv, v and part in `workspace`. */
+/* Projections, gate and conv from e: on bf16 tensor-core shapes (d a
+ * multiple of 128, J*D a multiple of 64) two tcgen05 GEMM passes, the first
+ * producing the gate partials from k, the second v with the gate, the conv
+ * and the residual applied in its epilogue (v is never stored); otherwise
+ * engram_project followed by engram_conv.  Scratch in `workspace`
+ * (engram_workspace_bytes(ctx, B, L); the index and e parts are unused). */
 ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, const void* h, const void* Wk,
                                const void* Wv, const float* gq, const float* gk, const float* conv_w,
                                int32_t B, int32_t L, float* conv_state, void* y, float* alpha_out,
@@ -184,8 +201,8 @@ ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, co
                                cudaStream_t stream);
 
 /* The whole forward: engram_hash (with remap) -> engram_gather ->
- * engram_project -> engram_conv, intermediates in `workspace`
- * (engram_workspace_bytes(ctx, B*(T-t_begin)) bytes, 256-byte aligned).
+ * engram_gate_conv, intermediates in `workspace`
+ * (engram_workspace_bytes(ctx, B, T-t_begin) bytes, 256-byte aligned).
  * tok is [B] rows of `tok_stride` raw ids; prefill uses t_begin = 0, a
  * decode step for the last position uses t_begin = T-1 with conv_state. */
 ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int32_t B, int32_t T,

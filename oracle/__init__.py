@@ -204,10 +204,11 @@ class Result:
 
 
 def _value_path(e, h, Wk, Wv, gq, gk, eps, bf16: bool):
+    # k and v are kept at full precision: the pages fix no storage point for
+    # them, and this build's rounding points are the stored tensors only
+    # (tables/e, h, W, Y)
     k = project(e, Wk)
     v = project(e, Wv)
-    if bf16:
-        v = round_bf16(v)  # v is stored as bf16 between the projection and the gate
     alpha = gate(h, k, gq, gk, eps)
     return k, v, alpha
 

@@ -87,4 +87,4 @@ def test_null_context_is_rejected(eb):
     from hashed_gram_embedding_02_b200 import binding
     assert binding._lib.engram_forward(None, None, 1, 1, 1, 0, None, None, None, None, None, None, None, None,
                                        None, None, None, 0, None, 0, None) == binding.ENGRAM_E_INVAL
-    assert eb.engram_workspace_bytes(None, 10) == 0
+    assert eb.engram_workspace_bytes(None, 2, 10) == 0
