@@ -88,17 +88,21 @@ bool tc_path(const engram_ctx* c, int64_t n) {
     return c->cfg.dtype == ENGRAM_BF16 && c->sm100 && project_tc_supported(n, c->d_mem, c->cfg.hidden);
 }
 
+// projections with the gate and the conv fused into the epilogue (conv width 4)
+bool fused_path(const engram_ctx* c, int64_t n) { return tc_path(c, n) && c->cfg.conv_width == 4; }
+
 struct Workspace {
     uint32_t* idx;
     void* e;
     float* part;
+    float* alpha;
     float* state_next;
     float* v;
     size_t bytes;
 };
 
-// idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | state_next [B][w-1][d] f32 |
-// v [n][d] f32 (CUDA-core path only), each 256-byte aligned
+// idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | alpha [n] f32 | state_next [B][w-1][d] f32 |
+// v [n][d] f32 (unfused paths only), each 256-byte aligned
 Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e) {
     const int64_t n = B * L;
     Workspace w{};
@@ -111,9 +115,11 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
     }
     w.part = reinterpret_cast<float*>(p);
     p += align256((size_t)n * c->G * 4 * sizeof(float));
+    w.alpha = reinterpret_cast<float*>(p);
+    p += align256((size_t)n * sizeof(float));
     w.state_next = reinterpret_cast<float*>(p);
     p += align256((size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
-    if (!tc_path(c, n)) {
+    if (!fused_path(c, n)) {
         w.v = reinterpret_cast<float*>(p);
         p += align256((size_t)n * c->cfg.hidden * sizeof(float));
     }
@@ -162,22 +168,27 @@ engram_status conv_impl(engram_ctx* c, const float* v, const float* part, const 
     return launched("gate/conv launch", e);
 }
 
-// projections + gate + conv; on the tensor-core path two GEMM passes with the
-// gate and the conv fused into the second one's epilogue
+// projections + gate + conv; on the fused path two tcgen05 GEMM passes with
+// the gate and the conv in the second one's epilogue, otherwise the
+// projection (tcgen05 or CUDA cores) followed by the CUDA-core gate/conv
 engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, const void* Wk, const void* Wv,
                              const float* gq, const float* gk, const float* conv_w, int32_t B, int32_t L,
                              float* state, void* y, float* alpha_out, int32_t add_residual, const Workspace& w,
                              cudaStream_t s) {
     const int64_t n = (int64_t)B * L;
-    if (tc_path(c, n)) {
+    if (fused_path(c, n)) {
         prof_begin(c, s, "gate_k_tc");
         cudaError_t e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, w.part, c->d_status,
                                          c->num_sms, s);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
+        prof_begin(c, s, "alpha");
+        e = launch_alpha(w.part, n, c->cfg.hidden, c->cfg.eps, w.alpha, alpha_out, c->num_sms, s);
+        prof_end(c, s);
+        if (e != cudaSuccess) return cuda_fail("alpha launch", e);
         prof_begin(c, s, "vconv_tc");
-        e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, c->cfg.eps,
-                            w.part, state, w.state_next, y, alpha_out, add_residual, c->d_status, c->num_sms, s);
+        e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha, state,
+                            w.state_next, y, add_residual, c->d_status, c->num_sms, s);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 value/conv launch", e);
         if (state) {

@@ -58,13 +58,17 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float* part, uint32_t* status, int num_sms,
                              cudaStream_t s);
-// Pass 2: v -> gate, causal conv, residual, Y (fused epilogue).  When state is
+// Pass 2: v -> gate (alpha from launch_alpha), causal conv, residual, Y (fused
+// epilogue, conv width 4).  When state is
 // non-null the new history goes to state_next ([B][w-1][d] fp32 scratch) and
 // launch_state_merge folds it into state afterwards.
+// alpha [n_tok] (and the caller's alpha_out, nullable) from the gate partials
+cudaError_t launch_alpha(const float* part, int64_t n_tok, int32_t d, float eps, float* alpha, float* alpha_out,
+                         int num_sms, cudaStream_t s);
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
-                            const float* conv_w, int32_t d, int32_t w, float eps, const float* part,
-                            const float* state, float* state_next, void* y, float* alpha_out, int32_t add_residual,
-                            uint32_t* status, int num_sms, cudaStream_t s);
+                            const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
+                            float* state_next, void* y, int32_t add_residual, uint32_t* status, int num_sms,
+                            cudaStream_t s);
 cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,
                                int num_sms, cudaStream_t s);
 // gate + conv from an fp32 v (CUDA cores)

@@ -12,23 +12,25 @@
 //              writes v (fp32) and the group's gate partials; the standalone
 //              engram_project.
 //   MODE_K     tile = 128 rows x BN k-channels: writes the gate partials
-//              (sum g_q g_k h k, sum k^2, sum h^2) of its BN/128 channel
-//              groups; k never leaves the SM.
-//   MODE_VCONV tile = 128 rows x BN v-channels, row tiles overlapping by the
-//              conv history (w-1 rows): each thread owns one TMEM lane (one
-//              row), reduces its row's partials into alpha, forms v~ = alpha v,
-//              takes v~ of the w-1 previous rows from the neighbouring lanes
-//              (warp shuffles, plus a shared-memory hand-over between the four
-//              epilogue warps), applies the conv taps, SiLU, the residual, and
-//              writes Y.  v itself never reaches global memory.
+//              (sum g_q g_k h k, sum k^2, sum h^2) of its channel groups;
+//              k never leaves the SM.
+//   MODE_VCONV tile = 4 row segments x BN v-channels.  Each epilogue warp owns
+//              32 TMEM lanes = 3 history rows + 29 output rows, so a row's
+//              conv history (rows t-1..t-3) sits in the same warp: v~ =
+//              alpha v is formed per lane and the history arrives by warp
+//              shuffles.  Taps, SiLU and the residual follow and Y is written;
+//              v never reaches global memory.  Consecutive segments overlap
+//              by 3 rows (116 output rows per 128-row MMA tile).
 //
-// Persistent kernel, one CTA per SM, warp-specialised:
-//   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of the A
-//              (e) tile and the W tile(s) into a shared-memory ring
+// Persistent kernel, one CTA per SM, warp-specialised (384 threads):
+//   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of A (e) and
+//              W into a shared-memory ring, and of the tile's h slice into a
+//              shared buffer the epilogue reads (issued after the tile's
+//              k-blocks, so it never holds back the MMA)
 //   warp 1     allocates TMEM (two fp32 accumulators) and issues
 //              tcgen05.mma kind::f16 (M=128, N=BN, K=16) from one thread
-//   warps 4-7  epilogue: tcgen05.ld of the accumulator; warp w reads TMEM
-//              lanes 32(w-4) .. 32(w-4)+31
+//   warps 4-11 epilogue: warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31;
+//              warps 4-7 and 8-11 take the two halves of the tile's channels
 // The double-buffered accumulator lets the epilogue of tile i overlap the
 // MMAs of tile i+1.  Tiles run channel-fastest so consecutive tiles share the
 // A block in L2; W stays L2-resident.
@@ -54,20 +56,29 @@ constexpr int BM = 128;                 // rows per tile (UMMA M)
 constexpr int BK = 64;                  // K per stage: 64 bf16 = 128 bytes = one swizzle row
 constexpr int UK = 16;                  // K per tcgen05.mma kind::f16
 constexpr int A_BYTES = BM * BK * 2;    // 16 KB
-constexpr int THREADS = 256;
-constexpr int kMaxHist = kMaxConv - 1;
+constexpr int THREADS = 640;            // warps 0-3 producer / MMA / idle, warps 4-19 epilogue
+constexpr int EPI_WARPS = 16;           // four per TMEM lane quarter
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int NPART = EPI_WARPS / 4;    // column parts per tile
+constexpr int CONV_W = 4;               // conv width of the fused epilogue
+constexpr int SEG = 32;                 // rows per epilogue warp
+constexpr int SEG_OUT = SEG - (CONV_W - 1);   // output rows per warp segment (29)
+constexpr int TILE_OUT = 4 * SEG_OUT;         // output rows per value tile (116)
 
-template <int BN>
+template <int MODE, int BN>
 struct Geo {
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (192 * 1024) / STAGE_BYTES;
+    static constexpr int STAGES = BN == 256 ? 3 : 4;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int SMEM_TILES = STAGES * STAGE_BYTES;
-    // tiles | barriers (1 KB) | conv taps [2][BN * 8] fp32 | hand-over [2][4][kMaxHist][32] fp32 | slack
-    static constexpr int CW_BYTES = 2 * BN * kMaxConv * 4;
-    static constexpr int XB_BYTES = 2 * 4 * kMaxHist * 32 * 4;
-    static constexpr int SMEM_BYTES = SMEM_TILES + 1024 + CW_BYTES + XB_BYTES + 1024;
+    static constexpr int HC = MODE == MODE_KV ? 128 : BN;      // h channels per tile
+    static constexpr int H_BYTES = BM * HC * 2;                // h tile, [HC/64][128 rows][128 B] swizzled
+    // tiles | h tile | barriers (1 KB) | per-tile gains [HC] or taps [BN][4] fp32 |
+    // partial hand-over [NPART][128] float4 | slack
+    static constexpr int GG_BYTES = BN * 16;
+    static constexpr int RED_BYTES = NPART * BM * 16;
+    static constexpr int SMEM_BYTES = SMEM_TILES + H_BYTES + 1024 + GG_BYTES + RED_BYTES + 1024;
 };
 
 struct __align__(8) Barriers {
@@ -75,34 +86,33 @@ struct __align__(8) Barriers {
     uint64_t empty[8];
     uint64_t tfull[2];
     uint64_t tempty[2];
+    uint64_t hfull;
+    uint64_t hempty;
     uint64_t drain;
     uint32_t tmem_base;
     volatile int abort_flag;
     int issued;       // k-block loads issued by the producer
     int consumed;     // k-block stages consumed by the MMA issuer
+    int h_issued;     // h tiles issued
+    int h_consumed;   // h tiles released by the epilogue
 };
 
 struct EpiParams {
-    const __nv_bfloat16* h;     // [n_tok][d]
     const float* gq;            // [d] or null
     const float* gk;            // [d] or null
     float* v;                   // MODE_KV: [n_tok][d] fp32
-    float4* part;               // [n_tok][G]: written (KV, K), read (VCONV)
-    const float* conv_w;        // [d][w]
-    const float* state;         // [B][w-1][d] history, or null (zero history)
-    float* state_next;          // [B][w-1][d] new history (merged by a second kernel), or null
+    float4* part;               // [n_tok][G]: written (KV, K)
+    const float* alpha;         // MODE_VCONV: [n_tok] gate values
+    const float* conv_w;        // [d][4]
+    const float* state;         // [B][3][d] history, or null (zero history)
+    float* state_next;          // [B][3][d] new history (merged by a second kernel), or null
     __nv_bfloat16* y;           // [n_tok][d]
-    float* alpha_out;           // [n_tok] or null
     uint32_t* status;
     int n_tok, d_mem, d, G;
     int n_groups;               // tiles along the channel dimension
     int num_tiles;
-    int m_stride;               // rows advanced per row tile (128, or 128 - (w-1) in MODE_VCONV)
-    int halo;                   // leading rows of a tile that are history only (MODE_VCONV)
     int L;                      // rows per sequence
-    int w;                      // conv width
     int add_residual;
-    float eps;
 };
 
 // Bounded wait: true when the phase with `parity` completed, false when the
@@ -182,10 +192,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// named barrier among the four epilogue warps (id 1; id 0 is __syncthreads)
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// wait for outstanding TMEM loads; the registers are passed through so no use
+// of them can be scheduled before the wait
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+// named barrier among the epilogue warps (id 1; id 0 is __syncthreads)
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory"); }
 
 // the same barrier as a vote: true on every epilogue thread when any passed true
 __device__ __forceinline__ bool epi_any(bool x) {
@@ -193,10 +222,10 @@ __device__ __forceinline__ bool epi_any(bool x) {
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}\n"
         : "=r"(r)
-        : "r"((uint32_t)x)
+        : "r"((uint32_t)x), "n"(EPI_THREADS)
         : "memory");
     return r != 0;
 }
@@ -210,34 +239,56 @@ __device__ __forceinline__ float silu_bf16out(float x) {
     return fmaf(hx, t, hx);
 }
 
+// 8 channels (16 bytes) of row i at tile-local channel cl (cl % 8 == 0) from
+// the h tile: boxes of 64 channels x 128 rows, 128-byte rows, 16-byte chunks
+// XOR-swizzled by the row index (the TMA 128-byte swizzle pattern)
+__device__ __forceinline__ uint4 h_chunk(const uint8_t* hs, int i, int cl) {
+    const int cb = cl >> 6;
+    const int ck = (cl & 63) >> 3;
+    return *reinterpret_cast<const uint4*>(hs + cb * (BM * 128) + i * 128 + ((ck ^ (i & 7)) << 4));
+}
+
+__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
+    f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x);
+    f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
+    f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z);
+    f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
+}
+
 // ---------------------------------------------------------------- epilogues
 
-// gate partials of one 128-channel group from 128 k columns at taddr
-__device__ __forceinline__ void partials_128(uint32_t taddr, const EpiParams& p, int64_t row, bool valid, int c0,
-                                             float& s_qk, float& s_kk, float& s_hh) {
+// Gate partials of row i over `ncols` k columns (multiple of 32) starting at
+// TMEM column taddr and tile-local channel cl; gains s_gg indexed
+// tile-locally.  TMEM loads run one 16-column chunk ahead of the math.
+__device__ __forceinline__ void partials_cols(uint32_t taddr, const uint8_t* hs, int i, bool valid, int cl,
+                                              int ncols, const float* s_gg, float& s_qk, float& s_kk, float& s_hh) {
+    uint32_t ka[16], kb[16];
+    const int nch = ncols / 16;
+    tmem_ld16(taddr, ka);
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-        uint32_t kr[32];
-        tmem_ld32(taddr + ch * 32, kr);
-        tmem_wait_ld();
-        if (valid) {
-            const uint4* hp = reinterpret_cast<const uint4*>(p.h + row * p.d + c0 + ch * 32);
+    for (int ch = 0; ch < nch; ch += 2) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint4 hv = __ldg(hp + u);
-                const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+        for (int sub = 0; sub < 2; ++sub) {
+            uint32_t(&cur)[16] = sub ? kb : ka;
+            uint32_t(&nxt)[16] = sub ? ka : kb;
+            const int c = ch + sub;
+            tmem_wait_ld(cur);
+            if (c + 1 < nch) tmem_ld16(taddr + (c + 1) * 16, nxt);
+            if (valid) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int u = 0; u < 2; ++u) {
+                    const int c8 = cl + c * 16 + u * 8;
+                    float hf[8];
+                    unpack8(h_chunk(hs, i, c8), hf);
+                    const float4 g0 = *reinterpret_cast<const float4*>(s_gg + c8);
+                    const float4 g1 = *reinterpret_cast<const float4*>(s_gg + c8 + 4);
+                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int i = u * 8 + q * 2 + half;
-                        const int c = c0 + ch * 32 + i;
-                        const float hf = half ? bf16_hi(hw[q]) : bf16_lo(hw[q]);
-                        const float kf = __uint_as_float(kr[i]);
-                        const float gg = (p.gq ? __ldg(p.gq + c) : 1.f) * (p.gk ? __ldg(p.gk + c) : 1.f);
-                        s_qk = fmaf(gg * hf, kf, s_qk);
+                    for (int e = 0; e < 8; ++e) {
+                        const float kf = __uint_as_float(cur[u * 8 + e]);
+                        s_qk = fmaf(gg[e] * hf[e], kf, s_qk);
                         s_kk = fmaf(kf, kf, s_kk);
-                        s_hh = fmaf(hf, hf, s_hh);
+                        s_hh = fmaf(hf[e], hf[e], s_hh);
                     }
                 }
             }
@@ -245,150 +296,181 @@ __device__ __forceinline__ void partials_128(uint32_t taddr, const EpiParams& p,
     }
 }
 
-__device__ __forceinline__ void epilogue_kv(uint32_t taddr, const EpiParams& p, int m0, int nt, int q, int lane) {
-    const int64_t row = (int64_t)m0 + q * 32 + lane;
+// g_q * g_k of channels [c0, c0 + n) into s_gg (all epilogue threads)
+__device__ __forceinline__ void load_gains(const EpiParams& p, int c0, int n, float* s_gg, int et) {
+    for (int k = et; k < n; k += EPI_THREADS) {
+        const int c = c0 + k;
+        s_gg[k] = (p.gq ? __ldg(p.gq + c) : 1.f) * (p.gk ? __ldg(p.gk + c) : 1.f);
+    }
+}
+
+// Partials over the channel slice [cl0, cl0 + ncols) of this warp's part,
+// added across the parts of each 128-channel group in a fixed order through
+// s_red, written by the group's first part.
+__device__ __forceinline__ void group_partials(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int64_t row,
+                                               int i, bool valid, int part, int cl0, int ncols, int parts_per_group,
+                                               int g, const float* s_gg, float4* s_red) {
+    float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+    partials_cols(taddr, hs, i, valid, cl0, ncols, s_gg, s_qk, s_kk, s_hh);
+    s_red[part * BM + i] = make_float4(s_qk, s_kk, s_hh, 0.f);
+    epi_sync();
+    if (part % parts_per_group == 0 && valid) {
+        float4 o = s_red[part * BM + i];
+        for (int k = 1; k < parts_per_group; ++k) {
+            const float4 x = s_red[(part + k) * BM + i];
+            o.x += x.x;
+            o.y += x.y;
+            o.z += x.z;
+        }
+        p.part[row * p.G + g] = o;
+    }
+}
+
+// [k | v] tile: parts 0-1 reduce the k half (128 channels, one group) into
+// the group's partials, parts 2-3 store the v half (fp32).
+__device__ __forceinline__ void epilogue_kv(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int m0, int nt,
+                                            int q, int part, int lane, int et, float* s_gg, float4* s_red) {
+    const int i = q * 32 + lane;
+    const int64_t row = (int64_t)m0 + i;
     const bool valid = row < p.n_tok;
     const int c0 = nt * 128;
-    float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-    partials_128(taddr, p, row, valid, c0, s_qk, s_kk, s_hh);
+    epi_sync();                       // previous tile's readers are done with s_gg and s_red
+    load_gains(p, c0, 128, s_gg, et);
+    epi_sync();
+    if (part < 2) {
+        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+        partials_cols(taddr + part * 64, hs, i, valid, part * 64, 64, s_gg, s_qk, s_kk, s_hh);
+        s_red[part * BM + i] = make_float4(s_qk, s_kk, s_hh, 0.f);
+    } else {
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-        uint32_t vr[32];
-        tmem_ld32(taddr + 128 + ch * 32, vr);
-        tmem_wait_ld();
-        if (valid) {
-            float4* vp = reinterpret_cast<float4*>(p.v + row * p.d + c0 + ch * 32);
+        for (int ch = 0; ch < 2; ++ch) {
+            const int cl = (part - 2) * 64 + ch * 32;
+            uint32_t vr[32];
+            tmem_ld32(taddr + 128 + cl, vr);
+            tmem_wait_ld();
+            if (valid) {
+                float4* vp = reinterpret_cast<float4*>(p.v + row * p.d + c0 + cl);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                vp[u] = make_float4(__uint_as_float(vr[4 * u]), __uint_as_float(vr[4 * u + 1]),
-                                    __uint_as_float(vr[4 * u + 2]), __uint_as_float(vr[4 * u + 3]));
+                for (int u = 0; u < 8; ++u)
+                    vp[u] = make_float4(__uint_as_float(vr[4 * u]), __uint_as_float(vr[4 * u + 1]),
+                                        __uint_as_float(vr[4 * u + 2]), __uint_as_float(vr[4 * u + 3]));
+            }
         }
     }
-    if (valid) p.part[row * p.G + nt] = make_float4(s_qk, s_kk, s_hh, 0.f);
-}
-
-template <int BN>
-__device__ __forceinline__ void epilogue_k(uint32_t taddr, const EpiParams& p, int m0, int nt, int q, int lane) {
-    const int64_t row = (int64_t)m0 + q * 32 + lane;
-    const bool valid = row < p.n_tok;
-#pragma unroll 1
-    for (int gi = 0; gi < BN / 128; ++gi) {
-        const int g = nt * (BN / 128) + gi;
-        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-        partials_128(taddr + gi * 128, p, row, valid, g * 128, s_qk, s_kk, s_hh);
-        if (valid) p.part[row * p.G + g] = make_float4(s_qk, s_kk, s_hh, 0.f);
+    epi_sync();
+    if (part == 0 && valid) {
+        const float4 a = s_red[i], b = s_red[BM + i];
+        p.part[row * p.G + nt] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, 0.f);
     }
 }
 
-// Gate + causal depthwise conv + residual on a v tile.  TMEM lane i holds flat
-// row m0 + i; lanes below `halo` are history rows of the previous tile.
+// k tile of BN channels: each of the NPART parts reduces BN/NPART columns,
+// the parts of one 128-channel group are then added in order.
 template <int BN>
-__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const EpiParams& p, int m0, int nt, int q, int lane,
-                                               int tcount, uint32_t& xcount, float* s_cw, float* s_xb) {
+__device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int m0, int nt,
+                                           int q, int part, int lane, int et, float* s_gg, float4* s_red) {
+    constexpr int PW = BN / NPART;                    // columns per part
+    constexpr int PPG = 128 / PW;                     // parts per 128-channel group
     const int i = q * 32 + lane;
-    const int64_t r = (int64_t)m0 + i;
+    const int64_t row = (int64_t)m0 + i;
+    const bool valid = row < p.n_tok;
+    const int n0 = nt * BN;
+    epi_sync();
+    load_gains(p, n0, BN, s_gg, et);
+    epi_sync();
+    group_partials(taddr + part * PW, hs, p, row, i, valid, part, part * PW, PW, PPG, (n0 + part * PW) / 128, s_gg,
+                   s_red);
+}
+
+// Gate + causal depthwise conv (width 4) + residual on a value tile of BN
+// channels.  Lane l of warp segment q holds row r0q + l; lanes 0..2 are the
+// history rows of the segment's first output row.  Each of the NPART parts
+// handles BN/NPART channels, 16 at a time, TMEM loads one chunk ahead.
+template <int BN, bool SLOW>
+__device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int i, int64_t r,
+                                             int64_t b, int t, float a, bool out_row, int n0, int cbeg,
+                                             const float4* s_cw) {
+    constexpr int H = CONV_W - 1;
+    constexpr int NCH = BN / NPART / 16;
+    const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
+    uint32_t va[16], vb[16];
+    tmem_ld16(taddr + cbeg, va);
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+        uint32_t(&cur)[16] = (ch & 1) ? vb : va;
+        uint32_t(&nxt)[16] = (ch & 1) ? va : vb;
+        const int cl = cbeg + ch * 16;
+        const int cg = n0 + cl;
+        float hv[16];
+        if (p.add_residual) {
+            unpack8(h_chunk(hs, i, cl), hv);
+            unpack8(h_chunk(hs, i, cl + 8), hv + 8);
+        }
+        tmem_wait_ld(cur);
+        if (ch + 1 < NCH) tmem_ld16(taddr + cl + 16, nxt);
+        float o[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const float vt = a * __uint_as_float(cur[c]);
+            float p1 = __shfl_up_sync(0xffffffffu, vt, 1);
+            float p2 = __shfl_up_sync(0xffffffffu, vt, 2);
+            float p3 = __shfl_up_sync(0xffffffffu, vt, 3);
+            if (SLOW && t < H) {
+                // rows before the sequence start come from the history (or are zero)
+                const float* st = p.state ? p.state + (b * H) * p.d + cg + c : nullptr;
+                if (t < 1) p1 = st ? st[(H - 1 + t) * p.d] : 0.f;
+                if (t < 2) p2 = st ? st[(H - 2 + t) * p.d] : 0.f;
+                p3 = st ? st[(H - 3 + t) * p.d] : 0.f;
+            }
+            const float4 w4 = s_cw[cl + c];
+            float u = w4.x * vt;
+            u = fmaf(w4.y, p1, u);
+            u = fmaf(w4.z, p2, u);
+            u = fmaf(w4.w, p3, u);
+            float res = vt + silu_bf16out(u);
+            if (p.add_residual) res += hv[c];
+            o[c] = res;
+            if (write_state) p.state_next[(b * H + (t - (p.L - H))) * p.d + cg + c] = vt;
+        }
+        if (out_row) {
+            uint4* yp = reinterpret_cast<uint4*>(p.y + r * p.d + cg);
+            yp[0] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                               pack_bf16x2(o[6], o[7]));
+            yp[1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
+                               pack_bf16x2(o[14], o[15]));
+        }
+    }
+}
+
+template <int BN>
+__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int mt,
+                                               int nt, int q, int part, int lane, int et, float* s_taps) {
+    constexpr int H = CONV_W - 1;
+    const int i = q * 32 + lane;
+    const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - H;
     const bool in_range = r >= 0 && r < p.n_tok;
-    const bool out_row = in_range && i >= p.halo;
-    const int W = p.w, H = W - 1;
+    const bool out_row = in_range && lane >= H;
     int64_t b = 0;
     int t = 0;
     if (in_range) {
         b = r / p.L;
         t = (int)(r - b * p.L);
     }
-    // alpha of this row: fixed-order sum of its G partials
-    float a = 0.f;
-    if (in_range) {
-        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-        const float4* pp = p.part + r * p.G;
-        for (int g = 0; g < p.G; ++g) {
-            const float4 v4 = pp[g];
-            s_qk += v4.x;
-            s_kk += v4.y;
-            s_hh += v4.z;
-        }
-        const float inv_d = 1.f / (float)p.d;
-        const float rh = sqrtf(s_hh * inv_d + p.eps);
-        const float rk = sqrtf(s_kk * inv_d + p.eps);
-        a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)p.d)));
-    }
-    if (out_row && nt == 0 && p.alpha_out) p.alpha_out[r] = a;
-
-    // conv taps of this tile's channels into shared memory (double-buffered by tile)
+    const float a = in_range ? __ldg(p.alpha + r) : 0.f;
     const int n0 = nt * BN;
-    float* cw = s_cw + (tcount & 1) * (BN * kMaxConv);
-    for (int k = i; k < BN * W; k += 128) cw[k] = __ldg(p.conv_w + (int64_t)n0 * W + k);
+    // conv taps of the tile's channels: [BN] float4
     epi_sync();
-
-    const bool has_state = p.state != nullptr;
-#pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t vr[32];
-        tmem_ld32(taddr + ch * 32, vr);
-        tmem_wait_ld();
-        float vt[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) vt[c] = a * __uint_as_float(vr[c]);
-        // hand the last H lanes' values to the next warp
-        float* xb = s_xb + (xcount & 1) * (4 * kMaxHist * 32);
-        if (lane >= 32 - H) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) xb[(q * kMaxHist + (lane - (32 - H))) * 32 + c] = vt[c];
-        }
-        epi_sync();
-        ++xcount;
-        const int cbase = n0 + ch * 32;
-        float yv[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) yv[c] = 0.f;
-#pragma unroll 1
-        for (int j = 1; j < W; ++j) {
-            const bool from_prev = lane < j;
-            const bool before_seq = t < j;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float pv = __shfl_up_sync(0xffffffffu, vt[c], j);
-                if (from_prev) pv = q > 0 ? xb[((q - 1) * kMaxHist + (H - j + lane)) * 32 + c] : 0.f;
-                if (before_seq) pv = has_state ? p.state[(b * H + (H + t - j)) * p.d + cbase + c] : 0.f;
-                yv[c] = fmaf(cw[(ch * 32 + c) * W + j], pv, yv[c]);
-            }
-        }
-        if (out_row) {
-            float hv[32];
-            if (p.add_residual) {
-                const uint4* hp = reinterpret_cast<const uint4*>(p.h + r * p.d + cbase);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint4 q4 = __ldg(hp + u);
-                    hv[8 * u + 0] = bf16_lo(q4.x); hv[8 * u + 1] = bf16_hi(q4.x);
-                    hv[8 * u + 2] = bf16_lo(q4.y); hv[8 * u + 3] = bf16_hi(q4.y);
-                    hv[8 * u + 4] = bf16_lo(q4.z); hv[8 * u + 5] = bf16_hi(q4.z);
-                    hv[8 * u + 6] = bf16_lo(q4.w); hv[8 * u + 7] = bf16_hi(q4.w);
-                }
-            }
-            uint4* yp = reinterpret_cast<uint4*>(p.y + r * p.d + cbase);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float o[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int c = 8 * u + e;
-                    const float uu = fmaf(cw[(ch * 32 + c) * W], vt[c], yv[c]);
-                    float res = vt[c] + silu_bf16out(uu);
-                    if (p.add_residual) res += hv[c];
-                    o[e] = res;
-                }
-                yp[u] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                                   pack_bf16x2(o[6], o[7]));
-            }
-            // the last H rows of a sequence become its next conv history
-            if (p.state_next && t >= p.L - H) {
-                float* sp = p.state_next + (b * H + (t - (p.L - H))) * p.d + cbase;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) sp[c] = vt[c];
-            }
-        }
-    }
+    for (int k = et; k < BN; k += EPI_THREADS)
+        reinterpret_cast<float4*>(s_taps)[k] = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + k);
+    epi_sync();
+    // warps whose rows all have their history inside the sequence and write no
+    // new history take the branch-free path
+    const bool slow_row = out_row && (t < H || (p.state_next && t >= p.L - H));
+    const int cbeg = part * (BN / NPART);
+    if (__any_sync(0xffffffffu, slow_row))
+        vconv_chunks<BN, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, reinterpret_cast<const float4*>(s_taps));
+    else
+        vconv_chunks<BN, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, reinterpret_cast<const float4*>(s_taps));
 }
 
 // ---------------------------------------------------------------- kernel
@@ -396,17 +478,19 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const EpiParams& 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
-                  const __grid_constant__ CUtensorMap map_b1, const EpiParams p) {
-    using GE = Geo<BN>;
+                  const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_h,
+                  const EpiParams p) {
+    using GE = Geo<MODE, BN>;
     constexpr int STAGES = GE::STAGES;
     constexpr int STAGE_BYTES = GE::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);   // 1024-byte aligned tile base
     const uint32_t tiles_u32 = smem_u32(smem);
-    Barriers* sb = reinterpret_cast<Barriers*>(smem + GE::SMEM_TILES);
-    float* s_cw = reinterpret_cast<float*>(smem + GE::SMEM_TILES + 1024);
-    float* s_xb = reinterpret_cast<float*>(smem + GE::SMEM_TILES + 1024 + GE::CW_BYTES);
+    uint8_t* s_h = smem + GE::SMEM_TILES;
+    Barriers* sb = reinterpret_cast<Barriers*>(smem + GE::SMEM_TILES + GE::H_BYTES);
+    float* s_gg = reinterpret_cast<float*>(smem + GE::SMEM_TILES + GE::H_BYTES + 1024);
+    float4* s_red = reinterpret_cast<float4*>(smem + GE::SMEM_TILES + GE::H_BYTES + 1024 + GE::GG_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -419,16 +503,21 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sb->tfull[a], 1);
-            mbar_init(&sb->tempty[a], 4);
+            mbar_init(&sb->tempty[a], EPI_WARPS);
         }
+        mbar_init(&sb->hfull, 1);
+        mbar_init(&sb->hempty, EPI_WARPS);
         mbar_init(&sb->drain, 1);
         sb->abort_flag = 0;
         sb->issued = 0;
         sb->consumed = 0;
+        sb->h_issued = 0;
+        sb->h_consumed = 0;
         mbar_fence_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b0);
+        tma_prefetch_desc(&map_h);
         if (MODE == MODE_KV) tma_prefetch_desc(&map_b1);
     }
     if (warp == 1) {
@@ -445,18 +534,30 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     if (warp == 0) {
         // ---------------- TMA producer
         if (lane == 0) {
-            int it = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !sb->abort_flag; tile += gridDim.x) {
+            int it = 0, tc = 0;
+            const uint32_t h_dst = smem_u32(s_h);
+            for (int tile = blockIdx.x; tile < p.num_tiles && !sb->abort_flag; tile += gridDim.x, ++tc) {
                 const int mt = tile / p.n_groups, nt = tile % p.n_groups;
-                const int m0 = mt * p.m_stride - p.halo;
+                bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!wait_bounded(&sb->empty[s], ph ^ 1u, sb, p.status)) break;
+                    if (!wait_bounded(&sb->empty[s], ph ^ 1u, sb, p.status)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t a_dst = tiles_u32 + s * STAGE_BYTES;
                     const uint32_t b_dst = a_dst + A_BYTES;
                     mbar_arrive_expect_tx(&sb->full[s], STAGE_BYTES);
-                    tma_load_2d(&map_a, a_dst, &sb->full[s], kb * BK, m0);
+                    if (MODE == MODE_VCONV) {
+                        // four 32-row segments, each starting 3 rows before its outputs
+#pragma unroll
+                        for (int sg = 0; sg < 4; ++sg)
+                            tma_load_2d(&map_a, a_dst + sg * (SEG * 128), &sb->full[s], kb * BK,
+                                        mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                    } else {
+                        tma_load_2d(&map_a, a_dst, &sb->full[s], kb * BK, mt * BM);
+                    }
                     if (MODE == MODE_KV) {
                         tma_load_2d(&map_b0, b_dst, &sb->full[s], kb * BK, nt * 128);
                         tma_load_2d(&map_b1, b_dst + 128 * BK * 2, &sb->full[s], kb * BK, nt * 128);
@@ -465,6 +566,23 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     }
                     sb->issued = it + 1;
                 }
+                if (!ok) break;
+                // the tile's h slice, once the epilogue has released the previous one
+                if (!wait_bounded(&sb->hempty, ((uint32_t)tc & 1u) ^ 1u, sb, p.status)) break;
+                mbar_arrive_expect_tx(&sb->hfull, GE::H_BYTES);
+                const int hc0 = MODE == MODE_KV ? nt * 128 : nt * BN;
+#pragma unroll 1
+                for (int cb = 0; cb < GE::HC / 64; ++cb) {
+                    if (MODE == MODE_VCONV) {
+#pragma unroll
+                        for (int sg = 0; sg < 4; ++sg)
+                            tma_load_2d(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull, hc0 + cb * 64,
+                                        mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                    } else {
+                        tma_load_2d(&map_h, h_dst + cb * (BM * 128), &sb->hfull, hc0 + cb * 64, mt * BM);
+                    }
+                }
+                sb->h_issued = tc + 1;
             }
         }
     } else if (warp == 1) {
@@ -502,37 +620,48 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             }
         }
     } else if (warp >= 4) {
-        // ---------------- epilogue
-        const int q = warp - 4;
+        // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) ..; the
+        // four warps of each lane quarter take the four column parts
+        const int q = warp & 3;
+        const int part = (warp - 4) >> 2;
+        const int et = threadIdx.x - 128;    // 0 .. EPI_THREADS-1
         int tc = 0;
-        uint32_t xcount = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tc) {
             const int acc = tc & 1;
             const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
-            const bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
-            if (epi_any(!ok)) break;          // one decision for all four warps
+            bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
+            ok = ok && wait_bounded(&sb->hfull, (uint32_t)tc & 1u, sb, p.status);
+            if (epi_any(!ok)) break;          // one decision for all epilogue warps
             tc_fence_after();
             const int mt = tile / p.n_groups, nt = tile % p.n_groups;
-            const int m0 = mt * p.m_stride - p.halo;
             const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-            if (MODE == MODE_KV) epilogue_kv(taddr, p, m0, nt, q, lane);
-            if (MODE == MODE_K) epilogue_k<BN>(taddr, p, m0, nt, q, lane);
-            if (MODE == MODE_VCONV) epilogue_vconv<BN>(taddr, p, m0, nt, q, lane, tc, xcount, s_cw, s_xb);
+            if (MODE == MODE_KV) epilogue_kv(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
+            if (MODE == MODE_K) epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
+            if (MODE == MODE_VCONV) epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sb->tempty[acc]);
+            if (lane == 0) {
+                mbar_arrive(&sb->tempty[acc]);
+                mbar_arrive(&sb->hempty);
+            }
+            if (threadIdx.x == 128) sb->h_consumed = tc + 1;
         }
     }
 
     __syncthreads();
     if (sb->abort_flag) {
-        // drain: copies this CTA issued but the MMA never consumed, then the MMAs
+        // drain: copies this CTA issued but nobody consumed, then the MMAs
         if (warp == 0 && lane == 0) {
             for (int it = sb->consumed; it < sb->issued; ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                 const long long t0 = clock64();
                 while (!mbar_try_wait(smem_u32(&sb->full[s]), ph) && clock64() - t0 < kWaitCycles) {
+                }
+            }
+            for (int k = sb->h_consumed; k < sb->h_issued; ++k) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(smem_u32(&sb->hfull), (uint32_t)k & 1u) && clock64() - t0 < kWaitCycles) {
                 }
             }
         }
@@ -548,6 +677,38 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GE::TMEM_COLS)
                      : "memory");
+    }
+}
+
+// alpha_t = sigmoid(<q^, k^> / sqrt(d)) from the G gate partials of row t:
+// one warp per row, lanes over the groups, fixed reduction order.
+__global__ void __launch_bounds__(256) alpha_kernel(const float4* __restrict__ part, int64_t n, int G, int d,
+                                                     float eps, float* __restrict__ alpha,
+                                                     float* __restrict__ alpha_out) {
+    const int lane = threadIdx.x & 31;
+    const float inv_d = 1.f / (float)d;
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n;
+         r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+        for (int g = lane; g < G; g += 32) {
+            const float4 v4 = part[r * G + g];
+            s_qk += v4.x;
+            s_kk += v4.y;
+            s_hh += v4.z;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            s_qk += __shfl_xor_sync(0xffffffffu, s_qk, off);
+            s_kk += __shfl_xor_sync(0xffffffffu, s_kk, off);
+            s_hh += __shfl_xor_sync(0xffffffffu, s_hh, off);
+        }
+        if (lane == 0) {
+            const float rh = sqrtf(s_hh * inv_d + eps);
+            const float rk = sqrtf(s_kk * inv_d + eps);
+            const float a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)d)));
+            alpha[r] = a;
+            if (alpha_out) alpha_out[r] = a;
+        }
     }
 }
 
@@ -601,9 +762,9 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 template <int MODE, int BN>
-cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, EpiParams p,
-                        int64_t m_tiles, int num_sms, cudaStream_t s) {
-    using GE = Geo<BN>;
+cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const CUtensorMap& mh,
+                        EpiParams p, int64_t m_tiles, int num_sms, cudaStream_t s) {
+    using GE = Geo<MODE, BN>;
     static unsigned long long attr_set = 0;   // one bit per device ordinal
     int dev = 0;
     cudaGetDevice(&dev);
@@ -617,7 +778,7 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
     if (tiles >= (int64_t)1 << 31) return cudaErrorInvalidValue;
     p.num_tiles = (int)tiles;
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    project_tc_kernel<MODE, BN><<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, p);
+    project_tc_kernel<MODE, BN><<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, mh, p);
     return cudaGetLastError();
 }
 
@@ -634,12 +795,11 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
                               const void* Wv, const float* gq, const float* gk, int32_t d, float* v, float* part,
                               uint32_t* status, int num_sms, cudaStream_t s) {
     if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
-    CUtensorMap ma, mk, mv;
+    CUtensorMap ma, mk, mv, mh;
     if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, 128) ||
-        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, 128))
+        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, 128) || !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, BM))
         return cudaErrorInvalidValue;
     EpiParams p{};
-    p.h = static_cast<const __nv_bfloat16*>(h);
     p.gq = gq;
     p.gk = gk;
     p.v = v;
@@ -650,9 +810,7 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
     p.d = d;
     p.G = d / 128;
     p.n_groups = d / 128;
-    p.m_stride = BM;
-    p.halo = 0;
-    return launch_mode<MODE_KV, 256>(ma, mk, mv, p, (n_tok + BM - 1) / BM, num_sms, s);
+    return launch_mode<MODE_KV, 256>(ma, mk, mv, mh, p, (n_tok + BM - 1) / BM, num_sms, s);
 }
 
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
@@ -660,11 +818,11 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
                              cudaStream_t s) {
     if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
     const int bn = pick_bn(d);
-    CUtensorMap ma, mk;
-    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn))
+    CUtensorMap ma, mk, mh;
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn) ||
+        !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, BM))
         return cudaErrorInvalidValue;
     EpiParams p{};
-    p.h = static_cast<const __nv_bfloat16*>(h);
     p.gq = gq;
     p.gk = gk;
     p.part = reinterpret_cast<float4*>(part);
@@ -674,32 +832,38 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     p.d = d;
     p.G = d / 128;
     p.n_groups = d / bn;
-    p.m_stride = BM;
-    p.halo = 0;
     const int64_t mt = (n_tok + BM - 1) / BM;
-    return bn == 256 ? launch_mode<MODE_K, 256>(ma, mk, mk, p, mt, num_sms, s)
-                     : launch_mode<MODE_K, 128>(ma, mk, mk, p, mt, num_sms, s);
+    return bn == 256 ? launch_mode<MODE_K, 256>(ma, mk, mk, mh, p, mt, num_sms, s)
+                     : launch_mode<MODE_K, 128>(ma, mk, mk, mh, p, mt, num_sms, s);
+}
+
+cudaError_t launch_alpha(const float* part, int64_t n_tok, int32_t d, float eps, float* alpha, float* alpha_out,
+                         int num_sms, cudaStream_t s) {
+    if (n_tok == 0) return cudaSuccess;
+    int64_t blocks = (n_tok + 7) / 8;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    alpha_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(part), n_tok, (d + 127) / 128, d,
+                                                  eps, alpha, alpha_out);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
-                            const float* conv_w, int32_t d, int32_t w, float eps, const float* part,
-                            const float* state, float* state_next, void* y, float* alpha_out, int32_t add_residual,
-                            uint32_t* status, int num_sms, cudaStream_t s) {
+                            const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
+                            float* state_next, void* y, int32_t add_residual, uint32_t* status, int num_sms,
+                            cudaStream_t s) {
     const int64_t n_tok = (int64_t)B * L;
-    if (!project_tc_supported(n_tok, d_mem, d) || w < 1 || w > kMaxConv) return cudaErrorNotSupported;
+    if (!project_tc_supported(n_tok, d_mem, d) || w != CONV_W) return cudaErrorNotSupported;
     const int bn = pick_bn(d);
-    const int H = w - 1;
-    CUtensorMap ma, mv;
-    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn))
+    CUtensorMap ma, mv, mh;
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, SEG) || !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn) ||
+        !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, SEG))
         return cudaErrorInvalidValue;
     EpiParams p{};
-    p.h = static_cast<const __nv_bfloat16*>(h);
-    p.part = const_cast<float4*>(reinterpret_cast<const float4*>(part));
+    p.alpha = alpha;
     p.conv_w = conv_w;
     p.state = state;
     p.state_next = state ? state_next : nullptr;
     p.y = static_cast<__nv_bfloat16*>(y);
-    p.alpha_out = alpha_out;
     p.status = status;
     p.n_tok = (int)n_tok;
     p.d_mem = d_mem;
@@ -707,15 +871,10 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     p.G = d / 128;
     p.n_groups = d / bn;
     p.L = L;
-    p.w = w;
     p.add_residual = add_residual;
-    p.eps = eps;
-    // row tiles overlap by the H history rows
-    p.m_stride = BM - H;
-    p.halo = H;
-    const int64_t mt = (n_tok + p.m_stride - 1) / p.m_stride;
-    return bn == 256 ? launch_mode<MODE_VCONV, 256>(ma, mv, mv, p, mt, num_sms, s)
-                     : launch_mode<MODE_VCONV, 128>(ma, mv, mv, p, mt, num_sms, s);
+    const int64_t mt = (n_tok + TILE_OUT - 1) / TILE_OUT;
+    return bn == 256 ? launch_mode<MODE_VCONV, 256>(ma, mv, mv, mh, p, mt, num_sms, s)
+                     : launch_mode<MODE_VCONV, 128>(ma, mv, mv, mh, p, mt, num_sms, s);
 }
 
 cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,

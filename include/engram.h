@@ -121,9 +121,10 @@ ENGRAM_API const char* engram_last_error(void);
 /* Bytes of scratch that engram_forward / engram_gate_conv need for B
  * sequences of L computed rows (n_tok = B*L): indices [n_tok][J] u32,
  * e [n_tok][J*D], gate partials [n_tok][G][4] f32 with G = ceil(d / 128), the
- * next conv history [B][w-1][d] f32 and, where the projection runs on CUDA
- * cores (fp32 configurations and shapes the tensor-core kernels do not tile),
- * v [n_tok][d] f32; each part 256-byte aligned.  0 for a null context. */
+ * gate values [n_tok] f32, the next conv history [B][w-1][d] f32 and, where
+ * the gate and conv are not
+ * fused into the projection (see engram_gate_conv), v [n_tok][d] f32; each
+ * part 256-byte aligned.  0 for a null context. */
 ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int32_t B, int32_t L);
 
 /* Per-kernel timing for benchmarks.  While enabled, every entry point records
@@ -189,10 +190,10 @@ ENGRAM_API engram_status engram_conv(engram_ctx* ctx, const float* v, const floa
                           float* alpha_out, int32_t add_residual, cudaStream_t stream);
 
 /* Projections, gate and conv from e: on bf16 tensor-core shapes (d a
- * multiple of 128, J*D a multiple of 64) two tcgen05 GEMM passes, the first
- * producing the gate partials from k, the second v with the gate, the conv
- * and the residual applied in its epilogue (v is never stored); otherwise
- * engram_project followed by engram_conv.  Scratch in `workspace`
+ * multiple of 128, J*D a multiple of 64) with conv width 4, two tcgen05 GEMM
+ * passes, the first producing the gate partials from k, the second v with
+ * the gate, the conv and the residual applied in its epilogue (v is never
+ * stored); otherwise engram_project followed by engram_conv.  Scratch in `workspace`
  * (engram_workspace_bytes(ctx, B, L); the index and e parts are unused). */
 ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, const void* h, const void* Wk,
                                const void* Wv, const float* gq, const float* gk, const float* conv_w,

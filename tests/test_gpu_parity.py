@@ -29,6 +29,8 @@ SMALL = {
     "f2": W["c1"].replace(name="f2", B=3, T=77, orders=(3,), K=3, D=8, d=136, w=2, seed=13),
     # bf16 tensor-core tiling with several row tiles and a ragged tail, d_mem 1024
     "b3": W["c2"].replace(name="b3", B=2, T=333, M=10007, d=512, seed=14),
+    # bf16 tensor-core projection with conv width 3 (unfused: CUDA-core gate/conv), d = 384
+    "b4": W["c1"].replace(name="b4", B=3, T=150, K=2, D=64, d=384, w=3, dtype="bf16", seed=15),
 }
 
 
