@@ -13,7 +13,8 @@ from typing import Optional
 from .binding import (  # noqa: F401  (re-exported C ABI names)
     ENGRAM_BF16, ENGRAM_F32, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
     ENGRAM_INVALID_INDEX, ENGRAM_OK, EXPORTS, LIB_PATH, EngramError, engram_config, engram_conv, engram_create,
-    engram_destroy, engram_device_status, engram_forward, engram_gate_conv, engram_gather, engram_hash,
+    ENGRAM_NOALLOC_SCRATCH_BYTES, engram_destroy, engram_device_status, engram_forward, engram_forward_noalloc,
+    engram_gate_conv, engram_gather, engram_hash,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 

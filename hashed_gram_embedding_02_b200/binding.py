@@ -34,7 +34,9 @@ ENGRAM_PART_GROUP = 128
 # exported symbol names declared in include/engram.h
 EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_error", "engram_workspace_bytes",
            "engram_profile_enable", "engram_profile_read", "engram_device_status", "engram_remap", "engram_hash",
-           "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward")
+           "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward",
+           "engram_forward_noalloc")
+ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class engram_config(ctypes.Structure):
@@ -82,6 +84,8 @@ _sigs = {
                          _st),
     "engram_forward": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                         _i32, _vp, _sz, _vp], _st),
+    "engram_forward_noalloc": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _vp, _i32, _vp], _st),
 }
 for _name, (_args, _res) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -204,3 +208,13 @@ def engram_forward(ctx, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq
                                _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w), _ptr(conv_state), _ptr(y),
                                _ptr(alpha_out), int(add_residual), _ptr(workspace), workspace_bytes,
                                _stream(stream)), "engram_forward")
+
+
+def engram_forward_noalloc(ctx, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
+                           alpha_out, add_residual, stream=None):
+    """engram_forward with its scratch in the library's static device array
+    (for callers that cannot allocate device memory)."""
+    _check(_lib.engram_forward_noalloc(ctx, _ptr(tok), B, T, tok_stride, t_begin, _ptr(P), _ptr(tables), _ptr(h),
+                                       _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w), _ptr(conv_state),
+                                       _ptr(y), _ptr(alpha_out), int(add_residual), _stream(stream)),
+           "engram_forward_noalloc")

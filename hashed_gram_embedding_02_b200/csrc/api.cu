@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "common.cuh"
@@ -494,6 +495,69 @@ engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32
     prof_end(c, s);
     if (e != cudaSuccess) return cuda_fail("gather launch", e);
     return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
+}
+
+// ---------------------------------------------------------------- forward without allocation
+//
+// For callers that cannot allocate device memory at all: an inference
+// engine's execution callback that forbids allocation, a process whose device
+// memory is already handed to another allocator, or a latency-critical loop
+// that must avoid cudaMalloc's implicit synchronisation.  They get the forward
+// with its scratch in this file-scope device array instead of a caller
+// workspace.  Every GPU that loads the library holds the array until exit.
+
+}  // extern "C"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ENGRAM_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64];   // device address of g_noalloc_scratch per device ordinal
+
+// Device address of the static scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device with that device current.
+engram_status noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= 64) return inval("device ordinal out of range for the static scratch");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress of the static scratch", e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ENGRAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+engram_status engram_forward_noalloc(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
+                                     int32_t t_begin, const int32_t* P, const void* tables, const void* h,
+                                     const void* Wk, const void* Wv, const float* gq, const float* gk,
+                                     const float* conv_w, float* conv_state, void* y, float* alpha_out,
+                                     int32_t add_residual, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (B < 0 || T < 0 || t_begin < 0 || t_begin > T) return inval("need B >= 0 and 0 <= t_begin <= T");
+    const size_t need = carve(c, nullptr, B, T - t_begin, true).bytes;
+    if (need > (size_t)ENGRAM_NOALLOC_SCRATCH_BYTES) {
+        std::snprintf(g_last_error, sizeof(g_last_error),
+                      "engram_forward_noalloc: %zu bytes of scratch needed, the static scratch holds %zu; "
+                      "use engram_forward with a workspace or split the batch",
+                      need, (size_t)ENGRAM_NOALLOC_SCRATCH_BYTES);
+        return ENGRAM_E_NOMEM;
+    }
+    void* scratch = nullptr;
+    engram_status st = noalloc_scratch(&scratch);
+    if (st != ENGRAM_OK) return st;
+    return engram_forward(c, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
+                          alpha_out, add_residual, scratch, (size_t)ENGRAM_NOALLOC_SCRATCH_BYTES, s);
 }
 
 }  // extern "C"

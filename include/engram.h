@@ -213,6 +213,30 @@ ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int
                              float* conv_state, void* y, float* alpha_out, int32_t add_residual,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* engram_forward for callers that cannot allocate device memory (an engine
+ * callback where allocation is forbidden, a process whose device memory is
+ * all owned by another allocator, a loop that cannot afford cudaMalloc's
+ * implicit synchronisation).  The pages have no counterpart: this is an
+ * interface of this library only.  Same arguments as engram_forward without
+ * the workspace: the scratch lives in a static device array of
+ * ENGRAM_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.  The first call on a device looks up that array's
+ * device address (cudaGetSymbolAddress), so make it before any stream
+ * capture.  Calls needing more than the array (engram_workspace_bytes(ctx,
+ * B, T - t_begin)) return ENGRAM_E_NOMEM with an explanation in
+ * engram_last_error and launch nothing.  No cudaMalloc or cudaFree is called.
+ * All calls share the one array, which keeps the last call's contents (the
+ * forward writes every scratch byte before reading it): calls that may
+ * overlap on the GPU (other streams, other host threads) race on it and must
+ * be serialised by the caller. */
+#define ENGRAM_NOALLOC_SCRATCH_BYTES (32u << 20)
+ENGRAM_API engram_status engram_forward_noalloc(engram_ctx* ctx, const int32_t* tok, int32_t B, int32_t T,
+                                     int64_t tok_stride, int32_t t_begin, const int32_t* P,
+                                     const void* tables, const void* h, const void* Wk, const void* Wv,
+                                     const float* gq, const float* gk, const float* conv_w,
+                                     float* conv_state, void* y, float* alpha_out, int32_t add_residual,
+                                     cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
