@@ -92,17 +92,22 @@ bool tc_path(const engram_ctx* c, int64_t n) {
 // projections with the gate and the conv fused into the epilogue (conv width 4)
 bool fused_path(const engram_ctx* c, int64_t n) { return tc_path(c, n) && c->cfg.conv_width == 4; }
 
+// per-128-row-band counters of the key pass
+size_t band_bytes(int64_t n) { return (size_t)((n + 127) / 128) * sizeof(int); }
+
 struct Workspace {
     uint32_t* idx;
     void* e;
     float* part;
     float* alpha;
+    int* band;
     float* state_next;
     float* v;
     size_t bytes;
 };
 
-// idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | alpha [n] f32 | state_next [B][w-1][d] f32 |
+// idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | alpha [n] f32 | band counters |
+// state_next [B][w-1][d] f32 |
 // v [n][d] f32 (unfused paths only), each 256-byte aligned
 Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e) {
     const int64_t n = B * L;
@@ -118,6 +123,8 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
     p += align256((size_t)n * c->G * 4 * sizeof(float));
     w.alpha = reinterpret_cast<float*>(p);
     p += align256((size_t)n * sizeof(float));
+    w.band = reinterpret_cast<int*>(p);
+    p += align256(band_bytes(n));
     w.state_next = reinterpret_cast<float*>(p);
     p += align256((size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
     if (!fused_path(c, n)) {
@@ -178,15 +185,13 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
                              cudaStream_t s) {
     const int64_t n = (int64_t)B * L;
     if (fused_path(c, n)) {
+        cudaError_t e = cudaMemsetAsync(w.band, 0, band_bytes(n), s);
+        if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
         prof_begin(c, s, "gate_k_tc");
-        cudaError_t e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, w.part, c->d_status,
-                                         c->num_sms, s);
+        e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band, w.alpha,
+                             alpha_out, c->d_status, c->num_sms, s);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
-        prof_begin(c, s, "alpha");
-        e = launch_alpha(w.part, n, c->cfg.hidden, c->cfg.eps, w.alpha, alpha_out, c->num_sms, s);
-        prof_end(c, s);
-        if (e != cudaSuccess) return cuda_fail("alpha launch", e);
         prof_begin(c, s, "vconv_tc");
         e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha, state,
                             w.state_next, y, add_residual, c->d_status, c->num_sms, s);

@@ -54,17 +54,16 @@ bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d);
 cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                               const void* Wv, const float* gq, const float* gk, int32_t d, float* v,
                               float* part, uint32_t* status, int num_sms, cudaStream_t s);
-// Pass 1: k -> gate partials [n_tok][G][4].
+// Pass 1: k -> gate partials [n_tok][G][4] and alpha [n_tok] (reduced by the
+// CTA that completes each 128-row band; band_count holds ceil(n_tok/128)
+// counters that must be zero on entry and are zero again on exit).
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
-                             const float* gq, const float* gk, int32_t d, float* part, uint32_t* status, int num_sms,
-                             cudaStream_t s);
-// Pass 2: v -> gate (alpha from launch_alpha), causal conv, residual, Y (fused
-// epilogue, conv width 4).  When state is
-// non-null the new history goes to state_next ([B][w-1][d] fp32 scratch) and
-// launch_state_merge folds it into state afterwards.
-// alpha [n_tok] (and the caller's alpha_out, nullable) from the gate partials
-cudaError_t launch_alpha(const float* part, int64_t n_tok, int32_t d, float eps, float* alpha, float* alpha_out,
-                         int num_sms, cudaStream_t s);
+                             const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
+                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, cudaStream_t s);
+// Pass 2: v -> gate (alpha from pass 1), causal conv, residual, Y (fused
+// epilogue, conv width 4).  When state is non-null the new history goes to
+// state_next ([B][w-1][d] fp32 scratch) and launch_state_merge folds it into
+// state afterwards.
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
                             float* state_next, void* y, int32_t add_residual, uint32_t* status, int num_sms,

@@ -7,18 +7,18 @@
 //   phi_{n,k}(g) = (XOR_{j<n} (s_j + 1) * a_{n,k,j} mod 2^64) mod M_{n,k},
 // s_j = x'_{t-j}, s_j = V' (PAD) before the sequence start.
 //
-// One thread per output row (b, t).  A warp covers consecutive positions of a
-// sequence, so the ids of the n-1 predecessors come from neighbouring lanes
-// by __shfl_up_sync; only lanes whose predecessor belongs to another warp (or
-// to the context before t_begin) read it from memory.  Indices are staged in
-// shared memory and written out as one contiguous block per CTA.
+// A CTA takes 256/J consecutive output rows (b, t).  It first stages each
+// row's window of canonical ids (x'_t, x'_{t-1}, ..., PAD before the start;
+// reading into [0, t_begin) for decode) in shared memory, one (row, j) pair
+// per thread, then hashes one (row, table) pair per thread, so consecutive
+// threads write consecutive indices.
 #include "common.cuh"
 
 namespace engram {
 
 namespace {
 
-constexpr int kHashThreads = 128;
+constexpr int kHashThreads = 256;
 
 __device__ __forceinline__ int32_t canon_at(const int32_t* ids, const int32_t* P, int64_t pos,
                                             int32_t V, int32_t Vc, uint32_t* status) {
@@ -39,66 +39,41 @@ __device__ __forceinline__ int32_t canon_at(const int32_t* ids, const int32_t* P
 
 __global__ void __launch_bounds__(kHashThreads)
 hash_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, int32_t B, int32_t T,
-            int64_t stride, int32_t t_begin, uint32_t* __restrict__ idx, const HashParams hp,
+            int64_t stride, int32_t t_begin, uint32_t* __restrict__ idx, const HashParams hp, int rows_per_cta,
             uint32_t* status) {
-    extern __shared__ uint32_t s_idx[];  // [kHashThreads][J]
+    __shared__ int32_t s_win[kHashThreads][4];   // [row][j]: canonical id at t - j (PAD before the start)
     const int64_t L = (int64_t)T - t_begin;
     const int64_t n = (int64_t)B * L;
-    const int64_t row0 = (int64_t)blockIdx.x * kHashThreads;
-    const int64_t row = row0 + threadIdx.x;
-    const bool active = row < n;
-    const int lane = threadIdx.x & 31;
-    int64_t b = 0, tl = 0;
-    if (active) {
-        b = row / L;
-        tl = row - b * L;
-    }
-    const int64_t t = t_begin + tl;
-    const int64_t base = b * stride;
+    const int64_t row0 = (int64_t)blockIdx.x * rows_per_cta;
+    const int R = (int)min((int64_t)rows_per_cta, n - row0);
+    const int W = hp.max_order;
 
-    const int32_t mine = active ? canon_at(ids, P, base + t, hp.V, hp.Vc, status) : -1;
-    int32_t s[4];
-    s[0] = mine;
-#pragma unroll
-    for (int j = 1; j < 4; ++j) {
-        const int32_t nb = __shfl_up_sync(0xffffffffu, mine, j);
-        if (j < hp.max_order) {
-            if (lane >= j && tl >= j) {
-                s[j] = nb;                       // row - j: same sequence, previous lane
-            } else if (t - j >= 0) {
-                s[j] = active ? canon_at(ids, P, base + t - j, hp.V, hp.Vc, status) : -1;
-            } else {
-                s[j] = hp.Vc;                    // PAD before the sequence start
-            }
-        } else {
-            s[j] = 0;
-        }
-    }
-
-    if (active) {
-        uint32_t* out = s_idx + threadIdx.x * hp.J;
-        for (int o = 0; o < hp.n_orders; ++o) {
-            const int n_o = hp.orders[o];
-            bool invalid = false;
-            for (int j = 0; j < n_o; ++j) invalid |= (s[j] < 0);
-            for (int k = 0; k < hp.K; ++k) {
-                const int jt = o * hp.K + k;
-                uint32_t r = ENGRAM_INVALID_INDEX;
-                if (!invalid) {
-                    uint64_t x = 0;
-                    for (int j = 0; j < n_o; ++j) x ^= (uint64_t)(uint32_t)(s[j] + 1) * hp.mult[jt][j];
-                    r = (uint32_t)(x % (uint64_t)hp.rows[jt]);
-                }
-                out[jt] = r;
-            }
-        }
+    // 1. the n-gram windows of this CTA's rows, one (row, j) pair per thread
+    for (int k = threadIdx.x; k < R * W; k += kHashThreads) {
+        const int rr = k / W, j = k - rr * W;
+        const int64_t row = row0 + rr;
+        const int64_t b = row / L;
+        const int64_t t = t_begin + (row - b * L);
+        s_win[rr][j] = (t - j >= 0) ? canon_at(ids, P, b * stride + t - j, hp.V, hp.Vc, status) : hp.Vc;
     }
     __syncthreads();
-    // coalesced write of this CTA's rows (contiguous in idx)
-    const int64_t rows_here = min((int64_t)kHashThreads, n - row0);
-    const int64_t words = rows_here * hp.J;
-    uint32_t* dst = idx + row0 * hp.J;
-    for (int64_t i = threadIdx.x; i < words; i += kHashThreads) dst[i] = s_idx[i];
+
+    // 2. one (row, table) pair per thread; consecutive threads write
+    //    consecutive words of idx
+    const int J = hp.J;
+    for (int k = threadIdx.x; k < R * J; k += kHashThreads) {
+        const int rr = k / J, jt = k - rr * J;
+        const int o = jt / hp.K;
+        const int n_o = hp.orders[o];
+        bool invalid = false;
+        uint64_t x = 0;
+        for (int j = 0; j < n_o; ++j) {
+            const int32_t sj = s_win[rr][j];
+            invalid |= (sj < 0);
+            x ^= (uint64_t)(uint32_t)(sj + 1) * hp.mult[jt][j];
+        }
+        idx[(row0 + rr) * J + jt] = invalid ? ENGRAM_INVALID_INDEX : (uint32_t)(x % (uint64_t)hp.rows[jt]);
+    }
 }
 
 __global__ void remap_kernel(const int32_t* __restrict__ tok, int64_t n, const int32_t* __restrict__ P,
@@ -133,9 +108,10 @@ cudaError_t launch_hash(const int32_t* ids, const int32_t* P, int32_t B, int32_t
                         cudaStream_t s) {
     const int64_t n = (int64_t)B * (T - t_begin);
     if (n == 0) return cudaSuccess;
-    const int64_t blocks = (n + kHashThreads - 1) / kHashThreads;
-    const size_t smem = (size_t)kHashThreads * hp.J * sizeof(uint32_t);
-    hash_kernel<<<(unsigned)blocks, kHashThreads, smem, s>>>(ids, P, B, T, stride, t_begin, idx, hp, status);
+    const int rows_per_cta = kHashThreads / hp.J;          // J <= 32, so at least 8
+    const int64_t blocks = (n + rows_per_cta - 1) / rows_per_cta;
+    hash_kernel<<<(unsigned)blocks, kHashThreads, 0, s>>>(ids, P, B, T, stride, t_begin, idx, hp, rows_per_cta,
+                                                          status);
     return cudaGetLastError();
 }
 

@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include <cuda_fp16.h>
 
 namespace engram {
 
@@ -95,6 +96,7 @@ struct __align__(8) Barriers {
     int consumed;     // k-block stages consumed by the MMA issuer
     int h_issued;     // h tiles issued
     int h_consumed;   // h tiles released by the epilogue
+    int band_last;    // this CTA completed a row band's partials (MODE_K)
 };
 
 struct EpiParams {
@@ -113,6 +115,10 @@ struct EpiParams {
     int num_tiles;
     int L;                      // rows per sequence
     int add_residual;
+    int* band_count;            // MODE_K: per row band, channel tiles done (zero on entry, zero on exit)
+    float* alpha_w;             // MODE_K: [n_tok] gate values written by each band's last CTA
+    float* alpha_out;           // MODE_K: caller's copy of alpha, or null
+    float eps;
 };
 
 // Bounded wait: true when the phase with `parity` completed, false when the
@@ -228,15 +234,6 @@ __device__ __forceinline__ bool epi_any(bool x) {
         : "r"((uint32_t)x), "n"(EPI_THREADS)
         : "memory");
     return r != 0;
-}
-
-__device__ __forceinline__ float silu_bf16out(float x) {
-    // x * sigmoid(x) = hx + hx * tanh(hx), hx = x/2; hardware tanh approximation
-    // (relative error about 2^-11, below the bf16 rounding of Y)
-    const float hx = 0.5f * x;
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hx));
-    return fmaf(hx, t, hx);
 }
 
 // 8 channels (16 bytes) of row i at tile-local channel cl (cl % 8 == 0) from
@@ -385,14 +382,21 @@ __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, co
 // Gate + causal depthwise conv (width 4) + residual on a value tile of BN
 // channels.  Lane l of warp segment q holds row r0q + l; lanes 0..2 are the
 // history rows of the segment's first output row.  Each of the NPART parts
-// handles BN/NPART channels, 16 at a time, TMEM loads one chunk ahead.
-template <int BN, bool SLOW>
+// handles BN/NPART channels, 16 at a time, TMEM loads one chunk ahead.  The
+// history values travel between lanes as fp16 pairs (one shuffle per two
+// channels per shift; relative error at most 2^-11 of each history term,
+// below the bf16 rounding of Y), which halves the shuffle traffic that
+// otherwise saturates the shared-memory/shuffle pipe.  The taps arrive
+// pre-halved, so the tap sum is x/2 and SiLU(x) = x/2 + x/2 * tanh(x/2)
+// needs no extra scaling.
+template <int BN, bool SLOW, bool RES>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
                                              const float4* s_cw) {
     constexpr int H = CONV_W - 1;
     constexpr int NCH = BN / NPART / 16;
     const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
+    uint4* yrow = reinterpret_cast<uint4*>(p.y + r * p.d + n0 + cbeg);
     uint32_t va[16], vb[16];
     tmem_ld16(taddr + cbeg, va);
 #pragma unroll
@@ -400,9 +404,8 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, 
         uint32_t(&cur)[16] = (ch & 1) ? vb : va;
         uint32_t(&nxt)[16] = (ch & 1) ? va : vb;
         const int cl = cbeg + ch * 16;
-        const int cg = n0 + cl;
         float hv[16];
-        if (p.add_residual) {
+        if (RES) {
             unpack8(h_chunk(hs, i, cl), hv);
             unpack8(h_chunk(hs, i, cl + 8), hv + 8);
         }
@@ -410,34 +413,43 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, 
         if (ch + 1 < NCH) tmem_ld16(taddr + cl + 16, nxt);
         float o[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const float vt = a * __uint_as_float(cur[c]);
-            float p1 = __shfl_up_sync(0xffffffffu, vt, 1);
-            float p2 = __shfl_up_sync(0xffffffffu, vt, 2);
-            float p3 = __shfl_up_sync(0xffffffffu, vt, 3);
-            if (SLOW && t < H) {
-                // rows before the sequence start come from the history (or are zero)
-                const float* st = p.state ? p.state + (b * H) * p.d + cg + c : nullptr;
-                if (t < 1) p1 = st ? st[(H - 1 + t) * p.d] : 0.f;
-                if (t < 2) p2 = st ? st[(H - 2 + t) * p.d] : 0.f;
-                p3 = st ? st[(H - 3 + t) * p.d] : 0.f;
+        for (int c = 0; c < 16; c += 2) {
+            const float v0 = a * __uint_as_float(cur[c]), v1 = a * __uint_as_float(cur[c + 1]);
+            __half2 pk = __floats2half2_rn(v0, v1);
+            const uint32_t u0 = *reinterpret_cast<uint32_t*>(&pk);
+            uint32_t s1 = __shfl_up_sync(0xffffffffu, u0, 1);
+            uint32_t s2 = __shfl_up_sync(0xffffffffu, u0, 2);
+            uint32_t s3 = __shfl_up_sync(0xffffffffu, u0, 3);
+            const float2 f1 = __half22float2(*reinterpret_cast<__half2*>(&s1));
+            const float2 f2 = __half22float2(*reinterpret_cast<__half2*>(&s2));
+            const float2 f3 = __half22float2(*reinterpret_cast<__half2*>(&s3));
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float vt = e ? v1 : v0;
+                float p1 = e ? f1.y : f1.x, p2 = e ? f2.y : f2.x, p3 = e ? f3.y : f3.x;
+                if (SLOW && t < H) {
+                    const float* st = p.state ? p.state + (b * H) * p.d + n0 + cl + c + e : nullptr;
+                    if (t < 1) p1 = st ? st[(H - 1 + t) * p.d] : 0.f;
+                    if (t < 2) p2 = st ? st[(H - 2 + t) * p.d] : 0.f;
+                    p3 = st ? st[(H - 3 + t) * p.d] : 0.f;
+                }
+                const float4 w4 = s_cw[cl + c + e];
+                float hx = w4.x * vt;
+                hx = fmaf(w4.y, p1, hx);
+                hx = fmaf(w4.z, p2, hx);
+                hx = fmaf(w4.w, p3, hx);
+                float th;
+                asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hx));
+                const float base = RES ? vt + hv[c + e] : vt;
+                o[c + e] = base + fmaf(hx, th, hx);
+                if (write_state) p.state_next[(b * H + (t - (p.L - H))) * p.d + n0 + cl + c + e] = vt;
             }
-            const float4 w4 = s_cw[cl + c];
-            float u = w4.x * vt;
-            u = fmaf(w4.y, p1, u);
-            u = fmaf(w4.z, p2, u);
-            u = fmaf(w4.w, p3, u);
-            float res = vt + silu_bf16out(u);
-            if (p.add_residual) res += hv[c];
-            o[c] = res;
-            if (write_state) p.state_next[(b * H + (t - (p.L - H))) * p.d + cg + c] = vt;
         }
         if (out_row) {
-            uint4* yp = reinterpret_cast<uint4*>(p.y + r * p.d + cg);
-            yp[0] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                               pack_bf16x2(o[6], o[7]));
-            yp[1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
-                               pack_bf16x2(o[14], o[15]));
+            yrow[2 * ch] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                      pack_bf16x2(o[6], o[7]));
+            yrow[2 * ch + 1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
+                                          pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
         }
     }
 }
@@ -458,19 +470,72 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const uint8_t* hs
     }
     const float a = in_range ? __ldg(p.alpha + r) : 0.f;
     const int n0 = nt * BN;
-    // conv taps of the tile's channels: [BN] float4
+    // conv taps of the tile's channels, halved: [BN] float4
     epi_sync();
-    for (int k = et; k < BN; k += EPI_THREADS)
-        reinterpret_cast<float4*>(s_taps)[k] = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + k);
+    for (int k = et; k < BN; k += EPI_THREADS) {
+        const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + k);
+        reinterpret_cast<float4*>(s_taps)[k] = make_float4(0.5f * w.x, 0.5f * w.y, 0.5f * w.z, 0.5f * w.w);
+    }
     epi_sync();
     // warps whose rows all have their history inside the sequence and write no
     // new history take the branch-free path
     const bool slow_row = out_row && (t < H || (p.state_next && t >= p.L - H));
     const int cbeg = part * (BN / NPART);
-    if (__any_sync(0xffffffffu, slow_row))
-        vconv_chunks<BN, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, reinterpret_cast<const float4*>(s_taps));
-    else
-        vconv_chunks<BN, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, reinterpret_cast<const float4*>(s_taps));
+    const float4* cw = reinterpret_cast<const float4*>(s_taps);
+    const bool slow = __any_sync(0xffffffffu, slow_row);
+    if (p.add_residual) {
+        if (slow) vconv_chunks<BN, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        else vconv_chunks<BN, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+    } else {
+        if (slow) vconv_chunks<BN, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        else vconv_chunks<BN, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+    }
+}
+
+// After a key tile's partials are written: the CTA that completes a row band
+// (the last of its n_groups channel tiles) reduces the band's G partials per
+// row into alpha, in the same fixed order as any other reduction of them,
+// and re-arms the counter.  One thread counts with a release/acquire atomic
+// at device scope after the CTA barrier; the band's partials (written by
+// other CTAs, read through L2) are staged in one pass into the h buffer,
+// which this tile no longer needs and the producer refills only after the
+// epilogue releases it.
+__device__ __forceinline__ int atomic_add_acq_rel(int* addr, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void band_alpha(const EpiParams& p, int mt, int et, Barriers* sb, float4* s_stage,
+                                           int stage_bytes) {
+    epi_sync();
+    if (et == 0) sb->band_last = (atomic_add_acq_rel(p.band_count + mt, 1) == p.n_groups - 1);
+    epi_sync();
+    if (!sb->band_last) return;
+    const int64_t row0 = (int64_t)mt * BM;
+    const int rows = (int)min((int64_t)BM, (int64_t)p.n_tok - row0);
+    const float4* src = p.part + row0 * p.G;
+    // wide hidden sizes whose band does not fit the buffer read L2 directly
+    const bool staged = rows * p.G * 16 <= stage_bytes;
+    if (staged)
+        for (int k = et; k < rows * p.G; k += EPI_THREADS) s_stage[k] = __ldcg(src + k);
+    epi_sync();
+    if (et < rows) {
+        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+        for (int g = 0; g < p.G; ++g) {
+            const float4 v4 = staged ? s_stage[et * p.G + g] : __ldcg(src + et * p.G + g);
+            s_qk += v4.x;
+            s_kk += v4.y;
+            s_hh += v4.z;
+        }
+        const float inv_d = 1.f / (float)p.d;
+        const float rh = sqrtf(s_hh * inv_d + p.eps);
+        const float rk = sqrtf(s_kk * inv_d + p.eps);
+        const float a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)p.d)));
+        p.alpha_w[row0 + et] = a;
+        if (p.alpha_out) p.alpha_out[row0 + et] = a;
+    }
+    if (et == 0) p.band_count[mt] = 0;
 }
 
 // ---------------------------------------------------------------- kernel
@@ -636,7 +701,10 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const int mt = tile / p.n_groups, nt = tile % p.n_groups;
             const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
             if (MODE == MODE_KV) epilogue_kv(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
-            if (MODE == MODE_K) epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
+            if (MODE == MODE_K) {
+                epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
+                band_alpha(p, mt, et, sb, reinterpret_cast<float4*>(s_h), GE::H_BYTES);
+            }
             if (MODE == MODE_VCONV) epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg);
             tc_fence_before();
             __syncwarp();
@@ -677,38 +745,6 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GE::TMEM_COLS)
                      : "memory");
-    }
-}
-
-// alpha_t = sigmoid(<q^, k^> / sqrt(d)) from the G gate partials of row t:
-// one warp per row, lanes over the groups, fixed reduction order.
-__global__ void __launch_bounds__(256) alpha_kernel(const float4* __restrict__ part, int64_t n, int G, int d,
-                                                     float eps, float* __restrict__ alpha,
-                                                     float* __restrict__ alpha_out) {
-    const int lane = threadIdx.x & 31;
-    const float inv_d = 1.f / (float)d;
-    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n;
-         r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-        for (int g = lane; g < G; g += 32) {
-            const float4 v4 = part[r * G + g];
-            s_qk += v4.x;
-            s_kk += v4.y;
-            s_hh += v4.z;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            s_qk += __shfl_xor_sync(0xffffffffu, s_qk, off);
-            s_kk += __shfl_xor_sync(0xffffffffu, s_kk, off);
-            s_hh += __shfl_xor_sync(0xffffffffu, s_hh, off);
-        }
-        if (lane == 0) {
-            const float rh = sqrtf(s_hh * inv_d + eps);
-            const float rk = sqrtf(s_kk * inv_d + eps);
-            const float a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)d)));
-            alpha[r] = a;
-            if (alpha_out) alpha_out[r] = a;
-        }
     }
 }
 
@@ -814,8 +850,8 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 }
 
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
-                             const float* gq, const float* gk, int32_t d, float* part, uint32_t* status, int num_sms,
-                             cudaStream_t s) {
+                             const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
+                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, cudaStream_t s) {
     if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
     const int bn = pick_bn(d);
     CUtensorMap ma, mk, mh;
@@ -826,6 +862,10 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     p.gq = gq;
     p.gk = gk;
     p.part = reinterpret_cast<float4*>(part);
+    p.band_count = band_count;
+    p.alpha_w = alpha;
+    p.alpha_out = alpha_out;
+    p.eps = eps;
     p.status = status;
     p.n_tok = (int)n_tok;
     p.d_mem = d_mem;
@@ -835,16 +875,6 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     const int64_t mt = (n_tok + BM - 1) / BM;
     return bn == 256 ? launch_mode<MODE_K, 256>(ma, mk, mk, mh, p, mt, num_sms, s)
                      : launch_mode<MODE_K, 128>(ma, mk, mk, mh, p, mt, num_sms, s);
-}
-
-cudaError_t launch_alpha(const float* part, int64_t n_tok, int32_t d, float eps, float* alpha, float* alpha_out,
-                         int num_sms, cudaStream_t s) {
-    if (n_tok == 0) return cudaSuccess;
-    int64_t blocks = (n_tok + 7) / 8;
-    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-    alpha_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(part), n_tok, (d + 127) / 128, d,
-                                                  eps, alpha, alpha_out);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,

@@ -121,7 +121,8 @@ ENGRAM_API const char* engram_last_error(void);
 /* Bytes of scratch that engram_forward / engram_gate_conv need for B
  * sequences of L computed rows (n_tok = B*L): indices [n_tok][J] u32,
  * e [n_tok][J*D], gate partials [n_tok][G][4] f32 with G = ceil(d / 128), the
- * gate values [n_tok] f32, the next conv history [B][w-1][d] f32 and, where
+ * gate values [n_tok] f32, ceil(n_tok/128) int32 counters, the next conv
+ * history [B][w-1][d] f32 and, where
  * the gate and conv are not
  * fused into the projection (see engram_gate_conv), v [n_tok][d] f32; each
  * part 256-byte aligned.  0 for a null context. */
@@ -226,7 +227,8 @@ ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int
  * B, T - t_begin)) return ENGRAM_E_NOMEM with an explanation in
  * engram_last_error and launch nothing.  No cudaMalloc or cudaFree is called.
  * All calls share the one array, which keeps the last call's contents (the
- * forward writes every scratch byte before reading it): calls that may
+ * forward clears the counters it needs zeroed and writes every other
+ * scratch byte before reading it): calls that may
  * overlap on the GPU (other streams, other host threads) race on it and must
  * be serialised by the caller. */
 #define ENGRAM_NOALLOC_SCRATCH_BYTES (32u << 20)
