@@ -14,7 +14,7 @@ from .binding import (  # noqa: F401  (re-exported C ABI names)
     ENGRAM_BF16, ENGRAM_F32, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
     ENGRAM_INVALID_INDEX, ENGRAM_OK, EXPORTS, LIB_PATH, EngramError, engram_config, engram_conv, engram_create,
     ENGRAM_NOALLOC_SCRATCH_BYTES, engram_destroy, engram_device_status, engram_forward, engram_forward_noalloc,
-    engram_gate_conv, engram_gather, engram_hash,
+    engram_forward_host, engram_gate_conv, engram_gather, engram_hash, engram_host_workspace_bytes,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 
@@ -62,6 +62,22 @@ class Engram:
         engram_forward(self.ctx, tok, B, T, tok.stride(0), t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w,
                        conv_state, y, alpha_out, add_residual, self.workspace, self.workspace_bytes, stream)
         return y
+
+    def forward_host(self, tok_host, P, tables, h_host, Wk, Wv, conv_w, y_host, *, t_begin: int = 0, gq=None,
+                     gk=None, conv_state=None, add_residual: bool = False, chunk_rows: int = 0, stream=None):
+        """The forward with tok, h and y in host memory (pinned CPU tensors
+        overlap their copies with the compute); returns y_host, complete once
+        the stream is synchronised."""
+        import torch
+        B, T = tok_host.shape[0], tok_host.shape[1]
+        need = engram_host_workspace_bytes(self.ctx, B, T, t_begin, chunk_rows)
+        if need > getattr(self, "host_workspace_bytes", 0):
+            self.host_workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self.host_workspace_bytes = need
+        engram_forward_host(self.ctx, tok_host, B, T, tok_host.stride(0), t_begin, P, tables, h_host, Wk, Wv, gq, gk,
+                            conv_w, conv_state, y_host, add_residual, chunk_rows, self.host_workspace,
+                            self.host_workspace_bytes, stream)
+        return y_host
 
     def status(self, stream=None):
         return engram_device_status(self.ctx, stream)

@@ -35,7 +35,7 @@ ENGRAM_PART_GROUP = 128
 EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_error", "engram_workspace_bytes",
            "engram_profile_enable", "engram_profile_read", "engram_device_status", "engram_remap", "engram_hash",
            "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward",
-           "engram_forward_noalloc")
+           "engram_forward_noalloc", "engram_host_workspace_bytes", "engram_forward_host")
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -86,6 +86,9 @@ _sigs = {
                         _i32, _vp, _sz, _vp], _st),
     "engram_forward_noalloc": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, _i32, _vp], _st),
+    "engram_host_workspace_bytes": ([_vp, _i32, _i32, _i32, _i32], _sz),
+    "engram_forward_host": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                             _i32, _vp, _sz, _vp], _st),
 }
 for _name, (_args, _res) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -218,3 +221,17 @@ def engram_forward_noalloc(ctx, tok, B, T, tok_stride, t_begin, P, tables, h, Wk
                                        _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w), _ptr(conv_state),
                                        _ptr(y), _ptr(alpha_out), int(add_residual), _stream(stream)),
            "engram_forward_noalloc")
+
+
+def engram_host_workspace_bytes(ctx: int, B: int, T: int, t_begin: int, chunk_rows: int = 0) -> int:
+    return int(_lib.engram_host_workspace_bytes(ctx, B, T, t_begin, chunk_rows))
+
+
+def engram_forward_host(ctx, tok_host, B, T, tok_stride, t_begin, P, tables, h_host, Wk, Wv, gq, gk, conv_w,
+                        conv_state, y_host, add_residual, chunk_rows, workspace, workspace_bytes, stream=None):
+    """engram_forward with tok, h and y in host memory (CPU tensors, ideally
+    pinned); the other tensors on the device."""
+    _check(_lib.engram_forward_host(ctx, _ptr(tok_host), B, T, tok_stride, t_begin, _ptr(P), _ptr(tables),
+                                    _ptr(h_host), _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w),
+                                    _ptr(conv_state), _ptr(y_host), int(add_residual), chunk_rows, _ptr(workspace),
+                                    workspace_bytes, _stream(stream)), "engram_forward_host")

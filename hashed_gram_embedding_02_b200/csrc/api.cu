@@ -8,34 +8,9 @@
 #include <mutex>
 #include <new>
 
-#include "common.cuh"
+#include "ctx.cuh"
 
-using namespace engram;
-
-namespace {
-constexpr int kMaxProf = 16;
-}
-
-struct engram_ctx {
-    engram_config cfg;
-    int device;
-    int num_sms;
-    bool sm100;
-    int J;
-    int d_mem;
-    int G;
-    int es;                 // element size of the storage dtype
-    HashParams hp;
-    GatherParams gp;
-    uint32_t* d_status;     // device status word (256-byte block)
-    // per-kernel timing (engram_profile_enable)
-    bool prof;
-    cudaEvent_t ev[2 * kMaxProf];
-    const char* prof_name[kMaxProf];
-    int prof_n;
-};
-
-namespace {
+namespace engram {
 
 thread_local char g_last_error[256] = "";
 
@@ -62,10 +37,6 @@ bool is_prime_u32(uint32_t n) {
         if (n % f == 0) return false;
     return true;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------------- profiling
 
@@ -95,20 +66,6 @@ bool fused_path(const engram_ctx* c, int64_t n) { return tc_path(c, n) && c->cfg
 // per-128-row-band counters of the key pass
 size_t band_bytes(int64_t n) { return (size_t)((n + 127) / 128) * sizeof(int); }
 
-struct Workspace {
-    uint32_t* idx;
-    void* e;
-    float* part;
-    float* alpha;
-    int* band;
-    float* state_next;
-    float* v;
-    size_t bytes;
-};
-
-// idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | alpha [n] f32 | band counters |
-// state_next [B][w-1][d] f32 |
-// v [n][d] f32 (unfused paths only), each 256-byte aligned
 Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e) {
     const int64_t n = B * L;
     Workspace w{};
@@ -210,7 +167,33 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
     return conv_impl(c, w.v, w.part, h, conv_w, B, L, state, y, alpha_out, add_residual, s);
 }
 
-}  // namespace
+engram_status check_forward_args(const engram_ctx* c, int32_t B, int32_t T, int64_t tok_stride, int32_t t_begin) {
+    if (!c) return inval("null context");
+    if (B < 0 || T < 0 || t_begin < 0 || t_begin > T) return inval("need B >= 0 and 0 <= t_begin <= T");
+    if (tok_stride < T) return inval("tok_stride must be >= T");
+    return ENGRAM_OK;
+}
+
+engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
+                           int32_t t_begin, const int32_t* P, const void* tables, const void* h, const void* Wk,
+                           const void* Wv, const float* gq, const float* gk, const float* conv_w, float* conv_state,
+                           void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s) {
+    const int32_t L = T - t_begin;
+    const int64_t n = (int64_t)B * L;
+    prof_begin(c, s, "hash");
+    cudaError_t e = launch_hash(tok, P, B, T, tok_stride, t_begin, w.idx, c->hp, c->d_status, s);
+    prof_end(c, s);
+    if (e != cudaSuccess) return cuda_fail("hash launch", e);
+    prof_begin(c, s, "gather");
+    e = launch_gather(w.idx, n, tables, c->gp, w.e, c->d_status, c->num_sms, s);
+    prof_end(c, s);
+    if (e != cudaSuccess) return cuda_fail("gather launch", e);
+    return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
+}
+
+}  // namespace engram
+
+using namespace engram;
 
 extern "C" {
 
@@ -302,10 +285,13 @@ engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
         return e == cudaErrorMemoryAllocation ? ENGRAM_E_NOMEM : cuda_fail("cudaMalloc status", e);
     }
     e = cudaMemset(c->d_status, 0, 256);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io_h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io_d2h, cudaStreamNonBlocking);
+    for (int i = 0; i < kIoEvents && e == cudaSuccess; ++i)
+        e = cudaEventCreateWithFlags(&c->io_ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
-        cudaFree(c->d_status);
-        delete c;
-        return cuda_fail("cudaMemset status", e);
+        engram_destroy(c);
+        return cuda_fail("context set-up (status word, copy streams, events)", e);
     }
     *out = c;
     return ENGRAM_OK;
@@ -315,6 +301,10 @@ void engram_destroy(engram_ctx* c) {
     if (!c) return;
     if (c->prof)
         for (int i = 0; i < 2 * kMaxProf; ++i) cudaEventDestroy(c->ev[i]);
+    for (int i = 0; i < kIoEvents; ++i)
+        if (c->io_ev[i]) cudaEventDestroy(c->io_ev[i]);
+    if (c->io_h2d) cudaStreamDestroy(c->io_h2d);
+    if (c->io_d2h) cudaStreamDestroy(c->io_d2h);
     if (c->d_status) cudaFree(c->d_status);
     delete c;
 }
@@ -475,9 +465,8 @@ engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32
                              const void* Wv, const float* gq, const float* gk, const float* conv_w,
                              float* conv_state, void* y, float* alpha_out, int32_t add_residual, void* workspace,
                              size_t workspace_bytes, cudaStream_t s) {
-    if (!c) return inval("null context");
-    if (B < 0 || T < 0 || t_begin < 0 || t_begin > T) return inval("need B >= 0 and 0 <= t_begin <= T");
-    if (tok_stride < T) return inval("tok_stride must be >= T");
+    engram_status st = check_forward_args(c, B, T, tok_stride, t_begin);
+    if (st != ENGRAM_OK) return st;
     const int32_t L = T - t_begin;
     const int64_t n = (int64_t)B * L;
     if (n == 0) return ENGRAM_OK;
@@ -488,18 +477,11 @@ engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32
     if (!aligned16(tables) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
         (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
         return inval("tables, h, Wk, Wv, y, conv_w and conv_state must be 16-byte aligned");
-    engram_status st = check_device(c);
+    st = check_device(c);
     if (st != ENGRAM_OK) return st;
     prof_reset(c);
-    prof_begin(c, s, "hash");
-    cudaError_t e = launch_hash(tok, P, B, T, tok_stride, t_begin, w.idx, c->hp, c->d_status, s);
-    prof_end(c, s);
-    if (e != cudaSuccess) return cuda_fail("hash launch", e);
-    prof_begin(c, s, "gather");
-    e = launch_gather(w.idx, n, tables, c->gp, w.e, c->d_status, c->num_sms, s);
-    prof_end(c, s);
-    if (e != cudaSuccess) return cuda_fail("gather launch", e);
-    return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
+    return forward_impl(c, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
+                        alpha_out, add_residual, w, s);
 }
 
 // ---------------------------------------------------------------- forward without allocation

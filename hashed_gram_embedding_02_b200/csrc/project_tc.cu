@@ -22,15 +22,16 @@
 //              v never reaches global memory.  Consecutive segments overlap
 //              by 3 rows (116 output rows per 128-row MMA tile).
 //
-// Persistent kernel, one CTA per SM, warp-specialised (384 threads):
+// Persistent kernel, one CTA per SM, warp-specialised (640 threads):
 //   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of A (e) and
 //              W into a shared-memory ring, and of the tile's h slice into a
 //              shared buffer the epilogue reads (issued after the tile's
 //              k-blocks, so it never holds back the MMA)
 //   warp 1     allocates TMEM (two fp32 accumulators) and issues
 //              tcgen05.mma kind::f16 (M=128, N=BN, K=16) from one thread
-//   warps 4-11 epilogue: warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31;
-//              warps 4-7 and 8-11 take the two halves of the tile's channels
+//   warps 4-19 epilogue: warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31;
+//              the four groups of four warps take four column parts of
+//              the tile's channels
 // The double-buffered accumulator lets the epilogue of tile i overlap the
 // MMAs of tile i+1.  Tiles run channel-fastest so consecutive tiles share the
 // A block in L2; W stays L2-resident.
@@ -382,20 +383,32 @@ __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, co
 // Gate + causal depthwise conv (width 4) + residual on a value tile of BN
 // channels.  Lane l of warp segment q holds row r0q + l; lanes 0..2 are the
 // history rows of the segment's first output row.  Each of the NPART parts
-// handles BN/NPART channels, 16 at a time, TMEM loads one chunk ahead.  The
-// history values travel between lanes as fp16 pairs (one shuffle per two
-// channels per shift; relative error at most 2^-11 of each history term,
-// below the bf16 rounding of Y), which halves the shuffle traffic that
-// otherwise saturates the shared-memory/shuffle pipe.  The taps arrive
-// pre-halved, so the tap sum is x/2 and SiLU(x) = x/2 + x/2 * tanh(x/2)
-// needs no extra scaling.
+// handles BN/NPART channels, 16 at a time, TMEM loads one chunk ahead.
+// v~ = alpha v is formed in fp32 per lane; the conv and SiLU run on channel
+// pairs in fp16x2: the history values travel between lanes as the same
+// fp16 pairs (one shuffle per two channels per shift), the taps are fp16
+// pairs, and SiLU(x) = x/2 + x/2 tanh(x/2) uses the paired hardware tanh.
+// Each term of the tap sum carries a relative rounding of at most about
+// 2^-10, below the bf16 rounding of Y; the skip term v~ and the residual
+// stay fp32.  The taps arrive pre-halved, so the tap sum is already x/2.
+// The fp16 range bounds |v~| and the tap sum by 65504.
+__device__ __forceinline__ uint32_t h2u(__half2 x) { return *reinterpret_cast<uint32_t*>(&x); }
+__device__ __forceinline__ __half2 u2h(uint32_t x) { return *reinterpret_cast<__half2*>(&x); }
+
+__device__ __forceinline__ __half2 tanh_h2(__half2 x) {
+    uint32_t r;
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h2u(x)));
+    return u2h(r);
+}
+
 template <int BN, bool SLOW, bool RES>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
-                                             const float4* s_cw) {
+                                             const uint4* s_cw) {
     constexpr int H = CONV_W - 1;
     constexpr int NCH = BN / NPART / 16;
     const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
+    const bool from_state = SLOW && t < H && p.state;
     uint4* yrow = reinterpret_cast<uint4*>(p.y + r * p.d + n0 + cbeg);
     uint32_t va[16], vb[16];
     tmem_ld16(taddr + cbeg, va);
@@ -415,35 +428,39 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, 
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
             const float v0 = a * __uint_as_float(cur[c]), v1 = a * __uint_as_float(cur[c + 1]);
-            __half2 pk = __floats2half2_rn(v0, v1);
-            const uint32_t u0 = *reinterpret_cast<uint32_t*>(&pk);
+            const __half2 vh = __floats2half2_rn(v0, v1);
+            const uint32_t u0 = h2u(vh);
             uint32_t s1 = __shfl_up_sync(0xffffffffu, u0, 1);
             uint32_t s2 = __shfl_up_sync(0xffffffffu, u0, 2);
             uint32_t s3 = __shfl_up_sync(0xffffffffu, u0, 3);
-            const float2 f1 = __half22float2(*reinterpret_cast<__half2*>(&s1));
-            const float2 f2 = __half22float2(*reinterpret_cast<__half2*>(&s2));
-            const float2 f3 = __half22float2(*reinterpret_cast<__half2*>(&s3));
+            if (SLOW && t < H) {
+                // history before the slab start: conv_state (zero without one);
+                // the row t-k comes from state row H-k+t
+                uint32_t ps[H] = {0u, 0u, 0u};
+                if (from_state) {
+                    const float* st = p.state + (b * H) * p.d + n0 + cl + c;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float vt = e ? v1 : v0;
-                float p1 = e ? f1.y : f1.x, p2 = e ? f2.y : f2.x, p3 = e ? f3.y : f3.x;
-                if (SLOW && t < H) {
-                    const float* st = p.state ? p.state + (b * H) * p.d + n0 + cl + c + e : nullptr;
-                    if (t < 1) p1 = st ? st[(H - 1 + t) * p.d] : 0.f;
-                    if (t < 2) p2 = st ? st[(H - 2 + t) * p.d] : 0.f;
-                    p3 = st ? st[(H - 3 + t) * p.d] : 0.f;
+                    for (int k = 1; k <= H; ++k)
+                        if (t < k) {
+                            const float2 x = __ldg(reinterpret_cast<const float2*>(st + (int64_t)(H - k + t) * p.d));
+                            ps[k - 1] = h2u(__floats2half2_rn(x.x, x.y));
+                        }
                 }
-                const float4 w4 = s_cw[cl + c + e];
-                float hx = w4.x * vt;
-                hx = fmaf(w4.y, p1, hx);
-                hx = fmaf(w4.z, p2, hx);
-                hx = fmaf(w4.w, p3, hx);
-                float th;
-                asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hx));
-                const float base = RES ? vt + hv[c + e] : vt;
-                o[c + e] = base + fmaf(hx, th, hx);
-                if (write_state) p.state_next[(b * H + (t - (p.L - H))) * p.d + n0 + cl + c + e] = vt;
+                if (t < 1) s1 = ps[0];
+                if (t < 2) s2 = ps[1];
+                s3 = ps[2];
             }
+            if (write_state)
+                *reinterpret_cast<float2*>(p.state_next + (b * H + (t - (p.L - H))) * p.d + n0 + cl + c) =
+                    make_float2(v0, v1);
+            const uint4 w = s_cw[(cl + c) >> 1];          // halved taps c_0..c_3 of the channel pair
+            __half2 hx = __hmul2(u2h(w.x), vh);
+            hx = __hfma2(u2h(w.y), u2h(s1), hx);
+            hx = __hfma2(u2h(w.z), u2h(s2), hx);
+            hx = __hfma2(u2h(w.w), u2h(s3), hx);
+            const float2 sl = __half22float2(__hfma2(hx, tanh_h2(hx), hx));
+            o[c] = (RES ? v0 + hv[c] : v0) + sl.x;
+            o[c + 1] = (RES ? v1 + hv[c + 1] : v1) + sl.y;
         }
         if (out_row) {
             yrow[2 * ch] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
@@ -470,18 +487,22 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const uint8_t* hs
     }
     const float a = in_range ? __ldg(p.alpha + r) : 0.f;
     const int n0 = nt * BN;
-    // conv taps of the tile's channels, halved: [BN] float4
+    // conv taps of the tile's channel pairs, halved, as fp16 pairs: [BN/2]
+    // x {c_0, c_1, c_2, c_3} of (channel 2m, channel 2m+1)
     epi_sync();
-    for (int k = et; k < BN; k += EPI_THREADS) {
-        const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + k);
-        reinterpret_cast<float4*>(s_taps)[k] = make_float4(0.5f * w.x, 0.5f * w.y, 0.5f * w.z, 0.5f * w.w);
+    for (int k = et; k < BN / 2; k += EPI_THREADS) {
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k);
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k + 1);
+        reinterpret_cast<uint4*>(s_taps)[k] =
+            make_uint4(h2u(__floats2half2_rn(0.5f * w0.x, 0.5f * w1.x)), h2u(__floats2half2_rn(0.5f * w0.y, 0.5f * w1.y)),
+                       h2u(__floats2half2_rn(0.5f * w0.z, 0.5f * w1.z)), h2u(__floats2half2_rn(0.5f * w0.w, 0.5f * w1.w)));
     }
     epi_sync();
     // warps whose rows all have their history inside the sequence and write no
     // new history take the branch-free path
     const bool slow_row = out_row && (t < H || (p.state_next && t >= p.L - H));
     const int cbeg = part * (BN / NPART);
-    const float4* cw = reinterpret_cast<const float4*>(s_taps);
+    const uint4* cw = reinterpret_cast<const uint4*>(s_taps);
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
         if (slow) vconv_chunks<BN, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);

@@ -239,6 +239,41 @@ ENGRAM_API engram_status engram_forward_noalloc(engram_ctx* ctx, const int32_t* 
                                      float* conv_state, void* y, float* alpha_out, int32_t add_residual,
                                      cudaStream_t stream);
 
+/* The whole forward from and to HOST memory: the end-to-end call of a caller
+ * whose hidden states live on the host.  The pages (the Synced repost,
+ * section "System efficiency: decoupling compute and storage") describe the
+ * retrieval as depending only on token ids, which is what lets transfers
+ * overlap compute; this entry point applies that to the per-token tensors.
+ *   tok_host  int32 [B][tok_stride] raw ids, host memory;
+ *   h_host    [B][L][d] hidden states (model dtype), host memory;
+ *   y_host    [B][L][d] output (model dtype), host memory, L = T - t_begin;
+ *   P, tables, Wk, Wv, gq, gk, conv_w, conv_state: device memory, as in
+ *             engram_forward (conv_state nullable: zero history).
+ * The rows are processed in chunks of `chunk_rows` positions of every
+ * sequence (0: about 8 MiB of h per chunk).  While chunk i computes on
+ * `stream`, the h of chunk i+1 is copied in on one of the context's copy
+ * streams and the Y of chunk i-1 is copied out on the other
+ * (cudaMemcpy2DAsync).  The conv history passes from chunk to chunk through
+ * conv_state, or through a zeroed copy in the workspace when conv_state is
+ * null, so the result equals engram_forward's.  Only the id window each
+ * sequence needs (from t_begin - (max order - 1)) is copied in.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister); with
+ * pageable memory the copies are correct but do not overlap.
+ * Device scratch: `workspace`, engram_host_workspace_bytes(ctx, B, T,
+ * t_begin, chunk_rows) bytes, 256-byte aligned.
+ * Returns once everything is enqueued; y_host (and conv_state) are complete
+ * when `stream` completes.  Host buffers must stay valid until then.  Errors
+ * are as engram_forward's, checked before anything is enqueued. */
+ENGRAM_API size_t engram_host_workspace_bytes(const engram_ctx* ctx, int32_t B, int32_t T, int32_t t_begin,
+                                              int32_t chunk_rows);
+ENGRAM_API engram_status engram_forward_host(engram_ctx* ctx, const int32_t* tok_host, int32_t B, int32_t T,
+                                             int64_t tok_stride, int32_t t_begin, const int32_t* P,
+                                             const void* tables, const void* h_host, const void* Wk,
+                                             const void* Wv, const float* gq, const float* gk,
+                                             const float* conv_w, float* conv_state, void* y_host,
+                                             int32_t add_residual, int32_t chunk_rows, void* workspace,
+                                             size_t workspace_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

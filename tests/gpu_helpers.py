@@ -36,12 +36,17 @@ def bf16_bound(y_ref: np.ndarray, vt_win: np.ndarray, cw: np.ndarray) -> np.ndar
     """Elementwise bound on |Y_gpu - Y_oracle| for the bf16 path.
 
     Sources: (1) Y is rounded once to bf16 (half an ulp, 2^-8 relative);
-    (2) v is stored as bf16 after an fp32 (GPU) or fp64 (oracle) accumulation,
-    so the two may land one bf16 ulp apart (2^-7 relative); such a flip in
-    v_{t-j} moves v~_{t-j} by at most 2^-7 |v~_{t-j}| and reaches Y_t through
-    the skip (j = 0, weight 1) and through SiLU(u) (weight |c_j| * max SiLU',
-    max SiLU' < 1.1); (3) fp32 arithmetic in the gate and conv, well below
-    1e-5 at these magnitudes.  A factor 1.5 covers both (1) and (2) at once."""
+    (2) the fused epilogue evaluates the tap sum and SiLU on fp16 pairs:
+    each history value and tap is rounded to fp16 (2^-11 relative), each
+    product and partial sum rounds to fp16, and the paired tanh
+    approximation errs by about 2^-10.7 relative; together well under
+    2^-8 of sum_j |c_j| |v~_{t-j}|.  The accumulation order of v (fp32)
+    differs from the oracle's (fp64) only in the last bits.  An error of
+    relative size r in v~_{t-j} reaches Y_t through the skip (j = 0, weight 1)
+    and through SiLU(u) (weight |c_j| * max SiLU', max SiLU' < 1.1).  The
+    bound allows r = 2^-7 per term and a factor 1.5 on the sum; (3) fp32
+    arithmetic in the gate and the skip/residual add stays well below 1e-5
+    at these magnitudes."""
     w = cw.shape[1]
     s = np.abs(vt_win[:, 0]) * (1.0 + 1.1 * np.abs(cw[None, :, 0]))
     for j in range(1, w):

@@ -88,3 +88,6 @@ def test_null_context_is_rejected(eb):
     assert binding._lib.engram_forward(None, None, 1, 1, 1, 0, None, None, None, None, None, None, None, None,
                                        None, None, None, 0, None, 0, None) == binding.ENGRAM_E_INVAL
     assert eb.engram_workspace_bytes(None, 2, 10) == 0
+    assert eb.engram_host_workspace_bytes(None, 2, 10, 0, 0) == 0
+    assert binding._lib.engram_forward_host(None, None, 1, 1, 1, 0, None, None, None, None, None, None, None, None,
+                                            None, None, 0, 0, None, 0, None) == binding.ENGRAM_E_INVAL
