@@ -14,7 +14,9 @@ from .binding import (  # noqa: F401  (re-exported C ABI names)
     ENGRAM_BF16, ENGRAM_F32, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
     ENGRAM_INVALID_INDEX, ENGRAM_OK, EXPORTS, LIB_PATH, EngramError, engram_config, engram_conv, engram_create,
     ENGRAM_NOALLOC_SCRATCH_BYTES, engram_destroy, engram_device_status, engram_forward, engram_forward_noalloc,
-    engram_forward_host, engram_gate_conv, engram_gather, engram_hash, engram_host_workspace_bytes,
+    engram_forward_host, engram_gate_conv, engram_gather, engram_gather_staged, engram_hash, engram_host_dedupe,
+    engram_host_fetch, engram_host_tier_create, engram_host_tier_destroy, engram_host_tier_stats,
+    engram_host_workspace_bytes, engram_pack_rows,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 
@@ -81,3 +83,37 @@ class Engram:
 
     def status(self, stream=None):
         return engram_device_status(self.ctx, stream)
+
+
+class HostTier:
+    """Owns one engram_host_tier: tables in host memory, rows fetched per
+    batch (engram_host_dedupe -> engram_host_fetch -> engram_gather_staged)."""
+
+    def __init__(self, engram: "Engram", host_tables, max_lookups: int, n_threads: int = 8):
+        self.engram = engram
+        self.host_tables = host_tables          # keeps the host memory alive
+        self.tier = engram_host_tier_create(engram.ctx, host_tables, max_lookups, n_threads)
+
+    def close(self):
+        if self.tier:
+            engram_host_tier_destroy(self.tier)
+            self.tier = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def dedupe(self, idx, n_tok: int, stream=None):
+        engram_host_dedupe(self.tier, idx, n_tok, stream)
+
+    def fetch(self, side_stream) -> int:
+        return engram_host_fetch(self.tier, side_stream)
+
+    def gather(self, n_tok: int, e_cat, stream=None):
+        engram_gather_staged(self.tier, n_tok, e_cat, stream)
+        return e_cat
+
+    def stats(self):
+        return engram_host_tier_stats(self.tier)

@@ -35,7 +35,9 @@ ENGRAM_PART_GROUP = 128
 EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_error", "engram_workspace_bytes",
            "engram_profile_enable", "engram_profile_read", "engram_device_status", "engram_remap", "engram_hash",
            "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward",
-           "engram_forward_noalloc", "engram_host_workspace_bytes", "engram_forward_host")
+           "engram_forward_noalloc", "engram_host_workspace_bytes", "engram_forward_host", "engram_host_tier_create",
+           "engram_host_tier_destroy", "engram_host_dedupe", "engram_host_fetch", "engram_gather_staged",
+           "engram_host_tier_stats", "engram_pack_rows")
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -87,6 +89,13 @@ _sigs = {
     "engram_forward_noalloc": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, _i32, _vp], _st),
     "engram_host_workspace_bytes": ([_vp, _i32, _i32, _i32, _i32], _sz),
+    "engram_host_tier_create": ([_vp, _vp, _i64, _i32, ctypes.POINTER(_vp)], _st),
+    "engram_host_tier_destroy": ([_vp], None),
+    "engram_host_dedupe": ([_vp, _vp, _i64, _vp], _st),
+    "engram_host_fetch": ([_vp, _vp, ctypes.POINTER(_i64)], _st),
+    "engram_gather_staged": ([_vp, _i64, _vp, _vp], _st),
+    "engram_host_tier_stats": ([_vp, ctypes.c_void_p], _st),
+    "engram_pack_rows": ([_vp, _i64, _sz, _vp, _i64, _vp, _i32], _st),
     "engram_forward_host": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                              _i32, _vp, _sz, _vp], _st),
 }
@@ -235,3 +244,53 @@ def engram_forward_host(ctx, tok_host, B, T, tok_stride, t_begin, P, tables, h_h
                                     _ptr(h_host), _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w),
                                     _ptr(conv_state), _ptr(y_host), int(add_residual), chunk_rows, _ptr(workspace),
                                     workspace_bytes, _stream(stream)), "engram_forward_host")
+
+
+# ---------------------------------------------------------------- host tier
+
+def engram_host_tier_create(ctx, host_tables, max_lookups: int, n_threads: int) -> int:
+    """host_tables: a CPU tensor (or anything with data_ptr()) holding the
+    [J][M][D] tables; it must outlive the tier."""
+    out = _vp()
+    _check(_lib.engram_host_tier_create(ctx, _ptr(host_tables), max_lookups, n_threads, ctypes.byref(out)),
+           "engram_host_tier_create")
+    return out.value
+
+
+def engram_host_tier_destroy(tier: int) -> None:
+    _lib.engram_host_tier_destroy(tier)
+
+
+def engram_host_dedupe(tier, idx, n_tok, stream=None):
+    _check(_lib.engram_host_dedupe(tier, _ptr(idx), n_tok, _stream(stream)), "engram_host_dedupe")
+
+
+def engram_host_fetch(tier, side_stream) -> int:
+    n = _i64(0)
+    _check(_lib.engram_host_fetch(tier, _stream(side_stream), ctypes.byref(n)), "engram_host_fetch")
+    return int(n.value)
+
+
+def engram_gather_staged(tier, n_tok, e_cat, stream=None):
+    _check(_lib.engram_gather_staged(tier, n_tok, _ptr(e_cat), _stream(stream)), "engram_gather_staged")
+
+
+class engram_host_tier_stats_t(ctypes.Structure):
+    _fields_ = [("n_unique", ctypes.c_int64), ("n_copies", ctypes.c_int64), ("wait_ms", ctypes.c_double),
+                ("pack_ms", ctypes.c_double), ("copy_ms", ctypes.c_double)]
+
+
+def engram_host_tier_stats(tier) -> dict:
+    """Figures of the last fetch: distinct rows, copies, host wait / packing
+    ms, device copy ms (-1 while in flight)."""
+    out = engram_host_tier_stats_t()
+    _check(_lib.engram_host_tier_stats(tier, ctypes.addressof(out)), "engram_host_tier_stats")
+    return {f: getattr(out, f) for f, _ in out._fields_}
+
+
+def engram_pack_rows(host_tables, total_rows: int, row_bytes: int, rows, n: int, dst, n_threads: int = 1):
+    """Host-only packing: rows[i] of the tables into dst[i] (CPU tensors or numpy arrays)."""
+    def addr(x):
+        return x.ctypes.data if hasattr(x, "ctypes") else x.data_ptr()
+    _check(_lib.engram_pack_rows(addr(host_tables), total_rows, row_bytes, addr(rows), n, addr(dst), n_threads),
+           "engram_pack_rows")

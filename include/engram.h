@@ -27,8 +27,11 @@
  *   conv      u_t = sum_{j<w} c[ch][j] * v~_{t-j} (per channel, causal;
  *             history before the first computed position from conv_state,
  *             else zero), Y_t = v~_t + SiLU(u_t) (+ h_t with add_residual).
- *   storage   bf16 configurations store e and v as bf16 and Y as bf16;
- *             k, alpha, u and the conv history stay fp32.
+ *   storage   bf16 configurations store e and Y as bf16; k, v, alpha and
+ *             the conv history stay fp32 (v is stored, in fp32, only where
+ *             the gate and conv are not fused into the projection).  The
+ *             fused path evaluates the tap sum and SiLU on fp16 pairs, so
+ *             |v~| and the tap sum must stay within the fp16 range.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are caller-owned DEVICE memory unless stated; the
@@ -273,6 +276,80 @@ ENGRAM_API engram_status engram_forward_host(engram_ctx* ctx, const int32_t* tok
                                              const float* conv_w, float* conv_state, void* y_host,
                                              int32_t add_residual, int32_t chunk_rows, void* workspace,
                                              size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- host tier
+ *
+ * Tables too large for HBM stay in host memory; each batch fetches over PCIe
+ * only the rows its n-grams activate.  The pages (the "DeepSeek AI II"
+ * digest, section "DeepSeek Engram", system efficiency; the Synced repost,
+ * section "System efficiency: decoupling compute and storage"; the QbitAI
+ * repost on the 100B-parameter table held in host memory) base this on the
+ * indices depending only on token ids: they are computed ahead of the layer,
+ * the distinct rows are copied while the preceding layers run, and the
+ * Zipf-skewed n-gram distribution keeps the distinct rows far fewer than the
+ * lookups.  A batch is three calls, in this order, with dedupe and
+ * gather_staged on the same stream:
+ *   engram_hash(...)                     indices [n_tok][J] on the device
+ *   engram_host_dedupe(tier, idx, n_tok, s)
+ *   ... other work on s (the preceding layers) ...
+ *   engram_host_fetch(tier, side, &n_unique)     blocks the calling thread
+ *                                                 while the rows are packed
+ *   engram_gather_staged(tier, n_tok, e_cat, s)  then engram_gate_conv.
+ */
+typedef struct engram_host_tier engram_host_tier;
+
+/* host_tables: [J][M_j][D] rows (model dtype) in host memory, back to back
+ * in table order; pageable memory is fine (it is only read by the packing
+ * threads).  max_lookups: the largest n_tok * J of any batch.  The tier
+ * allocates, once: a device hash set of 2^ceil(log2(2 max_lookups)) keys,
+ * the distinct-row list, the slot map and the staged rows on the device
+ * (max_lookups * D * elem bytes), and pinned host buffers for the list and
+ * the staging; it starts n_threads packing threads.  Returns
+ * ENGRAM_E_NOMEM when an allocation fails, ENGRAM_E_HOST when the threads
+ * cannot start.  The host tables must outlive the tier. */
+ENGRAM_API engram_status engram_host_tier_create(engram_ctx* ctx, const void* host_tables, int64_t max_lookups,
+                                                 int32_t n_threads, engram_host_tier** out);
+/* Waits (bounded) for copies in flight into the tier's pinned buffers, stops
+ * the threads and frees everything the tier allocated. */
+ENGRAM_API void engram_host_tier_destroy(engram_host_tier* tier);
+
+/* Enqueue on `stream`: clear the set; one kernel inserts every valid lookup's
+ * global row (row_off[j] + idx) and gives each distinct row the next slot;
+ * a second kernel writes each lookup's slot (invalid indices keep
+ * ENGRAM_INVALID_INDEX and later gather a zero row); the count and the
+ * distinct-row list are copied to pinned host memory.  Slot order depends
+ * on the atomics' timing; the gathered rows do not.  A set that overflows
+ * (impossible at its load factor of 1/2) sets ENGRAM_ERR_INDEX. */
+ENGRAM_API engram_status engram_host_dedupe(engram_host_tier* tier, const uint32_t* idx, int64_t n_tok,
+                                            cudaStream_t stream);
+/* Host side: waits (bounded, 20 s) for the distinct-row list, then the
+ * packing threads copy the rows from the host tables into pinned staging in
+ * chunks of 4096 rows; this thread hands the finished chunks, in order and
+ * at least 4 MB at a time (but the last), to cudaMemcpyAsync calls on
+ * `side_stream`.  Returns once every copy is
+ * enqueued, with the number of distinct rows in *n_unique (nullable).
+ * ENGRAM_E_TIMEOUT / ENGRAM_E_HOST when a wait or a packing thread runs out
+ * of time. */
+ENGRAM_API engram_status engram_host_fetch(engram_host_tier* tier, cudaStream_t side_stream, int64_t* n_unique);
+/* Enqueue on `stream`: wait for the fetched rows, then gather
+ * e_cat [n_tok][J*D] (device, 16-byte aligned) from the staged rows through
+ * the slot map: the same kernel and layout as engram_gather. */
+ENGRAM_API engram_status engram_gather_staged(engram_host_tier* tier, int64_t n_tok, void* e_cat,
+                                              cudaStream_t stream);
+/* Figures of the last fetch. */
+typedef struct {
+    int64_t n_unique;   /* distinct rows fetched */
+    int64_t n_copies;   /* cudaMemcpyAsync calls that carried them */
+    double wait_ms;     /* host wait for the distinct-row list (and the previous batch's copies) */
+    double pack_ms;     /* host: packing start to the last copy enqueued */
+    double copy_ms;     /* device: first row copy enqueued to the last one done; -1 while in flight */
+} engram_host_tier_stats_t;
+ENGRAM_API engram_status engram_host_tier_stats(const engram_host_tier* tier, engram_host_tier_stats_t* out);
+/* The packing step alone, on the host (no device involved): rows[i] of the
+ * [total_rows][row_bytes] host tables into dst[i], split over n_threads
+ * threads.  Every row number is checked (< total_rows) before any copy. */
+ENGRAM_API engram_status engram_pack_rows(const void* host_tables, int64_t total_rows, size_t row_bytes,
+                                          const uint64_t* rows, int64_t n, void* dst, int32_t n_threads);
 
 #ifdef __cplusplus
 }

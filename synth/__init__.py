@@ -117,6 +117,31 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
+def _is_prime(n: int) -> bool:
+    if n < 2:
+        return False
+    if n % 2 == 0:
+        return n == 2
+    f = 3
+    while f * f <= n:
+        if n % f == 0:
+            return False
+        f += 2
+    return True
+
+
+def host_scaled(wl: Workload, mem_bytes: int) -> Workload:
+    """The host-memory workload with its tables shrunk to fit ``mem_bytes``:
+    rows per table = the largest prime not above the stated size whose
+    J x rows x D tables fit (the sizing rule for a box with less host memory
+    than the stated 200 GB)."""
+    per_row = wl.J * wl.D * wl.elem_bytes
+    m = min(wl.M, int(mem_bytes // per_row))
+    while m > 2 and not _is_prime(m):
+        m -= 1
+    return wl if m == wl.M else wl.replace(M=m)
+
+
 def workload(name_or_wl) -> Workload:
     if isinstance(name_or_wl, Workload):
         return name_or_wl
@@ -317,6 +342,19 @@ class Inputs:
         for s in range(0, n, chunk):
             e = min(n, s + chunk)
             out[s:e] = normal_torch(wl.seed, TAG_TABLES, s, e - s, wl.table_sd, device).to(tdt)
+        return out.view(wl.J, self.M, wl.D)
+
+    def host_tables(self, device, chunk: int = 1 << 27, pin: bool = False):
+        """[J][M][D] tables in host memory (torch CPU tensor), the same values
+        as device_tables: generated on ``device`` in chunks and copied out."""
+        import torch
+        wl = self.wl
+        n = wl.J * self.M * wl.D
+        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        out = torch.empty(n, dtype=tdt, pin_memory=pin)
+        for s in range(0, n, chunk):
+            e = min(n, s + chunk)
+            out[s:e].copy_(normal_torch(wl.seed, TAG_TABLES, s, e - s, wl.table_sd, device).to(tdt))
         return out.view(wl.J, self.M, wl.D)
 
     def device_hidden(self, device, chunk: int = 1 << 27):
