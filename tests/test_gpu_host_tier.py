@@ -149,3 +149,35 @@ def test_host_tier_rejects_batches_beyond_its_capacity(eb):
         tier.dedupe(idx, 101)
     with pytest.raises(eb.EngramError):
         tier.fetch(torch.cuda.Stream())                  # no dedupe yet
+
+
+def test_c5_batch_forward_sampled_matches_oracle(eb):
+    """The host-memory configuration's batch (8 x 4096 tokens, d_mem 2048)
+    through dedupe, fetch, staged gather and the fused passes, checked
+    against the oracle at sampled rows (first rows, sequence ends included)."""
+    wl = FULL_BATCH
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    tier = eb.HostTier(ctx, inp.host_tables("cuda:0"), max_lookups=wl.n_tok * wl.J, n_threads=8)
+    idx = _indices(eb, ctx, di, wl)
+    e_t, _ = _staged_e(eb, ctx, tier, idx, wl, torch.cuda.Stream())
+    ws_bytes = eb.engram_workspace_bytes(ctx.ctx, wl.B, wl.T)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    y = di.empty_y()
+    alpha = torch.empty(wl.n_tok, dtype=torch.float32, device="cuda")
+    eb.engram_gate_conv(ctx.ctx, e_t, di.h, di.Wk, di.Wv, di.gq, di.gk, di.conv_w, wl.B, wl.T, None, y, alpha, 1,
+                        ws, ws_bytes)
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    canon_ref, _ = oracle.remap(inp.tok, inp.P)
+    idx_ref, _ = oracle.hash_ids(canon_ref, wl.Vc, wl.orders, wl.K, inp.mult, inp.rows)
+    assert np.array_equal(idx.cpu().numpy().view(np.uint32), idx_ref)
+    pos = synth.sample_positions(wl, 96, seed=9)
+    ref = oracle.forward_rows(inp, pos, add_residual=True, idx=idx_ref)
+    sel = torch.from_numpy(pos).cuda()
+    np.testing.assert_allclose(to_np(alpha[sel]), ref.alpha, rtol=0, atol=2e-6)
+    y_s = to_np(y[sel])
+    err = np.abs(y_s - ref.y)
+    assert err.max() <= 2e-2
+    assert not (err > bf16_bound(ref.y, ref.vt_win, inp.conv_w)).any()
