@@ -67,11 +67,15 @@ constexpr int SEG = 32;                 // rows per epilogue warp
 constexpr int SEG_OUT = SEG - (CONV_W - 1);   // output rows per warp segment (29)
 constexpr int TILE_OUT = 4 * SEG_OUT;         // output rows per value tile (116)
 
-template <int MODE, int BN>
+// PAIR: a cluster of two CTAs runs one M = 256 tcgen05 MMA (cta_group::2);
+// each CTA stages its own 128 rows of A and half of the BN columns of W, so a
+// stage costs each CTA 32 KB instead of 48 KB and four stages fit.
+template <int MODE, int BN, bool PAIR = false>
 struct Geo {
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;          // W rows (channels) this CTA stages
+    static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = BN == 256 ? 3 : 4;
+    static constexpr int STAGES = PAIR ? 4 : (BN == 256 ? 3 : 4);
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int SMEM_TILES = STAGES * STAGE_BYTES;
     static constexpr int HC = MODE == MODE_KV ? 128 : BN;      // h channels per tile
@@ -86,6 +90,7 @@ struct Geo {
 struct __align__(8) Barriers {
     uint64_t full[8];
     uint64_t empty[8];
+    uint64_t pfull[8];    // PAIR, leader: the peer's stage is full (one remote arrival)
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t hfull;
@@ -98,6 +103,7 @@ struct __align__(8) Barriers {
     int h_issued;     // h tiles issued
     int h_consumed;   // h tiles released by the epilogue
     int band_last;    // this CTA completed a row band's partials (MODE_K)
+    uint32_t peer_abort;   // PAIR: cluster address of the other CTA's abort_flag, else 0
 };
 
 struct EpiParams {
@@ -124,16 +130,24 @@ struct EpiParams {
 
 // Bounded wait: true when the phase with `parity` completed, false when the
 // CTA aborted or the wait ran out (then the status bit and abort flag are set).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity);
+__device__ __forceinline__ void st_remote_s32(uint32_t cluster_addr, int v);
+
+// CLUSTER: the barrier also receives arrivals from the other CTA of a pair
+// (acquire at cluster scope).  A timeout also raises the peer's abort flag.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Barriers* sb, uint32_t* status) {
     const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
+    auto try_wait = [&]() { return CLUSTER ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity); };
+    if (try_wait()) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(a, parity)) return true;
+        if (try_wait()) return true;
         if (sb->abort_flag) return false;
         if (clock64() - t0 > kWaitCycles) {
             flag(status, ENGRAM_ERR_TIMEOUT);
             sb->abort_flag = 1;
+            if (sb->peer_abort) st_remote_s32(sb->peer_abort, 1);
             return false;
         }
     }
@@ -164,10 +178,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
 // K-major, N = BN, M = 128.
-template <int BN>
+template <int BN, int M = BM>
 struct Idesc {
     static constexpr uint32_t value =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 };
 
 template <int BN>
@@ -182,6 +196,97 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
+}
+
+// ---- CTA pair (cluster of 2, cta_group::2)
+
+// M = 256 x N = BN MMA over both CTAs of the pair, issued by the leader:
+// A rows 0-127 from the leader's shared memory and 128-255 from the peer's,
+// W columns split the same way; D rows land in each CTA's own TMEM.
+template <int BN>
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN, 2 * BM>::value), "r"(accumulate));
+}
+
+// arrive on the barrier at the same offset in both CTAs once the pair's
+// earlier MMAs complete
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\t"
+        "mov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}\n"
+        ::"r"(smem_u32(bar))
+        : "memory");
+}
+
+// arrive on this CTA's barrier once the pair's earlier MMAs complete
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_addr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr), "r"(bytes)
+                 : "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// a barrier of the other CTA of the pair (cta_group::2 form, no multicast)
+__device__ __forceinline__ void tma_load_2d_peer_bar(const CUtensorMap* map, uint32_t dst, uint32_t bar_cluster, int x,
+                                                     int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(dst),
+        "l"(map), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ int ld_remote_s32(uint32_t cluster_addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_remote_s32(uint32_t cluster_addr, int v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// all threads of both CTAs
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -244,6 +349,12 @@ __device__ __forceinline__ uint4 h_chunk(const uint8_t* hs, int i, int cl) {
     const int cb = cl >> 6;
     const int ck = (cl & 63) >> 3;
     return *reinterpret_cast<const uint4*>(hs + cb * (BM * 128) + i * 128 + ((ck ^ (i & 7)) << 4));
+}
+
+__device__ __forceinline__ uint4* h_chunk_ptr(uint8_t* hs, int i, int cl) {
+    const int cb = cl >> 6;
+    const int ck = (cl & 63) >> 3;
+    return reinterpret_cast<uint4*>(hs + cb * (BM * 128) + i * 128 + ((ck ^ (i & 7)) << 4));
 }
 
 __device__ __forceinline__ void unpack8(const uint4& q, float* f) {
@@ -402,14 +513,13 @@ __device__ __forceinline__ __half2 tanh_h2(__half2 x) {
 }
 
 template <int BN, bool SLOW, bool RES>
-__device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int i, int64_t r,
+__device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
                                              const uint4* s_cw) {
     constexpr int H = CONV_W - 1;
     constexpr int NCH = BN / NPART / 16;
     const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
     const bool from_state = SLOW && t < H && p.state;
-    uint4* yrow = reinterpret_cast<uint4*>(p.y + r * p.d + n0 + cbeg);
     uint32_t va[16], vb[16];
     tmem_ld16(taddr + cbeg, va);
 #pragma unroll
@@ -462,17 +572,18 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, const uint8_t* hs, 
             o[c] = (RES ? v0 + hv[c] : v0) + sl.x;
             o[c + 1] = (RES ? v1 + hv[c + 1] : v1) + sl.y;
         }
-        if (out_row) {
-            yrow[2 * ch] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                                      pack_bf16x2(o[6], o[7]));
-            yrow[2 * ch + 1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
-                                          pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
-        }
+        // Y replaces this row's h in the staged tile (each element of the tile
+        // is read and written by one lane only); the warp stores its block
+        // with row-contiguous lanes afterwards
+        *h_chunk_ptr(hs, i, cl) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                             pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+        *h_chunk_ptr(hs, i, cl + 8) = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
+                                                 pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
     }
 }
 
 template <int BN>
-__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int mt,
+__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt,
                                                int nt, int q, int part, int lane, int et, float* s_taps) {
     constexpr int H = CONV_W - 1;
     const int i = q * 32 + lane;
@@ -510,6 +621,24 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, const uint8_t* hs
     } else {
         if (slow) vconv_chunks<BN, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
         else vconv_chunks<BN, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+    }
+    // the warp's Y block (its 32 rows x BN/NPART channels, in place of h) to
+    // global memory: LPR lanes cover one row's contiguous bytes, so each store
+    // instruction writes whole rows; the segment's history rows are skipped
+    __syncwarp();
+    constexpr int PW = BN / NPART;
+    constexpr int LPR = PW * 2 / 16;
+    constexpr int RPI = 32 / LPR;
+    const int cb = cbeg >> 6;
+    const int j = ((cbeg & 63) >> 3) + lane % LPR;
+    const int64_t seg0 = (int64_t)mt * TILE_OUT + q * SEG_OUT - H;   // global row of the segment's lane 0
+#pragma unroll
+    for (int k = 0; k < 32 / RPI; ++k) {
+        const int rr = k * RPI + lane / LPR;
+        const int ii = q * 32 + rr;
+        const uint4 v = *reinterpret_cast<const uint4*>(hs + cb * (BM * 128) + ii * 128 + ((j ^ (ii & 7)) << 4));
+        const int64_t rg = seg0 + rr;
+        if (rr >= H && rg < p.n_tok) *reinterpret_cast<uint4*>(p.y + rg * p.d + n0 + cb * 64 + j * 8) = v;
     }
 }
 
@@ -561,14 +690,27 @@ __device__ __forceinline__ void band_alpha(const EpiParams& p, int mt, int et, B
 
 // ---------------------------------------------------------------- kernel
 
-template <int MODE, int BN>
+// PAIR (cluster of two CTAs, MODE_K / MODE_VCONV): both CTAs walk the same
+// pair tiles; CTA r takes row tile 2 * mt2 + r and W channels
+// [n0 + r * BN/2, n0 + (r + 1) * BN/2).  The leader's TMA loads complete on
+// its full barrier; the peer announces its bytes on the leader's pfull
+// barrier and its TMA loads (cta_group::2 form) complete there too, so the
+// leader's warp 1 issues the M = 256 MMAs once both barriers flip and commits
+// the stage's empty barrier (and the accumulator's full barrier) in both
+// CTAs.  Each CTA's epilogue reads its own TMEM rows; the accumulator is free
+// once the 32 epilogue warps of both CTAs have arrived on the leader's tempty.
+// On an abort both CTAs stop issuing, meet at a cluster barrier, and the
+// leader drains every stage either CTA issued before both leave together.
+template <int MODE, int BN, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
                   const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_h,
                   const EpiParams p) {
-    using GE = Geo<MODE, BN>;
+    static_assert(!PAIR || MODE != MODE_KV, "the KV tile runs on one CTA");
+    using GE = Geo<MODE, BN, PAIR>;
     constexpr int STAGES = GE::STAGES;
     constexpr int STAGE_BYTES = GE::STAGE_BYTES;
+    constexpr int NCTA = PAIR ? 2 : 1;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);   // 1024-byte aligned tile base
@@ -581,15 +723,22 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int KB = p.d_mem / BK;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
+    const bool leader = rank == 0;
+    // work units: single tiles, or pair tiles shared by the two CTAs of a cluster
+    const int unit0 = (int)blockIdx.x / NCTA;
+    const int units_step = (int)gridDim.x / NCTA;
+    const int num_units = p.num_tiles;   // pair tiles when PAIR
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sb->full[s], 1);
             mbar_init(&sb->empty[s], 1);
+            mbar_init(&sb->pfull[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sb->tfull[a], 1);
-            mbar_init(&sb->tempty[a], EPI_WARPS);
+            mbar_init(&sb->tempty[a], NCTA * EPI_WARPS);
         }
         mbar_init(&sb->hfull, 1);
         mbar_init(&sb->hempty, EPI_WARPS);
@@ -599,6 +748,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         sb->consumed = 0;
         sb->h_issued = 0;
         sb->h_consumed = 0;
+        sb->peer_abort = PAIR ? peer_addr(const_cast<const int*>(&sb->abort_flag), rank ^ 1u) : 0u;
         mbar_fence_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&map_a);
@@ -607,23 +757,37 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         if (MODE == MODE_KV) tma_prefetch_desc(&map_b1);
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sb->tmem_base)),
-                     "r"(GE::TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(&sb->tmem_base)),
+                         "r"(GE::TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(&sb->tmem_base)),
+                         "r"(GE::TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // barriers of both CTAs initialised before any remote arrival
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = sb->tmem_base;
 
+    // row tile of this CTA for unit u; channel tile
+    auto unit_mt = [&](int u) { return PAIR ? 2 * (u / p.n_groups) + (int)rank : u / p.n_groups; };
+    auto unit_nt = [&](int u) { return u % p.n_groups; };
+
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- TMA producer (each CTA loads its own rows and W half)
         if (lane == 0) {
             int it = 0, tc = 0;
             const uint32_t h_dst = smem_u32(s_h);
-            for (int tile = blockIdx.x; tile < p.num_tiles && !sb->abort_flag; tile += gridDim.x, ++tc) {
-                const int mt = tile / p.n_groups, nt = tile % p.n_groups;
+            for (int u = unit0; u < num_units && !sb->abort_flag; u += units_step, ++tc) {
+                const int mt = unit_mt(u), nt = unit_nt(u);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % STAGES;
@@ -634,21 +798,28 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     }
                     const uint32_t a_dst = tiles_u32 + s * STAGE_BYTES;
                     const uint32_t b_dst = a_dst + A_BYTES;
-                    mbar_arrive_expect_tx(&sb->full[s], STAGE_BYTES);
+                    // the leader counts its stage on full[s]; the peer on the leader's pfull[s]
+                    const bool remote = PAIR && !leader;
+                    const uint32_t bar = remote ? peer_addr(&sb->pfull[s], 0u) : smem_u32(&sb->full[s]);
+                    auto load = [&](const CUtensorMap* m, uint32_t dst, int x, int y) {
+                        if (remote) tma_load_2d_peer_bar(m, dst, bar, x, y);
+                        else tma_load_2d(m, dst, &sb->full[s], x, y);
+                    };
+                    if (remote) mbar_arrive_expect_tx_remote(bar, STAGE_BYTES);
+                    else mbar_arrive_expect_tx(&sb->full[s], STAGE_BYTES);
                     if (MODE == MODE_VCONV) {
                         // four 32-row segments, each starting 3 rows before its outputs
 #pragma unroll
                         for (int sg = 0; sg < 4; ++sg)
-                            tma_load_2d(&map_a, a_dst + sg * (SEG * 128), &sb->full[s], kb * BK,
-                                        mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                            load(&map_a, a_dst + sg * (SEG * 128), kb * BK, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
                     } else {
-                        tma_load_2d(&map_a, a_dst, &sb->full[s], kb * BK, mt * BM);
+                        load(&map_a, a_dst, kb * BK, mt * BM);
                     }
                     if (MODE == MODE_KV) {
-                        tma_load_2d(&map_b0, b_dst, &sb->full[s], kb * BK, nt * 128);
-                        tma_load_2d(&map_b1, b_dst + 128 * BK * 2, &sb->full[s], kb * BK, nt * 128);
+                        load(&map_b0, b_dst, kb * BK, nt * 128);
+                        load(&map_b1, b_dst + 128 * BK * 2, kb * BK, nt * 128);
                     } else {
-                        tma_load_2d(&map_b0, b_dst, &sb->full[s], kb * BK, nt * BN);
+                        load(&map_b0, b_dst, kb * BK, nt * BN + (int)rank * GE::B_ROWS);
                     }
                     sb->issued = it + 1;
                 }
@@ -671,11 +842,11 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 sb->h_issued = tc + 1;
             }
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer
+    } else if (warp == 1 && (!PAIR || leader)) {
+        // ---------------- MMA issuer (the leader of a pair)
         if (lane == 0) {
             int it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !sb->abort_flag; tile += gridDim.x, ++tc) {
+            for (int u = unit0; u < num_units && !sb->abort_flag; u += units_step, ++tc) {
                 const int acc = tc & 1;
                 const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
                 if (!wait_bounded(&sb->tempty[acc], aph ^ 1u, sb, p.status)) break;
@@ -685,7 +856,8 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!wait_bounded(&sb->full[s], ph, sb, p.status)) {
+                    if (!wait_bounded(&sb->full[s], ph, sb, p.status) ||
+                        (PAIR && !wait_bounded(&sb->pfull[s], ph, sb, p.status))) {
                         ok = false;
                         break;
                     }
@@ -696,13 +868,18 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
                         // +32 bytes along K inside the swizzled 128-byte row
-                        umma_bf16<BN>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
+                        if constexpr (PAIR)
+                            umma_bf16_pair<BN>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
+                        else
+                            umma_bf16<BN>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
                     }
-                    umma_commit(&sb->empty[s]);
+                    if constexpr (PAIR) umma_commit_pair_both(&sb->empty[s]);
+                    else umma_commit(&sb->empty[s]);
                     sb->consumed = it + 1;
                 }
                 if (!ok) break;
-                umma_commit(&sb->tfull[acc]);
+                if constexpr (PAIR) umma_commit_pair_both(&sb->tfull[acc]);
+                else umma_commit(&sb->tfull[acc]);
             }
         }
     } else if (warp >= 4) {
@@ -711,26 +888,31 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         const int q = warp & 3;
         const int part = (warp - 4) >> 2;
         const int et = threadIdx.x - 128;    // 0 .. EPI_THREADS-1
+        const uint32_t tempty_leader0 = PAIR ? peer_addr(&sb->tempty[0], 0u) : 0u;
+        const uint32_t tempty_leader1 = PAIR ? peer_addr(&sb->tempty[1], 0u) : 0u;
         int tc = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tc) {
+        for (int u = unit0; u < num_units; u += units_step, ++tc) {
             const int acc = tc & 1;
             const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
             bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
             ok = ok && wait_bounded(&sb->hfull, (uint32_t)tc & 1u, sb, p.status);
             if (epi_any(!ok)) break;          // one decision for all epilogue warps
             tc_fence_after();
-            const int mt = tile / p.n_groups, nt = tile % p.n_groups;
+            const int mt = unit_mt(u), nt = unit_nt(u);
             const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+            // the odd CTA of the last pair may hold a row tile past the end
+            const bool rows_live = MODE == MODE_VCONV ? (int64_t)mt * TILE_OUT < p.n_tok : (int64_t)mt * BM < p.n_tok;
             if (MODE == MODE_KV) epilogue_kv(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
-            if (MODE == MODE_K) {
+            if (MODE == MODE_K && rows_live) {
                 epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
                 band_alpha(p, mt, et, sb, reinterpret_cast<float4*>(s_h), GE::H_BYTES);
             }
-            if (MODE == MODE_VCONV) epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg);
+            if (MODE == MODE_VCONV && rows_live) epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&sb->tempty[acc]);
+                if (PAIR && !leader) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+                else mbar_arrive(&sb->tempty[acc]);
                 mbar_arrive(&sb->hempty);
             }
             if (threadIdx.x == 128) sb->h_consumed = tc + 1;
@@ -738,14 +920,34 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     }
 
     __syncthreads();
-    if (sb->abort_flag) {
-        // drain: copies this CTA issued but nobody consumed, then the MMAs
+    // a pair decides together: both CTAs have stopped issuing once they meet here
+    bool aborted = sb->abort_flag != 0;
+    if constexpr (PAIR) {
+        cluster_sync_all();
+        aborted = aborted || ld_remote_s32(sb->peer_abort) != 0;
+    }
+    if (aborted) {
+        // drain: copies issued but not consumed (for a pair, the leader also
+        // waits out the peer's stages, which complete on its pfull), the h
+        // tiles, then the MMAs
         if (warp == 0 && lane == 0) {
-            for (int it = sb->consumed; it < sb->issued; ++it) {
-                const int s = it % STAGES;
-                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                const long long t0 = clock64();
-                while (!mbar_try_wait(smem_u32(&sb->full[s]), ph) && clock64() - t0 < kWaitCycles) {
+            if (!PAIR || leader) {
+                for (int it = sb->consumed; it < sb->issued; ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(smem_u32(&sb->full[s]), ph) && clock64() - t0 < kWaitCycles) {
+                    }
+                }
+            }
+            if (PAIR && leader) {
+                const int peer_issued = ld_remote_s32(peer_addr(&sb->issued, 1u));
+                for (int it = sb->consumed; it < peer_issued; ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(smem_u32(&sb->pfull[s]), ph) && clock64() - t0 < kWaitCycles) {
+                    }
                 }
             }
             for (int k = sb->h_consumed; k < sb->h_issued; ++k) {
@@ -754,18 +956,25 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 }
             }
         }
-        if (warp == 1 && lane == 0) {
-            umma_commit(&sb->drain);
+        if (warp == 1 && lane == 0 && (!PAIR || leader)) {
+            if constexpr (PAIR) umma_commit_pair_local(&sb->drain);
+            else umma_commit(&sb->drain);
             const long long t0 = clock64();
             while (!mbar_try_wait(smem_u32(&sb->drain), 0) && clock64() - t0 < kWaitCycles) {
             }
         }
         __syncthreads();
     }
+    // a pair leaves together: no remote arrival may reach a CTA that has exited
+    if constexpr (PAIR) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GE::TMEM_COLS)
-                     : "memory");
+        if constexpr (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GE::TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(GE::TMEM_COLS)
+                         : "memory");
     }
 }
 
@@ -818,28 +1027,67 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const CUtensorMap& mh,
                         EpiParams p, int64_t m_tiles, int num_sms, cudaStream_t s) {
-    using GE = Geo<MODE, BN>;
+    using GE = Geo<MODE, BN, PAIR>;
+    auto kernel = project_tc_kernel<MODE, BN, PAIR>;
     static unsigned long long attr_set = 0;   // one bit per device ordinal
+    static int max_clusters[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !(attr_set >> dev & 1ull)) {
-        cudaError_t err = cudaFuncSetAttribute(project_tc_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               GE::SMEM_BYTES);
+        cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GE::SMEM_BYTES);
         if (err != cudaSuccess) return err;
+        if (PAIR) {
+            err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+            (void)err;
+        }
         attr_set |= 1ull << dev;
     }
-    const int64_t tiles = m_tiles * p.n_groups;
-    if (tiles >= (int64_t)1 << 31) return cudaErrorInvalidValue;
-    p.num_tiles = (int)tiles;
-    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    project_tc_kernel<MODE, BN><<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, mh, p);
-    return cudaGetLastError();
+    const int64_t units = (PAIR ? (m_tiles + 1) / 2 : m_tiles) * p.n_groups;
+    if (units >= (int64_t)1 << 31) return cudaErrorInvalidValue;
+    p.num_tiles = (int)units;
+    if (!PAIR) {
+        const int grid = (int)(units < num_sms ? units : num_sms);
+        kernel<<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, mh, p);
+        return cudaGetLastError();
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = GE::SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (dev < 64 && max_clusters[dev] == 0) {
+        cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
+        int mc = 0;
+        if (cudaOccupancyMaxActiveClusters(&mc, kernel, &cfg) != cudaSuccess || mc < 1) {
+            cudaGetLastError();
+            mc = num_sms / 2;
+        }
+        max_clusters[dev] = mc;
+    }
+    const int64_t cap = dev < 64 ? max_clusters[dev] : num_sms / 2;
+    const int64_t clusters = units < cap ? units : cap;
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb0, mb1, mh, p);
 }
 
 int pick_bn(int32_t d) { return d % 256 == 0 ? 256 : 128; }
+
+// CTA pairs once there are enough row tiles to give every SM pair work
+bool use_pair(int64_t m_tiles, int n_groups, int num_sms) { return m_tiles * n_groups >= 2 * (int64_t)num_sms; }
+
+// The value pass is bound by its epilogue, not by the operand feed, and a
+// pair couples the two CTAs' epilogues through the shared accumulator: on
+// B200 it ran 136 us against 111 us single (c2).  It stays on single CTAs.
+bool use_pair_vconv(int64_t, int, int) { return false; }
 
 }  // namespace
 
@@ -867,7 +1115,7 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
     p.d = d;
     p.G = d / 128;
     p.n_groups = d / 128;
-    return launch_mode<MODE_KV, 256>(ma, mk, mv, mh, p, (n_tok + BM - 1) / BM, num_sms, s);
+    return launch_mode<MODE_KV, 256, false>(ma, mk, mv, mh, p, (n_tok + BM - 1) / BM, num_sms, s);
 }
 
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
@@ -894,8 +1142,13 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     p.G = d / 128;
     p.n_groups = d / bn;
     const int64_t mt = (n_tok + BM - 1) / BM;
-    return bn == 256 ? launch_mode<MODE_K, 256>(ma, mk, mk, mh, p, mt, num_sms, s)
-                     : launch_mode<MODE_K, 128>(ma, mk, mk, mh, p, mt, num_sms, s);
+    if (bn == 256 && use_pair(mt, p.n_groups, num_sms)) {
+        CUtensorMap mk2;
+        if (!make_map(&mk2, Wk, (uint64_t)d, (uint64_t)d_mem, 128)) return cudaErrorInvalidValue;
+        return launch_mode<MODE_K, 256, true>(ma, mk2, mk2, mh, p, mt, num_sms, s);
+    }
+    return bn == 256 ? launch_mode<MODE_K, 256, false>(ma, mk, mk, mh, p, mt, num_sms, s)
+                     : launch_mode<MODE_K, 128, false>(ma, mk, mk, mh, p, mt, num_sms, s);
 }
 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
@@ -924,8 +1177,13 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     p.L = L;
     p.add_residual = add_residual;
     const int64_t mt = (n_tok + TILE_OUT - 1) / TILE_OUT;
-    return bn == 256 ? launch_mode<MODE_VCONV, 256>(ma, mv, mv, mh, p, mt, num_sms, s)
-                     : launch_mode<MODE_VCONV, 128>(ma, mv, mv, mh, p, mt, num_sms, s);
+    if (bn == 256 && use_pair_vconv(mt, p.n_groups, num_sms)) {
+        CUtensorMap mv2;
+        if (!make_map(&mv2, Wv, (uint64_t)d, (uint64_t)d_mem, 128)) return cudaErrorInvalidValue;
+        return launch_mode<MODE_VCONV, 256, true>(ma, mv2, mv2, mh, p, mt, num_sms, s);
+    }
+    return bn == 256 ? launch_mode<MODE_VCONV, 256, false>(ma, mv, mv, mh, p, mt, num_sms, s)
+                     : launch_mode<MODE_VCONV, 128, false>(ma, mv, mv, mh, p, mt, num_sms, s);
 }
 
 cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,

@@ -31,6 +31,8 @@ SMALL = {
     "b3": W["c2"].replace(name="b3", B=2, T=333, M=10007, d=512, seed=14),
     # bf16 tensor-core projection with conv width 3 (unfused: CUDA-core gate/conv), d = 384
     "b4": W["c1"].replace(name="b4", B=3, T=150, K=2, D=64, d=384, w=3, dtype="bf16", seed=15),
+    # fused passes with 128-channel tiles (d = 384 is not a multiple of 256), ragged rows
+    "b5": W["c1"].replace(name="b5", B=2, T=237, K=4, D=64, d=384, w=4, dtype="bf16", seed=16),
 }
 
 
@@ -198,6 +200,37 @@ def test_forward_full_size_sampled(eb, name):
     assert np.array_equal(idx.cpu().numpy().view(np.uint32), idx_ref)
     pos = synth.sample_positions(wl, 96, seed=5)
     ref = oracle.forward_rows(inp, pos, add_residual=True, idx=idx_ref)
+    sel = torch.from_numpy(pos).cuda()
+    np.testing.assert_allclose(to_np(alpha[sel]), ref.alpha, rtol=0, atol=2e-6)
+    _check_y(wl, to_np(y[sel]), ref.y, ref.vt_win, inp.conv_w)
+
+
+# CTA-pair tiling (two CTAs per M = 256 MMA) engages once there are enough row
+# tiles to occupy every SM pair; these shapes reach it with ragged ends: an odd
+# number of value row tiles leaves the second CTA of the last pair without rows
+PAIR_CASES = {
+    "pair_a": W["c2"].replace(name="pair_a", B=2, T=2000, M=10007, seed=31),       # 4000 rows, 35 value tiles
+    "pair_b": W["c2"].replace(name="pair_b", B=3, T=1501, M=10007, seed=32),       # 4503 rows, ragged 128-row band
+}
+
+
+@pytest.mark.parametrize("name", sorted(PAIR_CASES))
+def test_cta_pair_tiling_sampled(eb, name):
+    wl = PAIR_CASES[name]
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    y, alpha = _run_forward(eb, ctx, di, add_residual=True)
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    # rows around every 116-row value tile edge and 128-row band edge, the
+    # sequence ends, and random rows
+    edges = set()
+    for base in list(range(0, wl.n_tok, 116)) + list(range(0, wl.n_tok, 128)):
+        for r in (base - 4, base - 1, base, base + 3):
+            if 0 <= r < wl.n_tok:
+                edges.add(r)
+    pos = np.array(sorted(edges | set(synth.sample_positions(wl, 64, seed=7).tolist())), dtype=np.int64)
+    ref = oracle.forward_rows(inp, pos, add_residual=True)
     sel = torch.from_numpy(pos).cuda()
     np.testing.assert_allclose(to_np(alpha[sel]), ref.alpha, rtol=0, atol=2e-6)
     _check_y(wl, to_np(y[sel]), ref.y, ref.vt_win, inp.conv_w)
