@@ -169,15 +169,12 @@ CSRC = os.path.join(ROOT, "hashed_gram_embedding_02_b200", "csrc")
 KERNEL_SOURCES = {
     "gate_k_tc": ("project_tc.cu", "common.cuh", "ptx.cuh"),
     "vconv_tc": ("project_tc.cu", "common.cuh", "ptx.cuh"),
-    "gather": ("gather.cu", "common.cuh"),
-    "hash": ("hash.cu", "common.cuh"),
+    "retrieve": ("retrieve.cu", "common.cuh"),
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
     ("c2", "vconv_tc"): ("c53c7049c3cf0f12", 123025920 + 47182848),
     ("c2", "gate_k_tc"): ("c53c7049c3cf0f12", 122742784 + 5212672),
-    ("c2", "gather"): ("71fc7b1a17174b45", 29688064 + 563456),
-    ("c2", "hash"): ("990ca7387ce2f5f1", 296704 + 0),
 }
 
 
@@ -498,8 +495,9 @@ def main():
     pass_flops = 2.0 * n * wl.d_mem * wl.d                      # one of the two projection passes
     work = {
         # name: (bound, algorithmic units per launch, unit)
-        "hash": ("hbm", n * (4.0 + wl.J * 4) + wl.B * 4.0 * min(wl.T, 3), "bytes"),
-        "gather": ("hbm", n * wl.J * 4 + 2.0 * n * wl.d_mem * es, "bytes"),
+        # remap + n-grams + hash + gather in one kernel: ids in, indices out,
+        # table rows in, e_cat out
+        "retrieve": ("hbm", n * (4.0 + wl.J * 4) + wl.B * 4.0 * min(wl.T, 3) + 2.0 * n * wl.d_mem * es, "bytes"),
         "gate_k_tc": ("tensor", pass_flops, "flop"),
         "vconv_tc": ("tensor", pass_flops, "flop"),
         "state_merge": ("hbm", wl.B * (wl.w - 1) * wl.d * 8.0, "bytes"),
@@ -524,8 +522,8 @@ def main():
                 "peak_source": f"{peak_src} " + ("bf16 burst" if dk.get("bound") == "tensor" else "HBM copy"),
                 "algorithmic": (f"2*n*d_mem*d = {pass_flops:.4g} FLOP per launch" if dk.get("bound") == "tensor"
                                 else f"{work.get(dominant, (0, 0))[1]:.4g} bytes per launch")}
-    gather_gbs = kern["gather"]["achieved"] if "gather" in kern else None
-    gather_bytes = work["gather"][1]
+    gather_gbs = kern["retrieve"]["achieved"] if "retrieve" in kern else None
+    gather_bytes = work["retrieve"][1]
 
     # ---- end to end through the C ABI with HOST buffers: engram_forward_host
     # copies the ids and h in from pinned host memory and Y back out, chunk by
@@ -574,8 +572,9 @@ def main():
                    "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write outside the events)"},
         "roofline": roofline,
-        "gather": {"achieved_gbs": gather_gbs, "frac_of_8000": gather_gbs / SPEC_HBM_GBS,
-                   "frac_of_measured": gather_gbs / hbm, "bytes_per_launch": gather_bytes},
+        "gather": {"kernel": "retrieve (remap + n-grams + hash + gather)", "achieved_gbs": gather_gbs,
+                   "frac_of_8000": gather_gbs / SPEC_HBM_GBS, "frac_of_measured": gather_gbs / hbm,
+                   "bytes_per_launch": gather_bytes},
         "kernels": kern, "kernels_ms": kms,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": per_step_launches * K, "clocks": clocks.summary(),
     }

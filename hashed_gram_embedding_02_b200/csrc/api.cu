@@ -179,15 +179,10 @@ engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t
                            const void* Wv, const float* gq, const float* gk, const float* conv_w, float* conv_state,
                            void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s) {
     const int32_t L = T - t_begin;
-    const int64_t n = (int64_t)B * L;
-    prof_begin(c, s, "hash");
-    cudaError_t e = launch_hash(tok, P, B, T, tok_stride, t_begin, w.idx, c->hp, c->d_status, s);
+    prof_begin(c, s, "retrieve");
+    cudaError_t e = launch_retrieve(tok, P, B, T, tok_stride, t_begin, c->hp, c->gp, tables, w.idx, w.e, c->d_status, s);
     prof_end(c, s);
-    if (e != cudaSuccess) return cuda_fail("hash launch", e);
-    prof_begin(c, s, "gather");
-    e = launch_gather(w.idx, n, tables, c->gp, w.e, c->d_status, c->num_sms, s);
-    prof_end(c, s);
-    if (e != cudaSuccess) return cuda_fail("gather launch", e);
+    if (e != cudaSuccess) return cuda_fail("retrieve (hash + gather) launch", e);
     return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
 }
 
@@ -260,6 +255,7 @@ engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
     for (int j = 0; j < J; ++j) {
         for (int q = 0; q < 4; ++q) c->hp.mult[j][q] = k.mult[j][q];
         c->hp.rows[j] = k.rows[j];
+        c->hp.recip[j] = ~(uint64_t)0 / k.rows[j];
     }
     for (int o = 0; o < 4; ++o) c->hp.orders[o] = o < k.n_orders ? k.orders[o] : 0;
     c->hp.n_orders = k.n_orders;

@@ -17,6 +17,7 @@ constexpr int kMaxConv = 8;
 // kernel parameters; dynamic indexing reads the constant bank).
 struct HashParams {
     uint64_t mult[kMaxTables][4];
+    uint64_t recip[kMaxTables];   // floor((2^64 - 1) / rows[j]) for the Barrett reduction
     uint32_t rows[kMaxTables];
     int32_t orders[4];
     int32_t n_orders;
@@ -35,6 +36,17 @@ struct GatherParams {
     int32_t chunks_per_row;        // 16-byte chunks per table row
 };
 
+// x mod m for a 64-bit x and a 32-bit m, by Barrett's reduction (P. Barrett,
+// CRYPTO '86) with recip = floor((2^64 - 1) / m): q = floor(x * recip / 2^64)
+// undershoots floor(x / m) by at most 2, so at most two subtractions follow.
+__device__ __forceinline__ uint32_t mod_u64(uint64_t x, uint32_t m, uint64_t recip) {
+    const uint64_t q = __umul64hi(x, recip);
+    uint64_t r = x - q * (uint64_t)m;
+    if (r >= m) r -= m;
+    if (r >= m) r -= m;
+    return (uint32_t)r;
+}
+
 // ---------------------------------------------------------------- launches
 // Each returns cudaGetLastError() of its launch.
 cudaError_t launch_remap(const int32_t* tok, int64_t n, const int32_t* P, int32_t V, int32_t* canon,
@@ -44,6 +56,10 @@ cudaError_t launch_hash(const int32_t* ids, const int32_t* P, int32_t B, int32_t
                         cudaStream_t s);
 cudaError_t launch_gather(const uint32_t* idx, int64_t n_tok, const void* tables, const GatherParams& gp,
                           void* e_cat, uint32_t* status, int num_sms, cudaStream_t s);
+// launch_hash followed by launch_gather in one kernel (indices still written to idx)
+cudaError_t launch_retrieve(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
+                            int32_t t_begin, const HashParams& hp, const GatherParams& gp, const void* tables,
+                            uint32_t* idx, void* e_cat, uint32_t* status, cudaStream_t s);
 // CUDA-core projection (fp32 or bf16 operands, fp32 accumulation); v in fp32
 cudaError_t launch_project_simt(bool bf16, const void* e, int64_t n_tok, int32_t d_mem, const void* h,
                                 const void* Wk, const void* Wv, const float* gq, const float* gk, int32_t d,

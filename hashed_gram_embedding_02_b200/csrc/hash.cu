@@ -72,7 +72,7 @@ hash_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, int3
             invalid |= (sj < 0);
             x ^= (uint64_t)(uint32_t)(sj + 1) * hp.mult[jt][j];
         }
-        idx[(row0 + rr) * J + jt] = invalid ? ENGRAM_INVALID_INDEX : (uint32_t)(x % (uint64_t)hp.rows[jt]);
+        idx[(row0 + rr) * J + jt] = invalid ? ENGRAM_INVALID_INDEX : mod_u64(x, hp.rows[jt], hp.recip[jt]);
     }
 }
 

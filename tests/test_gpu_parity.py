@@ -129,6 +129,29 @@ def test_hash_strided_context_and_t_begin(eb):
         assert np.array_equal(idx.cpu().numpy().view(np.uint32), ref), t_begin
 
 
+def test_hash_extreme_primes(eb):
+    """The device reduction of the 64-bit hash modulo each table size, at the
+    smallest primes and at the largest allowed one (2^31 - 1), against the
+    oracle's plain remainder, on ids drawn over the whole canonical range."""
+    wl = W["c2"].replace(name="primes", B=3, T=2000, seed=41)
+    inp = synth.Inputs(wl)
+    rows = np.array([2, 3, 5, 2147483647, 2147483629, 1000003, 65521, 7919,
+                     2, 3, 2147483647, 999983, 7, 11, 13, 2147483587], dtype=np.int64)
+    assert all(synth._is_prime(int(r)) for r in rows)
+    cfg = eb.make_config(orders=wl.orders, heads=wl.K, rows=[int(x) for x in rows], mult=inp.mult, row_dim=wl.D,
+                         hidden=wl.d, conv_width=wl.w, vocab=wl.V, canon_vocab=wl.Vc, dtype=eb.ENGRAM_BF16)
+    ctx = eb.Engram(cfg)
+    rng = np.random.default_rng(5)
+    inp.tok[:] = rng.integers(0, wl.V, size=inp.tok.shape)      # uniform ids: every bit of the products varies
+    canon_ref, _ = oracle.remap(inp.tok, inp.P)
+    ref, _ = oracle.hash_ids(canon_ref, wl.Vc, wl.orders, wl.K, inp.mult, rows.astype(np.uint32))
+    idx = torch.empty(wl.n_tok, wl.J, dtype=torch.int32, device="cuda")
+    eb.engram_hash(ctx.ctx, torch.from_numpy(inp.tok).cuda(), torch.from_numpy(inp.P).cuda(), wl.B, wl.T, wl.T, 0,
+                   idx)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy().view(np.uint32), ref)
+
+
 @pytest.mark.parametrize("name", ["c1", "b2", "c2"])
 def test_gather_bitexact(eb, name):
     wl = SMALL.get(name) or W[name]
