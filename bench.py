@@ -173,8 +173,9 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("c53c7049c3cf0f12", 123025920 + 47182848),
-    ("c2", "gate_k_tc"): ("c53c7049c3cf0f12", 122742784 + 5212672),
+    ("c2", "vconv_tc"): ("42410853cdb27c94", 123009280 + 50473728),
+    ("c2", "gate_k_tc"): ("42410853cdb27c94", 122741760 + 5350400),
+    ("c2", "retrieve"): ("917d9ef9fd4eee03", 28935424 + 470016),
 }
 
 

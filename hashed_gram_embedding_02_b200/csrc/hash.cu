@@ -42,6 +42,18 @@ hash_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, int3
             int64_t stride, int32_t t_begin, uint32_t* __restrict__ idx, const HashParams hp, int rows_per_cta,
             uint32_t* status) {
     __shared__ int32_t s_win[kHashThreads][4];   // [row][j]: canonical id at t - j (PAD before the start)
+    // per-table constants in shared memory (lanes index them by table; divergent
+    // indexing of kernel parameters would serialise on the constant cache)
+    __shared__ uint64_t s_mult[kMaxTables][4];
+    __shared__ uint64_t s_recip[kMaxTables];
+    __shared__ uint32_t s_rows[kMaxTables];
+    __shared__ int32_t s_order[kMaxTables];
+    for (int k = threadIdx.x; k < hp.J * 4; k += kHashThreads) s_mult[k >> 2][k & 3] = hp.mult[k >> 2][k & 3];
+    for (int k = threadIdx.x; k < hp.J; k += kHashThreads) {
+        s_recip[k] = hp.recip[k];
+        s_rows[k] = hp.rows[k];
+        s_order[k] = hp.orders[k / hp.K];
+    }
     const int64_t L = (int64_t)T - t_begin;
     const int64_t n = (int64_t)B * L;
     const int64_t row0 = (int64_t)blockIdx.x * rows_per_cta;
@@ -63,16 +75,15 @@ hash_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, int3
     const int J = hp.J;
     for (int k = threadIdx.x; k < R * J; k += kHashThreads) {
         const int rr = k / J, jt = k - rr * J;
-        const int o = jt / hp.K;
-        const int n_o = hp.orders[o];
+        const int n_o = s_order[jt];
         bool invalid = false;
         uint64_t x = 0;
         for (int j = 0; j < n_o; ++j) {
             const int32_t sj = s_win[rr][j];
             invalid |= (sj < 0);
-            x ^= (uint64_t)(uint32_t)(sj + 1) * hp.mult[jt][j];
+            x ^= (uint64_t)(uint32_t)(sj + 1) * s_mult[jt][j];
         }
-        idx[(row0 + rr) * J + jt] = invalid ? ENGRAM_INVALID_INDEX : mod_u64(x, hp.rows[jt], hp.recip[jt]);
+        idx[(row0 + rr) * J + jt] = invalid ? ENGRAM_INVALID_INDEX : mod_u64(x, s_rows[jt], s_recip[jt]);
     }
 }
 

@@ -46,12 +46,27 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
                 uint32_t* status) {
     __shared__ int32_t s_win[kThreads][4];
     __shared__ uint32_t s_idx[kThreads];
+    // per-table constants in shared memory: lanes index them by table, and
+    // divergent indexing of kernel parameters would serialise on the
+    // constant cache
+    __shared__ uint64_t s_mult[kMaxTables][4];
+    __shared__ uint64_t s_recip[kMaxTables];
+    __shared__ int64_t s_off[kMaxTables];
+    __shared__ uint32_t s_rows[kMaxTables];
+    __shared__ int32_t s_order[kMaxTables];
     const int64_t L = (int64_t)T - t_begin;
     const int64_t n = (int64_t)B * L;
     const int64_t row0 = (int64_t)blockIdx.x * rows_per_cta;
     const int R = (int)min((int64_t)rows_per_cta, n - row0);
     const int W = hp.max_order;
     const int J = hp.J;
+    for (int k = threadIdx.x; k < J * 4; k += kThreads) s_mult[k >> 2][k & 3] = hp.mult[k >> 2][k & 3];
+    for (int k = threadIdx.x; k < J; k += kThreads) {
+        s_recip[k] = hp.recip[k];
+        s_off[k] = gp.row_off[k];
+        s_rows[k] = hp.rows[k];
+        s_order[k] = hp.orders[k / hp.K];
+    }
 
     // 1. n-gram windows (PAD before the sequence start)
     for (int k = threadIdx.x; k < R * W; k += kThreads) {
@@ -66,15 +81,15 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
     // 2. hash heads, one (row, table) pair per thread
     for (int k = threadIdx.x; k < R * J; k += kThreads) {
         const int rr = k / J, jt = k - rr * J;
-        const int n_o = hp.orders[jt / hp.K];
+        const int n_o = s_order[jt];
         bool invalid = false;
         uint64_t x = 0;
         for (int j = 0; j < n_o; ++j) {
             const int32_t sj = s_win[rr][j];
             invalid |= (sj < 0);
-            x ^= (uint64_t)(uint32_t)(sj + 1) * hp.mult[jt][j];
+            x ^= (uint64_t)(uint32_t)(sj + 1) * s_mult[jt][j];
         }
-        const uint32_t v = invalid ? ENGRAM_INVALID_INDEX : mod_u64(x, hp.rows[jt], hp.recip[jt]);
+        const uint32_t v = invalid ? ENGRAM_INVALID_INDEX : mod_u64(x, s_rows[jt], s_recip[jt]);
         s_idx[k] = v;
         idx[(row0 + rr) * J + jt] = v;
     }
@@ -98,7 +113,7 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
                 const int jt = cpr_shift >= 0 ? rem >> cpr_shift : rem / cpr;
                 const int c = rem - jt * cpr;
                 const uint32_t r = s_idx[rr * J + jt];
-                if (r < gp.rows[jt]) v[u] = __ldg(tables + (gp.row_off[jt] + r) * cpr + c);
+                if (r < s_rows[jt]) v[u] = __ldg(tables + (s_off[jt] + r) * cpr + c);
                 else if (r != ENGRAM_INVALID_INDEX) flag(status, ENGRAM_ERR_INDEX);
             }
         }
