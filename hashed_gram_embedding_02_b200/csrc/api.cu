@@ -63,6 +63,12 @@ bool tc_path(const engram_ctx* c, int64_t n) {
 // projections with the gate and the conv fused into the epilogue (conv width 4)
 bool fused_path(const engram_ctx* c, int64_t n) { return tc_path(c, n) && c->cfg.conv_width == 4; }
 
+// Decode-shaped calls (a few positions per sequence) hand the fused value pass
+// the conv history in the sequence-minor layout [w-1][d][B]: consecutive lanes
+// then read consecutive sequences' history instead of rows d floats apart.
+constexpr int32_t kDecodeRows = 8;
+bool decode_shaped(const engram_ctx* c, int64_t n, int64_t L) { return fused_path(c, n) && L <= kDecodeRows; }
+
 // per-128-row-band counters of the key pass
 size_t band_bytes(int64_t n) { return (size_t)((n + 127) / 128) * sizeof(int); }
 
@@ -82,8 +88,13 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
     p += align256((size_t)n * sizeof(float));
     w.band = reinterpret_cast<int*>(p);
     p += align256(band_bytes(n));
+    const size_t hist_bytes = align256((size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
     w.state_next = reinterpret_cast<float*>(p);
-    p += align256((size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
+    p += hist_bytes;
+    if (decode_shaped(c, n, L)) {
+        w.state_t = reinterpret_cast<float*>(p);
+        p += hist_bytes;
+    }
     if (!fused_path(c, n)) {
         w.v = reinterpret_cast<float*>(p);
         p += align256((size_t)n * c->cfg.hidden * sizeof(float));
@@ -149,14 +160,23 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
                              alpha_out, c->d_status, c->num_sms, s);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
+        const bool tr = state && decode_shaped(c, n, L);
+        if (tr) {
+            prof_begin(c, s, "state_to_tr");
+            e = launch_state_to_tr(state, w.state_t, B, c->cfg.conv_width, c->cfg.hidden, s);
+            prof_end(c, s);
+            if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
+        }
         prof_begin(c, s, "vconv_tc");
-        e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha, state,
-                            w.state_next, y, add_residual, c->d_status, c->num_sms, s);
+        e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha,
+                            tr ? w.state_t : state, w.state_next, tr ? 1 : 0, y, add_residual, c->d_status,
+                            c->num_sms, s);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 value/conv launch", e);
         if (state) {
             prof_begin(c, s, "state_merge");
-            e = launch_state_merge(state, w.state_next, B, L, c->cfg.conv_width, c->cfg.hidden, c->num_sms, s);
+            e = tr ? launch_state_merge_tr(state, w.state_next, B, L, c->cfg.conv_width, c->cfg.hidden, s)
+                   : launch_state_merge(state, w.state_next, B, L, c->cfg.conv_width, c->cfg.hidden, c->num_sms, s);
             prof_end(c, s);
             if (e != cudaSuccess) return cuda_fail("conv-state merge launch", e);
         }

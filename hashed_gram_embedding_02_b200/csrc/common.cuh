@@ -82,8 +82,14 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
 // state afterwards.
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
-                            float* state_next, void* y, int32_t add_residual, uint32_t* status, int num_sms,
-                            cudaStream_t s);
+                            float* state_next, int32_t state_tr, void* y, int32_t add_residual, uint32_t* status,
+                            int num_sms, cudaStream_t s);
+// conv history [B][w-1][d] -> the sequence-minor [w-1][d][B] that decode-shaped
+// value passes read (state_tr), and the merge of such a pass's new history
+// back into the caller's [B][w-1][d]
+cudaError_t launch_state_to_tr(const float* state, float* state_t, int32_t B, int32_t w, int32_t d, cudaStream_t s);
+cudaError_t launch_state_merge_tr(float* state, const float* state_next_t, int32_t B, int32_t L, int32_t w, int32_t d,
+                                  cudaStream_t s);
 cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,
                                int num_sms, cudaStream_t s);
 // gate + conv from an fp32 v (CUDA cores)

@@ -55,8 +55,9 @@ engram_status check_device(const engram_ctx* c);
 
 // Scratch of one forward over B sequences of L computed rows:
 // idx [n][J] u32 | e [n][J*D] | part [n][G][4] f32 | alpha [n] f32 | band
-// counters | state_next [B][w-1][d] f32 | v [n][d] f32 (unfused paths only),
-// each 256-byte aligned.  With base == nullptr only `bytes` is meaningful.
+// counters | state_next [B][w-1][d] f32 | state_t [w-1][d][B] f32 (fused
+// decode-shaped calls, L <= 8) | v [n][d] f32 (unfused paths only), each
+// 256-byte aligned.  With base == nullptr only `bytes` is meaningful.
 struct Workspace {
     uint32_t* idx;
     void* e;
@@ -64,6 +65,7 @@ struct Workspace {
     float* alpha;
     int* band;
     float* state_next;
+    float* state_t;     // decode-shaped fused calls: the history, sequence-minor
     float* v;
     size_t bytes;
 };

@@ -95,6 +95,8 @@ struct __align__(8) Barriers {
     uint64_t tempty[2];
     uint64_t hfull;
     uint64_t hempty;
+    uint64_t hfull_v[2];    // MODE_VCONV: the two channel halves of the tile's h slice
+    uint64_t hempty_v[2];
     uint64_t drain;
     uint32_t tmem_base;
     volatile int abort_flag;
@@ -103,6 +105,8 @@ struct __align__(8) Barriers {
     int h_issued;     // h tiles issued
     int h_consumed;   // h tiles released by the epilogue
     int band_last;    // this CTA completed a row band's partials (MODE_K)
+    int h_issued_v[2];      // MODE_VCONV: h halves issued / released, per half
+    int h_consumed_v[2];
     uint32_t peer_abort;   // PAIR: cluster address of the other CTA's abort_flag, else 0
 };
 
@@ -113,8 +117,10 @@ struct EpiParams {
     float4* part;               // [n_tok][G]: written (KV, K)
     const float* alpha;         // MODE_VCONV: [n_tok] gate values
     const float* conv_w;        // [d][4]
-    const float* state;         // [B][3][d] history, or null (zero history)
-    float* state_next;          // [B][3][d] new history (merged by a second kernel), or null
+    const float* state;         // history, or null (zero history): [B][3][d], or [3][d][B] with state_tr
+    float* state_next;          // new history (merged by a second kernel), or null; same layout as state
+    int state_tr;               // history in the sequence-minor layout [3][d][B] (decode: lanes = sequences)
+    int B;
     __nv_bfloat16* y;           // [n_tok][d]
     uint32_t* status;
     int n_tok, d_mem, d, G;
@@ -512,12 +518,11 @@ __device__ __forceinline__ __half2 tanh_h2(__half2 x) {
     return u2h(r);
 }
 
-template <int BN, bool SLOW, bool RES>
+template <int NCH, bool SLOW, bool RES>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
                                              const uint4* s_cw) {
     constexpr int H = CONV_W - 1;
-    constexpr int NCH = BN / NPART / 16;
     const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
     const bool from_state = SLOW && t < H && p.state;
     uint32_t va[16], vb[16];
@@ -548,11 +553,18 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
                 // the row t-k comes from state row H-k+t
                 uint32_t ps[H] = {0u, 0u, 0u};
                 if (from_state) {
-                    const float* st = p.state + (b * H) * p.d + n0 + cl + c;
+                    const int ch = n0 + cl + c;
 #pragma unroll
                     for (int k = 1; k <= H; ++k)
                         if (t < k) {
-                            const float2 x = __ldg(reinterpret_cast<const float2*>(st + (int64_t)(H - k + t) * p.d));
+                            const int hr = H - k + t;            // history row holding v~_{t-k}
+                            float2 x;
+                            if (p.state_tr) {                     // [3][d][B]: consecutive lanes, consecutive b
+                                const float* st = p.state + ((int64_t)hr * p.d + ch) * p.B + b;
+                                x = make_float2(__ldg(st), __ldg(st + p.B));
+                            } else {
+                                x = __ldg(reinterpret_cast<const float2*>(p.state + (b * H + hr) * p.d + ch));
+                            }
                             ps[k - 1] = h2u(__floats2half2_rn(x.x, x.y));
                         }
                 }
@@ -560,9 +572,17 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
                 if (t < 2) s2 = ps[1];
                 s3 = ps[2];
             }
-            if (write_state)
-                *reinterpret_cast<float2*>(p.state_next + (b * H + (t - (p.L - H))) * p.d + n0 + cl + c) =
-                    make_float2(v0, v1);
+            if (write_state) {
+                const int hr = t - (p.L - H);
+                const int ch = n0 + cl + c;
+                if (p.state_tr) {
+                    float* sn = p.state_next + ((int64_t)hr * p.d + ch) * p.B + b;
+                    sn[0] = v0;
+                    sn[p.B] = v1;
+                } else {
+                    *reinterpret_cast<float2*>(p.state_next + (b * H + hr) * p.d + ch) = make_float2(v0, v1);
+                }
+            }
             const uint4 w = s_cw[(cl + c) >> 1];          // halved taps c_0..c_3 of the channel pair
             __half2 hx = __hmul2(u2h(w.x), vh);
             hx = __hfma2(u2h(w.y), u2h(s1), hx);
@@ -582,9 +602,12 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
     }
 }
 
+// The value tile's epilogue runs in two phases over the two channel halves of
+// the tile, so that the h half of phase 0 can be refilled for the next tile
+// while phase 1 runs.  In each phase part `part` takes BN/8 channels.
 template <int BN>
-__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt,
-                                               int nt, int q, int part, int lane, int et, float* s_taps) {
+__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt, int nt,
+                                               int q, int part, int lane, int et, float* s_taps, int phase) {
     constexpr int H = CONV_W - 1;
     const int i = q * 32 + lane;
     const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - H;
@@ -598,35 +621,38 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     }
     const float a = in_range ? __ldg(p.alpha + r) : 0.f;
     const int n0 = nt * BN;
-    // conv taps of the tile's channel pairs, halved, as fp16 pairs: [BN/2]
-    // x {c_0, c_1, c_2, c_3} of (channel 2m, channel 2m+1)
-    epi_sync();
-    for (int k = et; k < BN / 2; k += EPI_THREADS) {
-        const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k);
-        const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k + 1);
-        reinterpret_cast<uint4*>(s_taps)[k] =
-            make_uint4(h2u(__floats2half2_rn(0.5f * w0.x, 0.5f * w1.x)), h2u(__floats2half2_rn(0.5f * w0.y, 0.5f * w1.y)),
-                       h2u(__floats2half2_rn(0.5f * w0.z, 0.5f * w1.z)), h2u(__floats2half2_rn(0.5f * w0.w, 0.5f * w1.w)));
+    if (phase == 0) {
+        // conv taps of the tile's channel pairs, halved, as fp16 pairs: [BN/2]
+        // x {c_0, c_1, c_2, c_3} of (channel 2m, channel 2m+1)
+        epi_sync();
+        for (int k = et; k < BN / 2; k += EPI_THREADS) {
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k);
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k + 1);
+            reinterpret_cast<uint4*>(s_taps)[k] = make_uint4(
+                h2u(__floats2half2_rn(0.5f * w0.x, 0.5f * w1.x)), h2u(__floats2half2_rn(0.5f * w0.y, 0.5f * w1.y)),
+                h2u(__floats2half2_rn(0.5f * w0.z, 0.5f * w1.z)), h2u(__floats2half2_rn(0.5f * w0.w, 0.5f * w1.w)));
+        }
+        epi_sync();
     }
-    epi_sync();
+    constexpr int PW = BN / (2 * NPART);     // channels of this part in this phase
+    constexpr int NCHK = PW / 16;
+    const int cbeg = phase * (BN / 2) + part * PW;
     // warps whose rows all have their history inside the sequence and write no
     // new history take the branch-free path
     const bool slow_row = out_row && (t < H || (p.state_next && t >= p.L - H));
-    const int cbeg = part * (BN / NPART);
     const uint4* cw = reinterpret_cast<const uint4*>(s_taps);
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
-        if (slow) vconv_chunks<BN, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
-        else vconv_chunks<BN, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        else vconv_chunks<NCHK, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
     } else {
-        if (slow) vconv_chunks<BN, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
-        else vconv_chunks<BN, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        if (slow) vconv_chunks<NCHK, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        else vconv_chunks<NCHK, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
     }
-    // the warp's Y block (its 32 rows x BN/NPART channels, in place of h) to
-    // global memory: LPR lanes cover one row's contiguous bytes, so each store
-    // instruction writes whole rows; the segment's history rows are skipped
+    // the warp's Y block (its 32 rows x PW channels, in place of h) to global
+    // memory: LPR lanes cover one row's contiguous bytes, so each store
+    // instruction writes whole row pieces; the segment's history rows are skipped
     __syncwarp();
-    constexpr int PW = BN / NPART;
     constexpr int LPR = PW * 2 / 16;
     constexpr int RPI = 32 / LPR;
     const int cb = cbeg >> 6;
@@ -742,6 +768,12 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         }
         mbar_init(&sb->hfull, 1);
         mbar_init(&sb->hempty, EPI_WARPS);
+        for (int hf = 0; hf < 2; ++hf) {
+            mbar_init(&sb->hfull_v[hf], 1);
+            mbar_init(&sb->hempty_v[hf], EPI_WARPS);
+            sb->h_issued_v[hf] = 0;
+            sb->h_consumed_v[hf] = 0;
+        }
         mbar_init(&sb->drain, 1);
         sb->abort_flag = 0;
         sb->issued = 0;
@@ -824,6 +856,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     sb->issued = it + 1;
                 }
                 if (!ok) break;
+                if (MODE == MODE_VCONV) continue;   // warp 2 loads the value tile's h
                 // the tile's h slice, once the epilogue has released the previous one
                 if (!wait_bounded(&sb->hempty, ((uint32_t)tc & 1u) ^ 1u, sb, p.status)) break;
                 mbar_arrive_expect_tx(&sb->hfull, GE::H_BYTES);
@@ -882,6 +915,34 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 else umma_commit(&sb->tfull[acc]);
             }
         }
+    } else if (warp == 2 && MODE == MODE_VCONV) {
+        // ---------------- h loader of the value pass: the two channel halves of
+        // each tile's h slice, each as soon as the epilogue has released it, so
+        // neither the operand stream nor the next tile waits on an h load
+        if (lane == 0) {
+            const uint32_t h_dst = smem_u32(s_h);
+            constexpr int CB_HALF = GE::HC / 128;   // 64-channel blocks per half
+            int tc = 0;
+            for (int u = unit0; u < num_units && !sb->abort_flag; u += units_step, ++tc) {
+                const int mt = unit_mt(u), nt = unit_nt(u);
+                bool ok = true;
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (!wait_bounded(&sb->hempty_v[hf], ((uint32_t)tc & 1u) ^ 1u, sb, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sb->hfull_v[hf], GE::H_BYTES / 2);
+                    for (int cb = hf * CB_HALF; cb < (hf + 1) * CB_HALF; ++cb) {
+#pragma unroll
+                        for (int sg = 0; sg < 4; ++sg)
+                            tma_load_2d(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull_v[hf],
+                                        nt * BN + cb * 64, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                    }
+                    sb->h_issued_v[hf] = tc + 1;
+                }
+                if (!ok) break;
+            }
+        }
     } else if (warp >= 4) {
         // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) ..; the
         // four warps of each lane quarter take the four column parts
@@ -894,12 +955,35 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         for (int u = unit0; u < num_units; u += units_step, ++tc) {
             const int acc = tc & 1;
             const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
+            const int mt = unit_mt(u), nt = unit_nt(u);
+            const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+            if (MODE == MODE_VCONV) {
+                // phase 0 on the first channel half, release its h, phase 1
+                bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
+                ok = ok && wait_bounded(&sb->hfull_v[0], (uint32_t)tc & 1u, sb, p.status);
+                if (epi_any(!ok)) break;
+                tc_fence_after();
+                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 0);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sb->hempty_v[0]);
+                if (threadIdx.x == 128) sb->h_consumed_v[0] = tc + 1;
+                ok = wait_bounded(&sb->hfull_v[1], (uint32_t)tc & 1u, sb, p.status);
+                if (epi_any(!ok)) break;
+                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (PAIR && !leader) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+                    else mbar_arrive(&sb->tempty[acc]);
+                    mbar_arrive(&sb->hempty_v[1]);
+                }
+                if (threadIdx.x == 128) sb->h_consumed_v[1] = tc + 1;
+                continue;
+            }
             bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
             ok = ok && wait_bounded(&sb->hfull, (uint32_t)tc & 1u, sb, p.status);
             if (epi_any(!ok)) break;          // one decision for all epilogue warps
             tc_fence_after();
-            const int mt = unit_mt(u), nt = unit_nt(u);
-            const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
             // the odd CTA of the last pair may hold a row tile past the end
             const bool rows_live = MODE == MODE_VCONV ? (int64_t)mt * TILE_OUT < p.n_tok : (int64_t)mt * BM < p.n_tok;
             if (MODE == MODE_KV) epilogue_kv(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
@@ -907,7 +991,6 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
                 band_alpha(p, mt, et, sb, reinterpret_cast<float4*>(s_h), GE::H_BYTES);
             }
-            if (MODE == MODE_VCONV && rows_live) epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -955,6 +1038,14 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 while (!mbar_try_wait(smem_u32(&sb->hfull), (uint32_t)k & 1u) && clock64() - t0 < kWaitCycles) {
                 }
             }
+            for (int hf = 0; hf < 2; ++hf) {
+                for (int k = sb->h_consumed_v[hf]; k < sb->h_issued_v[hf]; ++k) {
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(smem_u32(&sb->hfull_v[hf]), (uint32_t)k & 1u) &&
+                           clock64() - t0 < kWaitCycles) {
+                    }
+                }
+            }
         }
         if (warp == 1 && lane == 0 && (!PAIR || leader)) {
             if constexpr (PAIR) umma_commit_pair_local(&sb->drain);
@@ -990,6 +1081,51 @@ __global__ void state_merge_kernel(float* state, const float* state_next, int B,
             const float val = p >= 0 ? state_next[(b * H + i) * d + c] : state[(b * H + (L + i)) * d + c];
             state[(b * H + i) * d + c] = val;
         }
+    }
+}
+
+// The history in the sequence-minor layout for decode-shaped calls: tiles of
+// 32 sequences x 32 channels go through shared memory so that both the read
+// and the write are coalesced.  state [B][H][d] -> state_t [H][d][B].
+__global__ void state_to_tr_kernel(const float* __restrict__ state, float* __restrict__ state_t, int B, int H, int d) {
+    __shared__ float tile[32][33];
+    const int c0 = blockIdx.x * 32, b0 = blockIdx.y * 32, i = blockIdx.z;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const int b = b0 + r, c = c0 + threadIdx.x;
+        tile[r][threadIdx.x] = (b < B && c < d) ? state[((int64_t)b * H + i) * d + c] : 0.f;
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const int c = c0 + r, b = b0 + threadIdx.x;
+        if (b < B && c < d) state_t[((int64_t)i * d + c) * B + b] = tile[threadIdx.x][r];
+    }
+}
+
+// merge for the sequence-minor layout: new history row i of sequence b is
+// state_next_t[i][c][b] when position L - H + i was computed, else the old
+// row L + i (L < H); each block walks i upwards, so the in-place shift reads
+// a row before the block overwrites it.
+__global__ void state_merge_tr_kernel(float* __restrict__ state, const float* __restrict__ state_next_t, int B, int L,
+                                      int H, int d) {
+    __shared__ float tile[32][33];
+    const int c0 = blockIdx.x * 32, b0 = blockIdx.y * 32;
+    for (int i = 0; i < H; ++i) {
+        const bool fresh = L - H + i >= 0;
+        if (fresh) {
+            for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+                const int c = c0 + r, b = b0 + threadIdx.x;
+                tile[r][threadIdx.x] = (b < B && c < d) ? state_next_t[((int64_t)i * d + c) * B + b] : 0.f;
+            }
+        }
+        __syncthreads();
+        for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+            const int b = b0 + r, c = c0 + threadIdx.x;
+            if (b < B && c < d) {
+                const float v = fresh ? tile[threadIdx.x][r] : state[((int64_t)b * H + (L + i)) * d + c];
+                state[((int64_t)b * H + i) * d + c] = v;
+            }
+        }
+        __syncthreads();
     }
 }
 
@@ -1153,8 +1289,8 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
-                            float* state_next, void* y, int32_t add_residual, uint32_t* status, int num_sms,
-                            cudaStream_t s) {
+                            float* state_next, int32_t state_tr, void* y, int32_t add_residual, uint32_t* status,
+                            int num_sms, cudaStream_t s) {
     const int64_t n_tok = (int64_t)B * L;
     if (!project_tc_supported(n_tok, d_mem, d) || w != CONV_W) return cudaErrorNotSupported;
     const int bn = pick_bn(d);
@@ -1167,6 +1303,8 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     p.conv_w = conv_w;
     p.state = state;
     p.state_next = state ? state_next : nullptr;
+    p.state_tr = state_tr;
+    p.B = B;
     p.y = static_cast<__nv_bfloat16*>(y);
     p.status = status;
     p.n_tok = (int)n_tok;
@@ -1184,6 +1322,23 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     }
     return bn == 256 ? launch_mode<MODE_VCONV, 256, false>(ma, mv, mv, mh, p, mt, num_sms, s)
                      : launch_mode<MODE_VCONV, 128, false>(ma, mv, mv, mh, p, mt, num_sms, s);
+}
+
+cudaError_t launch_state_to_tr(const float* state, float* state_t, int32_t B, int32_t w, int32_t d, cudaStream_t s) {
+    const int H = w - 1;
+    if (H <= 0 || B == 0) return cudaSuccess;
+    const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((B + 31) / 32), (unsigned)H);
+    state_to_tr_kernel<<<grid, dim3(32, 8), 0, s>>>(state, state_t, B, H, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_merge_tr(float* state, const float* state_next_t, int32_t B, int32_t L, int32_t w, int32_t d,
+                                  cudaStream_t s) {
+    const int H = w - 1;
+    if (H <= 0 || B == 0) return cudaSuccess;
+    const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((B + 31) / 32), 1);
+    state_merge_tr_kernel<<<grid, dim3(32, 8), 0, s>>>(state, state_next_t, B, L, H, d);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_state_merge(float* state, const float* state_next, int32_t B, int32_t L, int32_t w, int32_t d,

@@ -125,7 +125,9 @@ ENGRAM_API const char* engram_last_error(void);
  * sequences of L computed rows (n_tok = B*L): indices [n_tok][J] u32,
  * e [n_tok][J*D], gate partials [n_tok][G][4] f32 with G = ceil(d / 128), the
  * gate values [n_tok] f32, ceil(n_tok/128) int32 counters, the next conv
- * history [B][w-1][d] f32 and, where
+ * history [B][w-1][d] f32, for fused calls with L <= 8 a second history
+ * buffer (the history in the sequence-minor layout [w-1][d][B] that the
+ * value pass reads coalesced across sequences) and, where
  * the gate and conv are not
  * fused into the projection (see engram_gate_conv), v [n_tok][d] f32; each
  * part 256-byte aligned.  0 for a null context. */
