@@ -479,11 +479,38 @@ __device__ __forceinline__ void epilogue_kv(uint32_t taddr, const uint8_t* hs, c
     }
 }
 
+// Per-tile values the epilogue reads from global memory (the conv taps or the
+// RMSNorm gains of the tile's channels, the gate of the thread's row), loaded
+// one tile ahead so their latency hides behind the current tile's epilogue.
+struct TilePre {
+    float4 w0, w1;   // MODE_VCONV: taps of channel pair et (channels 2 et, 2 et + 1)
+    float g;         // MODE_K: g_q * g_k of channel et
+    float a;         // MODE_VCONV: alpha of this thread's row
+};
+
+template <int MODE, int BN>
+__device__ __forceinline__ TilePre tile_pre_load(const EpiParams& p, int mt, int nt, int q, int lane, int et) {
+    TilePre t{};
+    const int n0 = nt * BN;
+    if (MODE == MODE_VCONV) {
+        if (et < BN / 2) {
+            t.w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * et);
+            t.w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * et + 1);
+        }
+        const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - (CONV_W - 1);
+        t.a = (r >= 0 && r < p.n_tok) ? __ldg(p.alpha + r) : 0.f;
+    } else if (MODE == MODE_K) {
+        if (et < BN) t.g = (p.gq ? __ldg(p.gq + n0 + et) : 1.f) * (p.gk ? __ldg(p.gk + n0 + et) : 1.f);
+    }
+    return t;
+}
+
 // k tile of BN channels: each of the NPART parts reduces BN/NPART columns,
 // the parts of one 128-channel group are then added in order.
 template <int BN>
 __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int m0, int nt,
-                                           int q, int part, int lane, int et, float* s_gg, float4* s_red) {
+                                           int q, int part, int lane, int et, float* s_gg, float4* s_red,
+                                           TilePre& pre, bool has_next, int mt_next, int nt_next) {
     constexpr int PW = BN / NPART;                    // columns per part
     constexpr int PPG = 128 / PW;                     // parts per 128-channel group
     const int i = q * 32 + lane;
@@ -491,8 +518,9 @@ __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, co
     const bool valid = row < p.n_tok;
     const int n0 = nt * BN;
     epi_sync();
-    load_gains(p, n0, BN, s_gg, et);
+    if (et < BN) s_gg[et] = pre.g;
     epi_sync();
+    if (has_next) pre = tile_pre_load<MODE_K, BN>(p, mt_next, nt_next, q, lane, et);
     group_partials(taddr + part * PW, hs, p, row, i, valid, part, part * PW, PW, PPG, (n0 + part * PW) / 128, s_gg,
                    s_red);
 }
@@ -607,7 +635,8 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
 // while phase 1 runs.  In each phase part `part` takes BN/8 channels.
 template <int BN>
 __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt, int nt,
-                                               int q, int part, int lane, int et, float* s_taps, int phase) {
+                                               int q, int part, int lane, int et, float* s_taps, int phase,
+                                               float a, const TilePre& pre) {
     constexpr int H = CONV_W - 1;
     const int i = q * 32 + lane;
     const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - H;
@@ -619,16 +648,14 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
         b = r / p.L;
         t = (int)(r - b * p.L);
     }
-    const float a = in_range ? __ldg(p.alpha + r) : 0.f;
     const int n0 = nt * BN;
     if (phase == 0) {
-        // conv taps of the tile's channel pairs, halved, as fp16 pairs: [BN/2]
-        // x {c_0, c_1, c_2, c_3} of (channel 2m, channel 2m+1)
+        // conv taps of the tile's channel pairs (loaded a tile ahead), halved,
+        // as fp16 pairs: [BN/2] x {c_0, c_1, c_2, c_3} of (channel 2m, 2m+1)
         epi_sync();
-        for (int k = et; k < BN / 2; k += EPI_THREADS) {
-            const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k);
-            const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * k + 1);
-            reinterpret_cast<uint4*>(s_taps)[k] = make_uint4(
+        if (et < BN / 2) {
+            const float4 w0 = pre.w0, w1 = pre.w1;
+            reinterpret_cast<uint4*>(s_taps)[et] = make_uint4(
                 h2u(__floats2half2_rn(0.5f * w0.x, 0.5f * w1.x)), h2u(__floats2half2_rn(0.5f * w0.y, 0.5f * w1.y)),
                 h2u(__floats2half2_rn(0.5f * w0.z, 0.5f * w1.z)), h2u(__floats2half2_rn(0.5f * w0.w, 0.5f * w1.w)));
         }
@@ -952,24 +979,30 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         const uint32_t tempty_leader0 = PAIR ? peer_addr(&sb->tempty[0], 0u) : 0u;
         const uint32_t tempty_leader1 = PAIR ? peer_addr(&sb->tempty[1], 0u) : 0u;
         int tc = 0;
+        TilePre pre{};
+        if (unit0 < num_units) pre = tile_pre_load<MODE, BN>(p, unit_mt(unit0), unit_nt(unit0), q, lane, et);
         for (int u = unit0; u < num_units; u += units_step, ++tc) {
             const int acc = tc & 1;
             const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
             const int mt = unit_mt(u), nt = unit_nt(u);
             const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+            const int un = u + units_step;
+            const bool has_next = un < num_units;
             if (MODE == MODE_VCONV) {
                 // phase 0 on the first channel half, release its h, phase 1
                 bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
                 ok = ok && wait_bounded(&sb->hfull_v[0], (uint32_t)tc & 1u, sb, p.status);
                 if (epi_any(!ok)) break;
                 tc_fence_after();
-                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 0);
+                const float a_row = pre.a;
+                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 0, a_row, pre);
+                if (has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sb->hempty_v[0]);
                 if (threadIdx.x == 128) sb->h_consumed_v[0] = tc + 1;
                 ok = wait_bounded(&sb->hfull_v[1], (uint32_t)tc & 1u, sb, p.status);
                 if (epi_any(!ok)) break;
-                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 1);
+                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 1, a_row, pre);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -988,8 +1021,11 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const bool rows_live = MODE == MODE_VCONV ? (int64_t)mt * TILE_OUT < p.n_tok : (int64_t)mt * BM < p.n_tok;
             if (MODE == MODE_KV) epilogue_kv(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
             if (MODE == MODE_K && rows_live) {
-                epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
+                epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red, pre, has_next,
+                               unit_mt(un), unit_nt(un));
                 band_alpha(p, mt, et, sb, reinterpret_cast<float4*>(s_h), GE::H_BYTES);
+            } else if (MODE == MODE_K && has_next) {
+                pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
             }
             tc_fence_before();
             __syncwarp();

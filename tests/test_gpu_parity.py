@@ -234,6 +234,7 @@ def test_forward_full_size_sampled(eb, name):
 PAIR_CASES = {
     "pair_a": W["c2"].replace(name="pair_a", B=2, T=2000, M=10007, seed=31),       # 4000 rows, 35 value tiles
     "pair_b": W["c2"].replace(name="pair_b", B=3, T=1501, M=10007, seed=32),       # 4503 rows, ragged 128-row band
+    "pair_c": W["c2"].replace(name="pair_c", B=3, T=1376, M=10007, seed=33),       # 4128 rows, 33 key tiles (odd)
 }
 
 
