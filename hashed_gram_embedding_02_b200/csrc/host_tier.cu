@@ -35,6 +35,10 @@
 #include <thread>
 #include <vector>
 
+#if defined(__SSE2__)
+#include <emmintrin.h>
+#endif
+
 #include "ctx.cuh"
 
 namespace engram {
@@ -125,19 +129,43 @@ __global__ void dedupe_slot_kernel(const uint32_t* __restrict__ idx, int64_t n_l
 // Copy rows [r0, r1) of the distinct-row list from the host tables into the
 // staging buffer, prefetching a few rows ahead.  A row number outside the
 // tables (impossible for lists the dedupe kernel wrote) gives a zero row.
+// On x86 the staging writes are non-temporal (streaming) stores: the staging
+// buffer is read next by the copy engine, not by this core, and skipping the
+// read-for-ownership of each line leaves more host memory bandwidth to the
+// PCIe copies running at the same time.  A store fence ends the range, so
+// the rows are in memory before the chunk is marked packed.
 void pack_range(const uint8_t* tables, int64_t total_rows, size_t row_bytes, const uint64_t* rows, int64_t r0,
                 int64_t r1, uint8_t* dst) {
     constexpr int kAhead = 8;
+#if defined(__SSE2__)
+    const bool stream = (row_bytes % 16) == 0 && (reinterpret_cast<uintptr_t>(dst) % 16) == 0;
+#else
+    const bool stream = false;
+#endif
     for (int64_t r = r0; r < r1; ++r) {
         if (r + kAhead < r1 && rows[r + kAhead] < (uint64_t)total_rows) {
             const uint8_t* pf = tables + rows[r + kAhead] * row_bytes;
             for (size_t o = 0; o < row_bytes; o += 64) __builtin_prefetch(pf + o);
         }
-        if (rows[r] < (uint64_t)total_rows)
-            std::memcpy(dst + (size_t)r * row_bytes, tables + rows[r] * row_bytes, row_bytes);
-        else
-            std::memset(dst + (size_t)r * row_bytes, 0, row_bytes);
+        uint8_t* out = dst + (size_t)r * row_bytes;
+        if (rows[r] >= (uint64_t)total_rows) {
+            std::memset(out, 0, row_bytes);
+            continue;
+        }
+        const uint8_t* in = tables + rows[r] * row_bytes;
+#if defined(__SSE2__)
+        if (stream) {
+            for (size_t o = 0; o < row_bytes; o += 16)
+                _mm_stream_si128(reinterpret_cast<__m128i*>(out + o),
+                                 _mm_loadu_si128(reinterpret_cast<const __m128i*>(in + o)));
+            continue;
+        }
+#endif
+        std::memcpy(out, in, row_bytes);
     }
+#if defined(__SSE2__)
+    if (stream) _mm_sfence();
+#endif
 }
 
 }  // namespace
