@@ -18,7 +18,7 @@
 namespace engram {
 namespace {
 
-constexpr size_t kDefaultChunkBytes = 8u << 20;   // h bytes per chunk when chunk_rows = 0
+constexpr size_t kDefaultChunkBytes = 4u << 20;   // h bytes per chunk when chunk_rows = 0 (c2 sweep: 4 MiB best)
 
 enum IoEvent { EV_START = 0, EV_H_READY = 1, EV_COMPUTED = 3, EV_DRAINED = 5, EV_DONE = 7 };
 static_assert(EV_DONE < kIoEvents, "event slots");

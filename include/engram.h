@@ -255,7 +255,7 @@ ENGRAM_API engram_status engram_forward_noalloc(engram_ctx* ctx, const int32_t* 
  *   P, tables, Wk, Wv, gq, gk, conv_w, conv_state: device memory, as in
  *             engram_forward (conv_state nullable: zero history).
  * The rows are processed in chunks of `chunk_rows` positions of every
- * sequence (0: about 8 MiB of h per chunk).  While chunk i computes on
+ * sequence (0: about 4 MiB of h per chunk).  While chunk i computes on
  * `stream`, the h of chunk i+1 is copied in on one of the context's copy
  * streams and the Y of chunk i-1 is copied out on the other
  * (cudaMemcpy2DAsync).  The conv history passes from chunk to chunk through
