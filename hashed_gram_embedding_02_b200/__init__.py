@@ -12,11 +12,13 @@ from typing import Optional
 
 from .binding import (  # noqa: F401  (re-exported C ABI names)
     ENGRAM_BF16, ENGRAM_F32, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
+    ENGRAM_E_CUDA, ENGRAM_E_DEVICE, ENGRAM_E_HOST, ENGRAM_E_INVAL, ENGRAM_E_NOMEM, ENGRAM_E_TIMEOUT,
+    ENGRAM_E_UNSUPPORTED,
     ENGRAM_INVALID_INDEX, ENGRAM_OK, EXPORTS, LIB_PATH, EngramError, engram_config, engram_conv, engram_create,
     ENGRAM_NOALLOC_SCRATCH_BYTES, engram_destroy, engram_device_status, engram_forward, engram_forward_noalloc,
     engram_forward_host, engram_gate_conv, engram_gather, engram_gather_staged, engram_hash, engram_host_dedupe,
     engram_host_fetch, engram_host_tier_create, engram_host_tier_destroy, engram_host_tier_stats,
-    engram_host_workspace_bytes, engram_pack_rows,
+    engram_host_workspace_bytes, engram_pack_rows, engram_debug_stall_next,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 

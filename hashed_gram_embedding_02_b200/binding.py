@@ -37,7 +37,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_er
            "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward",
            "engram_forward_noalloc", "engram_host_workspace_bytes", "engram_forward_host", "engram_host_tier_create",
            "engram_host_tier_destroy", "engram_host_dedupe", "engram_host_fetch", "engram_gather_staged",
-           "engram_host_tier_stats", "engram_pack_rows")
+           "engram_host_tier_stats", "engram_pack_rows", "engram_debug_stall_next")
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -96,6 +96,7 @@ _sigs = {
     "engram_gather_staged": ([_vp, _i64, _vp, _vp], _st),
     "engram_host_tier_stats": ([_vp, ctypes.c_void_p], _st),
     "engram_pack_rows": ([_vp, _i64, _sz, _vp, _i64, _vp, _i32], _st),
+    "engram_debug_stall_next": ([_vp], _st),
     "engram_forward_host": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                              _i32, _vp, _sz, _vp], _st),
 }
@@ -294,3 +295,8 @@ def engram_pack_rows(host_tables, total_rows: int, row_bytes: int, rows, n: int,
         return x.ctypes.data if hasattr(x, "ctypes") else x.data_ptr()
     _check(_lib.engram_pack_rows(addr(host_tables), total_rows, row_bytes, addr(rows), n, addr(dst), n_threads),
            "engram_pack_rows")
+
+
+def engram_debug_stall_next(ctx) -> None:
+    """Test hook: the next fused key pass lets one bounded wait run out."""
+    _check(_lib.engram_debug_stall_next(ctx), "engram_debug_stall_next")

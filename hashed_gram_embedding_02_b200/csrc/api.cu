@@ -157,7 +157,8 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
         if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
         prof_begin(c, s, "gate_k_tc");
         e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band, w.alpha,
-                             alpha_out, c->d_status, c->num_sms, s);
+                             alpha_out, c->d_status, c->num_sms, c->debug_stall, s);
+        c->debug_stall = 0;
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
         const bool tr = state && decode_shaped(c, n, L);
@@ -328,6 +329,12 @@ void engram_destroy(engram_ctx* c) {
 size_t engram_workspace_bytes(const engram_ctx* c, int32_t B, int32_t L) {
     if (!c || B < 0 || L < 0) return 0;
     return carve(c, nullptr, B, L, true).bytes;
+}
+
+engram_status engram_debug_stall_next(engram_ctx* c) {
+    if (!c) return inval("null context");
+    c->debug_stall = 1;
+    return ENGRAM_OK;
 }
 
 engram_status engram_profile_enable(engram_ctx* c, int32_t enable) {

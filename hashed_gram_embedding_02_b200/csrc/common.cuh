@@ -75,7 +75,8 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 // counters that must be zero on entry and are zero again on exit).
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
-                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, cudaStream_t s);
+                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall,
+                             cudaStream_t s);
 // Pass 2: v -> gate (alpha from pass 1), causal conv, residual, Y (fused
 // epilogue, conv width 4).  When state is non-null the new history goes to
 // state_next ([B][w-1][d] fp32 scratch) and launch_state_merge folds it into

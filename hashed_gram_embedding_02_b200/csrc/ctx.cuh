@@ -29,6 +29,7 @@ struct engram_ctx {
     cudaEvent_t ev[2 * engram::kMaxProf];
     const char* prof_name[engram::kMaxProf];
     int prof_n;
+    int debug_stall;        // engram_debug_stall_next: the next fused key pass stalls (one shot)
     // copy streams and events of the host-buffer pipeline, made at create time
     cudaStream_t io_h2d;
     cudaStream_t io_d2h;

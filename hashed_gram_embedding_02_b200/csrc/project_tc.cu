@@ -129,6 +129,7 @@ struct EpiParams {
     int L;                      // rows per sequence
     int add_residual;
     int* band_count;            // MODE_K: per row band, channel tiles done (zero on entry, zero on exit)
+    int stall;                  // test hook: CTA 0 announces its first stage but never loads it
     float* alpha_w;             // MODE_K: [n_tok] gate values written by each band's last CTA
     float* alpha_out;           // MODE_K: caller's copy of alpha, or null
     float eps;
@@ -866,6 +867,12 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     };
                     if (remote) mbar_arrive_expect_tx_remote(bar, STAGE_BYTES);
                     else mbar_arrive_expect_tx(&sb->full[s], STAGE_BYTES);
+                    if (p.stall && it == 0 && blockIdx.x == 0) {
+                        // bounded-wait test: the stage's bytes are announced
+                        // and never arrive, so the MMA's wait on it runs out
+                        sb->issued = it + 1;
+                        continue;
+                    }
                     if (MODE == MODE_VCONV) {
                         // four 32-row segments, each starting 3 rows before its outputs
 #pragma unroll
@@ -1292,7 +1299,8 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
-                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, cudaStream_t s) {
+                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall,
+                             cudaStream_t s) {
     if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
     const int bn = pick_bn(d);
     CUtensorMap ma, mk, mh;
@@ -1304,6 +1312,7 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     p.gk = gk;
     p.part = reinterpret_cast<float4*>(part);
     p.band_count = band_count;
+    p.stall = stall;
     p.alpha_w = alpha;
     p.alpha_out = alpha_out;
     p.eps = eps;

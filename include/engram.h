@@ -142,6 +142,17 @@ ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int32_t B, int32
 ENGRAM_API engram_status engram_profile_enable(engram_ctx* ctx, int32_t enable);
 ENGRAM_API int32_t engram_profile_read(engram_ctx* ctx, float* ms, const char** names, int32_t max);
 
+/* Test hook for the bounded device waits (failure detection without a
+ * fault): the next fused key pass (tcgen05 path) of this context announces
+ * the bytes of its first operand stage in CTA 0 but never loads them, so the
+ * MMA warp's wait on that stage runs out after about 2 s.  The kernel then
+ * sets ENGRAM_ERR_TIMEOUT, raises its abort flag, drains the copies and MMAs
+ * it issued (bounded again), frees its tensor memory and returns; the
+ * following kernels run to completion.  engram_device_status then reports
+ * ENGRAM_E_TIMEOUT, and the context and its workspace stay usable for the
+ * next call.  The outputs of the stalled call are undefined.  One shot. */
+ENGRAM_API engram_status engram_debug_stall_next(engram_ctx* ctx);
+
 /* Synchronise `stream`, return the device status word in *flags (nullable)
  * and clear it.  ENGRAM_OK when it was zero, ENGRAM_E_TIMEOUT when the
  * timeout bit was set, else ENGRAM_E_DEVICE. */
