@@ -259,7 +259,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_ad
 }
 
 // TMA tile load into this CTA's shared memory whose completion is counted on
-// a barrier of the other CTA of the pair (cta_group::2 form, no multicast)
+// a barrier of the other CTA of the pair (the cta_group::2 form of the load)
 __device__ __forceinline__ void tma_load_2d_peer_bar(const CUtensorMap* map, uint32_t dst, uint32_t bar_cluster, int x,
                                                      int y) {
     asm volatile(
