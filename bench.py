@@ -173,9 +173,9 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("42410853cdb27c94", 123009280 + 50473728),
-    ("c2", "gate_k_tc"): ("42410853cdb27c94", 122741760 + 5350400),
-    ("c2", "retrieve"): ("917d9ef9fd4eee03", 28935424 + 470016),
+    ("c2", "vconv_tc"): ("e283855af9a8f06b", 123129856 + 51037184),
+    ("c2", "gate_k_tc"): ("e283855af9a8f06b", 122802176 + 5524992),
+    ("c2", "retrieve"): ("d3e72d4b3266f802", 28942848 + 869120),
 }
 
 
