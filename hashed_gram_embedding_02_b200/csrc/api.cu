@@ -153,7 +153,22 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
                              cudaStream_t s) {
     const int64_t n = (int64_t)B * L;
     if (fused_path(c, n)) {
-        cudaError_t e = cudaMemsetAsync(w.band, 0, band_bytes(n), s);
+        const bool tr = state && decode_shaped(c, n, L);
+        cudaError_t e = cudaSuccess;
+        if (tr) {
+            // the history transpose only needs the caller's conv_state: it runs on
+            // the side stream while the key pass (a few dozen CTAs at decode
+            // sizes) computes, and the value pass waits for it
+            e = cudaEventRecord(c->aux_ev[0], s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(c->aux, c->aux_ev[0], 0);
+            if (e != cudaSuccess) return cuda_fail("ordering the history transpose", e);
+            prof_begin(c, c->aux, "state_to_tr");
+            e = launch_state_to_tr(state, w.state_t, B, c->cfg.conv_width, c->cfg.hidden, c->aux);
+            prof_end(c, c->aux);
+            if (e == cudaSuccess) e = cudaEventRecord(c->aux_ev[1], c->aux);
+            if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
+        }
+        e = cudaMemsetAsync(w.band, 0, band_bytes(n), s);
         if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
         prof_begin(c, s, "gate_k_tc");
         e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band, w.alpha,
@@ -161,12 +176,9 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
         c->debug_stall = 0;
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
-        const bool tr = state && decode_shaped(c, n, L);
         if (tr) {
-            prof_begin(c, s, "state_to_tr");
-            e = launch_state_to_tr(state, w.state_t, B, c->cfg.conv_width, c->cfg.hidden, s);
-            prof_end(c, s);
-            if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
+            e = cudaStreamWaitEvent(s, c->aux_ev[1], 0);
+            if (e != cudaSuccess) return cuda_fail("joining the history transpose", e);
         }
         prof_begin(c, s, "vconv_tc");
         e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha,
@@ -306,6 +318,8 @@ engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io_d2h, cudaStreamNonBlocking);
     for (int i = 0; i < kIoEvents && e == cudaSuccess; ++i)
         e = cudaEventCreateWithFlags(&c->io_ev[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->aux, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&c->aux_ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
         engram_destroy(c);
         return cuda_fail("context set-up (status word, copy streams, events)", e);
@@ -320,6 +334,9 @@ void engram_destroy(engram_ctx* c) {
         for (int i = 0; i < 2 * kMaxProf; ++i) cudaEventDestroy(c->ev[i]);
     for (int i = 0; i < kIoEvents; ++i)
         if (c->io_ev[i]) cudaEventDestroy(c->io_ev[i]);
+    for (int i = 0; i < 2; ++i)
+        if (c->aux_ev[i]) cudaEventDestroy(c->aux_ev[i]);
+    if (c->aux) cudaStreamDestroy(c->aux);
     if (c->io_h2d) cudaStreamDestroy(c->io_h2d);
     if (c->io_d2h) cudaStreamDestroy(c->io_d2h);
     if (c->d_status) cudaFree(c->d_status);

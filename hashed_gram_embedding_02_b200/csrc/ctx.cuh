@@ -34,6 +34,9 @@ struct engram_ctx {
     cudaStream_t io_h2d;
     cudaStream_t io_d2h;
     cudaEvent_t io_ev[engram::kIoEvents];
+    // side stream for work that overlaps the key pass (the decode history transpose)
+    cudaStream_t aux;
+    cudaEvent_t aux_ev[2];
 };
 
 namespace engram {
