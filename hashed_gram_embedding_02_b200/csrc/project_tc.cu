@@ -484,19 +484,31 @@ __device__ __forceinline__ void epilogue_kv(uint32_t taddr, const uint8_t* hs, c
 // RMSNorm gains of the tile's channels, the gate of the thread's row), loaded
 // one tile ahead so their latency hides behind the current tile's epilogue.
 struct TilePre {
-    float4 w0, w1;   // MODE_VCONV: taps of channel pair et (channels 2 et, 2 et + 1)
+    float4 w0, w1;   // MODE_VCONV: taps of this lane's channel pair of its warp's part (see vconv_pair)
     float g;         // MODE_K: g_q * g_k of channel et
     float a;         // MODE_VCONV: alpha of this thread's row
 };
+
+// The value epilogue's warp (q, part) uses, per phase, BN/(2 NPART) channels =
+// VPP channel pairs; lane l of the warp loads pair l % 16 of phase l / 16
+// (when it exists), so a warp stages its own taps and needs no barrier with
+// the other warps.  Tile-local pair index of that lane, or -1.
+template <int BN>
+__device__ __forceinline__ int vconv_pair(int part, int lane) {
+    constexpr int VPP = BN / (4 * NPART);
+    const int ph = lane >> 4, k = lane & 15;
+    return k < VPP ? ph * (BN / 4) + part * VPP + k : -1;
+}
 
 template <int MODE, int BN>
 __device__ __forceinline__ TilePre tile_pre_load(const EpiParams& p, int mt, int nt, int q, int lane, int et) {
     TilePre t{};
     const int n0 = nt * BN;
     if (MODE == MODE_VCONV) {
-        if (et < BN / 2) {
-            t.w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * et);
-            t.w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * et + 1);
+        const int pr = vconv_pair<BN>((et >> 5) >> 2, lane);
+        if (pr >= 0) {
+            t.w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * pr);
+            t.w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * pr + 1);
         }
         const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - (CONV_W - 1);
         t.a = (r >= 0 && r < p.n_tok) ? __ldg(p.alpha + r) : 0.f;
@@ -650,17 +662,20 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
         t = (int)(r - b * p.L);
     }
     const int n0 = nt * BN;
+    // the warp's own taps (both phases), halved, as fp16 pairs: slot
+    // [warp][phase][pair] x {c_0, c_1, c_2, c_3} of (channel 2m, 2m+1); staged
+    // in phase 0 from the values loaded a tile ahead, read by this warp only
+    constexpr int VPP = BN / (4 * NPART);
+    uint4* s_tw = reinterpret_cast<uint4*>(s_taps) + (size_t)(q * NPART + part) * 2 * 16;
     if (phase == 0) {
-        // conv taps of the tile's channel pairs (loaded a tile ahead), halved,
-        // as fp16 pairs: [BN/2] x {c_0, c_1, c_2, c_3} of (channel 2m, 2m+1)
-        epi_sync();
-        if (et < BN / 2) {
+        const int k = lane & 15, ph = lane >> 4;
+        if (k < VPP) {
             const float4 w0 = pre.w0, w1 = pre.w1;
-            reinterpret_cast<uint4*>(s_taps)[et] = make_uint4(
+            s_tw[ph * 16 + k] = make_uint4(
                 h2u(__floats2half2_rn(0.5f * w0.x, 0.5f * w1.x)), h2u(__floats2half2_rn(0.5f * w0.y, 0.5f * w1.y)),
                 h2u(__floats2half2_rn(0.5f * w0.z, 0.5f * w1.z)), h2u(__floats2half2_rn(0.5f * w0.w, 0.5f * w1.w)));
         }
-        epi_sync();
+        __syncwarp();
     }
     constexpr int PW = BN / (2 * NPART);     // channels of this part in this phase
     constexpr int NCHK = PW / 16;
@@ -668,7 +683,8 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     // warps whose rows all have their history inside the sequence and write no
     // new history take the branch-free path
     const bool slow_row = out_row && (t < H || (p.state_next && t >= p.L - H));
-    const uint4* cw = reinterpret_cast<const uint4*>(s_taps);
+    // indexed by tile-local pair: this warp's slot, shifted to the phase's first pair
+    const uint4* cw = s_tw + phase * 16 - (cbeg >> 1);
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
         if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
@@ -997,19 +1013,23 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const bool has_next = un < num_units;
             if (MODE == MODE_VCONV) {
                 // phase 0 on the first channel half, release its h, phase 1
+                // each warp decides alone: the value epilogue has no barrier
+                // across warps, so a warp that stops cannot strand the others
                 bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
                 ok = ok && wait_bounded(&sb->hfull_v[0], (uint32_t)tc & 1u, sb, p.status);
-                if (epi_any(!ok)) break;
+                if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const float a_row = pre.a;
-                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 0, a_row, pre);
+                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, reinterpret_cast<float*>(s_red), 0,
+                                   a_row, pre);
                 if (has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sb->hempty_v[0]);
                 if (threadIdx.x == 128) sb->h_consumed_v[0] = tc + 1;
                 ok = wait_bounded(&sb->hfull_v[1], (uint32_t)tc & 1u, sb, p.status);
-                if (epi_any(!ok)) break;
-                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, 1, a_row, pre);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, reinterpret_cast<float*>(s_red), 1,
+                                   a_row, pre);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
