@@ -173,9 +173,9 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("e283855af9a8f06b", 123129856 + 51037184),
-    ("c2", "gate_k_tc"): ("e283855af9a8f06b", 122802176 + 5524992),
-    ("c2", "retrieve"): ("d3e72d4b3266f802", 28942848 + 869120),
+    ("c2", "vconv_tc"): ("659729a2018476a5", 123122944 + 51145216),
+    ("c2", "gate_k_tc"): ("659729a2018476a5", 122744320 + 5186816),
+    ("c2", "retrieve"): ("d3e72d4b3266f802", 28940800 + 617984),
 }
 
 
