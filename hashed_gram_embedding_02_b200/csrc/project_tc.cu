@@ -1278,7 +1278,13 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
     return cudaLaunchKernelEx(&cfg, kernel, ma, mb0, mb1, mh, p);
 }
 
-int pick_bn(int32_t d) { return d % 256 == 0 ? 256 : 128; }
+// 256-channel tiles where d allows them, except for decode-sized calls (a few
+// hundred rows) where they would leave most SMs idle: 128-channel tiles
+// double the CTAs there
+int pick_bn(int32_t d, int64_t n_tok, int64_t m_tiles, int num_sms) {
+    if (d % 256 != 0) return 128;
+    return (n_tok <= 1024 && m_tiles * (d / 256) < num_sms / 2) ? 128 : 256;
+}
 
 // CTA pairs once there are enough row tiles to give every SM pair work
 bool use_pair(int64_t m_tiles, int n_groups, int num_sms) { return m_tiles * n_groups >= 2 * (int64_t)num_sms; }
@@ -1322,7 +1328,7 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
                              float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall,
                              cudaStream_t s) {
     if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
-    const int bn = pick_bn(d);
+    const int bn = pick_bn(d, n_tok, (n_tok + BM - 1) / BM, num_sms);
     CUtensorMap ma, mk, mh;
     if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn) ||
         !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, BM))
@@ -1358,7 +1364,7 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
                             int num_sms, cudaStream_t s) {
     const int64_t n_tok = (int64_t)B * L;
     if (!project_tc_supported(n_tok, d_mem, d) || w != CONV_W) return cudaErrorNotSupported;
-    const int bn = pick_bn(d);
+    const int bn = pick_bn(d, n_tok, (n_tok + TILE_OUT - 1) / TILE_OUT, num_sms);
     CUtensorMap ma, mv, mh;
     if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, SEG) || !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn) ||
         !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, SEG))
