@@ -173,9 +173,9 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("659729a2018476a5", 123122944 + 51145216),
-    ("c2", "gate_k_tc"): ("659729a2018476a5", 122744320 + 5186816),
-    ("c2", "retrieve"): ("d3e72d4b3266f802", 28940800 + 617984),
+    ("c2", "vconv_tc"): ("8eddbe3a11629114", 123166208 + 47900672),
+    ("c2", "gate_k_tc"): ("8eddbe3a11629114", 122763264 + 2032128),
+    ("c2", "retrieve"): ("d3e72d4b3266f802", 28957696 + 437248),
 }
 
 
