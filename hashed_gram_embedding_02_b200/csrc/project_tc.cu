@@ -562,7 +562,7 @@ __device__ __forceinline__ __half2 tanh_h2(__half2 x) {
 template <int NCH, bool SLOW, bool RES>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
-                                             const uint4* s_cw) {
+                                             const uint4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3) {
     constexpr int H = CONV_W - 1;
     const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
     const bool from_state = SLOW && t < H && p.state;
@@ -589,6 +589,12 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
             uint32_t s1 = __shfl_up_sync(0xffffffffu, u0, 1);
             uint32_t s2 = __shfl_up_sync(0xffffffffu, u0, 2);
             uint32_t s3 = __shfl_up_sync(0xffffffffu, u0, 3);
+            if (!SLOW) {
+                // rows before the sequence start (no conv_state): zero history
+                s1 &= m1;
+                s2 &= m2;
+                s3 &= m3;
+            }
             if (SLOW && t < H) {
                 // history before the slab start: conv_state (zero without one);
                 // the row t-k comes from state row H-k+t
@@ -680,18 +686,23 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     constexpr int PW = BN / (2 * NPART);     // channels of this part in this phase
     constexpr int NCHK = PW / 16;
     const int cbeg = phase * (BN / 2) + part * PW;
-    // warps whose rows all have their history inside the sequence and write no
-    // new history take the branch-free path
-    const bool slow_row = out_row && (t < H || (p.state_next && t >= p.L - H));
+    // Rows whose history reaches back into conv_state, and rows among a
+    // sequence's last H when the new history is written, take the slow path
+    // (only warps holding such rows).  Without conv_state the history before
+    // a sequence start is zero, which the fast path applies through per-lane
+    // masks: a separate path that one warp in a few tiles runs stalled that
+    // warp, and with it the CTA's next tiles, for about 15 us.
+    const bool slow_row = out_row && ((t < H && p.state) || (p.state_next && t >= p.L - H));
+    const uint32_t m1 = t >= 1 ? ~0u : 0u, m2 = t >= 2 ? ~0u : 0u, m3 = t >= 3 ? ~0u : 0u;
     // indexed by tile-local pair: this warp's slot, shifted to the phase's first pair
     const uint4* cw = s_tw + phase * 16 - (cbeg >> 1);
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
-        if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
-        else vconv_chunks<NCHK, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
+        else vconv_chunks<NCHK, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
     } else {
-        if (slow) vconv_chunks<NCHK, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
-        else vconv_chunks<NCHK, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw);
+        if (slow) vconv_chunks<NCHK, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
+        else vconv_chunks<NCHK, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
     }
     // the warp's Y block (its 32 rows x PW channels, in place of h) to global
     // memory: LPR lanes cover one row's contiguous bytes, so each store
@@ -1012,32 +1023,34 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const int un = u + units_step;
             const bool has_next = un < num_units;
             if (MODE == MODE_VCONV) {
-                // phase 0 on the first channel half, release its h, phase 1
+                // phase 0 on the first channel half, release its h, phase 1;
                 // each warp decides alone: the value epilogue has no barrier
-                // across warps, so a warp that stops cannot strand the others
+                // across warps, so a warp that stops cannot strand the others.
+                // Both phases run one copy of the code (not unrolled), so the
+                // first tile fetches the epilogue's instructions once.
                 bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
-                ok = ok && wait_bounded(&sb->hfull_v[0], (uint32_t)tc & 1u, sb, p.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const float a_row = pre.a;
-                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, reinterpret_cast<float*>(s_red), 0,
-                                   a_row, pre);
-                if (has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sb->hempty_v[0]);
-                if (threadIdx.x == 128) sb->h_consumed_v[0] = tc + 1;
-                ok = wait_bounded(&sb->hfull_v[1], (uint32_t)tc & 1u, sb, p.status);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, reinterpret_cast<float*>(s_red), 1,
-                                   a_row, pre);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if (PAIR && !leader) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
-                    else mbar_arrive(&sb->tempty[acc]);
-                    mbar_arrive(&sb->hempty_v[1]);
+#pragma unroll 1
+                for (int phase = 0; phase < 2; ++phase) {
+                    ok = wait_bounded(&sb->hfull_v[phase], (uint32_t)tc & 1u, sb, p.status);
+                    if (!__all_sync(0xffffffffu, ok)) break;
+                    epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, reinterpret_cast<float*>(s_red),
+                                       phase, a_row, pre);
+                    if (phase == 0 && has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
+                    if (phase == 1) tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (phase == 1) {
+                            if (PAIR && !leader) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+                            else mbar_arrive(&sb->tempty[acc]);
+                        }
+                        mbar_arrive(&sb->hempty_v[phase]);
+                    }
+                    if (threadIdx.x == 128) sb->h_consumed_v[phase] = tc + 1;
                 }
-                if (threadIdx.x == 128) sb->h_consumed_v[1] = tc + 1;
+                if (!__all_sync(0xffffffffu, ok)) break;
                 continue;
             }
             bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
