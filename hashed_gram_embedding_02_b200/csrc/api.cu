@@ -146,11 +146,16 @@ engram_status conv_impl(engram_ctx* c, const float* v, const float* part, const 
 
 // projections + gate + conv; on the fused path two tcgen05 GEMM passes with
 // the gate and the conv in the second one's epilogue, otherwise the
-// projection (tcgen05 or CUDA cores) followed by the CUDA-core gate/conv
+// projection (tcgen05 or CUDA cores) followed by the CUDA-core gate/conv.
+// after_retrieve: the band counters are already cleared and the kernel just
+// before on the stream is the retrieval that wrote e_cat, so the key pass
+// can be its programmatic dependent (unless the decode history transpose
+// records an event in between).  Timed runs (engram_profile_enable) put
+// events between the kernels and launch them plainly.
 engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, const void* Wk, const void* Wv,
                              const float* gq, const float* gk, const float* conv_w, int32_t B, int32_t L,
                              float* state, void* y, float* alpha_out, int32_t add_residual, const Workspace& w,
-                             cudaStream_t s) {
+                             cudaStream_t s, bool after_retrieve = false) {
     const int64_t n = (int64_t)B * L;
     if (fused_path(c, n)) {
         const bool tr = state && decode_shaped(c, n, L);
@@ -168,11 +173,14 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
             if (e == cudaSuccess) e = cudaEventRecord(c->aux_ev[1], c->aux);
             if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
         }
-        e = cudaMemsetAsync(w.band, 0, band_bytes(n), s);
-        if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
+        if (!after_retrieve) {
+            e = cudaMemsetAsync(w.band, 0, band_bytes(n), s);
+            if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
+        }
         prof_begin(c, s, "gate_k_tc");
         e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band, w.alpha,
-                             alpha_out, c->d_status, c->num_sms, c->debug_stall, s);
+                             alpha_out, c->d_status, c->num_sms, c->debug_stall, after_retrieve && !tr && !c->prof,
+                             s);
         c->debug_stall = 0;
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
@@ -183,7 +191,7 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
         prof_begin(c, s, "vconv_tc");
         e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha,
                             tr ? w.state_t : state, w.state_next, tr ? 1 : 0, y, add_residual, c->d_status,
-                            c->num_sms, s);
+                            c->num_sms, !tr && !c->prof, s);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 value/conv launch", e);
         if (state) {
@@ -212,11 +220,18 @@ engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t
                            const void* Wv, const float* gq, const float* gk, const float* conv_w, float* conv_state,
                            void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s) {
     const int32_t L = T - t_begin;
+    const bool fused = fused_path(c, (int64_t)B * L);
+    if (fused) {
+        // cleared ahead of the retrieval, so that the key pass directly follows it
+        cudaError_t e = cudaMemsetAsync(w.band, 0, band_bytes((int64_t)B * L), s);
+        if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
+    }
     prof_begin(c, s, "retrieve");
     cudaError_t e = launch_retrieve(tok, P, B, T, tok_stride, t_begin, c->hp, c->gp, tables, w.idx, w.e, c->d_status, s);
     prof_end(c, s);
     if (e != cudaSuccess) return cuda_fail("retrieve (hash + gather) launch", e);
-    return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s);
+    return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s,
+                          fused);
 }
 
 }  // namespace engram

@@ -73,18 +73,24 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 // Pass 1: k -> gate partials [n_tok][G][4] and alpha [n_tok] (reduced by the
 // CTA that completes each 128-row band; band_count holds ceil(n_tok/128)
 // counters that must be zero on entry and are zero again on exit).
+// pdl: launched as a programmatic dependent of the kernel just before it on
+// the stream (which produced e); every thread waits for that kernel's
+// completion before any global access, then lets the next pass launch.
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
-                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall,
+                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
                              cudaStream_t s);
 // Pass 2: v -> gate (alpha from pass 1), causal conv, residual, Y (fused
 // epilogue, conv width 4).  When state is non-null the new history goes to
 // state_next ([B][w-1][d] fp32 scratch) and launch_state_merge folds it into
-// state afterwards.
+// state afterwards.  pdl: launched as a programmatic dependent of pass 1,
+// which must be the kernel just before it on the stream; the operand loads
+// and MMAs start on SMs as pass 1's CTAs leave, and the epilogue waits for
+// pass 1's completion before it reads alpha.
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
                             float* state_next, int32_t state_tr, void* y, int32_t add_residual, uint32_t* status,
-                            int num_sms, cudaStream_t s);
+                            int num_sms, bool pdl, cudaStream_t s);
 // conv history [B][w-1][d] -> the sequence-minor [w-1][d][B] that decode-shaped
 // value passes read (state_tr), and the merge of such a pass's new history
 // back into the caller's [B][w-1][d]

@@ -279,6 +279,15 @@ __device__ __forceinline__ void st_remote_s32(uint32_t cluster_addr, int v) {
     asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
+// programmatic dependent launch: wait for the kernel this grid depends on
+// to complete (its memory operations visible; returns at once when the grid
+// was launched without such a dependency), and let this grid's own
+// dependent launch
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // all threads of both CTAs
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -863,6 +872,12 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = sb->tmem_base;
+    if (MODE != MODE_VCONV) {
+        // e comes from the kernel before this one: wait for it, then let the
+        // value pass launch (its CTAs take SMs as this pass's CTAs leave)
+        grid_dep_wait();
+        grid_dep_launch_dependents();
+    }
 
     // row tile of this CTA for unit u; channel tile
     auto unit_mt = [&](int u) { return PAIR ? 2 * (u / p.n_groups) + (int)rank : u / p.n_groups; };
@@ -1014,6 +1029,9 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         const uint32_t tempty_leader1 = PAIR ? peer_addr(&sb->tempty[1], 0u) : 0u;
         int tc = 0;
         TilePre pre{};
+        // alpha comes from the key pass, which may still be running when this
+        // grid was launched as its programmatic dependent
+        if (MODE == MODE_VCONV) grid_dep_wait();
         if (unit0 < num_units) pre = tile_pre_load<MODE, BN>(p, unit_mt(unit0), unit_nt(unit0), q, lane, et);
         for (int u = unit0; u < num_units; u += units_step, ++tc) {
             const int acc = tc & 1;
@@ -1241,7 +1259,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 template <int MODE, int BN, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const CUtensorMap& mh,
-                        EpiParams p, int64_t m_tiles, int num_sms, cudaStream_t s) {
+                        EpiParams p, int64_t m_tiles, int num_sms, cudaStream_t s, bool pdl = false) {
     using GE = Geo<MODE, BN, PAIR>;
     auto kernel = project_tc_kernel<MODE, BN, PAIR>;
     static unsigned long long attr_set = 0;   // one bit per device ordinal
@@ -1260,26 +1278,39 @@ cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
     const int64_t units = (PAIR ? (m_tiles + 1) / 2 : m_tiles) * p.n_groups;
     if (units >= (int64_t)1 << 31) return cudaErrorInvalidValue;
     p.num_tiles = (int)units;
-    if (!PAIR) {
-        const int grid = (int)(units < num_sms ? units : num_sms);
-        kernel<<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, mh, p);
-        return cudaGetLastError();
-    }
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = GE::SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 0;
+    if (pdl) {
+        attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+        ++cfg.numAttrs;
+    }
+    if (!PAIR) {
+        const int grid = (int)(units < num_sms ? units : num_sms);
+        if (!pdl) {
+            kernel<<<grid, THREADS, GE::SMEM_BYTES, s>>>(ma, mb0, mb1, mh, p);
+            return cudaGetLastError();
+        }
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        return cudaLaunchKernelEx(&cfg, kernel, ma, mb0, mb1, mh, p);
+    }
+    attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+    attr[cfg.numAttrs].val.clusterDim.x = 2;
+    attr[cfg.numAttrs].val.clusterDim.y = 1;
+    attr[cfg.numAttrs].val.clusterDim.z = 1;
+    ++cfg.numAttrs;
     if (dev < 64 && max_clusters[dev] == 0) {
         cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
         int mc = 0;
-        if (cudaOccupancyMaxActiveClusters(&mc, kernel, &cfg) != cudaSuccess || mc < 1) {
+        cudaLaunchConfig_t qcfg = cfg;                 // the cluster shape alone
+        qcfg.attrs = &attr[cfg.numAttrs - 1];
+        qcfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&mc, kernel, &qcfg) != cudaSuccess || mc < 1) {
             cudaGetLastError();
             mc = num_sms / 2;
         }
@@ -1338,7 +1369,7 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
-                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall,
+                             float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
                              cudaStream_t s) {
     if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
     const int bn = pick_bn(d, n_tok, (n_tok + BM - 1) / BM, num_sms);
@@ -1365,16 +1396,16 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     if (bn == 256 && use_pair(mt, p.n_groups, num_sms)) {
         CUtensorMap mk2;
         if (!make_map(&mk2, Wk, (uint64_t)d, (uint64_t)d_mem, 128)) return cudaErrorInvalidValue;
-        return launch_mode<MODE_K, 256, true>(ma, mk2, mk2, mh, p, mt, num_sms, s);
+        return launch_mode<MODE_K, 256, true>(ma, mk2, mk2, mh, p, mt, num_sms, s, pdl);
     }
-    return bn == 256 ? launch_mode<MODE_K, 256, false>(ma, mk, mk, mh, p, mt, num_sms, s)
-                     : launch_mode<MODE_K, 128, false>(ma, mk, mk, mh, p, mt, num_sms, s);
+    return bn == 256 ? launch_mode<MODE_K, 256, false>(ma, mk, mk, mh, p, mt, num_sms, s, pdl)
+                     : launch_mode<MODE_K, 128, false>(ma, mk, mk, mh, p, mt, num_sms, s, pdl);
 }
 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
                             float* state_next, int32_t state_tr, void* y, int32_t add_residual, uint32_t* status,
-                            int num_sms, cudaStream_t s) {
+                            int num_sms, bool pdl, cudaStream_t s) {
     const int64_t n_tok = (int64_t)B * L;
     if (!project_tc_supported(n_tok, d_mem, d) || w != CONV_W) return cudaErrorNotSupported;
     const int bn = pick_bn(d, n_tok, (n_tok + TILE_OUT - 1) / TILE_OUT, num_sms);
@@ -1402,10 +1433,10 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     if (bn == 256 && use_pair_vconv(mt, p.n_groups, num_sms)) {
         CUtensorMap mv2;
         if (!make_map(&mv2, Wv, (uint64_t)d, (uint64_t)d_mem, 128)) return cudaErrorInvalidValue;
-        return launch_mode<MODE_VCONV, 256, true>(ma, mv2, mv2, mh, p, mt, num_sms, s);
+        return launch_mode<MODE_VCONV, 256, true>(ma, mv2, mv2, mh, p, mt, num_sms, s, pdl);
     }
-    return bn == 256 ? launch_mode<MODE_VCONV, 256, false>(ma, mv, mv, mh, p, mt, num_sms, s)
-                     : launch_mode<MODE_VCONV, 128, false>(ma, mv, mv, mh, p, mt, num_sms, s);
+    return bn == 256 ? launch_mode<MODE_VCONV, 256, false>(ma, mv, mv, mh, p, mt, num_sms, s, pdl)
+                     : launch_mode<MODE_VCONV, 128, false>(ma, mv, mv, mh, p, mt, num_sms, s, pdl);
 }
 
 cudaError_t launch_state_to_tr(const float* state, float* state_t, int32_t B, int32_t w, int32_t d, cudaStream_t s) {

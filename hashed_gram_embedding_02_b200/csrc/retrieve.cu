@@ -54,6 +54,9 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
     __shared__ int64_t s_off[kMaxTables];
     __shared__ uint32_t s_rows[kMaxTables];
     __shared__ int32_t s_order[kMaxTables];
+    // the key pass that follows may launch now: its CTAs take SMs as these
+    // leave and wait for this grid's completion before they read e_cat
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t L = (int64_t)T - t_begin;
     const int64_t n = (int64_t)B * L;
     const int64_t row0 = (int64_t)blockIdx.x * rows_per_cta;
