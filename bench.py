@@ -173,9 +173,9 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("8eddbe3a11629114", 123166208 + 47900672),
-    ("c2", "gate_k_tc"): ("8eddbe3a11629114", 122763264 + 2032128),
-    ("c2", "retrieve"): ("d3e72d4b3266f802", 28957696 + 437248),
+    ("c2", "vconv_tc"): ("8bc6e756c5446080", 123009792 + 51139840),
+    ("c2", "gate_k_tc"): ("8bc6e756c5446080", 122744832 + 5460480),
+    ("c2", "retrieve"): ("1ca1613a79a9c90b", 28940800 + 632832),
 }
 
 

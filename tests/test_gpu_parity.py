@@ -336,6 +336,31 @@ def test_forward_is_deterministic(eb):
     assert torch.equal(y1, y2) and torch.equal(a1, a2)
 
 
+@pytest.mark.parametrize("name", ["b3", "pair_a"])
+def test_dependent_launches_match_plain_launches(eb, name):
+    """engram_forward launches the key pass as a programmatic dependent of the
+    retrieval and the value pass as one of the key pass; with kernel timing
+    on, events separate the kernels and the launches are plain.  Both must
+    give the same bits.  A forward on other hidden states runs first, so a
+    value epilogue that read alpha before the key pass completed would see
+    different values."""
+    wl = {**SMALL, **PAIR_CASES}[name]
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    y0 = di.empty_y()
+    ctx.forward(di.tok, di.P, di.tables, (di.h * 3).contiguous(), di.Wk, di.Wv, di.conv_w, y0, gq=di.gq, gk=di.gk,
+                add_residual=True)
+    y1, a1 = _run_forward(eb, ctx, di, add_residual=True)
+    eb.engram_profile_enable(ctx.ctx, True)
+    try:
+        y2, a2 = _run_forward(eb, ctx, di, add_residual=True)
+    finally:
+        eb.engram_profile_enable(ctx.ctx, False)
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    assert torch.equal(y1, y2) and torch.equal(a1, a2)
+
+
 @pytest.mark.parametrize("B,T,t_begin", [(1, 1, 0), (1, 2, 0), (2, 3, 1), (1, 129, 0), (5, 1, 0), (3, 4, 4)])
 def test_edge_shapes(eb, B, T, t_begin):
     wl = SMALL["b1"].replace(B=B, T=T, t_begin=t_begin)
