@@ -383,7 +383,9 @@ def run_host_tier(args, wl, rank, world, dev):
                       "fetch_ms": fetch_ms, "last_fetch": tstats, "pack_threads": n_threads,
                       "layer_gemm_ms": layer_ms, "engram_alone_ms": alone_ms, "step_ms": step_ms,
                       "overhead_over_layer": (step_ms - layer_ms) / layer_ms, "table_generation_s": gen_s},
-        "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": clocks.summary(),
+        # per step: hash, dedupe insert, dedupe slot, staged gather, key pass,
+        # value pass (the stand-in GEMM and the memsets are not this library's)
+        "cpu_baseline": None, "e2e": None, "gpu_launches": 6 * K, "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)
 
