@@ -173,8 +173,8 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("8bc6e756c5446080", 123009792 + 51139840),
-    ("c2", "gate_k_tc"): ("8bc6e756c5446080", 122744832 + 5460480),
+    ("c2", "vconv_tc"): ("6ddf1a4b0328cd9b", 123190528 + 28159232),
+    ("c2", "gate_k_tc"): ("6ddf1a4b0328cd9b", 122743552 + 86016),
     ("c2", "retrieve"): ("1ca1613a79a9c90b", 28940800 + 632832),
 }
 

@@ -167,6 +167,24 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint32_t dst
         : "memory");
 }
 
+// The same load with an L2 eviction-priority hint (a policy made by
+// createpolicy): h is read once per pass, so its lines go first and e and W
+// stay in L2
+__device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap* map, uint32_t dst, uint64_t* bar, int x, int y,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(dst), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -728,7 +746,7 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
         const int ii = q * 32 + rr;
         const uint4 v = *reinterpret_cast<const uint4*>(hs + cb * (BM * 128) + ii * 128 + ((j ^ (ii & 7)) << 4));
         const int64_t rg = seg0 + rr;
-        if (rr >= H && rg < p.n_tok) *reinterpret_cast<uint4*>(p.y + rg * p.d + n0 + cb * 64 + j * 8) = v;
+        if (rr >= H && rg < p.n_tok) __stcs(reinterpret_cast<uint4*>(p.y + rg * p.d + n0 + cb * 64 + j * 8), v);
     }
 }
 
@@ -888,6 +906,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         if (lane == 0) {
             int it = 0, tc = 0;
             const uint32_t h_dst = smem_u32(s_h);
+            const uint64_t h_pol = l2_policy_evict_first();
             for (int u = unit0; u < num_units && !sb->abort_flag; u += units_step, ++tc) {
                 const int mt = unit_mt(u), nt = unit_nt(u);
                 bool ok = true;
@@ -942,10 +961,10 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     if (MODE == MODE_VCONV) {
 #pragma unroll
                         for (int sg = 0; sg < 4; ++sg)
-                            tma_load_2d(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull, hc0 + cb * 64,
-                                        mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                            tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull, hc0 + cb * 64,
+                                             mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1), h_pol);
                     } else {
-                        tma_load_2d(&map_h, h_dst + cb * (BM * 128), &sb->hfull, hc0 + cb * 64, mt * BM);
+                        tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128), &sb->hfull, hc0 + cb * 64, mt * BM, h_pol);
                     }
                 }
                 sb->h_issued = tc + 1;
@@ -997,6 +1016,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         // neither the operand stream nor the next tile waits on an h load
         if (lane == 0) {
             const uint32_t h_dst = smem_u32(s_h);
+            const uint64_t h_pol = l2_policy_evict_first();
             constexpr int CB_HALF = GE::HC / 128;   // 64-channel blocks per half
             int tc = 0;
             for (int u = unit0; u < num_units && !sb->abort_flag; u += units_step, ++tc) {
@@ -1011,8 +1031,8 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     for (int cb = hf * CB_HALF; cb < (hf + 1) * CB_HALF; ++cb) {
 #pragma unroll
                         for (int sg = 0; sg < 4; ++sg)
-                            tma_load_2d(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull_v[hf],
-                                        nt * BN + cb * 64, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                            tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull_v[hf],
+                                             nt * BN + cb * 64, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1), h_pol);
                     }
                     sb->h_issued_v[hf] = tc + 1;
                 }
