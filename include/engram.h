@@ -218,11 +218,15 @@ ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, co
                                int32_t add_residual, void* workspace, size_t workspace_bytes,
                                cudaStream_t stream);
 
-/* The whole forward: engram_hash (with remap) -> engram_gather ->
- * engram_gate_conv, intermediates in `workspace`
- * (engram_workspace_bytes(ctx, B, T-t_begin) bytes, 256-byte aligned).
- * tok is [B] rows of `tok_stride` raw ids; prefill uses t_begin = 0, a
- * decode step for the last position uses t_begin = T-1 with conv_state. */
+/* The whole forward: what engram_hash (with remap), engram_gather and
+ * engram_gate_conv compute, with the first two fused into one retrieval
+ * kernel; intermediates in `workspace` (engram_workspace_bytes(ctx, B,
+ * T-t_begin) bytes, 256-byte aligned).  tok is [B] rows of `tok_stride` raw
+ * ids; prefill uses t_begin = 0, a decode step for the last position uses
+ * t_begin = T-1 with conv_state.  On the tensor-core path the two GEMM passes
+ * are launched as programmatic dependents of the kernel before each (they
+ * overlap its last CTAs and wait for its results on the device); seen from
+ * the stream, the call is ordered like any other work on `stream`. */
 ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int32_t B, int32_t T,
                              int64_t tok_stride, int32_t t_begin, const int32_t* P,
                              const void* tables, const void* h, const void* Wk, const void* Wv,
