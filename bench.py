@@ -21,6 +21,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import sys
 import threading
 import time
@@ -162,9 +163,10 @@ def oracle_sample_time(wl, n_tokens: int):
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture of each kernel on a workload, with the digest of the kernel's
-# sources at capture time: once a source changes, the figure no longer
-# describes the kernel and the line reports null.  profiles/ holds the
-# capture's summary and the command that made it.
+# sources at capture time (their code, comments and blank lines left out):
+# once the code changes, the figure no longer describes the kernel and the
+# line reports null.  profiles/ holds the capture's summary and the command
+# that made it.
 CSRC = os.path.join(ROOT, "hashed_gram_embedding_02_b200", "csrc")
 KERNEL_SOURCES = {
     "gate_k_tc": ("project_tc.cu", "common.cuh", "ptx.cuh"),
@@ -173,17 +175,30 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    ("c2", "vconv_tc"): ("6ddf1a4b0328cd9b", 123190528 + 28159232),
-    ("c2", "gate_k_tc"): ("6ddf1a4b0328cd9b", 122743552 + 86016),
-    ("c2", "retrieve"): ("1ca1613a79a9c90b", 28940800 + 632832),
+    ("c2", "vconv_tc"): ("ece15e492f5dcb2f", 123190528 + 28159232),
+    ("c2", "gate_k_tc"): ("ece15e492f5dcb2f", 122743552 + 86016),
+    ("c2", "retrieve"): ("8c46903b0c8d286e", 28940800 + 632832),
 }
 
 
-def source_digest(files) -> str:
+def _code_only(text: str) -> str:
+    """The source without comments and blank lines: editing a comment does
+    not change the compiled kernel, so it keeps the capture valid."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
+def source_digest(files, read=None) -> str:
+    """Digest of the kernel's sources (code only).  `read(name)` returns a
+    file's text; by default the file under csrc/."""
+    if read is None:
+        def read(name):
+            with open(os.path.join(CSRC, name), encoding="utf-8") as fh:
+                return fh.read()
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        h.update(_code_only(read(f)).encode())
     return h.hexdigest()[:16]
 
 

@@ -24,17 +24,22 @@
 //
 // Persistent kernel, one CTA per SM, warp-specialised (640 threads):
 //   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of A (e) and
-//              W into a shared-memory ring, and of the tile's h slice into a
-//              shared buffer the epilogue reads (issued after the tile's
-//              k-blocks, so it never holds back the MMA)
+//              W into a shared-memory ring; in MODE_K/MODE_KV also the tile's
+//              h slice into a shared buffer the epilogue reads (issued after
+//              the tile's k-blocks, so it never holds back the MMA)
 //   warp 1     allocates TMEM (two fp32 accumulators) and issues
 //              tcgen05.mma kind::f16 (M=128, N=BN, K=16) from one thread
+//   warp 2     MODE_VCONV: loads each channel half of the tile's h slice as
+//              soon as the epilogue has released it
 //   warps 4-19 epilogue: warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31;
 //              the four groups of four warps take four column parts of
 //              the tile's channels
 // The double-buffered accumulator lets the epilogue of tile i overlap the
 // MMAs of tile i+1.  Tiles run channel-fastest so consecutive tiles share the
-// A block in L2; W stays L2-resident.
+// A block in L2; W stays L2-resident, and h, read once per pass, is loaded
+// with an evict-first hint.  In engram_forward the key pass is a
+// programmatic dependent of the retrieval and the value pass one of the key
+// pass: only the value epilogue's read of alpha waits for the key pass.
 //
 // Every mbarrier wait is bounded (about 2 s of clock64 time).  A wait that runs
 // out sets ENGRAM_ERR_TIMEOUT, raises a CTA-wide abort flag that makes the
