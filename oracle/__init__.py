@@ -68,10 +68,6 @@ def lib():
         L.orc_silu.restype = f64
         L.orc_output.argtypes = [P, P, P, i64, i32, i32, P]
         L.orc_output.restype = None
-        L.orc_round_bf16.argtypes = [f64]
-        L.orc_round_bf16.restype = f64
-        L.orc_round_bf16_array.argtypes = [P, i64]
-        L.orc_round_bf16_array.restype = None
         _lib = L
     return _lib
 
@@ -187,13 +183,6 @@ def silu(x: float) -> float:
     return lib().orc_silu(float(x))
 
 
-def round_bf16(x) -> np.ndarray:
-    a = np.array(x, dtype=np.float64, copy=True)
-    flat = a.reshape(-1)
-    lib().orc_round_bf16_array(_p(flat), flat.size)
-    return flat.reshape(a.shape)
-
-
 # ---------------------------------------------------------------- composites
 
 class Result:
@@ -203,7 +192,7 @@ class Result:
         self.__dict__.update(kw)
 
 
-def _value_path(e, h, Wk, Wv, gq, gk, eps, bf16: bool):
+def _value_path(e, h, Wk, Wv, gq, gk, eps):
     # k and v are kept at full precision: the pages fix no storage point for
     # them, and this build's rounding points are the stored tensors only
     # (tables/e, h, W, Y)
@@ -222,7 +211,7 @@ def forward_full(inp, add_residual: bool = False, eps: float = 1e-6, hist: Optio
     tables = inp.all_tables() if tables is None else tables
     e = gather(idx, inp.rows, tables)
     h = inp.all_hidden() if h is None else h
-    k, v, alpha = _value_path(e, h, inp.Wk, inp.Wv, inp.gq, inp.gk, eps, wl.dtype == "bf16")
+    k, v, alpha = _value_path(e, h, inp.Wk, inp.Wv, inp.gq, inp.gk, eps)
     vt = alpha[:, None] * v
     L = wl.T - wl.t_begin
     u = np.empty_like(vt)
@@ -254,7 +243,7 @@ def forward_rows(inp, positions: np.ndarray, add_residual: bool = False, eps: fl
     slot = {int(r): i for i, r in enumerate(need)}
     e = gather_rows(idx[need], inp.rows, inp.table_rows)
     h = inp.hidden_rows(need)
-    k, v, alpha = _value_path(e, h, inp.Wk, inp.Wv, inp.gq, inp.gk, eps, wl.dtype == "bf16")
+    k, v, alpha = _value_path(e, h, inp.Wk, inp.Wv, inp.gq, inp.gk, eps)
     vt = alpha[:, None] * v
     y = np.empty((len(positions), wl.d))
     al = np.empty(len(positions))

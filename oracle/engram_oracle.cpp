@@ -187,18 +187,4 @@ void orc_output(const double* vt, const double* u, const double* h, int64_t n, i
     }
 }
 
-// Round to the nearest bf16 value (8 significant bits), ties to even, for
-// normal-range values; the storage point of v in the bf16 path.
-double orc_round_bf16(double x) {
-    if (x == 0.0 || !std::isfinite(x)) return x;
-    int e = 0;
-    const double m = std::frexp(x, &e);          // x = m * 2^e, 0.5 <= |m| < 1
-    const double r = std::nearbyint(std::ldexp(m, 8));  // 8 significant bits, ties-to-even
-    return std::ldexp(r, e - 8);
-}
-
-void orc_round_bf16_array(double* x, int64_t n) {
-    for (int64_t i = 0; i < n; ++i) x[i] = orc_round_bf16(x[i]);
-}
-
 }  // extern "C"

@@ -1,9 +1,12 @@
 """Plant plausible mistakes in a copy of the oracle source and check that the
 pins in test_oracle_pins.py catch each one (CPU only).
 
-Each mutant is compiled into a temporary library and the pin tests are run
-against it in a child process through ``ORACLE_LIB``; a mutant survives if all
-pins still pass."""
+A mutant of the C++ steps is compiled into a temporary library and the pin
+tests run against it in a child process through ``ORACLE_LIB``.  A mutant of
+the Python composition (``oracle/__init__.py``: the per-sequence split of the
+conv, the zero rows of the row gather, the sequence of a sampled row) goes
+into a copy of the package that ``ORACLE_PKG`` puts first on the child's
+import path.  A mutant survives if all pins still pass."""
 
 import os
 import subprocess
@@ -14,6 +17,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "engram_oracle.cpp")
+PY = os.path.join(ROOT, "oracle", "__init__.py")
 
 MUTANTS = {
     "remap_identity": ("canon[i] = P[x];", "canon[i] = x;"),
@@ -33,8 +37,29 @@ MUTANTS = {
     "conv_history_reversed": ("hist[(int64_t)(w - 1 + tt) * d + c]", "hist[(int64_t)(-tt - 1) * d + c]"),
     "silu_is_sigmoid": ("return x / (1.0 + std::exp(-x));", "return 1.0 / (1.0 + std::exp(-x));"),
     "residual_dropped": ("if (add_residual) r += h[i];", "(void)add_residual;"),
-    "bf16_truncates": ("std::nearbyint(std::ldexp(m, 8))", "std::trunc(std::ldexp(m, 8))"),
 }
+
+PY_MUTANTS = {
+    # one conv over the flat [B*L][d] rows: history leaks from sequence b-1 into b
+    "conv_no_sequence_split": ("        seg = slice(b * L, (b + 1) * L)\n",
+                               "        seg = slice(0, wl.B * L)\n"),
+    # every sequence takes the first sequence's conv history
+    "conv_history_wrong_sequence": ("u[seg] = conv(vt[seg], inp.conv_w, None if hist is None else hist[b])",
+                                    "u[seg] = conv(vt[seg], inp.conv_w, None if hist is None else hist[0])"),
+    "rows_history_wrong_sequence": ("u = conv(seg, inp.conv_w, hist[b])[-1:]",
+                                    "u = conv(seg, inp.conv_w, hist[0])[-1:]"),
+    # an index >= M_j gathers row 0 instead of a zero row
+    "gather_rows_no_zeroing": ("        vals = np.where(ok[:, None], vals, 0)\n", ""),
+    # a sampled row's window taken from the wrong sequence
+    "rows_sequence_index": ("    for p in positions:\n        b, t = divmod(int(p), L)\n",
+                            "    for p in positions:\n        b, t = divmod(int(p), L + 1)\n"),
+}
+
+
+def _run_pins(env):
+    return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                           os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -48,7 +73,30 @@ def test_pins_kill_mutant(name, tmp_path):
     subprocess.check_call(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-shared", "-fPIC",
                            "-o", str(lib), str(mutant_src)])
     env = dict(os.environ, ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    r = _run_pins(env)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_kill_python_mutant(name, tmp_path):
+    import oracle
+    old, new = PY_MUTANTS[name]
+    src = open(PY).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique in the oracle package"
+    pkg = tmp_path / "oracle"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(src.replace(old, new))
+    env = dict(os.environ, ORACLE_PKG=str(tmp_path), ORACLE_LIB=oracle.build())
+    r = _run_pins(env)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    """The copy mechanism itself: the unchanged package passes the pins."""
+    import oracle
+    pkg = tmp_path / "oracle"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(open(PY).read())
+    env = dict(os.environ, ORACLE_PKG=str(tmp_path), ORACLE_LIB=oracle.build())
+    r = _run_pins(env)
+    assert r.returncode == 0, r.stdout[-2000:]

@@ -181,6 +181,22 @@ def test_gather_rows_matches_full_gather(c1):
 
 # ------------------------------------------------------------------ projections
 
+def test_gather_rows_zero_rows_for_invalid_indices():
+    """An index >= M_j, and the invalid-n-gram marker 0xFFFFFFFF, gather a zero
+    row; every other index gathers its table row (numpy indexing)."""
+    M, D, J = 11, 4, 3
+    tables = (np.arange(J * M * D, dtype=np.float64).reshape(J, M, D) + 1.0)
+    idx = np.array([[0, 10, 11], [0xFFFFFFFF, 5, 12], [3, 0xFFFFFFFF, 0], [11, 11, 10]], dtype=np.uint32)
+    got = oracle.gather_rows(idx, np.full(J, M, dtype=np.uint32), lambda j, r: tables[j][r])
+    want = np.zeros((idx.shape[0], J * D))
+    for i in range(idx.shape[0]):
+        for j in range(J):
+            if idx[i, j] < M:
+                want[i, j * D:(j + 1) * D] = tables[j, idx[i, j]]
+    assert np.array_equal(got, want)
+    assert np.count_nonzero(np.all(got.reshape(-1, J, D) == 0, axis=2)) == 6
+
+
 def test_project_matches_numpy_matmul():
     rng = np.random.default_rng(5)
     e = rng.standard_normal((9, 13))
@@ -300,22 +316,6 @@ def test_output_special_cases():
             assert abs(y[t, c] - (vt[t, c] + x / (1 + math.exp(-x)))) < 1e-14
 
 
-# ------------------------------------------------------------------ bf16 rounding
-
-def test_round_bf16_matches_torch_and_ties():
-    import torch
-    rng = np.random.default_rng(14)
-    x32 = (rng.standard_normal(20000) * rng.choice([1e-3, 1.0, 300.0], 20000)).astype(np.float32)
-    want = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
-    assert np.array_equal(oracle.round_bf16(x32.astype(np.float64)), want)
-    # ties to even: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7
-    assert oracle.round_bf16(1.0 + 2.0 ** -8) == 1.0
-    assert oracle.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
-    assert oracle.round_bf16(-(1.0 + 3 * 2.0 ** -8)) == -(1.0 + 2.0 ** -6)
-    # a double just above the tie rounds up (no double rounding through fp32)
-    assert oracle.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -40) == 1.0 + 2.0 ** -7
-
-
 # ------------------------------------------------------------------ whole path
 
 def test_forward_full_c1_properties(c1):
@@ -348,3 +348,61 @@ def test_decode_step_equals_last_prefill_row(c1):
     dec.hidden_rows = lambda rows: inp.hidden_rows(np.asarray(rows) + (wl.T - 1))
     r = oracle.forward_rows(dec, np.array([0]), hist=hist)
     np.testing.assert_allclose(r.y[0], full.y[wl.T - 1], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ batches of sequences
+
+def _one_sequence(inp, b, tables, h_all):
+    """The inputs of sequence b alone, as a workload with B = 1."""
+    import types
+    wl = inp.wl
+    L = wl.T - wl.t_begin
+    one = types.SimpleNamespace(**{k: getattr(inp, k) for k in ("P", "mult", "rows", "Wk", "Wv", "gq", "gk",
+                                                                    "conv_w")})
+    one.wl = wl.replace(B=1)
+    one.tok = inp.tok[b:b + 1]
+    return one, h_all[b * L:(b + 1) * L]
+
+
+@pytest.fixture(scope="module")
+def c1_batch():
+    inp = synth.Inputs(synth.WORKLOADS["c1"].replace(name="c1b3", B=3, T=96, seed=21), gamma="random")
+    return inp, inp.all_tables(), inp.all_hidden()
+
+
+@pytest.mark.parametrize("with_hist", [False, True])
+def test_batch_equals_independent_sequences(c1_batch, with_hist):
+    """The conv is causal within each sequence ("DeepSeek AI II" digest,
+    section "DeepSeek Engram": per-channel causal convolution over a
+    sequence): a batch of three sequences gives, row for row, what three
+    single-sequence runs give, each with its own history (zero or its own
+    conv_state row)."""
+    inp, tables, h_all = c1_batch
+    wl = inp.wl
+    L = wl.T
+    hist = inp.state_rows(np.arange(wl.B)) if with_hist else None
+    batch = oracle.forward_full(inp, add_residual=True, tables=tables, h=h_all, hist=hist)
+    for b in range(wl.B):
+        one, h_b = _one_sequence(inp, b, tables, h_all)
+        r = oracle.forward_full(one, add_residual=True, tables=tables, h=h_b,
+                                hist=None if hist is None else hist[b:b + 1])
+        np.testing.assert_array_equal(batch.y[b * L:(b + 1) * L], r.y)
+        np.testing.assert_array_equal(batch.alpha[b * L:(b + 1) * L], r.alpha)
+    # the sequences differ, so a history leaking across them would show
+    assert not np.allclose(batch.y[:4], batch.y[L:L + 4])
+
+
+@pytest.mark.parametrize("with_hist", [False, True])
+def test_forward_rows_equals_forward_full_batch(c1_batch, with_hist):
+    """forward_rows (one position at a time, its window rebuilt per sequence)
+    against forward_full on B = 3: every sequence's first four and last rows."""
+    inp, tables, h_all = c1_batch
+    wl = inp.wl
+    L = wl.T
+    hist = inp.state_rows(np.arange(wl.B)) if with_hist else None
+    full = oracle.forward_full(inp, add_residual=True, tables=tables, h=h_all, hist=hist)
+    pos = np.array([b * L + t for b in range(wl.B) for t in (0, 1, 2, 3, L - 1)], dtype=np.int64)
+    rows = oracle.forward_rows(inp, pos, add_residual=True, hist=hist)
+    np.testing.assert_allclose(rows.y, full.y[pos], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(rows.alpha, full.alpha[pos], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(rows.vt_win, oracle.vt_windows(full.vt, wl.B, L, wl.w, hist)[pos], rtol=0, atol=1e-15)
