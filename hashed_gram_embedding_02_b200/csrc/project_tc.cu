@@ -18,7 +18,8 @@
 //              32 TMEM lanes = 3 history rows + 29 output rows, so a row's
 //              conv history (rows t-1..t-3) sits in the same warp: v~ =
 //              alpha v is formed per lane and the history arrives by warp
-//              shuffles.  Taps, SiLU and the residual follow and Y is written;
+//              shuffles.  Taps, SiLU and the residual follow (all fp32) and
+//              Y is written;
 //              v never reaches global memory.  Consecutive segments overlap
 //              by 3 rows (116 output rows per 128-row MMA tile).
 //
@@ -49,7 +50,6 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
-#include <cuda_fp16.h>
 
 namespace engram {
 
@@ -85,9 +85,11 @@ struct Geo {
     static constexpr int SMEM_TILES = STAGES * STAGE_BYTES;
     static constexpr int HC = MODE == MODE_KV ? 128 : BN;      // h channels per tile
     static constexpr int H_BYTES = BM * HC * 2;                // h tile, [HC/64][128 rows][128 B] swizzled
-    // tiles | h tile | barriers (1 KB) | per-tile gains [HC] or taps [BN][4] fp32 |
+    // tiles | h tile | barriers (1 KB) | per-tile gains [HC] fp32 or taps |
     // partial hand-over [NPART][128] float4 | slack
-    static constexpr int GG_BYTES = BN * 16;
+    // MODE_VCONV: the gains area and the partial hand-over together hold the
+    // epilogue warps' fp32 taps, 16 warps x 2 phases x BN/16 pairs x 32 bytes
+    static constexpr int GG_BYTES = MODE == MODE_VCONV ? BN * 32 : BN * 16;
     static constexpr int RED_BYTES = NPART * BM * 16;
     static constexpr int SMEM_BYTES = SMEM_TILES + H_BYTES + 1024 + GG_BYTES + RED_BYTES + 1024;
 };
@@ -574,27 +576,24 @@ __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, co
 // channels.  Lane l of warp segment q holds row r0q + l; lanes 0..2 are the
 // history rows of the segment's first output row.  Each of the NPART parts
 // handles BN/NPART channels, 16 at a time, TMEM loads one chunk ahead.
-// v~ = alpha v is formed in fp32 per lane; the conv and SiLU run on channel
-// pairs in fp16x2: the history values travel between lanes as the same
-// fp16 pairs (one shuffle per two channels per shift), the taps are fp16
-// pairs, and SiLU(x) = x/2 + x/2 tanh(x/2) uses the paired hardware tanh.
-// Each term of the tap sum carries a relative rounding of at most about
-// 2^-10, below the bf16 rounding of Y; the skip term v~ and the residual
-// stay fp32.  The taps arrive pre-halved, so the tap sum is already x/2.
-// The fp16 range bounds |v~| and the tap sum by 65504.
-__device__ __forceinline__ uint32_t h2u(__half2 x) { return *reinterpret_cast<uint32_t*>(&x); }
-__device__ __forceinline__ __half2 u2h(uint32_t x) { return *reinterpret_cast<__half2*>(&x); }
-
-__device__ __forceinline__ __half2 tanh_h2(__half2 x) {
-    uint32_t r;
-    asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h2u(x)));
-    return u2h(r);
+// Everything is fp32: v~ = alpha v per lane, the history rows t-1..t-3 by
+// warp shuffles, the tap sum by fused multiply-adds in tap order, and
+// SiLU(x) = x/2 + x/2 tanh(x/2) with the hardware tanh approximation
+// (relative error about 2^-11, below the bf16 rounding of Y).  The taps
+// arrive pre-halved, so the tap sum is already x/2.  Only Y is rounded, once,
+// to bf16.
+__device__ __forceinline__ float tanh_f32(float x) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
+
+__device__ __forceinline__ float mask_f(float x, uint32_t m) { return __uint_as_float(__float_as_uint(x) & m); }
 
 template <int NCH, bool SLOW, bool RES>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
-                                             const uint4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3) {
+                                             const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3) {
     constexpr int H = CONV_W - 1;
     const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
     const bool from_state = SLOW && t < H && p.state;
@@ -616,60 +615,71 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
             const float v0 = a * __uint_as_float(cur[c]), v1 = a * __uint_as_float(cur[c + 1]);
-            const __half2 vh = __floats2half2_rn(v0, v1);
-            const uint32_t u0 = h2u(vh);
-            uint32_t s1 = __shfl_up_sync(0xffffffffu, u0, 1);
-            uint32_t s2 = __shfl_up_sync(0xffffffffu, u0, 2);
-            uint32_t s3 = __shfl_up_sync(0xffffffffu, u0, 3);
+            float s1a = __shfl_up_sync(0xffffffffu, v0, 1), s1b = __shfl_up_sync(0xffffffffu, v1, 1);
+            float s2a = __shfl_up_sync(0xffffffffu, v0, 2), s2b = __shfl_up_sync(0xffffffffu, v1, 2);
+            float s3a = __shfl_up_sync(0xffffffffu, v0, 3), s3b = __shfl_up_sync(0xffffffffu, v1, 3);
             if (!SLOW) {
                 // rows before the sequence start (no conv_state): zero history
-                s1 &= m1;
-                s2 &= m2;
-                s3 &= m3;
+                s1a = mask_f(s1a, m1);
+                s1b = mask_f(s1b, m1);
+                s2a = mask_f(s2a, m2);
+                s2b = mask_f(s2b, m2);
+                s3a = mask_f(s3a, m3);
+                s3b = mask_f(s3b, m3);
             }
             if (SLOW && t < H) {
                 // history before the slab start: conv_state (zero without one);
                 // the row t-k comes from state row H-k+t
-                uint32_t ps[H] = {0u, 0u, 0u};
+                float2 ps[H] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 if (from_state) {
-                    const int ch = n0 + cl + c;
+                    const int chn = n0 + cl + c;
 #pragma unroll
                     for (int k = 1; k <= H; ++k)
                         if (t < k) {
                             const int hr = H - k + t;            // history row holding v~_{t-k}
-                            float2 x;
                             if (p.state_tr) {                     // [3][d][B]: consecutive lanes, consecutive b
-                                const float* st = p.state + ((int64_t)hr * p.d + ch) * p.B + b;
-                                x = make_float2(__ldg(st), __ldg(st + p.B));
+                                const float* st = p.state + ((int64_t)hr * p.d + chn) * p.B + b;
+                                ps[k - 1] = make_float2(__ldg(st), __ldg(st + p.B));
                             } else {
-                                x = __ldg(reinterpret_cast<const float2*>(p.state + (b * H + hr) * p.d + ch));
+                                ps[k - 1] = __ldg(reinterpret_cast<const float2*>(p.state + (b * H + hr) * p.d + chn));
                             }
-                            ps[k - 1] = h2u(__floats2half2_rn(x.x, x.y));
                         }
                 }
-                if (t < 1) s1 = ps[0];
-                if (t < 2) s2 = ps[1];
-                s3 = ps[2];
+                if (t < 1) {
+                    s1a = ps[0].x;
+                    s1b = ps[0].y;
+                }
+                if (t < 2) {
+                    s2a = ps[1].x;
+                    s2b = ps[1].y;
+                }
+                s3a = ps[2].x;
+                s3b = ps[2].y;
             }
             if (write_state) {
                 const int hr = t - (p.L - H);
-                const int ch = n0 + cl + c;
+                const int chn = n0 + cl + c;
                 if (p.state_tr) {
-                    float* sn = p.state_next + ((int64_t)hr * p.d + ch) * p.B + b;
+                    float* sn = p.state_next + ((int64_t)hr * p.d + chn) * p.B + b;
                     sn[0] = v0;
                     sn[p.B] = v1;
                 } else {
-                    *reinterpret_cast<float2*>(p.state_next + (b * H + hr) * p.d + ch) = make_float2(v0, v1);
+                    *reinterpret_cast<float2*>(p.state_next + (b * H + hr) * p.d + chn) = make_float2(v0, v1);
                 }
             }
-            const uint4 w = s_cw[(cl + c) >> 1];          // halved taps c_0..c_3 of the channel pair
-            __half2 hx = __hmul2(u2h(w.x), vh);
-            hx = __hfma2(u2h(w.y), u2h(s1), hx);
-            hx = __hfma2(u2h(w.z), u2h(s2), hx);
-            hx = __hfma2(u2h(w.w), u2h(s3), hx);
-            const float2 sl = __half22float2(__hfma2(hx, tanh_h2(hx), hx));
-            o[c] = (RES ? v0 + hv[c] : v0) + sl.x;
-            o[c + 1] = (RES ? v1 + hv[c + 1] : v1) + sl.y;
+            // halved taps of the channel pair: (c_0 ch0, c_0 ch1, c_1 ch0, c_1 ch1), (c_2 .., c_3 ..)
+            const float4 wa = s_cw[(cl + c)], wb = s_cw[(cl + c) + 1];
+            float hx0 = wa.x * v0, hx1 = wa.y * v1;
+            hx0 = fmaf(wa.z, s1a, hx0);
+            hx1 = fmaf(wa.w, s1b, hx1);
+            hx0 = fmaf(wb.x, s2a, hx0);
+            hx1 = fmaf(wb.y, s2b, hx1);
+            hx0 = fmaf(wb.z, s3a, hx0);
+            hx1 = fmaf(wb.w, s3b, hx1);
+            const float sl0 = fmaf(hx0, tanh_f32(hx0), hx0);
+            const float sl1 = fmaf(hx1, tanh_f32(hx1), hx1);
+            o[c] = (RES ? v0 + hv[c] : v0) + sl0;
+            o[c + 1] = (RES ? v1 + hv[c + 1] : v1) + sl1;
         }
         // Y replaces this row's h in the staged tile (each element of the tile
         // is read and written by one lane only); the warp stores its block
@@ -700,18 +710,18 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
         t = (int)(r - b * p.L);
     }
     const int n0 = nt * BN;
-    // the warp's own taps (both phases), halved, as fp16 pairs: slot
-    // [warp][phase][pair] x {c_0, c_1, c_2, c_3} of (channel 2m, 2m+1); staged
-    // in phase 0 from the values loaded a tile ahead, read by this warp only
+    // the warp's own taps (both phases), halved, fp32: slot [warp][phase][pair]
+    // holds two float4, (c_0, c_0', c_1, c_1') and (c_2, c_2', c_3, c_3') of
+    // channels (2m, 2m+1); staged in phase 0 from the values loaded a tile
+    // ahead, read by this warp only
     constexpr int VPP = BN / (4 * NPART);
-    uint4* s_tw = reinterpret_cast<uint4*>(s_taps) + (size_t)(q * NPART + part) * 2 * 16;
+    float4* s_tw = reinterpret_cast<float4*>(s_taps) + (size_t)(q * NPART + part) * 2 * VPP * 2;
     if (phase == 0) {
         const int k = lane & 15, ph = lane >> 4;
         if (k < VPP) {
             const float4 w0 = pre.w0, w1 = pre.w1;
-            s_tw[ph * 16 + k] = make_uint4(
-                h2u(__floats2half2_rn(0.5f * w0.x, 0.5f * w1.x)), h2u(__floats2half2_rn(0.5f * w0.y, 0.5f * w1.y)),
-                h2u(__floats2half2_rn(0.5f * w0.z, 0.5f * w1.z)), h2u(__floats2half2_rn(0.5f * w0.w, 0.5f * w1.w)));
+            s_tw[(ph * VPP + k) * 2] = make_float4(0.5f * w0.x, 0.5f * w1.x, 0.5f * w0.y, 0.5f * w1.y);
+            s_tw[(ph * VPP + k) * 2 + 1] = make_float4(0.5f * w0.z, 0.5f * w1.z, 0.5f * w0.w, 0.5f * w1.w);
         }
         __syncwarp();
     }
@@ -726,8 +736,8 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     // warp, and with it the CTA's next tiles, for about 15 us.
     const bool slow_row = out_row && ((t < H && p.state) || (p.state_next && t >= p.L - H));
     const uint32_t m1 = t >= 1 ? ~0u : 0u, m2 = t >= 2 ? ~0u : 0u, m3 = t >= 3 ? ~0u : 0u;
-    // indexed by tile-local pair: this warp's slot, shifted to the phase's first pair
-    const uint4* cw = s_tw + phase * 16 - (cbeg >> 1);
+    // indexed by tile-local channel (even): this warp's slot, shifted to the phase's first pair
+    const float4* cw = s_tw + phase * VPP * 2 - cbeg;
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
         if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
@@ -1079,7 +1089,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 for (int phase = 0; phase < 2; ++phase) {
                     ok = wait_bounded(&sb->hfull_v[phase], (uint32_t)tc & 1u, sb, p.status);
                     if (!__all_sync(0xffffffffu, ok)) break;
-                    epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, reinterpret_cast<float*>(s_red),
+                    epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg,
                                        phase, a_row, pre);
                     if (phase == 0 && has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
                     if (phase == 1) tc_fence_before();

@@ -30,8 +30,8 @@
  *   storage   bf16 configurations store e and Y as bf16; k, v, alpha and
  *             the conv history stay fp32 (v is stored, in fp32, only where
  *             the gate and conv are not fused into the projection).  The
- *             fused path evaluates the tap sum and SiLU on fp16 pairs, so
- *             |v~| and the tap sum must stay within the fp16 range.
+ *             gate, the tap sum, SiLU and the residual add are fp32
+ *             arithmetic on every path; Y is rounded once, when stored.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are caller-owned DEVICE memory unless stated; the

@@ -36,10 +36,8 @@ def bf16_bound(y_ref: np.ndarray, vt_win: np.ndarray, cw: np.ndarray) -> np.ndar
     """Elementwise bound on |Y_gpu - Y_oracle| for the bf16 path.
 
     Sources: (1) Y is rounded once to bf16 (half an ulp, 2^-8 relative);
-    (2) the fused epilogue evaluates the tap sum and SiLU on fp16 pairs:
-    each history value and tap is rounded to fp16 (2^-11 relative), each
-    product and partial sum rounds to fp16, and the paired tanh
-    approximation errs by about 2^-10.7 relative; together well under
+    (2) the fused epilogue evaluates the tap sum in fp32 and SiLU through the
+    hardware tanh approximation (relative error about 2^-11), both far under
     2^-8 of sum_j |c_j| |v~_{t-j}|.  The accumulation order of v (fp32)
     differs from the oracle's (fp64) only in the last bits.  An error of
     relative size r in v~_{t-j} reaches Y_t through the skip (j = 0, weight 1)

@@ -208,6 +208,43 @@ def test_forward_full_small(eb, name, add_residual):
     _check_y(wl, to_np(y), ref.y, win, inp.conv_w)
 
 
+@pytest.mark.parametrize("name", ["b3", "b5"])
+@pytest.mark.parametrize("state", [False, True])
+def test_forward_large_magnitude(eb, name, state):
+    """Values far outside the test distribution: W_V scaled by 2^18 (|v~| and
+    the tap sums beyond 65504, the fp16 range) and h by 2^6 with
+    the residual.  Both scalings are powers of two, so the bf16 inputs stay
+    exact and the oracle sees the same numbers.  Y must stay finite and within
+    the relative bound (one bf16 rounding of Y plus the conv inputs' terms);
+    an absolute 2e-2 has no meaning at these magnitudes."""
+    wl = SMALL[name]
+    inp = synth.Inputs(wl, gamma="random")
+    inp.Wv = inp.Wv * np.float32(2.0 ** 18)
+    di = DeviceInputs(inp)
+    assert torch.equal(di.Wv.float().cpu(), torch.from_numpy(inp.Wv))
+    di.h = di.h * 64.0
+    h_host = inp.all_hidden() * 64.0
+    hist = None
+    st_dev = None
+    if state:
+        hist = inp.state_rows(np.arange(wl.B)) * 2.0 ** 14
+        st_dev = torch.from_numpy(hist.astype(np.float32)).cuda().contiguous()
+    ctx = eb.Engram(config_for(inp, eb))
+    y, alpha = _run_forward(eb, ctx, di, add_residual=True, state=st_dev)
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    ref = oracle.forward_full(inp, add_residual=True, h=h_host, hist=hist)
+    # beyond the fp16 range, both the gated values and the tap sums
+    assert np.max(np.abs(ref.vt)) > 65504 and np.max(np.abs(ref.u)) > 65504
+    win = oracle.vt_windows(ref.vt, wl.B, wl.T - wl.t_begin, wl.w, hist)
+    yg = to_np(y)
+    assert np.all(np.isfinite(yg))
+    np.testing.assert_allclose(to_np(alpha), ref.alpha, rtol=0, atol=2e-6)
+    err = np.abs(yg - ref.y)
+    bound = bf16_bound(ref.y, win, inp.conv_w)
+    bad = err > bound
+    assert not bad.any(), (int(bad.sum()), float(err.max()), float((err - bound).max()))
+
+
 @pytest.mark.parametrize("name", ["c2", "c3"])
 def test_forward_full_size_sampled(eb, name):
     wl = W[name]
