@@ -3,10 +3,16 @@
 
 One step = the whole forward (remap + hash, gather, W_K/W_V projections with
 gate partials, gate + causal conv) over one batch of the workload, through
-the C ABI.  Default workload: B=4 sequences x 4096 tokens, 16 tables of
-1000003 x 64 bf16 (about 2 GB), d_mem 1024, d 2560, conv width 4.
+the C ABI.  Default workload: the largest single-GPU prefill, B=8 sequences x
+4096 tokens, 16 tables of 2781271 x 128 bf16 (11.4 GB), d_mem 2048, d 2560,
+conv width 4.  --workload c2 runs B=4 x 4096 with 16 tables of 1000003 x 64
+(d_mem 1024), c4 the decode shape, c5 the host-memory tier.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload c3] [--batch B --table-rows M]
+
+--batch and --table-rows shrink the workload (fewer sequences, smaller prime
+tables) for ncu captures that must stay a few GB in size.
 
 Under torchrun every rank runs an independent replica (no collective on the
 data path: the forward shards by sequence); timing is the max over ranks.
@@ -175,9 +181,14 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
+    # c2, before the value epilogue's conv math moved to fp32 (profiles/launches_c2.md)
     ("c2", "vconv_tc"): ("ece15e492f5dcb2f", 123190528 + 28159232),
     ("c2", "gate_k_tc"): ("ece15e492f5dcb2f", 122743552 + 86016),
     ("c2", "retrieve"): ("8c46903b0c8d286e", 28940800 + 632832),
+    # c3 kernels on 2 sequences and 499979-row tables (profiles/dram_c3_small.md)
+    ("c3-B2-M499979", "vconv_tc"): ("59d2794a31cc0db6", 86297856 + 2050304),
+    ("c3-B2-M499979", "gate_k_tc"): ("59d2794a31cc0db6", 86043136 + 130048),
+    ("c3-B2-M499979", "retrieve"): ("8c46903b0c8d286e", 29667072 + 480512),
 }
 
 
@@ -238,10 +249,36 @@ def job_tokens_per_s(tokens_per_rank: int, world: int, ms: float) -> float:
 
 # ---------------------------------------------------------------- reference arm
 
+def selected_workload(args):
+    """The workload named on the command line, with --batch / --table-rows applied."""
+    wl = synth.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.replace(name=f"{wl.name}-B{args.batch}", B=args.batch)
+    if args.table_rows:
+        if not synth._is_prime(args.table_rows):
+            raise SystemExit(f"--table-rows {args.table_rows} is not prime")
+        wl = wl.replace(name=f"{wl.name}-M{args.table_rows}", M=args.table_rows)
+    return wl
+
+
+def host_cpu():
+    """The host's CPU model and logical core count (reported beside the oracle's rate)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_cores": os.cpu_count()}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl = synth.WORKLOADS[args.workload]
+    wl = selected_workload(args)
     n = args.ref_tokens
     if n <= 0:
         # size each step so that warm-up + timed steps take about 90 s
@@ -258,7 +295,8 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": describe(wl), "sample": f"first {n} tokens of sequence 0 per step"},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {n} tokens of sequence 0, single-threaded fp64 C++ oracle"},
+                         "sample": f"first {n} tokens of sequence 0, single-threaded fp64 C++ oracle",
+                         **host_cpu()},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -413,8 +451,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--cpu-tokens", type=int, default=2048, help="oracle sample for cpu_baseline")
+    ap.add_argument("--workload", default="c3", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0, help="override B (0: the workload's)")
+    ap.add_argument("--table-rows", type=int, default=0, help="override the rows per table (a prime; 0: the workload's)")
+    ap.add_argument("--cpu-tokens", type=int, default=4096,
+                    help="oracle sample for cpu_baseline (default: one full 4096-token sequence)")
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="oracle sample per reference step (0: sized so the run takes about 90 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -442,7 +483,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    wl = synth.WORKLOADS[args.workload]
+    wl = selected_workload(args)
     wl = replica_workload(wl, rank, world)
     if wl.host_tables:
         run_host_tier(args, wl, rank, world, dev)
@@ -531,7 +572,7 @@ def main():
                         "frac": rate / 1e12 / tf_burst}
         else:
             kern[nm] = {"ms": t, "bound": "hbm", "achieved": rate / 1e9, "unit": "GB/s", "frac": rate / 1e9 / hbm}
-        kern[nm]["traffic"] = captured_traffic(args.workload, nm)
+        kern[nm]["traffic"] = captured_traffic(wl.name, nm)
     dominant = max(kms, key=kms.get)
     dk = kern.get(dominant, {})
     roofline = {"kernel": dominant, "bound": dk.get("bound"), "achieved": dk.get("achieved"),
@@ -575,7 +616,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec = oracle_sample_time(wl, args.cpu_tokens)
         cpu = {"value": args.cpu_tokens / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {args.cpu_tokens} tokens of sequence 0 ({sec:.1f} s), single-threaded fp64 C++"}
+               "sample": f"first {args.cpu_tokens} tokens of sequence 0 ({sec:.1f} s), single-threaded fp64 C++",
+               **host_cpu()}
 
     if world > 1:
         barrier()
