@@ -278,3 +278,78 @@ def vt_windows(vt: np.ndarray, B: int, L: int, w: int, hist: Optional[np.ndarray
             elif hist is not None:
                 win[r, j] = hist[b][w - 1 + t - j]
     return win
+
+
+def forward_multibranch(branches, add_residual: bool = False, eps: float = 1e-6,
+                        hist: Optional[np.ndarray] = None, tables: Optional[np.ndarray] = None,
+                        h: Optional[np.ndarray] = None) -> Result:
+    """Multi-branch Engram ("DeepSeek AI II" digest, section "DeepSeek
+    Engram", the multi-branch paragraphs): the M branches share the tables
+    and W_V, branch m has its own W_K^(m), hidden state h^(m) and gate
+    alpha^(m) = sigmoid(<RMSNorm(h^(m)), RMSNorm(W_K^(m) e)> / sqrt(d)), and
+    u^(m) = alpha^(m) * (W_V e).  Each branch's gated value then goes through
+    the single-branch conv and output (shared taps, a history per branch).
+
+    branches[m] holds branch m's W_K, gains and hidden rows; branches[0] also
+    the shared tokens, tables, W_V and conv taps.  hist: [M][B][w-1][d] or
+    None; h: [M][n][d] or None (then each branch's all_hidden())."""
+    inp = branches[0]
+    wl = inp.wl
+    M = len(branches)
+    canon, _ = remap(inp.tok, inp.P)
+    idx, _ = hash_ids(canon, wl.Vc, wl.orders, wl.K, inp.mult, inp.rows, wl.t_begin)
+    tables = inp.all_tables() if tables is None else tables
+    e = gather(idx, inp.rows, tables)
+    v = project(e, inp.Wv)
+    L = wl.T - wl.t_begin
+    ys, alphas, vts = [], [], []
+    for m, br in enumerate(branches):
+        hm = br.all_hidden() if h is None else h[m]
+        k = project(e, br.Wk)
+        alpha = gate(hm, k, br.gq, br.gk, eps)
+        vt = alpha[:, None] * v
+        u = np.empty_like(vt)
+        for b in range(wl.B):
+            seg = slice(b * L, (b + 1) * L)
+            u[seg] = conv(vt[seg], inp.conv_w, None if hist is None else hist[m][b])
+        ys.append(output(vt, u, hm, add_residual))
+        alphas.append(alpha)
+        vts.append(vt)
+    return Result(idx=idx, e=e, v=v, alpha=np.stack(alphas), vt=np.stack(vts), y=np.stack(ys))
+
+
+def table_grad(idx: np.ndarray, rows: np.ndarray, de: np.ndarray, D: int):
+    """Gradient of the tables from dL/de ("DeepSeek AI II" digest, section
+    "DeepSeek Engram", training): e_t concatenates E_j[idx_j(t)], so the
+    gradient of table j's row r is the sum of slice j of dL/de_t over the
+    lookups with idx_j(t) = r.  Returns (sorted distinct global rows
+    sum_{i<j} M_i + r, fp64 [U][D] gradients); invalid indices contribute
+    nothing."""
+    idx = np.asarray(idx, dtype=np.uint32)
+    n, J = idx.shape
+    de = np.asarray(de, dtype=np.float64).reshape(n, J, D)
+    off = np.concatenate([[0], np.cumsum(np.asarray(rows, dtype=np.int64)[:-1])])
+    r = idx.astype(np.int64)
+    valid = r < np.asarray(rows, dtype=np.int64)[None, :]
+    keys = (r + off[None, :])[valid]
+    uniq, inv = np.unique(keys, return_inverse=True)
+    grad = np.zeros((len(uniq), D))
+    np.add.at(grad, inv, de[valid])
+    return uniq, grad
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """Values of FP8 E4M3 codes, from the format's definition (OCP 8-bit
+    floating point, E4M3): bit 7 the sign, bits 6-3 the exponent with bias 7,
+    bits 2-0 the mantissa; exponent 0 holds the subnormals m/8 * 2^-6; the
+    code with exponent 15 and mantissa 7 is NaN; there are no infinities
+    (largest finite value 448).  The tables and weights of the FP8 path are
+    such codes ("DeepSeek AI II" digest, section "DeepSeek Engram": the fused
+    projections run as one dense FP8 GEMM)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag

@@ -83,7 +83,8 @@ class Workload:
 
     @property
     def elem_bytes(self) -> int:
-        return 4 if self.dtype == "f32" else 2
+        """bytes of a table element (h and Y are bf16 for "bf16" and "fp8")"""
+        return {"f32": 4, "bf16": 2, "fp8": 1}[self.dtype]
 
     @property
     def w_sd(self) -> float:
@@ -115,6 +116,28 @@ WORKLOADS: Dict[str, Workload] = {
                    orders=(2, 3), K=8, M=48828139, D=128, d=2560, w=4, dtype="bf16", seed=4,
                    host_tables=True),
 }
+
+
+# FP8 (E4M3) inputs: the tables are stored as E4M3 codes of value / FP8_TABLE_SCALE
+# (the Irwin-Hall tails, 3.46 sigma, stay below the format's largest value, 448),
+# each weight row as E4M3 codes of W[c] / s_W[c] with s_W[c] = max |W[c]| / 448.
+FP8_MAX = 448.0
+
+
+def fp8_table_scale(wl: "Workload") -> float:
+    return float(np.float32(3.5 * wl.table_sd / FP8_MAX))
+
+
+def fp8_codes(x: np.ndarray) -> np.ndarray:
+    """uint8 E4M3 codes of fp32 values (torch's round-to-nearest conversion)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def fp8_values(codes: np.ndarray) -> np.ndarray:
+    """fp32 values of E4M3 codes (torch's conversion)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).to(torch.float32).numpy()
 
 
 def _is_prime(n: int) -> bool:
@@ -300,10 +323,31 @@ class Inputs:
         if wl.dtype == "bf16":
             self.Wk = to_bf16_values(self.Wk)
             self.Wv = to_bf16_values(self.Wv)
+        self.k_scale = self.v_scale = None
+        if wl.dtype == "fp8":
+            # codes per row, and the per-channel scale the GEMM epilogue applies:
+            # table scale x row scale; Wk / Wv hold scale[c] * decoded codes, so that
+            # W e over the decoded table values is the device's k and v
+            te = fp8_table_scale(wl)
+            self.Wk_codes, self.k_scale = self._fp8_rows(self.Wk, te)
+            self.Wv_codes, self.v_scale = self._fp8_rows(self.Wv, te)
+            self.Wk = self.k_scale.astype(np.float64)[:, None] * fp8_values(self.Wk_codes).astype(np.float64)
+            self.Wv = self.v_scale.astype(np.float64)[:, None] * fp8_values(self.Wv_codes).astype(np.float64)
+
+    @staticmethod
+    def _fp8_rows(W: np.ndarray, table_scale: float):
+        W = np.asarray(W, dtype=np.float32)
+        s_w = (np.max(np.abs(W), axis=1) / np.float32(FP8_MAX)).astype(np.float32)
+        codes = fp8_codes(W / s_w[:, None])
+        return codes, (s_w * np.float32(table_scale)).astype(np.float32)
 
     # -- rows of the big tensors, computed on the host on demand
     def table_rows(self, j: int, rows: np.ndarray) -> np.ndarray:
+        """Table values as the path sees them: bf16-rounded, or, for FP8, the
+        decoded E4M3 values (the table scale is in k_scale / v_scale)."""
         v = table_rows_np(self.wl, j, rows, self.M)
+        if self.wl.dtype == "fp8":
+            return fp8_values(fp8_codes(v / np.float32(fp8_table_scale(self.wl))))
         return to_bf16_values(v) if self.wl.dtype == "bf16" else v
 
     def hidden_rows(self, rows: np.ndarray) -> np.ndarray:
@@ -312,7 +356,7 @@ class Inputs:
         d = self.wl.d
         base = rows[:, None] * d + np.arange(d, dtype=np.int64)[None, :]
         v = normal_np(self.wl.seed, TAG_HIDDEN, base.reshape(-1), 1.0).reshape(len(rows), d)
-        return to_bf16_values(v) if self.wl.dtype == "bf16" else v
+        return v if self.wl.dtype == "f32" else to_bf16_values(v)
 
     def state_rows(self, b: np.ndarray) -> np.ndarray:
         """Conv history [len(b)][w-1][d] fp32 used by decode tests (scale 0.25)."""
@@ -322,7 +366,7 @@ class Inputs:
         return normal_np(self.wl.seed, TAG_STATE, base.reshape(-1), 0.25).reshape(len(b), self.wl.w - 1, self.wl.d)
 
     def all_tables(self) -> np.ndarray:
-        """[J][M][D] fp32 values (small workloads only)."""
+        """[J][M][D] fp32 values (small workloads only; FP8: the decoded codes)."""
         wl = self.wl
         out = np.empty((wl.J, self.M, wl.D), dtype=np.float32)
         for j in range(wl.J):
@@ -333,16 +377,39 @@ class Inputs:
         return self.hidden_rows(np.arange(self.wl.n_tok))
 
     # -- device tensors (torch); tables and h generated on the device
+    def _table_dtype(self):
+        import torch
+        return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8}[self.wl.dtype]
+
+    def _to_table(self, x):
+        """fp32 generator values -> the stored table element (FP8: E4M3 codes)"""
+        import torch
+        if self.wl.dtype == "fp8":
+            return (x / float(np.float32(fp8_table_scale(self.wl)))).to(torch.float8_e4m3fn).view(torch.uint8)
+        return x.to(self._table_dtype())
+
     def device_tables(self, device, chunk: int = 1 << 27):
         import torch
         wl = self.wl
         n = wl.J * self.M * wl.D
-        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
-        out = torch.empty(n, dtype=tdt, device=device)
+        out = torch.empty(n, dtype=self._table_dtype(), device=device)
         for s in range(0, n, chunk):
             e = min(n, s + chunk)
-            out[s:e] = normal_torch(wl.seed, TAG_TABLES, s, e - s, wl.table_sd, device).to(tdt)
+            out[s:e] = self._to_table(normal_torch(wl.seed, TAG_TABLES, s, e - s, wl.table_sd, device))
         return out.view(wl.J, self.M, wl.D)
+
+    def device_table_range(self, first_row: int, n_rows: int, out, chunk: int = 1 << 27):
+        """Rows [first_row, first_row + n_rows) of the J tables numbered back to
+        back (table j's row r is row j * M + r) into ``out`` ([n_rows][D] on a
+        device): the same values as device_tables, for one shard of them."""
+        wl = self.wl
+        flat = out.view(-1)
+        n = n_rows * wl.D
+        for s in range(0, n, chunk):
+            e = min(n, s + chunk)
+            flat[s:e] = self._to_table(normal_torch(wl.seed, TAG_TABLES, first_row * wl.D + s, e - s, wl.table_sd,
+                                                    out.device))
+        return out
 
     def host_tables(self, device, chunk: int = 1 << 27, pin: bool = False):
         """[J][M][D] tables in host memory (torch CPU tensor), the same values
@@ -350,18 +417,17 @@ class Inputs:
         import torch
         wl = self.wl
         n = wl.J * self.M * wl.D
-        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
-        out = torch.empty(n, dtype=tdt, pin_memory=pin)
+        out = torch.empty(n, dtype=self._table_dtype(), pin_memory=pin)
         for s in range(0, n, chunk):
             e = min(n, s + chunk)
-            out[s:e].copy_(normal_torch(wl.seed, TAG_TABLES, s, e - s, wl.table_sd, device).to(tdt))
+            out[s:e].copy_(self._to_table(normal_torch(wl.seed, TAG_TABLES, s, e - s, wl.table_sd, device)))
         return out.view(wl.J, self.M, wl.D)
 
     def device_hidden(self, device, chunk: int = 1 << 27):
         import torch
         wl = self.wl
         n = wl.n_tok * wl.d
-        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16     # h: bf16 for bf16 and FP8
         out = torch.empty(n, dtype=tdt, device=device)
         for s in range(0, n, chunk):
             e = min(n, s + chunk)
@@ -375,18 +441,35 @@ class Inputs:
         return normal_torch(wl.seed, TAG_STATE, 0, n, 0.25, device).view(wl.B, wl.w - 1, wl.d)
 
     def device_dense(self, device):
-        """dict of small device tensors: tok, P, Wk, Wv, conv_w, gq, gk."""
+        """dict of small device tensors: tok, P, Wk, Wv, conv_w, gq, gk (and, for
+        FP8, Wk/Wv as E4M3 codes plus k_scale, v_scale)."""
         import torch
         tdt = torch.float32 if self.wl.dtype == "f32" else torch.bfloat16
+        if self.wl.dtype == "fp8":
+            w = {"Wk": torch.from_numpy(self.Wk_codes).to(device), "Wv": torch.from_numpy(self.Wv_codes).to(device),
+                 "k_scale": torch.from_numpy(self.k_scale).to(device),
+                 "v_scale": torch.from_numpy(self.v_scale).to(device)}
+        else:
+            w = {"Wk": torch.from_numpy(self.Wk).to(tdt).to(device), "Wv": torch.from_numpy(self.Wv).to(tdt).to(device),
+                 "k_scale": None, "v_scale": None}
         return {
             "tok": torch.from_numpy(self.tok).to(device),
             "P": torch.from_numpy(self.P).to(device),
-            "Wk": torch.from_numpy(self.Wk).to(tdt).to(device),
-            "Wv": torch.from_numpy(self.Wv).to(tdt).to(device),
+            **w,
             "conv_w": torch.from_numpy(self.conv_w).to(device),
             "gq": torch.from_numpy(self.gq).to(device),
             "gk": torch.from_numpy(self.gk).to(device),
         }
+
+
+def branch_inputs(inp: "Inputs", m: int, gamma: str = "random") -> "Inputs":
+    """Inputs of branch m of a multi-branch module: its own key projection,
+    RMSNorm gains and hidden states, drawn from a seed of their own; branch 0
+    is ``inp`` itself.  The tokens, tables, W_V and conv taps of the module
+    are branch 0's (the caller uses those of ``inp``)."""
+    if m == 0:
+        return inp
+    return Inputs(inp.wl.replace(seed=inp.wl.seed * 31 + 977 * m), gamma=gamma, M=inp.M)
 
 
 def to_bf16_values(x: np.ndarray) -> np.ndarray:

@@ -41,8 +41,10 @@ MUTANTS = {
 
 PY_MUTANTS = {
     # one conv over the flat [B*L][d] rows: history leaks from sequence b-1 into b
-    "conv_no_sequence_split": ("        seg = slice(b * L, (b + 1) * L)\n",
-                               "        seg = slice(0, wl.B * L)\n"),
+    "conv_no_sequence_split": ("    for b in range(wl.B):\n        seg = slice(b * L, (b + 1) * L)\n",
+                               "    for b in range(wl.B):\n        seg = slice(0, wl.B * L)\n"),
+    "multibranch_no_sequence_split": ("        for b in range(wl.B):\n            seg = slice(b * L, (b + 1) * L)\n",
+                                      "        for b in range(wl.B):\n            seg = slice(0, wl.B * L)\n"),
     # every sequence takes the first sequence's conv history
     "conv_history_wrong_sequence": ("u[seg] = conv(vt[seg], inp.conv_w, None if hist is None else hist[b])",
                                     "u[seg] = conv(vt[seg], inp.conv_w, None if hist is None else hist[0])"),
@@ -50,6 +52,19 @@ PY_MUTANTS = {
                                     "u = conv(seg, inp.conv_w, hist[0])[-1:]"),
     # an index >= M_j gathers row 0 instead of a zero row
     "gather_rows_no_zeroing": ("        vals = np.where(ok[:, None], vals, 0)\n", ""),
+    # every branch gated with branch 0's key projection
+    "multibranch_shared_key": ("        k = project(e, br.Wk)\n", "        k = project(e, branches[0].Wk)\n"),
+    # every branch convolved with branch 0's history
+    "multibranch_history_of_branch0": ("None if hist is None else hist[m][b])", "None if hist is None else hist[0][b])"),
+    # the table gradient counts invalid lookups as row 0's
+    "table_grad_keeps_invalid": ("    valid = r < np.asarray(rows, dtype=np.int64)[None, :]\n",
+                                 "    valid = r < np.iinfo(np.int64).max\n"),
+    # the table gradient without the table offsets (tables' rows collide)
+    "table_grad_no_offset": ("    keys = (r + off[None, :])[valid]\n", "    keys = r[valid]\n"),
+    # E4M3 exponent bias 8 instead of 7
+    "e4m3_bias": ("np.exp2((e - 7).astype(np.float64))", "np.exp2((e - 8).astype(np.float64))"),
+    # subnormals without the 2^-6 scale
+    "e4m3_subnormal": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
     # a sampled row's window taken from the wrong sequence
     "rows_sequence_index": ("    for p in positions:\n        b, t = divmod(int(p), L)\n",
                             "    for p in positions:\n        b, t = divmod(int(p), L + 1)\n"),

@@ -406,3 +406,109 @@ def test_forward_rows_equals_forward_full_batch(c1_batch, with_hist):
     np.testing.assert_allclose(rows.y, full.y[pos], rtol=0, atol=1e-12)
     np.testing.assert_allclose(rows.alpha, full.alpha[pos], rtol=0, atol=1e-15)
     np.testing.assert_allclose(rows.vt_win, oracle.vt_windows(full.vt, wl.B, L, wl.w, hist)[pos], rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ multi-branch
+
+@pytest.fixture(scope="module")
+def mb():
+    inp = synth.Inputs(synth.WORKLOADS["c1"].replace(name="mb", B=2, T=80, seed=23), gamma="random")
+    branches = [synth.branch_inputs(inp, m) for m in range(3)]
+    return inp, branches, inp.all_tables()
+
+
+def _hybrid(inp, br):
+    """branch br's key, gains and hidden rows on inp's tokens, tables, W_V and taps."""
+    import types
+    one = types.SimpleNamespace(**{k: getattr(inp, k) for k in ("wl", "tok", "P", "mult", "rows", "Wv", "conv_w")})
+    one.Wk, one.gq, one.gk = br.Wk, br.gq, br.gk
+    one.hidden_rows = br.hidden_rows
+    one.table_rows = inp.table_rows
+    return one
+
+
+def test_multibranch_one_branch_is_the_single_branch_forward(mb):
+    inp, branches, tables = mb
+    r = oracle.forward_multibranch(branches[:1], add_residual=True, tables=tables)
+    f = oracle.forward_full(inp, add_residual=True, tables=tables)
+    np.testing.assert_array_equal(r.y[0], f.y)
+    np.testing.assert_array_equal(r.alpha[0], f.alpha)
+
+
+@pytest.mark.parametrize("with_hist", [False, True])
+def test_multibranch_branch_m_uses_its_own_key_and_hidden(mb, with_hist):
+    """Branch m equals the single-branch module run with W_K^(m), its gains and
+    h^(m) on the shared tables, W_V and taps (the pages: one W_V, M W_K, a gate
+    per branch applied to the shared value)."""
+    inp, branches, tables = mb
+    M = len(branches)
+    hist = np.stack([b.state_rows(np.arange(inp.wl.B)) for b in branches]) if with_hist else None
+    r = oracle.forward_multibranch(branches, add_residual=True, tables=tables, hist=hist)
+    assert r.y.shape == (M, inp.wl.n_tok, inp.wl.d)
+    for m in range(M):
+        f = oracle.forward_full(_hybrid(inp, branches[m]), add_residual=True, tables=tables,
+                                h=branches[m].all_hidden(), hist=None if hist is None else hist[m])
+        np.testing.assert_array_equal(r.y[m], f.y)
+        np.testing.assert_array_equal(r.alpha[m], f.alpha)
+    # the branches differ, and they share v: v~^(m) / alpha^(m) is the same vector
+    assert not np.allclose(r.alpha[0], r.alpha[1])
+    np.testing.assert_allclose(r.vt[1] / r.alpha[1][:, None], r.vt[2] / r.alpha[2][:, None], rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------------------------------ table backward
+
+def test_table_grad_brute_force():
+    """Against a plain loop over the lookups, on a case small enough to read:
+    three tables of 5 rows, rows touched several times, one invalid index."""
+    D = 2
+    rows = np.array([5, 5, 5], dtype=np.uint32)
+    idx = np.array([[0, 4, 2], [0, 1, 2], [3, 0xFFFFFFFF, 2], [0, 4, 7]], dtype=np.uint32)
+    de = np.arange(idx.shape[0] * 3 * D, dtype=np.float64).reshape(idx.shape[0], 3 * D) + 1.0
+    want = {}
+    for t in range(idx.shape[0]):
+        for j in range(3):
+            if idx[t, j] < 5:
+                key = j * 5 + int(idx[t, j])
+                want[key] = want.get(key, 0) + de[t, j * D:(j + 1) * D]
+    keys, grad = oracle.table_grad(idx, rows, de, D)
+    assert keys.tolist() == sorted(want)
+    for k, g in zip(keys, grad):
+        np.testing.assert_array_equal(g, want[int(k)])
+    # table 0 row 0 three times: 1+2, 7+8, 19+20 -> [1+7+19, 2+8+20]
+    np.testing.assert_array_equal(grad[list(keys).index(0)], [27.0, 30.0])
+
+
+def test_table_grad_conserves_the_total(c1):
+    """The gradients of all rows add up to the sum of every valid slice of
+    dL/de (nothing lost, nothing counted twice)."""
+    inp, _, idx = c1
+    wl = inp.wl
+    rng = np.random.default_rng(3)
+    de = rng.standard_normal((wl.n_tok, wl.d_mem))
+    keys, grad = oracle.table_grad(idx, inp.rows, de, wl.D)
+    assert len(np.unique(keys)) == len(keys)
+    valid = (idx.astype(np.int64) < inp.rows[None, :].astype(np.int64))
+    total = de.reshape(wl.n_tok, wl.J, wl.D)[valid].sum(axis=0)
+    np.testing.assert_allclose(grad.sum(axis=0), total, rtol=0, atol=1e-9)
+    assert len(keys) == len(np.unique((idx.astype(np.int64) + (np.arange(wl.J) * wl.M)[None, :])[valid]))
+
+
+# ------------------------------------------------------------------ FP8 E4M3 codes
+
+def test_decode_e4m3_hand_values_and_all_codes():
+    assert oracle.decode_e4m3(np.array([0x38]))[0] == 1.0          # exponent 7 = bias, mantissa 0
+    assert oracle.decode_e4m3(np.array([0xB8]))[0] == -1.0
+    assert oracle.decode_e4m3(np.array([0x7E]))[0] == 448.0        # 1.75 * 2^8, the largest finite value
+    assert oracle.decode_e4m3(np.array([0x01]))[0] == 2.0 ** -9    # smallest subnormal, 1/8 * 2^-6
+    assert oracle.decode_e4m3(np.array([0x08]))[0] == 2.0 ** -6    # smallest normal
+    assert oracle.decode_e4m3(np.array([0x3C]))[0] == 1.5
+    assert np.isnan(oracle.decode_e4m3(np.array([0x7F, 0xFF]))).all()
+    assert oracle.decode_e4m3(np.array([0x80]))[0] == 0.0
+    # every code against torch's float8_e4m3fn conversion (a library routine)
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.decode_e4m3(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
