@@ -189,6 +189,10 @@ CAPTURED_TRAFFIC = {
     ("c3-B2-M499979", "vconv_tc"): ("59d2794a31cc0db6", 86297856 + 2050304),
     ("c3-B2-M499979", "gate_k_tc"): ("59d2794a31cc0db6", 86043136 + 130048),
     ("c3-B2-M499979", "retrieve"): ("8c46903b0c8d286e", 29667072 + 480512),
+    # c3 at full size, mean of the five timed steps' launches (profiles/launches_c3.md)
+    ("c3", "vconv_tc"): ("3341a08adf82f52a", 314786253 + 123717939),
+    ("c3", "gate_k_tc"): ("3341a08adf82f52a", 312558797 + 7296461),
+    ("c3", "retrieve"): ("7fd2473de48a2d96", 115571456 + 81190400),
 }
 
 
@@ -258,6 +262,8 @@ def selected_workload(args):
         if not synth._is_prime(args.table_rows):
             raise SystemExit(f"--table-rows {args.table_rows} is not prime")
         wl = wl.replace(name=f"{wl.name}-M{args.table_rows}", M=args.table_rows)
+    if getattr(args, "fp8", False):
+        wl = wl.replace(name=f"{wl.name}-fp8", dtype="fp8")
     return wl
 
 
@@ -316,9 +322,13 @@ def run_host_tier(args, wl, rank, world, dev):
     """Tables in host memory: per step, hash -> dedupe (GPU) -> stand-in
     layer GEMM [n x 2560] x [2560 x 10240] on the compute stream while the
     host packs the distinct rows and copies them on a side stream -> staged
-    gather -> projections, gate and conv.  The tables are shrunk to the
-    largest prime row count that fits in 30 % of the available host memory
-    (the stated 200 GB does not fit), and the line states the size."""
+    gather -> projections, gate and conv.  Every step takes a fresh token
+    batch (its own seed), so rows found in the HBM hot-row cache are rows an
+    earlier batch admitted, not the same batch again.  Before timing, the
+    cache is filled by --cache-warm batches (retrieval only).  The tables are
+    shrunk to the largest prime row count that fits in 30 % of the available
+    host memory (the stated 200 GB does not fit), and the line states the
+    size."""
     import torch
     import torch.distributed as dist
 
@@ -339,6 +349,9 @@ def run_host_tier(args, wl, rank, world, dev):
     eng = eb.Engram(cfg, B=wl.B, L=wl.T)
     n_threads = max(1, min(16, (os.cpu_count() or 2) - 2))
     tier = eb.HostTier(eng, host, max_lookups=n * wl.J, n_threads=n_threads)
+    cache_rows = args.cache_rows
+    if cache_rows > 0:
+        tier.enable_cache(cache_rows, min_count=2)
     idx = torch.empty(n, wl.J, dtype=torch.int32, device=dev)
     e = torch.empty(n, wl.d_mem, dtype=torch.bfloat16, device=dev)
     y = torch.empty(n, wl.d, dtype=torch.bfloat16, device=dev)
@@ -350,9 +363,18 @@ def run_host_tier(args, wl, rank, world, dev):
     stream = torch.cuda.current_stream()
     side = torch.cuda.Stream(priority=-1)
     stats = []
+    cstats = []
+    batch_no = [0]
 
-    def engram_part(with_layer: bool, ev_fetch=None):
-        eb.engram_hash(eng.ctx, dd["tok"], dd["P"], wl.B, wl.T, wl.T, 0, idx)
+    def next_tokens():
+        # a fresh seeded Zipf batch of the same shape for every call
+        k = batch_no[0]
+        batch_no[0] += 1
+        return torch.from_numpy(synth.zipf_tokens(wl.replace(seed=wl.seed + 1000 + k))).to(dev, non_blocking=True)
+
+    def engram_part(with_layer: bool, ev_fetch=None, tok=None, full=True):
+        tok = next_tokens() if tok is None else tok
+        eb.engram_hash(eng.ctx, tok, dd["P"], wl.B, wl.T, wl.T, 0, idx)
         tier.dedupe(idx, n)
         if with_layer:
             torch.matmul(x_layer, w_layer)                      # the preceding layer's work
@@ -362,8 +384,9 @@ def run_host_tier(args, wl, rank, world, dev):
         if ev_fetch is not None:
             ev_fetch[1].record(side)
         tier.gather(n, e)
-        eb.engram_gate_conv(eng.ctx, e, h, dd["Wk"], dd["Wv"], dd["gq"], dd["gk"], dd["conv_w"], wl.B, wl.T, None,
-                            y, None, 1, ws, ws_bytes)
+        if full:
+            eb.engram_gate_conv(eng.ctx, e, h, dd["Wk"], dd["Wv"], dd["gq"], dd["gk"], dd["conv_w"], wl.B, wl.T,
+                                None, y, None, 1, ws, ws_bytes)
         return n_unique
 
     def timed(fn, K):
@@ -378,6 +401,8 @@ def run_host_tier(args, wl, rank, world, dev):
         torch.cuda.synchronize()
         return float(np.mean([a.elapsed_time(b) for a, b in out]))
 
+    for _ in range(args.cache_warm if cache_rows > 0 else 0):
+        engram_part(False, full=False)
     for _ in range(args.warmup):
         engram_part(True)
     torch.cuda.synchronize()
@@ -385,11 +410,13 @@ def run_host_tier(args, wl, rank, world, dev):
     if st != eb.ENGRAM_OK:
         raise RuntimeError(f"device status {st} flags {flags:#x} after warm-up")
     K = args.steps
+    toks = [next_tokens() for _ in range(K)]
     fetch_ev = []
 
     def step():
         ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        stats.append(engram_part(True, ev))
+        stats.append(engram_part(True, ev, tok=toks[len(fetch_ev)]))
+        cstats.append(tier.cache_stats())
         fetch_ev.append(ev)
 
     if world > 1:
@@ -400,10 +427,24 @@ def run_host_tier(args, wl, rank, world, dev):
     step_ms = max_over_ranks(step_ms, world, dev)
     fetch_ms = float(np.mean([a.elapsed_time(b) for a, b in fetch_ev]))
     layer_ms = timed(lambda: torch.matmul(x_layer, w_layer), max(3, K // 2))
-    alone_ms = timed(lambda: engram_part(False), max(3, K // 2))
+    toks_alone = [next_tokens() for _ in range(max(3, K // 2))]
+    it_alone = iter(toks_alone)
+    alone_ms = timed(lambda: engram_part(False, tok=next(it_alone)), len(toks_alone))
     tstats = tier.stats()
     uniq = float(np.mean(stats))
     fetch_bytes = uniq * wl.D * 2
+    cache = None
+    if cache_rows > 0:
+        cached_rows = float(np.mean([c["cached_rows"] for c in cstats]))
+        cached_lookups = float(np.mean([c["cached_lookups"] for c in cstats]))
+        lookups = float(np.mean([c["lookups"] for c in cstats]))
+        cache = {"capacity_rows": cache_rows, "capacity_gb": cache_rows * wl.D * 2 / 1e9, "admit_min_count": 2,
+                 "warm_batches": args.cache_warm, "resident_rows_last": cstats[-1]["resident"],
+                 "lookup_hit_rate": cached_lookups / lookups,
+                 "distinct_rows_per_step": uniq + cached_rows, "cached_rows_per_step": cached_rows,
+                 "row_hit_rate": cached_rows / (uniq + cached_rows),
+                 "pcie_bytes_saved_per_step": cached_rows * wl.D * 2,
+                 "pcie_mb_per_step_without_cache": (uniq + cached_rows) * wl.D * 2 / 1e6}
     # pinned host -> device copy peak of this machine, for the roofline
     probe_h = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
     probe_d = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -420,27 +461,62 @@ def run_host_tier(args, wl, rank, world, dev):
         "metric": METRIC, "value": job_tokens_per_s(n, world, step_ms), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic: seeded Zipf tokens, counter-based N(0,s^2) tables (host memory)/hidden/weights",
+        "data": "synthetic: seeded Zipf tokens (a fresh batch every step), counter-based N(0,s^2) tables (host "
+                "memory)/hidden/weights",
         "config": {"workload": describe(wl), "B": wl.B, "seq_len": wl.T, "tokens_per_step": n * world,
                    "host_tables_gb": wl.J * wl.M * wl.D * 2 / 1e9,
                    "table_sizing": f"rows per table = largest prime fitting 30% of MemAvailable ({budget / 1e9:.1f} GB)",
-                   "step": "hash, dedupe, stand-in layer GEMM 32768x2560x10240 (cuBLAS) overlapping the host "
-                           "packing and side-stream copies, staged gather, projections+gate+conv",
+                   "step": "hash, dedupe (against the HBM hot-row cache), stand-in layer GEMM 32768x2560x10240 "
+                           "(cuBLAS) overlapping the host packing and side-stream copies, staged gather, cache "
+                           "admission, projections+gate+conv",
                    "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write outside the events)"},
         "roofline": {"kernel": "host fetch (pack + PCIe copy)", "bound": "pcie", "achieved": achieved,
                      "peak": h2d_peak, "unit": "GB/s", "frac": achieved / h2d_peak, "traffic": None,
                      "peak_source": "pinned 256 MiB H2D copy measured in this run",
-                     "algorithmic": f"distinct rows x {wl.D * 2} B = {fetch_bytes / 1e6:.1f} MB per step"},
-        "host_tier": {"lookups": n * wl.J, "distinct_rows": uniq, "fetch_mb": fetch_bytes / 1e6,
+                     "algorithmic": f"fetched distinct rows x {wl.D * 2} B = {fetch_bytes / 1e6:.1f} MB per step"},
+        "host_tier": {"lookups": n * wl.J, "fetched_rows": uniq, "fetch_mb": fetch_bytes / 1e6,
                       "fetch_ms": fetch_ms, "last_fetch": tstats, "pack_threads": n_threads,
                       "layer_gemm_ms": layer_ms, "engram_alone_ms": alone_ms, "step_ms": step_ms,
                       "overhead_over_layer": (step_ms - layer_ms) / layer_ms, "table_generation_s": gen_s},
-        # per step: hash, dedupe insert, dedupe slot, staged gather, key pass,
-        # value pass (the stand-in GEMM and the memsets are not this library's)
-        "cpu_baseline": None, "e2e": None, "gpu_launches": 6 * K, "clocks": clocks.summary(),
+        "hot_row_cache": cache,
+        # per step: hash, dedupe insert, dedupe slot, staged gather, cache
+        # admission (with the cache), key pass, value pass (the stand-in GEMM
+        # and the memsets are not this library's)
+        "cpu_baseline": None, "e2e": None, "gpu_launches": (7 if cache_rows > 0 else 6) * K,
+        "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)
+
+
+def e2e_host(args, eng, inp, dd, tables, h, state, wl, tdt, es, n, K, flush, stream, world, dev):
+    """The same step end to end through the C ABI with HOST buffers:
+    engram_forward_host copies the ids and h in from pinned host memory and Y
+    back out, chunk by chunk, overlapped with the compute; all of it inside
+    the events."""
+    import torch
+    tok_h = torch.from_numpy(inp.tok).pin_memory()
+    h_h = h.cpu().pin_memory()
+    y_h = torch.empty(n, wl.d, dtype=tdt).pin_memory()
+    Ke = max(3, min(K, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    for i in range(Ke + 3):
+        flush.zero_()
+        if i >= 3:
+            e2e_ev[i - 3][0].record(stream)
+        eng.forward_host(tok_h, dd["P"], tables, h_h, dd["Wk"], dd["Wv"], dd["conv_w"], y_h, t_begin=wl.t_begin,
+                         gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
+        if i >= 3:
+            e2e_ev[i - 3][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])), world, dev)
+    ids_copied = wl.B * (wl.T - max(0, wl.t_begin - (max(wl.orders) - 1)))
+    e2e = {"value": job_tokens_per_s(n, world, e2e_ms), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(ids_copied * 4 + h_h.numel() * es),
+           "d2h_bytes_per_step": int(y_h.numel() * es), "ms_per_step": e2e_ms,
+           "path": "engram_forward_host: pinned host ids + h in, Y out to pinned host, chunked and overlapped"}
+
+    return e2e
 
 
 # ---------------------------------------------------------------- our arm
@@ -459,6 +535,18 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="oracle sample per reference step (0: sized so the run takes about 90 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--branches", type=int, default=1,
+                    help="multi-branch module: M residual branches (own W_K, h, gate and Y each; shared tables, "
+                         "W_V and conv)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="tables, W_K and W_V as FP8 E4M3 codes: the projections as FP8 tcgen05 GEMMs")
+    ap.add_argument("--sharded", action="store_true",
+                    help="split the tables over the ranks (rank r holds shard r); each rank's retrieval reads "
+                         "the other ranks' rows over NVLink (CUDA IPC mappings)")
+    ap.add_argument("--cache-rows", type=int, default=1 << 22,
+                    help="host-memory workload: rows of the HBM hot-row cache (0: none)")
+    ap.add_argument("--cache-warm", type=int, default=32,
+                    help="host-memory workload: batches that fill the hot-row cache before timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -492,23 +580,61 @@ def main():
         return
     inp = synth.Inputs(wl)
     dd = inp.device_dense(dev)
-    tables = inp.device_tables(dev)
     h = inp.device_hidden(dev)
-    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    es = 2 if wl.dtype == "bf16" else 4
+    tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16      # h and Y
+    es = wl.elem_bytes                                                 # tables, e
     cfg = eb.make_config(orders=wl.orders, heads=wl.K, rows=[int(x) for x in inp.rows], mult=inp.mult,
                          row_dim=wl.D, hidden=wl.d, conv_width=wl.w, vocab=wl.V, canon_vocab=wl.Vc,
-                         dtype=eb.ENGRAM_BF16 if wl.dtype == "bf16" else eb.ENGRAM_F32)
+                         dtype={"bf16": eb.ENGRAM_BF16, "f32": eb.ENGRAM_F32, "fp8": eb.ENGRAM_FP8}[wl.dtype])
     eng = eb.Engram(cfg, B=wl.B, L=wl.T - wl.t_begin)
     n = wl.n_tok
-    y = torch.empty(n, wl.d, dtype=tdt, device=dev)
-    state = (torch.zeros(wl.B, wl.w - 1, wl.d, dtype=torch.float32, device=dev) if wl.t_begin > 0 else None)
+    sharded = None
+    tables = None
+    if args.sharded:
+        # every rank's tables are the same seeded values (the workload's own
+        # seed, before the per-replica seeds), split by global row
+        tab_inp = synth.Inputs(selected_workload(args))
+
+        def all_gather(obj):
+            every = [None] * world
+            dist.all_gather_object(every, obj)
+            return every
+        sharded = eb.ShardedTables(eng, world, rank, wl.D, tdt, dev,
+                                   lambda first, cnt, out: tab_inp.device_table_range(first, cnt, out),
+                                   all_gather=all_gather)
+    else:
+        tables = inp.device_tables(dev)
+    M = args.branches
+    mb = M > 1 or wl.dtype == "fp8"          # the multi-branch entry point (FP8 takes its scales)
+    if mb:
+        if args.sharded:
+            raise SystemExit("--branches / --fp8 and --sharded are separate modes")
+        branches = [synth.branch_inputs(inp, m) for m in range(M)]
+        bdd = [dd] + [b.device_dense(dev) for b in branches[1:]]
+        h = torch.stack([h] + [b.device_hidden(dev) for b in branches[1:]]).contiguous()
+        Wk_mb = torch.stack([x["Wk"] for x in bdd]).contiguous()
+        ks_mb = torch.stack([x["k_scale"] for x in bdd]).contiguous() if wl.dtype == "fp8" else None
+        gq_mb = torch.stack([x["gq"] for x in bdd]).contiguous()
+        gk_mb = torch.stack([x["gk"] for x in bdd]).contiguous()
+        y = torch.empty(M, n, wl.d, dtype=tdt, device=dev)
+    else:
+        y = torch.empty(n, wl.d, dtype=tdt, device=dev)
+    state = (torch.zeros(M, wl.B, wl.w - 1, wl.d, dtype=torch.float32, device=dev).squeeze(0)
+             if wl.t_begin > 0 else None)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        eng.forward(dd["tok"], dd["P"], tables, h, dd["Wk"], dd["Wv"], dd["conv_w"], y, t_begin=wl.t_begin,
-                    gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
+        if mb:
+            eng.forward_multibranch(dd["tok"], dd["P"], tables, h, Wk_mb, dd["Wv"], dd["conv_w"], y,
+                                    t_begin=wl.t_begin, gq=gq_mb, gk=gk_mb, k_scale=ks_mb, v_scale=dd["v_scale"],
+                                    conv_state=state, add_residual=True)
+        elif sharded is not None:
+            eng.forward_sharded(dd["tok"], dd["P"], sharded.ptrs, h, dd["Wk"], dd["Wv"], dd["conv_w"], y,
+                                t_begin=wl.t_begin, gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
+        else:
+            eng.forward(dd["tok"], dd["P"], tables, h, dd["Wk"], dd["Wv"], dd["conv_w"], y, t_begin=wl.t_begin,
+                        gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
 
     for _ in range(args.warmup):
         step()
@@ -549,6 +675,9 @@ def main():
     per_step_launches = len(names)
 
     hbm, tf_burst, tf_sust, peak_src = _peaks()
+    if wl.dtype == "fp8":
+        # FP8 contraction: the bf16 peak times the nominal dense ratio 4.5 / 2.25
+        tf_burst, tf_sust, peak_src = 2.0 * tf_burst, 2.0 * tf_sust, peak_src + " bf16 x 2 (FP8/bf16 nominal)"
     G = (wl.d + 127) // 128
     L = wl.T - wl.t_begin
     pass_flops = 2.0 * n * wl.d_mem * wl.d                      # one of the two projection passes
@@ -557,7 +686,9 @@ def main():
         # remap + n-grams + hash + gather in one kernel: ids in, indices out,
         # table rows in, e_cat out
         "retrieve": ("hbm", n * (4.0 + wl.J * 4) + wl.B * 4.0 * min(wl.T, 3) + 2.0 * n * wl.d_mem * es, "bytes"),
-        "gate_k_tc": ("tensor", pass_flops, "flop"),
+        "retrieve_sharded": ("hbm", n * (4.0 + wl.J * 4) + wl.B * 4.0 * min(wl.T, 3) + 2.0 * n * wl.d_mem * es,
+                             "bytes"),
+        "gate_k_tc": ("tensor", M * pass_flops, "flop"),
         "vconv_tc": ("tensor", pass_flops, "flop"),
         "state_merge": ("hbm", wl.B * (wl.w - 1) * wl.d * 8.0, "bytes"),
     }
@@ -579,34 +710,21 @@ def main():
                 "peak": tf_burst if dk.get("bound") == "tensor" else hbm, "unit": dk.get("unit"),
                 "frac": dk.get("frac"), "traffic": dk.get("traffic"),
                 "peak_source": f"{peak_src} " + ("bf16 burst" if dk.get("bound") == "tensor" else "HBM copy"),
-                "algorithmic": (f"2*n*d_mem*d = {pass_flops:.4g} FLOP per launch" if dk.get("bound") == "tensor"
-                                else f"{work.get(dominant, (0, 0))[1]:.4g} bytes per launch")}
-    gather_gbs = kern["retrieve"]["achieved"] if "retrieve" in kern else None
+                "algorithmic": (f"{work[dominant][1]:.4g} FLOP per launch (2*n*d_mem*d per projection)"
+                                if dk.get("bound") == "tensor" else f"{work.get(dominant, (0, 0))[1]:.4g} bytes per launch")}
+    rname = "retrieve_sharded" if sharded is not None else "retrieve"
+    gather_gbs = kern[rname]["achieved"] if rname in kern else None
     gather_bytes = work["retrieve"][1]
 
     # ---- end to end through the C ABI with HOST buffers: engram_forward_host
     # copies the ids and h in from pinned host memory and Y back out, chunk by
     # chunk, overlapped with the compute; all of it inside the events
-    tok_h = torch.from_numpy(inp.tok).pin_memory()
-    h_h = h.cpu().pin_memory()
-    y_h = torch.empty(n, wl.d, dtype=tdt).pin_memory()
-    Ke = max(3, min(K, 50))
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
-    for i in range(Ke + 3):
-        flush.zero_()
-        if i >= 3:
-            e2e_ev[i - 3][0].record(stream)
-        eng.forward_host(tok_h, dd["P"], tables, h_h, dd["Wk"], dd["Wv"], dd["conv_w"], y_h, t_begin=wl.t_begin,
-                         gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
-        if i >= 3:
-            e2e_ev[i - 3][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])), world, dev)
-    ids_copied = wl.B * (wl.T - max(0, wl.t_begin - (max(wl.orders) - 1)))
-    e2e = {"value": job_tokens_per_s(n, world, e2e_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(ids_copied * 4 + h_h.numel() * es),
-           "d2h_bytes_per_step": int(y_h.numel() * es), "ms_per_step": e2e_ms,
-           "path": "engram_forward_host: pinned host ids + h in, Y out to pinned host, chunked and overlapped"}
+    e2e = None
+    if sharded is None and not mb:
+        e2e = e2e_host(args, eng, inp, dd, tables, h, state, wl, tdt, es, n, K, flush, stream, world, dev)
+    elif sharded is not None:
+        barrier()                  # every rank is done reading the others' shards
+        sharded.close()
 
     st, flags = eng.status()
     if st != eb.ENGRAM_OK:
@@ -627,9 +745,12 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.dtype, "data": "synthetic: seeded Zipf tokens, counter-based N(0,s^2) tables/hidden/weights",
-        "config": {"workload": describe(wl), "B": wl.B, "seq_len": wl.T, "tokens_per_step": n * world,
-                   "parallelism": f"replicas x{world} (no collective)",
+        "dtype": "fp8-e4m3 (h, Y bf16)" if wl.dtype == "fp8" else wl.dtype,
+        "data": "synthetic: seeded Zipf tokens, counter-based N(0,s^2) tables/hidden/weights",
+        "config": {"workload": describe(wl) + (f", {M} branches" if M > 1 else ""), "B": wl.B, "seq_len": wl.T,
+                   "tokens_per_step": n * world,
+                   "parallelism": (f"tables sharded over {world} GPUs, rows read over NVLink by the retrieval"
+                                   if sharded is not None else f"replicas x{world} (no collective)"),
                    "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write outside the events)"},
         "roofline": roofline,
         "gather": {"kernel": "retrieve (remap + n-grams + hash + gather)", "achieved_gbs": gather_gbs,

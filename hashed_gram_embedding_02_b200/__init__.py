@@ -11,14 +11,19 @@ from __future__ import annotations
 from typing import Optional
 
 from .binding import (  # noqa: F401  (re-exported C ABI names)
-    ENGRAM_BF16, ENGRAM_F32, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
+    ENGRAM_BF16, ENGRAM_F32, ENGRAM_FP8, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_TOKEN,
     ENGRAM_E_CUDA, ENGRAM_E_DEVICE, ENGRAM_E_HOST, ENGRAM_E_INVAL, ENGRAM_E_NOMEM, ENGRAM_E_TIMEOUT,
     ENGRAM_E_UNSUPPORTED,
     ENGRAM_INVALID_INDEX, ENGRAM_OK, EXPORTS, LIB_PATH, EngramError, engram_config, engram_conv, engram_create,
     ENGRAM_NOALLOC_SCRATCH_BYTES, engram_destroy, engram_device_status, engram_forward, engram_forward_noalloc,
     engram_forward_host, engram_gate_conv, engram_gather, engram_gather_staged, engram_hash, engram_host_dedupe,
     engram_host_fetch, engram_host_tier_create, engram_host_tier_destroy, engram_host_tier_stats,
-    engram_host_workspace_bytes, engram_pack_rows, engram_debug_stall_next,
+    engram_host_workspace_bytes, engram_pack_rows, engram_debug_stall_next, engram_host_tier_debug,
+    ENGRAM_INJECT_LIST_WAIT, ENGRAM_INJECT_PACK_ABANDON, engram_host_cache_enable, engram_host_cache_reset,
+    engram_host_cache_stats, engram_shard_range, engram_forward_sharded, engram_ipc_export, engram_ipc_open,
+    engram_ipc_close, ENGRAM_IPC_HANDLE_BYTES, ENGRAM_MAX_SHARDS, engram_multibranch_workspace_bytes,
+    engram_forward_multibranch, ENGRAM_MAX_BRANCHES, engram_table_grad_workspace_bytes, engram_table_grad,
+    engram_table_sgd,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 
@@ -67,6 +72,33 @@ class Engram:
                        conv_state, y, alpha_out, add_residual, self.workspace, self.workspace_bytes, stream)
         return y
 
+    def forward_multibranch(self, tok, P, tables, h, Wk, Wv, conv_w, y, *, t_begin: int = 0, gq=None, gk=None,
+                            k_scale=None, v_scale=None, conv_state=None, alpha_out=None, add_residual: bool = False,
+                            stream=None):
+        """M-branch forward: h [M][n][d], Wk [M][d][d_mem], gq/gk [M][d],
+        conv_state [M][B][w-1][d], y [M][n][d], alpha_out [M][n]."""
+        import torch
+        M = h.shape[0]
+        B, T = tok.shape[0], tok.shape[1]
+        need = engram_multibranch_workspace_bytes(self.ctx, M, B, T - t_begin)
+        if need > getattr(self, "mb_workspace_bytes", 0):
+            self.mb_workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self.mb_workspace_bytes = need
+        engram_forward_multibranch(self.ctx, M, tok, B, T, tok.stride(0), t_begin, P, tables, h, Wk, Wv, gq, gk,
+                                   k_scale, v_scale, conv_w, conv_state, y, alpha_out, add_residual, self.mb_workspace,
+                                   self.mb_workspace_bytes, stream)
+        return y
+
+    def forward_sharded(self, tok, P, shard_ptrs, h, Wk, Wv, conv_w, y, *, t_begin: int = 0, gq=None, gk=None,
+                        conv_state=None, alpha_out=None, add_residual: bool = False, stream=None):
+        """The forward with the tables split into shards (device pointers
+        valid on this GPU, in shard order: ShardedTables.ptrs)."""
+        B, T = tok.shape[0], tok.shape[1]
+        self.reserve(B, T - t_begin)
+        engram_forward_sharded(self.ctx, tok, B, T, tok.stride(0), t_begin, P, shard_ptrs, h, Wk, Wv, gq, gk, conv_w,
+                               conv_state, y, alpha_out, add_residual, self.workspace, self.workspace_bytes, stream)
+        return y
+
     def forward_host(self, tok_host, P, tables, h_host, Wk, Wv, conv_w, y_host, *, t_begin: int = 0, gq=None,
                      gk=None, conv_state=None, add_residual: bool = False, chunk_rows: int = 0, stream=None):
         """The forward with tok, h and y in host memory (pinned CPU tensors
@@ -82,6 +114,21 @@ class Engram:
                             conv_w, conv_state, y_host, add_residual, chunk_rows, self.host_workspace,
                             self.host_workspace_bytes, stream)
         return y_host
+
+    def table_grad(self, idx, d_e, stream=None):
+        """Sparse gradient of the tables from dL/de: (rows [U] int64 global
+        rows, grad [U][D] fp32), U read back from the device (a sync)."""
+        import torch
+        n_tok = idx.shape[0]
+        n = max(1, n_tok * idx.shape[1])
+        need = engram_table_grad_workspace_bytes(self.ctx, n_tok)
+        ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        rows = torch.empty(n, dtype=torch.int64, device=self.device)
+        grad = torch.empty(n, self.cfg.row_dim, dtype=torch.float32, device=self.device)
+        cnt = torch.zeros(1, dtype=torch.int64, device=self.device)
+        engram_table_grad(self.ctx, idx, n_tok, d_e, rows, grad, cnt, ws, need, stream)
+        U = int(cnt.item())
+        return rows[:U], grad[:U], cnt
 
     def status(self, stream=None):
         return engram_device_status(self.ctx, stream)
@@ -119,3 +166,69 @@ class HostTier:
 
     def stats(self):
         return engram_host_tier_stats(self.tier)
+
+    def enable_cache(self, capacity_rows: int, min_count: int = 2):
+        engram_host_cache_enable(self.tier, capacity_rows, min_count)
+
+    def reset_cache(self, stream=None):
+        engram_host_cache_reset(self.tier, stream)
+
+    def cache_stats(self):
+        return engram_host_cache_stats(self.tier)
+
+    def debug(self, inject: int, wait_limit_s: float):
+        engram_host_tier_debug(self.tier, inject, wait_limit_s)
+
+
+def exchange_shards(local_ptr: int, rank: int, world: int, all_gather, export=None, open_=None):
+    """Shard pointers valid on this rank's GPU for every rank's shard.
+
+    One process per GPU; rank r holds shard r at the device pointer
+    ``local_ptr``.  Each rank exports its shard (an IPC handle and offset),
+    ``all_gather(obj) -> [obj of rank 0, ..., obj of rank world-1]`` collects
+    every rank's export (``torch.distributed.all_gather_object`` in a job),
+    and each rank maps the others' shards into its own address space.
+    Returns (pointers in shard order, mapping bases to close later).  The
+    export/open functions default to the library's IPC calls; the host logic
+    is the same with any pair."""
+    export = engram_ipc_export if export is None else export
+    open_ = engram_ipc_open if open_ is None else open_
+    mine = export(local_ptr) if world > 1 else None
+    every = all_gather(mine) if world > 1 else [mine]
+    if len(every) != world:
+        raise RuntimeError(f"expected {world} shard exports, got {len(every)}")
+    ptrs, bases = [], []
+    for g in range(world):
+        if g == rank:
+            ptrs.append(int(local_ptr))
+            continue
+        handle, offset = every[g]
+        ptr, base = open_(handle, offset)
+        ptrs.append(ptr)
+        bases.append(base)
+    return ptrs, bases
+
+
+class ShardedTables:
+    """This rank's shard of the tables (rank r of ``world`` holds shard r, the
+    global rows ``engram_shard_range`` gives it) and the pointers of every
+    shard on this rank's GPU.  ``fill(first_row, n_rows, out)`` writes the
+    shard's rows into ``out`` ([n_rows][D] on the device).  Mappings of
+    other ranks' shards are closed by :meth:`close`; all ranks must keep
+    their shard alive until every rank is done with it (a barrier)."""
+
+    def __init__(self, engram: "Engram", world: int, rank: int, row_dim: int, dtype, device, fill, all_gather=None,
+                 export=None, open_=None, close=None):
+        import torch
+        self.first, self.rows = engram_shard_range(engram.ctx, world, rank)
+        self.local = torch.empty(max(1, self.rows), row_dim, dtype=dtype, device=device)
+        if self.rows:
+            fill(self.first, self.rows, self.local[: self.rows])
+        torch.cuda.synchronize(device)
+        self._close = engram_ipc_close if close is None else close
+        self.ptrs, self._bases = exchange_shards(self.local.data_ptr(), rank, world, all_gather, export, open_)
+
+    def close(self):
+        for b in self._bases:
+            self._close(b)
+        self._bases = []

@@ -25,8 +25,9 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 ENGRAM_OK, ENGRAM_E_INVAL, ENGRAM_E_CUDA, ENGRAM_E_NOMEM, ENGRAM_E_UNSUPPORTED, ENGRAM_E_TIMEOUT, \
     ENGRAM_E_HOST, ENGRAM_E_DEVICE = range(8)
-ENGRAM_F32, ENGRAM_BF16 = 0, 1
+ENGRAM_F32, ENGRAM_BF16, ENGRAM_FP8 = 0, 1, 2
 ENGRAM_ERR_TOKEN, ENGRAM_ERR_CANON, ENGRAM_ERR_INDEX, ENGRAM_ERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+ENGRAM_INJECT_LIST_WAIT, ENGRAM_INJECT_PACK_ABANDON = 0x1, 0x2
 ENGRAM_INVALID_INDEX = 0xFFFFFFFF
 ENGRAM_MAX_TABLES = 32
 ENGRAM_PART_GROUP = 128
@@ -37,7 +38,14 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_er
            "engram_gather", "engram_project", "engram_conv", "engram_gate_conv", "engram_forward",
            "engram_forward_noalloc", "engram_host_workspace_bytes", "engram_forward_host", "engram_host_tier_create",
            "engram_host_tier_destroy", "engram_host_dedupe", "engram_host_fetch", "engram_gather_staged",
-           "engram_host_tier_stats", "engram_pack_rows", "engram_debug_stall_next")
+           "engram_host_tier_stats", "engram_pack_rows", "engram_debug_stall_next", "engram_host_tier_debug",
+           "engram_host_cache_enable", "engram_host_cache_reset", "engram_host_cache_stats",
+           "engram_shard_range", "engram_forward_sharded", "engram_ipc_export", "engram_ipc_open", "engram_ipc_close",
+           "engram_multibranch_workspace_bytes", "engram_forward_multibranch", "engram_table_grad_workspace_bytes",
+           "engram_table_grad", "engram_table_sgd")
+ENGRAM_MAX_BRANCHES = 4
+ENGRAM_IPC_HANDLE_BYTES = 64
+ENGRAM_MAX_SHARDS = 16
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -97,6 +105,22 @@ _sigs = {
     "engram_host_tier_stats": ([_vp, ctypes.c_void_p], _st),
     "engram_pack_rows": ([_vp, _i64, _sz, _vp, _i64, _vp, _i32], _st),
     "engram_debug_stall_next": ([_vp], _st),
+    "engram_host_tier_debug": ([_vp, ctypes.c_uint32, ctypes.c_double], _st),
+    "engram_host_cache_enable": ([_vp, _i64, _i32], _st),
+    "engram_host_cache_reset": ([_vp, _vp], _st),
+    "engram_host_cache_stats": ([_vp, ctypes.c_void_p], _st),
+    "engram_shard_range": ([_vp, _i32, _i32, ctypes.POINTER(_i64), ctypes.POINTER(_i64)], _st),
+    "engram_multibranch_workspace_bytes": ([_vp, _i32, _i32, _i32], _sz),
+    "engram_table_grad_workspace_bytes": ([_vp, _i64], _sz),
+    "engram_table_grad": ([_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _st),
+    "engram_table_sgd": ([_vp, _vp, _vp, _vp, _i64, _vp, ctypes.c_float, _vp], _st),
+    "engram_forward_multibranch": ([_vp, _i32, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp], _st),
+    "engram_forward_sharded": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, ctypes.POINTER(_vp), _i32, _vp, _vp, _vp, _vp,
+                                _vp, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp], _st),
+    "engram_ipc_export": ([_vp, _vp, ctypes.POINTER(ctypes.c_uint64)], _st),
+    "engram_ipc_open": ([_vp, ctypes.c_uint64, ctypes.POINTER(_vp), ctypes.POINTER(_vp)], _st),
+    "engram_ipc_close": ([_vp], _st),
     "engram_forward_host": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                              _i32, _vp, _sz, _vp], _st),
 }
@@ -247,6 +271,80 @@ def engram_forward_host(ctx, tok_host, B, T, tok_stride, t_begin, P, tables, h_h
                                     workspace_bytes, _stream(stream)), "engram_forward_host")
 
 
+# ---------------------------------------------------------------- multi-branch
+
+def engram_multibranch_workspace_bytes(ctx, M: int, B: int, L: int) -> int:
+    return int(_lib.engram_multibranch_workspace_bytes(ctx, M, B, L))
+
+
+def engram_forward_multibranch(ctx, M, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, k_scale,
+                               v_scale, conv_w, conv_state, y, alpha_out, add_residual, workspace, workspace_bytes,
+                               stream=None):
+    _check(_lib.engram_forward_multibranch(ctx, M, _ptr(tok), B, T, tok_stride, t_begin, _ptr(P), _ptr(tables),
+                                           _ptr(h), _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(k_scale),
+                                           _ptr(v_scale), _ptr(conv_w),
+                                           _ptr(conv_state), _ptr(y), _ptr(alpha_out), int(add_residual),
+                                           _ptr(workspace), workspace_bytes, _stream(stream)),
+           "engram_forward_multibranch")
+
+
+# ---------------------------------------------------------------- table backward
+
+def engram_table_grad_workspace_bytes(ctx, n_tok: int) -> int:
+    return int(_lib.engram_table_grad_workspace_bytes(ctx, n_tok))
+
+
+def engram_table_grad(ctx, idx, n_tok, d_e, rows_out, grad_out, n_unique, workspace, workspace_bytes, stream=None):
+    _check(_lib.engram_table_grad(ctx, _ptr(idx), n_tok, _ptr(d_e), _ptr(rows_out), _ptr(grad_out), _ptr(n_unique),
+                                  _ptr(workspace), workspace_bytes, _stream(stream)), "engram_table_grad")
+
+
+def engram_table_sgd(ctx, rows, grad, n_unique, max_rows, tables, lr, stream=None):
+    _check(_lib.engram_table_sgd(ctx, _ptr(rows), _ptr(grad), _ptr(n_unique), max_rows, _ptr(tables), float(lr),
+                                 _stream(stream)), "engram_table_sgd")
+
+
+# ---------------------------------------------------------------- sharded tables
+
+def engram_shard_range(ctx, n_shards: int, shard: int):
+    """(first global row, row count) of shard `shard` of n_shards."""
+    lo, cnt = _i64(0), _i64(0)
+    _check(_lib.engram_shard_range(ctx, n_shards, shard, ctypes.byref(lo), ctypes.byref(cnt)), "engram_shard_range")
+    return int(lo.value), int(cnt.value)
+
+
+def engram_forward_sharded(ctx, tok, B, T, tok_stride, t_begin, P, shard_ptrs, h, Wk, Wv, gq, gk, conv_w,
+                           conv_state, y, alpha_out, add_residual, workspace, workspace_bytes, stream=None):
+    """shard_ptrs: device pointers (ints) of the shards, valid on the current device."""
+    arr = (_vp * len(shard_ptrs))(*[int(p) if p else None for p in shard_ptrs])
+    _check(_lib.engram_forward_sharded(ctx, _ptr(tok), B, T, tok_stride, t_begin, _ptr(P), arr, len(shard_ptrs),
+                                       _ptr(h), _ptr(Wk), _ptr(Wv), _ptr(gq), _ptr(gk), _ptr(conv_w),
+                                       _ptr(conv_state), _ptr(y), _ptr(alpha_out), int(add_residual),
+                                       _ptr(workspace), workspace_bytes, _stream(stream)),
+           "engram_forward_sharded")
+
+
+def engram_ipc_export(dev_ptr: int):
+    """(64-byte handle, offset) of the allocation holding dev_ptr."""
+    buf = ctypes.create_string_buffer(ENGRAM_IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    _check(_lib.engram_ipc_export(dev_ptr, buf, ctypes.byref(off)), "engram_ipc_export")
+    return buf.raw, int(off.value)
+
+
+def engram_ipc_open(handle: bytes, offset: int):
+    """(pointer, mapping base) of an exported allocation, on the current device."""
+    if len(handle) != ENGRAM_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is 64 bytes")
+    ptr, base = _vp(), _vp()
+    _check(_lib.engram_ipc_open(handle, offset, ctypes.byref(ptr), ctypes.byref(base)), "engram_ipc_open")
+    return int(ptr.value), int(base.value)
+
+
+def engram_ipc_close(base: int) -> None:
+    _check(_lib.engram_ipc_close(base), "engram_ipc_close")
+
+
 # ---------------------------------------------------------------- host tier
 
 def engram_host_tier_create(ctx, host_tables, max_lookups: int, n_threads: int) -> int:
@@ -256,6 +354,12 @@ def engram_host_tier_create(ctx, host_tables, max_lookups: int, n_threads: int) 
     _check(_lib.engram_host_tier_create(ctx, _ptr(host_tables), max_lookups, n_threads, ctypes.byref(out)),
            "engram_host_tier_create")
     return out.value
+
+
+def engram_host_tier_debug(tier, inject: int, wait_limit_s: float) -> None:
+    """Test hook: arm one-shot host-side faults of the next fetch and set the
+    tier's host wait limit."""
+    _check(_lib.engram_host_tier_debug(tier, inject, wait_limit_s), "engram_host_tier_debug")
 
 
 def engram_host_tier_destroy(tier: int) -> None:
@@ -286,6 +390,26 @@ def engram_host_tier_stats(tier) -> dict:
     ms, device copy ms (-1 while in flight)."""
     out = engram_host_tier_stats_t()
     _check(_lib.engram_host_tier_stats(tier, ctypes.addressof(out)), "engram_host_tier_stats")
+    return {f: getattr(out, f) for f, _ in out._fields_}
+
+
+def engram_host_cache_enable(tier, capacity_rows: int, min_count: int = 2) -> None:
+    _check(_lib.engram_host_cache_enable(tier, capacity_rows, min_count), "engram_host_cache_enable")
+
+
+def engram_host_cache_reset(tier, stream=None) -> None:
+    _check(_lib.engram_host_cache_reset(tier, _stream(stream)), "engram_host_cache_reset")
+
+
+class engram_host_cache_stats_t(ctypes.Structure):
+    _fields_ = [("capacity", ctypes.c_int64), ("resident", ctypes.c_int64), ("lookups", ctypes.c_int64),
+                ("cached_lookups", ctypes.c_int64), ("cached_rows", ctypes.c_int64), ("fetched_rows", ctypes.c_int64)]
+
+
+def engram_host_cache_stats(tier) -> dict:
+    """Hot-row cache figures of the last batch."""
+    out = engram_host_cache_stats_t()
+    _check(_lib.engram_host_cache_stats(tier, ctypes.addressof(out)), "engram_host_cache_stats")
     return {f: getattr(out, f) for f, _ in out._fields_}
 
 

@@ -2,11 +2,15 @@
 // kernel sequencing.  Every entry point validates on the host and launches
 // nothing on error; kernels report data errors through the context's device
 // status word instead of trapping.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <new>
+
+#include <cuda.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "ctx.cuh"
 
@@ -30,6 +34,8 @@ engram_status cuda_fail(const char* what, cudaError_t e) {
     return ENGRAM_E_CUDA;
 }
 
+int n_tables_of(const engram_config& k) { return k.n_orders * k.heads; }
+
 bool is_prime_u32(uint32_t n) {
     if (n < 2) return false;
     if (n % 2 == 0) return n == 2;
@@ -42,13 +48,18 @@ bool is_prime_u32(uint32_t n) {
 
 void prof_reset(engram_ctx* c) { c->prof_n = 0; }
 
+// Every launch is also an NVTX range named for the kernel's role, so a
+// profiler timeline of a step shows which launch is which (NVTX costs a
+// pointer test when no tool is attached).
 void prof_begin(engram_ctx* c, cudaStream_t s, const char* name) {
+    nvtxRangePushA(name);
     if (!c->prof || c->prof_n >= kMaxProf) return;
     c->prof_name[c->prof_n] = name;
     cudaEventRecord(c->ev[2 * c->prof_n], s);
 }
 
 void prof_end(engram_ctx* c, cudaStream_t s) {
+    nvtxRangePop();
     if (!c->prof || c->prof_n >= kMaxProf) return;
     cudaEventRecord(c->ev[2 * c->prof_n + 1], s);
     ++c->prof_n;
@@ -57,7 +68,8 @@ void prof_end(engram_ctx* c, cudaStream_t s) {
 // ---------------------------------------------------------------- workspace
 
 bool tc_path(const engram_ctx* c, int64_t n) {
-    return c->cfg.dtype == ENGRAM_BF16 && c->sm100 && project_tc_supported(n, c->d_mem, c->cfg.hidden);
+    return (c->cfg.dtype == ENGRAM_BF16 || c->cfg.dtype == ENGRAM_FP8) && c->sm100 &&
+           project_tc_supported(n, c->d_mem, c->cfg.hidden, c->cfg.dtype == ENGRAM_FP8);
 }
 
 // projections with the gate and the conv fused into the epilogue (conv width 4)
@@ -72,7 +84,7 @@ bool decode_shaped(const engram_ctx* c, int64_t n, int64_t L) { return fused_pat
 // per-128-row-band counters of the key pass
 size_t band_bytes(int64_t n) { return (size_t)((n + 127) / 128) * sizeof(int); }
 
-Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e) {
+Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e, int M) {
     const int64_t n = B * L;
     Workspace w{};
     char* p = static_cast<char*>(base);
@@ -83,12 +95,13 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
         p += align256((size_t)n * c->d_mem * c->es);
     }
     w.part = reinterpret_cast<float*>(p);
-    p += align256((size_t)n * c->G * 4 * sizeof(float));
+    p += align256((size_t)n * M * c->G * 4 * sizeof(float));
     w.alpha = reinterpret_cast<float*>(p);
-    p += align256((size_t)n * sizeof(float));
+    p += align256((size_t)M * n * sizeof(float));
     w.band = reinterpret_cast<int*>(p);
     p += align256(band_bytes(n));
-    const size_t hist_bytes = align256((size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
+    const size_t hist_bytes =
+        align256((size_t)M * B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
     w.state_next = reinterpret_cast<float*>(p);
     p += hist_bytes;
     if (decode_shaped(c, n, L)) {
@@ -155,8 +168,11 @@ engram_status conv_impl(engram_ctx* c, const float* v, const float* part, const 
 engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, const void* Wk, const void* Wv,
                              const float* gq, const float* gk, const float* conv_w, int32_t B, int32_t L,
                              float* state, void* y, float* alpha_out, int32_t add_residual, const Workspace& w,
-                             cudaStream_t s, bool after_retrieve = false) {
+                             cudaStream_t s, bool after_retrieve = false, int M = 1, const float* kscale = nullptr,
+                             const float* vscale = nullptr) {
+    const bool f8 = c->cfg.dtype == ENGRAM_FP8;
     const int64_t n = (int64_t)B * L;
+    const size_t hist_elems = (size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden;   // one branch's history
     if (fused_path(c, n)) {
         const bool tr = state && decode_shaped(c, n, L);
         cudaError_t e = cudaSuccess;
@@ -168,7 +184,9 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
             if (e == cudaSuccess) e = cudaStreamWaitEvent(c->aux, c->aux_ev[0], 0);
             if (e != cudaSuccess) return cuda_fail("ordering the history transpose", e);
             prof_begin(c, c->aux, "state_to_tr");
-            e = launch_state_to_tr(state, w.state_t, B, c->cfg.conv_width, c->cfg.hidden, c->aux);
+            for (int m = 0; m < M && e == cudaSuccess; ++m)
+                e = launch_state_to_tr(state + m * hist_elems, w.state_t + m * hist_elems, B, c->cfg.conv_width,
+                                       c->cfg.hidden, c->aux);
             prof_end(c, c->aux);
             if (e == cudaSuccess) e = cudaEventRecord(c->aux_ev[1], c->aux);
             if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
@@ -180,7 +198,7 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
         prof_begin(c, s, "gate_k_tc");
         e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band, w.alpha,
                              alpha_out, c->d_status, c->num_sms, c->debug_stall, after_retrieve && !tr && !c->prof,
-                             s);
+                             s, M, f8, kscale);
         c->debug_stall = 0;
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 key/gate launch", e);
@@ -191,17 +209,24 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
         prof_begin(c, s, "vconv_tc");
         e = launch_vconv_tc(e_cat, B, L, c->d_mem, h, Wv, conv_w, c->cfg.hidden, c->cfg.conv_width, w.alpha,
                             tr ? w.state_t : state, w.state_next, tr ? 1 : 0, y, add_residual, c->d_status,
-                            c->num_sms, !tr && !c->prof, s);
+                            c->num_sms, !tr && !c->prof, s, M, f8, vscale);
         prof_end(c, s);
         if (e != cudaSuccess) return cuda_fail("tcgen05 value/conv launch", e);
         if (state) {
             prof_begin(c, s, "state_merge");
-            e = tr ? launch_state_merge_tr(state, w.state_next, B, L, c->cfg.conv_width, c->cfg.hidden, s)
-                   : launch_state_merge(state, w.state_next, B, L, c->cfg.conv_width, c->cfg.hidden, c->num_sms, s);
+            for (int m = 0; m < M && e == cudaSuccess; ++m)
+                e = tr ? launch_state_merge_tr(state + m * hist_elems, w.state_next + m * hist_elems, B, L,
+                                               c->cfg.conv_width, c->cfg.hidden, s)
+                       : launch_state_merge(state + m * hist_elems, w.state_next + m * hist_elems, B, L,
+                                            c->cfg.conv_width, c->cfg.hidden, c->num_sms, s);
             prof_end(c, s);
             if (e != cudaSuccess) return cuda_fail("conv-state merge launch", e);
         }
         return ENGRAM_OK;
+    }
+    if (M != 1 || f8 || kscale || vscale) {
+        set_error("multi-branch, FP8 and scaled projections run on the fused tensor-core path only");
+        return ENGRAM_E_UNSUPPORTED;
     }
     engram_status st = project_impl(c, e_cat, n, h, Wk, Wv, gq, gk, w.v, w.part, s);
     if (st != ENGRAM_OK) return st;
@@ -218,7 +243,8 @@ engram_status check_forward_args(const engram_ctx* c, int32_t B, int32_t T, int6
 engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
                            int32_t t_begin, const int32_t* P, const void* tables, const void* h, const void* Wk,
                            const void* Wv, const float* gq, const float* gk, const float* conv_w, float* conv_state,
-                           void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s) {
+                           void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s,
+                           const ShardParams* shards, int M, const float* kscale, const float* vscale) {
     const int32_t L = T - t_begin;
     const bool fused = fused_path(c, (int64_t)B * L);
     if (fused) {
@@ -226,12 +252,15 @@ engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t
         cudaError_t e = cudaMemsetAsync(w.band, 0, band_bytes((int64_t)B * L), s);
         if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
     }
-    prof_begin(c, s, "retrieve");
-    cudaError_t e = launch_retrieve(tok, P, B, T, tok_stride, t_begin, c->hp, c->gp, tables, w.idx, w.e, c->d_status, s);
+    prof_begin(c, s, shards ? "retrieve_sharded" : "retrieve");
+    cudaError_t e = shards ? launch_retrieve_sharded(tok, P, B, T, tok_stride, t_begin, c->hp, c->gp, *shards, w.idx,
+                                                     w.e, c->d_status, c->num_sms, s)
+                           : launch_retrieve(tok, P, B, T, tok_stride, t_begin, c->hp, c->gp, tables, w.idx, w.e,
+                                             c->d_status, c->num_sms, s);
     prof_end(c, s);
     if (e != cudaSuccess) return cuda_fail("retrieve (hash + gather) launch", e);
     return gate_conv_impl(c, w.e, h, Wk, Wv, gq, gk, conv_w, B, L, conv_state, y, alpha_out, add_residual, w, s,
-                          fused);
+                          fused, M, kscale, vscale);
 }
 
 }  // namespace engram
@@ -273,8 +302,11 @@ engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
     for (int j = 0; j < J; ++j) {
         if (k.rows[j] >= 0x80000000u || !is_prime_u32(k.rows[j])) return inval("every table size must be a prime < 2^31");
     }
-    if (k.dtype != ENGRAM_F32 && k.dtype != ENGRAM_BF16) return inval("unknown dtype");
-    const int es = k.dtype == ENGRAM_F32 ? 4 : 2;
+    if (k.dtype != ENGRAM_F32 && k.dtype != ENGRAM_BF16 && k.dtype != ENGRAM_FP8) return inval("unknown dtype");
+    const int es = k.dtype == ENGRAM_F32 ? 4 : (k.dtype == ENGRAM_BF16 ? 2 : 1);
+    if (k.dtype == ENGRAM_FP8 &&
+        (k.hidden % 128 != 0 || ((int64_t)n_tables_of(k) * k.row_dim) % 128 != 0 || k.conv_width != 4))
+        return inval("FP8 needs hidden and J*row_dim multiples of 128 and conv width 4 (the fused path)");
     if (k.row_dim < 1 || ((int64_t)k.row_dim * es) % 16 != 0) return inval("row_dim * element size must be a multiple of 16 bytes");
     if (k.hidden < 8 || k.hidden % 8 != 0) return inval("hidden must be a positive multiple of 8");
     if (k.conv_width < 1 || k.conv_width > kMaxConv) return inval("conv_width must be in 1..8");
@@ -287,6 +319,7 @@ engram_status engram_create(const engram_config* cfg, engram_ctx** out) {
     c->cfg = k;
     c->J = J;
     c->es = es;
+    c->hs = k.dtype == ENGRAM_F32 ? 4 : 2;
     c->d_mem = J * k.row_dim;
     c->G = (k.hidden + kGroup - 1) / kGroup;
     cudaError_t e = cudaGetDevice(&c->device);
@@ -470,6 +503,10 @@ engram_status engram_project(engram_ctx* c, const void* e_cat, int64_t n_tok, co
     if (n_tok < 0) return inval("n_tok must be >= 0");
     if (n_tok == 0) return ENGRAM_OK;
     if (!e_cat || !h || !Wk || !Wv || !v || !part) return inval("null tensor pointer");
+    if (c->cfg.dtype == ENGRAM_FP8) {
+        set_error("engram_project: FP8 runs on the fused forward only");
+        return ENGRAM_E_UNSUPPORTED;
+    }
     if (!aligned16(e_cat) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(v) || !aligned16(part))
         return inval("e_cat, h, Wk, Wv, v and part must be 16-byte aligned");
     engram_status st = check_device(c);
@@ -485,6 +522,10 @@ engram_status engram_conv(engram_ctx* c, const float* v, const float* part, cons
     if (B < 0 || L < 0) return inval("B and L must be >= 0");
     if ((int64_t)B * L == 0) return ENGRAM_OK;
     if (!v || !part || !conv_w || !y || (add_residual && !h)) return inval("null tensor pointer");
+    if (c->cfg.dtype == ENGRAM_FP8) {
+        set_error("engram_conv: FP8 runs on the fused forward only");
+        return ENGRAM_E_UNSUPPORTED;
+    }
     if (!aligned16(v) || !aligned16(part) || !aligned16(y) || (add_residual && !aligned16(h)) ||
         (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
         return inval("v, part, y, h, conv_w and conv_state must be 16-byte aligned");
@@ -539,6 +580,146 @@ engram_status engram_forward(engram_ctx* c, const int32_t* tok, int32_t B, int32
                         alpha_out, add_residual, w, s);
 }
 
+// ---------------------------------------------------------------- multi-branch
+
+size_t engram_multibranch_workspace_bytes(const engram_ctx* c, int32_t M, int32_t B, int32_t L) {
+    if (!c || M < 1 || M > ENGRAM_MAX_BRANCHES || B < 0 || L < 0) return 0;
+    return carve(c, nullptr, B, L, true, M).bytes;
+}
+
+engram_status engram_forward_multibranch(engram_ctx* c, int32_t M, const int32_t* tok, int32_t B, int32_t T,
+                                         int64_t tok_stride, int32_t t_begin, const int32_t* P, const void* tables,
+                                         const void* h, const void* Wk, const void* Wv, const float* gq,
+                                         const float* gk, const float* k_scale, const float* v_scale,
+                                         const float* conv_w, float* conv_state, void* y, float* alpha_out,
+                                         int32_t add_residual, void* workspace, size_t workspace_bytes,
+                                         cudaStream_t s) {
+    engram_status st = check_forward_args(c, B, T, tok_stride, t_begin);
+    if (st != ENGRAM_OK) return st;
+    if (M < 1 || M > ENGRAM_MAX_BRANCHES) return inval("M must be in 1..4");
+    const int32_t L = T - t_begin;
+    const int64_t n = (int64_t)B * L;
+    if (n == 0) return ENGRAM_OK;
+    if (!fused_path(c, n)) {
+        set_error("the multi-branch forward runs on the fused tensor-core path only (bf16 or FP8, conv width 4, d "
+                  "a multiple of 128, J*D a multiple of 64 (128 for FP8))");
+        return ENGRAM_E_UNSUPPORTED;
+    }
+    if ((k_scale && !aligned16(k_scale)) || (v_scale && !aligned16(v_scale)))
+        return inval("k_scale and v_scale must be 16-byte aligned");
+    if (!tok || !P || !tables || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    Workspace w = carve(c, workspace, B, L, true, M);
+    if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
+    if (!aligned16(tables) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
+        (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
+        return inval("tables, h, Wk, Wv, y, conv_w and conv_state must be 16-byte aligned");
+    st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    prof_reset(c);
+    return forward_impl(c, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
+                        alpha_out, add_residual, w, s, nullptr, M, k_scale, v_scale);
+}
+
+// ---------------------------------------------------------------- tables sharded across GPUs
+
+engram_status engram_shard_range(const engram_ctx* c, int32_t n_shards, int32_t shard, int64_t* first_row,
+                                 int64_t* n_rows) {
+    if (!c || !first_row || !n_rows) return inval("null context or output pointer");
+    if (n_shards < 1 || n_shards > kMaxShards) return inval("n_shards must be in 1..16");
+    if (shard < 0 || shard >= n_shards) return inval("shard must be in [0, n_shards)");
+    int64_t total = 0;
+    for (int j = 0; j < c->J; ++j) total += c->cfg.rows[j];
+    const int64_t per = (total + n_shards - 1) / n_shards;
+    const int64_t lo = std::min<int64_t>(total, (int64_t)shard * per);
+    const int64_t hi = std::min<int64_t>(total, lo + per);
+    *first_row = lo;
+    *n_rows = hi - lo;
+    return ENGRAM_OK;
+}
+
+engram_status engram_forward_sharded(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
+                                     int32_t t_begin, const int32_t* P, const void* const* shard_tables,
+                                     int32_t n_shards, const void* h, const void* Wk, const void* Wv, const float* gq,
+                                     const float* gk, const float* conv_w, float* conv_state, void* y,
+                                     float* alpha_out, int32_t add_residual, void* workspace, size_t workspace_bytes,
+                                     cudaStream_t s) {
+    engram_status st = check_forward_args(c, B, T, tok_stride, t_begin);
+    if (st != ENGRAM_OK) return st;
+    if (n_shards < 1 || n_shards > kMaxShards) return inval("n_shards must be in 1..16");
+    if (!shard_tables) return inval("null shard table list");
+    ShardParams sp{};
+    sp.n = n_shards;
+    for (int g = 0; g < n_shards; ++g) {
+        int64_t lo = 0, cnt = 0;
+        engram_shard_range(c, n_shards, g, &lo, &cnt);
+        if (cnt > 0 && !shard_tables[g]) return inval("null shard pointer");
+        if (!aligned16(shard_tables[g])) return inval("every shard must be 16-byte aligned");
+        sp.base[g] = static_cast<const uint4*>(shard_tables[g]);
+        sp.bound[g] = lo;
+        sp.bound[g + 1] = lo + cnt;
+    }
+    const int32_t L = T - t_begin;
+    const int64_t n = (int64_t)B * L;
+    if (n == 0) return ENGRAM_OK;
+    if (!tok || !P || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    Workspace w = carve(c, workspace, B, L, true);
+    if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
+    if (!aligned16(h) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(y) ||
+        (conv_state && !aligned16(conv_state)) || !aligned16(conv_w))
+        return inval("h, Wk, Wv, y, conv_w and conv_state must be 16-byte aligned");
+    st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    prof_reset(c);
+    return forward_impl(c, tok, B, T, tok_stride, t_begin, P, nullptr, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
+                        alpha_out, add_residual, w, s, &sp);
+}
+
+// Cross-process mapping of a shard: the allocation that holds `ptr` is
+// exported as a CUDA IPC handle plus the offset of `ptr` inside it.
+engram_status engram_ipc_export(const void* ptr, void* handle_out, uint64_t* offset_out) {
+    if (!ptr || !handle_out || !offset_out) return inval("null pointer");
+    static CUresult (*get_range)(CUdeviceptr*, size_t*, CUdeviceptr) = nullptr;
+    if (!get_range) {
+        void* q = nullptr;
+        cudaDriverEntryPointQueryResult res;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &q, cudaEnableDefault, &res) != cudaSuccess ||
+            res != cudaDriverEntryPointSuccess)
+            return cuda_fail("cuMemGetAddressRange entry point", cudaErrorNotSupported);
+        get_range = reinterpret_cast<CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr)>(q);
+    }
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (get_range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+        return inval("the pointer is not inside a device allocation");
+    cudaIpcMemHandle_t hd;
+    cudaError_t e = cudaIpcGetMemHandle(&hd, reinterpret_cast<void*>(base));
+    if (e != cudaSuccess) return cuda_fail("cudaIpcGetMemHandle", e);
+    std::memcpy(handle_out, &hd, sizeof(hd));
+    *offset_out = reinterpret_cast<uint64_t>(ptr) - (uint64_t)base;
+    return ENGRAM_OK;
+}
+
+engram_status engram_ipc_open(const void* handle, uint64_t offset, void** ptr_out, void** base_out) {
+    if (!handle || !ptr_out || !base_out) return inval("null pointer");
+    cudaIpcMemHandle_t hd;
+    std::memcpy(&hd, handle, sizeof(hd));
+    void* base = nullptr;
+    cudaError_t e = cudaIpcOpenMemHandle(&base, hd, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail("cudaIpcOpenMemHandle", e);
+    *base_out = base;
+    *ptr_out = static_cast<char*>(base) + offset;
+    return ENGRAM_OK;
+}
+
+engram_status engram_ipc_close(void* base) {
+    if (!base) return inval("null pointer");
+    cudaError_t e = cudaIpcCloseMemHandle(base);
+    if (e != cudaSuccess) return cuda_fail("cudaIpcCloseMemHandle", e);
+    return ENGRAM_OK;
+}
+
 // ---------------------------------------------------------------- forward without allocation
 //
 // For callers that cannot allocate device memory at all: an inference
@@ -555,22 +736,31 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ENGRAM_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64];   // device address of g_noalloc_scratch per device ordinal
+void* g_noalloc_ptr[64];   // device address of g_noalloc_scratch per device ordinal, from the last lookup
 
 // Device address of the static scratch on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device with that device current.
-engram_status noalloc_scratch(void** out) {
+// with that device current.  The lookup is repeated on every call whose
+// stream is not capturing (a cheap table lookup once the module is loaded),
+// so a device reset or a new primary context never leaves a stale address;
+// a capturing stream uses the address of the last uncaptured call, so the
+// first call on a device must come before any stream capture.
+engram_status noalloc_scratch(cudaStream_t s, void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
     if (dev < 0 || dev >= 64) return inval("device ordinal out of range for the static scratch");
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(s, &cap);
+    if (e != cudaSuccess) return cuda_fail("cudaStreamIsCapturing", e);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress of the static scratch", e);
         g_noalloc_ptr[dev] = p;
+    } else if (!g_noalloc_ptr[dev]) {
+        return inval("engram_forward_noalloc: the first call on a device must come before any stream capture");
     }
     *out = g_noalloc_ptr[dev];
     return ENGRAM_OK;
@@ -585,8 +775,11 @@ engram_status engram_forward_noalloc(engram_ctx* c, const int32_t* tok, int32_t 
                                      const void* Wk, const void* Wv, const float* gq, const float* gk,
                                      const float* conv_w, float* conv_state, void* y, float* alpha_out,
                                      int32_t add_residual, cudaStream_t s) {
-    if (!c) return inval("null context");
-    if (B < 0 || T < 0 || t_begin < 0 || t_begin > T) return inval("need B >= 0 and 0 <= t_begin <= T");
+    engram_status st = check_forward_args(c, B, T, tok_stride, t_begin);
+    if (st != ENGRAM_OK) return st;
+    // on the wrong device nothing (not even the scratch lookup) touches it
+    st = check_device(c);
+    if (st != ENGRAM_OK) return st;
     const size_t need = carve(c, nullptr, B, T - t_begin, true).bytes;
     if (need > (size_t)ENGRAM_NOALLOC_SCRATCH_BYTES) {
         std::snprintf(g_last_error, sizeof(g_last_error),
@@ -596,7 +789,7 @@ engram_status engram_forward_noalloc(engram_ctx* c, const int32_t* tok, int32_t 
         return ENGRAM_E_NOMEM;
     }
     void* scratch = nullptr;
-    engram_status st = noalloc_scratch(&scratch);
+    st = noalloc_scratch(s, &scratch);
     if (st != ENGRAM_OK) return st;
     return engram_forward(c, tok, B, T, tok_stride, t_begin, P, tables, h, Wk, Wv, gq, gk, conv_w, conv_state, y,
                           alpha_out, add_residual, scratch, (size_t)ENGRAM_NOALLOC_SCRATCH_BYTES, s);

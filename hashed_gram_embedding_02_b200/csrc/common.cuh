@@ -36,6 +36,17 @@ struct GatherParams {
     int32_t chunks_per_row;        // 16-byte chunks per table row
 };
 
+// Tables split across GPUs by global row (table j's row r is global row
+// row_off[j] + r): shard g holds global rows [bound[g], bound[g + 1]) at
+// base[g], a device pointer valid on the launching GPU (its own memory, or
+// another GPU's mapped into this one's address space).
+constexpr int kMaxShards = 16;
+struct ShardParams {
+    const uint4* base[kMaxShards];
+    int64_t bound[kMaxShards + 1];
+    int32_t n;
+};
+
 // x mod m for a 64-bit x and a 32-bit m, by Barrett's reduction (P. Barrett,
 // CRYPTO '86) with recip = floor((2^64 - 1) / m): q = floor(x * recip / 2^64)
 // undershoots floor(x / m) by at most 2, so at most two subtractions follow.
@@ -59,17 +70,27 @@ cudaError_t launch_gather(const uint32_t* idx, int64_t n_tok, const void* tables
 // launch_hash followed by launch_gather in one kernel (indices still written to idx)
 cudaError_t launch_retrieve(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
                             int32_t t_begin, const HashParams& hp, const GatherParams& gp, const void* tables,
-                            uint32_t* idx, void* e_cat, uint32_t* status, cudaStream_t s);
+                            uint32_t* idx, void* e_cat, uint32_t* status, int num_sms, cudaStream_t s);
+// the same with the table rows read from the shards of sp (plain, L2-only
+// loads, which reach peer memory over NVLink)
+cudaError_t launch_retrieve_sharded(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
+                                    int32_t t_begin, const HashParams& hp, const GatherParams& gp,
+                                    const ShardParams& sp, uint32_t* idx, void* e_cat, uint32_t* status,
+                                    int num_sms, cudaStream_t s);
 // CUDA-core projection (fp32 or bf16 operands, fp32 accumulation); v in fp32
 cudaError_t launch_project_simt(bool bf16, const void* e, int64_t n_tok, int32_t d_mem, const void* h,
                                 const void* Wk, const void* Wv, const float* gq, const float* gk, int32_t d,
                                 float* v, float* part, cudaStream_t s);
 // tcgen05 kernels (bf16 operands, fp32 accumulation in tensor memory); both
 // return cudaErrorNotSupported when the shape does not fit their tiling.
-bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d);
+// f8: e and W in FP8 E4M3 (kind::f8f6f4), else bf16
+bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d, bool f8 = false);
 cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                               const void* Wv, const float* gq, const float* gk, int32_t d, float* v,
                               float* part, uint32_t* status, int num_sms, cudaStream_t s);
+// Multi-branch (M in 1..4): Wk is the M branches' W_K stacked [M*d][d_mem];
+// h, gq, gk, alpha, Y, the conv history and its scratch are [M][...] of the
+// single-branch shapes; e and W_V are shared.
 // Pass 1: k -> gate partials [n_tok][G][4] and alpha [n_tok] (reduced by the
 // CTA that completes each 128-row band; band_count holds ceil(n_tok/128)
 // counters that must be zero on entry and are zero again on exit).
@@ -79,7 +100,7 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
                              float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
-                             cudaStream_t s);
+                             cudaStream_t s, int32_t M = 1, bool f8 = false, const float* kscale = nullptr);
 // Pass 2: v -> gate (alpha from pass 1), causal conv, residual, Y (fused
 // epilogue, conv width 4).  When state is non-null the new history goes to
 // state_next ([B][w-1][d] fp32 scratch) and launch_state_merge folds it into
@@ -90,7 +111,8 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
                             float* state_next, int32_t state_tr, void* y, int32_t add_residual, uint32_t* status,
-                            int num_sms, bool pdl, cudaStream_t s);
+                            int num_sms, bool pdl, cudaStream_t s, int32_t M = 1, bool f8 = false,
+                            const float* vscale = nullptr);
 // conv history [B][w-1][d] -> the sequence-minor [w-1][d][B] that decode-shaped
 // value passes read (state_tr), and the merge of such a pass's new history
 // back into the caller's [B][w-1][d]

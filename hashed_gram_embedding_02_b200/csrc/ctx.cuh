@@ -20,7 +20,8 @@ struct engram_ctx {
     int J;
     int d_mem;
     int G;
-    int es;                 // element size of the storage dtype
+    int es;                 // element size of the tables, e and W (4, 2, or 1 for FP8)
+    int hs;                 // element size of h and Y (4 for fp32, else 2: bf16)
     engram::HashParams hp;
     engram::GatherParams gp;
     uint32_t* d_status;     // device status word (256-byte block)
@@ -73,7 +74,9 @@ struct Workspace {
     float* v;
     size_t bytes;
 };
-Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e);
+// M > 1 (multi-branch, fused path only): part [n][M*G][4], alpha [M][n],
+// state_next / state_t [M][...].
+Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e, int M = 1);
 
 // Argument checks shared by the forward entry points (device pointers).
 engram_status check_forward_args(const engram_ctx* c, int32_t B, int32_t T, int64_t tok_stride, int32_t t_begin);
@@ -83,6 +86,8 @@ engram_status check_forward_args(const engram_ctx* c, int32_t B, int32_t T, int6
 engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t T, int64_t tok_stride,
                            int32_t t_begin, const int32_t* P, const void* tables, const void* h, const void* Wk,
                            const void* Wv, const float* gq, const float* gk, const float* conv_w, float* conv_state,
-                           void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s);
+                           void* y, float* alpha_out, int32_t add_residual, const Workspace& w, cudaStream_t s,
+                           const ShardParams* shards = nullptr, int M = 1, const float* kscale = nullptr,
+                           const float* vscale = nullptr);
 
 }  // namespace engram

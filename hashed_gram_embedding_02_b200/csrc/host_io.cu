@@ -38,7 +38,7 @@ HostPlan make_plan(const engram_ctx* c, int32_t B, int32_t T, int32_t t_begin, i
     const int32_t L = T - t_begin;
     p.lo = std::max(0, t_begin - (c->hp.max_order - 1));
     p.Tw = T - p.lo;
-    p.row_bytes = (size_t)c->cfg.hidden * c->es;
+    p.row_bytes = (size_t)c->cfg.hidden * c->hs;
     int64_t R = chunk_rows;
     if (R <= 0) R = (int64_t)std::max<size_t>(1, kDefaultChunkBytes / std::max<size_t>(1, (size_t)B * p.row_bytes));
     R = std::min<int64_t>(R, std::max(L, 1));

@@ -25,6 +25,18 @@
 //                        slot[t][j] of the staged rows into e_cat[t][j].
 // Between dedupe and gather_staged the caller's stream is free for other
 // work (the preceding layers), which the fetch overlaps.
+//
+// Hot-row cache (engram_host_cache_enable): the same sections, and the
+// Synced repost's last paragraph of "System efficiency", keep the frequent
+// n-grams' rows in a faster tier, because a few patterns take most of the
+// accesses.  Here C rows of HBM in front of the host tables: a device hash
+// set maps (table, row) to a cache slot.  The dedupe kernel resolves each
+// distinct row of the batch against it; a resident row is read from its
+// slot and is not fetched.  After the staged gather, the rows that this
+// batch fetched and looked up at least min_count times are admitted into
+// free slots (device-to-device, from the staged copy) until the cache is
+// full.  Slots and staged rows share one device buffer (slots first), so
+// the gather reads both through one slot map.
 #include <algorithm>
 #include <atomic>
 #include <chrono>
@@ -48,7 +60,7 @@ constexpr uint64_t kEmpty = 0;               // hash-set key of an empty slot (k
 constexpr int64_t kPackChunkRows = 4096;     // rows per packing chunk (1 MB at 256-byte rows)
 constexpr size_t kMinCopyBytes = 4u << 20;   // smallest row copy but the last: PCIe copies of a few MB
                                              // run faster than 1 MB or 100 MB ones
-constexpr double kHostWaitSeconds = 20.0;    // bound on every host-side wait
+constexpr double kHostWaitSeconds = 20.0;    // default bound on every host-side wait
 
 // Murmur3's 64-bit finaliser (Appleby), to spread row numbers over the set.
 __device__ __forceinline__ uint64_t mix64(uint64_t k) {
@@ -66,13 +78,38 @@ struct TierParams {
     int32_t J;
 };
 
-// Insert every valid lookup's global row (+1) into the open-addressing set;
-// the thread whose CAS claims an empty slot assigns the row the next unique
-// id and records it.  Probing is bounded by the set size (half empty at most
-// load), so a full set flags ERR_INDEX instead of looping.
+// Cache lookup: slot of global row key-1 in the hot-row set, or -1.
+__device__ __forceinline__ int64_t cache_find(const unsigned long long* __restrict__ ckeys,
+                                              const uint32_t* __restrict__ cvals, uint32_t cmask,
+                                              unsigned long long key) {
+    uint32_t h = (uint32_t)mix64(key) & cmask;
+    for (uint32_t probe = 0; probe <= cmask; ++probe) {
+        const unsigned long long k = ckeys[h];
+        if (k == key) return (int64_t)cvals[h];
+        if (k == kEmpty) return -1;
+        h = (h + 1u) & cmask;
+    }
+    return -1;
+}
+
+struct CacheParams {
+    const unsigned long long* keys;   // hot-row set (null: no cache)
+    const uint32_t* vals;             // its slots
+    uint32_t mask;
+    uint32_t capacity;                // C: staged rows start at slot C
+};
+
+// Insert every valid lookup's global row (+1) into the open-addressing set
+// and count the lookups per entry; the thread whose CAS claims an empty slot
+// resolves the row once: a row resident in the hot-row cache gets its cache
+// slot (counted in count[1]), any other row the next fetch id (count[0]),
+// recorded in the fetch list, and slot C + id.  Probing is bounded by the
+// set size (half empty at most load), so a full set flags ERR_INDEX instead
+// of looping.
 __global__ void dedupe_insert_kernel(const uint32_t* __restrict__ idx, int64_t n_lookups, TierParams tp,
-                                     unsigned long long* set_keys, uint32_t* set_vals, uint32_t mask,
-                                     unsigned long long* ukeys, uint32_t* count, uint32_t* status) {
+                                     unsigned long long* set_keys, uint32_t* set_vals, uint32_t* set_cnt,
+                                     uint32_t mask, CacheParams cp, unsigned long long* ukeys, uint32_t* count,
+                                     uint32_t* status) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int j = (int)(i % tp.J);
@@ -84,13 +121,21 @@ __global__ void dedupe_insert_kernel(const uint32_t* __restrict__ idx, int64_t n
         for (uint32_t probe = 0; probe <= mask; ++probe) {
             const unsigned long long prev = atomicCAS(set_keys + h, (unsigned long long)kEmpty, key);
             if (prev == kEmpty) {
-                const uint32_t id = atomicAdd(count, 1u);
-                set_vals[h] = id;
-                ukeys[id] = key - 1ull;
+                const int64_t cs = cp.keys ? cache_find(cp.keys, cp.vals, cp.mask, key) : -1;
+                if (cs >= 0) {
+                    set_vals[h] = (uint32_t)cs;
+                    atomicAdd(count + 1, 1u);
+                } else {
+                    const uint32_t id = atomicAdd(count, 1u);
+                    set_vals[h] = cp.capacity + id;
+                    ukeys[id] = key - 1ull;
+                }
+                atomicAdd(set_cnt + h, 1u);
                 placed = true;
                 break;
             }
             if (prev == key) {
+                atomicAdd(set_cnt + h, 1u);
                 placed = true;
                 break;
             }
@@ -100,12 +145,80 @@ __global__ void dedupe_insert_kernel(const uint32_t* __restrict__ idx, int64_t n
     }
 }
 
-// Slot of every lookup (a separate launch, so every insert and id is visible).
+// Admission into the hot-row cache, after the staged gather: every entry of
+// the batch set that was fetched (slot >= C) and looked up at least
+// min_count times takes the next free cache slot, while any is left; its row
+// is copied from the staged rows (16-byte chunks, one warp per row) and its
+// key enters the cache set.  count[2] is the number of slots in use.
+__global__ void cache_admit_kernel(const unsigned long long* __restrict__ set_keys,
+                                   const uint32_t* __restrict__ set_vals, const uint32_t* __restrict__ set_cnt,
+                                   uint32_t set_slots, uint32_t min_count, unsigned long long* ckeys, uint32_t* cvals,
+                                   uint32_t cmask, uint32_t capacity, uint4* rows, int chunks_per_row, uint32_t* count,
+                                   uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t base = warp0 * 32; base < set_slots; base += nwarps * 32) {
+        // each lane inspects one set entry; admitted entries are then copied by the whole warp
+        const int64_t h = base + lane;
+        bool want = false;
+        unsigned long long key = kEmpty;
+        uint32_t src = 0;
+        if (h < set_slots) {
+            key = set_keys[h];
+            src = set_vals[h];
+            want = key != kEmpty && src >= capacity && set_cnt[h] >= min_count;
+        }
+        uint32_t slot = 0xFFFFFFFFu;
+        if (want) {
+            const uint32_t s = atomicAdd(count + 2, 1u);
+            if (s < capacity) {
+                slot = s;
+            } else {
+                atomicSub(count + 2, 1u);    // full: the count stays at capacity
+            }
+        }
+        if (slot != 0xFFFFFFFFu) {
+            uint32_t hh = (uint32_t)mix64(key) & cmask;
+            bool placed = false;
+            for (uint32_t probe = 0; probe <= cmask; ++probe) {
+                const unsigned long long prev = atomicCAS(ckeys + hh, (unsigned long long)kEmpty, key);
+                if (prev == kEmpty) {
+                    cvals[hh] = slot;
+                    placed = true;
+                    break;
+                }
+                hh = (hh + 1u) & cmask;
+            }
+            if (!placed) flag(status, ENGRAM_ERR_INDEX);
+        }
+        uint32_t todo = __ballot_sync(0xffffffffu, slot != 0xFFFFFFFFu);
+        while (todo) {
+            const int l = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const uint32_t dst = __shfl_sync(0xffffffffu, slot, l);
+            const uint32_t from = __shfl_sync(0xffffffffu, src, l);
+            for (int c = lane; c < chunks_per_row; c += 32)
+                rows[(int64_t)dst * chunks_per_row + c] = rows[(int64_t)from * chunks_per_row + c];
+        }
+    }
+}
+
+// Slot of every lookup (a separate launch, so every insert and slot is
+// visible): a cache slot, C + fetch id, or ENGRAM_INVALID_INDEX.
 __global__ void dedupe_slot_kernel(const uint32_t* __restrict__ idx, int64_t n_lookups, TierParams tp,
                                    const unsigned long long* __restrict__ set_keys,
-                                   const uint32_t* __restrict__ set_vals, uint32_t mask, uint32_t* __restrict__ slot) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
-         i += (int64_t)gridDim.x * blockDim.x) {
+                                   const uint32_t* __restrict__ set_vals, uint32_t mask, uint32_t capacity,
+                                   uint32_t* __restrict__ slot, uint32_t* count) {
+    // every thread of the grid runs the same number of iterations (the bound
+    // is rounded up to the grid), so the warp-wide vote below is uniform
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t n_iter = (n_lookups + stride - 1) / stride * stride;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_iter; i += stride) {
+        if (i >= n_lookups) {
+            __ballot_sync(0xffffffffu, false);
+            continue;
+        }
         const int j = (int)(i % tp.J);
         const uint32_t r = __ldg(idx + i);
         uint32_t out = ENGRAM_INVALID_INDEX;
@@ -123,6 +236,9 @@ __global__ void dedupe_slot_kernel(const uint32_t* __restrict__ idx, int64_t n_l
             }
         }
         slot[i] = out;
+        // lookups served from the hot-row cache, one atomic per warp
+        const uint32_t hits = __ballot_sync(0xffffffffu, out < capacity);
+        if ((threadIdx.x & 31) == 0 && hits) atomicAdd(count + 3, (uint32_t)__popc(hits));
     }
 }
 
@@ -186,9 +302,17 @@ struct engram_host_tier {
     uint32_t* d_set_vals;
     uint32_t set_mask;
     unsigned long long* d_ukeys;
-    uint32_t* d_count;
+    uint32_t* d_set_cnt;    // lookups per set entry in this batch
+    uint32_t* d_count;      // [0] rows to fetch, [1] distinct rows found in the cache, [2] cache slots in use,
+                            // [3] lookups served from the cache
     uint32_t* d_slot;
-    uint8_t* d_rows;
+    uint8_t* d_rows;        // cache slots [0, C) then the staged rows [C, C + max_lookups)
+    // hot-row cache (capacity 0: none)
+    uint32_t cache_cap;
+    uint32_t cache_min_count;
+    unsigned long long* d_ckeys;
+    uint32_t* d_cvals;
+    uint32_t cache_mask;
     // pinned host
     unsigned long long* h_ukeys;
     uint32_t* h_count;
@@ -196,6 +320,10 @@ struct engram_host_tier {
     cudaEvent_t ev_keys, ev_ready, ev_consumed;
     cudaEvent_t ev_copy0, ev_copy1;   // timing: first row copy enqueued, last one done
     bool have_keys, fetched, consumed_recorded;
+    bool copies_recorded;   // ev_ready marks the end of every copy enqueued so far (success or failure)
+    // failure injection (engram_host_tier_debug): one-shot faults made on the host
+    std::atomic<uint32_t> inject;
+    double wait_limit_s;    // bound on every host-side wait
     int64_t pending_lookups;
     // packing pool
     std::vector<std::thread> workers;
@@ -229,6 +357,9 @@ void worker_main(engram_host_tier* t) {
         for (;;) {
             const int64_t k = t->next_chunk.fetch_add(1);
             if (k >= t->job_chunks) break;
+            if (k == t->job_chunks - 1 &&
+                (t->inject.fetch_and(~ENGRAM_INJECT_PACK_ABANDON) & ENGRAM_INJECT_PACK_ABANDON))
+                continue;   // injected: this thread gives up its chunk without packing or marking it
             const int64_t r0 = k * kPackChunkRows;
             const int64_t r1 = std::min(t->job_n, r0 + kPackChunkRows);
             pack_range(t->host_tables, t->total_rows, t->row_bytes, t->job_rows, r0, r1, t->h_stage);
@@ -237,14 +368,17 @@ void worker_main(engram_host_tier* t) {
     }
 }
 
-// Host wait on an event, bounded: ENGRAM_E_TIMEOUT if it does not complete.
-engram_status wait_event_bounded(cudaEvent_t ev, const char* what) {
+// Host wait on an event, bounded by `limit` seconds: ENGRAM_E_TIMEOUT if it
+// does not complete.  `never` fakes an event that never completes (the
+// injected list-wait failure): the query's answer is replaced, nothing else.
+engram_status wait_event_bounded(cudaEvent_t ev, const char* what, double limit = kHostWaitSeconds,
+                                 bool never = false) {
     const auto t0 = std::chrono::steady_clock::now();
     for (;;) {
-        const cudaError_t e = cudaEventQuery(ev);
+        const cudaError_t e = never ? cudaErrorNotReady : cudaEventQuery(ev);
         if (e == cudaSuccess) return ENGRAM_OK;
         if (e != cudaErrorNotReady) return cuda_fail(what, e);
-        if (std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count() > kHostWaitSeconds) {
+        if (std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count() > limit) {
             set_error(what);
             return ENGRAM_E_TIMEOUT;
         }
@@ -269,6 +403,9 @@ void tier_free(engram_host_tier* t) {
     cudaFree(t->d_set_vals);
     cudaFree(t->d_ukeys);
     cudaFree(t->d_count);
+    cudaFree(t->d_set_cnt);
+    cudaFree(t->d_ckeys);
+    cudaFree(t->d_cvals);
     cudaFree(t->d_slot);
     cudaFree(t->d_rows);
     cudaFreeHost(t->h_ukeys);
@@ -315,6 +452,8 @@ engram_status engram_host_tier_create(engram_ctx* c, const void* host_tables, in
     engram_host_tier* t = new (std::nothrow) engram_host_tier();
     if (!t) return ENGRAM_E_NOMEM;
     t->c = c;
+    t->wait_limit_s = kHostWaitSeconds;
+    t->inject.store(0);
     t->host_tables = static_cast<const uint8_t*>(host_tables);
     t->row_bytes = (size_t)c->cfg.row_dim * c->es;
     t->max_lookups = max_lookups;
@@ -334,8 +473,10 @@ engram_status engram_host_tier_create(engram_ctx* c, const void* host_tables, in
     cudaError_t e = t->chunk_done ? cudaSuccess : cudaErrorMemoryAllocation;
     if (e == cudaSuccess) e = cudaMalloc(&t->d_set_keys, (size_t)cap * sizeof(unsigned long long));
     if (e == cudaSuccess) e = cudaMalloc(&t->d_set_vals, (size_t)cap * sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMalloc(&t->d_set_cnt, (size_t)cap * sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMalloc(&t->d_ukeys, (size_t)max_lookups * sizeof(unsigned long long));
     if (e == cudaSuccess) e = cudaMalloc(&t->d_count, 256);
+    if (e == cudaSuccess) e = cudaMemset(t->d_count, 0, 256);
     if (e == cudaSuccess) e = cudaMalloc(&t->d_slot, (size_t)max_lookups * sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMalloc(&t->d_rows, (size_t)max_lookups * t->row_bytes);
     if (e == cudaSuccess) e = cudaHostAlloc(&t->h_ukeys, (size_t)max_lookups * sizeof(unsigned long long), 0);
@@ -368,7 +509,7 @@ engram_status engram_host_tier_create(engram_ctx* c, const void* host_tables, in
 void engram_host_tier_destroy(engram_host_tier* t) {
     if (!t) return;
     // copies of the last batch may still be in flight into the pinned buffers
-    if (t->fetched) wait_event_bounded(t->ev_ready, "host tier: draining the last fetch");
+    if (t->copies_recorded) wait_event_bounded(t->ev_ready, "host tier: draining the last fetch");
     if (t->have_keys) wait_event_bounded(t->ev_keys, "host tier: draining the last dedupe");
     tier_free(t);
 }
@@ -384,24 +525,28 @@ engram_status engram_host_dedupe(engram_host_tier* t, const uint32_t* idx, int64
     // fetches run on the caller's thread, so by now that fetch has returned
     const int64_t n = n_tok * c->J;
     cudaError_t e = cudaMemsetAsync(t->d_set_keys, 0, (size_t)(t->set_mask + 1) * sizeof(unsigned long long), s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(t->d_count, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->d_set_cnt, 0, (size_t)(t->set_mask + 1) * sizeof(uint32_t), s);
+    // the batch's counters; count[2] (cache slots in use) carries over
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->d_count, 0, 2 * sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->d_count + 3, 0, sizeof(uint32_t), s);
     if (e != cudaSuccess) return cuda_fail("host tier: clearing the set", e);
     if (n > 0) {
         const int threads = 256;
         const int64_t want = (n + threads - 1) / threads;
         const int blocks = (int)std::min<int64_t>(want, (int64_t)c->num_sms * 8);
-        dedupe_insert_kernel<<<blocks, threads, 0, s>>>(idx, n, t->tp, t->d_set_keys, t->d_set_vals, t->set_mask,
-                                                        t->d_ukeys, t->d_count, c->d_status);
+        CacheParams cp{t->cache_cap ? t->d_ckeys : nullptr, t->d_cvals, t->cache_mask, t->cache_cap};
+        dedupe_insert_kernel<<<blocks, threads, 0, s>>>(idx, n, t->tp, t->d_set_keys, t->d_set_vals, t->d_set_cnt,
+                                                        t->set_mask, cp, t->d_ukeys, t->d_count, c->d_status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail("dedupe insert launch", e);
         dedupe_slot_kernel<<<blocks, threads, 0, s>>>(idx, n, t->tp, t->d_set_keys, t->d_set_vals, t->set_mask,
-                                                      t->d_slot);
+                                                      t->cache_cap, t->d_slot, t->d_count);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail("dedupe slot launch", e);
     }
     // distinct-row count and list to pinned host memory (the list at its
     // largest possible length: one copy, no round trip for the count)
-    e = cudaMemcpyAsync(t->h_count, t->d_count, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(t->h_count, t->d_count, 4 * sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess && n > 0)
         e = cudaMemcpyAsync(t->h_ukeys, t->d_ukeys, (size_t)n * sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaEventRecord(t->ev_keys, s);
@@ -416,12 +561,16 @@ engram_status engram_host_fetch(engram_host_tier* t, cudaStream_t side, int64_t*
     if (!t->have_keys) return inval("engram_host_fetch needs a preceding engram_host_dedupe");
     engram_status st = check_device(t->c);
     if (st != ENGRAM_OK) return st;
+    // until this fetch succeeds, gather_staged must not read the staged rows
+    t->fetched = false;
     const auto tw = std::chrono::steady_clock::now();
-    st = wait_event_bounded(t->ev_keys, "host tier: waiting for the row list");
+    const bool fake_list = (t->inject.fetch_and(~ENGRAM_INJECT_LIST_WAIT) & ENGRAM_INJECT_LIST_WAIT) != 0;
+    st = wait_event_bounded(t->ev_keys, "host tier: waiting for the row list", t->wait_limit_s, fake_list);
     if (st != ENGRAM_OK) return st;
-    // the staging buffer and the device rows may still serve the previous batch
-    if (t->fetched) {
-        st = wait_event_bounded(t->ev_ready, "host tier: waiting for the previous copies");
+    // the staging buffer and the device rows may still serve the previous
+    // batch, or hold copies that a failed fetch left in flight
+    if (t->copies_recorded) {
+        st = wait_event_bounded(t->ev_ready, "host tier: waiting for the previous copies", t->wait_limit_s);
         if (st != ENGRAM_OK) return st;
     }
     cudaError_t e = cudaSuccess;
@@ -451,7 +600,7 @@ engram_status engram_host_fetch(engram_host_tier* t, cudaStream_t side, int64_t*
     auto wait_chunk = [&](int64_t k) -> bool {
         const auto w0 = std::chrono::steady_clock::now();
         while (!(*t->chunk_done)[k].load(std::memory_order_acquire)) {
-            if (std::chrono::duration<double>(std::chrono::steady_clock::now() - w0).count() > kHostWaitSeconds)
+            if (std::chrono::duration<double>(std::chrono::steady_clock::now() - w0).count() > t->wait_limit_s)
                 return false;
             std::this_thread::yield();
         }
@@ -476,18 +625,30 @@ engram_status engram_host_fetch(engram_host_tier* t, cudaStream_t side, int64_t*
         const int64_t rn = std::min(U, k1 * kPackChunkRows) - r0;
         if (copies == 0) e = cudaEventRecord(t->ev_copy0, side);
         if (e == cudaSuccess)
-            e = cudaMemcpyAsync(t->d_rows + (size_t)r0 * t->row_bytes, t->h_stage + (size_t)r0 * t->row_bytes,
+            e = cudaMemcpyAsync(t->d_rows + ((size_t)t->cache_cap + r0) * t->row_bytes,
+                                t->h_stage + (size_t)r0 * t->row_bytes,
                                 (size_t)rn * t->row_bytes, cudaMemcpyHostToDevice, side);
         if (e != cudaSuccess) result = cuda_fail("host tier: row copy", e);
         ++copies;
         k = k1;
     }
     if (result != ENGRAM_OK) {
+        // copies already enqueued still read the pinned staging: the next
+        // fetch (and destroy) must wait for them before the staging is
+        // packed again, so their end is recorded like a successful fetch's
+        if (copies > 0) {
+            if (cudaEventRecord(t->ev_ready, side) == cudaSuccess) {
+                t->copies_recorded = true;
+            } else {
+                cudaStreamSynchronize(side);
+                t->copies_recorded = false;
+            }
+        }
         // let the workers run out of chunks before anyone reuses the job
         const auto w0 = std::chrono::steady_clock::now();
         for (int64_t q = 0; q < n_chunks; ++q)
             while (!(*t->chunk_done)[q].load(std::memory_order_acquire) &&
-                   std::chrono::duration<double>(std::chrono::steady_clock::now() - w0).count() < kHostWaitSeconds)
+                   std::chrono::duration<double>(std::chrono::steady_clock::now() - w0).count() < t->wait_limit_s)
                 std::this_thread::yield();
         return result;
     }
@@ -496,6 +657,7 @@ engram_status engram_host_fetch(engram_host_tier* t, cudaStream_t side, int64_t*
     if (e == cudaSuccess) e = cudaEventRecord(t->ev_ready, side);
     if (e != cudaSuccess) return cuda_fail("host tier: recording the ready event", e);
     t->fetched = true;
+    t->copies_recorded = true;
     t->have_keys = false;
     t->last_unique = U;
     t->last_copies = copies;
@@ -508,7 +670,7 @@ engram_status engram_host_fetch(engram_host_tier* t, cudaStream_t side, int64_t*
 engram_status engram_gather_staged(engram_host_tier* t, int64_t n_tok, void* e_cat, cudaStream_t s) {
     if (!t) return inval("null host tier");
     engram_ctx* c = t->c;
-    if (!t->fetched) return inval("engram_gather_staged needs a preceding engram_host_fetch");
+    if (!t->fetched) return inval("engram_gather_staged needs a preceding successful engram_host_fetch");
     if (n_tok < 0 || n_tok * c->J > t->pending_lookups) return inval("n_tok differs from the deduplicated batch");
     if (n_tok == 0) return ENGRAM_OK;
     if (!e_cat || !aligned16(e_cat)) return inval("e_cat must be a 16-byte aligned device pointer");
@@ -519,16 +681,103 @@ engram_status engram_gather_staged(engram_host_tier* t, int64_t n_tok, void* e_c
     GatherParams gp = c->gp;
     for (int j = 0; j < c->J; ++j) {
         gp.row_off[j] = 0;
-        gp.rows[j] = (uint32_t)std::min<int64_t>(t->max_lookups, 0xFFFFFFFEll);
+        gp.rows[j] = (uint32_t)std::min<int64_t>((int64_t)t->cache_cap + t->max_lookups, 0xFFFFFFFEll);
     }
     prof_reset(c);
     prof_begin(c, s, "gather_staged");
     e = launch_gather(t->d_slot, n_tok, t->d_rows, gp, e_cat, c->d_status, c->num_sms, s);
     prof_end(c, s);
     if (e != cudaSuccess) return cuda_fail("staged gather launch", e);
+    if (t->cache_cap) {
+        // admission reads the staged rows, so it runs before the next fetch may overwrite them
+        const uint32_t slots = t->set_mask + 1;
+        const int blocks = (int)std::min<int64_t>((slots + 255) / 256, (int64_t)c->num_sms * 8);
+        prof_begin(c, s, "cache_admit");
+        cache_admit_kernel<<<blocks, 256, 0, s>>>(t->d_set_keys, t->d_set_vals, t->d_set_cnt, slots,
+                                                  t->cache_min_count, t->d_ckeys, t->d_cvals, t->cache_mask,
+                                                  t->cache_cap, reinterpret_cast<uint4*>(t->d_rows),
+                                                  (int)(t->row_bytes / 16), t->d_count, c->d_status);
+        prof_end(c, s);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("cache admission launch", e);
+    }
     e = cudaEventRecord(t->ev_consumed, s);
     if (e != cudaSuccess) return cuda_fail("host tier: recording the consumed event", e);
     t->consumed_recorded = true;
+    return ENGRAM_OK;
+}
+
+engram_status engram_host_cache_enable(engram_host_tier* t, int64_t capacity_rows, int32_t min_count) {
+    if (!t) return inval("null host tier");
+    if (capacity_rows < 1 || capacity_rows > ((int64_t)1 << 30)) return inval("capacity_rows must be in [1, 2^30]");
+    if (min_count < 1) return inval("min_count must be >= 1");
+    if (t->cache_cap) return inval("the hot-row cache is already enabled");
+    if (t->have_keys || t->fetched) return inval("enable the hot-row cache before the first batch");
+    engram_status st = check_device(t->c);
+    if (st != ENGRAM_OK) return st;
+    if (t->copies_recorded) {
+        st = wait_event_bounded(t->ev_ready, "host tier: draining copies before the cache is set up", t->wait_limit_s);
+        if (st != ENGRAM_OK) return st;
+    }
+    uint32_t cap = 1;
+    while ((int64_t)cap < 2 * capacity_rows) cap <<= 1;   // load factor <= 1/2
+    uint8_t* rows = nullptr;
+    unsigned long long* ckeys = nullptr;
+    uint32_t* cvals = nullptr;
+    cudaError_t e = cudaMalloc(&rows, ((size_t)capacity_rows + (size_t)t->max_lookups) * t->row_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&ckeys, (size_t)cap * sizeof(unsigned long long));
+    if (e == cudaSuccess) e = cudaMalloc(&cvals, (size_t)cap * sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemset(ckeys, 0, (size_t)cap * sizeof(unsigned long long));
+    if (e == cudaSuccess) e = cudaMemset(t->d_count + 2, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        cudaFree(rows);
+        cudaFree(ckeys);
+        cudaFree(cvals);
+        if (e == cudaErrorMemoryAllocation) {
+            set_error("host tier: the hot-row cache does not fit in device memory");
+            return ENGRAM_E_NOMEM;
+        }
+        return cuda_fail("host tier: hot-row cache set-up", e);
+    }
+    cudaFree(t->d_rows);
+    t->d_rows = rows;
+    t->d_ckeys = ckeys;
+    t->d_cvals = cvals;
+    t->cache_mask = cap - 1;
+    t->cache_cap = (uint32_t)capacity_rows;
+    t->cache_min_count = (uint32_t)min_count;
+    return ENGRAM_OK;
+}
+
+engram_status engram_host_cache_reset(engram_host_tier* t, cudaStream_t s) {
+    if (!t) return inval("null host tier");
+    if (!t->cache_cap) return inval("the hot-row cache is not enabled");
+    engram_status st = check_device(t->c);
+    if (st != ENGRAM_OK) return st;
+    cudaError_t e = cudaMemsetAsync(t->d_ckeys, 0, (size_t)(t->cache_mask + 1) * sizeof(unsigned long long), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->d_count + 2, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return cuda_fail("host tier: clearing the hot-row cache", e);
+    return ENGRAM_OK;
+}
+
+engram_status engram_host_cache_stats(const engram_host_tier* t, engram_host_cache_stats_t* out) {
+    if (!t || !out) return inval("null host tier or output");
+    out->capacity = t->cache_cap;
+    out->lookups = t->have_keys || t->fetched ? t->pending_lookups : 0;
+    out->resident = t->h_count ? t->h_count[2] : 0;
+    out->cached_rows = t->h_count ? t->h_count[1] : 0;
+    out->fetched_rows = t->h_count ? t->h_count[0] : 0;
+    out->cached_lookups = t->h_count ? t->h_count[3] : 0;
+    return ENGRAM_OK;
+}
+
+engram_status engram_host_tier_debug(engram_host_tier* t, uint32_t inject, double wait_limit_s) {
+    if (!t) return inval("null host tier");
+    if (inject & ~(uint32_t)(ENGRAM_INJECT_LIST_WAIT | ENGRAM_INJECT_PACK_ABANDON)) return inval("unknown injection bit");
+    if (!(wait_limit_s > 0.0) || wait_limit_s > 3600.0) return inval("wait_limit_s must be in (0, 3600]");
+    t->wait_limit_s = wait_limit_s;
+    t->inject.fetch_or(inject);
     return ENGRAM_OK;
 }
 

@@ -62,6 +62,11 @@ constexpr int MODE_VCONV = 2;
 constexpr int BM = 128;                 // rows per tile (UMMA M)
 constexpr int BK = 64;                  // K per stage: 64 bf16 = 128 bytes = one swizzle row
 constexpr int UK = 16;                  // K per tcgen05.mma kind::f16
+// FP8 (E4M3) operands: the same 128-byte swizzle rows hold 128 elements, and
+// one tcgen05.mma kind::f8f6f4 covers K = 32 (32 bytes, like 16 bf16)
+template <bool F8> struct Elt {
+    static constexpr int BKE = F8 ? 128 : 64;   // K elements per stage
+};
 constexpr int A_BYTES = BM * BK * 2;    // 16 KB
 constexpr int THREADS = 640;            // warps 0-3 producer / MMA / idle, warps 4-19 epilogue
 constexpr int EPI_WARPS = 16;           // four per TMEM lane quarter
@@ -140,7 +145,23 @@ struct EpiParams {
     float* alpha_w;             // MODE_K: [n_tok] gate values written by each band's last CTA
     float* alpha_out;           // MODE_K: caller's copy of alpha, or null
     float eps;
+    // multi-branch: M residual branches share e and W_V and have their own
+    // W_K (stacked [M*d][d_mem]), h, gains, gate, conv history and Y, each
+    // [M][...] with the single-branch layout per branch
+    int M;
+    int Gb;                     // 128-channel groups per branch (d / 128); G = M * Gb in MODE_K
+    // per output channel dequantisation of the accumulators (null: none):
+    // k = kscale[c] * acc over the stacked [M*d] key channels, v = vscale[c] * acc
+    const float* kscale;
+    const float* vscale;
+    // tile order: 0 = channel-fastest (a row band's tiles run together, A is
+    // read once); rb > 0 = groups of rb row units per channel tile, so that a
+    // W slice is reused by rb bands in a row (wide N: the stacked W_K of
+    // several branches does not stay in L2 under channel-fastest order)
+    int raster_rb;
 };
+
+constexpr int kMaxBranches = ENGRAM_MAX_BRANCHES;
 
 // Bounded wait: true when the phase with `parity` completed, false when the
 // CTA aborted or the wait ran out (then the status bit and abort flag are set).
@@ -208,21 +229,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N = BN, M = 128.
-template <int BN, int M = BM>
+// Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A and B K-major,
+// N = BN (bits 17-22, N/8), M (bits 24-28, M/16); operand formats in bits
+// 7-9 (A) and 10-12 (B): bf16 = 1 for kind::f16, E4M3 = 0 for kind::f8f6f4.
+template <int BN, int M = BM, bool F8 = false>
 struct Idesc {
-    static constexpr uint32_t value =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    static constexpr uint32_t value = (1u << 4) | (F8 ? 0u : ((1u << 7) | (1u << 10))) |
+                                      ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 };
 
-template <int BN>
+template <int BN, bool F8 = false>
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
-        ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN>::value), "r"(accumulate));
+    if constexpr (F8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n"
+            ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN, BM, true>::value), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+            ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN>::value), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -235,13 +264,20 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 // M = 256 x N = BN MMA over both CTAs of the pair, issued by the leader:
 // A rows 0-127 from the leader's shared memory and 128-255 from the peer's,
 // W columns split the same way; D rows land in each CTA's own TMEM.
-template <int BN>
+template <int BN, bool F8 = false>
 __device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
-        ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN, 2 * BM>::value), "r"(accumulate));
+    if constexpr (F8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n"
+            ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN, 2 * BM, true>::value), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+            ::"r"(tmem_d), "l"(da), "l"(db), "n"(Idesc<BN, 2 * BM>::value), "r"(accumulate));
 }
 
 // arrive on the barrier at the same offset in both CTAs once the pair's
@@ -408,10 +444,12 @@ __device__ __forceinline__ void unpack8(const uint4& q, float* f) {
 // ---------------------------------------------------------------- epilogues
 
 // Gate partials of row i over `ncols` k columns (multiple of 32) starting at
-// TMEM column taddr and tile-local channel cl; gains s_gg indexed
-// tile-locally.  TMEM loads run one 16-column chunk ahead of the math.
+// TMEM column taddr and tile-local channel cl; gains s_gg and the key
+// channels' dequantisation scales s_ks indexed tile-locally.  TMEM loads run
+// one 16-column chunk ahead of the math.
 __device__ __forceinline__ void partials_cols(uint32_t taddr, const uint8_t* hs, int i, bool valid, int cl,
-                                              int ncols, const float* s_gg, float& s_qk, float& s_kk, float& s_hh) {
+                                              int ncols, const float* s_gg, const float* s_ks, float& s_qk,
+                                              float& s_kk, float& s_hh) {
     uint32_t ka[16], kb[16];
     const int nch = ncols / 16;
     tmem_ld16(taddr, ka);
@@ -433,9 +471,12 @@ __device__ __forceinline__ void partials_cols(uint32_t taddr, const uint8_t* hs,
                     const float4 g0 = *reinterpret_cast<const float4*>(s_gg + c8);
                     const float4 g1 = *reinterpret_cast<const float4*>(s_gg + c8 + 4);
                     const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const float4 k0 = *reinterpret_cast<const float4*>(s_ks + c8);
+                    const float4 k1 = *reinterpret_cast<const float4*>(s_ks + c8 + 4);
+                    const float ks[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float kf = __uint_as_float(cur[u * 8 + e]);
+                        const float kf = __uint_as_float(cur[u * 8 + e]) * ks[e];
                         s_qk = fmaf(gg[e] * hf[e], kf, s_qk);
                         s_kk = fmaf(kf, kf, s_kk);
                         s_hh = fmaf(hf[e], hf[e], s_hh);
@@ -459,9 +500,9 @@ __device__ __forceinline__ void load_gains(const EpiParams& p, int c0, int n, fl
 // s_red, written by the group's first part.
 __device__ __forceinline__ void group_partials(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int64_t row,
                                                int i, bool valid, int part, int cl0, int ncols, int parts_per_group,
-                                               int g, const float* s_gg, float4* s_red) {
+                                               int g, const float* s_gg, const float* s_ks, float4* s_red) {
     float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-    partials_cols(taddr, hs, i, valid, cl0, ncols, s_gg, s_qk, s_kk, s_hh);
+    partials_cols(taddr, hs, i, valid, cl0, ncols, s_gg, s_ks, s_qk, s_kk, s_hh);
     s_red[part * BM + i] = make_float4(s_qk, s_kk, s_hh, 0.f);
     epi_sync();
     if (part % parts_per_group == 0 && valid) {
@@ -486,10 +527,11 @@ __device__ __forceinline__ void epilogue_kv(uint32_t taddr, const uint8_t* hs, c
     const int c0 = nt * 128;
     epi_sync();                       // previous tile's readers are done with s_gg and s_red
     load_gains(p, c0, 128, s_gg, et);
+    if (et < 128) s_gg[128 + et] = 1.f;    // no key scales on this path
     epi_sync();
     if (part < 2) {
         float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-        partials_cols(taddr + part * 64, hs, i, valid, part * 64, 64, s_gg, s_qk, s_kk, s_hh);
+        partials_cols(taddr + part * 64, hs, i, valid, part * 64, 64, s_gg, s_gg + 128, s_qk, s_kk, s_hh);
         s_red[part * BM + i] = make_float4(s_qk, s_kk, s_hh, 0.f);
     } else {
 #pragma unroll 1
@@ -520,7 +562,8 @@ __device__ __forceinline__ void epilogue_kv(uint32_t taddr, const uint8_t* hs, c
 struct TilePre {
     float4 w0, w1;   // MODE_VCONV: taps of this lane's channel pair of its warp's part (see vconv_pair)
     float g;         // MODE_K: g_q * g_k of channel et
-    float a;         // MODE_VCONV: alpha of this thread's row
+    float ks;        // MODE_K: dequantisation scale of key channel et
+    float a;         // MODE_VCONV: alpha of this thread's row (branch 0; other branches load theirs in turn)
 };
 
 // The value epilogue's warp (q, part) uses, per phase, BN/(2 NPART) channels =
@@ -547,7 +590,10 @@ __device__ __forceinline__ TilePre tile_pre_load(const EpiParams& p, int mt, int
         const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - (CONV_W - 1);
         t.a = (r >= 0 && r < p.n_tok) ? __ldg(p.alpha + r) : 0.f;
     } else if (MODE == MODE_K) {
-        if (et < BN) t.g = (p.gq ? __ldg(p.gq + n0 + et) : 1.f) * (p.gk ? __ldg(p.gk + n0 + et) : 1.f);
+        if (et < BN) {
+            t.g = (p.gq ? __ldg(p.gq + n0 + et) : 1.f) * (p.gk ? __ldg(p.gk + n0 + et) : 1.f);
+            t.ks = p.kscale ? __ldg(p.kscale + n0 + et) : 1.f;
+        }
     }
     return t;
 }
@@ -565,11 +611,14 @@ __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, co
     const bool valid = row < p.n_tok;
     const int n0 = nt * BN;
     epi_sync();
-    if (et < BN) s_gg[et] = pre.g;
+    if (et < BN) {
+        s_gg[et] = pre.g;
+        s_gg[BN + et] = pre.ks;
+    }
     epi_sync();
     if (has_next) pre = tile_pre_load<MODE_K, BN>(p, mt_next, nt_next, q, lane, et);
     group_partials(taddr + part * PW, hs, p, row, i, valid, part, part * PW, PW, PPG, (n0 + part * PW) / 128, s_gg,
-                   s_red);
+                   s_gg + BN, s_red);
 }
 
 // Gate + causal depthwise conv (width 4) + residual on a value tile of BN
@@ -593,10 +642,14 @@ __device__ __forceinline__ float mask_f(float x, uint32_t m) { return __uint_as_
 template <int NCH, bool SLOW, bool RES>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
-                                             const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3) {
+                                             const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3, int br) {
     constexpr int H = CONV_W - 1;
-    const bool write_state = SLOW && p.state_next && out_row && t >= p.L - H;
-    const bool from_state = SLOW && t < H && p.state;
+    // this branch's history and new history (the same size in both layouts)
+    const int64_t hist_off = (int64_t)br * p.B * H * p.d;
+    const float* state = p.state ? p.state + hist_off : nullptr;
+    float* state_next = p.state_next ? p.state_next + hist_off : nullptr;
+    const bool write_state = SLOW && state_next && out_row && t >= p.L - H;
+    const bool from_state = SLOW && t < H && state;
     uint32_t va[16], vb[16];
     tmem_ld16(taddr + cbeg, va);
 #pragma unroll
@@ -614,7 +667,10 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
         float o[16];
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
-            const float v0 = a * __uint_as_float(cur[c]), v1 = a * __uint_as_float(cur[c + 1]);
+            // warp-uniform address: one broadcast load per channel pair
+            const float2 vs = p.vscale ? __ldg(reinterpret_cast<const float2*>(p.vscale + n0 + cl + c))
+                                       : make_float2(1.f, 1.f);
+            const float v0 = a * vs.x * __uint_as_float(cur[c]), v1 = a * vs.y * __uint_as_float(cur[c + 1]);
             float s1a = __shfl_up_sync(0xffffffffu, v0, 1), s1b = __shfl_up_sync(0xffffffffu, v1, 1);
             float s2a = __shfl_up_sync(0xffffffffu, v0, 2), s2b = __shfl_up_sync(0xffffffffu, v1, 2);
             float s3a = __shfl_up_sync(0xffffffffu, v0, 3), s3b = __shfl_up_sync(0xffffffffu, v1, 3);
@@ -638,10 +694,10 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
                         if (t < k) {
                             const int hr = H - k + t;            // history row holding v~_{t-k}
                             if (p.state_tr) {                     // [3][d][B]: consecutive lanes, consecutive b
-                                const float* st = p.state + ((int64_t)hr * p.d + chn) * p.B + b;
+                                const float* st = state + ((int64_t)hr * p.d + chn) * p.B + b;
                                 ps[k - 1] = make_float2(__ldg(st), __ldg(st + p.B));
                             } else {
-                                ps[k - 1] = __ldg(reinterpret_cast<const float2*>(p.state + (b * H + hr) * p.d + chn));
+                                ps[k - 1] = __ldg(reinterpret_cast<const float2*>(state + (b * H + hr) * p.d + chn));
                             }
                         }
                 }
@@ -660,11 +716,11 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
                 const int hr = t - (p.L - H);
                 const int chn = n0 + cl + c;
                 if (p.state_tr) {
-                    float* sn = p.state_next + ((int64_t)hr * p.d + chn) * p.B + b;
+                    float* sn = state_next + ((int64_t)hr * p.d + chn) * p.B + b;
                     sn[0] = v0;
                     sn[p.B] = v1;
                 } else {
-                    *reinterpret_cast<float2*>(p.state_next + (b * H + hr) * p.d + chn) = make_float2(v0, v1);
+                    *reinterpret_cast<float2*>(state_next + (b * H + hr) * p.d + chn) = make_float2(v0, v1);
                 }
             }
             // halved taps of the channel pair: (c_0 ch0, c_0 ch1, c_1 ch0, c_1 ch1), (c_2 .., c_3 ..)
@@ -693,11 +749,13 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
 
 // The value tile's epilogue runs in two phases over the two channel halves of
 // the tile, so that the h half of phase 0 can be refilled for the next tile
-// while phase 1 runs.  In each phase part `part` takes BN/8 channels.
+// while phase 1 runs; with M branches, 2M phases: both halves for branch 0,
+// then for branch 1, ... (the accumulator holds v for all of them).  In each
+// phase part `part` takes BN/8 channels.
 template <int BN>
 __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt, int nt,
                                                int q, int part, int lane, int et, float* s_taps, int phase,
-                                               float a, const TilePre& pre) {
+                                               float a, const TilePre& pre, int br) {
     constexpr int H = CONV_W - 1;
     const int i = q * 32 + lane;
     const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - H;
@@ -716,7 +774,7 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     // ahead, read by this warp only
     constexpr int VPP = BN / (4 * NPART);
     float4* s_tw = reinterpret_cast<float4*>(s_taps) + (size_t)(q * NPART + part) * 2 * VPP * 2;
-    if (phase == 0) {
+    if (phase == 0 && br == 0) {
         const int k = lane & 15, ph = lane >> 4;
         if (k < VPP) {
             const float4 w0 = pre.w0, w1 = pre.w1;
@@ -740,11 +798,15 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     const float4* cw = s_tw + phase * VPP * 2 - cbeg;
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
-        if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
-        else vconv_chunks<NCHK, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
+        if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+                                                            br);
+        else vconv_chunks<NCHK, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+                                                            br);
     } else {
-        if (slow) vconv_chunks<NCHK, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
-        else vconv_chunks<NCHK, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3);
+        if (slow) vconv_chunks<NCHK, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+                                                            br);
+        else vconv_chunks<NCHK, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+                                                            br);
     }
     // the warp's Y block (its 32 rows x PW channels, in place of h) to global
     // memory: LPR lanes cover one row's contiguous bytes, so each store
@@ -755,13 +817,14 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     const int cb = cbeg >> 6;
     const int j = ((cbeg & 63) >> 3) + lane % LPR;
     const int64_t seg0 = (int64_t)mt * TILE_OUT + q * SEG_OUT - H;   // global row of the segment's lane 0
+    __nv_bfloat16* y = p.y + (int64_t)br * p.n_tok * p.d;
 #pragma unroll
     for (int k = 0; k < 32 / RPI; ++k) {
         const int rr = k * RPI + lane / LPR;
         const int ii = q * 32 + rr;
         const uint4 v = *reinterpret_cast<const uint4*>(hs + cb * (BM * 128) + ii * 128 + ((j ^ (ii & 7)) << 4));
         const int64_t rg = seg0 + rr;
-        if (rr >= H && rg < p.n_tok) __stcs(reinterpret_cast<uint4*>(p.y + rg * p.d + n0 + cb * 64 + j * 8), v);
+        if (rr >= H && rg < p.n_tok) __stcs(reinterpret_cast<uint4*>(y + rg * p.d + n0 + cb * 64 + j * 8), v);
     }
 }
 
@@ -793,10 +856,12 @@ __device__ __forceinline__ void band_alpha(const EpiParams& p, int mt, int et, B
     if (staged)
         for (int k = et; k < rows * p.G; k += EPI_THREADS) s_stage[k] = __ldcg(src + k);
     epi_sync();
-    if (et < rows) {
+    // one (row, branch) per thread: branch m's gate reduces its Gb groups
+    for (int k = et; k < rows * p.M; k += EPI_THREADS) {
+        const int m = k / rows, rr = k - m * rows;
         float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-        for (int g = 0; g < p.G; ++g) {
-            const float4 v4 = staged ? s_stage[et * p.G + g] : __ldcg(src + et * p.G + g);
+        for (int g = m * p.Gb; g < (m + 1) * p.Gb; ++g) {
+            const float4 v4 = staged ? s_stage[rr * p.G + g] : __ldcg(src + rr * p.G + g);
             s_qk += v4.x;
             s_kk += v4.y;
             s_hh += v4.z;
@@ -805,8 +870,9 @@ __device__ __forceinline__ void band_alpha(const EpiParams& p, int mt, int et, B
         const float rh = sqrtf(s_hh * inv_d + p.eps);
         const float rk = sqrtf(s_kk * inv_d + p.eps);
         const float a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)p.d)));
-        p.alpha_w[row0 + et] = a;
-        if (p.alpha_out) p.alpha_out[row0 + et] = a;
+        const int64_t o = (int64_t)m * p.n_tok + row0 + rr;
+        p.alpha_w[o] = a;
+        if (p.alpha_out) p.alpha_out[o] = a;
     }
     if (et == 0) p.band_count[mt] = 0;
 }
@@ -824,7 +890,7 @@ __device__ __forceinline__ void band_alpha(const EpiParams& p, int mt, int et, B
 // once the 32 epilogue warps of both CTAs have arrived on the leader's tempty.
 // On an abort both CTAs stop issuing, meet at a cluster barrier, and the
 // leader drains every stage either CTA issued before both leave together.
-template <int MODE, int BN, bool PAIR>
+template <int MODE, int BN, bool PAIR, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
                   const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_h,
@@ -845,7 +911,8 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int KB = p.d_mem / BK;
+    constexpr int BKE = Elt<F8>::BKE;
+    const int KB = p.d_mem / BKE;
     const uint32_t rank = PAIR ? cluster_rank() : 0u;
     const bool leader = rank == 0;
     // work units: single tiles, or pair tiles shared by the two CTAs of a cluster
@@ -913,8 +980,22 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     }
 
     // row tile of this CTA for unit u; channel tile
-    auto unit_mt = [&](int u) { return PAIR ? 2 * (u / p.n_groups) + (int)rank : u / p.n_groups; };
-    auto unit_nt = [&](int u) { return u % p.n_groups; };
+    const int m_units = num_units / p.n_groups;
+    auto unit_row = [&](int u) {
+        if (p.raster_rb <= 0) return u / p.n_groups;
+        const int per = p.raster_rb * p.n_groups;
+        const int g = u / per, local = u - g * per;
+        const int rows_g = min(p.raster_rb, m_units - g * p.raster_rb);
+        return g * p.raster_rb + local % rows_g;
+    };
+    auto unit_nt = [&](int u) {
+        if (p.raster_rb <= 0) return u % p.n_groups;
+        const int per = p.raster_rb * p.n_groups;
+        const int g = u / per, local = u - g * per;
+        const int rows_g = min(p.raster_rb, m_units - g * p.raster_rb);
+        return local / rows_g;
+    };
+    auto unit_mt = [&](int u) { return PAIR ? 2 * unit_row(u) + (int)rank : unit_row(u); };
 
     if (warp == 0) {
         // ---------------- TMA producer (each CTA loads its own rows and W half)
@@ -953,15 +1034,15 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                         // four 32-row segments, each starting 3 rows before its outputs
 #pragma unroll
                         for (int sg = 0; sg < 4; ++sg)
-                            load(&map_a, a_dst + sg * (SEG * 128), kb * BK, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
+                            load(&map_a, a_dst + sg * (SEG * 128), kb * BKE, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1));
                     } else {
-                        load(&map_a, a_dst, kb * BK, mt * BM);
+                        load(&map_a, a_dst, kb * BKE, mt * BM);
                     }
                     if (MODE == MODE_KV) {
-                        load(&map_b0, b_dst, kb * BK, nt * 128);
-                        load(&map_b1, b_dst + 128 * BK * 2, kb * BK, nt * 128);
+                        load(&map_b0, b_dst, kb * BKE, nt * 128);
+                        load(&map_b1, b_dst + 128 * 128, kb * BKE, nt * 128);
                     } else {
-                        load(&map_b0, b_dst, kb * BK, nt * BN + (int)rank * GE::B_ROWS);
+                        load(&map_b0, b_dst, kb * BKE, nt * BN + (int)rank * GE::B_ROWS);
                     }
                     sb->issued = it + 1;
                 }
@@ -970,18 +1051,14 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 // the tile's h slice, once the epilogue has released the previous one
                 if (!wait_bounded(&sb->hempty, ((uint32_t)tc & 1u) ^ 1u, sb, p.status)) break;
                 mbar_arrive_expect_tx(&sb->hfull, GE::H_BYTES);
-                const int hc0 = MODE == MODE_KV ? nt * 128 : nt * BN;
+                // the tile's channels in the stacked [M*d] key space: branch m, channel hc0 within
+                // it; branch m's rows start at row m * n_tok of the stacked [M * n_tok][d] h
+                const int ck = MODE == MODE_KV ? nt * 128 : nt * BN;
+                const int hm = ck / p.d, hc0 = ck - hm * p.d;
 #pragma unroll 1
-                for (int cb = 0; cb < GE::HC / 64; ++cb) {
-                    if (MODE == MODE_VCONV) {
-#pragma unroll
-                        for (int sg = 0; sg < 4; ++sg)
-                            tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull, hc0 + cb * 64,
-                                             mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1), h_pol);
-                    } else {
-                        tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128), &sb->hfull, hc0 + cb * 64, mt * BM, h_pol);
-                    }
-                }
+                for (int cb = 0; cb < GE::HC / 64; ++cb)
+                    tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128), &sb->hfull, hc0 + cb * 64, hm * p.n_tok + mt * BM,
+                                     h_pol);
                 sb->h_issued = tc + 1;
             }
         }
@@ -1010,11 +1087,12 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     const uint64_t db = smem_desc_sw128(a_addr + A_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
-                        // +32 bytes along K inside the swizzled 128-byte row
+                        // +32 bytes along K inside the swizzled 128-byte row (16 bf16 or 32 FP8)
                         if constexpr (PAIR)
-                            umma_bf16_pair<BN>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
+                            umma_bf16_pair<BN, F8>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2),
+                                                   (kb | kk) != 0);
                         else
-                            umma_bf16<BN>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
+                            umma_bf16<BN, F8>(d_tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0);
                     }
                     if constexpr (PAIR) umma_commit_pair_both(&sb->empty[s]);
                     else umma_commit(&sb->empty[s]);
@@ -1037,19 +1115,24 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             for (int u = unit0; u < num_units && !sb->abort_flag; u += units_step, ++tc) {
                 const int mt = unit_mt(u), nt = unit_nt(u);
                 bool ok = true;
-                for (int hf = 0; hf < 2; ++hf) {
-                    if (!wait_bounded(&sb->hempty_v[hf], ((uint32_t)tc & 1u) ^ 1u, sb, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&sb->hfull_v[hf], GE::H_BYTES / 2);
-                    for (int cb = hf * CB_HALF; cb < (hf + 1) * CB_HALF; ++cb) {
+                // each half is filled once per branch: use k = tc * M + m
+                for (int m = 0; m < p.M && ok; ++m) {
+                    const int k = tc * p.M + m;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        if (!wait_bounded(&sb->hempty_v[hf], ((uint32_t)k & 1u) ^ 1u, sb, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&sb->hfull_v[hf], GE::H_BYTES / 2);
+                        for (int cb = hf * CB_HALF; cb < (hf + 1) * CB_HALF; ++cb) {
 #pragma unroll
-                        for (int sg = 0; sg < 4; ++sg)
-                            tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull_v[hf],
-                                             nt * BN + cb * 64, mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1), h_pol);
+                            for (int sg = 0; sg < 4; ++sg)
+                                tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull_v[hf],
+                                                 nt * BN + cb * 64,
+                                                 m * p.n_tok + mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1), h_pol);
+                        }
+                        sb->h_issued_v[hf] = k + 1;
                     }
-                    sb->h_issued_v[hf] = tc + 1;
                 }
                 if (!ok) break;
             }
@@ -1084,24 +1167,31 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 bool ok = wait_bounded(&sb->tfull[acc], aph, sb, p.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
-                const float a_row = pre.a;
+                const float a0 = pre.a;
+                const int64_t r_lane = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - (CONV_W - 1);
+                const bool r_ok = r_lane >= 0 && r_lane < p.n_tok;
+                float a_br = a0;
+                const int n_ph = 2 * p.M;
 #pragma unroll 1
-                for (int phase = 0; phase < 2; ++phase) {
-                    ok = wait_bounded(&sb->hfull_v[phase], (uint32_t)tc & 1u, sb, p.status);
+                for (int ph = 0; ph < n_ph; ++ph) {
+                    const int phase = ph & 1, br = ph >> 1;
+                    const int k = tc * p.M + br;
+                    ok = wait_bounded(&sb->hfull_v[phase], (uint32_t)k & 1u, sb, p.status);
                     if (!__all_sync(0xffffffffu, ok)) break;
-                    epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg,
-                                       phase, a_row, pre);
-                    if (phase == 0 && has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
-                    if (phase == 1) tc_fence_before();
+                    if (br > 0 && phase == 0) a_br = r_ok ? __ldg(p.alpha + (int64_t)br * p.n_tok + r_lane) : 0.f;
+                    epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, phase, a_br, pre, br);
+                    if (ph == 0 && has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
+                    const bool last = ph == n_ph - 1;
+                    if (last) tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        if (phase == 1) {
+                        if (last) {
                             if (PAIR && !leader) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
                             else mbar_arrive(&sb->tempty[acc]);
                         }
                         mbar_arrive(&sb->hempty_v[phase]);
                     }
-                    if (threadIdx.x == 128) sb->h_consumed_v[phase] = tc + 1;
+                    if (threadIdx.x == 128) sb->h_consumed_v[phase] = k + 1;
                 }
                 if (!__all_sync(0xffffffffu, ok)) break;
                 continue;
@@ -1278,25 +1368,36 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 row-major [rows][cols] map with a box of box_rows x 64 columns
-// (128 bytes, 128-byte swizzle); rows outside [0, rows) read as zero.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D row-major [rows][cols] map with a box of box_rows x 128 bytes (64 bf16
+// or 128 FP8 bytes, 128-byte swizzle); rows outside [0, rows) read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, bool f8 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const uint64_t es = f8 ? 1 : 2;
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    const cuuint64_t strides[1] = {cols * es};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / es), box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    return fn(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+              dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BN, bool PAIR>
+// h of M branches stacked as a 2-D bf16 [M * rows][cols] map (box_rows x 64
+// columns, 128-byte swizzle).  A tile's rows before its branch's row 0 or
+// past its last row read the neighbouring branch (or zeros at the ends);
+// those rows are never used: they are conv history rows, whose h the value
+// epilogue does not read, or rows past n_tok, which neither epilogue keeps.
+bool make_map_h(CUtensorMap* m, const void* base, uint64_t branches, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return make_map(m, base, branches * rows, cols, box_rows);
+}
+
+template <int MODE, int BN, bool PAIR, bool F8 = false>
 cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const CUtensorMap& mh,
                         EpiParams p, int64_t m_tiles, int num_sms, cudaStream_t s, bool pdl = false) {
     using GE = Geo<MODE, BN, PAIR>;
-    auto kernel = project_tc_kernel<MODE, BN, PAIR>;
+    auto kernel = project_tc_kernel<MODE, BN, PAIR, F8>;
     static unsigned long long attr_set = 0;   // one bit per device ordinal
     static int max_clusters[64] = {};
     int dev = 0;
@@ -1368,27 +1469,29 @@ int pick_bn(int32_t d, int64_t n_tok, int64_t m_tiles, int num_sms) {
 // CTA pairs once there are enough row tiles to give every SM pair work
 bool use_pair(int64_t m_tiles, int n_groups, int num_sms) { return m_tiles * n_groups >= 2 * (int64_t)num_sms; }
 
-// A pair couples the two CTAs' value epilogues through the shared
-// accumulator; on B200 the value pass ran 124 us as pairs against 101 us on
-// single CTAs (c2).  It stays on single CTAs.
-bool use_pair_vconv(int64_t, int, int) { return false; }
+// The value pass stays on single CTAs: a pair couples the two CTAs' value
+// epilogues through the shared accumulator, and on B200 the value pass ran
+// 124 us as pairs against 101 us on single CTAs (c2), 399 against 322 us (c3).
 
 }  // namespace
 
-bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d) {
-    return n_tok > 0 && n_tok < (int64_t)1 << 30 && d_mem % BK == 0 && d_mem >= BK && d % 128 == 0 &&
+bool project_tc_supported(int64_t n_tok, int32_t d_mem, int32_t d, bool f8) {
+    const int bke = f8 ? Elt<true>::BKE : Elt<false>::BKE;
+    return n_tok > 0 && n_tok < (int64_t)1 << 30 && d_mem % bke == 0 && d_mem >= bke && d % 128 == 0 &&
            encode_fn() != nullptr;
 }
 
 cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                               const void* Wv, const float* gq, const float* gk, int32_t d, float* v, float* part,
                               uint32_t* status, int num_sms, cudaStream_t s) {
-    if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
+    if (!project_tc_supported(n_tok, d_mem, d, false)) return cudaErrorNotSupported;
     CUtensorMap ma, mk, mv, mh;
     if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, 128) ||
-        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, 128) || !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, BM))
+        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, 128) || !make_map_h(&mh, h, 1, (uint64_t)n_tok, (uint64_t)d, BM))
         return cudaErrorInvalidValue;
     EpiParams p{};
+    p.M = 1;
+    p.Gb = d / 128;
     p.gq = gq;
     p.gk = gk;
     p.v = v;
@@ -1405,14 +1508,19 @@ cudaError_t launch_project_tc(const void* e, int64_t n_tok, int32_t d_mem, const
 cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const void* h, const void* Wk,
                              const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
                              float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
-                             cudaStream_t s) {
-    if (!project_tc_supported(n_tok, d_mem, d)) return cudaErrorNotSupported;
+                             cudaStream_t s, int32_t M, bool f8, const float* kscale) {
+    if (!project_tc_supported(n_tok, d_mem, d, f8) || M < 1 || M > kMaxBranches || (int64_t)M * n_tok >= (1ll << 31))
+        return cudaErrorNotSupported;
     const int bn = pick_bn(d, n_tok, (n_tok + BM - 1) / BM, num_sms);
     CUtensorMap ma, mk, mh;
-    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn) ||
-        !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, BM))
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, BM, f8) ||
+        !make_map(&mk, Wk, (uint64_t)M * d, (uint64_t)d_mem, bn, f8) ||
+        !make_map_h(&mh, h, (uint64_t)M, (uint64_t)n_tok, (uint64_t)d, BM))
         return cudaErrorInvalidValue;
     EpiParams p{};
+    p.M = M;
+    p.Gb = d / 128;
+    p.kscale = kscale;
     p.gq = gq;
     p.gk = gk;
     p.part = reinterpret_cast<float4*>(part);
@@ -1425,14 +1533,19 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     p.n_tok = (int)n_tok;
     p.d_mem = d_mem;
     p.d = d;
-    p.G = d / 128;
-    p.n_groups = d / bn;
+    p.G = M * (d / 128);
+    p.n_groups = M * (d / bn);
+    p.raster_rb = p.n_groups > 16 ? 8 : 0;
     const int64_t mt = (n_tok + BM - 1) / BM;
     if (bn == 256 && use_pair(mt, p.n_groups, num_sms)) {
         CUtensorMap mk2;
-        if (!make_map(&mk2, Wk, (uint64_t)d, (uint64_t)d_mem, 128)) return cudaErrorInvalidValue;
-        return launch_mode<MODE_K, 256, true>(ma, mk2, mk2, mh, p, mt, num_sms, s, pdl);
+        if (!make_map(&mk2, Wk, (uint64_t)M * d, (uint64_t)d_mem, 128, f8)) return cudaErrorInvalidValue;
+        return f8 ? launch_mode<MODE_K, 256, true, true>(ma, mk2, mk2, mh, p, mt, num_sms, s, pdl)
+                  : launch_mode<MODE_K, 256, true, false>(ma, mk2, mk2, mh, p, mt, num_sms, s, pdl);
     }
+    if (f8)
+        return bn == 256 ? launch_mode<MODE_K, 256, false, true>(ma, mk, mk, mh, p, mt, num_sms, s, pdl)
+                         : launch_mode<MODE_K, 128, false, true>(ma, mk, mk, mh, p, mt, num_sms, s, pdl);
     return bn == 256 ? launch_mode<MODE_K, 256, false>(ma, mk, mk, mh, p, mt, num_sms, s, pdl)
                      : launch_mode<MODE_K, 128, false>(ma, mk, mk, mh, p, mt, num_sms, s, pdl);
 }
@@ -1440,15 +1553,21 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
 cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, const void* h, const void* Wv,
                             const float* conv_w, int32_t d, int32_t w, const float* alpha, const float* state,
                             float* state_next, int32_t state_tr, void* y, int32_t add_residual, uint32_t* status,
-                            int num_sms, bool pdl, cudaStream_t s) {
+                            int num_sms, bool pdl, cudaStream_t s, int32_t M, bool f8, const float* vscale) {
     const int64_t n_tok = (int64_t)B * L;
-    if (!project_tc_supported(n_tok, d_mem, d) || w != CONV_W) return cudaErrorNotSupported;
+    if (!project_tc_supported(n_tok, d_mem, d, f8) || w != CONV_W || M < 1 || M > kMaxBranches ||
+        (int64_t)M * n_tok >= (1ll << 31))
+        return cudaErrorNotSupported;
     const int bn = pick_bn(d, n_tok, (n_tok + TILE_OUT - 1) / TILE_OUT, num_sms);
     CUtensorMap ma, mv, mh;
-    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, SEG) || !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn) ||
-        !make_map(&mh, h, (uint64_t)n_tok, (uint64_t)d, SEG))
+    if (!make_map(&ma, e, (uint64_t)n_tok, (uint64_t)d_mem, SEG, f8) ||
+        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn, f8) ||
+        !make_map_h(&mh, h, (uint64_t)M, (uint64_t)n_tok, (uint64_t)d, SEG))
         return cudaErrorInvalidValue;
     EpiParams p{};
+    p.M = M;
+    p.Gb = d / 128;
+    p.vscale = vscale;
     p.alpha = alpha;
     p.conv_w = conv_w;
     p.state = state;
@@ -1465,11 +1584,9 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     p.L = L;
     p.add_residual = add_residual;
     const int64_t mt = (n_tok + TILE_OUT - 1) / TILE_OUT;
-    if (bn == 256 && use_pair_vconv(mt, p.n_groups, num_sms)) {
-        CUtensorMap mv2;
-        if (!make_map(&mv2, Wv, (uint64_t)d, (uint64_t)d_mem, 128)) return cudaErrorInvalidValue;
-        return launch_mode<MODE_VCONV, 256, true>(ma, mv2, mv2, mh, p, mt, num_sms, s, pdl);
-    }
+    if (f8)
+        return bn == 256 ? launch_mode<MODE_VCONV, 256, false, true>(ma, mv, mv, mh, p, mt, num_sms, s, pdl)
+                         : launch_mode<MODE_VCONV, 128, false, true>(ma, mv, mv, mh, p, mt, num_sms, s, pdl);
     return bn == 256 ? launch_mode<MODE_VCONV, 256, false>(ma, mv, mv, mh, p, mt, num_sms, s, pdl)
                      : launch_mode<MODE_VCONV, 128, false>(ma, mv, mv, mh, p, mt, num_sms, s, pdl);
 }

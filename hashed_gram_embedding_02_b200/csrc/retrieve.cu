@@ -13,6 +13,17 @@
 // then copies the R x J table rows as 16-byte chunks, each thread issuing a
 // batch of independent loads before its stores, consecutive threads on
 // consecutive chunks of e_cat (coalesced stores).
+//
+// Sharded tables (the pages' training layout, "DeepSeek AI II" digest,
+// section "DeepSeek Engram", and the Synced repost, "System efficiency":
+// the tables are split over the GPUs and the accessed rows are brought to
+// the GPU that needs them).  The SHARDED variant resolves, in the hash
+// phase, each (row, table) pair to the shard that owns the row and to the
+// row's address there; the gather phase then reads every row straight from
+// its owner's memory (over NVLink for another GPU's shard) into this GPU's
+// e_cat.  The all-to-all of indices and rows becomes one-sided reads inside
+// the kernel that needs them, and every remote row lands in local HBM
+// before the projections use it.
 #include "common.cuh"
 
 namespace engram {
@@ -39,13 +50,18 @@ __device__ __forceinline__ int32_t canon_id(const int32_t* ids, const int32_t* P
     return x;
 }
 
+template <bool SHARDED>
 __global__ void __launch_bounds__(kThreads, 8)
 retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, int32_t B, int32_t T, int64_t stride,
                 int32_t t_begin, const HashParams hp, const GatherParams gp, const uint4* __restrict__ tables,
-                uint32_t* __restrict__ idx, uint4* __restrict__ e_cat, int rows_per_cta, int cpr_shift, int pr_shift,
-                uint32_t* status) {
+                const ShardParams sp, uint32_t* __restrict__ idx, uint4* __restrict__ e_cat, int rows_per_cta,
+                int cpr_shift, int pr_shift, uint32_t* status) {
     __shared__ int32_t s_win[kThreads][4];
     __shared__ uint32_t s_idx[kThreads];
+    // SHARDED: the first chunk of each (row, table) pair's table row, or null
+    __shared__ const uint4* s_src[SHARDED ? kThreads : 1];
+    __shared__ const uint4* s_base[SHARDED ? kMaxShards : 1];
+    __shared__ int64_t s_bound[SHARDED ? kMaxShards + 1 : 1];
     // per-table constants in shared memory: lanes index them by table, and
     // divergent indexing of kernel parameters would serialise on the
     // constant cache
@@ -69,6 +85,10 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
         s_off[k] = gp.row_off[k];
         s_rows[k] = hp.rows[k];
         s_order[k] = hp.orders[k / hp.K];
+    }
+    if constexpr (SHARDED) {
+        for (int k = threadIdx.x; k < sp.n; k += kThreads) s_base[k] = sp.base[k];
+        for (int k = threadIdx.x; k <= sp.n; k += kThreads) s_bound[k] = sp.bound[k];
     }
 
     // 1. n-gram windows (PAD before the sequence start)
@@ -95,6 +115,17 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
         const uint32_t v = invalid ? ENGRAM_INVALID_INDEX : mod_u64(x, s_rows[jt], s_recip[jt]);
         s_idx[k] = v;
         idx[(row0 + rr) * J + jt] = v;
+        if constexpr (SHARDED) {
+            const uint4* src = nullptr;
+            if (v < s_rows[jt]) {
+                const int64_t g_row = s_off[jt] + v;
+                int g = 0;
+                while (g + 1 < sp.n && g_row >= s_bound[g + 1]) ++g;
+                if (g_row >= s_bound[g] && g_row < s_bound[g + 1])
+                    src = s_base[g] + (g_row - s_bound[g]) * gp.chunks_per_row;
+            }
+            s_src[k] = src;
+        }
     }
     __syncthreads();
 
@@ -116,8 +147,14 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
                 const int jt = cpr_shift >= 0 ? rem >> cpr_shift : rem / cpr;
                 const int c = rem - jt * cpr;
                 const uint32_t r = s_idx[rr * J + jt];
-                if (r < s_rows[jt]) v[u] = __ldg(tables + (s_off[jt] + r) * cpr + c);
-                else if (r != ENGRAM_INVALID_INDEX) flag(status, ENGRAM_ERR_INDEX);
+                if constexpr (SHARDED) {
+                    const uint4* src = s_src[rr * J + jt];
+                    if (src) v[u] = __ldcg(src + c);
+                    else if (r != ENGRAM_INVALID_INDEX) flag(status, ENGRAM_ERR_INDEX);
+                } else {
+                    if (r < s_rows[jt]) v[u] = __ldg(tables + (s_off[jt] + r) * cpr + c);
+                    else if (r != ENGRAM_INVALID_INDEX) flag(status, ENGRAM_ERR_INDEX);
+                }
             }
         }
 #pragma unroll
@@ -130,26 +167,54 @@ retrieve_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ P, 
 
 }  // namespace
 
-cudaError_t launch_retrieve(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
-                            int32_t t_begin, const HashParams& hp, const GatherParams& gp, const void* tables,
-                            uint32_t* idx, void* e_cat, uint32_t* status, cudaStream_t s) {
+namespace {
+
+int log2_or_neg(int v) {
+    if (v <= 0 || (v & (v - 1))) return -1;
+    int k = 0;
+    while ((1 << k) < v) ++k;
+    return k;
+}
+
+template <bool SHARDED>
+cudaError_t launch_retrieve_impl(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
+                                 int32_t t_begin, const HashParams& hp, const GatherParams& gp, const void* tables,
+                                 const ShardParams& sp, uint32_t* idx, void* e_cat, uint32_t* status, int num_sms,
+                                 cudaStream_t s) {
     const int64_t n = (int64_t)B * (T - t_begin);
     if (n == 0) return cudaSuccess;
-    const int rows_per_cta = kThreads / hp.J;
+    // 256 / J rows per CTA, or fewer when the batch is small (decode: a few
+    // hundred rows), so that the grid still spreads over every SM: the
+    // kernel is a chain of dependent loads, and a CTA's rows run one batch
+    // of loads after another
+    int rows_per_cta = kThreads / hp.J;
+    const int64_t spread = (n + 2 * (int64_t)num_sms - 1) / (2 * (int64_t)num_sms);
+    if (spread < rows_per_cta) rows_per_cta = (int)(spread < 1 ? 1 : spread);
     const int64_t blocks = (n + rows_per_cta - 1) / rows_per_cta;
-    auto log2_or_neg = [](int v) {
-        if (v <= 0 || (v & (v - 1))) return -1;
-        int k = 0;
-        while ((1 << k) < v) ++k;
-        return k;
-    };
     const int cpr_shift = log2_or_neg(gp.chunks_per_row);
     const int pr_shift = log2_or_neg(hp.J * gp.chunks_per_row);
-    retrieve_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(ids, P, B, T, stride, t_begin, hp, gp,
-                                                          static_cast<const uint4*>(tables), idx,
-                                                          static_cast<uint4*>(e_cat), rows_per_cta, cpr_shift,
-                                                          pr_shift, status);
+    retrieve_kernel<SHARDED><<<(unsigned)blocks, kThreads, 0, s>>>(
+        ids, P, B, T, stride, t_begin, hp, gp, static_cast<const uint4*>(tables), sp, idx, static_cast<uint4*>(e_cat),
+        rows_per_cta, cpr_shift, pr_shift, status);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_retrieve(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
+                            int32_t t_begin, const HashParams& hp, const GatherParams& gp, const void* tables,
+                            uint32_t* idx, void* e_cat, uint32_t* status, int num_sms, cudaStream_t s) {
+    ShardParams none{};
+    return launch_retrieve_impl<false>(ids, P, B, T, stride, t_begin, hp, gp, tables, none, idx, e_cat, status,
+                                       num_sms, s);
+}
+
+cudaError_t launch_retrieve_sharded(const int32_t* ids, const int32_t* P, int32_t B, int32_t T, int64_t stride,
+                                    int32_t t_begin, const HashParams& hp, const GatherParams& gp,
+                                    const ShardParams& sp, uint32_t* idx, void* e_cat, uint32_t* status, int num_sms,
+                                    cudaStream_t s) {
+    return launch_retrieve_impl<true>(ids, P, B, T, stride, t_begin, hp, gp, nullptr, sp, idx, e_cat, status,
+                                      num_sms, s);
 }
 
 }  // namespace engram

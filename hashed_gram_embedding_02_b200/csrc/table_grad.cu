@@ -1,0 +1,409 @@
+// Training backward for the tables: the gradient of every table row that a
+// batch looked up, as a sparse list of (row, summed gradient).
+//
+// "DeepSeek AI II" digest, section "DeepSeek Engram", the training
+// paragraph (and the Synced repost, "System efficiency"): the embedding
+// tables are trained with the model; the backward sends each accessed row's
+// gradient to the shard that stores it.  Since e_t is the concatenation of
+// the rows E_j[idx_j(t)], the gradient of row r of table j is the sum, over
+// the lookups (t, j) with idx_j(t) = r, of the slice j of dL/de_t.
+//
+// Deterministic: the sum of every row runs in increasing lookup order
+// (t * J + j), whatever order the atomics gave the work.
+//   1. dedupe: every valid lookup's global row (row_off[j] + idx) goes into an
+//      open-addressing set; the thread that claims a row gives it the next id
+//      and records the row; every lookup then learns its row's id and counts
+//      itself into its id's bucket.
+//   2. scan: exclusive prefix sum of the bucket sizes (three levels of
+//      4096-element blocks), the start of every row's segment.
+//   3. place: every lookup writes its position into its row's segment (in
+//      the order the atomics give).
+//   4. reduce: one warp per row orders its segment by position (each lookup's
+//      rank is the number of smaller positions in the segment) and sums the
+//      slices of dL/de in that order, in fp32, 16 bytes of the row per lane.
+// The cost of step 4 grows with the square of a row's lookup count: fine for
+// Zipf batches (the largest segments hold hundreds of lookups), slow for a
+// degenerate batch in which one n-gram fills it.
+#include <algorithm>
+
+#include "ctx.cuh"
+
+namespace engram {
+namespace {
+
+constexpr uint64_t kEmptyKey = 0;   // set key of an empty slot (keys are row + 1)
+constexpr int kScanThreads = 1024;
+constexpr int kScanPer = 4;         // elements per thread
+constexpr int kScanBlock = kScanThreads * kScanPer;
+
+__device__ __forceinline__ uint64_t mix64(uint64_t k) {
+    // Murmur3's 64-bit finaliser (Appleby), to spread row numbers over the set
+    k ^= k >> 33;
+    k *= 0xff51afd7ed558ccdull;
+    k ^= k >> 33;
+    k *= 0xc4ceb9fe1a85ec53ull;
+    k ^= k >> 33;
+    return k;
+}
+
+struct GradGeo {
+    int64_t row_off[kMaxTables];
+    uint32_t rows[kMaxTables];
+    int32_t J;
+};
+
+__device__ __forceinline__ int64_t find_slot(const unsigned long long* keys, uint32_t mask, unsigned long long key) {
+    uint32_t h = (uint32_t)mix64(key) & mask;
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+        const unsigned long long k = keys[h];
+        if (k == key) return h;
+        if (k == kEmptyKey) return -1;
+        h = (h + 1u) & mask;
+    }
+    return -1;
+}
+
+__global__ void grad_insert_kernel(const uint32_t* __restrict__ idx, int64_t n_lookups, GradGeo g,
+                                   unsigned long long* keys, uint32_t* vals, uint32_t mask, uint64_t* rows_out,
+                                   unsigned long long* count, uint32_t* status) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int j = (int)(i % g.J);
+        const uint32_t r = __ldg(idx + i);
+        if (r >= g.rows[j]) continue;                  // invalid n-gram: no row, no gradient
+        const unsigned long long key = (unsigned long long)(g.row_off[j] + r) + 1ull;
+        uint32_t h = (uint32_t)mix64(key) & mask;
+        bool placed = false;
+        for (uint32_t probe = 0; probe <= mask; ++probe) {
+            const unsigned long long prev = atomicCAS(keys + h, kEmptyKey, key);
+            if (prev == kEmptyKey) {
+                const unsigned long long id = atomicAdd(count, 1ull);
+                vals[h] = (uint32_t)id;
+                rows_out[id] = key - 1ull;
+                placed = true;
+                break;
+            }
+            if (prev == key) {
+                placed = true;
+                break;
+            }
+            h = (h + 1u) & mask;
+        }
+        if (!placed) flag(status, ENGRAM_ERR_INDEX);
+    }
+}
+
+// each valid lookup's row id (or 0xFFFFFFFF), and the size of every id's bucket
+__global__ void grad_id_kernel(const uint32_t* __restrict__ idx, int64_t n_lookups, GradGeo g,
+                               const unsigned long long* __restrict__ keys, const uint32_t* __restrict__ vals,
+                               uint32_t mask, uint32_t* __restrict__ lid, uint32_t* bucket) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int j = (int)(i % g.J);
+        const uint32_t r = __ldg(idx + i);
+        uint32_t id = 0xFFFFFFFFu;
+        if (r < g.rows[j]) {
+            const int64_t h = find_slot(keys, mask, (unsigned long long)(g.row_off[j] + r) + 1ull);
+            if (h >= 0) {
+                id = vals[h];
+                atomicAdd(bucket + id, 1u);
+            }
+        }
+        lid[i] = id;
+    }
+}
+
+// Exclusive scan of x[0, n) in blocks of kScanBlock: out gets the in-block
+// prefix, block_sum[b] the block's total.
+__global__ void __launch_bounds__(kScanThreads) scan_block_kernel(const uint32_t* __restrict__ x, int64_t n,
+                                                                  uint32_t* __restrict__ out,
+                                                                  uint32_t* __restrict__ block_sum) {
+    __shared__ uint32_t s_warp[kScanThreads / 32];
+    const int64_t base = (int64_t)blockIdx.x * kScanBlock + (int64_t)threadIdx.x * kScanPer;
+    uint32_t v[kScanPer];
+    uint32_t tsum = 0;
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) {
+        v[k] = base + k < n ? x[base + k] : 0u;
+        tsum += v[k];
+    }
+    // inclusive scan of the thread sums within the warp, then across warps
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t inc = tsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    uint32_t run = inc - tsum + (warp > 0 ? s_warp[warp - 1] : 0u);
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) {
+        if (base + k < n) out[base + k] = run;
+        run += v[k];
+    }
+    if (threadIdx.x == kScanThreads - 1) block_sum[blockIdx.x] = run;
+}
+
+__global__ void scan_add_kernel(uint32_t* __restrict__ out, int64_t n, const uint32_t* __restrict__ block_off) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] += block_off[i / kScanBlock];
+}
+
+// every lookup's position into its row's segment (order within a segment:
+// whatever the atomics give; the reduction orders it)
+__global__ void grad_place_kernel(const uint32_t* __restrict__ lid, int64_t n_lookups,
+                                  const uint32_t* __restrict__ start, uint32_t* cursor, uint32_t* __restrict__ seg) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t id = lid[i];
+        if (id == 0xFFFFFFFFu) continue;
+        seg[start[id] + atomicAdd(cursor + id, 1u)] = (uint32_t)i;
+    }
+}
+
+// One warp per distinct row: order the segment by position (into `sorted`,
+// each element's rank = the count of smaller positions), then sum the
+// slices of dL/de in that order.  Lane l owns the row's 16-byte chunks
+// l, l + 32, ... (D*elem/16 chunks in all).
+template <typename T>
+__global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint32_t* __restrict__ start,
+                                   const uint32_t* __restrict__ bucket, const unsigned long long* __restrict__ count,
+                                   uint32_t* __restrict__ sorted, const T* __restrict__ de, int J, int D,
+                                   float* __restrict__ grad) {
+    constexpr int EPC = 16 / sizeof(T);   // elements per 16-byte chunk
+    const int lane = threadIdx.x & 31;
+    const int64_t U = (int64_t)*count;
+    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int chunks = D / EPC;
+    const int64_t d_mem = (int64_t)J * D;
+    for (int64_t id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; id < U; id += warps) {
+        const uint32_t s0 = start[id], k = bucket[id];
+        const uint32_t* in = seg + s0;
+        uint32_t* srt = sorted + s0;
+        for (uint32_t a = lane; a < k; a += 32) {
+            const uint32_t x = in[a];
+            uint32_t rank = 0;
+            for (uint32_t b = 0; b < k; ++b) rank += in[b] < x;
+            srt[rank] = x;
+        }
+        __syncwarp();
+        for (int c = lane; c < chunks; c += 32) {
+            float acc[EPC];
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+            for (uint32_t a = 0; a < k; ++a) {
+                const uint32_t pos = srt[a];                   // lookup t * J + j
+                const int64_t t = pos / J, j = pos - t * J;
+                float f[EPC];
+                Vec<T>::load(de + t * d_mem + j * D + c * EPC, f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+            }
+            float* o = grad + id * D + c * EPC;
+#pragma unroll
+            for (int e = 0; e < EPC; e += 4) *reinterpret_cast<float4*>(o + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+        }
+    }
+}
+
+// tables[row] -= lr * grad, in the tables' dtype (fp32 arithmetic, one
+// rounding to the storage type); one warp per row
+template <typename T>
+__global__ void table_sgd_kernel(const uint64_t* __restrict__ rows, const float* __restrict__ grad,
+                                 const unsigned long long* __restrict__ count, int64_t max_rows, uint64_t total_rows,
+                                 int D, float lr, T* tables, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t U = min((int64_t)*count, max_rows);
+    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
+        const uint64_t r = rows[u];
+        if (r >= total_rows) {
+            if (lane == 0) flag(status, ENGRAM_ERR_INDEX);
+            continue;
+        }
+        for (int c = lane; c < D; c += 32) {
+            T& x = tables[r * D + c];
+            from_f(x, fmaf(-lr, grad[u * D + c], to_f(x)));
+        }
+    }
+}
+
+size_t set_slots(int64_t n_lookups) {
+    size_t cap = 1;
+    while ((int64_t)cap < 2 * n_lookups) cap <<= 1;
+    return cap;
+}
+
+struct GradWs {
+    unsigned long long* keys;
+    uint32_t* vals;
+    unsigned long long* count;
+    uint32_t* lid;
+    uint32_t* bucket;
+    uint32_t* start;
+    uint32_t* cursor;
+    uint32_t* seg;
+    uint32_t* sorted;
+    uint32_t* bsum1;
+    uint32_t* bsum2;
+    uint32_t* bsum3;
+    size_t bytes;
+};
+
+GradWs grad_carve(void* base, int64_t n) {
+    GradWs w{};
+    char* p = static_cast<char*>(base);
+    const size_t cap = set_slots(n);
+    const int64_t nb1 = (n + kScanBlock - 1) / kScanBlock;
+    const int64_t nb2 = (nb1 + kScanBlock - 1) / kScanBlock;
+    auto take = [&](size_t bytes) {
+        char* q = p;
+        p += align256(bytes);
+        return q;
+    };
+    w.keys = reinterpret_cast<unsigned long long*>(take(cap * 8));
+    w.vals = reinterpret_cast<uint32_t*>(take(cap * 4));
+    w.count = reinterpret_cast<unsigned long long*>(take(8));
+    w.lid = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
+    w.bucket = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
+    w.start = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
+    w.cursor = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
+    w.seg = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
+    w.sorted = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
+    w.bsum1 = reinterpret_cast<uint32_t*>(take((size_t)nb1 * 4));
+    w.bsum2 = reinterpret_cast<uint32_t*>(take((size_t)nb2 * 4));
+    w.bsum3 = reinterpret_cast<uint32_t*>(take(4));
+    w.bytes = (size_t)(p - static_cast<char*>(base));
+    return w;
+}
+
+constexpr int64_t kMaxGradLookups = (int64_t)kScanBlock * kScanBlock;   // two scan levels of 4096
+
+}  // namespace
+}  // namespace engram
+
+using namespace engram;
+
+extern "C" {
+
+size_t engram_table_grad_workspace_bytes(const engram_ctx* c, int64_t n_tok) {
+    if (!c || n_tok < 0) return 0;
+    return grad_carve(nullptr, std::max<int64_t>(1, n_tok * c->J)).bytes;
+}
+
+engram_status engram_table_grad(engram_ctx* c, const uint32_t* idx, int64_t n_tok, const void* d_e,
+                                uint64_t* rows_out, float* grad_out, uint64_t* n_unique, void* workspace,
+                                size_t workspace_bytes, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (n_tok < 0) return inval("n_tok must be >= 0");
+    const int64_t n = n_tok * c->J;
+    if (n > kMaxGradLookups) return inval("n_tok * J must be at most 2^24 lookups");
+    if (c->cfg.dtype == ENGRAM_FP8) {
+        set_error("engram_table_grad: FP8 tables are not trained here");
+        return ENGRAM_E_UNSUPPORTED;
+    }
+    if (!n_unique) return inval("null n_unique pointer");
+    if (n > 0 && (!idx || !d_e || !rows_out || !grad_out || !workspace)) return inval("null tensor pointer");
+    if (!aligned16(d_e) || !aligned16(grad_out)) return inval("d_e and grad_out must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    GradWs w = grad_carve(workspace, std::max<int64_t>(1, n));
+    if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    prof_reset(c);
+    const size_t cap = set_slots(std::max<int64_t>(1, n));
+    cudaError_t e = cudaMemsetAsync(w.keys, 0, cap * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(w.count, 0, 8, s);
+    if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.bucket, 0, (size_t)n * 4, s);
+    if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.cursor, 0, (size_t)n * 4, s);
+    if (e != cudaSuccess) return cuda_fail("table gradient: clearing the scratch", e);
+    if (n == 0) {
+        e = cudaMemcpyAsync(n_unique, w.count, 8, cudaMemcpyDeviceToDevice, s);
+        return e == cudaSuccess ? ENGRAM_OK : cuda_fail("table gradient: count", e);
+    }
+    GradGeo g{};
+    for (int j = 0; j < c->J; ++j) {
+        g.row_off[j] = c->gp.row_off[j];
+        g.rows[j] = c->gp.rows[j];
+    }
+    g.J = c->J;
+    const int threads = 256;
+    const int blocks = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)c->num_sms * 8);
+    const uint32_t mask = (uint32_t)(cap - 1);
+    prof_begin(c, s, "grad_dedupe");
+    grad_insert_kernel<<<blocks, threads, 0, s>>>(idx, n, g, w.keys, w.vals, mask, rows_out, w.count, c->d_status);
+    grad_id_kernel<<<blocks, threads, 0, s>>>(idx, n, g, w.keys, w.vals, mask, w.lid, w.bucket);
+    prof_end(c, s);
+    // segment starts: scan of the bucket sizes (ids >= U have empty buckets)
+    const int64_t nb1 = (n + kScanBlock - 1) / kScanBlock;
+    const int64_t nb2 = (nb1 + kScanBlock - 1) / kScanBlock;
+    prof_begin(c, s, "grad_scan");
+    scan_block_kernel<<<(unsigned)nb1, kScanThreads, 0, s>>>(w.bucket, n, w.start, w.bsum1);
+    scan_block_kernel<<<(unsigned)nb2, kScanThreads, 0, s>>>(w.bsum1, nb1, w.bsum1, w.bsum2);
+    scan_block_kernel<<<1, kScanThreads, 0, s>>>(w.bsum2, nb2, w.bsum2, w.bsum3);
+    if (nb2 > 1) scan_add_kernel<<<(unsigned)((nb1 + 255) / 256), 256, 0, s>>>(w.bsum1, nb1, w.bsum2);
+    if (nb1 > 1) scan_add_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.start, n, w.bsum1);
+    prof_end(c, s);
+    prof_begin(c, s, "grad_place");
+    grad_place_kernel<<<blocks, threads, 0, s>>>(w.lid, n, w.start, w.cursor, w.seg);
+    prof_end(c, s);
+    prof_begin(c, s, "grad_reduce");
+    const int rblocks = (int)std::min<int64_t>((n + 7) / 8, (int64_t)c->num_sms * 16);
+    if (c->cfg.dtype == ENGRAM_BF16)
+        grad_reduce_kernel<__nv_bfloat16><<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted,
+                                                                  static_cast<const __nv_bfloat16*>(d_e), c->J,
+                                                                  c->cfg.row_dim, grad_out);
+    else
+        grad_reduce_kernel<float><<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted,
+                                                          static_cast<const float*>(d_e), c->J, c->cfg.row_dim,
+                                                          grad_out);
+    prof_end(c, s);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaMemcpyAsync(n_unique, w.count, 8, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail("table gradient launches", e);
+    return ENGRAM_OK;
+}
+
+engram_status engram_table_sgd(engram_ctx* c, const uint64_t* rows, const float* grad, const uint64_t* n_unique,
+                               int64_t max_rows, void* tables, float lr, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (max_rows < 0) return inval("max_rows must be >= 0");
+    if (max_rows == 0) return ENGRAM_OK;
+    if (!rows || !grad || !n_unique || !tables) return inval("null tensor pointer");
+    if (c->cfg.dtype == ENGRAM_FP8) {
+        set_error("engram_table_sgd: FP8 tables are not trained here");
+        return ENGRAM_E_UNSUPPORTED;
+    }
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    uint64_t total = 0;
+    for (int j = 0; j < c->J; ++j) total += c->cfg.rows[j];
+    prof_reset(c);
+    prof_begin(c, s, "table_sgd");
+    const int blocks = (int)std::min<int64_t>((max_rows + 7) / 8, (int64_t)c->num_sms * 16);
+    if (c->cfg.dtype == ENGRAM_BF16)
+        table_sgd_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+            rows, grad, reinterpret_cast<const unsigned long long*>(n_unique), max_rows, total, c->cfg.row_dim, lr,
+            static_cast<__nv_bfloat16*>(tables), c->d_status);
+    else
+        table_sgd_kernel<float><<<blocks, 256, 0, s>>>(rows, grad, reinterpret_cast<const unsigned long long*>(n_unique),
+                                                       max_rows, total, c->cfg.row_dim, lr,
+                                                       static_cast<float*>(tables), c->d_status);
+    prof_end(c, s);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ENGRAM_OK : cuda_fail("table update launch", e);
+}
+
+}  // extern "C"

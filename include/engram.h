@@ -80,7 +80,14 @@ typedef enum engram_status {
 
 typedef enum engram_dtype {
     ENGRAM_F32 = 0,   /* tables, e, W, h, v, Y in fp32; projections on CUDA cores */
-    ENGRAM_BF16 = 1   /* tables, e, W, h, v, Y in bf16; projections on tcgen05 tensor cores */
+    ENGRAM_BF16 = 1,  /* tables, e, W, h, v, Y in bf16; projections on tcgen05 tensor cores */
+    ENGRAM_FP8 = 2    /* tables, e, W_K, W_V in FP8 E4M3 (1 byte: sign, 4 exponent bits with bias 7, 3
+                         mantissa bits; no infinities); h and Y in bf16; the projections as FP8 tcgen05
+                         GEMMs (kind::f8f6f4) with fp32 accumulation, dequantised per output channel by
+                         the k_scale / v_scale arguments of engram_forward_multibranch.  Needs d and J*D
+                         multiples of 128 and conv width 4 (the fused path); only the forward entry
+                         points take it ("DeepSeek AI II" digest, section "DeepSeek Engram": the
+                         multi-branch projections fuse into one dense FP8 GEMM) */
 } engram_dtype;
 
 /* device status word bits (engram_device_status) */
@@ -111,7 +118,8 @@ typedef struct engram_config {
 typedef struct engram_ctx engram_ctx;
 
 /* Validate cfg (orders ascending in 1..4, J <= 32, every M prime and < 2^31,
- * D*elem a multiple of 16 bytes, d a multiple of 8, V' < 2^31 - 1) and bind a
+ * D*elem a multiple of 16 bytes, d a multiple of 8, V' < 2^31 - 1; for
+ * ENGRAM_FP8 also d and J*D multiples of 128 and conv width 4) and bind a
  * context to the CURRENT device.  Allocates a 256-byte device status block.
  * Returns ENGRAM_E_INVAL for a bad config, ENGRAM_E_CUDA/NOMEM on failure. */
 ENGRAM_API engram_status engram_create(const engram_config* cfg, engram_ctx** out);
@@ -234,6 +242,129 @@ ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int
                              float* conv_state, void* y, float* alpha_out, int32_t add_residual,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ------------------------------------------------------------ multi-branch
+ *
+ * The pages ("DeepSeek AI II" digest, section "DeepSeek Engram", the
+ * multi-branch paragraphs; the Synced repost, "context-aware gating") use a
+ * backbone whose residual stream has M parallel branches.  All branches share
+ * the sparse tables and the value projection W_V; branch m has its own key
+ * projection W_K^(m) and hidden state h^(m), hence its own gate
+ *   alpha^(m)_t = sigmoid(<RMSNorm(h^(m)_t), RMSNorm(W_K^(m) e_t)> / sqrt(d)),
+ * applied to the shared value: u^(m)_t = alpha^(m)_t * (W_V e_t).  The
+ * projections fuse into dense GEMMs over [W_V; W_K^(1..M)]: here one key pass
+ * over the stacked W_K^(1..M) (N = M*d) yields the M gates per token, and one
+ * value pass computes v once and, in its epilogue, applies each branch's
+ * gate, the causal depthwise conv, SiLU and the residual, writing M outputs.
+ * Readings (the pages stop at u^(m)): each branch's u^(m) goes through the
+ * same conv as the single-branch module (shared conv_w, a history per
+ * branch), and the RMSNorm gains are per branch.
+ *   h          [M][B*L][d] (model dtype), branch-major;
+ *   Wk         [M][d][J*D]: W_K^(m) stacked;       Wv [d][J*D], shared;
+ *   gq, gk     [M][d] fp32 or null (ones);           conv_w [d][w], shared;
+ *   conv_state [M][B][w-1][d] fp32 or null;          y [M][B*L][d];
+ *   alpha_out  [M][B*L] fp32 or null;
+ *   k_scale    [M][d] fp32 or null, v_scale [d] fp32 or null: per output
+ *              channel factors applied to the GEMM accumulators, k^(m)_c =
+ *              k_scale[m][c] * (W_K^(m) e)_c and v_c = v_scale[c] * (W_V e)_c:
+ *              the dequantisation of FP8 operands (the tables' scale times
+ *              the weight row's scale), or null for 1 (16-byte aligned).
+ * M in 1..ENGRAM_MAX_BRANCHES.  With ENGRAM_FP8 tables, e, W_K and W_V are
+ * E4M3 bytes and the fused GEMM over [W_V; W_K^(1..M)] runs as FP8 MMAs, as
+ * the pages describe.  Runs on the fused tensor-core path only
+ * (bf16, conv width 4, d a multiple of 128, J*D a multiple of 64);
+ * otherwise ENGRAM_E_UNSUPPORTED.  Scratch: engram_multibranch_workspace_bytes
+ * (M = 1 gives engram_workspace_bytes). */
+#define ENGRAM_MAX_BRANCHES 4
+ENGRAM_API size_t engram_multibranch_workspace_bytes(const engram_ctx* ctx, int32_t M, int32_t B, int32_t L);
+ENGRAM_API engram_status engram_forward_multibranch(engram_ctx* ctx, int32_t M, const int32_t* tok, int32_t B,
+                                                    int32_t T, int64_t tok_stride, int32_t t_begin, const int32_t* P,
+                                                    const void* tables, const void* h, const void* Wk, const void* Wv,
+                                                    const float* gq, const float* gk, const float* k_scale,
+                                                    const float* v_scale, const float* conv_w, float* conv_state,
+                                                    void* y, float* alpha_out, int32_t add_residual,
+                                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------ sharded tables
+ *
+ * Tables split across GPUs.  The pages ("DeepSeek AI II" digest, section
+ * "DeepSeek Engram", the training paragraph; the Synced repost, section
+ * "System efficiency: decoupling compute and storage") shard the embedding
+ * tables over the available GPUs so that capacity grows with their number,
+ * and bring the accessed rows to each GPU in the forward (an all-to-all).
+ * Here the rows of all J tables, numbered globally (table j's row r is global
+ * row sum_{i<j} M_i + r), are split into n_shards contiguous ranges of
+ * ceil(R / n_shards) rows (R = sum of M_j; the last range may be shorter or
+ * empty); engram_shard_range gives the range of shard g.  Shard g stores its
+ * rows back to back, D elements of the model dtype per row.  The forward's
+ * retrieval kernel reads every row directly from the shard that owns it:
+ * shard_tables[g] is a device pointer valid on THIS GPU, to this GPU's own
+ * memory or to another GPU's memory mapped here (engram_ipc_open, or peer
+ * access).  Remote rows cross NVLink once, with plain loads, and land in
+ * this GPU's e_cat before the projections read them: the all-to-all of
+ * indices and rows is one-sided reads inside the retrieval. */
+ENGRAM_API engram_status engram_shard_range(const engram_ctx* ctx, int32_t n_shards, int32_t shard,
+                                            int64_t* first_row, int64_t* n_rows);
+/* engram_forward with the tables given as n_shards (1..16) shards instead of
+ * one array: shard_tables is a HOST array of n_shards device pointers (16-byte
+ * aligned; null only for an empty shard).  Every other argument and the
+ * result are engram_forward's; an index whose row no shard covers gathers a
+ * zero row and sets ENGRAM_ERR_INDEX.  The shards must stay mapped until the
+ * call completes on `stream`; nothing is exchanged between GPUs except these
+ * reads, so the caller's only ordering duty is that the shards hold their
+ * rows before the call (they are read-only here). */
+ENGRAM_API engram_status engram_forward_sharded(engram_ctx* ctx, const int32_t* tok, int32_t B, int32_t T,
+                                                int64_t tok_stride, int32_t t_begin, const int32_t* P,
+                                                const void* const* shard_tables, int32_t n_shards, const void* h,
+                                                const void* Wk, const void* Wv, const float* gq, const float* gk,
+                                                const float* conv_w, float* conv_state, void* y, float* alpha_out,
+                                                int32_t add_residual, void* workspace, size_t workspace_bytes,
+                                                cudaStream_t stream);
+/* Cross-process mapping of a shard (plumbing for one process per GPU).
+ * engram_ipc_export: the cudaMalloc allocation that contains the device
+ * pointer `ptr`, as a 64-byte CUDA IPC handle (handle_out) plus the offset of
+ * `ptr` in it.  engram_ipc_open (in another process, any GPU with peer
+ * access to the owner): maps that allocation into the calling process on the
+ * current device and returns the pointer at the offset (*ptr_out) and the
+ * mapping's base (*base_out, for engram_ipc_close).  Memory from a
+ * virtual-memory (cuMemMap) allocator cannot be exported: ENGRAM_E_CUDA. */
+#define ENGRAM_IPC_HANDLE_BYTES 64
+ENGRAM_API engram_status engram_ipc_export(const void* ptr, void* handle_out, uint64_t* offset_out);
+ENGRAM_API engram_status engram_ipc_open(const void* handle, uint64_t offset, void** ptr_out, void** base_out);
+ENGRAM_API engram_status engram_ipc_close(void* base);
+
+/* ------------------------------------------------------------ table backward
+ *
+ * The tables are trained with the model ("DeepSeek AI II" digest, section
+ * "DeepSeek Engram", the training paragraph: the backward sends each
+ * accessed row's gradient to the shard that holds it).  e_t concatenates
+ * the rows E_j[idx_j(t)], so the gradient of table j's row r is the sum of
+ * slice j of dL/de_t over the lookups (t, j) with idx_j(t) = r; rows no
+ * lookup touched have zero gradient and are not listed.
+ *
+ * engram_table_grad: idx [n_tok][J] (engram_hash's output), d_e
+ * [n_tok][J*D] in the context dtype (16-byte aligned).  Writes, for the U
+ * distinct rows the valid lookups touched: rows_out[u] = the global row
+ * (sum_{i<j} M_i + r) and grad_out[u][D] (fp32, 16-byte aligned) its
+ * summed gradient, u < U; *n_unique (DEVICE uint64) = U.  Capacity: n_tok*J
+ * rows in rows_out and grad_out.  Invalid indices (an n-gram with an
+ * invalid id) contribute nothing.  Each row's sum runs in increasing lookup
+ * order (t * J + j) in fp32, so the (row, gradient) pairs are the same on
+ * every run; which u a row lands at depends on the device's atomics.
+ * n_tok * J <= 2^24.  Scratch: engram_table_grad_workspace_bytes(ctx, n_tok)
+ * bytes, 256-byte aligned.
+ *
+ * engram_table_sgd: tables[rows[u]] -= lr * grad[u] for u < min(*n_unique,
+ * max_rows), in fp32 arithmetic with one rounding to the tables' dtype;
+ * tables as in engram_gather.  A row outside the tables sets
+ * ENGRAM_ERR_INDEX and is skipped. */
+ENGRAM_API size_t engram_table_grad_workspace_bytes(const engram_ctx* ctx, int64_t n_tok);
+ENGRAM_API engram_status engram_table_grad(engram_ctx* ctx, const uint32_t* idx, int64_t n_tok, const void* d_e,
+                                           uint64_t* rows_out, float* grad_out, uint64_t* n_unique, void* workspace,
+                                           size_t workspace_bytes, cudaStream_t stream);
+ENGRAM_API engram_status engram_table_sgd(engram_ctx* ctx, const uint64_t* rows, const float* grad,
+                                          const uint64_t* n_unique, int64_t max_rows, void* tables, float lr,
+                                          cudaStream_t stream);
+
 /* engram_forward for callers that cannot allocate device memory (an engine
  * callback where allocation is forbidden, a process whose device memory is
  * all owned by another allocator, a loop that cannot afford cudaMalloc's
@@ -241,9 +372,11 @@ ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int
  * interface of this library only.  Same arguments as engram_forward without
  * the workspace: the scratch lives in a static device array of
  * ENGRAM_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
- * the process exits.  The first call on a device looks up that array's
- * device address (cudaGetSymbolAddress), so make it before any stream
- * capture.  Calls needing more than the array (engram_workspace_bytes(ctx,
+ * the process exits.  Every call whose stream is not capturing looks up that
+ * array's device address on the current device (cudaGetSymbolAddress); a
+ * call on a capturing stream reuses the last address looked up, so the first
+ * call on a device must come before any stream capture.  The context's device
+ * must be current (ENGRAM_E_INVAL otherwise, before anything is looked up).  Calls needing more than the array (engram_workspace_bytes(ctx,
  * B, T - t_begin)) return ENGRAM_E_NOMEM with an explanation in
  * engram_last_error and launch nothing.  No cudaMalloc or cudaFree is called.
  * All calls share the one array, which keeps the last call's contents (the
@@ -353,6 +486,57 @@ ENGRAM_API engram_status engram_host_fetch(engram_host_tier* tier, cudaStream_t 
  * the slot map: the same kernel and layout as engram_gather. */
 ENGRAM_API engram_status engram_gather_staged(engram_host_tier* tier, int64_t n_tok, void* e_cat,
                                               cudaStream_t stream);
+/* Hot-row cache in HBM in front of the host tables.  The pages (the
+ * "DeepSeek AI II" digest, section "DeepSeek Engram", last paragraph; the
+ * Synced repost, section "System efficiency: decoupling compute and
+ * storage", last paragraph) keep the frequently accessed n-gram rows in a
+ * faster tier, since a few patterns take most accesses under the Zipf law.
+ * capacity_rows rows of device memory (plus a hash set of 2^ceil(log2(2 C))
+ * 12-byte entries) are allocated once, here; the tier's staged-row buffer
+ * is re-allocated to hold the cache slots in front of the staged rows.
+ * From the next batch on, engram_host_dedupe resolves every distinct row
+ * against the cache: resident rows are gathered from HBM and not fetched.
+ * engram_gather_staged then admits the rows this batch fetched and looked up
+ * at least min_count times (2 keeps the one-off tail out) into free slots
+ * until the cache is full; nothing is evicted (engram_host_cache_reset
+ * empties it).  Which rows win the last free slots depends on the device's
+ * atomics; the gathered e_cat never does.  Call before the first batch.
+ * ENGRAM_E_NOMEM when the device memory is short. */
+ENGRAM_API engram_status engram_host_cache_enable(engram_host_tier* tier, int64_t capacity_rows, int32_t min_count);
+/* Enqueue on `stream`: empty the hot-row cache. */
+ENGRAM_API engram_status engram_host_cache_reset(engram_host_tier* tier, cudaStream_t stream);
+/* Figures of the last batch (valid once its fetch has returned). */
+typedef struct {
+    int64_t capacity;        /* cache slots */
+    int64_t resident;        /* slots in use when the batch was deduplicated */
+    int64_t lookups;         /* the batch's lookups (n_tok * J) */
+    int64_t cached_lookups;  /* lookups served from the cache */
+    int64_t cached_rows;     /* distinct rows served from the cache (not fetched) */
+    int64_t fetched_rows;    /* distinct rows fetched over PCIe */
+} engram_host_cache_stats_t;
+ENGRAM_API engram_status engram_host_cache_stats(const engram_host_tier* tier, engram_host_cache_stats_t* out);
+
+/* Test hook for the host-side failure paths (failure detection without a
+ * GPU fault; every failure is made on the host).  `inject` arms one-shot
+ * faults for the next fetch:
+ *   ENGRAM_INJECT_LIST_WAIT     the wait for the distinct-row list is told the
+ *                               list never arrives (the event query's answer
+ *                               is replaced), so the fetch returns
+ *                               ENGRAM_E_TIMEOUT after the wait limit;
+ *   ENGRAM_INJECT_PACK_ABANDON  the packing thread that takes the last chunk
+ *                               of the batch gives it up without packing or
+ *                               marking it, so the fetch returns ENGRAM_E_HOST
+ *                               after the wait limit; the copies of the
+ *                               earlier chunks, already enqueued, are
+ *                               recorded, and the next fetch waits for them.
+ * wait_limit_s replaces the 20 s bound of every host-side wait of the tier
+ * (list, previous copies, packed chunks) from now on.  After either failure
+ * the tier stays usable: the next dedupe + fetch + gather_staged is correct;
+ * engram_gather_staged refuses to run on the failed batch. */
+#define ENGRAM_INJECT_LIST_WAIT 0x1u
+#define ENGRAM_INJECT_PACK_ABANDON 0x2u
+ENGRAM_API engram_status engram_host_tier_debug(engram_host_tier* tier, uint32_t inject, double wait_limit_s);
+
 /* Figures of the last fetch. */
 typedef struct {
     int64_t n_unique;   /* distinct rows fetched */

@@ -12,7 +12,7 @@ def config_for(inp, eb, eps: float = 1e-6):
     wl = inp.wl
     return eb.make_config(orders=wl.orders, heads=wl.K, rows=[int(x) for x in inp.rows], mult=inp.mult,
                           row_dim=wl.D, hidden=wl.d, conv_width=wl.w, vocab=wl.V, canon_vocab=wl.Vc,
-                          dtype=eb.ENGRAM_BF16 if wl.dtype == "bf16" else eb.ENGRAM_F32, eps=eps)
+                          dtype={"bf16": eb.ENGRAM_BF16, "f32": eb.ENGRAM_F32, "fp8": eb.ENGRAM_FP8}[wl.dtype], eps=eps)
 
 
 class DeviceInputs:

@@ -181,3 +181,133 @@ def test_c5_batch_forward_sampled_matches_oracle(eb):
     err = np.abs(y_s - ref.y)
     assert err.max() <= 2e-2
     assert not (err > bf16_bound(ref.y, ref.vt_win, inp.conv_w)).any()
+
+
+# ---------------------------------------------------------------- failure paths (made on the host)
+
+@pytest.mark.parametrize("inject,status", [("list", "timeout"), ("pack", "host")])
+def test_fetch_failure_is_reported_and_the_tier_recovers(eb, inject, status):
+    """A host-side fault of one fetch: the distinct-row list that never
+    arrives (the event query's answer is faked), or a packing thread that
+    abandons the batch's last chunk.  The fetch returns ENGRAM_E_TIMEOUT or
+    ENGRAM_E_HOST within a few seconds, gather_staged refuses the failed
+    batch, and the next batch on the same tier matches the HBM gather bit for
+    bit.  Nothing faults or stalls the GPU."""
+    import time
+    wl = SMALL
+    inp = synth.Inputs(wl)
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    host = inp.host_tables("cuda:0")
+    # one thread: the abandoned chunk is the last one, after the earlier
+    # chunks' copies were enqueued (their end must be recorded for the next fetch)
+    tier = eb.HostTier(ctx, host, max_lookups=wl.n_tok * wl.J, n_threads=1)
+    idx = _indices(eb, ctx, di, wl)
+    side = torch.cuda.Stream()
+    tier.debug(eb.ENGRAM_INJECT_LIST_WAIT if inject == "list" else eb.ENGRAM_INJECT_PACK_ABANDON, 1.0)
+    tier.dedupe(idx, wl.n_tok)
+    t0 = time.time()
+    with pytest.raises(eb.EngramError) as err:
+        tier.fetch(side)
+    took = time.time() - t0
+    want = eb.ENGRAM_E_TIMEOUT if status == "timeout" else eb.ENGRAM_E_HOST
+    assert err.value.status == want
+    assert 0.9 <= took < 10.0, took
+    e = torch.empty(wl.n_tok, wl.d_mem, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(eb.EngramError) as err2:
+        tier.gather(wl.n_tok, e)
+    assert err2.value.status == eb.ENGRAM_E_INVAL
+    # the next batch, same tier
+    e_t, n_unique = _staged_e(eb, ctx, tier, idx, wl, side)
+    e_d = torch.empty_like(e_t)
+    eb.engram_gather(ctx.ctx, idx, wl.n_tok, di.tables, e_d)
+    torch.cuda.synchronize()
+    assert torch.equal(e_t, e_d)
+    assert n_unique == _distinct_rows(idx, inp)
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    tier.close()
+
+
+# ---------------------------------------------------------------- hot-row cache in HBM
+
+def _batches(wl, n):
+    """n token batches of the same workload (different seeds); the tables are batch 0's for all."""
+    return [synth.Inputs(wl.replace(seed=wl.seed + k)) for k in range(n)]
+
+
+def _distinct_split(idx, inp, cached_keys):
+    off = np.concatenate([[0], np.cumsum(inp.rows[:-1].astype(np.int64))])
+    ix = idx.cpu().numpy().view(np.uint32).astype(np.int64)
+    valid = ix < inp.rows[None, :].astype(np.int64)
+    keys, counts = np.unique((ix + off[None, :])[valid], return_counts=True)
+    return keys, counts
+
+
+@pytest.mark.parametrize("capacity", [60000, 500])
+def test_hot_row_cache_over_batches(eb, capacity):
+    """Five consecutive batches through a tier with a hot-row cache: each
+    batch's staged gather equals the HBM gather bit for bit; fetched +
+    cached rows = the batch's distinct rows; the first batch finds the cache
+    empty and fetches everything; the cache fills with rows looked up at
+    least twice, never beyond its capacity; later batches take rows from it;
+    a reset empties it."""
+    wl = SMALL
+    batches = _batches(wl, 5)
+    ctx = eb.Engram(config_for(batches[0], eb))
+    host = batches[0].host_tables("cuda:0")
+    tables_d = batches[0].device_tables("cuda:0")
+    tier = eb.HostTier(ctx, host, max_lookups=wl.n_tok * wl.J, n_threads=4)
+    tier.enable_cache(capacity, min_count=2)
+    side = torch.cuda.Stream()
+    admitted_possible = set()         # rows looked up >= 2 times in some earlier batch
+    resident_prev = 0
+    for k, inp in enumerate(batches):
+        tok = torch.from_numpy(inp.tok).cuda()
+        P = torch.from_numpy(inp.P).cuda()
+        idx = torch.empty(wl.n_tok, wl.J, dtype=torch.int32, device="cuda")
+        eb.engram_hash(ctx.ctx, tok, P, wl.B, wl.T, wl.T, 0, idx)
+        e_t = torch.full((wl.n_tok, wl.d_mem), float("nan"), dtype=torch.bfloat16, device="cuda")
+        tier.dedupe(idx, wl.n_tok)
+        n_fetched = tier.fetch(side)
+        tier.gather(wl.n_tok, e_t)
+        e_d = torch.empty_like(e_t)
+        eb.engram_gather(ctx.ctx, idx, wl.n_tok, tables_d, e_d)
+        torch.cuda.synchronize()
+        assert torch.equal(e_t, e_d), k
+        keys, counts = _distinct_split(idx, batches[0], None)
+        cs = tier.cache_stats()
+        assert cs["capacity"] == capacity
+        assert cs["fetched_rows"] == n_fetched
+        assert cs["fetched_rows"] + cs["cached_rows"] == len(keys)
+        assert cs["lookups"] == wl.n_tok * wl.J
+        assert cs["resident"] >= resident_prev and cs["resident"] <= capacity
+        if k == 0:
+            assert cs["cached_rows"] == 0 and cs["resident"] == 0
+        else:
+            # every row served from the cache was a candidate of an earlier batch
+            assert cs["cached_rows"] > 0
+            assert cs["cached_rows"] <= len(set(keys.tolist()) & admitted_possible)
+            assert cs["cached_lookups"] >= cs["cached_rows"]
+        admitted_possible |= set(keys[counts >= 2].tolist())
+        resident_prev = cs["resident"]
+    if capacity == 500:
+        assert resident_prev == 500
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    # a reset empties the cache: the next batch fetches every distinct row
+    tier.reset_cache()
+    inp = batches[1]
+    idx = torch.empty(wl.n_tok, wl.J, dtype=torch.int32, device="cuda")
+    eb.engram_hash(ctx.ctx, torch.from_numpy(inp.tok).cuda(), torch.from_numpy(inp.P).cuda(), wl.B, wl.T, wl.T, 0,
+                   idx)
+    e_t = torch.empty(wl.n_tok, wl.d_mem, dtype=torch.bfloat16, device="cuda")
+    tier.dedupe(idx, wl.n_tok)
+    tier.fetch(side)
+    tier.gather(wl.n_tok, e_t)
+    torch.cuda.synchronize()
+    cs = tier.cache_stats()
+    assert cs["cached_rows"] == 0 and cs["resident"] == 0
+    e_d = torch.empty_like(e_t)
+    eb.engram_gather(ctx.ctx, idx, wl.n_tok, tables_d, e_d)
+    torch.cuda.synchronize()
+    assert torch.equal(e_t, e_d)
+    tier.close()
