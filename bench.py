@@ -709,6 +709,8 @@ def main():
     roofline = {"kernel": dominant, "bound": dk.get("bound"), "achieved": dk.get("achieved"),
                 "peak": tf_burst if dk.get("bound") == "tensor" else hbm, "unit": dk.get("unit"),
                 "frac": dk.get("frac"), "traffic": dk.get("traffic"),
+                # context: the same rate against the sustained (power-capped) figure
+                "frac_of_sustained": (dk.get("achieved") / tf_sust) if dk.get("bound") == "tensor" else None,
                 "peak_source": f"{peak_src} " + ("bf16 burst" if dk.get("bound") == "tensor" else "HBM copy"),
                 "algorithmic": (f"{work[dominant][1]:.4g} FLOP per launch (2*n*d_mem*d per projection)"
                                 if dk.get("bound") == "tensor" else f"{work.get(dominant, (0, 0))[1]:.4g} bytes per launch")}

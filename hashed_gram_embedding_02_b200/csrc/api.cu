@@ -99,6 +99,7 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
     w.alpha = reinterpret_cast<float*>(p);
     p += align256((size_t)M * n * sizeof(float));
     w.band = reinterpret_cast<int*>(p);
+    w.counter_bytes = band_bytes(n);
     p += align256(band_bytes(n));
     const size_t hist_bytes =
         align256((size_t)M * B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
@@ -157,6 +158,25 @@ engram_status conv_impl(engram_ctx* c, const float* v, const float* part, const 
     return launched("gate/conv launch", e);
 }
 
+// Decode-shaped fused calls read the conv history from a sequence-minor copy
+// [w-1][d][B]: the transpose runs on the side stream (it needs only the
+// caller's conv_state), and the value pass waits for aux_ev[1].
+engram_status launch_history_transpose(engram_ctx* c, float* state, const Workspace& w, int32_t B, int M,
+                                       cudaStream_t s) {
+    const size_t hist_elems = (size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden;
+    cudaError_t e = cudaEventRecord(c->aux_ev[0], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(c->aux, c->aux_ev[0], 0);
+    if (e != cudaSuccess) return cuda_fail("ordering the history transpose", e);
+    prof_begin(c, c->aux, "state_to_tr");
+    for (int m = 0; m < M && e == cudaSuccess; ++m)
+        e = launch_state_to_tr(state + m * hist_elems, w.state_t + m * hist_elems, B, c->cfg.conv_width,
+                               c->cfg.hidden, c->aux);
+    prof_end(c, c->aux);
+    if (e == cudaSuccess) e = cudaEventRecord(c->aux_ev[1], c->aux);
+    if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
+    return ENGRAM_OK;
+}
+
 // projections + gate + conv; on the fused path two tcgen05 GEMM passes with
 // the gate and the conv in the second one's epilogue, otherwise the
 // projection (tcgen05 or CUDA cores) followed by the CUDA-core gate/conv.
@@ -176,28 +196,19 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
     if (fused_path(c, n)) {
         const bool tr = state && decode_shaped(c, n, L);
         cudaError_t e = cudaSuccess;
-        if (tr) {
-            // the history transpose only needs the caller's conv_state: it runs on
-            // the side stream while the key pass (a few dozen CTAs at decode
-            // sizes) computes, and the value pass waits for it
-            e = cudaEventRecord(c->aux_ev[0], s);
-            if (e == cudaSuccess) e = cudaStreamWaitEvent(c->aux, c->aux_ev[0], 0);
-            if (e != cudaSuccess) return cuda_fail("ordering the history transpose", e);
-            prof_begin(c, c->aux, "state_to_tr");
-            for (int m = 0; m < M && e == cudaSuccess; ++m)
-                e = launch_state_to_tr(state + m * hist_elems, w.state_t + m * hist_elems, B, c->cfg.conv_width,
-                                       c->cfg.hidden, c->aux);
-            prof_end(c, c->aux);
-            if (e == cudaSuccess) e = cudaEventRecord(c->aux_ev[1], c->aux);
-            if (e != cudaSuccess) return cuda_fail("conv-state transpose launch", e);
+        // after_retrieve: the forward launched the transpose ahead of the
+        // retrieval, so nothing stands between the retrieval and the key pass
+        if (tr && !after_retrieve) {
+            engram_status st = launch_history_transpose(c, state, w, B, M, s);
+            if (st != ENGRAM_OK) return st;
         }
         if (!after_retrieve) {
-            e = cudaMemsetAsync(w.band, 0, band_bytes(n), s);
+            e = cudaMemsetAsync(w.band, 0, w.counter_bytes, s);
             if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
         }
         prof_begin(c, s, "gate_k_tc");
         e = launch_gate_k_tc(e_cat, n, c->d_mem, h, Wk, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band, w.alpha,
-                             alpha_out, c->d_status, c->num_sms, c->debug_stall, after_retrieve && !tr && !c->prof,
+                             alpha_out, c->d_status, c->num_sms, c->debug_stall, after_retrieve && !c->prof,
                              s, M, f8, kscale);
         c->debug_stall = 0;
         prof_end(c, s);
@@ -247,9 +258,13 @@ engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t
                            const ShardParams* shards, int M, const float* kscale, const float* vscale) {
     const int32_t L = T - t_begin;
     const bool fused = fused_path(c, (int64_t)B * L);
+    if (fused && conv_state && decode_shaped(c, (int64_t)B * L, L)) {
+        engram_status st = launch_history_transpose(c, conv_state, w, B, M, s);
+        if (st != ENGRAM_OK) return st;
+    }
     if (fused) {
         // cleared ahead of the retrieval, so that the key pass directly follows it
-        cudaError_t e = cudaMemsetAsync(w.band, 0, band_bytes((int64_t)B * L), s);
+        cudaError_t e = cudaMemsetAsync(w.band, 0, w.counter_bytes, s);
         if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
     }
     prof_begin(c, s, shards ? "retrieve_sharded" : "retrieve");
@@ -605,8 +620,12 @@ engram_status engram_forward_multibranch(engram_ctx* c, int32_t M, const int32_t
                   "a multiple of 128, J*D a multiple of 64 (128 for FP8))");
         return ENGRAM_E_UNSUPPORTED;
     }
-    if ((k_scale && !aligned16(k_scale)) || (v_scale && !aligned16(v_scale)))
-        return inval("k_scale and v_scale must be 16-byte aligned");
+    if (c->cfg.dtype == ENGRAM_FP8) {
+        if (!k_scale || !v_scale) return inval("FP8 needs k_scale and v_scale (the dequantisation scales)");
+        if (!aligned16(k_scale) || !aligned16(v_scale)) return inval("k_scale and v_scale must be 16-byte aligned");
+    } else if (k_scale || v_scale) {
+        return inval("k_scale and v_scale dequantise FP8 operands: pass null for other dtypes");
+    }
     if (!tok || !P || !tables || !h || !Wk || !Wv || !conv_w || !y || !workspace) return inval("null tensor pointer");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
     Workspace w = carve(c, workspace, B, L, true, M);

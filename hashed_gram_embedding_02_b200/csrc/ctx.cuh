@@ -72,6 +72,7 @@ struct Workspace {
     float* state_next;
     float* state_t;     // decode-shaped fused calls: the history, sequence-minor
     float* v;
+    size_t counter_bytes;   // band counters: cleared before every fused call
     size_t bytes;
 };
 // M > 1 (multi-branch, fused path only): part [n][M*G][4], alpha [M][n],

@@ -447,6 +447,7 @@ __device__ __forceinline__ void unpack8(const uint4& q, float* f) {
 // TMEM column taddr and tile-local channel cl; gains s_gg and the key
 // channels' dequantisation scales s_ks indexed tile-locally.  TMEM loads run
 // one 16-column chunk ahead of the math.
+template <bool SCALED>
 __device__ __forceinline__ void partials_cols(uint32_t taddr, const uint8_t* hs, int i, bool valid, int cl,
                                               int ncols, const float* s_gg, const float* s_ks, float& s_qk,
                                               float& s_kk, float& s_hh) {
@@ -471,12 +472,16 @@ __device__ __forceinline__ void partials_cols(uint32_t taddr, const uint8_t* hs,
                     const float4 g0 = *reinterpret_cast<const float4*>(s_gg + c8);
                     const float4 g1 = *reinterpret_cast<const float4*>(s_gg + c8 + 4);
                     const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                    const float4 k0 = *reinterpret_cast<const float4*>(s_ks + c8);
-                    const float4 k1 = *reinterpret_cast<const float4*>(s_ks + c8 + 4);
-                    const float ks[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    float ks[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                    if constexpr (SCALED) {
+                        const float4 k0 = *reinterpret_cast<const float4*>(s_ks + c8);
+                        const float4 k1 = *reinterpret_cast<const float4*>(s_ks + c8 + 4);
+                        ks[0] = k0.x; ks[1] = k0.y; ks[2] = k0.z; ks[3] = k0.w;
+                        ks[4] = k1.x; ks[5] = k1.y; ks[6] = k1.z; ks[7] = k1.w;
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float kf = __uint_as_float(cur[u * 8 + e]) * ks[e];
+                        const float kf = SCALED ? __uint_as_float(cur[u * 8 + e]) * ks[e] : __uint_as_float(cur[u * 8 + e]);
                         s_qk = fmaf(gg[e] * hf[e], kf, s_qk);
                         s_kk = fmaf(kf, kf, s_kk);
                         s_hh = fmaf(hf[e], hf[e], s_hh);
@@ -498,11 +503,12 @@ __device__ __forceinline__ void load_gains(const EpiParams& p, int c0, int n, fl
 // Partials over the channel slice [cl0, cl0 + ncols) of this warp's part,
 // added across the parts of each 128-channel group in a fixed order through
 // s_red, written by the group's first part.
+template <bool SCALED>
 __device__ __forceinline__ void group_partials(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int64_t row,
                                                int i, bool valid, int part, int cl0, int ncols, int parts_per_group,
                                                int g, const float* s_gg, const float* s_ks, float4* s_red) {
     float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-    partials_cols(taddr, hs, i, valid, cl0, ncols, s_gg, s_ks, s_qk, s_kk, s_hh);
+    partials_cols<SCALED>(taddr, hs, i, valid, cl0, ncols, s_gg, s_ks, s_qk, s_kk, s_hh);
     s_red[part * BM + i] = make_float4(s_qk, s_kk, s_hh, 0.f);
     epi_sync();
     if (part % parts_per_group == 0 && valid) {
@@ -527,11 +533,10 @@ __device__ __forceinline__ void epilogue_kv(uint32_t taddr, const uint8_t* hs, c
     const int c0 = nt * 128;
     epi_sync();                       // previous tile's readers are done with s_gg and s_red
     load_gains(p, c0, 128, s_gg, et);
-    if (et < 128) s_gg[128 + et] = 1.f;    // no key scales on this path
     epi_sync();
     if (part < 2) {
         float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-        partials_cols(taddr + part * 64, hs, i, valid, part * 64, 64, s_gg, s_gg + 128, s_qk, s_kk, s_hh);
+        partials_cols<false>(taddr + part * 64, hs, i, valid, part * 64, 64, s_gg, nullptr, s_qk, s_kk, s_hh);
         s_red[part * BM + i] = make_float4(s_qk, s_kk, s_hh, 0.f);
     } else {
 #pragma unroll 1
@@ -600,7 +605,7 @@ __device__ __forceinline__ TilePre tile_pre_load(const EpiParams& p, int mt, int
 
 // k tile of BN channels: each of the NPART parts reduces BN/NPART columns,
 // the parts of one 128-channel group are then added in order.
-template <int BN>
+template <int BN, bool SCALED>
 __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, const EpiParams& p, int m0, int nt,
                                            int q, int part, int lane, int et, float* s_gg, float4* s_red,
                                            TilePre& pre, bool has_next, int mt_next, int nt_next) {
@@ -613,11 +618,11 @@ __device__ __forceinline__ void epilogue_k(uint32_t taddr, const uint8_t* hs, co
     epi_sync();
     if (et < BN) {
         s_gg[et] = pre.g;
-        s_gg[BN + et] = pre.ks;
+        if (SCALED) s_gg[BN + et] = pre.ks;
     }
     epi_sync();
     if (has_next) pre = tile_pre_load<MODE_K, BN>(p, mt_next, nt_next, q, lane, et);
-    group_partials(taddr + part * PW, hs, p, row, i, valid, part, part * PW, PW, PPG, (n0 + part * PW) / 128, s_gg,
+    group_partials<SCALED>(taddr + part * PW, hs, p, row, i, valid, part, part * PW, PW, PPG, (n0 + part * PW) / 128, s_gg,
                    s_gg + BN, s_red);
 }
 
@@ -639,7 +644,7 @@ __device__ __forceinline__ float tanh_f32(float x) {
 
 __device__ __forceinline__ float mask_f(float x, uint32_t m) { return __uint_as_float(__float_as_uint(x) & m); }
 
-template <int NCH, bool SLOW, bool RES>
+template <int NCH, bool SLOW, bool RES, bool SCALED>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
                                              const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3, int br) {
@@ -667,10 +672,13 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
         float o[16];
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
-            // warp-uniform address: one broadcast load per channel pair
-            const float2 vs = p.vscale ? __ldg(reinterpret_cast<const float2*>(p.vscale + n0 + cl + c))
-                                       : make_float2(1.f, 1.f);
-            const float v0 = a * vs.x * __uint_as_float(cur[c]), v1 = a * vs.y * __uint_as_float(cur[c + 1]);
+            float v0 = a * __uint_as_float(cur[c]), v1 = a * __uint_as_float(cur[c + 1]);
+            if constexpr (SCALED) {
+                // warp-uniform address: one broadcast load per channel pair
+                const float2 vs = __ldg(reinterpret_cast<const float2*>(p.vscale + n0 + cl + c));
+                v0 *= vs.x;
+                v1 *= vs.y;
+            }
             float s1a = __shfl_up_sync(0xffffffffu, v0, 1), s1b = __shfl_up_sync(0xffffffffu, v1, 1);
             float s2a = __shfl_up_sync(0xffffffffu, v0, 2), s2b = __shfl_up_sync(0xffffffffu, v1, 2);
             float s3a = __shfl_up_sync(0xffffffffu, v0, 3), s3b = __shfl_up_sync(0xffffffffu, v1, 3);
@@ -752,7 +760,7 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
 // while phase 1 runs; with M branches, 2M phases: both halves for branch 0,
 // then for branch 1, ... (the accumulator holds v for all of them).  In each
 // phase part `part` takes BN/8 channels.
-template <int BN>
+template <int BN, bool SCALED>
 __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt, int nt,
                                                int q, int part, int lane, int et, float* s_taps, int phase,
                                                float a, const TilePre& pre, int br) {
@@ -798,14 +806,14 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     const float4* cw = s_tw + phase * VPP * 2 - cbeg;
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
-        if (slow) vconv_chunks<NCHK, true, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+        if (slow) vconv_chunks<NCHK, true, true, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
                                                             br);
-        else vconv_chunks<NCHK, false, true>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+        else vconv_chunks<NCHK, false, true, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
                                                             br);
     } else {
-        if (slow) vconv_chunks<NCHK, true, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+        if (slow) vconv_chunks<NCHK, true, false, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
                                                             br);
-        else vconv_chunks<NCHK, false, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
+        else vconv_chunks<NCHK, false, false, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
                                                             br);
     }
     // the warp's Y block (its 32 rows x PW channels, in place of h) to global
@@ -1179,7 +1187,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     ok = wait_bounded(&sb->hfull_v[phase], (uint32_t)k & 1u, sb, p.status);
                     if (!__all_sync(0xffffffffu, ok)) break;
                     if (br > 0 && phase == 0) a_br = r_ok ? __ldg(p.alpha + (int64_t)br * p.n_tok + r_lane) : 0.f;
-                    epilogue_vconv<BN>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, phase, a_br, pre, br);
+                    epilogue_vconv<BN, F8>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, phase, a_br, pre, br);
                     if (ph == 0 && has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
                     const bool last = ph == n_ph - 1;
                     if (last) tc_fence_before();
@@ -1204,7 +1212,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const bool rows_live = MODE == MODE_VCONV ? (int64_t)mt * TILE_OUT < p.n_tok : (int64_t)mt * BM < p.n_tok;
             if (MODE == MODE_KV) epilogue_kv(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red);
             if (MODE == MODE_K && rows_live) {
-                epilogue_k<BN>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red, pre, has_next,
+                epilogue_k<BN, F8>(taddr, s_h, p, mt * BM, nt, q, part, lane, et, s_gg, s_red, pre, has_next,
                                unit_mt(un), unit_nt(un));
                 band_alpha(p, mt, et, sb, reinterpret_cast<float4*>(s_h), GE::H_BYTES);
             } else if (MODE == MODE_K && has_next) {

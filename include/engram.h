@@ -214,7 +214,11 @@ ENGRAM_API engram_status engram_conv(engram_ctx* ctx, const float* v, const floa
                           const float* conv_w, int32_t B, int32_t L, float* conv_state, void* y,
                           float* alpha_out, int32_t add_residual, cudaStream_t stream);
 
-/* Projections, gate and conv from e: on bf16 tensor-core shapes (d a
+/* Projections, gate and conv from e ("DeepSeek AI II" digest, section
+ * "DeepSeek Engram": k = W_K e and v = W_V e, RMSNorm on the query h and the
+ * key, a scalar gate alpha in (0,1), v~ = alpha v, a short-kernel per-channel
+ * causal convolution, the residual H <- H + Y; Synced repost, section
+ * "context-aware gating").  On bf16 tensor-core shapes (d a
  * multiple of 128, J*D a multiple of 64) with conv width 4, two tcgen05 GEMM
  * passes, the first producing the gate partials from k, the second v with
  * the gate, the conv and the residual applied in its epilogue (v is never
@@ -226,7 +230,11 @@ ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, co
                                int32_t add_residual, void* workspace, size_t workspace_bytes,
                                cudaStream_t stream);
 
-/* The whole forward: what engram_hash (with remap), engram_gather and
+/* The whole forward ("DeepSeek AI II" digest, section "DeepSeek Engram": the
+ * module takes the token ids and the hidden states of a layer and returns Y,
+ * through retrieval (tokenizer compression, suffix n-grams, multi-head
+ * hashing into prime-sized tables, concatenation) and fusion (the gate and
+ * the causal convolution)): what engram_hash (with remap), engram_gather and
  * engram_gate_conv compute, with the first two fused into one retrieval
  * kernel; intermediates in `workspace` (engram_workspace_bytes(ctx, B,
  * T-t_begin) bytes, 256-byte aligned).  tok is [B] rows of `tok_stride` raw
@@ -263,11 +271,12 @@ ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int
  *   gq, gk     [M][d] fp32 or null (ones);           conv_w [d][w], shared;
  *   conv_state [M][B][w-1][d] fp32 or null;          y [M][B*L][d];
  *   alpha_out  [M][B*L] fp32 or null;
- *   k_scale    [M][d] fp32 or null, v_scale [d] fp32 or null: per output
- *              channel factors applied to the GEMM accumulators, k^(m)_c =
- *              k_scale[m][c] * (W_K^(m) e)_c and v_c = v_scale[c] * (W_V e)_c:
- *              the dequantisation of FP8 operands (the tables' scale times
- *              the weight row's scale), or null for 1 (16-byte aligned).
+ *   k_scale    [M][d] fp32, v_scale [d] fp32 (16-byte aligned): with
+ *              ENGRAM_FP8, the per output channel dequantisation of the GEMM
+ *              accumulators, k^(m)_c = k_scale[m][c] * (W_K^(m) e)_c and
+ *              v_c = v_scale[c] * (W_V e)_c (the tables' scale times the weight
+ *              row's scale); required there, and null for the other dtypes
+ *              (ENGRAM_E_INVAL otherwise).
  * M in 1..ENGRAM_MAX_BRANCHES.  With ENGRAM_FP8 tables, e, W_K and W_V are
  * E4M3 bytes and the fused GEMM over [W_V; W_K^(1..M)] runs as FP8 MMAs, as
  * the pages describe.  Runs on the fused tensor-core path only
