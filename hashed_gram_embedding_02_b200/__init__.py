@@ -23,7 +23,7 @@ from .binding import (  # noqa: F401  (re-exported C ABI names)
     engram_host_cache_stats, engram_shard_range, engram_forward_sharded, engram_ipc_export, engram_ipc_open,
     engram_ipc_close, ENGRAM_IPC_HANDLE_BYTES, ENGRAM_MAX_SHARDS, engram_multibranch_workspace_bytes,
     engram_forward_multibranch, ENGRAM_MAX_BRANCHES, engram_table_grad_workspace_bytes, engram_table_grad,
-    engram_table_sgd,
+    engram_table_sgd, engram_host_tier_map,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 
@@ -166,6 +166,10 @@ class HostTier:
 
     def stats(self):
         return engram_host_tier_stats(self.tier)
+
+    def map_tables(self):
+        """Fetch rows with a GPU kernel reading the mapped host tables."""
+        engram_host_tier_map(self.tier)
 
     def enable_cache(self, capacity_rows: int, min_count: int = 2):
         engram_host_cache_enable(self.tier, capacity_rows, min_count)

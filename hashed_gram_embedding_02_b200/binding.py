@@ -42,7 +42,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_er
            "engram_host_cache_enable", "engram_host_cache_reset", "engram_host_cache_stats",
            "engram_shard_range", "engram_forward_sharded", "engram_ipc_export", "engram_ipc_open", "engram_ipc_close",
            "engram_multibranch_workspace_bytes", "engram_forward_multibranch", "engram_table_grad_workspace_bytes",
-           "engram_table_grad", "engram_table_sgd")
+           "engram_table_grad", "engram_table_sgd", "engram_host_tier_map")
 ENGRAM_MAX_BRANCHES = 4
 ENGRAM_IPC_HANDLE_BYTES = 64
 ENGRAM_MAX_SHARDS = 16
@@ -107,6 +107,7 @@ _sigs = {
     "engram_debug_stall_next": ([_vp], _st),
     "engram_host_tier_debug": ([_vp, ctypes.c_uint32, ctypes.c_double], _st),
     "engram_host_cache_enable": ([_vp, _i64, _i32], _st),
+    "engram_host_tier_map": ([_vp], _st),
     "engram_host_cache_reset": ([_vp, _vp], _st),
     "engram_host_cache_stats": ([_vp, ctypes.c_void_p], _st),
     "engram_shard_range": ([_vp, _i32, _i32, ctypes.POINTER(_i64), ctypes.POINTER(_i64)], _st),
@@ -391,6 +392,11 @@ def engram_host_tier_stats(tier) -> dict:
     out = engram_host_tier_stats_t()
     _check(_lib.engram_host_tier_stats(tier, ctypes.addressof(out)), "engram_host_tier_stats")
     return {f: getattr(out, f) for f, _ in out._fields_}
+
+
+def engram_host_tier_map(tier) -> None:
+    """Map the host tables: the tier fetches rows with a GPU kernel over PCIe."""
+    _check(_lib.engram_host_tier_map(tier), "engram_host_tier_map")
 
 
 def engram_host_cache_enable(tier, capacity_rows: int, min_count: int = 2) -> None:

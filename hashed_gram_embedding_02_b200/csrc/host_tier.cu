@@ -242,6 +242,41 @@ __global__ void dedupe_slot_kernel(const uint32_t* __restrict__ idx, int64_t n_l
     }
 }
 
+// Mapped fetch (engram_host_tier_map): the distinct rows come straight from
+// the host tables, which are mapped into the device's address space, into
+// the staged rows [C + id]: every load crosses PCIe as a read request of the
+// GPU, issued by many warps at once, and no host thread packs anything.  The
+// row list and its length are read on the device.  Each thread issues
+// kBatchMapped independent 16-byte loads before its stores.
+constexpr int kBatchMapped = 4;
+__global__ void __launch_bounds__(256) mapped_fetch_kernel(const uint4* __restrict__ host_rows,
+                                                          const unsigned long long* __restrict__ ukeys,
+                                                          const uint32_t* __restrict__ count, int chunks_per_row,
+                                                          uint64_t total_rows, uint4* __restrict__ staged,
+                                                          uint32_t* status) {
+    const int64_t n = (int64_t)__ldg(count) * chunks_per_row;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t f0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; f0 < n; f0 += stride * kBatchMapped) {
+        uint4 v[kBatchMapped];
+#pragma unroll
+        for (int u = 0; u < kBatchMapped; ++u) {
+            const int64_t f = f0 + u * stride;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (f < n) {
+                const int64_t r = f / chunks_per_row, c = f - r * chunks_per_row;
+                const uint64_t row = __ldg(ukeys + r);
+                if (row < total_rows) v[u] = host_rows[row * chunks_per_row + c];
+                else flag(status, ENGRAM_ERR_INDEX);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatchMapped; ++u) {
+            const int64_t f = f0 + u * stride;
+            if (f < n) staged[f] = v[u];
+        }
+    }
+}
+
 // Copy rows [r0, r1) of the distinct-row list from the host tables into the
 // staging buffer, prefetching a few rows ahead.  A row number outside the
 // tables (impossible for lists the dedupe kernel wrote) gives a zero row.
@@ -307,6 +342,9 @@ struct engram_host_tier {
                             // [3] lookups served from the cache
     uint32_t* d_slot;
     uint8_t* d_rows;        // cache slots [0, C) then the staged rows [C, C + max_lookups)
+    // mapped mode (engram_host_tier_map): the host tables as device-visible memory
+    const uint4* d_host_tables;
+    bool mapped_registered;   // this tier registered the host range (and unregisters it)
     // hot-row cache (capacity 0: none)
     uint32_t cache_cap;
     uint32_t cache_min_count;
@@ -411,6 +449,7 @@ void tier_free(engram_host_tier* t) {
     cudaFreeHost(t->h_ukeys);
     cudaFreeHost(t->h_count);
     cudaFreeHost(t->h_stage);
+    if (t->mapped_registered) cudaHostUnregister(const_cast<uint8_t*>(t->host_tables));
     delete t->chunk_done;
     delete t;
 }
@@ -547,7 +586,8 @@ engram_status engram_host_dedupe(engram_host_tier* t, const uint32_t* idx, int64
     // distinct-row count and list to pinned host memory (the list at its
     // largest possible length: one copy, no round trip for the count)
     e = cudaMemcpyAsync(t->h_count, t->d_count, 4 * sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess && n > 0)
+    // the mapped fetch reads the list on the device: only the copy path needs it on the host
+    if (e == cudaSuccess && n > 0 && !t->d_host_tables)
         e = cudaMemcpyAsync(t->h_ukeys, t->d_ukeys, (size_t)n * sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaEventRecord(t->ev_keys, s);
     if (e != cudaSuccess) return cuda_fail("host tier: copying the row list out", e);
@@ -561,6 +601,35 @@ engram_status engram_host_fetch(engram_host_tier* t, cudaStream_t side, int64_t*
     if (!t->have_keys) return inval("engram_host_fetch needs a preceding engram_host_dedupe");
     engram_status st = check_device(t->c);
     if (st != ENGRAM_OK) return st;
+    if (t->d_host_tables) {
+        // mapped: everything stays on the GPU's queues; the side stream waits
+        // for the dedupe and for the previous staged gather, then one kernel
+        // pulls the distinct rows over PCIe.  The count is not known here.
+        t->fetched = false;
+        cudaError_t e = cudaStreamWaitEvent(side, t->ev_keys, 0);
+        if (e == cudaSuccess && t->consumed_recorded) e = cudaStreamWaitEvent(side, t->ev_consumed, 0);
+        if (e == cudaSuccess) e = cudaEventRecord(t->ev_copy0, side);
+        if (e != cudaSuccess) return cuda_fail("host tier: ordering the mapped fetch", e);
+        const int cpr = (int)(t->row_bytes / 16);
+        const int blocks = t->c->num_sms * 8;
+        mapped_fetch_kernel<<<blocks, 256, 0, side>>>(t->d_host_tables, t->d_ukeys, t->d_count, cpr,
+                                                      (uint64_t)t->total_rows,
+                                                      reinterpret_cast<uint4*>(t->d_rows) + (size_t)t->cache_cap * cpr,
+                                                      t->c->d_status);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaEventRecord(t->ev_copy1, side);
+        if (e == cudaSuccess) e = cudaEventRecord(t->ev_ready, side);
+        if (e != cudaSuccess) return cuda_fail("host tier: mapped fetch launch", e);
+        t->fetched = true;
+        t->copies_recorded = true;
+        t->have_keys = false;
+        t->last_unique = -1;
+        t->last_copies = 0;
+        t->last_wait_ms = 0.0;
+        t->last_pack_ms = 0.0;
+        if (n_unique) *n_unique = -1;
+        return ENGRAM_OK;
+    }
     // until this fetch succeeds, gather_staged must not read the staged rows
     t->fetched = false;
     const auto tw = std::chrono::steady_clock::now();
@@ -707,6 +776,37 @@ engram_status engram_gather_staged(engram_host_tier* t, int64_t n_tok, void* e_c
     return ENGRAM_OK;
 }
 
+engram_status engram_host_tier_map(engram_host_tier* t) {
+    if (!t) return inval("null host tier");
+    if (t->d_host_tables) return ENGRAM_OK;
+    if (t->have_keys || t->fetched) return inval("map the host tables before the first batch");
+    engram_status st = check_device(t->c);
+    if (st != ENGRAM_OK) return st;
+    const size_t bytes = (size_t)t->total_rows * t->row_bytes;
+    void* host = const_cast<uint8_t*>(t->host_tables);
+    cudaError_t e = cudaHostRegister(host, bytes, cudaHostRegisterMapped | cudaHostRegisterReadOnly);
+    if (e == cudaErrorHostMemoryAlreadyRegistered) {
+        cudaGetLastError();
+        e = cudaSuccess;       // the caller's registration (it must be mapped)
+    } else if (e == cudaSuccess) {
+        t->mapped_registered = true;
+    }
+    void* dev = nullptr;
+    if (e == cudaSuccess) e = cudaHostGetDevicePointer(&dev, host, 0);
+    if (e != cudaSuccess) {
+        if (t->mapped_registered) cudaHostUnregister(host);
+        t->mapped_registered = false;
+        return cuda_fail("host tier: mapping the host tables", e);
+    }
+    if ((reinterpret_cast<uintptr_t>(dev) & 15u) != 0) {
+        if (t->mapped_registered) cudaHostUnregister(host);
+        t->mapped_registered = false;
+        return inval("the mapped host tables are not 16-byte aligned");
+    }
+    t->d_host_tables = static_cast<const uint4*>(dev);
+    return ENGRAM_OK;
+}
+
 engram_status engram_host_cache_enable(engram_host_tier* t, int64_t capacity_rows, int32_t min_count) {
     if (!t) return inval("null host tier");
     if (capacity_rows < 1 || capacity_rows > ((int64_t)1 << 30)) return inval("capacity_rows must be in [1, 2^30]");
@@ -783,12 +883,13 @@ engram_status engram_host_tier_debug(engram_host_tier* t, uint32_t inject, doubl
 
 engram_status engram_host_tier_stats(const engram_host_tier* t, engram_host_tier_stats_t* out) {
     if (!t || !out) return inval("null host tier or output");
-    out->n_unique = t->last_unique;
+    // mapped fetches learn the count from the dedupe's copy of it, once the batch is done
+    out->n_unique = t->last_unique >= 0 ? t->last_unique : (int64_t)(t->h_count ? t->h_count[0] : 0);
     out->n_copies = t->last_copies;
     out->wait_ms = t->last_wait_ms;
     out->pack_ms = t->last_pack_ms;
     out->copy_ms = -1.0;
-    if (t->fetched && t->last_copies > 0 && cudaEventQuery(t->ev_copy1) == cudaSuccess) {
+    if (t->fetched && (t->last_copies > 0 || t->d_host_tables) && cudaEventQuery(t->ev_copy1) == cudaSuccess) {
         float ms = 0.f;
         if (cudaEventElapsedTime(&ms, t->ev_copy0, t->ev_copy1) == cudaSuccess) out->copy_ms = ms;
     }

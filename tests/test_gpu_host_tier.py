@@ -311,3 +311,42 @@ def test_hot_row_cache_over_batches(eb, capacity):
     torch.cuda.synchronize()
     assert torch.equal(e_t, e_d)
     tier.close()
+
+
+# ---------------------------------------------------------------- mapped fetch (GPU reads the host tables)
+
+@pytest.mark.parametrize("cache", [0, 20000])
+def test_mapped_fetch_equals_hbm_gather(eb, cache):
+    """With the host tables mapped into the device's address space, a GPU
+    kernel pulls the distinct rows over PCIe: three consecutive batches (with
+    and without the hot-row cache) must gather exactly what the HBM gather
+    gives, and the counts must match the copy path's."""
+    wl = SMALL
+    batches = _batches(wl, 3)
+    ctx = eb.Engram(config_for(batches[0], eb))
+    host = batches[0].host_tables("cuda:0")
+    tables_d = batches[0].device_tables("cuda:0")
+    tier = eb.HostTier(ctx, host, max_lookups=wl.n_tok * wl.J, n_threads=2)
+    tier.map_tables()
+    if cache:
+        tier.enable_cache(cache)
+    side = torch.cuda.Stream()
+    for k, inp in enumerate(batches):
+        idx = torch.empty(wl.n_tok, wl.J, dtype=torch.int32, device="cuda")
+        eb.engram_hash(ctx.ctx, torch.from_numpy(inp.tok).cuda(), torch.from_numpy(inp.P).cuda(), wl.B, wl.T, wl.T,
+                       0, idx)
+        e_t = torch.full((wl.n_tok, wl.d_mem), float("nan"), dtype=torch.bfloat16, device="cuda")
+        tier.dedupe(idx, wl.n_tok)
+        assert tier.fetch(side) == -1                  # not known on the host at this point
+        tier.gather(wl.n_tok, e_t)
+        e_d = torch.empty_like(e_t)
+        eb.engram_gather(ctx.ctx, idx, wl.n_tok, tables_d, e_d)
+        torch.cuda.synchronize()
+        assert torch.equal(e_t, e_d), k
+        keys, _ = _distinct_split(idx, batches[0], None)
+        cs = tier.cache_stats()
+        assert cs["fetched_rows"] + cs["cached_rows"] == len(keys)
+        st = tier.stats()
+        assert st["n_unique"] == cs["fetched_rows"] and st["copy_ms"] > 0
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    tier.close()
