@@ -560,6 +560,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="oracle sample per reference step (0: sized so the run takes about 90 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph replay")
     ap.add_argument("--branches", type=int, default=1,
                     help="multi-branch module: M residual branches (own W_K, h, gate and Y each; shared tables, "
                          "W_V and conv)")
@@ -671,6 +672,25 @@ def main():
     if st != eb.ENGRAM_OK:
         raise RuntimeError(f"device status {st} flags {flags:#x} after warm-up")
 
+    # ---- one forward captured as a CUDA graph: the timed loop replays it, so
+    # the host's launch work (argument checks, tensor maps, four launches)
+    # stays out of the device time of short steps such as decode
+    graph, launch = None, "eager"
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+            launch = "CUDA graph of one forward (captured after the warm-up), replayed each step"
+        except Exception as exc:                      # capture unsupported: time eager launches
+            graph, launch = None, f"eager (graph capture failed: {type(exc).__name__})"
+            torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+
     # ---- timed: K whole steps, L2 flushed before each (outside the events)
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -680,7 +700,7 @@ def main():
         for i in range(K):
             flush.zero_()
             ev[i][0].record(stream)
-            step()
+            run()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -718,6 +738,9 @@ def main():
                              "bytes"),
         "gate_k_tc": ("tensor", M * pass_flops, "flop"),
         "vconv_tc": ("tensor", pass_flops, "flop"),
+        # decode passes (one position per sequence): the same contraction
+        "gate_k_decode": ("tensor", pass_flops, "flop"),
+        "vconv_decode": ("tensor", pass_flops, "flop"),
         "state_merge": ("hbm", wl.B * (wl.w - 1) * wl.d * 8.0, "bytes"),
     }
     kern = {}
@@ -781,7 +804,8 @@ def main():
                    "tokens_per_step": n * world,
                    "parallelism": (f"tables sharded over {world} GPUs, rows read over NVLink by the retrieval"
                                    if sharded is not None else f"replicas x{world} (no collective)"),
-                   "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write outside the events)"},
+                   "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write outside the events)",
+                   "launch": launch},
         "roofline": roofline,
         "gather": {"kernel": "retrieve (remap + n-grams + hash + gather)", "achieved_gbs": gather_gbs,
                    "frac_of_8000": gather_gbs / SPEC_HBM_GBS, "frac_of_measured": gather_gbs / hbm,

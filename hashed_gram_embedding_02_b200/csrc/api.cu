@@ -81,8 +81,19 @@ bool fused_path(const engram_ctx* c, int64_t n) { return tc_path(c, n) && c->cfg
 constexpr int32_t kDecodeRows = 8;
 bool decode_shaped(const engram_ctx* c, int64_t n, int64_t L) { return fused_path(c, n) && L <= kDecodeRows; }
 
-// per-128-row-band counters of the key pass
-size_t band_bytes(int64_t n) { return (size_t)((n + 127) / 128) * sizeof(int); }
+// One new position per sequence for at most 256 sequences (bf16, one branch):
+// the decode passes, which read and update the caller's conv state in place.
+bool decode_kernels(const engram_ctx* c, int64_t n, int64_t L, int M) {
+    return fused_path(c, n) && decode_tc_supported(n, (int32_t)L, c->d_mem, c->cfg.hidden, M,
+                                                   c->cfg.dtype == ENGRAM_FP8);
+}
+
+// per-128-row-band counters of the key pass (at least 8: the decode key pass
+// counts four row blocks)
+size_t band_bytes(int64_t n) {
+    const int64_t k = (n + 127) / 128;
+    return (size_t)(k < 8 ? 8 : k) * sizeof(int);
+}
 
 Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with_idx_e, int M) {
     const int64_t n = B * L;
@@ -94,8 +105,10 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
         w.e = p;
         p += align256((size_t)n * c->d_mem * c->es);
     }
+    const bool dec = decode_kernels(c, n, L, M);
     w.part = reinterpret_cast<float*>(p);
-    p += align256((size_t)n * M * c->G * 4 * sizeof(float));
+    const int64_t groups = dec ? decode_tc_max_tiles(c->cfg.hidden) : c->G;
+    p += align256((size_t)n * M * groups * 4 * sizeof(float));
     w.alpha = reinterpret_cast<float*>(p);
     p += align256((size_t)M * n * sizeof(float));
     w.band = reinterpret_cast<int*>(p);
@@ -105,7 +118,7 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
         align256((size_t)M * B * (c->cfg.conv_width - 1) * c->cfg.hidden * sizeof(float));
     w.state_next = reinterpret_cast<float*>(p);
     p += hist_bytes;
-    if (decode_shaped(c, n, L)) {
+    if (decode_shaped(c, n, L) && !dec) {
         w.state_t = reinterpret_cast<float*>(p);
         p += hist_bytes;
     }
@@ -193,6 +206,25 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
     const bool f8 = c->cfg.dtype == ENGRAM_FP8;
     const int64_t n = (int64_t)B * L;
     const size_t hist_elems = (size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden;   // one branch's history
+    if (decode_kernels(c, n, L, M)) {
+        cudaError_t e = cudaSuccess;
+        if (!after_retrieve) {
+            e = cudaMemsetAsync(w.band, 0, w.counter_bytes, s);
+            if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
+        }
+        prof_begin(c, s, "gate_k_decode");
+        e = launch_decode_k(e_cat, (int32_t)n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band,
+                            w.alpha, alpha_out, c->d_status, c->num_sms, c->debug_stall, after_retrieve && !c->prof, s);
+        c->debug_stall = 0;
+        prof_end(c, s);
+        if (e != cudaSuccess) return cuda_fail("tcgen05 decode key/gate launch", e);
+        prof_begin(c, s, "vconv_decode");
+        e = launch_decode_v(e_cat, (int32_t)n, c->d_mem, h, Wv, conv_w, c->cfg.hidden, w.alpha, state, y,
+                            add_residual, c->d_status, c->num_sms, !c->prof, s);
+        prof_end(c, s);
+        if (e != cudaSuccess) return cuda_fail("tcgen05 decode value/conv launch", e);
+        return ENGRAM_OK;
+    }
     if (fused_path(c, n)) {
         const bool tr = state && decode_shaped(c, n, L);
         cudaError_t e = cudaSuccess;
@@ -258,7 +290,7 @@ engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t
                            const ShardParams* shards, int M, const float* kscale, const float* vscale) {
     const int32_t L = T - t_begin;
     const bool fused = fused_path(c, (int64_t)B * L);
-    if (fused && conv_state && decode_shaped(c, (int64_t)B * L, L)) {
+    if (fused && conv_state && decode_shaped(c, (int64_t)B * L, L) && !decode_kernels(c, (int64_t)B * L, L, M)) {
         engram_status st = launch_history_transpose(c, conv_state, w, B, M, s);
         if (st != ENGRAM_OK) return st;
     }

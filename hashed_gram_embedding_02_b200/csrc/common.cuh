@@ -58,6 +58,19 @@ __device__ __forceinline__ uint32_t mod_u64(uint64_t x, uint32_t m, uint64_t rec
     return (uint32_t)r;
 }
 
+// Decode passes (one new position per sequence, at most 256 sequences, bf16,
+// one branch): K split over clusters of four CTAs, partials added through
+// distributed shared memory, the conv state updated in place.
+bool decode_tc_supported(int64_t n, int32_t L, int32_t d_mem, int32_t d, int32_t M, bool f8);
+int32_t decode_tc_max_tiles(int32_t d);   // channel tiles per row at most (the gate partials' width)
+cudaError_t launch_decode_k(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wk, const void* Wv,
+                            const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
+                            float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
+                            cudaStream_t s);
+cudaError_t launch_decode_v(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wv,
+                            const float* conv_w, int32_t d, const float* alpha, float* state, void* y,
+                            int32_t add_residual, uint32_t* status, int num_sms, bool pdl, cudaStream_t s);
+
 // ---------------------------------------------------------------- launches
 // Each returns cudaGetLastError() of its launch.
 cudaError_t launch_remap(const int32_t* tok, int64_t n, const int32_t* P, int32_t V, int32_t* canon,

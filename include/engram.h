@@ -242,7 +242,13 @@ ENGRAM_API engram_status engram_gate_conv(engram_ctx* ctx, const void* e_cat, co
  * t_begin = T-1 with conv_state.  On the tensor-core path the two GEMM passes
  * are launched as programmatic dependents of the kernel before each (they
  * overlap its last CTAs and wait for its results on the device); seen from
- * the stream, the call is ordered like any other work on `stream`. */
+ * the stream, the call is ordered like any other work on `stream`.  A decode
+ * step (T - t_begin = 1) for at most 256 sequences of a bf16 context runs
+ * the decode passes: K split over clusters of four CTAs, and conv_state
+ * rewritten in place by the value pass (same result as above).  The call
+ * only enqueues work on `stream`, so it can be captured into a CUDA graph;
+ * a replay recomputes from the pointers given at capture, whose contents
+ * may change between replays. */
 ENGRAM_API engram_status engram_forward(engram_ctx* ctx, const int32_t* tok, int32_t B, int32_t T,
                              int64_t tok_stride, int32_t t_begin, const int32_t* P,
                              const void* tables, const void* h, const void* Wk, const void* Wv,

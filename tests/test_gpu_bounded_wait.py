@@ -68,3 +68,37 @@ def test_stalled_wait_times_out_and_context_recovers(eb, name):
     err = np.abs(to_np(y2[sel]) - ref.y)
     assert err.max() <= 2e-2
     assert not (err > bf16_bound(ref.y, ref.vt_win, inp.conv_w)).any()
+
+
+def test_decode_stalled_wait_times_out_and_context_recovers(eb):
+    """The same on the decode key pass (clusters of four CTAs splitting K): the
+    stalled CTA votes to abort, its cluster skips the partial exchange, and
+    every CTA still meets the cluster barriers and leaves."""
+    wl = W["c2"].replace(name="decode", B=64, T=4, t_begin=3, M=10007, seed=53)
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    state = inp.device_state("cuda:0").contiguous()
+    y = di.empty_y()
+    eb.engram_debug_stall_next(ctx.ctx)
+    t0 = time.time()
+    ctx.forward(di.tok, di.P, di.tables, di.h, di.Wk, di.Wv, di.conv_w, y, t_begin=wl.t_begin, gq=di.gq, gk=di.gk,
+                conv_state=state.clone(), add_residual=True)
+    st, flags = ctx.status()
+    elapsed = time.time() - t0
+    assert st == eb.ENGRAM_E_TIMEOUT and flags & eb.ENGRAM_ERR_TIMEOUT, (st, flags)
+    assert elapsed < 30.0
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+
+    y2 = di.empty_y()
+    alpha = torch.empty(wl.n_tok, dtype=torch.float32, device="cuda")
+    ctx.forward(di.tok, di.P, di.tables, di.h, di.Wk, di.Wv, di.conv_w, y2, t_begin=wl.t_begin, gq=di.gq, gk=di.gk,
+                conv_state=state, alpha_out=alpha, add_residual=True)
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    hist = inp.state_rows(np.arange(wl.B))
+    ref = oracle.forward_rows(inp, np.arange(wl.n_tok), add_residual=True, hist=hist)
+    np.testing.assert_allclose(to_np(alpha), ref.alpha, rtol=0, atol=2e-6)
+    err = np.abs(to_np(y2) - ref.y)
+    assert err.max() <= 2e-2
+    assert not (err > bf16_bound(ref.y, ref.vt_win, inp.conv_w)).any()

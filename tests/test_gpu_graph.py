@@ -1,0 +1,72 @@
+"""engram_forward captured into a CUDA graph: a replay gives the same bits as
+an eager call, for a prefill and for a decode step (whose conv state the
+replay updates in place, as the eager call does)."""
+
+import numpy as np
+import pytest
+
+import synth
+from gpu_helpers import DeviceInputs, config_for
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+CASES = {
+    "prefill": W["c2"].replace(name="prefill", B=2, T=333, M=10007, d=512, seed=71),
+    "decode": W["c4"].replace(name="decode", M=10007, T=16, t_begin=15, seed=72),
+}
+
+
+@pytest.fixture(scope="module")
+def eb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import hashed_gram_embedding_02_b200 as eb
+    return eb
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_graph_replay_matches_eager(eb, name):
+    wl = CASES[name]
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb), B=wl.B, L=wl.T - wl.t_begin)
+    s0 = inp.device_state("cuda:0").contiguous() if wl.t_begin > 0 else None
+    y = di.empty_y()
+    alpha = torch.empty(wl.n_tok, dtype=torch.float32, device="cuda")
+    state = s0.clone() if s0 is not None else None
+
+    def step():
+        ctx.forward(di.tok, di.P, di.tables, di.h, di.Wk, di.Wv, di.conv_w, y, t_begin=wl.t_begin, gq=di.gq,
+                    gk=di.gk, conv_state=state, alpha_out=alpha, add_residual=True)
+
+    step()
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    y_eager, a_eager = y.clone(), alpha.clone()
+    st_eager = state.clone() if state is not None else None
+
+    g = torch.cuda.CUDAGraph()
+    if state is not None:
+        state.copy_(s0)
+    with torch.cuda.graph(g):
+        step()
+    # capture records the launches without running them
+    if state is not None:
+        state.copy_(s0)
+    y.zero_()
+    alpha.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    assert torch.equal(y, y_eager) and torch.equal(alpha, a_eager)
+    if state is not None:
+        assert torch.equal(state, st_eager)
+    # a second replay from the same starting state: the same bits again
+    if state is not None:
+        state.copy_(s0)
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager)
