@@ -175,8 +175,10 @@ def oracle_sample_time(wl, n_tokens: int):
 # that made it.
 CSRC = os.path.join(ROOT, "hashed_gram_embedding_02_b200", "csrc")
 KERNEL_SOURCES = {
-    "gate_k_tc": ("project_tc.cu", "common.cuh", "ptx.cuh"),
-    "vconv_tc": ("project_tc.cu", "common.cuh", "ptx.cuh"),
+    "gate_k_tc": ("project_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
+    "vconv_tc": ("project_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
+    "gate_k_decode": ("decode_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
+    "vconv_decode": ("decode_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
     "retrieve": ("retrieve.cu", "common.cuh"),
 }
 CAPTURED_TRAFFIC = {
@@ -190,9 +192,15 @@ CAPTURED_TRAFFIC = {
     ("c3-B2-M499979", "gate_k_tc"): ("59d2794a31cc0db6", 86043136 + 130048),
     ("c3-B2-M499979", "retrieve"): ("8c46903b0c8d286e", 29667072 + 480512),
     # c3 at full size, mean of the five timed steps' launches (profiles/launches_c3.md)
-    ("c3", "vconv_tc"): ("3341a08adf82f52a", 314786253 + 123717939),
-    ("c3", "gate_k_tc"): ("3341a08adf82f52a", 312558797 + 7296461),
-    ("c3", "retrieve"): ("7fd2473de48a2d96", 115571456 + 81190400),
+    ("c3", "vconv_tc"): ("9ab3e6fa4d60f677", 314986291 + 123705805),
+    ("c3", "gate_k_tc"): ("9ab3e6fa4d60f677", 312567296 + 7406336),
+    ("c3", "retrieve"): ("466e8ddd712470f7", 115578931 + 81197158),
+    # c4 at full size, the same way (profiles/launches_c4.md); ncu flushes the
+    # caches before each launch, so the value pass's W_V, which the key pass
+    # brings into L2 in a real step, counts as DRAM reads here
+    ("c4", "gate_k_decode"): ("6c7cd3723eca9a47", 23403930 + 0),
+    ("c4", "vconv_decode"): ("6c7cd3723eca9a47", 20784845 + 0),
+    ("c4", "retrieve"): ("466e8ddd712470f7", 1207296 + 307),
 }
 
 
