@@ -51,17 +51,28 @@ void prof_reset(engram_ctx* c) { c->prof_n = 0; }
 // Every launch is also an NVTX range named for the kernel's role, so a
 // profiler timeline of a step shows which launch is which (NVTX costs a
 // pointer test when no tool is attached).
+// Under stream capture a plain event record only orders work inside the
+// graph; the external form makes it a record node that each replay records,
+// so a captured forward can be timed kernel by kernel.
+static void prof_record(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, s);
+}
+
 void prof_begin(engram_ctx* c, cudaStream_t s, const char* name) {
     nvtxRangePushA(name);
     if (!c->prof || c->prof_n >= kMaxProf) return;
     c->prof_name[c->prof_n] = name;
-    cudaEventRecord(c->ev[2 * c->prof_n], s);
+    prof_record(c->ev[2 * c->prof_n], s);
 }
 
 void prof_end(engram_ctx* c, cudaStream_t s) {
     nvtxRangePop();
     if (!c->prof || c->prof_n >= kMaxProf) return;
-    cudaEventRecord(c->ev[2 * c->prof_n + 1], s);
+    prof_record(c->ev[2 * c->prof_n + 1], s);
     ++c->prof_n;
 }
 
@@ -472,9 +483,12 @@ int32_t engram_profile_read(engram_ctx* c, float* ms, const char** names, int32_
     if (!c || !c->prof) return 0;
     int n = c->prof_n < max ? c->prof_n : max;
     for (int i = 0; i < n; ++i) {
-        cudaEventSynchronize(c->ev[2 * i + 1]);
-        float t = 0.f;
-        cudaEventElapsedTime(&t, c->ev[2 * i], c->ev[2 * i + 1]);
+        float t = -1.f;
+        if (cudaEventSynchronize(c->ev[2 * i + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&t, c->ev[2 * i], c->ev[2 * i + 1]) != cudaSuccess) {
+            t = -1.f;
+            cudaGetLastError();   // a failed query must not surface at the next launch
+        }
         if (ms) ms[i] = t;
         if (names) names[i] = c->prof_name[i];
     }

@@ -146,7 +146,10 @@ ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int32_t B, int32
  * kernel it launches on the caller's stream; engram_profile_read waits for
  * the events of the most recent call and writes up to `max` durations in
  * milliseconds and kernel names (library-owned strings) in launch order,
- * returning how many.  Not thread-safe; disable to free the events. */
+ * returning how many; a duration that could not be measured reads -1.
+ * Under stream capture the events become record nodes of the graph, so
+ * after a replay engram_profile_read returns that replay's durations.  Not
+ * thread-safe; disable to free the events. */
 ENGRAM_API engram_status engram_profile_enable(engram_ctx* ctx, int32_t enable);
 ENGRAM_API int32_t engram_profile_read(engram_ctx* ctx, float* ms, const char** names, int32_t max);
 

@@ -70,3 +70,38 @@ def test_graph_replay_matches_eager(eb, name):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(y, y_eager)
+
+
+def test_profile_events_inside_a_graph(eb):
+    """With kernel timing on, a captured forward records its events as graph
+    nodes: every replay yields positive per-kernel durations, and a failed
+    read leaves no pending error behind for the next launch."""
+    wl = CASES["decode"]
+    inp = synth.Inputs(wl)
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb), B=wl.B, L=1)
+    state = inp.device_state("cuda:0").contiguous()
+    y = di.empty_y()
+
+    def step():
+        ctx.forward(di.tok, di.P, di.tables, di.h, di.Wk, di.Wv, di.conv_w, y, t_begin=wl.t_begin, gq=di.gq,
+                    gk=di.gk, conv_state=state, add_residual=True)
+
+    step()
+    eb.engram_profile_enable(ctx.ctx, True)
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+            torch.cuda.synchronize()
+            prof = eb.engram_profile_read(ctx.ctx)
+            assert [n for n, _ in prof] == ["retrieve", "gate_k_decode", "vconv_decode"], prof
+            assert all(t > 0.0 for _, t in prof), prof
+        del g
+    finally:
+        eb.engram_profile_enable(ctx.ctx, False)
+    step()                                   # an eager call after the graph
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
