@@ -131,12 +131,12 @@ ENGRAM_API const char* engram_last_error(void);
 
 /* Bytes of scratch that engram_forward / engram_gate_conv need for B
  * sequences of L computed rows (n_tok = B*L): indices [n_tok][J] u32,
- * e [n_tok][J*D], gate partials [n_tok][G][4] f32 with G = ceil(d / 128), the
- * gate values [n_tok] f32, ceil(n_tok/128) int32 counters, the next conv
- * history [B][w-1][d] f32, for fused calls with L <= 8 a second history
- * buffer (the history in the sequence-minor layout [w-1][d][B] that the
- * value pass reads coalesced across sequences) and, where
- * the gate and conv are not
+ * e [n_tok][J*D], gate partials [n_tok][G][4] f32 with G = ceil(d / 128)
+ * (d / 64 for the decode passes of one-position bf16 calls), the gate values
+ * [n_tok] f32, max(ceil(n_tok/128), 8) int32 counters, the next conv history
+ * [B][w-1][d] f32, for other fused calls with L <= 8 a second history buffer
+ * (the history in the sequence-minor layout [w-1][d][B] that the value pass
+ * reads coalesced across sequences) and, where the gate and conv are not
  * fused into the projection (see engram_gate_conv), v [n_tok][d] f32; each
  * part 256-byte aligned.  0 for a null context. */
 ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int32_t B, int32_t L);
