@@ -177,8 +177,8 @@ CSRC = os.path.join(ROOT, "hashed_gram_embedding_02_b200", "csrc")
 KERNEL_SOURCES = {
     "gate_k_tc": ("project_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
     "vconv_tc": ("project_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
-    "gate_k_decode": ("decode_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
-    "vconv_decode": ("decode_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
+    "gate_kv_decode": ("decode_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
+    "conv_decode": ("decode_tc.cu", "tc.cuh", "common.cuh", "ptx.cuh"),
     "retrieve": ("retrieve.cu", "common.cuh"),
 }
 CAPTURED_TRAFFIC = {
@@ -195,11 +195,6 @@ CAPTURED_TRAFFIC = {
     ("c3", "vconv_tc"): ("9ab3e6fa4d60f677", 314986291 + 123705805),
     ("c3", "gate_k_tc"): ("9ab3e6fa4d60f677", 312567296 + 7406336),
     ("c3", "retrieve"): ("466e8ddd712470f7", 115578931 + 81197158),
-    # c4 at full size, the same way (profiles/launches_c4.md); ncu flushes the
-    # caches before each launch, so the value pass's W_V, which the key pass
-    # brings into L2 in a real step, counts as DRAM reads here
-    ("c4", "gate_k_decode"): ("6c7cd3723eca9a47", 23403930 + 0),
-    ("c4", "vconv_decode"): ("6c7cd3723eca9a47", 20784845 + 0),
     ("c4", "retrieve"): ("466e8ddd712470f7", 1207296 + 307),
 }
 
@@ -770,9 +765,11 @@ def main():
                              "bytes"),
         "gate_k_tc": ("tensor", M * pass_flops, "flop"),
         "vconv_tc": ("tensor", pass_flops, "flop"),
-        # decode passes (one position per sequence): the same contraction
-        "gate_k_decode": ("tensor", pass_flops, "flop"),
-        "vconv_decode": ("tensor", pass_flops, "flop"),
+        # decode (one position per sequence): both contractions in one kernel,
+        # then the conv over v: v and alpha in, the history read and
+        # rewritten, h in, Y out
+        "gate_kv_decode": ("tensor", 2 * pass_flops, "flop"),
+        "conv_decode": ("hbm", n * wl.d * (4.0 + 24.0 + 2.0 + 2.0) + n * 4.0 + wl.d * 16.0, "bytes"),
         "state_merge": ("hbm", wl.B * (wl.w - 1) * wl.d * 8.0, "bytes"),
     }
     kern = {}

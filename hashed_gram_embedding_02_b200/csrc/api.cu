@@ -133,7 +133,7 @@ Workspace carve(const engram_ctx* c, void* base, int64_t B, int64_t L, bool with
         w.state_t = reinterpret_cast<float*>(p);
         p += hist_bytes;
     }
-    if (!fused_path(c, n)) {
+    if (!fused_path(c, n) || dec) {
         w.v = reinterpret_cast<float*>(p);
         p += align256((size_t)n * c->cfg.hidden * sizeof(float));
     }
@@ -219,21 +219,17 @@ engram_status gate_conv_impl(engram_ctx* c, const void* e_cat, const void* h, co
     const size_t hist_elems = (size_t)B * (c->cfg.conv_width - 1) * c->cfg.hidden;   // one branch's history
     if (decode_kernels(c, n, L, M)) {
         cudaError_t e = cudaSuccess;
-        if (!after_retrieve) {
-            e = cudaMemsetAsync(w.band, 0, w.counter_bytes, s);
-            if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);
-        }
-        prof_begin(c, s, "gate_k_decode");
-        e = launch_decode_k(e_cat, (int32_t)n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, c->cfg.eps, w.part, w.band,
-                            w.alpha, alpha_out, c->d_status, c->num_sms, c->debug_stall, after_retrieve && !c->prof, s);
+        prof_begin(c, s, "gate_kv_decode");
+        e = launch_decode_kv(e_cat, (int32_t)n, c->d_mem, h, Wk, Wv, gq, gk, c->cfg.hidden, w.part, w.v, c->d_status,
+                             c->num_sms, c->debug_stall, after_retrieve && !c->prof, s);
         c->debug_stall = 0;
         prof_end(c, s);
-        if (e != cudaSuccess) return cuda_fail("tcgen05 decode key/gate launch", e);
-        prof_begin(c, s, "vconv_decode");
-        e = launch_decode_v(e_cat, (int32_t)n, c->d_mem, h, Wv, conv_w, c->cfg.hidden, w.alpha, state, y,
-                            add_residual, c->d_status, c->num_sms, !c->prof, s);
+        if (e != cudaSuccess) return cuda_fail("tcgen05 decode projections launch", e);
+        prof_begin(c, s, "conv_decode");
+        e = launch_decode_conv(w.v, w.part, (int32_t)n, h, conv_w, c->cfg.hidden, c->cfg.eps, w.alpha, alpha_out,
+                               state, y, add_residual, c->num_sms, !c->prof, s);
         prof_end(c, s);
-        if (e != cudaSuccess) return cuda_fail("tcgen05 decode value/conv launch", e);
+        if (e != cudaSuccess) return cuda_fail("decode conv launch", e);
         return ENGRAM_OK;
     }
     if (fused_path(c, n)) {
@@ -305,7 +301,7 @@ engram_status forward_impl(engram_ctx* c, const int32_t* tok, int32_t B, int32_t
         engram_status st = launch_history_transpose(c, conv_state, w, B, M, s);
         if (st != ENGRAM_OK) return st;
     }
-    if (fused) {
+    if (fused && !decode_kernels(c, (int64_t)B * L, L, M)) {
         // cleared ahead of the retrieval, so that the key pass directly follows it
         cudaError_t e = cudaMemsetAsync(w.band, 0, w.counter_bytes, s);
         if (e != cudaSuccess) return cuda_fail("clearing the band counters", e);

@@ -58,18 +58,20 @@ __device__ __forceinline__ uint32_t mod_u64(uint64_t x, uint32_t m, uint64_t rec
     return (uint32_t)r;
 }
 
-// Decode passes (one new position per sequence, at most 256 sequences, bf16,
-// one branch): K split over clusters of four CTAs, partials added through
-// distributed shared memory, the conv state updated in place.
+// Decode (one new position per sequence, at most 256 sequences, bf16, one
+// branch): both projections in one kernel, K split over clusters of four
+// CTAs, partials added through distributed shared memory, the rows' gate
+// partials and v [n][d] fp32 to the workspace; then the gate and conv
+// kernel, a programmatic dependent, which writes alpha and Y and updates the
+// conv state in place.
 bool decode_tc_supported(int64_t n, int32_t L, int32_t d_mem, int32_t d, int32_t M, bool f8);
 int32_t decode_tc_max_tiles(int32_t d);   // channel tiles per row at most (the gate partials' width)
-cudaError_t launch_decode_k(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wk, const void* Wv,
-                            const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
-                            float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
-                            cudaStream_t s);
-cudaError_t launch_decode_v(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wv,
-                            const float* conv_w, int32_t d, const float* alpha, float* state, void* y,
-                            int32_t add_residual, uint32_t* status, int num_sms, bool pdl, cudaStream_t s);
+cudaError_t launch_decode_kv(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wk, const void* Wv,
+                             const float* gq, const float* gk, int32_t d, float* part, float* v, uint32_t* status,
+                             int num_sms, int stall, bool pdl, cudaStream_t s);
+cudaError_t launch_decode_conv(const float* v, const float* part, int32_t n, const void* h, const float* conv_w,
+                               int32_t d, float eps, float* alpha, float* alpha_out, float* state, void* y,
+                               int32_t add_residual, int num_sms, bool pdl, cudaStream_t s);
 
 // ---------------------------------------------------------------- launches
 // Each returns cudaGetLastError() of its launch.

@@ -1,6 +1,6 @@
-// Decode passes: the key and value projections with the gate and the conv,
-// for a call that computes one new position per sequence (L = 1) for at most
-// 256 sequences.
+// Decode: the key and value projections with the gate and the conv, for a
+// call that computes one new position per sequence (L = 1) for at most 256
+// sequences.
 //
 // "DeepSeek AI II" digest, section "DeepSeek Engram": k_t = W_K e_t and
 // v_t = W_V e_t; the scalar gate alpha_t from the RMS-normalised h_t and k_t;
@@ -11,32 +11,44 @@
 // At decode the projections are 256-row GEMMs.  The 128-row tiles of the
 // prefill passes give 40-60 CTAs there, each streaming a full K extent of
 // operands (about 1 MB) through its ring, and the passes are bound by that
-// per-SM stream.  Here each pass spreads the work over the SMs three ways:
+// per-SM stream.  Here two kernels do the work:
 //
+// decode_kv_kernel (both projections, the gate): the work is spread over
+// the SMs three ways.
 //   - a cluster of kSplit = 4 CTAs splits K (d_mem): CTA r of the cluster
-//     multiplies its quarter of the 64-wide k-blocks, for every row (up to
-//     256, in two TMEM accumulators of 128 rows) and the cluster's BN
-//     channels, so a CTA streams a quarter of the K extent;
-//   - the four partial sums are added through distributed shared memory:
-//     each CTA stores every accumulator row into the shared memory of the CTA
-//     that owns the row (rows r*RP .. r*RP+RP-1 belong to CTA r, RP = rows/4),
-//     and the owner adds the four partials in rank order, so the sum does
-//     not depend on timing;
-//   - the owner finishes its RP rows x BN channels with threads running along
-//     the channels: the h, conv-state and output accesses are row pieces, and
-//     the conv state is updated in place (one thread per (sequence, channel)).
+//     multiplies the r-th quarter of the 64-wide k-blocks, for every row (up
+//     to 256, in 128-row TMEM accumulators) and the cluster's BN channels, by
+//     W_K and by W_V: each A stage (e) feeds both products, so e streams
+//     once for the two projections;
+//   - the four partial sums of k, then of v, are added through distributed
+//     shared memory: each CTA stages its accumulator rows in its own ring and
+//     sends each peer, in one bulk copy that completes on the peer's
+//     mbarrier, the rows the peer owns (rows r*RP .. r*RP+RP-1 belong to CTA
+//     r, RP = rows/4); the owner adds the four partials in rank order, so the
+//     sums do not depend on timing;
+//   - the owner finishes its RP rows x BN channels with threads running
+//     along channels: the rows' gate partials for the cluster's channel tile
+//     (sum g_q g_k h k, sum k^2, sum h^2), and v, written to the workspace.
+// decode_conv_kernel (the gate, the conv, SiLU and residual): each CTA
+// reduces the gate partials of the rows it covers into alpha (one warp per
+// row, in channel-tile order), then one thread per four channels of a row
+// reads v, the history and h, writes Y and rewrites the history in place
+// ([v~_{t-2}, v~_{t-1}, v~_t]; each (sequence, channel) belongs to one
+// thread).  It is a programmatic dependent of the first kernel: its CTAs take
+// the SMs' spare slots early and load the history, h and the taps before
+// they wait for v and the partials.
 //
-// The grid is d / BN clusters (BN = 64, 80 or 128, the narrowest that still
-// lets every cluster be resident at once).  The key pass reduces each row's
-// gate partials across its clusters through a per-row-block counter, the
-// last cluster to finish a block computing alpha.  Both passes issue their W
-// loads before waiting for the kernel they depend on (the retrieval, the key
-// pass), so the weight stream overlaps it.
+// The grid of the first kernel is d / BN clusters (BN = 64 or 80, the
+// narrowest whose clusters are all resident at once).  It issues its first W
+// stages before waiting for the retrieval.  Each cluster walks its k-blocks
+// from a different starting block (rotated by its channel tile): every
+// cluster reads the same quarter of e, and the rotation spreads those reads
+// over L2 instead of every cluster asking for the same lines at once.
 //
 // Every mbarrier wait is bounded.  A CTA whose wait runs out flags
 // ENGRAM_ERR_TIMEOUT and votes to abort; after the first cluster barrier every
-// CTA of the cluster reads the votes, and on any abort the cluster stores no
-// partials and writes no output.  The CTA drains its own copies and MMAs
+// CTA of the cluster reads the votes, and on any abort the cluster exchanges
+// nothing and writes nothing.  The CTA drains its own copies and MMAs
 // (bounded) before it frees its TMEM and leaves.
 #include "tc.cuh"
 
@@ -44,69 +56,74 @@ namespace engram {
 
 namespace {
 
-constexpr int DEC_K = 0;
-constexpr int DEC_V = 1;
 constexpr int kSplit = 4;             // CTAs per cluster (K split)
 constexpr int kDecThreads = 256;
 constexpr int kDecStages = 4;
 constexpr int kDecRows = 256;         // rows per call (two 128-row accumulators)
 constexpr int kDecRp = kDecRows / kSplit;   // rows owned by a CTA at most
-constexpr int kAccStride = 128;       // TMEM column of the second accumulator
-constexpr int kTmemCols = 256;
+constexpr int kAccK = 0;              // TMEM columns of the key accumulators (rows 0-127, +128: rows 128-255)
+constexpr int kAccV = 256;            // and of the value accumulators
+constexpr int kRowTile = 128;         // TMEM column offset of the second row tile's accumulator
+constexpr int kTmemCols = 512;
 constexpr int kABytes = 128 * 128;    // one 128-row x 64-element bf16 box
+constexpr int kConvThreads = 256;
 
 template <int BN>
 struct DecGeo {
-    static constexpr int B_BYTES = BN * 128;
-    static constexpr int STAGE_BYTES = 2 * kABytes + B_BYTES;
+    static constexpr int B_BYTES = BN * 128;                  // one W tile: BN rows x 64 elements
+    static constexpr int STAGE_BYTES = 2 * kABytes + 2 * B_BYTES;   // A (256 rows) | W_K tile | W_V tile
     static constexpr int RING = kDecStages * STAGE_BYTES;
     static constexpr int RS = BN + 4;   // floats per staged row (16-byte pad: conflict-free row-per-lane stores)
-    // after the MMAs the ring holds this CTA's partial sums, [256][RS], and
-    // the three peers' partials of the rows it owns, [3][64][RS]
+    // after the MMAs the ring holds this CTA's partial sums of one
+    // projection, [256][RS], and the three peers' partials of the rows it
+    // owns, [3][64][RS]
     static constexpr int STAGE_OFF = 0;
     static constexpr int RECV_OFF = kDecRows * RS * 4;
     static constexpr int EXCH_BYTES = RECV_OFF + (kSplit - 1) * kDecRp * RS * 4;
-    static constexpr int CONST_BYTES = BN * 16;   // conv taps (value pass) or gains (key pass)
+    static constexpr int CONST_BYTES = BN * 4;   // g_q g_k of the tile's channels
     static constexpr int SMEM_BYTES = RING + 1024 + CONST_BYTES + 1024;
-    static constexpr int ITEMS = kDecRp * (BN / 4) / kDecThreads;   // value items per thread at most
     static_assert(EXCH_BYTES <= RING, "the partials reuse the operand ring");
-    static_assert(BN % 16 == 0 && BN <= kAccStride, "UMMA N and the accumulator spacing");
+    static_assert(BN % 16 == 0 && BN <= kRowTile, "UMMA N and the accumulator spacing");
     static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
-    static_assert(kDecRp * (BN / 4) % kDecThreads == 0, "whole value items per thread");
 };
 
 struct __align__(8) DecBarriers {
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
     uint64_t tfull;
-    uint64_t rfull;   // the peers' partials of this CTA's rows have landed
+    uint64_t rfull;   // the peers' partials of this CTA's rows have landed (phase 0: k, phase 1: v)
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;   // this CTA's vote (read by the cluster after the first barrier)
     int issued;       // k-block stages whose loads were issued
     int consumed;     // stages the MMAs have taken
-    int last;         // key pass: this CTA completed its row block's partials
 };
 
 struct DecParams {
-    const __nv_bfloat16* w;        // this pass's weights [d][d_mem]
-    const __nv_bfloat16* w_next;   // key pass: W_V, brought into L2 for the value pass; else null
+    const __nv_bfloat16* wk;       // [d][d_mem]
+    const __nv_bfloat16* wv;       // [d][d_mem]
     const __nv_bfloat16* h;        // [n][d]
     const float* gq;               // [d] or null
     const float* gk;               // [d] or null
-    const float* conv_w;           // [d][4]
-    float* state;                  // [n][3][d] conv history, updated in place, or null (zero history)
-    const float* alpha;            // value pass: [n]
-    float* alpha_w;                // key pass: [n]
-    float* alpha_out;              // key pass: caller's copy, or null
-    float4* part;                  // key pass: [n][n_ct] (sum g h k, sum k^2, sum h^2, 0)
-    int* band_count;               // key pass: [kSplit] per row block (zero on entry, zero on exit)
-    __nv_bfloat16* y;              // value pass: [n][d]
+    float4* part;                  // [n][n_ct] (sum g h k, sum k^2, sum h^2, 0)
+    float* v;                      // [n][d] fp32, for the conv kernel
     uint32_t* status;
     int n, d, d_mem, n_ct;
+    int stall;                     // test hook: CTA 0 announces its first stage and never loads it
+};
+
+struct ConvParams {
+    const float* v;                // [n][d]
+    const float4* part;            // [n][n_ct] gate partials
+    float* alpha_w;                // [n] gate values (written)
+    float* alpha_out;              // caller's copy, or null
+    const __nv_bfloat16* h;        // [n][d]
+    const float* conv_w;           // [d][4]
+    float* state;                  // [n][3][d] conv history, updated in place, or null (zero history)
+    __nv_bfloat16* y;              // [n][d]
+    int n, d, n_ct;
     int add_residual;
     float eps;
-    int stall;                     // test hook: CTA 0 announces its first stage and never loads it
 };
 
 __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, DecBarriers* sb, uint32_t* status) {
@@ -128,12 +145,6 @@ __device__ __forceinline__ void dec_wait_drain(uint64_t* bar, uint32_t parity) {
     const long long t0 = clock64();
     while (!mbar_try_wait(smem_u32(bar), parity) && clock64() - t0 < kWaitCycles) {
     }
-}
-
-__device__ __forceinline__ int dec_atomic_add_acq_rel(int* addr, int v) {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
-    return old;
 }
 
 __device__ __forceinline__ float dec_tanh(float x) {
@@ -162,27 +173,20 @@ __device__ __forceinline__ int owned_rows(int n, int rank, int rp) {
     return r < 0 ? 0 : (r < rp ? r : rp);
 }
 
-// While the MMAs run, warps 2-7 stage the per-channel constants in shared
-// memory (g_q g_k for the key pass, the four conv taps for the value pass)
-// and bring into L2 the k-blocks of the CTA's W slice that the first round of
-// stages does not hold and (key pass) the same slice of W_V, which the value
-// pass CTA with the same cluster rank and channel tile will read.  Offsets
-// and lengths are multiples of 16 bytes (d_mem a multiple of 64).
-template <int MODE, int BN>
-__device__ __forceinline__ void dec_prefetch(const DecParams& p, int rank, int rp, int ct, int kb0, int nkb,
-                                             float* s_const, int t, int nt) {
+// While the MMAs run, warps 2-7 stage g_q g_k of the tile's channels in
+// shared memory and bring the CTA's W_K and W_V slices into L2, so the
+// stages after the first round find them there.  Offsets and lengths are
+// multiples of 16 bytes (d_mem a multiple of 64).
+template <int BN>
+__device__ __forceinline__ void dec_prefetch(const DecParams& p, int ct, int kb0, int nkb, float* s_g, int t, int nt) {
     const int c0 = ct * BN;
-    if (MODE == DEC_K) {
-        for (int c = t; c < BN; c += nt)
-            s_const[c] = (p.gq ? __ldg(p.gq + c0 + c) : 1.f) * (p.gk ? __ldg(p.gk + c0 + c) : 1.f);
-    } else {
-        for (int c = t; c < BN; c += nt)
-            reinterpret_cast<float4*>(s_const)[c] = __ldg(reinterpret_cast<const float4*>(p.conv_w) + c0 + c);
-    }
+    for (int c = t; c < BN; c += nt)
+        s_g[c] = (p.gq ? __ldg(p.gq + c0 + c) : 1.f) * (p.gk ? __ldg(p.gk + c0 + c) : 1.f);
+    if (nkb <= kDecStages) return;
     for (int c = t; c < BN; c += nt) {
         const int64_t wrow = (int64_t)(c0 + c) * p.d_mem + (int64_t)kb0 * 64;
-        if (nkb > kDecStages) prefetch_l2(p.w + wrow + kDecStages * 64, (uint32_t)(nkb - kDecStages) * 128u);
-        if (p.w_next) prefetch_l2(p.w_next + wrow, (uint32_t)nkb * 128u);
+        prefetch_l2(p.wk + wrow, (uint32_t)nkb * 128u);
+        prefetch_l2(p.wv + wrow, (uint32_t)nkb * 128u);
     }
 }
 
@@ -201,10 +205,9 @@ struct PartRows {
     }
 };
 
-// The epilogues' global inputs, loaded into registers before the
-// accumulators complete, so their latency hides behind the MMAs and the
-// exchange.  Key pass: warp w holds h of rows w, w + 8, .. of the CTA's
-// block, lane l channels l, l + 32, ..
+// h of the CTA's owned rows, in registers during the key exchange, so its
+// latency hides behind it: warp w holds rows w, w + 8, .., lane l channels
+// l, l + 32, ..
 template <int BN>
 struct KIn {
     static constexpr int NJ = (BN + 31) / 32;
@@ -227,41 +230,10 @@ struct KIn {
     }
 };
 
-// Value pass: the thread's items (four channels of a row each): history and h.
-template <int BN>
-struct VIn {
-    static constexpr int NQ = BN / 4;
-    static constexpr int NI = DecGeo<BN>::ITEMS;
-    float4 h0[NI], h1[NI], h2[NI];
-    uint2 hq[NI];
-    __device__ __forceinline__ void load(const DecParams& p, int rank, int rp, int ct) {
-        const int items = rp * NQ;
-#pragma unroll
-        for (int b = 0; b < NI; ++b) {
-            const int it = b * kDecThreads + threadIdx.x;
-            const int lr = it / NQ, q4 = it - lr * NQ;
-            const int row = rank * rp + lr;
-            h0[b] = h1[b] = h2[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-            hq[b] = make_uint2(0u, 0u);
-            if (it < items && row < p.n) {
-                const int64_t c = ct * BN + 4 * q4;
-                if (p.state) {
-                    const float4* st = reinterpret_cast<const float4*>(p.state + (int64_t)row * 3 * p.d + c);
-                    h0[b] = __ldcs(st);
-                    h1[b] = __ldcs(st + p.d / 4);
-                    h2[b] = __ldcs(st + p.d / 2);
-                }
-                if (p.add_residual) hq[b] = __ldcs(reinterpret_cast<const uint2*>(p.h + (int64_t)row * p.d + c));
-            }
-        }
-    }
-};
-
-// Gate partials of the CTA's rows over its BN channels, then the row block's
-// alpha by the last of the n_ct clusters to finish the block.
+// Gate partials of the CTA's rows over its BN channels.
 template <int BN>
 __device__ __forceinline__ void dec_epilogue_k(const DecParams& p, const PartRows<BN>& pr, const KIn<BN>& in,
-                                               const float* s_g, int rank, int rp, int ct, DecBarriers* sb) {
+                                               const float* s_g, int rank, int rp, int ct) {
     constexpr int NJ = KIn<BN>::NJ;
     constexpr int NW = KIn<BN>::NW;
     constexpr int RPW = KIn<BN>::RPW;
@@ -292,72 +264,18 @@ __device__ __forceinline__ void dec_epilogue_k(const DecParams& p, const PartRow
         }
         if (lane == 0) p.part[(int64_t)row * p.n_ct + ct] = make_float4(s_qk, s_kk, s_hh, 0.f);
     }
-    // the CTA barrier orders every thread's partials before thread 0's
-    // release at device scope (the count), and its acquire before every
-    // thread's reads of the other clusters' partials
-    __syncthreads();
-    if (threadIdx.x == 0) sb->last = dec_atomic_add_acq_rel(p.band_count + rank, 1) == p.n_ct - 1;
-    __syncthreads();
-    if (!sb->last) return;
-    // every cluster's partials of this row block are visible: four threads
-    // per row reduce a quarter of the channel tiles each, then combine
-    const int lr = threadIdx.x >> 2, qq = threadIdx.x & 3;
-    const int row = rank * rp + lr;
-    const bool live = lr < rp && row < p.n;
-    float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
-    if (live) {
-        const float4* src = p.part + (int64_t)row * p.n_ct;
-#pragma unroll 8
-        for (int t = qq; t < p.n_ct; t += 4) {
-            const float4 v = __ldcg(src + t);
-            s_qk += v.x;
-            s_kk += v.y;
-            s_hh += v.z;
-        }
-    }
-#pragma unroll
-    for (int o = 1; o < 4; o <<= 1) {
-        s_qk += __shfl_xor_sync(0xffffffffu, s_qk, o);
-        s_kk += __shfl_xor_sync(0xffffffffu, s_kk, o);
-        s_hh += __shfl_xor_sync(0xffffffffu, s_hh, o);
-    }
-    if (live && qq == 0) {
-        const float inv_d = 1.f / (float)p.d;
-        const float rh = sqrtf(s_hh * inv_d + p.eps);
-        const float rk = sqrtf(s_kk * inv_d + p.eps);
-        const float a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)p.d)));
-        p.alpha_w[row] = a;
-        if (p.alpha_out) p.alpha_out[row] = a;
-    }
-    if (threadIdx.x == 0) p.band_count[rank] = 0;
 }
 
-// Gate, conv over the history in the caller's state, SiLU, residual; four
-// channels per item, consecutive threads on consecutive channels of a row.
+// v of the CTA's rows over its BN channels: the four partials in rank order,
+// four channels per item, consecutive threads on consecutive channels
 template <int BN>
-__device__ __forceinline__ void dec_epilogue_v(const DecParams& p, const PartRows<BN>& pr, const VIn<BN>& in,
-                                               const float4* s_w, int rank, int rp, int ct) {
-    constexpr int NQ = VIn<BN>::NQ;
-    constexpr int NI = VIn<BN>::NI;
-    const int c0 = ct * BN;
+__device__ __forceinline__ void dec_write_v(const DecParams& p, const PartRows<BN>& pr, int rank, int rp, int ct) {
+    constexpr int NQ = BN / 4;
     const int items = rp * NQ;
-    const int dq = p.d / 4;
-    const auto &h0 = in.h0, &h1 = in.h1, &h2 = in.h2;
-    const auto& hq = in.hq;
-    float a[NI];
-#pragma unroll
-    for (int b = 0; b < NI; ++b) {
-        const int it = b * kDecThreads + threadIdx.x;
-        const int row = rank * rp + it / NQ;
-        a[b] = (it < items && row < p.n) ? __ldg(p.alpha + row) : 0.f;
-    }
-#pragma unroll
-    for (int b = 0; b < NI; ++b) {
-        const int it = b * kDecThreads + threadIdx.x;
+    for (int it = threadIdx.x; it < items; it += kDecThreads) {
         const int lr = it / NQ, q4 = it - lr * NQ;
         const int row = rank * rp + lr;
-        if (it >= items || row >= p.n) continue;
-        const int64_t c = c0 + 4 * q4;
+        if (row >= p.n) break;
         float4 v = *reinterpret_cast<const float4*>(pr.row(0, lr) + 4 * q4);
 #pragma unroll
         for (int src = 1; src < kSplit; ++src) {
@@ -367,46 +285,64 @@ __device__ __forceinline__ void dec_epilogue_v(const DecParams& p, const PartRow
             v.z += u.z;
             v.w += u.w;
         }
-        const float x[4] = {a[b] * v.x, a[b] * v.y, a[b] * v.z, a[b] * v.w};
-        const float s0[4] = {h0[b].x, h0[b].y, h0[b].z, h0[b].w};
-        const float s1[4] = {h1[b].x, h1[b].y, h1[b].z, h1[b].w};
-        const float s2[4] = {h2[b].x, h2[b].y, h2[b].z, h2[b].w};
-        const float hv[4] = {bf16_lo(hq[b].x), bf16_hi(hq[b].x), bf16_lo(hq[b].y), bf16_hi(hq[b].y)};
-        float yv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            // tap j multiplies the input j positions back: x_t, then the
-            // history rows 2, 1, 0 (oldest last)
-            const float4 w = s_w[4 * q4 + e];
-            float u = w.x * x[e];
-            u = fmaf(w.y, s2[e], u);
-            u = fmaf(w.z, s1[e], u);
-            u = fmaf(w.w, s0[e], u);
-            const float hu = 0.5f * u;
-            yv[e] = x[e] + fmaf(hu, dec_tanh(hu), hu) + hv[e];
-        }
-        *reinterpret_cast<uint2*>(p.y + (int64_t)row * p.d + c) =
-            make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
-        if (p.state) {
-            float4* st = reinterpret_cast<float4*>(p.state + (int64_t)row * 3 * p.d + c);
-            st[0] = h1[b];
-            st[dq] = h2[b];
-            st[2 * dq] = make_float4(x[0], x[1], x[2], x[3]);
-        }
+        *reinterpret_cast<float4*>(p.v + (int64_t)row * p.d + ct * BN + 4 * q4) = v;
     }
 }
 
-template <int MODE, int BN>
+// One accumulator pair (rows 0-127 and 128-255) into this CTA's staging
+// rows: warp w reads TMEM lanes 32 (w % 4) .. +31 and channel half w / 4,
+// one row per lane; the padded rows put the lanes' stores in distinct banks
+template <int BN>
+__device__ __forceinline__ void stage_acc(uint32_t tmem, float* stage, int nr) {
+    constexpr int HALF = BN / 2;
+    constexpr int NCH = HALF / 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3, col0 = (warp >> 2) * HALF;
+    for (int rt = 0; rt < nr; ++rt) {
+        const int row = rt * 128 + q * 32 + lane;
+        uint32_t v[NCH][8];
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch)
+            tmem_ld8(tmem + (uint32_t)(rt * kRowTile + col0 + ch * 8) + ((uint32_t)(q * 32) << 16), v[ch]);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(stage + row * DecGeo<BN>::RS + col0);
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) {
+            dst[2 * ch] = make_uint4(v[ch][0], v[ch][1], v[ch][2], v[ch][3]);
+            dst[2 * ch + 1] = make_uint4(v[ch][4], v[ch][5], v[ch][6], v[ch][7]);
+        }
+    }
+    // the bulk copies read the staged rows through the async proxy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// one bulk copy per peer: the staged rows the peer owns (contiguous, padded)
+// into its receive slot for this rank
+template <int BN>
+__device__ __forceinline__ void send_partials(const DecParams& p, DecBarriers* sb, float* stage, float* recv, int rank,
+                                              int rp) {
+    constexpr int RS = DecGeo<BN>::RS;
+    const int t = threadIdx.x;
+    if (t >= kSplit - 1) return;
+    const int o = t < rank ? t : t + 1;
+    const int rows = owned_rows(p.n, o, rp);
+    if (rows <= 0) return;
+    const int slot = rank < o ? rank : rank - 1;
+    bulk_s2cluster(peer_addr(recv + slot * rp * RS, (uint32_t)o), smem_u32(stage + o * rp * RS),
+                   (uint32_t)(rows * RS * 4), peer_addr(&sb->rfull, (uint32_t)o));
+}
+
+template <int BN>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                 const DecParams p) {
+decode_kv_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_bk,
+                 const __grid_constant__ CUtensorMap map_bv, const DecParams p) {
     using GE = DecGeo<BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);   // 1024-byte aligned ring
     const uint32_t ring = smem_u32(smem);
     DecBarriers* sb = reinterpret_cast<DecBarriers*>(smem + GE::RING);
-    float* s_const = reinterpret_cast<float*>(smem + GE::RING + 1024);
+    float* s_g = reinterpret_cast<float*>(smem + GE::RING + 1024);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_rank();
     const int ct = (int)blockIdx.x / kSplit;   // channel tile of the cluster
@@ -416,7 +352,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const int kb_total = p.d_mem / 64;
     const int kb0 = rank * kb_total / kSplit, kb1 = (rank + 1) * kb_total / kSplit;
     const int nkb = kb1 - kb0;
-    const uint32_t stage_tx = (uint32_t)(nr * kABytes + GE::B_BYTES);
+    const int rot = nkb > 0 ? ct % nkb : 0;   // this cluster's first k-block (see the header)
+    const uint32_t stage_tx = (uint32_t)(nr * kABytes + 2 * GE::B_BYTES);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecStages; ++s) {
@@ -429,11 +366,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         sb->abort_flag = 0;
         sb->issued = 0;
         sb->consumed = 0;
-        sb->last = 0;
         mbar_fence_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&map_a);
-        tma_prefetch_desc(&map_b);
+        tma_prefetch_desc(&map_bk);
+        tma_prefetch_desc(&map_bv);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sb->tmem_base)),
@@ -450,39 +387,38 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // ---------------- TMA producer
         if (lane == 0) {
             const int pre = nkb < kDecStages ? nkb : kDecStages;
-            auto load_b = [&](int j) {
+            auto kcol = [&](int j) { return (kb0 + (j + rot) % nkb) * 64; };
+            auto load_w = [&](int j) {
                 const int s = j % kDecStages;
                 mbar_arrive_expect_tx(&sb->full[s], stage_tx);
                 if (p.stall && j == 0 && blockIdx.x == 0) return;   // bounded-wait test: never loaded
-                tma_load_2d(&map_b, ring + s * GE::STAGE_BYTES + 2 * kABytes, &sb->full[s], (kb0 + j) * 64, ct * BN);
+                const uint32_t b = ring + s * GE::STAGE_BYTES + 2 * kABytes;
+                tma_load_2d(&map_bk, b, &sb->full[s], kcol(j), ct * BN);
+                tma_load_2d(&map_bv, b + GE::B_BYTES, &sb->full[s], kcol(j), ct * BN);
             };
             auto load_a = [&](int j) {
                 const int s = j % kDecStages;
                 if (p.stall && j == 0 && blockIdx.x == 0) return;
                 for (int rt = 0; rt < nr; ++rt)
-                    tma_load_2d(&map_a, ring + s * GE::STAGE_BYTES + rt * kABytes, &sb->full[s], (kb0 + j) * 64,
-                                rt * 128);
+                    tma_load_2d(&map_a, ring + s * GE::STAGE_BYTES + rt * kABytes, &sb->full[s], kcol(j), rt * 128);
             };
-            // the weights do not depend on the kernel before this one: their
-            // first stages stream while it finishes.  The key pass reads e,
-            // which the retrieval before it writes; the value pass reads e
-            // only after the key pass, which waited for the retrieval, let
-            // it launch
-            for (int j = 0; j < pre; ++j) load_b(j);
-            if (MODE == DEC_K) grid_dep_wait();
+            // the weights do not depend on the retrieval: their first stages
+            // stream while it finishes; e is read after it completes
+            for (int j = 0; j < pre; ++j) load_w(j);
+            grid_dep_wait();
             for (int j = 0; j < pre; ++j) load_a(j);
             sb->issued = pre;
             for (int j = pre; j < nkb; ++j) {
                 const int s = j % kDecStages;
                 if (!dec_wait(&sb->empty[s], ((uint32_t)(j / kDecStages) & 1u) ^ 1u, sb, p.status)) break;
-                load_b(j);
+                load_w(j);
                 load_a(j);
                 sb->issued = j + 1;
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: each A stage feeds k and v
         if (lane == 0) {
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
@@ -493,13 +429,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 }
                 tc_fence_after();
                 const uint32_t a_addr = ring + s * GE::STAGE_BYTES;
-                const uint64_t db = smem_desc_sw128(a_addr + 2 * kABytes);
+                const uint64_t dbk = smem_desc_sw128(a_addr + 2 * kABytes);
+                const uint64_t dbv = smem_desc_sw128(a_addr + 2 * kABytes + GE::B_BYTES);
                 for (int rt = 0; rt < nr; ++rt) {
                     const uint64_t da = smem_desc_sw128(a_addr + rt * kABytes);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16<BN>(tmem_base + (uint32_t)(rt * kAccStride), da + (uint64_t)(kk * 2),
-                                      db + (uint64_t)(kk * 2), (j | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        umma_bf16<BN>(tmem_base + (uint32_t)(kAccK + rt * kRowTile), da + (uint64_t)(kk * 2),
+                                      dbk + (uint64_t)(kk * 2), (j | kk) != 0);
+                        umma_bf16<BN>(tmem_base + (uint32_t)(kAccV + rt * kRowTile), da + (uint64_t)(kk * 2),
+                                      dbv + (uint64_t)(kk * 2), (j | kk) != 0);
+                    }
                 }
                 umma_commit(&sb->empty[s]);
                 sb->consumed = j + 1;
@@ -508,54 +448,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
         __syncwarp();
     } else {
-        dec_prefetch<MODE, BN>(p, rank, rp, ct, kb0, nkb, s_const, threadIdx.x - 64, kDecThreads - 64);
+        dec_prefetch<BN>(p, ct, kb0, nkb, s_g, threadIdx.x - 64, kDecThreads - 64);
     }
-    // key pass: the value pass may launch once every thread of every CTA is
-    // past the retrieval (warp 0 follows its lane 0, which waited above)
-    if (MODE == DEC_K) {
-        if (warp != 0) grid_dep_wait();
-        grid_dep_launch_dependents();
-    }
+    // the conv kernel may launch once every thread of every CTA is past the
+    // retrieval (warp 0 follows its lane 0, which waited above); its CTAs
+    // load the history and h while this grid runs
+    if (warp != 0) grid_dep_wait();
+    grid_dep_launch_dependents();
 
-    // ---------------- accumulators complete: stage them in this CTA's ring
+    // ---------------- accumulators complete
     const bool ok = nkb > 0 && dec_wait(&sb->tfull, 0, sb, p.status);
     const int cta_abort = __syncthreads_or(!ok || sb->abort_flag);
     tc_fence_after();
     float* stage = reinterpret_cast<float*>(smem + GE::STAGE_OFF);
     float* recv = reinterpret_cast<float*>(smem + GE::RECV_OFF);
-    if (!cta_abort) {
-        // warp w reads TMEM lanes 32 (w % 4) .. +31 and channel half w / 4;
-        // one row per lane, padded rows: the stores hit distinct banks
-        constexpr int HALF = BN / 2;
-        constexpr int NCH = HALF / 8;
-        const int q = warp & 3, col0 = (warp >> 2) * HALF;
-        for (int rt = 0; rt < nr; ++rt) {
-            const int row = rt * 128 + q * 32 + lane;
-            uint32_t v[NCH][8];
-#pragma unroll
-            for (int ch = 0; ch < NCH; ++ch)
-                tmem_ld8(tmem_base + (uint32_t)(rt * kAccStride + col0 + ch * 8) + ((uint32_t)(q * 32) << 16), v[ch]);
-            tmem_wait_ld();
-            uint4* dst = reinterpret_cast<uint4*>(stage + row * GE::RS + col0);
-#pragma unroll
-            for (int ch = 0; ch < NCH; ++ch) {
-                dst[2 * ch] = make_uint4(v[ch][0], v[ch][1], v[ch][2], v[ch][3]);
-                dst[2 * ch + 1] = make_uint4(v[ch][4], v[ch][5], v[ch][6], v[ch][7]);
-            }
-        }
-        // the bulk copies below read the staged rows through the async proxy
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    // the epilogue's global inputs, in flight during the exchange (issued
-    // after the proxy fence, which would otherwise wait for them)
-    KIn<BN> kin;
-    VIn<BN> vin;
-    if (MODE == DEC_K) kin.load(p, rank, rp, ct);
-    else vin.load(p, rank, rp, ct);
+    const PartRows<BN> pr{stage, recv, rank, rp};
+    const uint32_t rbytes = (uint32_t)((kSplit - 1) * owned_rows(p.n, rank, rp) * GE::RS * 4);
+
+    // ---- k: stage, exchange, gate partials and alpha
+    if (!cta_abort) stage_acc<BN>(tmem_base + kAccK, stage, nr);
     if (threadIdx.x == 0) {
         sb->abort_flag = cta_abort;
-        // the three peers' copies of the rows this CTA owns (padded rows)
-        mbar_arrive_expect_tx(&sb->rfull, (uint32_t)((kSplit - 1) * owned_rows(p.n, rank, rp) * GE::RS * 4));
+        mbar_arrive_expect_tx(&sb->rfull, rbytes);   // phase 0: the peers' k rows
     }
     tc_fence_before();
     // barrier 1: every CTA's MMAs have finished reading its ring, which now
@@ -565,35 +479,41 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     int any_abort = 0;
 #pragma unroll
     for (int r = 0; r < kSplit; ++r) any_abort |= ld_remote_s32(peer_addr(&sb->abort_flag, (uint32_t)r));
-
+    // h of the owned rows, in flight during the exchange (issued after the
+    // barrier, whose release would otherwise wait for the loads)
+    KIn<BN> kin;
+    kin.load(p, rank, rp, ct);
     bool have = false;
     if (!any_abort) {
-        // one bulk copy per peer: the staged rows the peer owns (contiguous,
-        // padded) into its receive slot for this rank
-        const int t = threadIdx.x;
-        if (t < kSplit - 1) {
-            const int o = t < rank ? t : t + 1;
-            const int rows = owned_rows(p.n, o, rp);
-            if (rows > 0) {
-                const int slot = rank < o ? rank : rank - 1;
-                bulk_s2cluster(peer_addr(recv + slot * rp * GE::RS, (uint32_t)o), smem_u32(stage + o * rp * GE::RS),
-                               (uint32_t)(rows * GE::RS * 4), peer_addr(&sb->rfull, (uint32_t)o));
-            }
-        }
+        send_partials<BN>(p, sb, stage, recv, rank, rp);
         have = dec_wait(&sb->rfull, 0, sb, p.status);
     }
-    // barrier 2: every copy has landed, so no CTA's staged rows are read any more
+    // barrier 2: every k copy has landed, so no CTA's staged rows are read any more
     __syncwarp();
     cluster_sync_all();
+    const bool go = !any_abort && __syncthreads_and(have);
+    if (go) dec_epilogue_k<BN>(p, pr, kin, s_g, rank, rp, ct);
+    __syncthreads();   // the k rows are read: the ring takes v
 
-    if (!any_abort && __syncthreads_and(have)) {
-        const PartRows<BN> pr{stage, recv, rank, rp};
-        if (MODE == DEC_K) {
-            dec_epilogue_k<BN>(p, pr, kin, s_const, rank, rp, ct, sb);
-        } else {
-            grid_dep_wait();   // alpha comes from the key pass
-            dec_epilogue_v<BN>(p, pr, vin, reinterpret_cast<const float4*>(s_const), rank, rp, ct);
-        }
+    // ---- v: stage, exchange, write
+    if (go) {
+        stage_acc<BN>(tmem_base + kAccV, stage, nr);
+        if (threadIdx.x == 0) mbar_arrive_expect_tx(&sb->rfull, rbytes);   // phase 1: the peers' v rows
+    }
+    tc_fence_before();
+    // barrier 3: every CTA has read its k rows, so the receive slots are free
+    __syncwarp();
+    cluster_sync_all();
+    bool have_v = false;
+    if (go) {
+        send_partials<BN>(p, sb, stage, recv, rank, rp);
+        have_v = dec_wait(&sb->rfull, 1, sb, p.status);
+    }
+    // barrier 4: every v copy has landed
+    __syncwarp();
+    cluster_sync_all();
+    if (go && __syncthreads_and(have_v)) {
+        dec_write_v<BN>(p, pr, rank, rp, ct);
     } else if (cta_abort) {
         // this CTA stopped early: wait out the copies and MMAs it issued
         if (warp == 0 && lane == 0)
@@ -612,15 +532,105 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
 }
 
+// Gate, conv over the history in the caller's state, SiLU, residual; one
+// thread per four channels of a row.  The history, h and the taps are read
+// before the wait for the kernel that writes v and the gate partials; then
+// warp w reduces the partials of the CTA's w-th row into alpha (a CTA covers
+// at most 8 rows: d is a multiple of 128, so a row is at least 32 items).
+constexpr int kConvRows = kConvThreads / 32;
+
+__global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const ConvParams q) {
+    __shared__ float s_alpha[kConvRows];
+    const int dq = q.d / 4;
+    const int64_t it0 = (int64_t)blockIdx.x * kConvThreads;
+    const int64_t it = it0 + threadIdx.x;
+    const bool live = it < (int64_t)q.n * dq;
+    const int64_t row = live ? it / dq : 0;
+    const int c = live ? (int)(it - row * dq) * 4 : 0;
+    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0, s2 = s0;
+    uint2 hq = make_uint2(0u, 0u);
+    float4 w[4];
+    float4* st = nullptr;
+    if (live) {
+        if (q.state) {
+            st = reinterpret_cast<float4*>(q.state + row * 3 * q.d + c);
+            s0 = __ldcs(st);
+            s1 = __ldcs(st + dq);
+            s2 = __ldcs(st + 2 * dq);
+        }
+        if (q.add_residual) hq = __ldcs(reinterpret_cast<const uint2*>(q.h + row * q.d + c));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = __ldg(reinterpret_cast<const float4*>(q.conv_w) + c + e);
+    }
+    grid_dep_wait();   // v and the gate partials come from the projection kernel
+
+    // alpha of the rows this CTA covers, each reduced in channel-tile order
+    const int64_t row0 = it0 / dq;
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r = row0 + wid;
+    if (r < q.n && r * dq < it0 + kConvThreads) {
+        float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
+        for (int t = lane; t < q.n_ct; t += 32) {
+            const float4 v = __ldcg(q.part + r * q.n_ct + t);
+            s_qk += v.x;
+            s_kk += v.y;
+            s_hh += v.z;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s_qk += __shfl_xor_sync(0xffffffffu, s_qk, o);
+            s_kk += __shfl_xor_sync(0xffffffffu, s_kk, o);
+            s_hh += __shfl_xor_sync(0xffffffffu, s_hh, o);
+        }
+        if (lane == 0) {
+            const float inv_d = 1.f / (float)q.d;
+            const float rh = sqrtf(s_hh * inv_d + q.eps);
+            const float rk = sqrtf(s_kk * inv_d + q.eps);
+            const float a = 1.f / (1.f + expf(-(s_qk / (rh * rk)) * rsqrtf((float)q.d)));
+            s_alpha[wid] = a;
+            // the CTA that holds the row's first channels publishes it
+            if (r * dq >= it0) {
+                q.alpha_w[r] = a;
+                if (q.alpha_out) q.alpha_out[r] = a;
+            }
+        }
+    }
+    __syncthreads();
+    if (!live) return;
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(q.v + row * q.d + c));
+    const float a = s_alpha[row - row0];
+    const float x[4] = {a * v.x, a * v.y, a * v.z, a * v.w};
+    const float h0[4] = {s0.x, s0.y, s0.z, s0.w}, h1[4] = {s1.x, s1.y, s1.z, s1.w}, h2[4] = {s2.x, s2.y, s2.z, s2.w};
+    const float hv[4] = {bf16_lo(hq.x), bf16_hi(hq.x), bf16_lo(hq.y), bf16_hi(hq.y)};
+    float yv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        // tap j multiplies the input j positions back: x_t, then the history
+        // rows 2, 1, 0 (oldest last)
+        float u = w[e].x * x[e];
+        u = fmaf(w[e].y, h2[e], u);
+        u = fmaf(w[e].z, h1[e], u);
+        u = fmaf(w[e].w, h0[e], u);
+        const float hu = 0.5f * u;
+        yv[e] = x[e] + fmaf(hu, dec_tanh(hu), hu) + hv[e];
+    }
+    *reinterpret_cast<uint2*>(q.y + row * q.d + c) = make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
+    if (st) {
+        st[0] = s1;
+        st[dq] = s2;
+        st[2 * dq] = make_float4(x[0], x[1], x[2], x[3]);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
-// clusters of kSplit CTAs of the largest decode kernel that the device holds at once
+// clusters of kSplit CTAs of the decode kernel that the device holds at once
 int resident_clusters(int num_sms) {
     static int cached[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && cached[dev] > 0) return cached[dev];
-    auto kernel = decode_tc_kernel<DEC_V, 80>;
+    auto kernel = decode_kv_kernel<80>;
     int mc = 0;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DecGeo<80>::SMEM_BYTES) ==
         cudaSuccess) {
@@ -645,9 +655,10 @@ int pick_dec_bn(int32_t d, int num_sms) {
     return 80;
 }
 
-template <int MODE, int BN>
-cudaError_t launch_dec(const CUtensorMap& ma, const CUtensorMap& mb, DecParams p, bool pdl, cudaStream_t s) {
-    auto kernel = decode_tc_kernel<MODE, BN>;
+template <int BN>
+cudaError_t launch_kv(const CUtensorMap& ma, const CUtensorMap& mk, const CUtensorMap& mv, DecParams p, bool pdl,
+                      cudaStream_t s) {
+    auto kernel = decode_kv_kernel<BN>;
     static unsigned long long attr_set = 0;   // one bit per device ordinal
     int dev = 0;
     cudaGetDevice(&dev);
@@ -671,13 +682,7 @@ cudaError_t launch_dec(const CUtensorMap& ma, const CUtensorMap& mb, DecParams p
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
-}
-
-template <int MODE>
-cudaError_t launch_dec_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, const DecParams& p, bool pdl,
-                          cudaStream_t s) {
-    return bn == 80 ? launch_dec<MODE, 80>(ma, mb, p, pdl, s) : launch_dec<MODE, 64>(ma, mb, p, pdl, s);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mk, mv, p);
 }
 
 }  // namespace
@@ -689,55 +694,62 @@ bool decode_tc_supported(int64_t n, int32_t L, int32_t d_mem, int32_t d, int32_t
 
 int32_t decode_tc_max_tiles(int32_t d) { return d / 64; }
 
-cudaError_t launch_decode_k(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wk, const void* Wv,
-                            const float* gq, const float* gk, int32_t d, float eps, float* part, int* band_count,
-                            float* alpha, float* alpha_out, uint32_t* status, int num_sms, int stall, bool pdl,
-                            cudaStream_t s) {
+cudaError_t launch_decode_kv(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wk, const void* Wv,
+                             const float* gq, const float* gk, int32_t d, float* part, float* v, uint32_t* status,
+                             int num_sms, int stall, bool pdl, cudaStream_t s) {
     if (!decode_tc_supported(n, 1, d_mem, d, 1, false)) return cudaErrorNotSupported;
     const int bn = pick_dec_bn(d, num_sms);
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, e, (uint64_t)n, (uint64_t)d_mem, 128) || !make_map(&mb, Wk, (uint64_t)d, (uint64_t)d_mem, bn))
+    CUtensorMap ma, mk, mv;
+    if (!make_map(&ma, e, (uint64_t)n, (uint64_t)d_mem, 128) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn) ||
+        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn))
         return cudaErrorInvalidValue;
     DecParams p{};
-    p.w = static_cast<const __nv_bfloat16*>(Wk);
-    p.w_next = static_cast<const __nv_bfloat16*>(Wv);
+    p.wk = static_cast<const __nv_bfloat16*>(Wk);
+    p.wv = static_cast<const __nv_bfloat16*>(Wv);
     p.h = static_cast<const __nv_bfloat16*>(h);
     p.gq = gq;
     p.gk = gk;
-    p.alpha_w = alpha;
-    p.alpha_out = alpha_out;
     p.part = reinterpret_cast<float4*>(part);
-    p.band_count = band_count;
+    p.v = v;
     p.status = status;
     p.n = n;
     p.d = d;
     p.d_mem = d_mem;
-    p.eps = eps;
     p.stall = stall;
-    return launch_dec_bn<DEC_K>(bn, ma, mb, p, pdl, s);
+    return bn == 80 ? launch_kv<80>(ma, mk, mv, p, pdl, s) : launch_kv<64>(ma, mk, mv, p, pdl, s);
 }
 
-cudaError_t launch_decode_v(const void* e, int32_t n, int32_t d_mem, const void* h, const void* Wv,
-                            const float* conv_w, int32_t d, const float* alpha, float* state, void* y,
-                            int32_t add_residual, uint32_t* status, int num_sms, bool pdl, cudaStream_t s) {
-    if (!decode_tc_supported(n, 1, d_mem, d, 1, false)) return cudaErrorNotSupported;
-    const int bn = pick_dec_bn(d, num_sms);
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, e, (uint64_t)n, (uint64_t)d_mem, 128) || !make_map(&mb, Wv, (uint64_t)d, (uint64_t)d_mem, bn))
-        return cudaErrorInvalidValue;
-    DecParams p{};
-    p.w = static_cast<const __nv_bfloat16*>(Wv);
-    p.h = static_cast<const __nv_bfloat16*>(h);
-    p.conv_w = conv_w;
-    p.state = state;
-    p.alpha = alpha;
-    p.y = static_cast<__nv_bfloat16*>(y);
-    p.status = status;
-    p.n = n;
-    p.d = d;
-    p.d_mem = d_mem;
-    p.add_residual = add_residual;
-    return launch_dec_bn<DEC_V>(bn, ma, mb, p, pdl, s);
+cudaError_t launch_decode_conv(const float* v, const float* part, int32_t n, const void* h, const float* conv_w,
+                               int32_t d, float eps, float* alpha, float* alpha_out, float* state, void* y,
+                               int32_t add_residual, int num_sms, bool pdl, cudaStream_t s) {
+    ConvParams q{};
+    q.v = v;
+    q.part = reinterpret_cast<const float4*>(part);
+    q.alpha_w = alpha;
+    q.alpha_out = alpha_out;
+    q.h = static_cast<const __nv_bfloat16*>(h);
+    q.conv_w = conv_w;
+    q.state = state;
+    q.y = static_cast<__nv_bfloat16*>(y);
+    q.n = n;
+    q.d = d;
+    q.n_ct = d / pick_dec_bn(d, num_sms);   // the projection kernel's channel tiles
+    q.add_residual = add_residual;
+    q.eps = eps;
+    const int64_t items = (int64_t)n * (d / 4);
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((items + kConvThreads - 1) / kConvThreads), 1, 1);
+    cfg.blockDim = dim3(kConvThreads, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, decode_conv_kernel, q);
 }
 
 }  // namespace engram

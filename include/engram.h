@@ -137,8 +137,9 @@ ENGRAM_API const char* engram_last_error(void);
  * [B][w-1][d] f32, for other fused calls with L <= 8 a second history buffer
  * (the history in the sequence-minor layout [w-1][d][B] that the value pass
  * reads coalesced across sequences) and, where the gate and conv are not
- * fused into the projection (see engram_gate_conv), v [n_tok][d] f32; each
- * part 256-byte aligned.  0 for a null context. */
+ * fused into the projection (see engram_gate_conv) or for the decode
+ * kernels, v [n_tok][d] f32; each part 256-byte aligned.  0 for a null
+ * context. */
 ENGRAM_API size_t engram_workspace_bytes(const engram_ctx* ctx, int32_t B, int32_t L);
 
 /* Per-kernel timing for benchmarks.  While enabled, every entry point records

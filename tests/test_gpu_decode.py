@@ -1,11 +1,12 @@
-"""The decode passes (one new position per sequence, at most 256 sequences,
+"""The decode path (one new position per sequence, at most 256 sequences,
 bf16) against the oracle, through engram_forward.
 
-These calls run the cluster split-K key and value passes: partial sums added
-through distributed shared memory, the gate's row sums across clusters, and
-the conv state read and rewritten in place.  Covered: one and two 128-row
-accumulators (1 to 256 sequences, ragged), every channel tile width (64, 80
-and 128 channels: d = 256, 384, 2560), K extents that split evenly and
+These calls run the decode kernels: both projections in one cluster split-K
+kernel (partial sums added through distributed shared memory, the gate's row
+sums across clusters), then the conv kernel, which reads and rewrites the
+conv state in place.  Covered: one and two 128-row accumulators (1 to 256
+sequences, ragged), both channel tile widths (64 channels: d = 256, 384, 512;
+80 channels: d = 2560 on a full B200), K extents that split evenly and
 unevenly over the four CTAs of a cluster, with and without conv state and
 residual, bitwise determinism, and dependent against plain launches."""
 
@@ -100,8 +101,8 @@ def test_decode_runs_the_decode_kernels(eb):
     ctx = eb.Engram(config_for(inp, eb))
     state = inp.device_state("cuda:0").contiguous()
     names = _kernels(eb, ctx, di, state)
-    # no history transpose and no merge: the value pass rewrites the state in place
-    assert names == ["retrieve", "gate_k_decode", "vconv_decode"], names
+    # no history transpose and no merge: the conv kernel rewrites the state in place
+    assert names == ["retrieve", "gate_kv_decode", "conv_decode"], names
 
 
 def test_decode_without_gains(eb):
@@ -122,8 +123,8 @@ def test_decode_without_gains(eb):
 def test_decode_deterministic_and_dependent_launches_match_plain(eb, name):
     """Same bits from two dependent-launch runs and from a run with kernel
     timing on (plain launches with events between them).  A decode on other
-    hidden states runs first, so a value pass that read alpha before the key
-    pass completed would see different values."""
+    hidden states runs first, so a conv kernel that read v or alpha before the
+    projection kernel completed would see different values."""
     wl = CASES[name]
     inp = synth.Inputs(wl, gamma="random")
     di = DeviceInputs(inp)

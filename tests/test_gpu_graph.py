@@ -97,7 +97,7 @@ def test_profile_events_inside_a_graph(eb):
             g.replay()
             torch.cuda.synchronize()
             prof = eb.engram_profile_read(ctx.ctx)
-            assert [n for n, _ in prof] == ["retrieve", "gate_k_decode", "vconv_decode"], prof
+            assert [n for n, _ in prof] == ["retrieve", "gate_kv_decode", "conv_decode"], prof
             assert all(t > 0.0 for _, t in prof), prof
         del g
     finally:
