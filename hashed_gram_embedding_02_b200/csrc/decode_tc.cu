@@ -13,21 +13,20 @@
 // operands (about 1 MB) through its ring, and the passes are bound by that
 // per-SM stream.  Here two kernels do the work:
 //
-// decode_kv_kernel (both projections, the gate): the work is spread over
-// the SMs three ways.
-//   - a cluster of kSplit = 4 CTAs splits K (d_mem): CTA r of the cluster
-//     multiplies the r-th quarter of the 64-wide k-blocks, for every row (up
-//     to 256, in 128-row TMEM accumulators) and the cluster's BN channels, by
-//     W_K and by W_V: each A stage (e) feeds both products, so e streams
-//     once for the two projections;
-//   - the four partial sums of k, then of v, are added through distributed
-//     shared memory: each CTA stages its accumulator rows in its own ring and
-//     sends each peer, in one bulk copy that completes on the peer's
-//     mbarrier, the rows the peer owns (rows r*RP .. r*RP+RP-1 belong to CTA
-//     r, RP = rows/4); the owner adds the four partials in rank order, so the
-//     sums do not depend on timing;
-//   - the owner finishes its RP rows x BN channels with threads running
-//     along channels: the rows' gate partials for the cluster's channel tile
+// decode_kv_kernel (both projections, the gate partials): a cluster of 4
+// CTAs per channel tile of BN channels, as two CTA pairs.
+//   - each pair multiplies one half of K (d_mem) with M = 256 tcgen05 MMAs
+//     (cta_group::2): each CTA of the pair stages its 128 rows of e and half
+//     of the tile's W_K and W_V rows, and its TMEM receives its 128 rows of
+//     k and v over all BN channels; each A stage of e feeds both products, so
+//     e streams once for the two projections;
+//   - the two halves of K are added through distributed shared memory: each
+//     CTA stages its k and v rows in its own ring and sends, in two bulk
+//     copies that complete on the receiver's mbarrier, the 64 rows that the
+//     CTA holding the same rows from the other half of K owns; the owner adds
+//     the two partials in K-half order, so the sums do not depend on timing;
+//   - the owner finishes its 64 rows x BN channels with threads running
+//     along channels: the rows' gate partials for the channel tile
 //     (sum g_q g_k h k, sum k^2, sum h^2), and v, written to the workspace.
 // decode_conv_kernel (the gate, the conv, SiLU and residual): each CTA
 // reduces the gate partials of the rows it covers into alpha (one warp per
@@ -42,7 +41,7 @@
 // narrowest whose clusters are all resident at once).  It issues its first W
 // stages before waiting for the retrieval.  Each cluster walks its k-blocks
 // from a different starting block (rotated by its channel tile): every
-// cluster reads the same quarter of e, and the rotation spreads those reads
+// cluster reads the same half of e, and the rotation spreads those reads
 // over L2 instead of every cluster asking for the same lines at once.
 //
 // Every mbarrier wait is bounded.  A CTA whose wait runs out flags
@@ -56,42 +55,48 @@ namespace engram {
 
 namespace {
 
-constexpr int kSplit = 4;             // CTAs per cluster (K split)
+constexpr int kCluster = 4;           // CTAs per cluster: two CTA pairs, one per half of K
 constexpr int kDecThreads = 256;
-constexpr int kDecStages = 4;
-constexpr int kDecRows = 256;         // rows per call (two 128-row accumulators)
-constexpr int kDecRp = kDecRows / kSplit;   // rows owned by a CTA at most
-constexpr int kAccK = 0;              // TMEM columns of the key accumulators (rows 0-127, +128: rows 128-255)
-constexpr int kAccV = 256;            // and of the value accumulators
-constexpr int kRowTile = 128;         // TMEM column offset of the second row tile's accumulator
-constexpr int kTmemCols = 512;
+constexpr int kDecStages = 8;
+constexpr int kDecRows = 256;         // rows per call: one M = 256 pair accumulator
+constexpr int kOwnRows = 64;          // rows a CTA finishes (half of its 128 accumulator rows)
+constexpr int kAccK = 0;              // TMEM columns of the key accumulator
+constexpr int kAccV = 128;            // and of the value accumulator
+constexpr int kTmemCols = 256;
 constexpr int kABytes = 128 * 128;    // one 128-row x 64-element bf16 box
 constexpr int kConvThreads = 256;
 
 template <int BN>
 struct DecGeo {
-    static constexpr int B_BYTES = BN * 128;                  // one W tile: BN rows x 64 elements
-    static constexpr int STAGE_BYTES = 2 * kABytes + 2 * B_BYTES;   // A (256 rows) | W_K tile | W_V tile
+    static constexpr int B_ROWS = BN / 2;                     // W rows (channels) this CTA of a pair stages
+    static constexpr int B_BYTES = B_ROWS * 128;
+    static constexpr int STAGE_BYTES = kABytes + 2 * B_BYTES;   // A (this CTA's 128 rows) | W_K half | W_V half
     static constexpr int RING = kDecStages * STAGE_BYTES;
     static constexpr int RS = BN + 4;   // floats per staged row (16-byte pad: conflict-free row-per-lane stores)
-    // after the MMAs the ring holds this CTA's partial sums of one
-    // projection, [256][RS], and the three peers' partials of the rows it
-    // owns, [3][64][RS]
-    static constexpr int STAGE_OFF = 0;
-    static constexpr int RECV_OFF = kDecRows * RS * 4;
-    static constexpr int EXCH_BYTES = RECV_OFF + (kSplit - 1) * kDecRp * RS * 4;
+    // after the MMAs the ring holds, for k and then for v, this CTA's
+    // partial sums [128][RS] and the partner's partials of the rows it owns
+    // [64][RS]
+    static constexpr int PART_BYTES = 128 * RS * 4;
+    static constexpr int RECV_BYTES = kOwnRows * RS * 4;
+    static constexpr int STAGE_K = 0;
+    static constexpr int RECV_K = STAGE_K + PART_BYTES;
+    static constexpr int STAGE_V = RECV_K + RECV_BYTES;
+    static constexpr int RECV_V = STAGE_V + PART_BYTES;
+    static constexpr int EXCH_BYTES = RECV_V + RECV_BYTES;
     static constexpr int CONST_BYTES = BN * 4;   // g_q g_k of the tile's channels
     static constexpr int SMEM_BYTES = RING + 1024 + CONST_BYTES + 1024;
     static_assert(EXCH_BYTES <= RING, "the partials reuse the operand ring");
-    static_assert(BN % 16 == 0 && BN <= kRowTile, "UMMA N and the accumulator spacing");
+    static_assert(BN % 16 == 0 && BN <= kAccV, "UMMA N and the accumulator spacing");
+    static_assert(B_ROWS % 8 == 0, "whole 8-row swizzle atoms per W half");
     static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 };
 
 struct __align__(8) DecBarriers {
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
+    uint64_t pfull[kDecStages];   // leader: the partner CTA's half of the stage is full
     uint64_t tfull;
-    uint64_t rfull;   // the peers' partials of this CTA's rows have landed (phase 0: k, phase 1: v)
+    uint64_t rfull;   // the other half of K's partials (k and v) of this CTA's rows have landed
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;   // this CTA's vote (read by the cluster after the first barrier)
@@ -168,40 +173,41 @@ __device__ __forceinline__ void bulk_s2cluster(uint32_t dst_cluster, uint32_t sr
         : "memory");
 }
 
-__device__ __forceinline__ int owned_rows(int n, int rank, int rp) {
-    const int r = n - rank * rp;
-    return r < 0 ? 0 : (r < rp ? r : rp);
+// rows of [first, first + kOwnRows) below n
+__device__ __forceinline__ int live_rows(int n, int first) {
+    const int r = n - first;
+    return r < 0 ? 0 : (r < kOwnRows ? r : kOwnRows);
 }
 
 // While the MMAs run, warps 2-7 stage g_q g_k of the tile's channels in
-// shared memory and bring the CTA's W_K and W_V slices into L2, so the
-// stages after the first round find them there.  Offsets and lengths are
-// multiples of 16 bytes (d_mem a multiple of 64).
+// shared memory and bring this CTA's halves of the W_K and W_V slices into
+// L2, so the stages after the first round find them there.  Offsets and
+// lengths are multiples of 16 bytes (d_mem a multiple of 64).
 template <int BN>
-__device__ __forceinline__ void dec_prefetch(const DecParams& p, int ct, int kb0, int nkb, float* s_g, int t, int nt) {
+__device__ __forceinline__ void dec_prefetch(const DecParams& p, int ct, int w_row0, int kb0, int nkb, float* s_g,
+                                             int t, int nt) {
     const int c0 = ct * BN;
     for (int c = t; c < BN; c += nt)
         s_g[c] = (p.gq ? __ldg(p.gq + c0 + c) : 1.f) * (p.gk ? __ldg(p.gk + c0 + c) : 1.f);
     if (nkb <= kDecStages) return;
-    for (int c = t; c < BN; c += nt) {
-        const int64_t wrow = (int64_t)(c0 + c) * p.d_mem + (int64_t)kb0 * 64;
+    for (int c = t; c < DecGeo<BN>::B_ROWS; c += nt) {
+        const int64_t wrow = (int64_t)(w_row0 + c) * p.d_mem + (int64_t)kb0 * 64;
         prefetch_l2(p.wk + wrow, (uint32_t)nkb * 128u);
         prefetch_l2(p.wv + wrow, (uint32_t)nkb * 128u);
     }
 }
 
-// The four partial sums of an owned row, in rank order: this CTA's own from
-// its staging rows, the peers' from the receive slots.
+// The two partial sums of an owned row, in K-half order: this CTA's own from
+// its staging rows, the partner's from the receive rows.
 template <int BN>
 struct PartRows {
-    const float* stage;
-    const float* recv;
-    int rank, rp;
+    const float* stage;   // this CTA's 128 accumulator rows
+    const float* recv;    // the partner's partials of the owned rows
+    int own0;             // first owned row within the CTA's 128
+    int half;             // this CTA's half of K
     __device__ __forceinline__ const float* row(int src, int lr) const {
         constexpr int RS = DecGeo<BN>::RS;
-        if (src == rank) return stage + (rank * rp + lr) * RS;
-        const int slot = src < rank ? src : src - 1;
-        return recv + (slot * rp + lr) * RS;
+        return src == half ? stage + (own0 + lr) * RS : recv + lr * RS;
     }
 };
 
@@ -212,28 +218,26 @@ template <int BN>
 struct KIn {
     static constexpr int NJ = (BN + 31) / 32;
     static constexpr int NW = kDecThreads / 32;
-    static constexpr int RPW = kDecRp / NW;   // rows per warp at most (8)
+    static constexpr int RPW = kOwnRows / NW;   // rows per warp (8)
     float hv[RPW][NJ];
-    __device__ __forceinline__ void load(const DecParams& p, int rank, int rp, int ct) {
+    __device__ __forceinline__ void load(const DecParams& p, int row0, int ct) {
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
-            const int lr = warp + NW * i, row = rank * rp + lr;
+            const int row = row0 + warp + NW * i;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
                 const int c = lane + 32 * j;
-                hv[i][j] = (lr < rp && row < p.n && c < BN)
-                               ? __bfloat162float(p.h[(int64_t)row * p.d + ct * BN + c])
-                               : 0.f;
+                hv[i][j] = (row < p.n && c < BN) ? __bfloat162float(p.h[(int64_t)row * p.d + ct * BN + c]) : 0.f;
             }
         }
     }
 };
 
-// Gate partials of the CTA's rows over its BN channels.
+// Gate partials of the CTA's owned rows over its BN channels.
 template <int BN>
 __device__ __forceinline__ void dec_epilogue_k(const DecParams& p, const PartRows<BN>& pr, const KIn<BN>& in,
-                                               const float* s_g, int rank, int rp, int ct) {
+                                               const float* s_g, int row0, int ct) {
     constexpr int NJ = KIn<BN>::NJ;
     constexpr int NW = KIn<BN>::NW;
     constexpr int RPW = KIn<BN>::RPW;
@@ -241,16 +245,14 @@ __device__ __forceinline__ void dec_epilogue_k(const DecParams& p, const PartRow
     const auto& hv = in.hv;
 #pragma unroll
     for (int i = 0; i < RPW; ++i) {
-        const int lr = warp + NW * i, row = rank * rp + lr;
-        if (lr >= rp || row >= p.n) break;
+        const int lr = warp + NW * i, row = row0 + lr;
+        if (row >= p.n) break;
         float s_qk = 0.f, s_kk = 0.f, s_hh = 0.f;
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
             const int c = lane + 32 * j;
             if (c < BN) {
-                float k = pr.row(0, lr)[c];
-#pragma unroll
-                for (int src = 1; src < kSplit; ++src) k += pr.row(src, lr)[c];
+                const float k = pr.row(0, lr)[c] + pr.row(1, lr)[c];
                 s_qk = fmaf(s_g[c] * hv[i][j], k, s_qk);
                 s_kk = fmaf(k, k, s_kk);
                 s_hh = fmaf(hv[i][j], hv[i][j], s_hh);
@@ -266,74 +268,67 @@ __device__ __forceinline__ void dec_epilogue_k(const DecParams& p, const PartRow
     }
 }
 
-// v of the CTA's rows over its BN channels: the four partials in rank order,
-// four channels per item, consecutive threads on consecutive channels
+// v of the CTA's owned rows over its BN channels: the two partials in K-half
+// order, four channels per item, consecutive threads on consecutive channels
 template <int BN>
-__device__ __forceinline__ void dec_write_v(const DecParams& p, const PartRows<BN>& pr, int rank, int rp, int ct) {
+__device__ __forceinline__ void dec_write_v(const DecParams& p, const PartRows<BN>& pr, int row0, int ct) {
     constexpr int NQ = BN / 4;
-    const int items = rp * NQ;
-    for (int it = threadIdx.x; it < items; it += kDecThreads) {
+    for (int it = threadIdx.x; it < kOwnRows * NQ; it += kDecThreads) {
         const int lr = it / NQ, q4 = it - lr * NQ;
-        const int row = rank * rp + lr;
+        const int row = row0 + lr;
         if (row >= p.n) break;
-        float4 v = *reinterpret_cast<const float4*>(pr.row(0, lr) + 4 * q4);
-#pragma unroll
-        for (int src = 1; src < kSplit; ++src) {
-            const float4 u = *reinterpret_cast<const float4*>(pr.row(src, lr) + 4 * q4);
-            v.x += u.x;
-            v.y += u.y;
-            v.z += u.z;
-            v.w += u.w;
-        }
-        *reinterpret_cast<float4*>(p.v + (int64_t)row * p.d + ct * BN + 4 * q4) = v;
+        const float4 a = *reinterpret_cast<const float4*>(pr.row(0, lr) + 4 * q4);
+        const float4 b = *reinterpret_cast<const float4*>(pr.row(1, lr) + 4 * q4);
+        *reinterpret_cast<float4*>(p.v + (int64_t)row * p.d + ct * BN + 4 * q4) =
+            make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
     }
 }
 
-// One accumulator pair (rows 0-127 and 128-255) into this CTA's staging
-// rows: warp w reads TMEM lanes 32 (w % 4) .. +31 and channel half w / 4,
-// one row per lane; the padded rows put the lanes' stores in distinct banks
+// One accumulator (this CTA's 128 rows) into its staging rows: warp w reads
+// TMEM lanes 32 (w % 4) .. +31 and channel half w / 4, one row per lane;
+// the padded rows put the lanes' stores in distinct banks
 template <int BN>
-__device__ __forceinline__ void stage_acc(uint32_t tmem, float* stage, int nr) {
+__device__ __forceinline__ void stage_acc(uint32_t tmem, float* stage) {
     constexpr int HALF = BN / 2;
     constexpr int NCH = HALF / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3, col0 = (warp >> 2) * HALF;
-    for (int rt = 0; rt < nr; ++rt) {
-        const int row = rt * 128 + q * 32 + lane;
-        uint32_t v[NCH][8];
+    const int row = q * 32 + lane;
+    uint32_t v[NCH][8];
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch)
-            tmem_ld8(tmem + (uint32_t)(rt * kRowTile + col0 + ch * 8) + ((uint32_t)(q * 32) << 16), v[ch]);
-        tmem_wait_ld();
-        uint4* dst = reinterpret_cast<uint4*>(stage + row * DecGeo<BN>::RS + col0);
+    for (int ch = 0; ch < NCH; ++ch)
+        tmem_ld8(tmem + (uint32_t)(col0 + ch * 8) + ((uint32_t)(q * 32) << 16), v[ch]);
+    tmem_wait_ld();
+    uint4* dst = reinterpret_cast<uint4*>(stage + row * DecGeo<BN>::RS + col0);
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) {
-            dst[2 * ch] = make_uint4(v[ch][0], v[ch][1], v[ch][2], v[ch][3]);
-            dst[2 * ch + 1] = make_uint4(v[ch][4], v[ch][5], v[ch][6], v[ch][7]);
-        }
+    for (int ch = 0; ch < NCH; ++ch) {
+        dst[2 * ch] = make_uint4(v[ch][0], v[ch][1], v[ch][2], v[ch][3]);
+        dst[2 * ch + 1] = make_uint4(v[ch][4], v[ch][5], v[ch][6], v[ch][7]);
     }
-    // the bulk copies read the staged rows through the async proxy
+    // the bulk copy reads the staged rows through the async proxy
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// one bulk copy per peer: the staged rows the peer owns (contiguous, padded)
-// into its receive slot for this rank
+// one bulk copy: the staged rows the partner owns (contiguous, padded) into
+// its receive rows (thread 0)
 template <int BN>
-__device__ __forceinline__ void send_partials(const DecParams& p, DecBarriers* sb, float* stage, float* recv, int rank,
-                                              int rp) {
+__device__ __forceinline__ void send_partials(DecBarriers* sb, float* stage, float* recv, int partner,
+                                              int partner_own0, int rows) {
     constexpr int RS = DecGeo<BN>::RS;
-    const int t = threadIdx.x;
-    if (t >= kSplit - 1) return;
-    const int o = t < rank ? t : t + 1;
-    const int rows = owned_rows(p.n, o, rp);
-    if (rows <= 0) return;
-    const int slot = rank < o ? rank : rank - 1;
-    bulk_s2cluster(peer_addr(recv + slot * rp * RS, (uint32_t)o), smem_u32(stage + o * rp * RS),
-                   (uint32_t)(rows * RS * 4), peer_addr(&sb->rfull, (uint32_t)o));
+    if (threadIdx.x != 0 || rows <= 0) return;
+    bulk_s2cluster(peer_addr(recv, (uint32_t)partner), smem_u32(stage + partner_own0 * RS), (uint32_t)(rows * RS * 4),
+                   peer_addr(&sb->rfull, (uint32_t)partner));
 }
 
+// Cluster of 4: rank 2h + m.  The pair {2h, 2h+1} multiplies the h-th half
+// of K with M = 256 tcgen05 MMAs issued by its leader (m = 0): CTA m stages
+// rows 128m .. 128m+127 of e and channels m BN/2 .. (m+1) BN/2 - 1 of the
+// tile's W_K and W_V, and its TMEM receives its 128 rows of k and v over all
+// BN channels.  CTA (h, m) owns rows 128m + 64h .. +63 and exchanges its
+// other 64 rows (k and v) with CTA (1-h, m), which holds the same rows from
+// the other half of K; two cluster barriers bracket the exchange.
 template <int BN>
-__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 1)
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kDecThreads, 1)
 decode_kv_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_bk,
                  const __grid_constant__ CUtensorMap map_bv, const DecParams p) {
     using GE = DecGeo<BN>;
@@ -345,20 +340,26 @@ decode_kv_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     float* s_g = reinterpret_cast<float*>(smem + GE::RING + 1024);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_rank();
-    const int ct = (int)blockIdx.x / kSplit;   // channel tile of the cluster
-    const int nr = p.n > 128 ? 2 : 1;          // 128-row accumulators in use
-    const int rp = nr * 128 / kSplit;          // rows owned by each CTA of the cluster
-    // this CTA's k-blocks (64 elements each)
+    const int half = rank >> 1, m = rank & 1;
+    const bool leader = m == 0;
+    const int lead_rank = rank & ~1;            // the pair's leader
+    const uint16_t pair_mask = (uint16_t)(3u << lead_rank);
+    const int partner = rank ^ 2;               // same rows, other half of K
+    const int ct = (int)blockIdx.x / kCluster;  // channel tile of the cluster
+    const int own0 = half * kOwnRows;           // first owned row within the CTA's 128
+    const int row0 = m * 128 + own0;            // first owned row
+    // this pair's k-blocks (64 elements each)
     const int kb_total = p.d_mem / 64;
-    const int kb0 = rank * kb_total / kSplit, kb1 = (rank + 1) * kb_total / kSplit;
+    const int kb0 = half * kb_total / 2, kb1 = (half + 1) * kb_total / 2;
     const int nkb = kb1 - kb0;
-    const int rot = nkb > 0 ? ct % nkb : 0;   // this cluster's first k-block (see the header)
-    const uint32_t stage_tx = (uint32_t)(nr * kABytes + 2 * GE::B_BYTES);
+    const int rot = nkb > 0 ? ct % nkb : 0;     // this cluster's first k-block (see the header)
+    const int w_row0 = ct * BN + m * GE::B_ROWS;   // this CTA's W rows
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(&sb->full[s], 1);
             mbar_init(&sb->empty[s], 1);
+            mbar_init(&sb->pfull[s], 1);
         }
         mbar_init(&sb->tfull, 1);
         mbar_init(&sb->rfull, 1);
@@ -373,34 +374,43 @@ decode_kv_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         tma_prefetch_desc(&map_bv);
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sb->tmem_base)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sb->tmem_base)),
                      "n"(kTmemCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    cluster_sync_all();   // every CTA's barriers are initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = sb->tmem_base;
 
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- TMA producer (each CTA loads its own rows and W half;
+        // the partner of a pair counts its stages on the leader's pfull)
         if (lane == 0) {
             const int pre = nkb < kDecStages ? nkb : kDecStages;
             auto kcol = [&](int j) { return (kb0 + (j + rot) % nkb) * 64; };
+            auto bar_of = [&](int s) {
+                return leader ? smem_u32(&sb->full[s]) : peer_addr(&sb->pfull[s], (uint32_t)lead_rank);
+            };
+            auto load = [&](const CUtensorMap* map, uint32_t dst, int s, int x, int y) {
+                if (leader) tma_load_2d(map, dst, &sb->full[s], x, y);
+                else tma_load_2d_peer_bar(map, dst, bar_of(s), x, y);
+            };
             auto load_w = [&](int j) {
                 const int s = j % kDecStages;
-                mbar_arrive_expect_tx(&sb->full[s], stage_tx);
+                if (leader) mbar_arrive_expect_tx(&sb->full[s], GE::STAGE_BYTES);
+                else mbar_arrive_expect_tx_remote(bar_of(s), GE::STAGE_BYTES);
                 if (p.stall && j == 0 && blockIdx.x == 0) return;   // bounded-wait test: never loaded
-                const uint32_t b = ring + s * GE::STAGE_BYTES + 2 * kABytes;
-                tma_load_2d(&map_bk, b, &sb->full[s], kcol(j), ct * BN);
-                tma_load_2d(&map_bv, b + GE::B_BYTES, &sb->full[s], kcol(j), ct * BN);
+                const uint32_t b = ring + s * GE::STAGE_BYTES + kABytes;
+                load(&map_bk, b, s, kcol(j), w_row0);
+                load(&map_bv, b + GE::B_BYTES, s, kcol(j), w_row0);
             };
             auto load_a = [&](int j) {
                 const int s = j % kDecStages;
                 if (p.stall && j == 0 && blockIdx.x == 0) return;
-                for (int rt = 0; rt < nr; ++rt)
-                    tma_load_2d(&map_a, ring + s * GE::STAGE_BYTES + rt * kABytes, &sb->full[s], kcol(j), rt * 128);
+                load(&map_a, ring + s * GE::STAGE_BYTES, s, kcol(j), m * 128);
             };
             // the weights do not depend on the retrieval: their first stages
             // stream while it finishes; e is read after it completes
@@ -418,37 +428,36 @@ decode_kv_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer: each A stage feeds k and v
-        if (lane == 0) {
+        // ---------------- MMA issuer (the pair's leader): each stage feeds k and v
+        if (lane == 0 && leader) {
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
                 const int s = j % kDecStages;
-                if (!dec_wait(&sb->full[s], (uint32_t)(j / kDecStages) & 1u, sb, p.status)) {
+                const uint32_t ph = (uint32_t)(j / kDecStages) & 1u;
+                if (!dec_wait(&sb->full[s], ph, sb, p.status) || !dec_wait(&sb->pfull[s], ph, sb, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t a_addr = ring + s * GE::STAGE_BYTES;
-                const uint64_t dbk = smem_desc_sw128(a_addr + 2 * kABytes);
-                const uint64_t dbv = smem_desc_sw128(a_addr + 2 * kABytes + GE::B_BYTES);
-                for (int rt = 0; rt < nr; ++rt) {
-                    const uint64_t da = smem_desc_sw128(a_addr + rt * kABytes);
+                const uint64_t da = smem_desc_sw128(a_addr);
+                const uint64_t dbk = smem_desc_sw128(a_addr + kABytes);
+                const uint64_t dbv = smem_desc_sw128(a_addr + kABytes + GE::B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        umma_bf16<BN>(tmem_base + (uint32_t)(kAccK + rt * kRowTile), da + (uint64_t)(kk * 2),
-                                      dbk + (uint64_t)(kk * 2), (j | kk) != 0);
-                        umma_bf16<BN>(tmem_base + (uint32_t)(kAccV + rt * kRowTile), da + (uint64_t)(kk * 2),
-                                      dbv + (uint64_t)(kk * 2), (j | kk) != 0);
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    umma_bf16_pair<BN>(tmem_base + kAccK, da + (uint64_t)(kk * 2), dbk + (uint64_t)(kk * 2),
+                                       (j | kk) != 0);
+                    umma_bf16_pair<BN>(tmem_base + kAccV, da + (uint64_t)(kk * 2), dbv + (uint64_t)(kk * 2),
+                                       (j | kk) != 0);
                 }
-                umma_commit(&sb->empty[s]);
+                umma_commit_pair_mask(&sb->empty[s], pair_mask);
                 sb->consumed = j + 1;
             }
-            if (ok) umma_commit(&sb->tfull);
+            if (ok) umma_commit_pair_mask(&sb->tfull, pair_mask);
         }
         __syncwarp();
     } else {
-        dec_prefetch<BN>(p, ct, kb0, nkb, s_g, threadIdx.x - 64, kDecThreads - 64);
+        dec_prefetch<BN>(p, ct, w_row0, kb0, nkb, s_g, threadIdx.x - 64, kDecThreads - 64);
     }
     // the conv kernel may launch once every thread of every CTA is past the
     // retrieval (warp 0 follows its lane 0, which waited above); its CTAs
@@ -456,78 +465,74 @@ decode_kv_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     if (warp != 0) grid_dep_wait();
     grid_dep_launch_dependents();
 
-    // ---------------- accumulators complete
+    // ---------------- accumulators complete (the leader's commits arrive in both CTAs)
     const bool ok = nkb > 0 && dec_wait(&sb->tfull, 0, sb, p.status);
     const int cta_abort = __syncthreads_or(!ok || sb->abort_flag);
     tc_fence_after();
-    float* stage = reinterpret_cast<float*>(smem + GE::STAGE_OFF);
-    float* recv = reinterpret_cast<float*>(smem + GE::RECV_OFF);
-    const PartRows<BN> pr{stage, recv, rank, rp};
-    const uint32_t rbytes = (uint32_t)((kSplit - 1) * owned_rows(p.n, rank, rp) * GE::RS * 4);
+    float* stage_k = reinterpret_cast<float*>(smem + GE::STAGE_K);
+    float* recv_k = reinterpret_cast<float*>(smem + GE::RECV_K);
+    float* stage_v = reinterpret_cast<float*>(smem + GE::STAGE_V);
+    float* recv_v = reinterpret_cast<float*>(smem + GE::RECV_V);
+    const PartRows<BN> pk{stage_k, recv_k, own0, half}, pv{stage_v, recv_v, own0, half};
+    const int partner_own0 = (1 - half) * kOwnRows;
+    const int send_rows = live_rows(p.n, m * 128 + partner_own0);
+    const uint32_t rbytes = (uint32_t)(live_rows(p.n, row0) * GE::RS * 4);
 
-    // ---- k: stage, exchange, gate partials and alpha
-    if (!cta_abort) stage_acc<BN>(tmem_base + kAccK, stage, nr);
+    // ---- k and v: stage both, one exchange
+    if (!cta_abort) {
+        stage_acc<BN>(tmem_base + kAccK, stage_k);
+        stage_acc<BN>(tmem_base + kAccV, stage_v);
+    }
     if (threadIdx.x == 0) {
         sb->abort_flag = cta_abort;
-        mbar_arrive_expect_tx(&sb->rfull, rbytes);   // phase 0: the peers' k rows
+        mbar_arrive_expect_tx(&sb->rfull, 2 * rbytes);   // the partner's k and v rows
     }
     tc_fence_before();
     // barrier 1: every CTA's MMAs have finished reading its ring, which now
-    // receives the peers' partials; the abort votes are visible cluster-wide
+    // receives the partner's partials; the abort votes are visible cluster-wide
     __syncwarp();
     cluster_sync_all();
     int any_abort = 0;
 #pragma unroll
-    for (int r = 0; r < kSplit; ++r) any_abort |= ld_remote_s32(peer_addr(&sb->abort_flag, (uint32_t)r));
+    for (int r = 0; r < kCluster; ++r) any_abort |= ld_remote_s32(peer_addr(&sb->abort_flag, (uint32_t)r));
+    if (!any_abort) {
+        send_partials<BN>(sb, stage_k, recv_k, partner, partner_own0, send_rows);
+        send_partials<BN>(sb, stage_v, recv_v, partner, partner_own0, send_rows);
+    }
     // h of the owned rows, in flight during the exchange (issued after the
     // barrier, whose release would otherwise wait for the loads)
     KIn<BN> kin;
-    kin.load(p, rank, rp, ct);
-    bool have = false;
-    if (!any_abort) {
-        send_partials<BN>(p, sb, stage, recv, rank, rp);
-        have = dec_wait(&sb->rfull, 0, sb, p.status);
-    }
-    // barrier 2: every k copy has landed, so no CTA's staged rows are read any more
+    kin.load(p, row0, ct);
+    const bool have = !any_abort && dec_wait(&sb->rfull, 0, sb, p.status);
+    // barrier 2: every copy has landed, so no CTA's staged rows are read any more
     __syncwarp();
     cluster_sync_all();
-    const bool go = !any_abort && __syncthreads_and(have);
-    if (go) dec_epilogue_k<BN>(p, pr, kin, s_g, rank, rp, ct);
-    __syncthreads();   // the k rows are read: the ring takes v
-
-    // ---- v: stage, exchange, write
-    if (go) {
-        stage_acc<BN>(tmem_base + kAccV, stage, nr);
-        if (threadIdx.x == 0) mbar_arrive_expect_tx(&sb->rfull, rbytes);   // phase 1: the peers' v rows
-    }
-    tc_fence_before();
-    // barrier 3: every CTA has read its k rows, so the receive slots are free
-    __syncwarp();
-    cluster_sync_all();
-    bool have_v = false;
-    if (go) {
-        send_partials<BN>(p, sb, stage, recv, rank, rp);
-        have_v = dec_wait(&sb->rfull, 1, sb, p.status);
-    }
-    // barrier 4: every v copy has landed
-    __syncwarp();
-    cluster_sync_all();
-    if (go && __syncthreads_and(have_v)) {
-        dec_write_v<BN>(p, pr, rank, rp, ct);
-    } else if (cta_abort) {
-        // this CTA stopped early: wait out the copies and MMAs it issued
-        if (warp == 0 && lane == 0)
+    if (!any_abort && __syncthreads_and(have)) {
+        dec_epilogue_k<BN>(p, pk, kin, s_g, row0, ct);
+        dec_write_v<BN>(p, pv, row0, ct);
+    } else if (any_abort && leader) {
+        // the pair stopped early: the leader waits out every stage either CTA
+        // of the pair issued (the partner's complete on its pfull), then its MMAs
+        if (warp == 0 && lane == 0) {
             for (int j = sb->consumed; j < sb->issued; ++j)
                 dec_wait_drain(&sb->full[j % kDecStages], (uint32_t)(j / kDecStages) & 1u);
+            const int peer_issued = ld_remote_s32(peer_addr(&sb->issued, (uint32_t)(rank + 1)));
+            for (int j = sb->consumed; j < peer_issued; ++j)
+                dec_wait_drain(&sb->pfull[j % kDecStages], (uint32_t)(j / kDecStages) & 1u);
+        }
         if (warp == 1 && lane == 0) {
-            umma_commit(&sb->drain);
+            umma_commit_pair_local(&sb->drain);
             dec_wait_drain(&sb->drain, 0);
         }
     }
     __syncthreads();
+    // the cluster leaves together: no copy or MMA of a pair is in flight
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "n"(kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "n"(kTmemCols)
                      : "memory");
     }
 }
@@ -624,7 +629,7 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const ConvPar
 
 // ---------------------------------------------------------------- host side
 
-// clusters of kSplit CTAs of the decode kernel that the device holds at once
+// clusters of kCluster CTAs of the decode kernel that the device holds at once
 int resident_clusters(int num_sms) {
     static int cached[64] = {};
     int dev = 0;
@@ -635,13 +640,13 @@ int resident_clusters(int num_sms) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DecGeo<80>::SMEM_BYTES) ==
         cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(num_sms / kSplit * kSplit), 1, 1);
+        cfg.gridDim = dim3((unsigned)(num_sms / kCluster * kCluster), 1, 1);
         cfg.blockDim = dim3(kDecThreads, 1, 1);
         cfg.dynamicSmemBytes = DecGeo<80>::SMEM_BYTES;
         if (cudaOccupancyMaxActiveClusters(&mc, kernel, &cfg) != cudaSuccess) mc = 0;
     }
     cudaGetLastError();
-    if (mc < 1) mc = num_sms / kSplit;
+    if (mc < 1) mc = num_sms / kCluster;
     if (dev < 64) cached[dev] = mc;
     return mc;
 }
@@ -671,7 +676,7 @@ cudaError_t launch_kv(const CUtensorMap& ma, const CUtensorMap& mk, const CUtens
     p.n_ct = p.d / BN;
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.n_ct * kSplit), 1, 1);
+    cfg.gridDim = dim3((unsigned)(p.n_ct * kCluster), 1, 1);
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = DecGeo<BN>::SMEM_BYTES;
     cfg.stream = s;
@@ -689,7 +694,7 @@ cudaError_t launch_kv(const CUtensorMap& ma, const CUtensorMap& mk, const CUtens
 
 bool decode_tc_supported(int64_t n, int32_t L, int32_t d_mem, int32_t d, int32_t M, bool f8) {
     return L == 1 && n >= 1 && n <= kDecRows && M == 1 && !f8 && d % 64 == 0 && d_mem % 64 == 0 &&
-           d_mem / 64 >= kSplit && encode_fn() != nullptr;
+           d_mem / 64 >= 2 && encode_fn() != nullptr;
 }
 
 int32_t decode_tc_max_tiles(int32_t d) { return d / 64; }
@@ -700,8 +705,10 @@ cudaError_t launch_decode_kv(const void* e, int32_t n, int32_t d_mem, const void
     if (!decode_tc_supported(n, 1, d_mem, d, 1, false)) return cudaErrorNotSupported;
     const int bn = pick_dec_bn(d, num_sms);
     CUtensorMap ma, mk, mv;
-    if (!make_map(&ma, e, (uint64_t)n, (uint64_t)d_mem, 128) || !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn) ||
-        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn))
+    // each CTA of a pair stages half of the tile's W rows
+    if (!make_map(&ma, e, (uint64_t)n, (uint64_t)d_mem, 128) ||
+        !make_map(&mk, Wk, (uint64_t)d, (uint64_t)d_mem, bn / 2) ||
+        !make_map(&mv, Wv, (uint64_t)d, (uint64_t)d_mem, bn / 2))
         return cudaErrorInvalidValue;
     DecParams p{};
     p.wk = static_cast<const __nv_bfloat16*>(Wk);

@@ -114,6 +114,15 @@ __device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
         : "memory");
 }
 
+// the same for a pair anywhere in a larger cluster: arrive on the barrier at
+// the same offset in the CTAs whose ranks are set in `mask` (the pair's two)
+__device__ __forceinline__ void umma_commit_pair_mask(uint64_t* bar, uint16_t mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(smem_u32(bar)), "h"(mask)
+        : "memory");
+}
+
 // arrive on this CTA's barrier once the pair's earlier MMAs complete
 __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
