@@ -209,11 +209,14 @@ CAPTURED_TRAFFIC = {
     ("c3-B2-M499979", "vconv_tc"): ("59d2794a31cc0db6", 86297856 + 2050304),
     ("c3-B2-M499979", "gate_k_tc"): ("59d2794a31cc0db6", 86043136 + 130048),
     ("c3-B2-M499979", "retrieve"): ("8c46903b0c8d286e", 29667072 + 480512),
-    # c3 at full size, mean of the five timed steps' launches (profiles/launches_c3.md)
-    ("c3", "vconv_tc"): ("9ab3e6fa4d60f677", 314986291 + 123705805),
-    ("c3", "gate_k_tc"): ("9ab3e6fa4d60f677", 312567296 + 7406336),
-    ("c3", "retrieve"): ("466e8ddd712470f7", 115578931 + 81197158),
-    ("c4", "retrieve"): ("466e8ddd712470f7", 1207296 + 307),
+    # c3 and c4 at full size, mean of the five timed steps' launches
+    # (profiles/launches_c3.md, profiles/launches_c4.md)
+    ("c3", "vconv_tc"): ("6d29d9cc97972e11", 314932326 + 123619072),
+    ("c3", "gate_k_tc"): ("6d29d9cc97972e11", 312567450 + 7093248),
+    ("c3", "retrieve"): ("cd4c38c473a10c27", 115572480 + 81451725),
+    ("c4", "retrieve"): ("cd4c38c473a10c27", 1209139 + 2867),
+    ("c4", "gate_kv_decode"): ("6bc5ef79605ad072", 23401165 + 0),
+    ("c4", "conv_decode"): ("6bc5ef79605ad072", 11986534 + 0),
 }
 
 

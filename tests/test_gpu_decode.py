@@ -1,14 +1,16 @@
 """The decode path (one new position per sequence, at most 256 sequences,
-bf16) against the oracle, through engram_forward.
+bf16) against the oracle, through engram_forward and engram_gate_conv.
 
-These calls run the decode kernels: both projections in one cluster split-K
-kernel (partial sums added through distributed shared memory, the gate's row
-sums across clusters), then the conv kernel, which reads and rewrites the
-conv state in place.  Covered: one and two 128-row accumulators (1 to 256
-sequences, ragged), both channel tile widths (64 channels: d = 256, 384, 512;
-80 channels: d = 2560 on a full B200), K extents that split evenly and
-unevenly over the four CTAs of a cluster, with and without conv state and
-residual, bitwise determinism, and dependent against plain launches."""
+These calls run the decode kernels after the retrieval: both projections in
+one cluster kernel (the two halves of K on two CTA pairs, partial sums added
+through distributed shared memory, the gate's row sums across clusters),
+then the conv kernel, which reads and rewrites the conv state in place.
+Covered: one and two 128-row accumulators (1 to 256 sequences, ragged), both
+channel tile widths (64 channels: d = 256, 384, 512; 80 channels: d = 2560
+on a full B200), K extents that split evenly and unevenly over the two
+pairs, the indices, invalid ids (zero rows), engram_gate_conv on e, with and
+without conv state and residual, bitwise determinism, and dependent against
+plain launches."""
 
 import numpy as np
 import pytest
@@ -81,6 +83,11 @@ def test_decode_matches_oracle(eb, name, with_state):
     y, alpha = _decode(eb, ctx, di, state, add_residual)
     assert ctx.status() == (eb.ENGRAM_OK, 0)
     ref = oracle.forward_rows(inp, np.arange(wl.n_tok), add_residual=add_residual, hist=hist)
+    # the indices of the computed position, bit-exact
+    canon, _ = oracle.remap(inp.tok, inp.P)
+    idx_ref, _ = oracle.hash_ids(canon, wl.Vc, wl.orders, wl.K, inp.mult, inp.rows, wl.t_begin)
+    idx = ctx.workspace[: wl.n_tok * wl.J * 4].view(torch.int32).view(wl.n_tok, wl.J)
+    assert np.array_equal(idx.cpu().numpy().view(np.uint32), idx_ref)
     np.testing.assert_allclose(to_np(alpha), ref.alpha, rtol=0, atol=2e-6)
     err = np.abs(to_np(y) - ref.y)
     assert err.max() <= 2e-2, err.max()
@@ -103,6 +110,71 @@ def test_decode_runs_the_decode_kernels(eb):
     names = _kernels(eb, ctx, di, state)
     # no history transpose and no merge: the conv kernel rewrites the state in place
     assert names == ["retrieve", "gate_kv_decode", "conv_decode"], names
+
+
+def test_decode_invalid_ids_read_zero_rows(eb):
+    """Ids outside the vocabulary in the n-gram windows of some sequences:
+    every order whose window holds one reads zero rows and the status word
+    says ENGRAM_ERR_TOKEN."""
+    wl = CASES["n200_d2560"]
+    inp = synth.Inputs(wl, gamma="random")
+    t = wl.t_begin
+    inp.tok[3, t] = wl.V + 5        # every order of sequence 3
+    inp.tok[7, t - 1] = -3          # both orders of sequence 7
+    inp.tok[9, t - 2] = wl.V        # order 3 only (tables 8-15, the second half of K)
+    inp.tok[150, t - 2] = -1        # the same in the second 128-row block
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    state = inp.device_state("cuda:0").contiguous()
+    hist = inp.state_rows(np.arange(wl.B))
+    y, alpha = _decode(eb, ctx, di, state, True)
+    st, flags = ctx.status()
+    assert flags == eb.ENGRAM_ERR_TOKEN, (st, flags)
+    ref = oracle.forward_rows(inp, np.arange(wl.n_tok), add_residual=True, hist=hist)
+    np.testing.assert_allclose(to_np(alpha), ref.alpha, rtol=0, atol=2e-6)
+    err = np.abs(to_np(y) - ref.y)
+    bad = err > bf16_bound(ref.y, ref.vt_win, inp.conv_w)
+    assert not bad.any(), (int(bad.sum()), float(err.max()))
+    idx = ctx.workspace[: wl.n_tok * wl.J * 4].view(torch.int32).view(wl.n_tok, wl.J).cpu().numpy().view(np.uint32)
+    assert (idx[3] == eb.ENGRAM_INVALID_INDEX).all() and (idx[7] == eb.ENGRAM_INVALID_INDEX).all()
+    assert (idx[9, : wl.K] != eb.ENGRAM_INVALID_INDEX).all() and (idx[9, wl.K:] == eb.ENGRAM_INVALID_INDEX).all()
+
+
+@pytest.mark.parametrize("name", ["n200_d2560", "n5_d256"])
+def test_gate_conv_decode_from_e(eb, name):
+    """engram_gate_conv on one position per sequence runs the same decode
+    kernels on the caller's e (here made on the device by engram_hash and
+    engram_gather)."""
+    wl = CASES[name]
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    n = wl.n_tok
+    idx = torch.empty(n, wl.J, dtype=torch.int32, device="cuda")
+    eb.engram_hash(ctx.ctx, di.tok, di.P, wl.B, wl.T, wl.T, wl.t_begin, idx)
+    e = torch.empty(n, wl.J * wl.D, dtype=torch.bfloat16, device="cuda")
+    eb.engram_gather(ctx.ctx, idx, n, di.tables, e)
+    ws_bytes = eb.engram_workspace_bytes(ctx.ctx, wl.B, 1)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    state = inp.device_state("cuda:0").contiguous()
+    hist = inp.state_rows(np.arange(wl.B))
+    y = di.empty_y()
+    alpha = torch.empty(n, dtype=torch.float32, device="cuda")
+    eb.engram_profile_enable(ctx.ctx, True)
+    try:
+        eb.engram_gate_conv(ctx.ctx, e, di.h, di.Wk, di.Wv, di.gq, di.gk, di.conv_w, wl.B, 1, state, y, alpha, 1,
+                            ws, ws_bytes)
+        torch.cuda.synchronize()
+        names = [nm for nm, _ in eb.engram_profile_read(ctx.ctx)]
+    finally:
+        eb.engram_profile_enable(ctx.ctx, False)
+    assert names == ["gate_kv_decode", "conv_decode"], names
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    ref = oracle.forward_rows(inp, np.arange(n), add_residual=True, hist=hist)
+    np.testing.assert_allclose(to_np(alpha), ref.alpha, rtol=0, atol=2e-6)
+    err = np.abs(to_np(y) - ref.y)
+    bad = err > bf16_bound(ref.y, ref.vt_win, inp.conv_w)
+    assert not bad.any(), (int(bad.sum()), float(err.max()))
 
 
 def test_decode_without_gains(eb):
