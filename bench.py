@@ -201,10 +201,10 @@ KERNEL_SOURCES = {
 }
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
-    # c2, before the value epilogue's conv math moved to fp32 (profiles/launches_c2.md)
-    ("c2", "vconv_tc"): ("ece15e492f5dcb2f", 123190528 + 28159232),
-    ("c2", "gate_k_tc"): ("ece15e492f5dcb2f", 122743552 + 86016),
-    ("c2", "retrieve"): ("8c46903b0c8d286e", 28940800 + 632832),
+    # c2 at full size, mean of the five timed steps' launches (profiles/launches_c2.md)
+    ("c2", "vconv_tc"): ("6d29d9cc97972e11", 123251354 + 28427930),
+    ("c2", "gate_k_tc"): ("6d29d9cc97972e11", 122761472 + 378829),
+    ("c2", "retrieve"): ("cd4c38c473a10c27", 28944845 + 151552),
     # c3 kernels on 2 sequences and 499979-row tables (profiles/dram_c3_small.md)
     ("c3-B2-M499979", "vconv_tc"): ("59d2794a31cc0db6", 86297856 + 2050304),
     ("c3-B2-M499979", "gate_k_tc"): ("59d2794a31cc0db6", 86043136 + 130048),
