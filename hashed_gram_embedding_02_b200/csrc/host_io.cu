@@ -11,6 +11,13 @@
 // The conv history crosses chunk boundaries through conv_state (the caller's,
 // or a zeroed one in the workspace), exactly as a decode step continues a
 // prefill.
+//
+// Chunk sizes (chunk_rows = 0): a long batch runs 16 MiB chunks of h, whose
+// compute is short next to their copies, so the copies run back to back;
+// the first three chunks grow from 2 to 8 MiB and the last three shrink
+// again, so that the first compute starts early and the last copy out is
+// short.  A batch under four 16 MiB chunks runs uniform chunks of about
+// 4 MiB.  chunk_rows > 0 fixes uniform chunks of that many positions.
 #include <algorithm>
 
 #include "ctx.cuh"
@@ -18,7 +25,9 @@
 namespace engram {
 namespace {
 
-constexpr size_t kDefaultChunkBytes = 4u << 20;   // h bytes per chunk when chunk_rows = 0 (c2 sweep: 4 MiB best)
+constexpr size_t kShortChunkBytes = 4u << 20;   // h bytes per uniform chunk when chunk_rows = 0 (short batches)
+constexpr size_t kLongChunkBytes = 16u << 20;   // h bytes per middle chunk of a long batch
+constexpr int kRamp = 3;                        // chunks of 1/8, 1/4, 1/2 the middle size at each end
 
 enum IoEvent { EV_START = 0, EV_H_READY = 1, EV_COMPUTED = 3, EV_DRAINED = 5, EV_DONE = 7 };
 static_assert(EV_DONE < kIoEvents, "event slots");
@@ -26,7 +35,11 @@ static_assert(EV_DONE < kIoEvents, "event slots");
 struct HostPlan {
     int32_t lo;          // first id position copied per sequence
     int32_t Tw;          // ids copied per sequence (T - lo)
-    int32_t R;           // positions per chunk
+    int32_t R;           // positions per chunk at most (the buffers' size)
+    int32_t n_ramp;      // ramp chunks at each end (0: uniform chunks of R)
+    int32_t ramp_rows;   // positions in the chunks of one ramp
+    int32_t n_mid;       // middle chunks, each of R positions but the last
+    int32_t mid_rows;    // positions in the middle chunks
     int32_t n_chunks;
     size_t row_bytes;    // one position of h or Y
     size_t tok_off, state_off, h_off[2], y_off[2], fwd_off;
@@ -39,11 +52,22 @@ HostPlan make_plan(const engram_ctx* c, int32_t B, int32_t T, int32_t t_begin, i
     p.lo = std::max(0, t_begin - (c->hp.max_order - 1));
     p.Tw = T - p.lo;
     p.row_bytes = (size_t)c->cfg.hidden * c->hs;
+    const size_t seq_row = std::max<size_t>(1, (size_t)B * p.row_bytes);   // one position of every sequence
     int64_t R = chunk_rows;
-    if (R <= 0) R = (int64_t)std::max<size_t>(1, kDefaultChunkBytes / std::max<size_t>(1, (size_t)B * p.row_bytes));
+    const int64_t R_long = (int64_t)std::max<size_t>(1, kLongChunkBytes / seq_row);
+    if (R <= 0 && R_long >= 8 && (int64_t)L >= 4 * R_long) {
+        // ramp up, 16 MiB chunks, ramp down
+        R = R_long;
+        p.n_ramp = kRamp;
+        for (int i = 0; i < kRamp; ++i) p.ramp_rows += (int32_t)(R >> (kRamp - i));
+    } else if (R <= 0) {
+        R = (int64_t)std::max<size_t>(1, kShortChunkBytes / seq_row);
+    }
     R = std::min<int64_t>(R, std::max(L, 1));
     p.R = (int32_t)R;
-    p.n_chunks = L > 0 ? (int32_t)((L + R - 1) / R) : 0;
+    p.mid_rows = L - 2 * p.ramp_rows;
+    p.n_mid = p.mid_rows > 0 ? (int32_t)((p.mid_rows + R - 1) / R) : 0;
+    p.n_chunks = L > 0 ? p.n_mid + 2 * p.n_ramp : 0;
     const size_t chunk_bytes = (size_t)B * R * p.row_bytes;
     size_t off = 0;
     p.tok_off = off;
@@ -63,6 +87,28 @@ HostPlan make_plan(const engram_ctx* c, int32_t B, int32_t T, int32_t t_begin, i
     off += carve(c, nullptr, B, R, true).bytes;
     p.bytes = off;
     return p;
+}
+
+// positions [*r0, *r0 + *rc) of chunk ci
+void chunk_of(const HostPlan& p, int32_t ci, int32_t* r0, int32_t* rc) {
+    if (ci < p.n_ramp) {   // growing: R/8, R/4, R/2
+        int32_t o = 0;
+        for (int i = 0; i < ci; ++i) o += p.R >> (p.n_ramp - i);
+        *r0 = o;
+        *rc = p.R >> (p.n_ramp - ci);
+        return;
+    }
+    const int32_t j = ci - p.n_ramp;
+    if (j < p.n_mid) {
+        *r0 = p.ramp_rows + j * p.R;
+        *rc = std::min(p.R, p.mid_rows - j * p.R);
+        return;
+    }
+    const int32_t k = j - p.n_mid;   // shrinking: R/2, R/4, R/8
+    int32_t o = p.ramp_rows + p.mid_rows;
+    for (int i = 0; i < k; ++i) o += p.R >> (i + 1);
+    *r0 = o;
+    *rc = p.R >> (k + 1);
 }
 
 }  // namespace
@@ -130,8 +176,8 @@ engram_status engram_forward_host(engram_ctx* c, const int32_t* tok_host, int32_
 
     for (int32_t ci = 0; ci < p.n_chunks; ++ci) {
         const int b = ci & 1;
-        const int32_t r0 = ci * p.R;
-        const int32_t rc = std::min(p.R, L - r0);
+        int32_t r0 = 0, rc = 0;
+        chunk_of(p, ci, &r0, &rc);
         const size_t width = (size_t)rc * p.row_bytes;
         char* h_d = base + p.h_off[b];
         char* y_d = base + p.y_off[b];

@@ -422,7 +422,10 @@ ENGRAM_API engram_status engram_forward_noalloc(engram_ctx* ctx, const int32_t* 
  *   P, tables, Wk, Wv, gq, gk, conv_w, conv_state: device memory, as in
  *             engram_forward (conv_state nullable: zero history).
  * The rows are processed in chunks of `chunk_rows` positions of every
- * sequence (0: about 4 MiB of h per chunk).  While chunk i computes on
+ * sequence.  With chunk_rows = 0, a batch of at least four 16 MiB chunks of
+ * h runs 16 MiB chunks, entered and left through chunks of 2, 4 and 8 MiB
+ * (the first compute starts early, the last copy out is short); a shorter
+ * batch runs chunks of about 4 MiB.  While chunk i computes on
  * `stream`, the h of chunk i+1 is copied in on one of the context's copy
  * streams and the Y of chunk i-1 is copied out on the other
  * (cudaMemcpy2DAsync).  The conv history passes from chunk to chunk through

@@ -62,6 +62,30 @@ def test_host_forward_matches_oracle(eb, wl, chunk_rows):
     _check(wl, y_h.double().numpy(), ref.y, win, inp.conv_w)
 
 
+def test_host_forward_ramped_chunks_match_oracle(eb):
+    """A batch long enough for the default schedule's ramp (16 sequences of
+    1000 positions, d = 2560: 16 MiB middle chunks of 204 positions, ends of
+    25, 51 and 102): rows at and next to every chunk boundary match the
+    oracle, and the workspace is the one of 204-position chunks."""
+    wl = W["c2"].replace(name="ramp", B=16, T=1000, M=10007, seed=15)
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    assert (eb.engram_host_workspace_bytes(ctx.ctx, wl.B, wl.T, 0, 0)
+            == eb.engram_host_workspace_bytes(ctx.ctx, wl.B, wl.T, 0, 204))
+    y_h = torch.full((wl.n_tok, wl.d), float("nan"), dtype=di.dtype).pin_memory()
+    ctx.forward_host(_host(di.tok, True), di.P, di.tables, _host(di.h, True), di.Wk, di.Wv, di.conv_w, y_h,
+                     gq=di.gq, gk=di.gk, add_residual=True)
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    assert not torch.isnan(y_h.float()).any()
+    bounds = [0, 25, 76, 178, 382, 586, 790, 822, 924, 975]
+    ts = sorted({t for b0 in bounds for t in (b0 - 1, b0, b0 + 1, b0 + 2, b0 + 3) if 0 <= t < wl.T})
+    pos = np.array([b * wl.T + t for b in (0, 7, 15) for t in ts], dtype=np.int64)
+    ref = oracle.forward_rows(inp, pos, add_residual=True)
+    _check(wl, y_h[torch.from_numpy(pos)].double().numpy(), ref.y, ref.vt_win, inp.conv_w)
+
+
 def test_host_forward_pageable_equals_pinned(eb):
     wl = B3
     inp = synth.Inputs(wl)
