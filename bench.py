@@ -542,29 +542,52 @@ def e2e_host(args, eng, inp, dd, tables, h, state, wl, tdt, es, n, K, flush, str
     """The same step end to end through the C ABI with HOST buffers:
     engram_forward_host copies the ids and h in from pinned host memory and Y
     back out, chunk by chunk, overlapped with the compute; all of it inside
-    the events."""
+    the events.  Timed as eager calls and as replays of a CUDA graph that
+    captured one call (its copies are graph nodes that run again on every
+    replay, from and to the same pinned buffers); `value` is the graph
+    replay unless the capture failed, as for the device-time figure."""
     import torch
     tok_h = torch.from_numpy(inp.tok).pin_memory()
     h_h = h.cpu().pin_memory()
     y_h = torch.empty(n, wl.d, dtype=tdt).pin_memory()
     Ke = max(3, min(K, 50))
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
-    for i in range(Ke + 3):
-        flush()
-        if i >= 3:
-            e2e_ev[i - 3][0].record(stream)
+
+    def call():
         eng.forward_host(tok_h, dd["P"], tables, h_h, dd["Wk"], dd["Wv"], dd["conv_w"], y_h, t_begin=wl.t_begin,
                          gq=dd["gq"], gk=dd["gk"], conv_state=state, add_residual=True)
-        if i >= 3:
-            e2e_ev[i - 3][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])), world, dev)
+
+    def timed(run):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+        for i in range(Ke + 3):
+            flush()
+            if i >= 3:
+                ev[i - 3][0].record(stream)
+            run()
+            if i >= 3:
+                ev[i - 3][1].record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev])), world, dev)
+
+    eager_ms = timed(call)
+    graph_ms, path = None, "eager calls"
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call()
+            torch.cuda.synchronize()
+            graph_ms, path = timed(g.replay), "replays of a CUDA graph of one call"
+        except Exception as exc:                      # capture unsupported: the eager figure stands
+            torch.cuda.synchronize()
+            path = f"eager calls (graph capture failed: {type(exc).__name__})"
+    e2e_ms = graph_ms if graph_ms is not None else eager_ms
     ids_copied = wl.B * (wl.T - max(0, wl.t_begin - (max(wl.orders) - 1)))
     e2e = {"value": job_tokens_per_s(n, world, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": int(ids_copied * 4 + h_h.numel() * es),
            "d2h_bytes_per_step": int(y_h.numel() * es), "ms_per_step": e2e_ms,
-           "path": "engram_forward_host: pinned host ids + h in, Y out to pinned host, chunked and overlapped"}
-
+           "eager": {"value": job_tokens_per_s(n, world, eager_ms), "ms_per_step": eager_ms},
+           "path": "engram_forward_host: pinned host ids + h in, Y out to pinned host, chunked and overlapped; "
+                   + path}
     return e2e
 
 
