@@ -1,6 +1,7 @@
-"""engram_forward captured into a CUDA graph: a replay gives the same bits as
-an eager call, for a prefill and for a decode step (whose conv state the
-replay updates in place, as the eager call does)."""
+"""engram_forward and engram_forward_host captured into a CUDA graph: a replay
+gives the same bits as an eager call, for a prefill and for a decode step
+(whose conv state the replay updates in place, as the eager call does); the
+host-buffer call's copies replay from and to the same pinned buffers."""
 
 import numpy as np
 import pytest
@@ -105,3 +106,43 @@ def test_profile_events_inside_a_graph(eb):
     step()                                   # an eager call after the graph
     torch.cuda.synchronize()
     assert ctx.status() == (eb.ENGRAM_OK, 0)
+
+
+@pytest.mark.parametrize("name,chunk_rows", [("prefill", 0), ("prefill", 50), ("decode", 0)])
+def test_host_forward_graph_replay_matches_eager(eb, name, chunk_rows):
+    wl = CASES[name]
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb), B=wl.B, L=wl.T - wl.t_begin)
+    s0 = inp.device_state("cuda:0").contiguous() if wl.t_begin > 0 else None
+    state = s0.clone() if s0 is not None else None
+    tok_h = di.tok.cpu().contiguous().pin_memory()
+    h_h = di.h.cpu().contiguous().pin_memory()
+    y_h = torch.empty(wl.n_tok, wl.d, dtype=di.dtype).pin_memory()
+
+    def step():
+        ctx.forward_host(tok_h, di.P, di.tables, h_h, di.Wk, di.Wv, di.conv_w, y_h, t_begin=wl.t_begin, gq=di.gq,
+                         gk=di.gk, conv_state=state, add_residual=True, chunk_rows=chunk_rows)
+
+    step()
+    torch.cuda.synchronize()
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    y_eager = y_h.clone()
+    st_eager = state.clone() if state is not None else None
+    g = torch.cuda.CUDAGraph()
+    if state is not None:
+        state.copy_(s0)
+    with torch.cuda.graph(g):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(2):
+        if state is not None:
+            state.copy_(s0)
+        y_h.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert ctx.status() == (eb.ENGRAM_OK, 0)
+        assert torch.equal(y_h, y_eager)
+        if state is not None:
+            assert torch.equal(state, st_eager)
+    del g
