@@ -73,6 +73,12 @@ constexpr int CONV_W = 4;               // conv width of the fused epilogue
 constexpr int SEG = 32;                 // rows per epilogue warp
 constexpr int SEG_OUT = SEG - (CONV_W - 1);   // output rows per warp segment (29)
 constexpr int TILE_OUT = 4 * SEG_OUT;         // output rows per value tile (116)
+// The value pass on CTA pairs reads each CTA's 128 rows as one contiguous
+// block (3 history rows, then 125 output rows); a warp's first three rows
+// take their conv history from the previous warp's last three (halo slots
+// in shared memory)
+constexpr int TILE_OUT_C = BM - (CONV_W - 1);   // output rows per contiguous value tile (125)
+constexpr int HALO_SLOTS = 4;                   // (tile parity, channel half)
 
 // PAIR: a cluster of two CTAs runs one M = 256 tcgen05 MMA (cta_group::2);
 // each CTA stages its own 128 rows of A and half of the BN columns of W, so a
@@ -91,9 +97,16 @@ struct Geo {
     // partial hand-over [NPART][128] float4 | slack
     // MODE_VCONV: the gains area and the partial hand-over together hold the
     // epilogue warps' fp32 taps, 16 warps x 2 phases x BN/16 pairs x 32 bytes
+    // MODE_VCONV on pairs (contiguous tiles): the warps stage the taps of one
+    // phase at a time (16 warps x BN/16 pairs x 32 bytes, the gains area
+    // alone), and the halo slots follow:
+    // [slot][warp q < 3][part][3 rows][BN/8 channels] fp32
+    static constexpr bool CONTIG = MODE == MODE_VCONV && PAIR;
     static constexpr int GG_BYTES = MODE == MODE_VCONV ? BN * 32 : BN * 16;
-    static constexpr int RED_BYTES = NPART * BM * 16;
-    static constexpr int SMEM_BYTES = SMEM_TILES + H_BYTES + 1024 + GG_BYTES + RED_BYTES + 1024;
+    static constexpr int RED_BYTES = CONTIG ? 0 : NPART * BM * 16;
+    static constexpr int HALO_PW = BN / (2 * NPART);   // channels of one part in one phase
+    static constexpr int HALO_BYTES = CONTIG ? HALO_SLOTS * 3 * NPART * 3 * HALO_PW * 4 : 0;
+    static constexpr int SMEM_BYTES = SMEM_TILES + H_BYTES + 1024 + GG_BYTES + RED_BYTES + HALO_BYTES + 1024;
 };
 
 struct __align__(8) Barriers {
@@ -107,6 +120,7 @@ struct __align__(8) Barriers {
     uint64_t hfull_v[2];    // MODE_VCONV: the two channel halves of the tile's h slice
     uint64_t hempty_v[2];
     uint64_t drain;
+    uint64_t hx[HALO_SLOTS][3][NPART];   // contiguous value tiles: warp q's halo rows are in the slot
     uint32_t tmem_base;
     volatile int abort_flag;
     int issued;       // k-block loads issued by the producer
@@ -362,7 +376,14 @@ __device__ __forceinline__ int vconv_pair(int part, int lane) {
     return k < VPP ? ph * (BN / 4) + part * VPP + k : -1;
 }
 
-template <int MODE, int BN>
+// first row of a value tile's lane quarter q (its lane 0), both layouts
+template <bool CONTIG>
+__device__ __forceinline__ int64_t vrow0(int mt, int q) {
+    return CONTIG ? (int64_t)mt * TILE_OUT_C + q * 32 - (CONV_W - 1)
+                  : (int64_t)mt * TILE_OUT + q * SEG_OUT - (CONV_W - 1);
+}
+
+template <int MODE, int BN, bool CONTIG = false>
 __device__ __forceinline__ TilePre tile_pre_load(const EpiParams& p, int mt, int nt, int q, int lane, int et) {
     TilePre t{};
     const int n0 = nt * BN;
@@ -372,7 +393,7 @@ __device__ __forceinline__ TilePre tile_pre_load(const EpiParams& p, int mt, int
             t.w0 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * pr);
             t.w1 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + 2 * pr + 1);
         }
-        const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - (CONV_W - 1);
+        const int64_t r = vrow0<CONTIG>(mt, q) + lane;
         t.a = (r >= 0 && r < p.n_tok) ? __ldg(p.alpha + r) : 0.f;
     } else if (MODE == MODE_K) {
         if (et < BN) {
@@ -424,10 +445,14 @@ __device__ __forceinline__ float tanh_f32(float x) {
 
 __device__ __forceinline__ float mask_f(float x, uint32_t m) { return __uint_as_float(__float_as_uint(x) & m); }
 
-template <int NCH, bool SLOW, bool RES, bool SCALED>
+// CONTIG: halo_r is the previous warp's slot (its last three rows' v~ over
+// this part's channels of the phase, [3][NCH * 16]; null for the first
+// warp, whose first three rows are history only)
+template <int NCH, bool SLOW, bool RES, bool SCALED, bool CONTIG = false>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
-                                             const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3, int br) {
+                                             const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3, int br,
+                                             const float* halo_r = nullptr) {
     constexpr int H = CONV_W - 1;
     // this branch's history and new history (the same size in both layouts)
     const int64_t hist_off = (int64_t)br * p.B * H * p.d;
@@ -462,6 +487,23 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
             float s1a = __shfl_up_sync(0xffffffffu, v0, 1), s1b = __shfl_up_sync(0xffffffffu, v1, 1);
             float s2a = __shfl_up_sync(0xffffffffu, v0, 2), s2b = __shfl_up_sync(0xffffffffu, v1, 2);
             float s3a = __shfl_up_sync(0xffffffffu, v0, 3), s3b = __shfl_up_sync(0xffffffffu, v1, 3);
+            if (CONTIG && halo_r != nullptr && (i & 31) < 3) {
+                // rows t-k before this warp's first row: slot row 3-k+lane
+                // holds the previous warp's lane 29+(3-k+lane)
+                const int ln = i & 31;
+                const float* hr = halo_r + (cl + c - cbeg);
+                constexpr int PWC = NCH * 16;
+                if (ln < 1) {
+                    s1a = hr[2 * PWC];
+                    s1b = hr[2 * PWC + 1];
+                }
+                if (ln < 2) {
+                    s2a = hr[(1 + ln) * PWC];
+                    s2b = hr[(1 + ln) * PWC + 1];
+                }
+                s3a = hr[ln * PWC];
+                s3b = hr[ln * PWC + 1];
+            }
             if (!SLOW) {
                 // rows before the sequence start (no conv_state): zero history
                 s1a = mask_f(s1a, m1);
@@ -540,15 +582,25 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
 // while phase 1 runs; with M branches, 2M phases: both halves for branch 0,
 // then for branch 1, ... (the accumulator holds v for all of them).  In each
 // phase part `part` takes BN/8 channels.
-template <int BN, bool SCALED>
-__device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt, int nt,
+//
+// CONTIG (contiguous tiles, one branch): warp q < 3 first publishes the
+// gated values of its last three rows over the part's channels in the
+// phase's halo slot, and warp q > 0 waits for warp q-1's slot before its
+// first three rows read their history from it.  Slots rotate over (tile
+// parity, phase): a warp is never more than one tile ahead of another (the
+// accumulator it needs next is released only by all of them), so a slot is
+// rewritten only after its reader has finished that tile.  False when a
+// wait ran out.
+template <int BN, bool SCALED, bool CONTIG = false>
+__device__ __forceinline__ bool epilogue_vconv(uint32_t taddr, uint8_t* hs, const EpiParams& p, int mt, int nt,
                                                int q, int part, int lane, int et, float* s_taps, int phase,
-                                               float a, const TilePre& pre, int br) {
+                                               float a, const TilePre& pre, int br, Barriers* sb = nullptr,
+                                               float* s_halo = nullptr, int tc = 0) {
     constexpr int H = CONV_W - 1;
     const int i = q * 32 + lane;
-    const int64_t r = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - H;
+    const int64_t r = vrow0<CONTIG>(mt, q) + lane;
     const bool in_range = r >= 0 && r < p.n_tok;
-    const bool out_row = in_range && lane >= H;
+    const bool out_row = in_range && (lane >= H || (CONTIG && q > 0));
     int64_t b = 0;
     int t = 0;
     if (in_range) {
@@ -559,21 +611,55 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     // the warp's own taps (both phases), halved, fp32: slot [warp][phase][pair]
     // holds two float4, (c_0, c_0', c_1, c_1') and (c_2, c_2', c_3, c_3') of
     // channels (2m, 2m+1); staged in phase 0 from the values loaded a tile
-    // ahead, read by this warp only
+    // ahead, read by this warp only.  CONTIG stages one phase at a time
+    // (slot [warp][pair]).
     constexpr int VPP = BN / (4 * NPART);
-    float4* s_tw = reinterpret_cast<float4*>(s_taps) + (size_t)(q * NPART + part) * 2 * VPP * 2;
-    if (phase == 0 && br == 0) {
+    float4* s_tw = reinterpret_cast<float4*>(s_taps) + (size_t)(q * NPART + part) * (CONTIG ? 1 : 2) * VPP * 2;
+    if (CONTIG || (phase == 0 && br == 0)) {
         const int k = lane & 15, ph = lane >> 4;
-        if (k < VPP) {
+        if (k < VPP && (!CONTIG || ph == phase)) {
             const float4 w0 = pre.w0, w1 = pre.w1;
-            s_tw[(ph * VPP + k) * 2] = make_float4(0.5f * w0.x, 0.5f * w1.x, 0.5f * w0.y, 0.5f * w1.y);
-            s_tw[(ph * VPP + k) * 2 + 1] = make_float4(0.5f * w0.z, 0.5f * w1.z, 0.5f * w0.w, 0.5f * w1.w);
+            // (CONTIG: the previous phase's reads of the slot ended at its
+            // __syncwarp before the Y stores)
+            const int at = CONTIG ? k : ph * VPP + k;
+            s_tw[at * 2] = make_float4(0.5f * w0.x, 0.5f * w1.x, 0.5f * w0.y, 0.5f * w1.y);
+            s_tw[at * 2 + 1] = make_float4(0.5f * w0.z, 0.5f * w1.z, 0.5f * w0.w, 0.5f * w1.w);
         }
         __syncwarp();
     }
     constexpr int PW = BN / (2 * NPART);     // channels of this part in this phase
     constexpr int NCHK = PW / 16;
     const int cbeg = phase * (BN / 2) + part * PW;
+    const float* halo_r = nullptr;
+    if constexpr (CONTIG) {
+        static_assert(PW == 32, "halo rows hold one 32-channel part");
+        const int slot = (tc & 1) * 2 + phase;
+        float* slot_base = s_halo + (size_t)slot * 3 * NPART * 3 * PW;
+        if (q < 3) {
+            // this warp's last three rows (lanes 29-31), gated as in the
+            // chunk loop, into its slot; each writer arrives on the slot
+            uint32_t va[16], vb[16];
+            tmem_ld16(taddr + cbeg, va);
+            tmem_ld16(taddr + cbeg + 16, vb);
+            tmem_wait_ld(va);
+            tmem_wait_ld(vb);
+            if (lane >= 32 - H) {
+                float* w = slot_base + ((size_t)(q * NPART + part) * 3 + (lane - (32 - H))) * PW;
+#pragma unroll
+                for (int c = 0; c < PW; ++c) {
+                    float v = a * __uint_as_float(c < 16 ? va[c] : vb[c - 16]);
+                    if constexpr (SCALED) v *= __ldg(p.vscale + n0 + cbeg + c);
+                    w[c] = v;
+                }
+                mbar_arrive(&sb->hx[slot][q][part]);
+            }
+        }
+        if (q > 0) {
+            const bool ok = wait_bounded(&sb->hx[slot][q - 1][part], (uint32_t)(tc >> 1) & 1u, sb, p.status);
+            if (!__all_sync(0xffffffffu, ok)) return false;
+            halo_r = slot_base + (size_t)((q - 1) * NPART + part) * 3 * PW;
+        }
+    }
     // Rows whose history reaches back into conv_state, and rows among a
     // sequence's last H when the new history is written, take the slow path
     // (only warps holding such rows).  Without conv_state the history before
@@ -583,28 +669,32 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     const bool slow_row = out_row && ((t < H && p.state) || (p.state_next && t >= p.L - H));
     const uint32_t m1 = t >= 1 ? ~0u : 0u, m2 = t >= 2 ? ~0u : 0u, m3 = t >= 3 ? ~0u : 0u;
     // indexed by tile-local channel (even): this warp's slot, shifted to the phase's first pair
-    const float4* cw = s_tw + phase * VPP * 2 - cbeg;
+    const float4* cw = s_tw + (CONTIG ? 0 : phase * VPP * 2) - cbeg;
     const bool slow = __any_sync(0xffffffffu, slow_row);
     if (p.add_residual) {
-        if (slow) vconv_chunks<NCHK, true, true, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
-                                                            br);
-        else vconv_chunks<NCHK, false, true, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
-                                                            br);
+        if (slow)
+            vconv_chunks<NCHK, true, true, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2,
+                                                           m3, br, halo_r);
+        else
+            vconv_chunks<NCHK, false, true, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2,
+                                                            m3, br, halo_r);
     } else {
-        if (slow) vconv_chunks<NCHK, true, false, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
-                                                            br);
-        else vconv_chunks<NCHK, false, false, SCALED>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2, m3,
-                                                            br);
+        if (slow)
+            vconv_chunks<NCHK, true, false, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1,
+                                                            m2, m3, br, halo_r);
+        else
+            vconv_chunks<NCHK, false, false, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1,
+                                                             m2, m3, br, halo_r);
     }
     // the warp's Y block (its 32 rows x PW channels, in place of h) to global
     // memory: LPR lanes cover one row's contiguous bytes, so each store
-    // instruction writes whole row pieces; the segment's history rows are skipped
+    // instruction writes whole row pieces; history-only rows are skipped
     __syncwarp();
     constexpr int LPR = PW * 2 / 16;
     constexpr int RPI = 32 / LPR;
     const int cb = cbeg >> 6;
     const int j = ((cbeg & 63) >> 3) + lane % LPR;
-    const int64_t seg0 = (int64_t)mt * TILE_OUT + q * SEG_OUT - H;   // global row of the segment's lane 0
+    const int64_t seg0 = vrow0<CONTIG>(mt, q);   // global row of the warp's lane 0
     __nv_bfloat16* y = p.y + (int64_t)br * p.n_tok * p.d;
 #pragma unroll
     for (int k = 0; k < 32 / RPI; ++k) {
@@ -612,8 +702,10 @@ __device__ __forceinline__ void epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
         const int ii = q * 32 + rr;
         const uint4 v = *reinterpret_cast<const uint4*>(hs + cb * (BM * 128) + ii * 128 + ((j ^ (ii & 7)) << 4));
         const int64_t rg = seg0 + rr;
-        if (rr >= H && rg < p.n_tok) __stcs(reinterpret_cast<uint4*>(y + rg * p.d + n0 + cb * 64 + j * 8), v);
+        if ((rr >= H || (CONTIG && q > 0)) && rg < p.n_tok)
+            __stcs(reinterpret_cast<uint4*>(y + rg * p.d + n0 + cb * 64 + j * 8), v);
     }
+    return true;
 }
 
 // After a key tile's partials are written: the CTA that completes a row band
@@ -684,7 +776,11 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                   const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_h,
                   const EpiParams p) {
     static_assert(!PAIR || MODE != MODE_KV, "the KV tile runs on one CTA");
+    static_assert(sizeof(Barriers) <= 1024, "the barrier block");
     using GE = Geo<MODE, BN, PAIR>;
+    static_assert(!GE::CONTIG || GE::GG_BYTES >= EPI_WARPS * (BN / (4 * NPART)) * 32, "one phase of taps per warp");
+    static_assert(GE::SMEM_BYTES <= 232448, "shared memory per CTA");
+    constexpr bool CONTIG = GE::CONTIG;
     constexpr int STAGES = GE::STAGES;
     constexpr int STAGE_BYTES = GE::STAGE_BYTES;
     constexpr int NCTA = PAIR ? 2 : 1;
@@ -696,6 +792,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     Barriers* sb = reinterpret_cast<Barriers*>(smem + GE::SMEM_TILES + GE::H_BYTES);
     float* s_gg = reinterpret_cast<float*>(smem + GE::SMEM_TILES + GE::H_BYTES + 1024);
     float4* s_red = reinterpret_cast<float4*>(smem + GE::SMEM_TILES + GE::H_BYTES + 1024 + GE::GG_BYTES);
+    float* s_halo = reinterpret_cast<float*>(smem + GE::SMEM_TILES + GE::H_BYTES + 1024 + GE::GG_BYTES + GE::RED_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -727,6 +824,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             sb->h_consumed_v[hf] = 0;
         }
         mbar_init(&sb->drain, 1);
+        for (int k = 0; k < HALO_SLOTS * 3 * NPART; ++k) mbar_init(&sb->hx[0][0][0] + k, CONV_W - 1);
         sb->abort_flag = 0;
         sb->issued = 0;
         sb->consumed = 0;
@@ -818,7 +916,10 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                         sb->issued = it + 1;
                         continue;
                     }
-                    if (MODE == MODE_VCONV) {
+                    if (MODE == MODE_VCONV && CONTIG) {
+                        // one 128-row block, starting 3 rows before its outputs
+                        load(&map_a, a_dst, kb * BKE, (int)vrow0<true>(mt, 0));
+                    } else if (MODE == MODE_VCONV) {
                         // four 32-row segments, each starting 3 rows before its outputs
 #pragma unroll
                         for (int sg = 0; sg < 4; ++sg)
@@ -916,8 +1017,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
 #pragma unroll
                             for (int sg = 0; sg < 4; ++sg)
                                 tma_load_2d_hint(&map_h, h_dst + cb * (BM * 128) + sg * (SEG * 128), &sb->hfull_v[hf],
-                                                 nt * BN + cb * 64,
-                                                 m * p.n_tok + mt * TILE_OUT + sg * SEG_OUT - (CONV_W - 1), h_pol);
+                                                 nt * BN + cb * 64, m * p.n_tok + (int)vrow0<CONTIG>(mt, sg), h_pol);
                         }
                         sb->h_issued_v[hf] = k + 1;
                     }
@@ -938,7 +1038,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         // alpha comes from the key pass, which may still be running when this
         // grid was launched as its programmatic dependent
         if (MODE == MODE_VCONV) grid_dep_wait();
-        if (unit0 < num_units) pre = tile_pre_load<MODE, BN>(p, unit_mt(unit0), unit_nt(unit0), q, lane, et);
+        if (unit0 < num_units) pre = tile_pre_load<MODE, BN, CONTIG>(p, unit_mt(unit0), unit_nt(unit0), q, lane, et);
         for (int u = unit0; u < num_units; u += units_step, ++tc) {
             const int acc = tc & 1;
             const uint32_t aph = (uint32_t)(tc >> 1) & 1u;
@@ -956,7 +1056,7 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const float a0 = pre.a;
-                const int64_t r_lane = (int64_t)mt * TILE_OUT + q * SEG_OUT + lane - (CONV_W - 1);
+                const int64_t r_lane = vrow0<CONTIG>(mt, q) + lane;
                 const bool r_ok = r_lane >= 0 && r_lane < p.n_tok;
                 float a_br = a0;
                 const int n_ph = 2 * p.M;
@@ -967,8 +1067,13 @@ project_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     ok = wait_bounded(&sb->hfull_v[phase], (uint32_t)k & 1u, sb, p.status);
                     if (!__all_sync(0xffffffffu, ok)) break;
                     if (br > 0 && phase == 0) a_br = r_ok ? __ldg(p.alpha + (int64_t)br * p.n_tok + r_lane) : 0.f;
-                    epilogue_vconv<BN, F8>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, phase, a_br, pre, br);
-                    if (ph == 0 && has_next) pre = tile_pre_load<MODE, BN>(p, unit_mt(un), unit_nt(un), q, lane, et);
+                    ok = epilogue_vconv<BN, F8, CONTIG>(taddr, s_h, p, mt, nt, q, part, lane, et, s_gg, phase, a_br,
+                                                        pre, br, sb, s_halo, tc);
+                    if (!ok) break;
+                    // the next tile's taps and gates, once this tile's last use of
+                    // them is staged (contiguous tiles stage the taps phase by phase)
+                    if (ph == (CONTIG ? n_ph - 1 : 0) && has_next)
+                        pre = tile_pre_load<MODE, BN, CONTIG>(p, unit_mt(un), unit_nt(un), q, lane, et);
                     const bool last = ph == n_ph - 1;
                     if (last) tc_fence_before();
                     __syncwarp();
@@ -1223,9 +1328,17 @@ int pick_bn(int32_t d, int64_t n_tok, int64_t m_tiles, int num_sms) {
 // CTA pairs once there are enough row tiles to give every SM pair work
 bool use_pair(int64_t m_tiles, int n_groups, int num_sms) { return m_tiles * n_groups >= 2 * (int64_t)num_sms; }
 
-// The value pass stays on single CTAs: a pair couples the two CTAs' value
-// epilogues through the shared accumulator, and on B200 the value pass ran
-// 124 us as pairs against 101 us on single CTAs (c2), 399 against 322 us (c3).
+// The value pass runs on CTA pairs with contiguous 128-row tiles (one A box
+// per CTA and stage, 125 output rows) for one bf16 branch, 256-channel tiles
+// and K >= 2048: there a tile's MMAs outlast the epilogue's halo exchange
+// between warps (about 2.5 us a tile), which at K = 1024 sits on the
+// critical path (B200, c2: 131 against 108 us single; c3: 323-331 against
+// 351-376 us).  On pairs the layout of four overlapping 32-row boxes per
+// stage starves the MMAs (124 against 101 us on single CTAs at c2, 399
+// against 322 us at c3), so that layout stays on single CTAs.
+bool use_contig_pair(int bn, int32_t M, bool f8, int32_t d_mem, int64_t m_tiles_c, int n_groups, int num_sms) {
+    return bn == 256 && M == 1 && !f8 && d_mem >= 2048 && use_pair(m_tiles_c, n_groups, num_sms);
+}
 
 }  // namespace
 
@@ -1338,6 +1451,16 @@ cudaError_t launch_vconv_tc(const void* e, int32_t B, int32_t L, int32_t d_mem, 
     p.L = L;
     p.add_residual = add_residual;
     const int64_t mt = (n_tok + TILE_OUT - 1) / TILE_OUT;
+    const int64_t mt_c = (n_tok + TILE_OUT_C - 1) / TILE_OUT_C;
+    if (use_contig_pair(bn, M, f8, d_mem, mt_c, p.n_groups, num_sms)) {
+        // contiguous tiles on CTA pairs: each CTA's A block is 128 rows, its
+        // half of the W_V tile 128 channels
+        CUtensorMap ma_c, mv_c;
+        if (!make_map(&ma_c, e, (uint64_t)n_tok, (uint64_t)d_mem, BM) ||
+            !make_map(&mv_c, Wv, (uint64_t)d, (uint64_t)d_mem, 128))
+            return cudaErrorInvalidValue;
+        return launch_mode<MODE_VCONV, 256, true, false>(ma_c, mv_c, mv_c, mh, p, mt_c, num_sms, s, pdl);
+    }
     if (f8)
         return bn == 256 ? launch_mode<MODE_VCONV, 256, false, true>(ma, mv, mv, mh, p, mt, num_sms, s, pdl)
                          : launch_mode<MODE_VCONV, 128, false, true>(ma, mv, mv, mh, p, mt, num_sms, s, pdl);

@@ -265,6 +265,29 @@ def test_forward_full_size_sampled(eb, name):
     _check_y(wl, to_np(y[sel]), ref.y, ref.vt_win, inp.conv_w)
 
 
+def _value_rows(wl, tiles=None):
+    """Rows at the value pass's tile and warp boundaries.  With K >= 2048 the
+    value pass runs contiguous tiles on CTA pairs (125 output rows per
+    128-row CTA tile, starting 3 rows before), and the first three rows of
+    warps 1-3 take their conv history from the previous warp's halo slot;
+    otherwise tiles of four 29-row segments (116 rows).  `tiles`: the tile
+    indices to cover (default all)."""
+    contig = wl.d_mem >= 2048 and wl.dtype == "bf16"
+    out, step = (125, 32) if contig else (116, 29)
+    rows = set()
+    n_tiles = (wl.n_tok + out - 1) // out
+    for mt in (range(n_tiles) if tiles is None else [m % n_tiles for m in tiles]):
+        base = mt * out - 3
+        for q in range(4):
+            for lane in ((3, 4) if q == 0 else ((0, 1, 2, 31) if contig else (3, 4))):
+                r = base + step * q + lane
+                if 0 <= r < wl.n_tok:
+                    rows.add(r)
+        if 0 <= base + 2 < wl.n_tok:
+            rows.add(base + 2)
+    return rows
+
+
 # CTA-pair tiling (two CTAs per M = 256 MMA) engages once there are enough row
 # tiles to occupy every SM pair; these shapes reach it with ragged ends: an odd
 # number of value row tiles leaves the second CTA of the last pair without rows
@@ -272,6 +295,9 @@ PAIR_CASES = {
     "pair_a": W["c2"].replace(name="pair_a", B=2, T=2000, M=10007, seed=31),       # 4000 rows, 35 value tiles
     "pair_b": W["c2"].replace(name="pair_b", B=3, T=1501, M=10007, seed=32),       # 4503 rows, ragged 128-row band
     "pair_c": W["c2"].replace(name="pair_c", B=3, T=1376, M=10007, seed=33),       # 4128 rows, 33 key tiles (odd)
+    # K = 2048: the value pass on contiguous pair tiles, 31 of them (the last
+    # pair's second CTA holds no rows)
+    "contig_a": W["c3"].replace(name="contig_a", B=2, T=1900, M=10007, seed=35),
 }
 
 
@@ -283,13 +309,14 @@ def test_cta_pair_tiling_sampled(eb, name):
     ctx = eb.Engram(config_for(inp, eb))
     y, alpha = _run_forward(eb, ctx, di, add_residual=True)
     assert ctx.status() == (eb.ENGRAM_OK, 0)
-    # rows around every 116-row value tile edge and 128-row band edge, the
-    # sequence ends, and random rows
+    # rows around every 128-row key band edge, the value pass's warp and tile
+    # boundaries, the sequence ends, and random rows
     edges = set()
-    for base in list(range(0, wl.n_tok, 116)) + list(range(0, wl.n_tok, 128)):
+    for base in range(0, wl.n_tok, 128):
         for r in (base - 4, base - 1, base, base + 3):
             if 0 <= r < wl.n_tok:
                 edges.add(r)
+    edges |= _value_rows(wl, tiles=(0, 1, 2, 15, 16, -3, -2, -1))
     pos = np.array(sorted(edges | set(synth.sample_positions(wl, 64, seed=7).tolist())), dtype=np.int64)
     ref = oracle.forward_rows(inp, pos, add_residual=True)
     sel = torch.from_numpy(pos).cuda()
@@ -507,6 +534,34 @@ def test_unfused_project_then_conv_matches_oracle(eb, name):
     # new history = the last w-1 gated rows of every sequence
     want = ref.vt.reshape(wl.B, wl.T, wl.d)[:, wl.T - (wl.w - 1):]
     np.testing.assert_allclose(state.cpu().numpy(), want, rtol=0, atol=1e-5)
+
+
+def test_pair_value_pass_with_history(eb):
+    """A continued prefill on the contiguous pair tiles: each sequence's first
+    three rows take their history from conv_state, rows at warp boundaries
+    from the halo slots, and the last three rows become the new state."""
+    wl = W["c3"].replace(name="pair_hist", B=2, T=2000, t_begin=100, M=10007, seed=34)
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    hist = inp.state_rows(np.arange(wl.B))
+    state = inp.device_state("cuda:0").contiguous()
+    L = wl.T - wl.t_begin
+    y, alpha = _run_forward(eb, ctx, di, t_begin=wl.t_begin, state=state, add_residual=True)
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    rows = _value_rows(wl, tiles=(0, 1, 14, 15, 16, 29, 30))
+    for b in range(wl.B):
+        rows |= {b * L + t for t in (0, 1, 2, 3, L - 1)}
+    pos = np.array(sorted(rows), dtype=np.int64)
+    ref = oracle.forward_rows(inp, pos, add_residual=True, hist=hist)
+    sel = torch.from_numpy(pos).cuda()
+    np.testing.assert_allclose(to_np(alpha[sel]), ref.alpha, rtol=0, atol=2e-6)
+    _check_y(wl, to_np(y[sel]), ref.y, ref.vt_win, inp.conv_w)
+    last = oracle.forward_rows(inp, np.array([b * L + t for b in range(wl.B) for t in range(L - 3, L)]),
+                               hist=hist)
+    want = last.vt_win[:, 0].reshape(wl.B, 3, wl.d)
+    vmax = float(np.abs(want).max())
+    assert float(np.abs(state.cpu().numpy() - want).max()) <= 2.0 ** -10 * vmax + 1e-6
 
 
 @pytest.mark.parametrize("name", ["b1", "b3"])
