@@ -21,7 +21,11 @@
 //              shuffles.  Taps, SiLU and the residual follow (all fp32) and
 //              Y is written;
 //              v never reaches global memory.  Consecutive segments overlap
-//              by 3 rows (116 output rows per 128-row MMA tile).
+//              by 3 rows (116 output rows per 128-row MMA tile).  On CTA
+//              pairs (bf16, K >= 2048) the tile is instead 128 contiguous
+//              rows per CTA (3 history rows, then 125 output rows): the
+//              first three rows of warps 1-3 take their history from the
+//              previous warp's last three through shared-memory halo slots.
 //
 // Persistent kernel, one CTA per SM, warp-specialised (640 threads):
 //   warp 0     TMA producer: 2-D tiled loads (128-byte swizzle) of A (e) and
