@@ -1332,6 +1332,31 @@ int pick_bn(int32_t d, int64_t n_tok, int64_t m_tiles, int num_sms) {
 // CTA pairs once there are enough row tiles to give every SM pair work
 bool use_pair(int64_t m_tiles, int n_groups, int num_sms) { return m_tiles * n_groups >= 2 * (int64_t)num_sms; }
 
+// Row units per group of the grouped tile order of a wide key pass (stacked
+// W_K of several branches): a group's rows of e and the whole stacked W_K
+// stay in L2 together, in 70 % of it (the rest holds the streaming h and the
+// gate partials).  Measured at c3 with four bf16 branches (row units of 256
+// rows, W_K 42 MB): 8 / 16 / 32 / 48 / 64 / 128 units per group gave a key
+// pass of 1780 / 1437 / 1200 / 1157 / 1235 / 1308 us; this rule gives 44.
+int raster_group(int32_t M, int32_t d, int32_t d_mem, bool f8, bool pair) {
+    static int64_t l2_bytes[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int64_t l2 = dev < 64 ? l2_bytes[dev] : 0;
+    if (l2 == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess || v <= 0) v = 96 << 20;
+        cudaGetLastError();
+        l2 = v;
+        if (dev < 64) l2_bytes[dev] = l2;
+    }
+    const double es = f8 ? 1.0 : 2.0;
+    const double w_bytes = (double)M * d * d_mem * es;
+    const double unit_bytes = (double)(pair ? 2 * BM : BM) * d_mem * es;
+    const double rb = (0.7 * (double)l2 - w_bytes) / unit_bytes;
+    return rb < 8.0 ? 8 : (rb > 4096.0 ? 4096 : (int)rb);
+}
+
 // The value pass runs on CTA pairs with contiguous 128-row tiles (one A box
 // per CTA and stage, 125 output rows) for one bf16 branch, 256-channel tiles
 // and K >= 2048: there a tile's MMAs outlast the epilogue's halo exchange
@@ -1406,9 +1431,10 @@ cudaError_t launch_gate_k_tc(const void* e, int64_t n_tok, int32_t d_mem, const 
     p.d = d;
     p.G = M * (d / 128);
     p.n_groups = M * (d / bn);
-    p.raster_rb = p.n_groups > 16 ? 8 : 0;
     const int64_t mt = (n_tok + BM - 1) / BM;
-    if (bn == 256 && use_pair(mt, p.n_groups, num_sms)) {
+    const bool pair = bn == 256 && use_pair(mt, p.n_groups, num_sms);
+    p.raster_rb = p.n_groups > 16 ? raster_group(M, d, d_mem, f8, pair) : 0;
+    if (pair) {
         CUtensorMap mk2;
         if (!make_map(&mk2, Wk, (uint64_t)M * d, (uint64_t)d_mem, 128, f8)) return cudaErrorInvalidValue;
         return f8 ? launch_mode<MODE_K, 256, true, true>(ma, mk2, mk2, mh, p, mt, num_sms, s, pdl)
