@@ -564,6 +564,36 @@ def test_pair_value_pass_with_history(eb):
     assert float(np.abs(state.cpu().numpy() - want).max()) <= 2.0 ** -10 * vmax + 1e-6
 
 
+def test_pair_value_pass_short_sequences_with_history(eb):
+    """1024 sequences of 4 new positions each (a decode-shaped call, L <= 8)
+    at K = 2048: the value pass runs contiguous pair tiles and reads the conv
+    history in the sequence-minor layout, and every row's history reaches
+    into conv_state (the slow path), including rows at warp boundaries that
+    otherwise take it from the halo slots."""
+    wl = W["c3"].replace(name="ds_contig", B=1024, T=68, t_begin=64, M=10007, seed=36)
+    inp = synth.Inputs(wl, gamma="random")
+    di = DeviceInputs(inp)
+    ctx = eb.Engram(config_for(inp, eb))
+    hist = inp.state_rows(np.arange(wl.B))
+    state = inp.device_state("cuda:0").contiguous()
+    L = wl.T - wl.t_begin
+    y, alpha = _run_forward(eb, ctx, di, t_begin=wl.t_begin, state=state, add_residual=True)
+    assert ctx.status() == (eb.ENGRAM_OK, 0)
+    rows = _value_rows(wl, tiles=(0, 1, 2, 16, 17, -2, -1))
+    rows |= set(synth.sample_positions(wl, 48, seed=9).tolist())
+    pos = np.array(sorted(rows), dtype=np.int64)
+    ref = oracle.forward_rows(inp, pos, add_residual=True, hist=hist)
+    sel = torch.from_numpy(pos).cuda()
+    np.testing.assert_allclose(to_np(alpha[sel]), ref.alpha, rtol=0, atol=2e-6)
+    _check_y(wl, to_np(y[sel]), ref.y, ref.vt_win, inp.conv_w)
+    # the new history of a few sequences: their last three gated rows
+    bs = np.array([0, 5, 511, 1023])
+    last = oracle.forward_rows(inp, np.array([b * L + t for b in bs for t in range(L - 3, L)]), hist=hist)
+    want = last.vt_win[:, 0].reshape(len(bs), 3, wl.d)
+    got = state.cpu().numpy()[bs]
+    assert float(np.abs(got - want).max()) <= 2.0 ** -10 * float(np.abs(want).max()) + 1e-6
+
+
 @pytest.mark.parametrize("name", ["b1", "b3"])
 def test_fused_prefill_with_history(eb, name):
     """Fused tensor-core path with a conv history at the start of every
