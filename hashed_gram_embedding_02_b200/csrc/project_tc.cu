@@ -451,8 +451,11 @@ __device__ __forceinline__ float mask_f(float x, uint32_t m) { return __uint_as_
 
 // CONTIG: halo_r is the previous warp's slot (its last three rows' v~ over
 // this part's channels of the phase, [3][NCH * 16]; null for the first
-// warp, whose first three rows are history only)
-template <int NCH, bool SLOW, bool RES, bool SCALED, bool CONTIG = false>
+// warp, whose first three rows are history only).  MASK: some row of the
+// warp is among its sequence's first three (the fast path then zeroes the
+// history before the start; without such a row the masks are all ones and
+// are skipped)
+template <int NCH, bool SLOW, bool RES, bool SCALED, bool CONTIG = false, bool MASK = true>
 __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const EpiParams& p, int i, int64_t r,
                                              int64_t b, int t, float a, bool out_row, int n0, int cbeg,
                                              const float4* s_cw, uint32_t m1, uint32_t m2, uint32_t m3, int br,
@@ -508,7 +511,7 @@ __device__ __forceinline__ void vconv_chunks(uint32_t taddr, uint8_t* hs, const 
                 s3a = hr[ln * PWC];
                 s3b = hr[ln * PWC + 1];
             }
-            if (!SLOW) {
+            if (!SLOW && MASK) {
                 // rows before the sequence start (no conv_state): zero history
                 s1a = mask_f(s1a, m1);
                 s1b = mask_f(s1b, m1);
@@ -675,13 +678,17 @@ __device__ __forceinline__ bool epilogue_vconv(uint32_t taddr, uint8_t* hs, cons
     // indexed by tile-local channel (even): this warp's slot, shifted to the phase's first pair
     const float4* cw = s_tw + (CONTIG ? 0 : phase * VPP * 2) - cbeg;
     const bool slow = __any_sync(0xffffffffu, slow_row);
+    const bool masked = __any_sync(0xffffffffu, t < H);
     if (p.add_residual) {
         if (slow)
             vconv_chunks<NCHK, true, true, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2,
                                                            m3, br, halo_r);
-        else
+        else if (masked)
             vconv_chunks<NCHK, false, true, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1, m2,
                                                             m3, br, halo_r);
+        else
+            vconv_chunks<NCHK, false, true, SCALED, CONTIG, false>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw,
+                                                                   m1, m2, m3, br, halo_r);
     } else {
         if (slow)
             vconv_chunks<NCHK, true, false, SCALED, CONTIG>(taddr, hs, p, i, r, b, t, a, out_row, n0, cbeg, cw, m1,
