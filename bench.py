@@ -202,18 +202,18 @@ KERNEL_SOURCES = {
 CAPTURED_TRAFFIC = {
     # (workload, kernel): (source digest, bytes per launch)
     # c2 at full size, mean of the five timed steps' launches (profiles/launches_c2.md)
-    ("c2", "vconv_tc"): ("63961e8b747035aa", 123218586 + 28744806),
-    ("c2", "gate_k_tc"): ("63961e8b747035aa", 122776576 + 384154),
-    ("c2", "retrieve"): ("cd4c38c473a10c27", 28944179 + 180122),
+    ("c2", "vconv_tc"): ("c854b247a509134b", 123174144 + 28366950),
+    ("c2", "gate_k_tc"): ("c854b247a509134b", 122753075 + 507085),
+    ("c2", "retrieve"): ("cd4c38c473a10c27", 28943667 + 190822),
     # c3 kernels on 2 sequences and 499979-row tables (profiles/dram_c3_small.md)
     ("c3-B2-M499979", "vconv_tc"): ("59d2794a31cc0db6", 86297856 + 2050304),
     ("c3-B2-M499979", "gate_k_tc"): ("59d2794a31cc0db6", 86043136 + 130048),
     ("c3-B2-M499979", "retrieve"): ("8c46903b0c8d286e", 29667072 + 480512),
     # c3 and c4 at full size, mean of the five timed steps' launches
     # (profiles/launches_c3.md, profiles/launches_c4.md)
-    ("c3", "vconv_tc"): ("63961e8b747035aa", 314450944 + 128533248),
-    ("c3", "gate_k_tc"): ("63961e8b747035aa", 312563302 + 7408026),
-    ("c3", "retrieve"): ("cd4c38c473a10c27", 115572787 + 80994406),
+    ("c3", "vconv_tc"): ("c854b247a509134b", 314464102 + 128461363),
+    ("c3", "gate_k_tc"): ("c854b247a509134b", 312547584 + 7371162),
+    ("c3", "retrieve"): ("cd4c38c473a10c27", 115575347 + 80895590),
     ("c4", "retrieve"): ("cd4c38c473a10c27", 1209139 + 2867),
     ("c4", "gate_kv_decode"): ("6bc5ef79605ad072", 23401165 + 0),
     ("c4", "conv_decode"): ("6bc5ef79605ad072", 11986534 + 0),
