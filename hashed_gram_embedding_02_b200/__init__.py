@@ -23,7 +23,8 @@ from .binding import (  # noqa: F401  (re-exported C ABI names)
     engram_host_cache_stats, engram_shard_range, engram_forward_sharded, engram_ipc_export, engram_ipc_open,
     engram_ipc_close, ENGRAM_IPC_HANDLE_BYTES, ENGRAM_MAX_SHARDS, engram_multibranch_workspace_bytes,
     engram_forward_multibranch, ENGRAM_MAX_BRANCHES, engram_table_grad_workspace_bytes, engram_table_grad,
-    engram_table_sgd, engram_host_tier_map,
+    engram_table_sgd, engram_host_tier_map, engram_grad_route_workspace_bytes, engram_grad_route,
+    engram_grad_combine_workspace_bytes, engram_grad_combine, engram_shard_sgd,
     engram_last_error, engram_profile_enable, engram_profile_read, engram_project, engram_remap, engram_strerror,
     engram_workspace_bytes, make_config)
 
@@ -129,6 +130,39 @@ class Engram:
         engram_table_grad(self.ctx, idx, n_tok, d_e, rows, grad, cnt, ws, need, stream)
         U = int(cnt.item())
         return rows[:U], grad[:U], cnt
+
+    def grad_route(self, rows, grad, n_pairs, n_shards: int, stream=None):
+        """This rank's (row, gradient) pairs split by the shard that owns the
+        row: (send_rows, send_grad, send_counts), the counts an int64 [n_shards]
+        tensor on the device, the segments in shard order."""
+        import torch
+        max_rows = rows.shape[0]
+        send_rows = torch.empty(max(1, max_rows), dtype=torch.int64, device=self.device)
+        send_grad = torch.empty(max(1, max_rows), self.cfg.row_dim, dtype=torch.float32, device=self.device)
+        send_counts = torch.empty(n_shards, dtype=torch.int64, device=self.device)
+        need = engram_grad_route_workspace_bytes(self.ctx)
+        ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        engram_grad_route(self.ctx, n_shards, rows, grad, n_pairs, max_rows, send_rows, send_grad, send_counts, ws,
+                          need, stream)
+        return send_rows, send_grad, send_counts
+
+    def grad_combine(self, pair_rows, pair_grad, n_shards: int, shard: int, stream=None):
+        """The pairs received by shard `shard`, summed per row: (rows [U]
+        int64 global rows, grad [U][D] fp32, count), U read back (a sync)."""
+        import torch
+        n = pair_rows.shape[0]
+        need = engram_grad_combine_workspace_bytes(self.ctx, n)
+        ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        rows = torch.empty(max(1, n), dtype=torch.int64, device=self.device)
+        grad = torch.empty(max(1, n), self.cfg.row_dim, dtype=torch.float32, device=self.device)
+        cnt = torch.zeros(1, dtype=torch.int64, device=self.device)
+        engram_grad_combine(self.ctx, n_shards, shard, pair_rows, pair_grad, n, rows, grad, cnt, ws, need, stream)
+        U = int(cnt.item())
+        return rows[:U], grad[:U], cnt
+
+    def shard_sgd(self, n_shards: int, shard: int, rows, grad, n_unique, shard_table, lr: float, stream=None):
+        """shard_table[row - first] -= lr * grad for the listed global rows."""
+        engram_shard_sgd(self.ctx, n_shards, shard, rows, grad, n_unique, rows.shape[0], shard_table, lr, stream)
 
     def status(self, stream=None):
         return engram_device_status(self.ctx, stream)
@@ -236,3 +270,52 @@ class ShardedTables:
         for b in self._bases:
             self._close(b)
         self._bases = []
+
+
+def all_to_all_pairs(send_rows, send_grad, send_counts, all_to_all_single=None):
+    """The backward's exchange of (row, gradient) pairs between the ranks.
+
+    ``send_counts[g]`` pairs of this rank are for rank g (one shard per rank),
+    in segments of ``send_rows`` / ``send_grad`` in rank order (what
+    :meth:`Engram.grad_route` writes).  First the counts go round (one int64
+    from every rank to every rank), then the segments, with the split sizes
+    those counts give.  Returns (recv_rows, recv_grad, recv_counts as a host
+    list): the pairs sent to this rank by rank 0, then rank 1, and so on.
+    ``all_to_all_single`` defaults to ``torch.distributed``'s (NCCL between
+    GPUs, gloo on CPU); reading the counts on the host is a sync."""
+    import torch
+    if all_to_all_single is None:
+        import torch.distributed as dist
+        all_to_all_single = dist.all_to_all_single
+    recv_counts = torch.empty_like(send_counts)
+    all_to_all_single(recv_counts, send_counts)
+    in_split = [int(x) for x in send_counts.tolist()]
+    out_split = [int(x) for x in recv_counts.tolist()]
+    if min(in_split + out_split, default=0) < 0:
+        raise RuntimeError(f"negative pair count in {in_split} / {out_split}")
+    n_send, n_recv = sum(in_split), sum(out_split)
+    if n_send > send_rows.shape[0]:
+        raise RuntimeError(f"{n_send} pairs to send, the send buffers hold {send_rows.shape[0]}")
+    D = send_grad.shape[1]
+    recv_rows = torch.empty(n_recv, dtype=send_rows.dtype, device=send_rows.device)
+    recv_grad = torch.empty(n_recv, D, dtype=send_grad.dtype, device=send_grad.device)
+    all_to_all_single(recv_rows, send_rows[:n_send], out_split, in_split)
+    all_to_all_single(recv_grad, send_grad[:n_send], out_split, in_split)
+    return recv_rows, recv_grad, out_split
+
+
+def sharded_table_step(engram: Engram, tables: ShardedTables, idx, d_e, lr: float, rank: int, world: int,
+                       all_to_all_single=None):
+    """One update of sharded tables from this rank's batch: the sparse
+    gradient of the rows the batch looked up (engram_table_grad), routed to
+    the ranks that own them (engram_grad_route), exchanged
+    (:func:`all_to_all_pairs`), summed per row in rank order
+    (engram_grad_combine) and applied to this rank's shard
+    (engram_shard_sgd).  Every rank calls it with its own batch; returns the
+    (rows, gradient) applied to this rank's shard."""
+    rows, grad, cnt = engram.table_grad(idx, d_e)
+    send_rows, send_grad, send_counts = engram.grad_route(rows, grad, cnt, world)
+    recv_rows, recv_grad, _ = all_to_all_pairs(send_rows, send_grad, send_counts, all_to_all_single)
+    r, g, u = engram.grad_combine(recv_rows, recv_grad, world, rank)
+    engram.shard_sgd(world, rank, r, g, u, tables.local, lr)
+    return r, g

@@ -42,7 +42,8 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_strerror", "engram_last_er
            "engram_host_cache_enable", "engram_host_cache_reset", "engram_host_cache_stats",
            "engram_shard_range", "engram_forward_sharded", "engram_ipc_export", "engram_ipc_open", "engram_ipc_close",
            "engram_multibranch_workspace_bytes", "engram_forward_multibranch", "engram_table_grad_workspace_bytes",
-           "engram_table_grad", "engram_table_sgd", "engram_host_tier_map")
+           "engram_table_grad", "engram_table_sgd", "engram_host_tier_map", "engram_grad_route_workspace_bytes",
+           "engram_grad_route", "engram_grad_combine_workspace_bytes", "engram_grad_combine", "engram_shard_sgd")
 ENGRAM_MAX_BRANCHES = 4
 ENGRAM_IPC_HANDLE_BYTES = 64
 ENGRAM_MAX_SHARDS = 16
@@ -115,6 +116,11 @@ _sigs = {
     "engram_table_grad_workspace_bytes": ([_vp, _i64], _sz),
     "engram_table_grad": ([_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _st),
     "engram_table_sgd": ([_vp, _vp, _vp, _vp, _i64, _vp, ctypes.c_float, _vp], _st),
+    "engram_grad_route_workspace_bytes": ([_vp], _sz),
+    "engram_grad_route": ([_vp, _i32, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp], _st),
+    "engram_grad_combine_workspace_bytes": ([_vp, _i64], _sz),
+    "engram_grad_combine": ([_vp, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp], _st),
+    "engram_shard_sgd": ([_vp, _i32, _i32, _vp, _vp, _vp, _i64, _vp, ctypes.c_float, _vp], _st),
     "engram_forward_multibranch": ([_vp, _i32, _vp, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp], _st),
     "engram_forward_sharded": ([_vp, _vp, _i32, _i32, _i64, _i32, _vp, ctypes.POINTER(_vp), _i32, _vp, _vp, _vp, _vp,
@@ -303,6 +309,33 @@ def engram_table_grad(ctx, idx, n_tok, d_e, rows_out, grad_out, n_unique, worksp
 def engram_table_sgd(ctx, rows, grad, n_unique, max_rows, tables, lr, stream=None):
     _check(_lib.engram_table_sgd(ctx, _ptr(rows), _ptr(grad), _ptr(n_unique), max_rows, _ptr(tables), float(lr),
                                  _stream(stream)), "engram_table_sgd")
+
+
+def engram_grad_route_workspace_bytes(ctx) -> int:
+    return int(_lib.engram_grad_route_workspace_bytes(ctx))
+
+
+def engram_grad_route(ctx, n_shards, rows, grad, n_pairs, max_rows, send_rows, send_grad, send_counts, workspace,
+                      workspace_bytes, stream=None):
+    _check(_lib.engram_grad_route(ctx, n_shards, _ptr(rows), _ptr(grad), _ptr(n_pairs), max_rows, _ptr(send_rows),
+                                  _ptr(send_grad), _ptr(send_counts), _ptr(workspace), workspace_bytes,
+                                  _stream(stream)), "engram_grad_route")
+
+
+def engram_grad_combine_workspace_bytes(ctx, n_pairs: int) -> int:
+    return int(_lib.engram_grad_combine_workspace_bytes(ctx, n_pairs))
+
+
+def engram_grad_combine(ctx, n_shards, shard, pair_rows, pair_grad, n_pairs, rows_out, grad_out, n_unique, workspace,
+                        workspace_bytes, stream=None):
+    _check(_lib.engram_grad_combine(ctx, n_shards, shard, _ptr(pair_rows), _ptr(pair_grad), n_pairs, _ptr(rows_out),
+                                    _ptr(grad_out), _ptr(n_unique), _ptr(workspace), workspace_bytes,
+                                    _stream(stream)), "engram_grad_combine")
+
+
+def engram_shard_sgd(ctx, n_shards, shard, rows, grad, n_unique, max_rows, shard_table, lr, stream=None):
+    _check(_lib.engram_shard_sgd(ctx, n_shards, shard, _ptr(rows), _ptr(grad), _ptr(n_unique), max_rows,
+                                 _ptr(shard_table), float(lr), _stream(stream)), "engram_shard_sgd")
 
 
 # ---------------------------------------------------------------- sharded tables

@@ -63,15 +63,43 @@ __device__ __forceinline__ int64_t find_slot(const unsigned long long* keys, uin
     return -1;
 }
 
-__global__ void grad_insert_kernel(const uint32_t* __restrict__ idx, int64_t n_lookups, GradGeo g,
-                                   unsigned long long* keys, uint32_t* vals, uint32_t mask, uint64_t* rows_out,
-                                   unsigned long long* count, uint32_t* status) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
-         i += (int64_t)gridDim.x * blockDim.x) {
+// Where a lookup's key (global row + 1) comes from.  LookupKeys: the
+// lookups (t, j) of a batch, global row row_off[j] + idx (an invalid n-gram
+// has no row and no gradient).  PairKeys: (row, gradient) pairs sent by the
+// ranks to the shard that owns rows [lo, hi); a row outside it is an error.
+struct LookupKeys {
+    const uint32_t* idx;
+    GradGeo g;
+    __device__ __forceinline__ bool key(int64_t i, unsigned long long& k, uint32_t*) const {
         const int j = (int)(i % g.J);
         const uint32_t r = __ldg(idx + i);
-        if (r >= g.rows[j]) continue;                  // invalid n-gram: no row, no gradient
-        const unsigned long long key = (unsigned long long)(g.row_off[j] + r) + 1ull;
+        if (r >= g.rows[j]) return false;
+        k = (unsigned long long)(g.row_off[j] + r) + 1ull;
+        return true;
+    }
+};
+
+struct PairKeys {
+    const uint64_t* rows;
+    uint64_t lo, hi;
+    __device__ __forceinline__ bool key(int64_t i, unsigned long long& k, uint32_t* status) const {
+        const uint64_t r = __ldg(reinterpret_cast<const unsigned long long*>(rows) + i);
+        if (r < lo || r >= hi) {
+            if (status) flag(status, ENGRAM_ERR_INDEX);
+            return false;
+        }
+        k = (unsigned long long)r + 1ull;
+        return true;
+    }
+};
+
+template <typename Keys>
+__global__ void grad_insert_kernel(Keys src, int64_t n_lookups, unsigned long long* keys, uint32_t* vals,
+                                   uint32_t mask, uint64_t* rows_out, unsigned long long* count, uint32_t* status) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        unsigned long long key;
+        if (!src.key(i, key, status)) continue;
         uint32_t h = (uint32_t)mix64(key) & mask;
         bool placed = false;
         for (uint32_t probe = 0; probe <= mask; ++probe) {
@@ -94,16 +122,16 @@ __global__ void grad_insert_kernel(const uint32_t* __restrict__ idx, int64_t n_l
 }
 
 // each valid lookup's row id (or 0xFFFFFFFF), and the size of every id's bucket
-__global__ void grad_id_kernel(const uint32_t* __restrict__ idx, int64_t n_lookups, GradGeo g,
-                               const unsigned long long* __restrict__ keys, const uint32_t* __restrict__ vals,
-                               uint32_t mask, uint32_t* __restrict__ lid, uint32_t* bucket) {
+template <typename Keys>
+__global__ void grad_id_kernel(Keys src, int64_t n_lookups, const unsigned long long* __restrict__ keys,
+                               const uint32_t* __restrict__ vals, uint32_t mask, uint32_t* __restrict__ lid,
+                               uint32_t* bucket) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lookups;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int j = (int)(i % g.J);
-        const uint32_t r = __ldg(idx + i);
         uint32_t id = 0xFFFFFFFFu;
-        if (r < g.rows[j]) {
-            const int64_t h = find_slot(keys, mask, (unsigned long long)(g.row_off[j] + r) + 1ull);
+        unsigned long long key;
+        if (src.key(i, key, nullptr)) {
+            const int64_t h = find_slot(keys, mask, key);
             if (h >= 0) {
                 id = vals[h];
                 atomicAdd(bucket + id, 1u);
@@ -173,21 +201,40 @@ __global__ void grad_place_kernel(const uint32_t* __restrict__ lid, int64_t n_lo
     }
 }
 
+// Where lookup `pos`'s gradient slice starts.  LookupSlices: slice j of
+// dL/de_t for pos = t * J + j.  PairSlices: the pos-th received gradient row.
+template <typename T>
+struct LookupSlices {
+    using Elem = T;
+    const T* de;
+    int J, D;
+    __device__ __forceinline__ const T* at(uint32_t pos) const {
+        const int64_t t = pos / J, j = pos - t * J;
+        return de + t * ((int64_t)J * D) + j * D;
+    }
+};
+
+struct PairSlices {
+    using Elem = float;
+    const float* g;
+    int D;
+    __device__ __forceinline__ const float* at(uint32_t pos) const { return g + (int64_t)pos * D; }
+};
+
 // One warp per distinct row: order the segment by position (into `sorted`,
 // each element's rank = the count of smaller positions), then sum the
-// slices of dL/de in that order.  Lane l owns the row's 16-byte chunks
+// gradient slices in that order.  Lane l owns the row's 16-byte chunks
 // l, l + 32, ... (D*elem/16 chunks in all).
-template <typename T>
+template <typename Slices>
 __global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint32_t* __restrict__ start,
                                    const uint32_t* __restrict__ bucket, const unsigned long long* __restrict__ count,
-                                   uint32_t* __restrict__ sorted, const T* __restrict__ de, int J, int D,
-                                   float* __restrict__ grad) {
+                                   uint32_t* __restrict__ sorted, Slices src, int D, float* __restrict__ grad) {
+    using T = typename Slices::Elem;
     constexpr int EPC = 16 / sizeof(T);   // elements per 16-byte chunk
     const int lane = threadIdx.x & 31;
     const int64_t U = (int64_t)*count;
     const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int chunks = D / EPC;
-    const int64_t d_mem = (int64_t)J * D;
     for (int64_t id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; id < U; id += warps) {
         const uint32_t s0 = start[id], k = bucket[id];
         const uint32_t* in = seg + s0;
@@ -204,10 +251,8 @@ __global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint3
 #pragma unroll
             for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
             for (uint32_t a = 0; a < k; ++a) {
-                const uint32_t pos = srt[a];                   // lookup t * J + j
-                const int64_t t = pos / J, j = pos - t * J;
                 float f[EPC];
-                Vec<T>::load(de + t * d_mem + j * D + c * EPC, f);
+                Vec<T>::load(src.at(srt[a]) + c * EPC, f);
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) acc[e] += f[e];
             }
@@ -218,25 +263,81 @@ __global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint3
     }
 }
 
-// tables[row] -= lr * grad, in the tables' dtype (fp32 arithmetic, one
-// rounding to the storage type); one warp per row
+// tables[row - first] -= lr * grad for rows in [first, first + n_rows), in
+// the tables' dtype (fp32 arithmetic, one rounding to the storage type); one
+// warp per row.  The whole table is first = 0, n_rows = sum of M_j; a shard
+// is its own range.
 template <typename T>
 __global__ void table_sgd_kernel(const uint64_t* __restrict__ rows, const float* __restrict__ grad,
-                                 const unsigned long long* __restrict__ count, int64_t max_rows, uint64_t total_rows,
-                                 int D, float lr, T* tables, uint32_t* status) {
+                                 const unsigned long long* __restrict__ count, int64_t max_rows, uint64_t first,
+                                 uint64_t n_rows, int D, float lr, T* tables, uint32_t* status) {
     const int lane = threadIdx.x & 31;
     const int64_t U = min((int64_t)*count, max_rows);
     const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
         const uint64_t r = rows[u];
-        if (r >= total_rows) {
+        if (r < first || r - first >= n_rows) {
             if (lane == 0) flag(status, ENGRAM_ERR_INDEX);
             continue;
         }
+        const uint64_t q = r - first;
         for (int c = lane; c < D; c += 32) {
-            T& x = tables[r * D + c];
+            T& x = tables[q * D + c];
             from_f(x, fmaf(-lr, grad[u * D + c], to_f(x)));
         }
+    }
+}
+
+// Routing of a rank's (row, gradient) pairs to the shards that own the rows
+// (shard g holds global rows [g * per, (g + 1) * per)).  First the count of
+// pairs for every shard, then every pair copied into its shard's segment of
+// the send buffers (segments in shard order; within a segment, in the order
+// the atomics give: the owner's sum does not depend on it, because a rank
+// sends every row at most once).
+__global__ void route_count_kernel(const uint64_t* __restrict__ rows, const unsigned long long* __restrict__ n_pairs,
+                                   int64_t max_rows, uint64_t per, uint64_t total, int n_shards,
+                                   unsigned long long* counts, uint32_t* status) {
+    __shared__ unsigned int s_cnt[kMaxShards];
+    if (threadIdx.x < kMaxShards) s_cnt[threadIdx.x] = 0u;
+    __syncthreads();
+    const int64_t U = min((int64_t)*n_pairs, max_rows);
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < U; u += (int64_t)gridDim.x * blockDim.x) {
+        const uint64_t r = rows[u];
+        if (r >= total) {
+            flag(status, ENGRAM_ERR_INDEX);
+            continue;
+        }
+        atomicAdd(&s_cnt[(int)(r / per)], 1u);
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < n_shards && s_cnt[threadIdx.x])
+        atomicAdd(counts + threadIdx.x, (unsigned long long)s_cnt[threadIdx.x]);
+}
+
+// one warp per pair: lane 0 takes the slot, the warp copies the D floats
+__global__ void route_place_kernel(const uint64_t* __restrict__ rows, const float* __restrict__ grad,
+                                   const unsigned long long* __restrict__ n_pairs, int64_t max_rows, uint64_t per,
+                                   uint64_t total, const unsigned long long* __restrict__ counts,
+                                   unsigned long long* cursor, int D, uint64_t* __restrict__ send_rows,
+                                   float* __restrict__ send_grad) {
+    const int lane = threadIdx.x & 31;
+    const int64_t U = min((int64_t)*n_pairs, max_rows);
+    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
+        const uint64_t r = rows[u];
+        if (r >= total) continue;
+        const int o = (int)(r / per);
+        unsigned long long slot = 0ull;
+        if (lane == 0) {
+            unsigned long long base = 0ull;
+            for (int g = 0; g < o; ++g) base += counts[g];
+            slot = base + atomicAdd(cursor + o, 1ull);
+            send_rows[slot] = r;
+        }
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        const float4* in = reinterpret_cast<const float4*>(grad + u * D);
+        float4* out = reinterpret_cast<float4*>(send_grad + (int64_t)slot * D);
+        for (int q = lane; q < D / 4; q += 32) out[q] = in[q];
     }
 }
 
@@ -291,6 +392,66 @@ GradWs grad_carve(void* base, int64_t n) {
 
 constexpr int64_t kMaxGradLookups = (int64_t)kScanBlock * kScanBlock;   // two scan levels of 4096
 
+// Clear the scratch, then steps 1-4 over n keyed gradient slices: the
+// distinct rows into rows_out, their ordered sums into grad_out, the count
+// into *n_unique.  `what` names the caller in errors.
+template <typename Keys, typename Slices>
+engram_status dedupe_and_sum(engram_ctx* c, const GradWs& w, int64_t n, Keys keys, Slices slices, int D,
+                             uint64_t* rows_out, float* grad_out, uint64_t* n_unique, const char* what,
+                             cudaStream_t s) {
+    const size_t cap = set_slots(std::max<int64_t>(1, n));
+    cudaError_t e = cudaMemsetAsync(w.keys, 0, cap * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(w.count, 0, 8, s);
+    if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.bucket, 0, (size_t)n * 4, s);
+    if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.cursor, 0, (size_t)n * 4, s);
+    if (e != cudaSuccess) return cuda_fail(what, e);
+    if (n > 0) {
+        const int threads = 256;
+        const int blocks = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)c->num_sms * 8);
+        const uint32_t mask = (uint32_t)(cap - 1);
+        prof_begin(c, s, "grad_dedupe");
+        grad_insert_kernel<<<blocks, threads, 0, s>>>(keys, n, w.keys, w.vals, mask, rows_out, w.count, c->d_status);
+        grad_id_kernel<<<blocks, threads, 0, s>>>(keys, n, w.keys, w.vals, mask, w.lid, w.bucket);
+        prof_end(c, s);
+        // segment starts: scan of the bucket sizes (ids >= U have empty buckets)
+        const int64_t nb1 = (n + kScanBlock - 1) / kScanBlock;
+        const int64_t nb2 = (nb1 + kScanBlock - 1) / kScanBlock;
+        prof_begin(c, s, "grad_scan");
+        scan_block_kernel<<<(unsigned)nb1, kScanThreads, 0, s>>>(w.bucket, n, w.start, w.bsum1);
+        scan_block_kernel<<<(unsigned)nb2, kScanThreads, 0, s>>>(w.bsum1, nb1, w.bsum1, w.bsum2);
+        scan_block_kernel<<<1, kScanThreads, 0, s>>>(w.bsum2, nb2, w.bsum2, w.bsum3);
+        if (nb2 > 1) scan_add_kernel<<<(unsigned)((nb1 + 255) / 256), 256, 0, s>>>(w.bsum1, nb1, w.bsum2);
+        if (nb1 > 1) scan_add_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.start, n, w.bsum1);
+        prof_end(c, s);
+        prof_begin(c, s, "grad_place");
+        grad_place_kernel<<<blocks, threads, 0, s>>>(w.lid, n, w.start, w.cursor, w.seg);
+        prof_end(c, s);
+        prof_begin(c, s, "grad_reduce");
+        const int rblocks = (int)std::min<int64_t>((n + 7) / 8, (int64_t)c->num_sms * 16);
+        grad_reduce_kernel<<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted, slices, D, grad_out);
+        prof_end(c, s);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(n_unique, w.count, 8, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(what, e);
+    return ENGRAM_OK;
+}
+
+uint64_t total_rows(const engram_ctx* c) {
+    uint64_t total = 0;
+    for (int j = 0; j < c->J; ++j) total += c->cfg.rows[j];
+    return total;
+}
+
+template <typename T>
+void launch_sgd(engram_ctx* c, const uint64_t* rows, const float* grad, const uint64_t* n_unique, int64_t max_rows,
+                uint64_t first, uint64_t n_rows, void* tables, float lr, cudaStream_t s) {
+    const int blocks = (int)std::min<int64_t>((max_rows + 7) / 8, (int64_t)c->num_sms * 16);
+    table_sgd_kernel<T><<<blocks, 256, 0, s>>>(rows, grad, reinterpret_cast<const unsigned long long*>(n_unique),
+                                               max_rows, first, n_rows, c->cfg.row_dim, lr, static_cast<T*>(tables),
+                                               c->d_status);
+}
+
 }  // namespace
 }  // namespace engram
 
@@ -323,57 +484,19 @@ engram_status engram_table_grad(engram_ctx* c, const uint32_t* idx, int64_t n_to
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
     prof_reset(c);
-    const size_t cap = set_slots(std::max<int64_t>(1, n));
-    cudaError_t e = cudaMemsetAsync(w.keys, 0, cap * 8, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(w.count, 0, 8, s);
-    if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.bucket, 0, (size_t)n * 4, s);
-    if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.cursor, 0, (size_t)n * 4, s);
-    if (e != cudaSuccess) return cuda_fail("table gradient: clearing the scratch", e);
-    if (n == 0) {
-        e = cudaMemcpyAsync(n_unique, w.count, 8, cudaMemcpyDeviceToDevice, s);
-        return e == cudaSuccess ? ENGRAM_OK : cuda_fail("table gradient: count", e);
-    }
     GradGeo g{};
     for (int j = 0; j < c->J; ++j) {
         g.row_off[j] = c->gp.row_off[j];
         g.rows[j] = c->gp.rows[j];
     }
     g.J = c->J;
-    const int threads = 256;
-    const int blocks = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)c->num_sms * 8);
-    const uint32_t mask = (uint32_t)(cap - 1);
-    prof_begin(c, s, "grad_dedupe");
-    grad_insert_kernel<<<blocks, threads, 0, s>>>(idx, n, g, w.keys, w.vals, mask, rows_out, w.count, c->d_status);
-    grad_id_kernel<<<blocks, threads, 0, s>>>(idx, n, g, w.keys, w.vals, mask, w.lid, w.bucket);
-    prof_end(c, s);
-    // segment starts: scan of the bucket sizes (ids >= U have empty buckets)
-    const int64_t nb1 = (n + kScanBlock - 1) / kScanBlock;
-    const int64_t nb2 = (nb1 + kScanBlock - 1) / kScanBlock;
-    prof_begin(c, s, "grad_scan");
-    scan_block_kernel<<<(unsigned)nb1, kScanThreads, 0, s>>>(w.bucket, n, w.start, w.bsum1);
-    scan_block_kernel<<<(unsigned)nb2, kScanThreads, 0, s>>>(w.bsum1, nb1, w.bsum1, w.bsum2);
-    scan_block_kernel<<<1, kScanThreads, 0, s>>>(w.bsum2, nb2, w.bsum2, w.bsum3);
-    if (nb2 > 1) scan_add_kernel<<<(unsigned)((nb1 + 255) / 256), 256, 0, s>>>(w.bsum1, nb1, w.bsum2);
-    if (nb1 > 1) scan_add_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.start, n, w.bsum1);
-    prof_end(c, s);
-    prof_begin(c, s, "grad_place");
-    grad_place_kernel<<<blocks, threads, 0, s>>>(w.lid, n, w.start, w.cursor, w.seg);
-    prof_end(c, s);
-    prof_begin(c, s, "grad_reduce");
-    const int rblocks = (int)std::min<int64_t>((n + 7) / 8, (int64_t)c->num_sms * 16);
+    const int D = c->cfg.row_dim;
     if (c->cfg.dtype == ENGRAM_BF16)
-        grad_reduce_kernel<__nv_bfloat16><<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted,
-                                                                  static_cast<const __nv_bfloat16*>(d_e), c->J,
-                                                                  c->cfg.row_dim, grad_out);
-    else
-        grad_reduce_kernel<float><<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted,
-                                                          static_cast<const float*>(d_e), c->J, c->cfg.row_dim,
-                                                          grad_out);
-    prof_end(c, s);
-    e = cudaGetLastError();
-    if (e == cudaSuccess) e = cudaMemcpyAsync(n_unique, w.count, 8, cudaMemcpyDeviceToDevice, s);
-    if (e != cudaSuccess) return cuda_fail("table gradient launches", e);
-    return ENGRAM_OK;
+        return dedupe_and_sum(c, w, n, LookupKeys{idx, g},
+                              LookupSlices<__nv_bfloat16>{static_cast<const __nv_bfloat16*>(d_e), c->J, D}, D,
+                              rows_out, grad_out, n_unique, "table gradient", s);
+    return dedupe_and_sum(c, w, n, LookupKeys{idx, g}, LookupSlices<float>{static_cast<const float*>(d_e), c->J, D},
+                          D, rows_out, grad_out, n_unique, "table gradient", s);
 }
 
 engram_status engram_table_sgd(engram_ctx* c, const uint64_t* rows, const float* grad, const uint64_t* n_unique,
@@ -388,22 +511,110 @@ engram_status engram_table_sgd(engram_ctx* c, const uint64_t* rows, const float*
     }
     engram_status st = check_device(c);
     if (st != ENGRAM_OK) return st;
-    uint64_t total = 0;
-    for (int j = 0; j < c->J; ++j) total += c->cfg.rows[j];
     prof_reset(c);
     prof_begin(c, s, "table_sgd");
-    const int blocks = (int)std::min<int64_t>((max_rows + 7) / 8, (int64_t)c->num_sms * 16);
     if (c->cfg.dtype == ENGRAM_BF16)
-        table_sgd_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-            rows, grad, reinterpret_cast<const unsigned long long*>(n_unique), max_rows, total, c->cfg.row_dim, lr,
-            static_cast<__nv_bfloat16*>(tables), c->d_status);
+        launch_sgd<__nv_bfloat16>(c, rows, grad, n_unique, max_rows, 0, total_rows(c), tables, lr, s);
     else
-        table_sgd_kernel<float><<<blocks, 256, 0, s>>>(rows, grad, reinterpret_cast<const unsigned long long*>(n_unique),
-                                                       max_rows, total, c->cfg.row_dim, lr,
-                                                       static_cast<float*>(tables), c->d_status);
+        launch_sgd<float>(c, rows, grad, n_unique, max_rows, 0, total_rows(c), tables, lr, s);
     prof_end(c, s);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ENGRAM_OK : cuda_fail("table update launch", e);
+}
+
+size_t engram_grad_route_workspace_bytes(const engram_ctx* c) {
+    return c ? (size_t)256 : 0;
+}
+
+engram_status engram_grad_route(engram_ctx* c, int32_t n_shards, const uint64_t* rows, const float* grad,
+                                const uint64_t* n_pairs, int64_t max_rows, uint64_t* send_rows, float* send_grad,
+                                int64_t* send_counts, void* workspace, size_t workspace_bytes, cudaStream_t s) {
+    if (!c) return inval("null context");
+    if (n_shards < 1 || n_shards > kMaxShards) return inval("n_shards must be in 1..16");
+    if (max_rows < 0) return inval("max_rows must be >= 0");
+    if (max_rows > kMaxGradLookups) return inval("max_rows must be at most 2^24 pairs");
+    if (!n_pairs || !send_counts || !workspace) return inval("null count, send_counts or workspace pointer");
+    if (max_rows > 0 && (!rows || !grad || !send_rows || !send_grad)) return inval("null tensor pointer");
+    if (!aligned16(grad) || !aligned16(send_grad)) return inval("grad and send_grad must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    if (workspace_bytes < engram_grad_route_workspace_bytes(c)) return ENGRAM_E_NOMEM;
+    engram_status st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    const uint64_t total = total_rows(c);
+    const uint64_t per = (total + (uint64_t)n_shards - 1) / (uint64_t)n_shards;
+    unsigned long long* counts = reinterpret_cast<unsigned long long*>(send_counts);
+    unsigned long long* cursor = static_cast<unsigned long long*>(workspace);
+    prof_reset(c);
+    cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)n_shards * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(cursor, 0, (size_t)n_shards * 8, s);
+    if (e != cudaSuccess) return cuda_fail("gradient routing: clearing the counts", e);
+    if (max_rows == 0) return ENGRAM_OK;
+    const int D = c->cfg.row_dim;
+    prof_begin(c, s, "grad_route");
+    const int cblocks = (int)std::min<int64_t>((max_rows + 255) / 256, (int64_t)c->num_sms * 4);
+    route_count_kernel<<<cblocks, 256, 0, s>>>(rows, reinterpret_cast<const unsigned long long*>(n_pairs), max_rows,
+                                               per, total, n_shards, counts, c->d_status);
+    const int pblocks = (int)std::min<int64_t>((max_rows + 7) / 8, (int64_t)c->num_sms * 16);
+    route_place_kernel<<<pblocks, 256, 0, s>>>(rows, grad, reinterpret_cast<const unsigned long long*>(n_pairs),
+                                               max_rows, per, total, counts, cursor, D, send_rows, send_grad);
+    prof_end(c, s);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? ENGRAM_OK : cuda_fail("gradient routing launches", e);
+}
+
+size_t engram_grad_combine_workspace_bytes(const engram_ctx* c, int64_t n_pairs) {
+    if (!c || n_pairs < 0) return 0;
+    return grad_carve(nullptr, std::max<int64_t>(1, n_pairs)).bytes;
+}
+
+engram_status engram_grad_combine(engram_ctx* c, int32_t n_shards, int32_t shard, const uint64_t* pair_rows,
+                                  const float* pair_grad, int64_t n_pairs, uint64_t* rows_out, float* grad_out,
+                                  uint64_t* n_unique, void* workspace, size_t workspace_bytes, cudaStream_t s) {
+    if (!c) return inval("null context");
+    int64_t lo = 0, cnt = 0;
+    engram_status st = engram_shard_range(c, n_shards, shard, &lo, &cnt);
+    if (st != ENGRAM_OK) return st;
+    if (n_pairs < 0) return inval("n_pairs must be >= 0");
+    if (n_pairs > kMaxGradLookups) return inval("n_pairs must be at most 2^24");
+    if (!n_unique || !workspace) return inval("null n_unique or workspace pointer");
+    if (n_pairs > 0 && (!pair_rows || !pair_grad || !rows_out || !grad_out)) return inval("null tensor pointer");
+    if (!aligned16(pair_grad) || !aligned16(grad_out)) return inval("pair_grad and grad_out must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return inval("workspace must be 256-byte aligned");
+    GradWs w = grad_carve(workspace, std::max<int64_t>(1, n_pairs));
+    if (workspace_bytes < w.bytes) return ENGRAM_E_NOMEM;
+    st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    prof_reset(c);
+    const int D = c->cfg.row_dim;
+    return dedupe_and_sum(c, w, n_pairs, PairKeys{pair_rows, (uint64_t)lo, (uint64_t)(lo + cnt)},
+                          PairSlices{pair_grad, D}, D, rows_out, grad_out, n_unique, "gradient combine", s);
+}
+
+engram_status engram_shard_sgd(engram_ctx* c, int32_t n_shards, int32_t shard, const uint64_t* rows,
+                               const float* grad, const uint64_t* n_unique, int64_t max_rows, void* shard_table,
+                               float lr, cudaStream_t s) {
+    if (!c) return inval("null context");
+    int64_t lo = 0, cnt = 0;
+    engram_status st = engram_shard_range(c, n_shards, shard, &lo, &cnt);
+    if (st != ENGRAM_OK) return st;
+    if (max_rows < 0) return inval("max_rows must be >= 0");
+    if (max_rows == 0) return ENGRAM_OK;
+    if (!rows || !grad || !n_unique || (cnt > 0 && !shard_table)) return inval("null tensor pointer");
+    if (c->cfg.dtype == ENGRAM_FP8) {
+        set_error("engram_shard_sgd: FP8 tables are not trained here");
+        return ENGRAM_E_UNSUPPORTED;
+    }
+    st = check_device(c);
+    if (st != ENGRAM_OK) return st;
+    prof_reset(c);
+    prof_begin(c, s, "table_sgd");
+    if (c->cfg.dtype == ENGRAM_BF16)
+        launch_sgd<__nv_bfloat16>(c, rows, grad, n_unique, max_rows, (uint64_t)lo, (uint64_t)cnt, shard_table, lr, s);
+    else
+        launch_sgd<float>(c, rows, grad, n_unique, max_rows, (uint64_t)lo, (uint64_t)cnt, shard_table, lr, s);
+    prof_end(c, s);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ENGRAM_OK : cuda_fail("shard update launch", e);
 }
 
 }  // extern "C"

@@ -384,6 +384,61 @@ ENGRAM_API engram_status engram_table_sgd(engram_ctx* ctx, const uint64_t* rows,
                                           const uint64_t* n_unique, int64_t max_rows, void* tables, float lr,
                                           cudaStream_t stream);
 
+/* ------------------------------------------------------------ table backward across shards
+ *
+ * With the tables sharded (shard g holds the global rows engram_shard_range
+ * gives it, one shard per rank), the backward sends every accessed row's
+ * gradient to the shard that stores it ("DeepSeek AI II" digest, section
+ * "DeepSeek Engram", the training paragraph; the Synced repost, section
+ * "System efficiency: decoupling compute and storage": the rows are gathered
+ * to each GPU by an all-to-all in the forward and their gradients are
+ * scattered back to the owners in the backward).  Three steps per rank:
+ *
+ * engram_grad_route: this rank's (row, gradient) pairs (engram_table_grad's
+ * rows_out, grad_out and DEVICE *n_pairs; pairs beyond max_rows are ignored)
+ * split by owner.  Writes send_counts[g] (DEVICE int64, n_shards entries) =
+ * the number of pairs for shard g, and the pairs themselves into send_rows
+ * (uint64 global rows) and send_grad ([.][D] fp32, 16-byte aligned), shard
+ * 0's segment first, then shard 1's, and so on (capacity max_rows each).
+ * Within a segment the order is whatever the device's atomics give.  A row
+ * beyond the tables sets ENGRAM_ERR_INDEX and is not sent.  Scratch:
+ * engram_grad_route_workspace_bytes(ctx) bytes, 256-byte aligned.
+ *
+ * The exchange itself is the caller's: an all-to-all (NCCL's, through
+ * torch.distributed.all_to_all_single) of send_counts, then of the segments,
+ * which leaves on every rank the pairs for its shard from rank 0, then rank
+ * 1, and so on.
+ *
+ * engram_grad_combine: the pairs received by shard `shard` of n_shards
+ * (pair_rows uint64 [n_pairs], pair_grad [n_pairs][D] fp32, 16-byte aligned;
+ * n_pairs <= 2^24 is a HOST count).  Writes the distinct rows into rows_out
+ * (global rows), their summed gradients into grad_out ([.][D] fp32, 16-byte
+ * aligned; capacity n_pairs each) and their number into DEVICE *n_unique.
+ * Each row's sum runs in increasing pair order, i.e. in rank order when the
+ * pairs arrive in rank order, in fp32; since every rank sends a row at most
+ * once, the result does not depend on the order within a rank's segment.  A
+ * pair whose row the shard does not hold sets ENGRAM_ERR_INDEX and is
+ * dropped.  Scratch: engram_grad_combine_workspace_bytes(ctx, n_pairs) bytes,
+ * 256-byte aligned.
+ *
+ * engram_shard_sgd: engram_table_sgd on one shard: shard_table holds the
+ * shard's rows back to back ([n_rows][D], the model dtype), rows are global;
+ * shard_table[row - first_row] -= lr * grad for u < min(*n_unique,
+ * max_rows).  A row outside the shard sets ENGRAM_ERR_INDEX and is skipped. */
+ENGRAM_API size_t engram_grad_route_workspace_bytes(const engram_ctx* ctx);
+ENGRAM_API engram_status engram_grad_route(engram_ctx* ctx, int32_t n_shards, const uint64_t* rows,
+                                           const float* grad, const uint64_t* n_pairs, int64_t max_rows,
+                                           uint64_t* send_rows, float* send_grad, int64_t* send_counts,
+                                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+ENGRAM_API size_t engram_grad_combine_workspace_bytes(const engram_ctx* ctx, int64_t n_pairs);
+ENGRAM_API engram_status engram_grad_combine(engram_ctx* ctx, int32_t n_shards, int32_t shard,
+                                             const uint64_t* pair_rows, const float* pair_grad, int64_t n_pairs,
+                                             uint64_t* rows_out, float* grad_out, uint64_t* n_unique,
+                                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+ENGRAM_API engram_status engram_shard_sgd(engram_ctx* ctx, int32_t n_shards, int32_t shard, const uint64_t* rows,
+                                          const float* grad, const uint64_t* n_unique, int64_t max_rows,
+                                          void* shard_table, float lr, cudaStream_t stream);
+
 /* engram_forward for callers that cannot allocate device memory (an engine
  * callback where allocation is forbidden, a process whose device memory is
  * all owned by another allocator, a loop that cannot afford cudaMalloc's
