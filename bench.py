@@ -538,6 +538,158 @@ def run_host_tier(args, wl, rank, world, dev):
     print(json.dumps(line), flush=True)
 
 
+def table_grad_bytes(n: int, J: int, D: int, es: int, U: int) -> dict:
+    """Algorithmic bytes of one table update from dL/de: what the step must
+    read and write at least once.  n tokens, J tables of D-wide rows in
+    `es`-byte elements, U distinct rows touched.
+      grad_reduce: every lookup's slice of dL/de read once (n*J*D*es), each
+        distinct row's fp32 sum written once (U*D*4);
+      table_sgd: the sums and row ids read (U*D*4 + U*8), the touched table
+        rows read and written (2*U*D*es);
+      step: the two, plus the indices read (n*J*4) and the row ids written
+        (U*8) by the dedupe."""
+    reduce_b = n * J * D * es + U * D * 4
+    sgd_b = U * D * 4 + U * 8 + 2 * U * D * es
+    return {"grad_reduce": reduce_b, "table_sgd": sgd_b, "step": reduce_b + sgd_b + n * J * 4 + U * 8}
+
+
+def run_table_grad(args, wl, rank, world, dev):
+    """The tables' training update from dL/de: per step, engram_table_grad
+    (dedupe, scan, place, ordered per-row sums) then engram_table_sgd on the
+    resident tables, with the batch's indices and a seeded dL/de resident in
+    HBM.  The row count is read back once after the warm-up, never inside a
+    step (the update takes it from device memory)."""
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_02_b200 as eb
+
+    if wl.dtype != "bf16":
+        raise SystemExit("--table-grad times bf16 workloads")
+    inp = synth.Inputs(wl)
+    dd = inp.device_dense(dev)
+    tables = inp.device_tables(dev)
+    n, J, D, es = wl.n_tok, wl.J, wl.D, 2
+    cfg = eb.make_config(orders=wl.orders, heads=wl.K, rows=[int(x) for x in inp.rows], mult=inp.mult,
+                         row_dim=D, hidden=wl.d, conv_width=wl.w, vocab=wl.V, canon_vocab=wl.Vc,
+                         dtype=eb.ENGRAM_BF16)
+    eng = eb.Engram(cfg)
+    idx = torch.empty(n, J, dtype=torch.int32, device=dev)
+    tok = torch.from_numpy(inp.tok).to(dev)
+    eb.engram_hash(eng.ctx, tok, dd["P"], wl.B, wl.T, wl.T, 0, idx)
+    g = torch.Generator(device=dev).manual_seed(wl.seed + 77)
+    d_e = (torch.randn(n, wl.d_mem, device=dev, generator=g) * 1e-2).to(torch.bfloat16)
+    cap = n * J
+    rows = torch.empty(cap, dtype=torch.int64, device=dev)
+    grad = torch.empty(cap, D, dtype=torch.float32, device=dev)
+    cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+    ws_bytes = eb.engram_table_grad_workspace_bytes(eng.ctx, n)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    lr = 1e-3
+    flush = L2Flush(dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        eb.engram_table_grad(eng.ctx, idx, n, d_e, rows, grad, cnt, ws, ws_bytes)
+        eb.engram_table_sgd(eng.ctx, rows, grad, cnt, cap, tables, lr)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    st, flags = eng.status()
+    if st != eb.ENGRAM_OK:
+        raise RuntimeError(f"device status {st} flags {flags:#x} after warm-up")
+    U = int(cnt.item())
+    K = args.steps
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = []
+    with ClockSampler(dev.index) as clocks:
+        for _ in range(K):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+    step_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev])), world, dev)
+
+    # per-kernel durations from the library's events, in separate profiled steps
+    eb.engram_profile_enable(eng.ctx, True)
+    rec = []
+    for i in range(K + args.warmup):
+        flush()
+        eb.engram_table_grad(eng.ctx, idx, n, d_e, rows, grad, cnt, ws, ws_bytes)
+        p1 = eb.engram_profile_read(eng.ctx)
+        eb.engram_table_sgd(eng.ctx, rows, grad, cnt, cap, tables, lr)
+        p2 = eb.engram_profile_read(eng.ctx)
+        if i >= args.warmup:
+            rec.append(p1 + p2)
+    eb.engram_profile_enable(eng.ctx, False)
+    names = [nm for nm, _ in rec[0]]
+    kms = {nm: float(np.mean([r[j][1] for r in rec])) for j, nm in enumerate(names)}
+    st, flags = eng.status()
+    if st != eb.ENGRAM_OK:
+        raise RuntimeError(f"device status {st} flags {flags:#x} after timing")
+    if rank != 0:
+        return
+    hbm, _, _, peak_src = _peaks()
+    nbytes = table_grad_bytes(n, J, D, es, U)
+    # the reduce is two launches (short segments by lane groups, long ones a
+    # CTA each) over one set of algorithmic bytes: its roofline takes both
+    kms_r = {nm: ms for nm, ms in kms.items() if nm != "grad_reduce_long"}
+    kms_r["grad_reduce"] = kms.get("grad_reduce", 0.0) + kms.get("grad_reduce_long", 0.0)
+    kernels = {nm: {"ms": ms} for nm, ms in kms.items()}
+    for nm, ms in kms_r.items():
+        if nm in nbytes and ms > 0:
+            gbs = nbytes[nm] / (ms / 1e3) / 1e9
+            kernels.setdefault(nm, {})
+            kernels[nm].update(bound="hbm", achieved=gbs, unit="GB/s", frac=gbs / hbm,
+                               **({"ms_both_launches": ms} if nm == "grad_reduce" else {}))
+    dom = max(kms_r, key=kms_r.get)
+    timed_dom = dom if dom in nbytes else max((nm for nm in kms_r if nm in nbytes), key=kms_r.get)
+    dk = kernels[timed_dom]
+    step_gbs = nbytes["step"] / (step_ms / 1e3) / 1e9
+    # launches per step: dedupe 2, scan 3 blocks + the adds, place 1, reduce 2 (short and long segments), sgd 1
+    nb1 = (cap + 4095) // 4096
+    nb2 = (nb1 + 4095) // 4096
+    per_step = 2 + 3 + (1 if nb2 > 1 else 0) + (1 if nb1 > 1 else 0) + 1 + 2 + 1
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        m = min(n, max(1, args.cpu_tokens))
+        idx_np = idx[:m].cpu().numpy().view(np.uint32)
+        de_np = d_e[:m].float().cpu().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.table_grad(idx_np, inp.rows, de_np, D)
+        cpu_s = time.perf_counter() - t0
+        cpu = {"value": m / cpu_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"the gradient of the first {m} tokens' lookups ({cpu_s:.2f} s), numpy fp64 "
+                         "(np.unique + np.add.at), no table update", **host_cpu()}
+    line = {
+        "metric": "Engram table backward (sparse gradient from dL/de + SGD update) tokens/sec on 1 B200",
+        "value": job_tokens_per_s(n, world, step_ms), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: the workload's seeded Zipf tokens hashed on the device, dL/de ~ N(0, 1e-4) bf16",
+        "config": {"workload": describe(wl), "B": wl.B, "seq_len": wl.T, "tokens_per_step": n * world,
+                   "lookups": cap, "distinct_rows": U, "parallelism": f"replicas x{world} (no collective)",
+                   "l2": L2_DESC, "launch": "eager"},
+        "roofline": {"kernel": timed_dom + (" (+ grad_reduce_long)" if timed_dom == "grad_reduce" else ""),
+                     "bound": "hbm", "achieved": dk.get("achieved"), "peak": hbm,
+                     "unit": "GB/s", "frac": dk.get("frac"), "traffic": None,
+                     "peak_source": f"{peak_src} HBM copy",
+                     "algorithmic": f"{nbytes[timed_dom] / 1e6:.1f} MB per launch"},
+        "step_bytes": {"algorithmic_mb": nbytes["step"] / 1e6, "achieved_gbs": step_gbs, "frac": step_gbs / hbm},
+        "kernels": kernels, "kernels_ms": kms, "dominant_kernel": dom,
+        "cpu_baseline": cpu, "e2e": None, "gpu_launches": per_step * K, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def e2e_host(args, eng, inp, dd, tables, h, state, wl, tdt, es, n, K, flush, stream, world, dev):
     """The same step end to end through the C ABI with HOST buffers:
     engram_forward_host copies the ids and h in from pinned host memory and Y
@@ -608,6 +760,9 @@ def main():
                     help="oracle sample per reference step (0: sized so the run takes about 90 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph replay")
+    ap.add_argument("--table-grad", action="store_true",
+                    help="time the tables' training update (engram_table_grad + engram_table_sgd) instead of the "
+                         "forward")
     ap.add_argument("--branches", type=int, default=1,
                     help="multi-branch module: M residual branches (own W_K, h, gate and Y each; shared tables, "
                          "W_V and conv)")
@@ -651,6 +806,11 @@ def main():
     wl = replica_workload(wl, rank, world)
     if wl.host_tables:
         run_host_tier(args, wl, rank, world, dev)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    if args.table_grad:
+        run_table_grad(args, wl, rank, world, dev)
         if world > 1:
             dist.destroy_process_group()
         return

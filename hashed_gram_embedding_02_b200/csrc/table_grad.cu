@@ -18,9 +18,11 @@
 //      4096-element blocks), the start of every row's segment.
 //   3. place: every lookup writes its position into its row's segment (in
 //      the order the atomics give).
-//   4. reduce: one warp per row orders its segment by position (each lookup's
-//      rank is the number of smaller positions in the segment) and sums the
-//      slices of dL/de in that order, in fp32, 16 bytes of the row per lane.
+//   4. reduce: a group of lanes per row (as many as the row has 16-byte
+//      chunks, rounded up to a power of two) orders its segment by position
+//      (each lookup's rank is the number of smaller positions in the segment)
+//      and sums the slices of dL/de in that order, in fp32; a row looked up
+//      once skips the ordering.
 // The cost of step 4 grows with the square of a row's lookup count: fine for
 // Zipf batches (the largest segments hold hundreds of lookups), slow for a
 // degenerate batch in which one n-gram fills it.
@@ -221,32 +223,69 @@ struct PairSlices {
     __device__ __forceinline__ const float* at(uint32_t pos) const { return g + (int64_t)pos * D; }
 };
 
-// One warp per distinct row: order the segment by position (into `sorted`,
-// each element's rank = the count of smaller positions), then sum the
-// gradient slices in that order.  Lane l owns the row's 16-byte chunks
-// l, l + 32, ... (D*elem/16 chunks in all).
+constexpr uint32_t kSmallSeg = 32;   // the longest segment a lane group orders by itself
+constexpr int kTile = 2048;          // segment positions staged in shared memory at a time for ranking
+constexpr int kPosCap = 4096;        // longest segment whose ordered positions stay in shared memory
+constexpr int kStage = 1024;         // 16-byte slice chunks staged per batch of the long-segment sum
+constexpr int kHeavyThreads = 256;
+
+// One group of `gs` lanes per distinct row: gs is a power of two, at least
+// the row's count of 16-byte chunks (D*elem/16) and at most 32, so a warp
+// takes 32 / gs rows at a time and no lane idles for 128-wide bf16 rows.
+// Lane l of a group owns its row's chunks l, l + gs, ...  A row looked up
+// once (most rows of a Zipf batch) is its one slice, added to zero in fp32;
+// a row looked up k > 1 times has its segment ordered by position (into
+// `sorted`, each element's rank = the count of smaller positions) and its
+// slices summed in that order, in fp32.  A row looked up more than kSmallSeg
+// times (a Zipf-frequent n-gram) is only listed in `heavy`: ordering it
+// costs k^2 comparisons, which one CTA does far faster than one lane group.
+// Every lane of a group takes the same branches (they share the row), so the
+// group's own mask serves its barrier.
 template <typename Slices>
 __global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint32_t* __restrict__ start,
                                    const uint32_t* __restrict__ bucket, const unsigned long long* __restrict__ count,
-                                   uint32_t* __restrict__ sorted, Slices src, int D, float* __restrict__ grad) {
+                                   uint32_t* __restrict__ sorted, Slices src, int D, int gs,
+                                   float* __restrict__ grad, uint32_t* __restrict__ heavy,
+                                   unsigned long long* n_heavy) {
     using T = typename Slices::Elem;
     constexpr int EPC = 16 / sizeof(T);   // elements per 16-byte chunk
     const int lane = threadIdx.x & 31;
+    const int grp = lane / gs, gl = lane - grp * gs;
+    const unsigned gmask = gs == 32 ? 0xffffffffu : ((1u << gs) - 1u) << (grp * gs);
+    const int rpw = 32 / gs;
     const int64_t U = (int64_t)*count;
-    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t groups = (((int64_t)gridDim.x * blockDim.x) >> 5) * rpw;
     const int chunks = D / EPC;
-    for (int64_t id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; id < U; id += warps) {
+    for (int64_t id = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * rpw + grp; id < U; id += groups) {
         const uint32_t s0 = start[id], k = bucket[id];
+        float* out = grad + id * D;
+        if (k > kSmallSeg) {             // a long segment: a whole CTA orders it (grad_reduce_heavy_kernel)
+            if (gl == 0) heavy[atomicAdd(n_heavy, 1ull)] = (uint32_t)id;
+            continue;
+        }
+        if (k == 1) {
+            const T* slice = src.at(seg[s0]);
+            for (int c = gl; c < chunks; c += gs) {
+                float f[EPC];
+                Vec<T>::load(slice + c * EPC, f);
+                float* o = out + c * EPC;
+#pragma unroll
+                for (int e = 0; e < EPC; e += 4)
+                    *reinterpret_cast<float4*>(o + e) =
+                        make_float4(0.f + f[e], 0.f + f[e + 1], 0.f + f[e + 2], 0.f + f[e + 3]);
+            }
+            continue;
+        }
         const uint32_t* in = seg + s0;
         uint32_t* srt = sorted + s0;
-        for (uint32_t a = lane; a < k; a += 32) {
+        for (uint32_t a = gl; a < k; a += gs) {
             const uint32_t x = in[a];
             uint32_t rank = 0;
             for (uint32_t b = 0; b < k; ++b) rank += in[b] < x;
             srt[rank] = x;
         }
-        __syncwarp();
-        for (int c = lane; c < chunks; c += 32) {
+        __syncwarp(gmask);
+        for (int c = gl; c < chunks; c += gs) {
             float acc[EPC];
 #pragma unroll
             for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
@@ -256,10 +295,109 @@ __global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint3
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) acc[e] += f[e];
             }
-            float* o = grad + id * D + c * EPC;
+            float* o = out + c * EPC;
 #pragma unroll
             for (int e = 0; e < EPC; e += 4) *reinterpret_cast<float4*>(o + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
         }
+    }
+}
+
+// One CTA per listed long segment.  Ordering: every thread ranks its
+// positions (the count of smaller positions in the segment, read from
+// shared-memory tiles of kTile positions, so any length works); the ordered
+// positions go to shared memory when the segment fits (kPosCap), else to
+// `sorted`.  Summing: the CTA stages the slices of up to 1024 / chunks
+// positions at a time in shared memory (all threads loading, several
+// 16-byte chunks each, so one memory round trip serves a whole batch), then
+// thread c adds chunk c of the batch's slices in increasing position order,
+// in fp32: the lane groups' order.  Rows wider than 256 chunks are summed
+// straight from memory, one thread per chunk.  All threads of the CTA share
+// the row and its length, so every barrier is reached by all of them.
+template <typename Slices>
+__global__ void __launch_bounds__(kHeavyThreads)
+    grad_reduce_heavy_kernel(const uint32_t* __restrict__ seg, const uint32_t* __restrict__ start,
+                             const uint32_t* __restrict__ bucket, const uint32_t* __restrict__ heavy,
+                             const unsigned long long* __restrict__ n_heavy, uint32_t* sorted, Slices src, int D,
+                             float* __restrict__ grad) {
+    using T = typename Slices::Elem;
+    constexpr int EPC = 16 / sizeof(T);
+    __shared__ uint32_t tile[kTile];
+    __shared__ uint32_t s_pos[kPosCap];
+    __shared__ uint4 stage[kStage];
+    const int64_t H = (int64_t)*n_heavy;
+    const int chunks = D / EPC;
+    const bool staged = chunks <= kHeavyThreads;
+    const int P = staged ? kStage / chunks : 0;   // positions per staged batch
+    for (int64_t hh = blockIdx.x; hh < H; hh += gridDim.x) {
+        const uint32_t id = heavy[hh];
+        const uint32_t s0 = start[id], k = bucket[id];
+        const uint32_t* in = seg + s0;
+        uint32_t* srt = sorted + s0;
+        const bool local = k <= (uint32_t)kPosCap;
+        for (uint32_t a0 = 0; a0 < k; a0 += blockDim.x) {
+            const uint32_t a = a0 + threadIdx.x;
+            const uint32_t x = a < k ? in[a] : 0u;
+            uint32_t rank = 0;
+            for (uint32_t t0 = 0; t0 < k; t0 += kTile) {
+                const uint32_t m = min((uint32_t)kTile, k - t0);
+                __syncthreads();
+                for (uint32_t b = threadIdx.x; b < m; b += blockDim.x) tile[b] = in[t0 + b];
+                __syncthreads();
+                if (a < k)
+                    for (uint32_t b = 0; b < m; ++b) rank += tile[b] < x;
+            }
+            if (a < k) {
+                if (local) s_pos[rank] = x;
+                else srt[rank] = x;
+            }
+        }
+        __syncthreads();   // the ordered positions (shared or global) are visible to the block
+        float* out = grad + (int64_t)id * D;
+        if (staged) {
+            const int c = threadIdx.x;   // this thread's chunk, when c < chunks
+            float acc[EPC];
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+            for (uint32_t a0 = 0; a0 < k; a0 += (uint32_t)P) {
+                const int np = (int)min((uint32_t)P, k - a0);
+                for (int q = threadIdx.x; q < np * chunks; q += blockDim.x) {
+                    const int p = q / chunks, cc = q - p * chunks;
+                    const uint32_t pos = local ? s_pos[a0 + p] : srt[a0 + p];
+                    stage[q] = *reinterpret_cast<const uint4*>(src.at(pos) + cc * EPC);
+                }
+                __syncthreads();
+                if (c < chunks) {
+                    for (int p = 0; p < np; ++p) {
+                        float f[EPC];
+                        Vec<T>::load(reinterpret_cast<const T*>(&stage[p * chunks + c]), f);
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+                    }
+                }
+                __syncthreads();
+            }
+            if (c < chunks) {
+#pragma unroll
+                for (int e = 0; e < EPC; e += 4)
+                    *reinterpret_cast<float4*>(out + c * EPC + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+            }
+        } else {
+            for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+                float acc[EPC];
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+                for (uint32_t a = 0; a < k; ++a) {
+                    float f[EPC];
+                    Vec<T>::load(src.at(local ? s_pos[a] : srt[a]) + c * EPC, f);
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+                }
+#pragma unroll
+                for (int e = 0; e < EPC; e += 4)
+                    *reinterpret_cast<float4*>(out + c * EPC + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+            }
+        }
+        __syncthreads();
     }
 }
 
@@ -351,6 +489,7 @@ struct GradWs {
     unsigned long long* keys;
     uint32_t* vals;
     unsigned long long* count;
+    unsigned long long* n_heavy;   // rows handed to grad_reduce_heavy_kernel (their ids go into lid)
     uint32_t* lid;
     uint32_t* bucket;
     uint32_t* start;
@@ -377,6 +516,7 @@ GradWs grad_carve(void* base, int64_t n) {
     w.keys = reinterpret_cast<unsigned long long*>(take(cap * 8));
     w.vals = reinterpret_cast<uint32_t*>(take(cap * 4));
     w.count = reinterpret_cast<unsigned long long*>(take(8));
+    w.n_heavy = reinterpret_cast<unsigned long long*>(take(8));
     w.lid = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
     w.bucket = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
     w.start = reinterpret_cast<uint32_t*>(take((size_t)n * 4));
@@ -402,6 +542,7 @@ engram_status dedupe_and_sum(engram_ctx* c, const GradWs& w, int64_t n, Keys key
     const size_t cap = set_slots(std::max<int64_t>(1, n));
     cudaError_t e = cudaMemsetAsync(w.keys, 0, cap * 8, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(w.count, 0, 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(w.n_heavy, 0, 8, s);
     if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.bucket, 0, (size_t)n * 4, s);
     if (e == cudaSuccess && n > 0) e = cudaMemsetAsync(w.cursor, 0, (size_t)n * 4, s);
     if (e != cudaSuccess) return cuda_fail(what, e);
@@ -427,8 +568,18 @@ engram_status dedupe_and_sum(engram_ctx* c, const GradWs& w, int64_t n, Keys key
         grad_place_kernel<<<blocks, threads, 0, s>>>(w.lid, n, w.start, w.cursor, w.seg);
         prof_end(c, s);
         prof_begin(c, s, "grad_reduce");
+        // lanes per row: the row's 16-byte chunks rounded up to a power of two, at most a warp
+        const int chunks = D / (16 / (int)sizeof(typename Slices::Elem));
+        int gs = 1;
+        while (gs < chunks && gs < 32) gs <<= 1;
         const int rblocks = (int)std::min<int64_t>((n + 7) / 8, (int64_t)c->num_sms * 16);
-        grad_reduce_kernel<<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted, slices, D, grad_out);
+        // lid (one entry per lookup, free once the lookups are placed) lists the long segments
+        grad_reduce_kernel<<<rblocks, 256, 0, s>>>(w.seg, w.start, w.bucket, w.count, w.sorted, slices, D, gs,
+                                                   grad_out, w.lid, w.n_heavy);
+        prof_end(c, s);
+        prof_begin(c, s, "grad_reduce_long");
+        grad_reduce_heavy_kernel<<<c->num_sms * 2, kHeavyThreads, 0, s>>>(w.seg, w.start, w.bucket, w.lid,
+                                                                         w.n_heavy, w.sorted, slices, D, grad_out);
         prof_end(c, s);
         e = cudaGetLastError();
     }

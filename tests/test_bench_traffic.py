@@ -53,3 +53,15 @@ def test_captured_traffic_matches_current_sources_or_is_none():
         assert got == (nbytes if current == digest else None)
     assert m.captured_traffic("c2", "no_such_kernel") is None
     assert m.captured_traffic("no_such_workload", "vconv_tc") is None
+
+
+def test_table_grad_bytes_by_hand():
+    """Two tokens, two tables of 4-wide bf16 rows, three distinct rows: the
+    reduce reads 2*2 slices of 8 bytes and writes 3 sums of 16 bytes; the
+    update reads the 3 sums and 3 row ids and reads and writes 3 rows of 8
+    bytes; the step adds the 4 indices read and the 3 row ids written."""
+    m = _bench()
+    b = m.table_grad_bytes(n=2, J=2, D=4, es=2, U=3)
+    assert b["grad_reduce"] == 4 * 8 + 3 * 16
+    assert b["table_sgd"] == 3 * 16 + 3 * 8 + 2 * 3 * 8
+    assert b["step"] == b["grad_reduce"] + b["table_sgd"] + 4 * 4 + 3 * 8
