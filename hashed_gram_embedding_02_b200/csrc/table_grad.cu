@@ -8,8 +8,11 @@
 // the rows E_j[idx_j(t)], the gradient of row r of table j is the sum, over
 // the lookups (t, j) with idx_j(t) = r, of the slice j of dL/de_t.
 //
-// Deterministic: the sum of every row runs in increasing lookup order
-// (t * J + j), whatever order the atomics gave the work.
+// Deterministic: the sum of every row runs in an order fixed by the row's
+// lookups alone, whatever order the atomics gave the work: increasing lookup
+// order (t * J + j) for a row looked up at most 32 times; for a longer row,
+// running sums over every slots-th lookup in increasing order, added in a
+// fixed order (grad_reduce_heavy_kernel).
 //   1. dedupe: every valid lookup's global row (row_off[j] + idx) goes into an
 //      open-addressing set; the thread that claims a row gives it the next id
 //      and records the row; every lookup then learns its row's id and counts
@@ -226,7 +229,7 @@ struct PairSlices {
 constexpr uint32_t kSmallSeg = 32;   // the longest segment a lane group orders by itself
 constexpr int kTile = 2048;          // segment positions staged in shared memory at a time for ranking
 constexpr int kPosCap = 4096;        // longest segment whose ordered positions stay in shared memory
-constexpr int kStage = 1024;         // 16-byte slice chunks staged per batch of the long-segment sum
+constexpr int kStage = 1024;         // 16-byte words of shared memory for the long-segment partial sums
 constexpr int kHeavyThreads = 256;
 
 // One group of `gs` lanes per distinct row: gs is a power of two, at least
@@ -306,11 +309,13 @@ __global__ void grad_reduce_kernel(const uint32_t* __restrict__ seg, const uint3
 // positions (the count of smaller positions in the segment, read from
 // shared-memory tiles of kTile positions, so any length works); the ordered
 // positions go to shared memory when the segment fits (kPosCap), else to
-// `sorted`.  Summing: the CTA stages the slices of up to 1024 / chunks
-// positions at a time in shared memory (all threads loading, several
-// 16-byte chunks each, so one memory round trip serves a whole batch), then
-// thread c adds chunk c of the batch's slices in increasing position order,
-// in fp32: the lane groups' order.  Rows wider than 256 chunks are summed
+// `sorted`.  Summing, for rows of at most 256 chunks: the CTA's threads are
+// `slots` = 256 / chunks running sums per chunk; slot p adds the slices at
+// ordered positions p, p + slots, p + 2 slots, ... in that order, in fp32,
+// and the slots' sums are then added in slot order (0 + s_0 + s_1 + ...).
+// The order is fixed by the row alone, so the result is the same on every
+// run; every thread has several loads in flight instead of one thread per
+// chunk walking the whole segment.  Wider rows are summed in position order
 // straight from memory, one thread per chunk.  All threads of the CTA share
 // the row and its length, so every barrier is reached by all of them.
 template <typename Slices>
@@ -327,7 +332,6 @@ __global__ void __launch_bounds__(kHeavyThreads)
     const int64_t H = (int64_t)*n_heavy;
     const int chunks = D / EPC;
     const bool staged = chunks <= kHeavyThreads;
-    const int P = staged ? kStage / chunks : 0;   // positions per staged batch
     for (int64_t hh = blockIdx.x; hh < H; hh += gridDim.x) {
         const uint32_t id = heavy[hh];
         const uint32_t s0 = start[id], k = bucket[id];
@@ -354,32 +358,41 @@ __global__ void __launch_bounds__(kHeavyThreads)
         __syncthreads();   // the ordered positions (shared or global) are visible to the block
         float* out = grad + (int64_t)id * D;
         if (staged) {
-            const int c = threadIdx.x;   // this thread's chunk, when c < chunks
+            // thread (slot p, chunk c) keeps a running sum of chunk c over the
+            // positions a = p, p + slots, ... in increasing order; the slots'
+            // sums are then added in slot order
+            const int slots = (int)blockDim.x / chunks;
+            const int p = (int)threadIdx.x / chunks, c = (int)threadIdx.x - p * chunks;
             float acc[EPC];
 #pragma unroll
             for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-            for (uint32_t a0 = 0; a0 < k; a0 += (uint32_t)P) {
-                const int np = (int)min((uint32_t)P, k - a0);
-                for (int q = threadIdx.x; q < np * chunks; q += blockDim.x) {
-                    const int p = q / chunks, cc = q - p * chunks;
-                    const uint32_t pos = local ? s_pos[a0 + p] : srt[a0 + p];
-                    stage[q] = *reinterpret_cast<const uint4*>(src.at(pos) + cc * EPC);
-                }
-                __syncthreads();
-                if (c < chunks) {
-                    for (int p = 0; p < np; ++p) {
-                        float f[EPC];
-                        Vec<T>::load(reinterpret_cast<const T*>(&stage[p * chunks + c]), f);
+            if (p < slots) {
+#pragma unroll 4
+                for (uint32_t a = (uint32_t)p; a < k; a += (uint32_t)slots) {
+                    float f[EPC];
+                    Vec<T>::load(src.at(local ? s_pos[a] : srt[a]) + c * EPC, f);
 #pragma unroll
-                        for (int e = 0; e < EPC; ++e) acc[e] += f[e];
-                    }
+                    for (int e = 0; e < EPC; ++e) acc[e] += f[e];
                 }
-                __syncthreads();
             }
-            if (c < chunks) {
+            float* part = reinterpret_cast<float*>(stage);   // slots x chunks x EPC floats
+            if (p < slots) {
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) part[(p * chunks + c) * EPC + e] = acc[e];
+            }
+            __syncthreads();
+            if ((int)threadIdx.x < chunks) {
+                const int cc = (int)threadIdx.x;
+                float tot[EPC];
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) tot[e] = 0.f;
+                for (int q = 0; q < slots; ++q) {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) tot[e] += part[(q * chunks + cc) * EPC + e];
+                }
 #pragma unroll
                 for (int e = 0; e < EPC; e += 4)
-                    *reinterpret_cast<float4*>(out + c * EPC + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                    *reinterpret_cast<float4*>(out + cc * EPC + e) = make_float4(tot[e], tot[e + 1], tot[e + 2], tot[e + 3]);
             }
         } else {
             for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
@@ -578,7 +591,7 @@ engram_status dedupe_and_sum(engram_ctx* c, const GradWs& w, int64_t n, Keys key
                                                    grad_out, w.lid, w.n_heavy);
         prof_end(c, s);
         prof_begin(c, s, "grad_reduce_long");
-        grad_reduce_heavy_kernel<<<c->num_sms * 2, kHeavyThreads, 0, s>>>(w.seg, w.start, w.bucket, w.lid,
+        grad_reduce_heavy_kernel<<<c->num_sms * 4, kHeavyThreads, 0, s>>>(w.seg, w.start, w.bucket, w.lid,
                                                                          w.n_heavy, w.sorted, slices, D, grad_out);
         prof_end(c, s);
         e = cudaGetLastError();

@@ -366,9 +366,13 @@ ENGRAM_API engram_status engram_ipc_close(void* base);
  * (sum_{i<j} M_i + r) and grad_out[u][D] (fp32, 16-byte aligned) its
  * summed gradient, u < U; *n_unique (DEVICE uint64) = U.  Capacity: n_tok*J
  * rows in rows_out and grad_out.  Invalid indices (an n-gram with an
- * invalid id) contribute nothing.  Each row's sum runs in increasing lookup
- * order (t * J + j) in fp32, so the (row, gradient) pairs are the same on
- * every run; which u a row lands at depends on the device's atomics.
+ * invalid id) contribute nothing.  Each row's sum runs in fp32 in an order
+ * fixed by its lookups alone: increasing lookup order (t * J + j) for a row
+ * looked up at most 32 times; for a longer row, S = 256 / (D*elem/16)
+ * running sums, the p-th over the row's lookups p, p + S, p + 2S, ... in
+ * increasing order, then added in order of p.  So the (row, gradient) pairs
+ * are the same on every run; which u a row lands at depends on the device's
+ * atomics.
  * n_tok * J <= 2^24.  Scratch: engram_table_grad_workspace_bytes(ctx, n_tok)
  * bytes, 256-byte aligned.
  *
