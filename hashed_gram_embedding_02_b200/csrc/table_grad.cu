@@ -415,26 +415,38 @@ __global__ void __launch_bounds__(kHeavyThreads)
 }
 
 // tables[row - first] -= lr * grad for rows in [first, first + n_rows), in
-// the tables' dtype (fp32 arithmetic, one rounding to the storage type); one
-// warp per row.  The whole table is first = 0, n_rows = sum of M_j; a shard
-// is its own range.
+// the tables' dtype (fp32 arithmetic, one rounding to the storage type).  The
+// whole table is first = 0, n_rows = sum of M_j; a shard is its own range.
+// A group of `gs` lanes per row (the row's 16-byte table chunks rounded up to
+// a power of two, at most 32), each lane updating whole 16-byte chunks of the
+// row (and reading the matching fp32 gradients as 16-byte vectors).
 template <typename T>
 __global__ void table_sgd_kernel(const uint64_t* __restrict__ rows, const float* __restrict__ grad,
                                  const unsigned long long* __restrict__ count, int64_t max_rows, uint64_t first,
-                                 uint64_t n_rows, int D, float lr, T* tables, uint32_t* status) {
+                                 uint64_t n_rows, int D, int gs, float lr, T* tables, uint32_t* status) {
+    constexpr int EPC = 16 / sizeof(T);   // table elements per 16-byte chunk
     const int lane = threadIdx.x & 31;
+    const int grp = lane / gs, gl = lane - grp * gs;
+    const int rpw = 32 / gs;
     const int64_t U = min((int64_t)*count, max_rows);
-    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
+    const int64_t groups = (((int64_t)gridDim.x * blockDim.x) >> 5) * rpw;
+    const int chunks = D / EPC;
+    for (int64_t u = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * rpw + grp; u < U; u += groups) {
         const uint64_t r = rows[u];
         if (r < first || r - first >= n_rows) {
-            if (lane == 0) flag(status, ENGRAM_ERR_INDEX);
+            if (gl == 0) flag(status, ENGRAM_ERR_INDEX);
             continue;
         }
-        const uint64_t q = r - first;
-        for (int c = lane; c < D; c += 32) {
-            T& x = tables[q * D + c];
-            from_f(x, fmaf(-lr, grad[u * D + c], to_f(x)));
+        T* row = tables + (r - first) * D;
+        const float* g = grad + u * D;
+        for (int c = gl; c < chunks; c += gs) {
+            float x[EPC], gv[EPC];
+            Vec<T>::load(row + c * EPC, x);
+#pragma unroll
+            for (int e = 0; e < EPC; e += 4) Vec<float>::load(g + c * EPC + e, gv + e);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) x[e] = fmaf(-lr, gv[e], x[e]);
+            Vec<T>::store(row + c * EPC, x);
         }
     }
 }
@@ -610,10 +622,13 @@ uint64_t total_rows(const engram_ctx* c) {
 template <typename T>
 void launch_sgd(engram_ctx* c, const uint64_t* rows, const float* grad, const uint64_t* n_unique, int64_t max_rows,
                 uint64_t first, uint64_t n_rows, void* tables, float lr, cudaStream_t s) {
+    const int chunks = c->cfg.row_dim / (16 / (int)sizeof(T));
+    int gs = 1;   // lanes per row: the row's 16-byte chunks rounded up to a power of two, at most a warp
+    while (gs < chunks && gs < 32) gs <<= 1;
     const int blocks = (int)std::min<int64_t>((max_rows + 7) / 8, (int64_t)c->num_sms * 16);
     table_sgd_kernel<T><<<blocks, 256, 0, s>>>(rows, grad, reinterpret_cast<const unsigned long long*>(n_unique),
-                                               max_rows, first, n_rows, c->cfg.row_dim, lr, static_cast<T*>(tables),
-                                               c->d_status);
+                                               max_rows, first, n_rows, c->cfg.row_dim, gs, lr,
+                                               static_cast<T*>(tables), c->d_status);
 }
 
 }  // namespace
@@ -669,6 +684,7 @@ engram_status engram_table_sgd(engram_ctx* c, const uint64_t* rows, const float*
     if (max_rows < 0) return inval("max_rows must be >= 0");
     if (max_rows == 0) return ENGRAM_OK;
     if (!rows || !grad || !n_unique || !tables) return inval("null tensor pointer");
+    if (!aligned16(tables) || !aligned16(grad)) return inval("tables and grad must be 16-byte aligned");
     if (c->cfg.dtype == ENGRAM_FP8) {
         set_error("engram_table_sgd: FP8 tables are not trained here");
         return ENGRAM_E_UNSUPPORTED;
@@ -764,6 +780,7 @@ engram_status engram_shard_sgd(engram_ctx* c, int32_t n_shards, int32_t shard, c
     if (max_rows < 0) return inval("max_rows must be >= 0");
     if (max_rows == 0) return ENGRAM_OK;
     if (!rows || !grad || !n_unique || (cnt > 0 && !shard_table)) return inval("null tensor pointer");
+    if (!aligned16(shard_table) || !aligned16(grad)) return inval("shard_table and grad must be 16-byte aligned");
     if (c->cfg.dtype == ENGRAM_FP8) {
         set_error("engram_shard_sgd: FP8 tables are not trained here");
         return ENGRAM_E_UNSUPPORTED;

@@ -378,8 +378,8 @@ ENGRAM_API engram_status engram_ipc_close(void* base);
  *
  * engram_table_sgd: tables[rows[u]] -= lr * grad[u] for u < min(*n_unique,
  * max_rows), in fp32 arithmetic with one rounding to the tables' dtype;
- * tables as in engram_gather.  A row outside the tables sets
- * ENGRAM_ERR_INDEX and is skipped. */
+ * tables as in engram_gather (16-byte aligned, as is grad).  A row outside
+ * the tables sets ENGRAM_ERR_INDEX and is skipped. */
 ENGRAM_API size_t engram_table_grad_workspace_bytes(const engram_ctx* ctx, int64_t n_tok);
 ENGRAM_API engram_status engram_table_grad(engram_ctx* ctx, const uint32_t* idx, int64_t n_tok, const void* d_e,
                                            uint64_t* rows_out, float* grad_out, uint64_t* n_unique, void* workspace,
