@@ -420,7 +420,10 @@ ENGRAM_API engram_status engram_table_sgd(engram_ctx* ctx, const uint64_t* rows,
  * aligned; capacity n_pairs each) and their number into DEVICE *n_unique.
  * Each row's sum runs in increasing pair order, i.e. in rank order when the
  * pairs arrive in rank order, in fp32; since every rank sends a row at most
- * once, the result does not depend on the order within a rank's segment.  A
+ * once, the result does not depend on the order within a rank's segment.
+ * (A row received more than 32 times, which at most 16 ranks sending it once
+ * each never produce, is summed in engram_table_grad's order for long
+ * rows.)  A
  * pair whose row the shard does not hold sets ENGRAM_ERR_INDEX and is
  * dropped.  Scratch: engram_grad_combine_workspace_bytes(ctx, n_pairs) bytes,
  * 256-byte aligned.

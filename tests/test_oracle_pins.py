@@ -493,6 +493,33 @@ def test_table_grad_conserves_the_total(c1):
     assert len(keys) == len(np.unique((idx.astype(np.int64) + (np.arange(wl.J) * wl.M)[None, :])[valid]))
 
 
+def test_table_grad_of_a_union_is_the_sum_of_the_parts():
+    """The sharded backward rests on linearity: the gradient of the union of
+    the ranks' batches is, row by row, the sum of each rank's own gradient
+    (a row missing from a rank contributes nothing).  Three batches with
+    integer-valued slices, so every sum is exact."""
+    D, J, M = 3, 2, 7
+    rows = np.full(J, M, dtype=np.uint32)
+    rng = np.random.default_rng(11)
+    parts = []
+    for r in range(3):
+        n = 5 + 4 * r
+        idx = rng.integers(0, M, size=(n, J)).astype(np.uint32)
+        idx[0, 1] = 0xFFFFFFFF                                   # an invalid lookup in every batch
+        de = rng.integers(-5, 6, size=(n, J * D)).astype(np.float64)
+        parts.append((idx, de))
+    keys_u, grad_u = oracle.table_grad(np.concatenate([p[0] for p in parts]), rows,
+                                       np.concatenate([p[1] for p in parts]), D)
+    total = {}
+    for idx, de in parts:
+        keys, grad = oracle.table_grad(idx, rows, de, D)
+        for k, g in zip(keys.tolist(), grad):
+            total[k] = total.get(k, 0) + g
+    assert keys_u.tolist() == sorted(total)
+    for k, g in zip(keys_u.tolist(), grad_u):
+        np.testing.assert_array_equal(g, total[k])
+
+
 # ------------------------------------------------------------------ FP8 E4M3 codes
 
 def test_decode_e4m3_hand_values_and_all_codes():
