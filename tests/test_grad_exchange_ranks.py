@@ -4,7 +4,10 @@ numpy (a stand-in for engram_grad_route, which needs a GPU; its side is in
 test_gpu_grad_exchange.py).  Each rank must receive, from every rank in rank
 order, exactly the segment that rank addressed to it, and the per-row sums
 of what it received must equal the sums over all ranks' pairs of its rows
-(integer-valued gradients, so every sum is exact)."""
+(integer-valued gradients, so every sum is exact).  Then the package's
+sharded_table_step on two gloo ranks, with numpy stand-ins for the library
+calls: each rank's shard must end as the whole table updated by the union
+batch's gradient."""
 
 import os
 import socket
@@ -138,3 +141,101 @@ def test_all_to_all_pairs_rejects_bad_counts():
         eb.all_to_all_pairs(rows, grad, torch.tensor([5], dtype=torch.int64), a2a)
     with pytest.raises(RuntimeError):   # a negative count
         eb.all_to_all_pairs(rows, grad, torch.tensor([-1], dtype=torch.int64), a2a)
+
+
+# ------------------------------------------------- the whole step, two ranks
+
+J_T, M_T, D_T, N_T = 2, 11, 3, 9          # 2 tables of 11 rows of width 3; 9 tokens per rank
+
+
+def _batch(rank):
+    rng = np.random.default_rng(40 + rank)
+    idx = rng.integers(0, M_T, size=(N_T, J_T)).astype(np.uint32)
+    de = rng.integers(-4, 5, size=(N_T, J_T * D_T)).astype(np.float64)
+    return idx, de
+
+
+class _HostEngram:
+    """Stand-ins for the library calls sharded_table_step makes, in numpy,
+    with the oracle's gradient: the step's wiring and its exchange are what
+    is tested here (the kernels are tested on the GPU)."""
+
+    def __init__(self, world):
+        self.world = world
+        self.R = J_T * M_T
+        self.per = (self.R + world - 1) // world
+
+    def table_grad(self, idx, d_e):
+        import oracle
+        keys, grad = oracle.table_grad(idx.numpy(), np.full(J_T, M_T, np.uint32), d_e.numpy(), D_T)
+        return torch.from_numpy(keys.astype(np.int64)), torch.from_numpy(grad), torch.tensor([len(keys)])
+
+    def grad_route(self, rows, grad, n_pairs, n_shards):
+        owner = rows.numpy() // self.per
+        order = np.argsort(owner, kind="stable")
+        counts = np.bincount(owner, minlength=n_shards).astype(np.int64)
+        return rows[order].contiguous(), grad[order].contiguous(), torch.from_numpy(counts)
+
+    def grad_combine(self, pair_rows, pair_grad, n_shards, shard):
+        got = {}
+        for r, g in zip(pair_rows.tolist(), pair_grad.numpy()):
+            assert r // self.per == shard
+            got[r] = got.get(r, 0) + g
+        keys = sorted(got)
+        grad = np.array([got[k] for k in keys]).reshape(len(keys), D_T)
+        return torch.tensor(keys, dtype=torch.int64), torch.from_numpy(grad), torch.tensor([len(keys)])
+
+    def shard_sgd(self, n_shards, shard, rows, grad, n_unique, shard_table, lr):
+        first = shard * self.per
+        for r, g in zip(rows.tolist(), grad):
+            shard_table[r - first] -= lr * g
+
+
+def _full_table():
+    return np.arange(J_T * M_T * D_T, dtype=np.float64).reshape(J_T * M_T, D_T) / 7.0
+
+
+def _step_main(rank, world, port, out):
+    import datetime
+    import types
+
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_02_b200 as eb
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        eng = _HostEngram(world)
+        lo, hi = rank * eng.per, min(eng.R, (rank + 1) * eng.per)
+        shards = types.SimpleNamespace(local=torch.from_numpy(_full_table()[lo:hi].copy()))
+        idx, de = _batch(rank)
+        eb.sharded_table_step(eng, shards, torch.from_numpy(idx), torch.from_numpy(de), 0.5, rank, world)
+        out.put((rank, lo, shards.local.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_table_step_two_ranks_gloo():
+    import torch.multiprocessing as mp
+
+    import oracle
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_step_main, args=(r, world, port, q)) for r in range(world)]
+    for p in ps:
+        p.start()
+    res = sorted((q.get(timeout=120) for _ in ps), key=lambda x: x[0])
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # the full table after one step on the union of the two batches
+    idx = np.concatenate([_batch(r)[0] for r in range(world)])
+    de = np.concatenate([_batch(r)[1] for r in range(world)])
+    keys, grad = oracle.table_grad(idx, np.full(J_T, M_T, np.uint32), de, D_T)
+    want = _full_table()
+    want[keys.astype(np.int64)] -= 0.5 * grad
+    for rank, lo, shard in res:
+        np.testing.assert_array_equal(shard, want[lo:lo + len(shard)])
+    assert sum(len(s) for _, _, s in res) == J_T * M_T
