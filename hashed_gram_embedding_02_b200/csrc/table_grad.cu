@@ -26,9 +26,11 @@
 //      (each lookup's rank is the number of smaller positions in the segment)
 //      and sums the slices of dL/de in that order, in fp32; a row looked up
 //      once skips the ordering.
-// The cost of step 4 grows with the square of a row's lookup count: fine for
-// Zipf batches (the largest segments hold hundreds of lookups), slow for a
-// degenerate batch in which one n-gram fills it.
+// Ordering a row's segment costs k^2 comparisons for k lookups, spread over
+// a lane group (k <= 32) or a CTA of 256 threads (longer rows): negligible
+// for Zipf batches, whose longest segments hold a few hundred lookups, but
+// a degenerate batch in which one n-gram fills a table of a million-token
+// batch costs about 4e9 comparisons per thread of that row's CTA.
 #include <algorithm>
 
 #include "ctx.cuh"
