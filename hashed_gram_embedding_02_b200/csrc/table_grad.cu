@@ -25,8 +25,8 @@
 //      chunks, rounded up to a power of two) orders its segment by position
 //      (each lookup's rank is the number of smaller positions in the segment)
 //      and sums the slices of dL/de in that order, in fp32; a row looked up
-//      once skips the ordering.  Rows looked up more than 32 times, listed
-//      by step 3, are ordered and summed by a CTA each in a second launch.
+//      once skips the ordering.  Rows looked up more than 32 times are only
+//      listed by that launch; a second launch orders and sums each with a CTA.
 // Ordering a row's segment costs k^2 comparisons for k lookups, spread over
 // a lane group (k <= 32) or a CTA of 256 threads (longer rows): negligible
 // for Zipf batches, whose longest segments hold a few hundred lookups, but
